@@ -1,0 +1,319 @@
+/*
+ * pgf8 CPU oracle — TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow, scalar C11 restatement of what the FP8 linear layer and the
+ * NestedFP dual-precision layer compute.  It exists so that tests, the
+ * smoke check and the benchmark's CPU-baseline leg can check the CUDA path
+ * against an independent definition.  Nothing in the product links, loads
+ * or calls this file; it shares no source, header, table or constant with
+ * the CUDA library, and it includes no CUDA header.
+ *
+ * Arithmetic rules:
+ *   - every floating-point quantity that the pages leave open is carried in
+ *     IEEE binary64 (double); format conversions are done on the exact value
+ *     with frexp/ldexp and nearbyint() under the default round-to-nearest-
+ *     even mode;
+ *   - where the method itself fixes a binary32 step (the per-token scale and
+ *     the scaled value that is then cast to FP8) the step is written as a
+ *     plain float operation, which C11 on x86-64 evaluates as a correctly
+ *     rounded IEEE binary32 division (FLT_EVAL_METHOD == 0);
+ *   - no blocking, reordering, vectorisation or threading: every result is
+ *     the textbook loop.
+ *
+ * Sources (pages of the "precision_gemm_fp8" subject):
+ *   [FP8-4060]  "7B on an RTX 4060 with FP8" (intelliparadigm.com 2151670):
+ *               §2.1 E4M3 format; §2.2 static weight / dynamic activation
+ *               scaling; §6.1 scale bound 448 and exponent saturation.
+ *   [CPP-FP8]   "C++ and FP8 quantization for LLM inference" (tqpw.cn 201730):
+ *               §3.1 E4M3 or E5M2; §3.3 kernel e4m3 x e4m3 -> f32 accumulate
+ *               -> bf16 output, TN; §4.2 per-channel / per-token flags.
+ *   [NestedFP]  "NestedFP dual-precision inference framework"
+ *               (intelliparadigm.com 2229392): §2.1 byte-plane split and the
+ *               (upper<<8)|lower rebuild; FP8 mode uses the upper byte;
+ *               §4.1 underflow handling of the E4M3 converter.
+ * The E4M3 ("FN" variant: no infinities, one NaN pattern per sign, largest
+ * finite 448) and E5M2 bit layouts are the public OCP 8-bit floating point
+ * definitions; binary16 is IEEE 754.
+ *
+ * Parity status of each function is stated in its comment; every function
+ * here is pinned by a CPU test (see tests/test_oracle_*.py).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#define ORC_OK 0
+#define ORC_ERR_NONFINITE 1
+#define ORC_ERR_BADSCALE 2
+#define ORC_ERR_ARG 3
+
+/* ------------------------------------------------------------------ */
+/* FP8 E4M3 (FN): sign | 4 exponent bits (bias 7) | 3 mantissa bits.   */
+/* [FP8-4060] §2.1 names E4M3; §6.1 fixes 448 as the largest value.    */
+/* ------------------------------------------------------------------ */
+
+double orc_e4m3_decode(uint8_t c)
+{
+    int s = (c >> 7) & 1;
+    int e = (c >> 3) & 0xF;
+    int m = c & 0x7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;                         /* the only NaN patterns: 0x7F, 0xFF */
+    if (e == 0)
+        v = ldexp((double)m, -9);           /* subnormal: m * 2^-9 */
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* Saturating, round-to-nearest-even cast of a binary32 value to E4M3.
+ * Values above 448 in magnitude (and infinities) become +-448; NaN stays
+ * NaN; the sign of zero is kept.  Subnormal results are produced by
+ * rounding on the 2^-9 grid ([NestedFP] §4.1 asks that underflow be
+ * handled). */
+uint8_t orc_e4m3_encode(float v)
+{
+    if (isnan(v))
+        return signbit(v) ? 0xFF : 0x7F;
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    double a = fabs((double)v);
+    if (a > 448.0)
+        return sign | 0x7E;                 /* satfinite */
+    if (a < ldexp(1.0, -6)) {               /* below the smallest normal */
+        double k = nearbyint(a * 512.0);    /* k in [0, 8]; 8 lands on 0x08 = 2^-6 */
+        return sign | (uint8_t)k;
+    }
+    int e;
+    (void)frexp(a, &e);                     /* a = f * 2^e, f in [0.5, 1) */
+    int E = e - 1;                          /* a = 1.xxx * 2^E */
+    double r = nearbyint((ldexp(a, -E) - 1.0) * 8.0);
+    if (r == 8.0) {                         /* mantissa carried into the exponent */
+        E += 1;
+        r = 0.0;
+    }
+    if (E > 8 || (E == 8 && r == 7.0))
+        return sign | 0x7E;
+    return sign | (uint8_t)(((E + 7) << 3) | (int)r);
+}
+
+/* ------------------------------------------------------------------ */
+/* FP8 E5M2: sign | 5 exponent bits (bias 15) | 2 mantissa bits.       */
+/* [CPP-FP8] §3.1 names it as the other FP8 layout; it is exactly the  */
+/* upper byte of an IEEE binary16 value ([NestedFP] §2.1).             */
+/* ------------------------------------------------------------------ */
+
+double orc_e5m2_decode(uint8_t c)
+{
+    int s = (c >> 7) & 1;
+    int e = (c >> 2) & 0x1F;
+    int m = c & 0x3;
+    double v;
+    if (e == 31)
+        return m == 0 ? (s ? -INFINITY : INFINITY) : NAN;
+    if (e == 0)
+        v = ldexp((double)m, -16);          /* subnormal: m * 2^-16 */
+    else
+        v = ldexp(1.0 + (double)m / 4.0, e - 15);
+    return s ? -v : v;
+}
+
+/* Saturating RNE cast to E5M2 (largest finite 57344 = 0x7B). */
+uint8_t orc_e5m2_encode(float v)
+{
+    if (isnan(v))
+        return signbit(v) ? 0xFF : 0x7F;
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    double a = fabs((double)v);
+    if (a > 57344.0)
+        return sign | 0x7B;
+    if (a < ldexp(1.0, -14)) {
+        double k = nearbyint(a * 65536.0);  /* k in [0, 4]; 4 lands on 0x04 = 2^-14 */
+        return sign | (uint8_t)k;
+    }
+    int e;
+    (void)frexp(a, &e);
+    int E = e - 1;
+    double r = nearbyint((ldexp(a, -E) - 1.0) * 4.0);
+    if (r == 4.0) {
+        E += 1;
+        r = 0.0;
+    }
+    if (E > 15 || (E == 15 && r == 3.0))
+        return sign | 0x7B;
+    return sign | (uint8_t)(((E + 15) << 2) | (int)r);
+}
+
+/* ------------------------------------------------------------------ */
+/* IEEE binary16 decode from its bit pattern.                          */
+/* ------------------------------------------------------------------ */
+
+double orc_fp16_decode(uint16_t b)
+{
+    int s = (b >> 15) & 1;
+    int e = (b >> 10) & 0x1F;
+    int m = b & 0x3FF;
+    double v;
+    if (e == 31)
+        return m == 0 ? (s ? -INFINITY : INFINITY) : NAN;
+    if (e == 0)
+        v = ldexp((double)m, -24);
+    else
+        v = ldexp(1.0 + (double)m / 1024.0, e - 15);
+    return s ? -v : v;
+}
+
+/* ------------------------------------------------------------------ */
+/* Per-row quantisation ([FP8-4060] §2.2 dynamic activation amax;      */
+/* [CPP-FP8] §4.2 per-token / per-channel granularity; [FP8-4060] §6.1 */
+/* the 448 bound applies to the scaled values).                        */
+/*                                                                     */
+/* For each row r (fixed order of the steps, since the pages leave it  */
+/* open):                                                              */
+/*   amax  = max_k |x[r,k]|                      (exact)               */
+/*   s     = fl32(amax / 448)                    (binary32 division)   */
+/*           s := 1 when that quotient is 0 (an all-zero row)          */
+/*   q[r,k]= E4M3_satfinite_RNE( fl32(x[r,k] / s) )                    */
+/* mode 0 (dynamic) writes s to scales[r]; mode 1 (static) reads it.   */
+/* ------------------------------------------------------------------ */
+
+static int quantize_one_row(const float *xr, int64_t cols, uint8_t *qr, float *s_io, int mode)
+{
+    float s;
+    if (mode == 0) {
+        float amax = 0.0f;
+        for (int64_t k = 0; k < cols; ++k) {
+            float a = fabsf(xr[k]);
+            if (!isfinite(a))
+                return ORC_ERR_NONFINITE;
+            if (a > amax)
+                amax = a;
+        }
+        s = amax / 448.0f;
+        if (s == 0.0f)
+            s = 1.0f;
+        *s_io = s;
+    } else {
+        s = *s_io;
+        if (!(s > 0.0f) || !isfinite(s))
+            return ORC_ERR_BADSCALE;
+        for (int64_t k = 0; k < cols; ++k)
+            if (!isfinite(xr[k]))
+                return ORC_ERR_NONFINITE;
+    }
+    for (int64_t k = 0; k < cols; ++k) {
+        float t = xr[k] / s;                /* correctly rounded binary32 quotient */
+        qr[k] = orc_e4m3_encode(t);
+    }
+    return ORC_OK;
+}
+
+/* x: rows x cols binary32 with row stride ldx (elements); q: rows x cols
+ * contiguous codes; scales: rows. */
+int orc_quantize_rows_f32(const float *x, int64_t rows, int64_t cols, int64_t ldx,
+                          uint8_t *q, float *scales, int mode)
+{
+    if (rows < 0 || cols < 0 || ldx < cols || (mode != 0 && mode != 1))
+        return ORC_ERR_ARG;
+    for (int64_t r = 0; r < rows; ++r) {
+        int st = quantize_one_row(x + r * ldx, cols, q + r * cols, scales + r, mode);
+        if (st != ORC_OK)
+            return st;
+    }
+    return ORC_OK;
+}
+
+/* Same for binary16 input bits: each element is widened exactly to
+ * binary32 first (every binary16 value is a binary32 value). */
+int orc_quantize_rows_f16(const uint16_t *x, int64_t rows, int64_t cols, int64_t ldx,
+                          uint8_t *q, float *scales, int mode, float *tmp_row)
+{
+    if (rows < 0 || cols < 0 || ldx < cols || (mode != 0 && mode != 1))
+        return ORC_ERR_ARG;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t k = 0; k < cols; ++k)
+            tmp_row[k] = (float)orc_fp16_decode(x[r * ldx + k]);
+        int st = quantize_one_row(tmp_row, cols, q + r * cols, scales + r, mode);
+        if (st != ORC_OK)
+            return st;
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* FP8 linear ([CPP-FP8] §3.3: E4M3 x E4M3 operands, both K-contiguous */
+/* ("TN"), f32 accumulation, bf16 output; scales from [FP8-4060] §2.2).*/
+/*   ref[m,n] = ( sum_k dec(aq[m,k]) * dec(wq[n,k]) ) * sa[m] * sw[n]  */
+/* evaluated in binary64.  Every product of two E4M3 values is exact   */
+/* in binary64.                                                        */
+/* ------------------------------------------------------------------ */
+
+void orc_fp8_linear(const uint8_t *aq, const float *sa, int64_t M, int64_t K,
+                    const uint8_t *wq, const float *sw, int64_t N, double *ref)
+{
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += orc_e4m3_decode(aq[m * K + k]) * orc_e4m3_decode(wq[n * K + k]);
+            ref[m * N + n] = acc * (double)sa[m] * (double)sw[n];
+        }
+}
+
+/* ------------------------------------------------------------------ */
+/* NestedFP ([NestedFP] §2.1).                                         */
+/* ------------------------------------------------------------------ */
+
+/* Split each binary16 bit pattern b into hi = b >> 8 (sign, the five
+ * exponent bits and the top two mantissa bits) and lo = b & 0xFF (the low
+ * eight mantissa bits). */
+void orc_nestedfp_split(const uint16_t *w, int64_t count, uint8_t *hi, uint8_t *lo)
+{
+    for (int64_t i = 0; i < count; ++i) {
+        hi[i] = (uint8_t)(w[i] >> 8);
+        lo[i] = (uint8_t)(w[i] & 0xFF);
+    }
+}
+
+uint16_t orc_nestedfp_rebuild(uint8_t hi, uint8_t lo)
+{
+    return (uint16_t)(((unsigned)hi << 8) | (unsigned)lo);
+}
+
+/* FP16 mode: the weight is the rebuilt binary16 value.
+ *   ref[m,n] = sum_k fp16(x[m,k]) * fp16((hi[n,k] << 8) | lo[n,k])   (binary64) */
+void orc_nestedfp_linear_fp16(const uint16_t *x, int64_t M, int64_t K,
+                              const uint8_t *hi, const uint8_t *lo, int64_t N, double *ref)
+{
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                uint16_t wb = orc_nestedfp_rebuild(hi[n * K + k], lo[n * K + k]);
+                acc += orc_fp16_decode(x[m * K + k]) * orc_fp16_decode(wb);
+            }
+            ref[m * N + n] = acc;
+        }
+}
+
+/* FP8 mode: the upper byte alone is the weight, read as an E5M2 code with
+ * unit scale; activations are quantised per token to E4M3 exactly as
+ * orc_quantize_rows_f16 does (dynamic mode).  aq (M x K) and sa (M) are
+ * outputs, tmp_row holds K floats.
+ *   ref[m,n] = ( sum_k dec_e4m3(aq[m,k]) * dec_e5m2(hi[n,k]) ) * sa[m]   */
+int orc_nestedfp_linear_fp8(const uint16_t *x, int64_t M, int64_t K,
+                            const uint8_t *hi, int64_t N, double *ref,
+                            uint8_t *aq, float *sa, float *tmp_row)
+{
+    int st = orc_quantize_rows_f16(x, M, K, K, aq, sa, 0, tmp_row);
+    if (st != ORC_OK)
+        return st;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += orc_e4m3_decode(aq[m * K + k]) * orc_e5m2_decode(hi[n * K + k]);
+            ref[m * N + n] = acc * (double)sa[m];
+        }
+    return ORC_OK;
+}
