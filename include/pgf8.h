@@ -1,0 +1,196 @@
+/*
+ * pgf8 — FP8 (E4M3) quantised linear layer and NestedFP dual-precision
+ * linear layer for NVIDIA B200 (sm_100a).  C ABI.
+ *
+ * The layer computed here is the one the "precision_gemm_fp8" pages
+ * describe:
+ *   - "7B on an RTX 4060 with FP8" (intelliparadigm.com 2151670), §2.1:
+ *     weights and activations in FP8 E4M3; §2.2: weights use static
+ *     (offline-calibrated) scales, activations dynamic scales from a
+ *     runtime amax; §6.1: scaled values must stay within 448.
+ *   - "C++ and FP8 quantization for LLM inference" (tqpw.cn 201730), §3.3:
+ *     an E4M3 x E4M3 GEMM with FP32 accumulation and BF16 output whose
+ *     operands are both K-contiguous ("TN"); §4.2: per-channel weight and
+ *     per-token activation granularity.
+ *   - "NestedFP dual-precision inference framework" (intelliparadigm.com
+ *     2229392), §2.1: one FP16 weight tensor stored as an upper-byte plane
+ *     and a lower-byte plane; FP16 mode rebuilds (upper << 8) | lower, FP8
+ *     mode feeds the upper byte alone to the compute units; §2.2: the
+ *     rebuild is fused into the GEMM's shared-memory stage.
+ *
+ * Conventions for every entry point
+ *   Memory      All pointers are DEVICE pointers owned by the caller.  The
+ *               library never allocates or frees device memory; the size of
+ *               any workspace is returned by the matching *_workspace_size().
+ *   Layout      Row-major, last index contiguous: activations x/aq [M, K],
+ *               weights w/wq/hi/lo [N, K] (K contiguous, "TN"), outputs
+ *               y [M, N].  Row strides equal the row length unless an
+ *               ld* argument is given.
+ *   Alignment   Every base pointer 16-byte aligned; K % 16 == 0 and
+ *               N % 16 == 0 (the tensor-memory-access unit moves 16-byte
+ *               granules); row strides in bytes a multiple of 16.
+ *   Execution   Asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *               default stream) on the current device.  A return of
+ *               PGF8_OK means the work was enqueued.
+ *   Errors      Argument errors are reported before anything is enqueued
+ *               (INVALID_ARG, ALIGNMENT, UNSUPPORTED).  A failed launch
+ *               returns PGF8_ERR_CUDA (details: pgf8_last_cuda_error).  Every
+ *               device-side wait is bounded; a kernel that gives up raises a
+ *               device error word, reported by pgf8_device_status() as
+ *               PGF8_ERR_TIMEOUT.  No C++ exception crosses this boundary.
+ *   Determinism Results are bit-identical from run to run for the same
+ *               inputs, shapes and options: split-K partial sums are added
+ *               in a fixed order, never with floating-point atomics.
+ */
+#ifndef PGF8_H
+#define PGF8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PGF8_OK = 0,
+    PGF8_ERR_INVALID_ARG = 1,
+    PGF8_ERR_ALIGNMENT = 2,
+    PGF8_ERR_UNSUPPORTED = 3,
+    PGF8_ERR_CUDA = 4,
+    PGF8_ERR_TIMEOUT = 5
+} pgf8_status;
+
+typedef enum { PGF8_F32 = 0, PGF8_F16 = 1, PGF8_BF16 = 2 } pgf8_dtype;
+
+typedef enum { PGF8_SCALE_DYNAMIC = 0, PGF8_SCALE_STATIC = 1 } pgf8_scale_mode;
+
+typedef enum { PGF8_NESTED_FP16 = 0, PGF8_NESTED_FP8 = 1 } pgf8_nested_mode;
+
+/* Kernel family used by the linear entry points. */
+typedef enum {
+    PGF8_PATH_AUTO = 0,    /* chosen from M, N, K */
+    PGF8_PATH_SKINNY = 1,  /* weight-streaming: weights are the 128-row MMA operand,
+                              tokens the narrow one (M <= 128) */
+    PGF8_PATH_TILED = 2    /* tokens are the 128-row MMA operand (any M) */
+} pgf8_path;
+
+/* Optional tuning of the linear entry points; a NULL pointer means all
+ * defaults.  Fields set to 0 mean "choose automatically". */
+typedef struct {
+    int32_t path;      /* pgf8_path */
+    int32_t split_k;   /* K split across a thread-block cluster, 1..8 */
+    int32_t tile_n;    /* narrow MMA operand rows: 16, 32, 64, 128 (skinny) or 128, 256 (tiled) */
+    int32_t reserved;
+} pgf8_linear_opts;
+
+/* ------------------------------------------------------------------------
+ * Per-row FP8 quantisation (activations per token, weights per output
+ * channel).  "7B on an RTX 4060 with FP8" §2.2 and §6.1; "C++ and FP8" §4.2.
+ *
+ * For each row r of x ([rows, cols], element type xdt = PGF8_F32 or
+ * PGF8_F16, row stride ldx elements):
+ *   DYNAMIC: amax = max_k |x[r,k]|; scales[r] = fl32(amax / 448), or 1.0
+ *            when that quotient is 0 (all-zero row);
+ *   STATIC:  scales[r] is read (must be positive and finite);
+ *   q[r,k] = E4M3 code of fl32(x[r,k] / scales[r]), rounded to nearest even,
+ *            saturated to +-448, sign of zero kept.
+ * q is [rows, cols] contiguous (uint8 codes, OCP E4M3 "FN" layout).
+ * Results are bit-exact with respect to that definition.  Non-finite input
+ * values give unspecified codes.
+ * ---------------------------------------------------------------------- */
+pgf8_status pgf8_fp8_quantize_rows(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols,
+                                   int64_t ldx, uint8_t *q, float *scales,
+                                   pgf8_scale_mode mode, void *stream);
+
+/* ------------------------------------------------------------------------
+ * FP8 linear with fused dequantisation ("C++ and FP8" §3.3):
+ *   y[m,n] = bf16_rn( (sum_k e4m3(aq[m,k]) * e4m3(wq[n,k])) * sa[m] * sw[n] )
+ * with FP32 accumulation.  aq [M,K] uint8, sa [M] f32, wq [N,K] uint8,
+ * sw [N] f32, y [M,N] bf16.  M >= 1.  workspace may be NULL when
+ * pgf8_fp8_linear_workspace_size() returns 0 (it currently always does).
+ * ---------------------------------------------------------------------- */
+pgf8_status pgf8_fp8_linear(const uint8_t *aq, const float *sa, int64_t M, int64_t K,
+                            const uint8_t *wq, const float *sw, int64_t N, void *y_bf16,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
+pgf8_status pgf8_fp8_linear_ex(const uint8_t *aq, const float *sa, int64_t M, int64_t K,
+                               const uint8_t *wq, const float *sw, int64_t N, void *y_bf16,
+                               void *workspace, size_t workspace_bytes,
+                               const pgf8_linear_opts *opts, void *stream);
+
+size_t pgf8_fp8_linear_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/* ------------------------------------------------------------------------
+ * Dynamic-activation FP8 linear: per-token quantisation of x (as
+ * pgf8_fp8_quantize_rows, DYNAMIC) followed by pgf8_fp8_linear, enqueued as
+ * one dependent pair so the GEMM's set-up and first weight loads overlap the
+ * quantisation ("7B on an RTX 4060 with FP8" §2.2: activations quantised at
+ * run time).  x [M,K] f32 or f16 with row stride ldx.  The workspace
+ * (size from pgf8_fp8_linear_dynamic_workspace_size) receives the E4M3
+ * activation codes [M,K] at offset 0 and the per-token scales [M] at offset
+ * pgf8_fp8_linear_dynamic_scales_offset(M, K); the caller may read both
+ * after the call completes.  wq must not be written by work enqueued
+ * between this call's quantisation and GEMM (nothing is).
+ * ---------------------------------------------------------------------- */
+pgf8_status pgf8_fp8_linear_dynamic(const void *x, pgf8_dtype xdt, int64_t M, int64_t K,
+                                    int64_t ldx, const uint8_t *wq, const float *sw, int64_t N,
+                                    void *y_bf16, void *workspace, size_t workspace_bytes,
+                                    const pgf8_linear_opts *opts, void *stream);
+
+size_t pgf8_fp8_linear_dynamic_workspace_size(int64_t M, int64_t N, int64_t K);
+size_t pgf8_fp8_linear_dynamic_scales_offset(int64_t M, int64_t K);
+
+/* ------------------------------------------------------------------------
+ * NestedFP byte-plane split ("NestedFP" §2.1): for each FP16 weight bit
+ * pattern b of w_f16 [N,K]: hi[n,k] = b >> 8 (sign, 5 exponent bits, top 2
+ * mantissa bits), lo[n,k] = b & 0xFF.  Bit-exact; (hi << 8) | lo == b.
+ * ---------------------------------------------------------------------- */
+pgf8_status pgf8_nestedfp_split(const void *w_f16, int64_t N, int64_t K, uint8_t *hi,
+                                uint8_t *lo, void *stream);
+
+/* ------------------------------------------------------------------------
+ * NestedFP linear ("NestedFP" §2.1-2.2).  x_f16 [M,K] FP16, y_f16 [M,N] FP16.
+ *   PGF8_NESTED_FP16: y = fp16_rn( sum_k x[m,k] * fp16((hi<<8)|lo)[n,k] ),
+ *     the weight rebuilt bit-exactly in shared memory inside the GEMM;
+ *     FP32 accumulation.  workspace unused (size 0).
+ *   PGF8_NESTED_FP8: x is quantised per token to E4M3 (as
+ *     pgf8_fp8_quantize_rows, DYNAMIC) into the workspace, and
+ *     y = fp16_rn( (sum_k e4m3(aq[m,k]) * e5m2(hi[n,k])) * sa[m] ): the upper
+ *     byte is read as an E5M2 code with unit scale, which is the FP16 weight
+ *     with its low 8 bits cleared.  lo is ignored and may be NULL.
+ * ---------------------------------------------------------------------- */
+pgf8_status pgf8_nestedfp_linear(const void *x_f16, int64_t M, int64_t K, const uint8_t *hi,
+                                 const uint8_t *lo, int64_t N, pgf8_nested_mode mode,
+                                 void *y_f16, void *workspace, size_t workspace_bytes,
+                                 void *stream);
+
+pgf8_status pgf8_nestedfp_linear_ex(const void *x_f16, int64_t M, int64_t K, const uint8_t *hi,
+                                    const uint8_t *lo, int64_t N, pgf8_nested_mode mode,
+                                    void *y_f16, void *workspace, size_t workspace_bytes,
+                                    const pgf8_linear_opts *opts, void *stream);
+
+size_t pgf8_nestedfp_linear_workspace_size(int64_t M, int64_t N, int64_t K,
+                                           pgf8_nested_mode mode);
+
+/* ------------------------------------------------------------------------
+ * Diagnostics.
+ * pgf8_last_cuda_error: the cudaError_t of the most recent failed CUDA call
+ *   made by this library on the calling thread (0 if none).
+ * pgf8_device_status: synchronises `stream`, then reads and clears the
+ *   device error word of the current device: PGF8_ERR_TIMEOUT if a kernel
+ *   gave up a bounded wait since the last check, PGF8_ERR_CUDA if the
+ *   synchronisation itself failed, else PGF8_OK.
+ * pgf8_status_str: static description of a status code.
+ * pgf8_version: library version as major*10000 + minor*100 + patch.
+ * ---------------------------------------------------------------------- */
+pgf8_status pgf8_last_cuda_error(int *cuda_err);
+pgf8_status pgf8_device_status(void *stream);
+const char *pgf8_status_str(pgf8_status status);
+int pgf8_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PGF8_H */

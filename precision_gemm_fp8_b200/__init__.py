@@ -1,0 +1,228 @@
+"""B200 (sm_100a) FP8 E4M3 quantised linear layer and NestedFP dual-precision
+linear layer.
+
+This module is the Python binding of ``libpgf8.so`` (the C ABI declared in
+``include/pgf8.h``).  It only marshals arguments: tensors are plain device
+buffers (PyTorch is used for device memory and streams), every computation
+runs in the library's CUDA kernels, and there is no other code path.  If the
+library has not been built the import fails; build it with
+``python -m precision_gemm_fp8_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libpgf8.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "pgf8.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m precision_gemm_fp8_b200.build` "
+                      "(the CUDA library is the only implementation)")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+OK, ERR_INVALID_ARG, ERR_ALIGNMENT, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = range(6)
+F32, F16, BF16 = 0, 1, 2
+SCALE_DYNAMIC, SCALE_STATIC = 0, 1
+NESTED_FP16, NESTED_FP8 = 0, 1
+PATH_AUTO, PATH_SKINNY, PATH_TILED = 0, 1, 2
+
+
+class LinearOpts(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int32), ("split_k", ctypes.c_int32), ("tile_n", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_sz = ctypes.c_size_t
+_i32 = ctypes.c_int
+_optp = ctypes.POINTER(LinearOpts)
+
+_SIGS = {
+    "pgf8_fp8_quantize_rows": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _i32, _vp], _i32),
+    "pgf8_fp8_linear": ([_vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _sz, _vp], _i32),
+    "pgf8_fp8_linear_ex": ([_vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _sz, _optp, _vp], _i32),
+    "pgf8_fp8_linear_workspace_size": ([_i64, _i64, _i64], _sz),
+    "pgf8_fp8_linear_dynamic": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _sz, _optp, _vp], _i32),
+    "pgf8_fp8_linear_dynamic_workspace_size": ([_i64, _i64, _i64], _sz),
+    "pgf8_fp8_linear_dynamic_scales_offset": ([_i64, _i64], _sz),
+    "pgf8_nestedfp_split": ([_vp, _i64, _i64, _vp, _vp, _vp], _i32),
+    "pgf8_nestedfp_linear": ([_vp, _i64, _i64, _vp, _vp, _i64, _i32, _vp, _vp, _sz, _vp], _i32),
+    "pgf8_nestedfp_linear_ex": ([_vp, _i64, _i64, _vp, _vp, _i64, _i32, _vp, _vp, _sz, _optp, _vp], _i32),
+    "pgf8_nestedfp_linear_workspace_size": ([_i64, _i64, _i64, _i32], _sz),
+    "pgf8_last_cuda_error": ([ctypes.POINTER(ctypes.c_int)], _i32),
+    "pgf8_device_status": ([_vp], _i32),
+    "pgf8_status_str": ([_i32], ctypes.c_char_p),
+    "pgf8_version": ([], _i32),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.argtypes = _args
+    _f.restype = _res
+
+
+def header_symbols() -> list[str]:
+    """Names of the functions declared in include/pgf8.h."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^\s*(?:pgf8_status|size_t|const char \*|int)\s*(pgf8_\w+)\s*\(", text, re.M)))
+
+
+class Pgf8Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = lib.pgf8_status_str(status).decode()
+        if status == ERR_CUDA:
+            e = ctypes.c_int(0)
+            lib.pgf8_last_cuda_error(ctypes.byref(e))
+            msg += f" (cudaError {e.value})"
+        super().__init__(f"{where}: {msg}")
+        self.status = status
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise Pgf8Error(status, where)
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("pgf8 takes device tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _opts(path=PATH_AUTO, split_k=0, tile_n=0):
+    if path == PATH_AUTO and split_k == 0 and tile_n == 0:
+        return None
+    return ctypes.byref(LinearOpts(path, split_k, tile_n, 0))
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.float16:
+        return F16
+    raise TypeError(f"unsupported activation dtype {t.dtype}")
+
+
+# ----------------------------------------------------------------- entry points
+def fp8_quantize_rows(x: torch.Tensor, q: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                      mode: int = SCALE_DYNAMIC, stream=None):
+    """Per-row E4M3 quantisation of x [rows, cols] (f32 or f16, row stride
+    x.stride(0)).  Returns (q uint8 [rows, cols], scales f32 [rows]).  In
+    static mode ``scales`` holds the given scales."""
+    rows, cols = x.shape
+    if x.stride(1) != 1:
+        raise ValueError("x rows must be contiguous")
+    if q is None:
+        q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        if mode == SCALE_STATIC:
+            raise ValueError("static mode needs scales")
+        scales = torch.empty(rows, dtype=torch.float32, device=x.device)
+    _check(lib.pgf8_fp8_quantize_rows(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(q), _ptr(scales),
+                                      mode, _stream(stream)), "fp8_quantize_rows")
+    return q, scales
+
+
+def fp8_linear(aq, sa, wq, sw, y=None, path=PATH_AUTO, split_k=0, tile_n=0, stream=None):
+    """y [M,N] bf16 = (E4M3 aq [M,K] x E4M3 wq [N,K]^T) * sa[m] * sw[n]."""
+    M, K = aq.shape
+    N = wq.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=aq.device)
+    _check(lib.pgf8_fp8_linear_ex(_ptr(aq), _ptr(sa), M, K, _ptr(wq), _ptr(sw), N, _ptr(y), None, 0,
+                                  _opts(path, split_k, tile_n), _stream(stream)), "fp8_linear")
+    return y
+
+
+def fp8_linear_dynamic_workspace_size(M: int, N: int, K: int) -> int:
+    return int(lib.pgf8_fp8_linear_dynamic_workspace_size(M, N, K))
+
+
+def fp8_linear_dynamic(x, wq, sw, y=None, workspace=None, path=PATH_AUTO, split_k=0, tile_n=0, stream=None):
+    """Per-token dynamic quantisation of x [M,K] (f32/f16) followed by the FP8
+    linear with weights wq [N,K] / sw [N].  Returns y [M,N] bf16."""
+    M, K = x.shape
+    N = wq.shape[0]
+    if x.stride(1) != 1:
+        raise ValueError("x rows must be contiguous")
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    need = fp8_linear_dynamic_workspace_size(M, N, K)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    _check(lib.pgf8_fp8_linear_dynamic(_ptr(x), _dtype_code(x), M, K, x.stride(0), _ptr(wq), _ptr(sw), N, _ptr(y),
+                                       _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                       _opts(path, split_k, tile_n), _stream(stream)), "fp8_linear_dynamic")
+    return y
+
+
+def dynamic_workspace_views(workspace: torch.Tensor, M: int, K: int):
+    """(aq [M,K] uint8, sa [M] f32) views of a dynamic-linear workspace."""
+    off = int(lib.pgf8_fp8_linear_dynamic_scales_offset(M, K))
+    aq = workspace[:M * K].view(M, K)
+    sa = workspace[off:off + 4 * M].view(torch.float32)
+    return aq, sa
+
+
+def nestedfp_split(w: torch.Tensor, hi=None, lo=None, stream=None):
+    """hi/lo byte planes [N,K] of an FP16 weight [N,K]."""
+    if w.dtype != torch.float16 or not w.is_contiguous():
+        raise ValueError("w must be a contiguous float16 tensor")
+    N, K = w.shape
+    if hi is None:
+        hi = torch.empty((N, K), dtype=torch.uint8, device=w.device)
+    if lo is None:
+        lo = torch.empty((N, K), dtype=torch.uint8, device=w.device)
+    _check(lib.pgf8_nestedfp_split(_ptr(w), N, K, _ptr(hi), _ptr(lo), _stream(stream)), "nestedfp_split")
+    return hi, lo
+
+
+def nestedfp_linear_workspace_size(M: int, N: int, K: int, mode: int) -> int:
+    return int(lib.pgf8_nestedfp_linear_workspace_size(M, N, K, mode))
+
+
+def nestedfp_linear(x, hi, lo, mode=NESTED_FP16, y=None, workspace=None, path=PATH_AUTO, split_k=0, tile_n=0,
+                    stream=None):
+    """NestedFP linear: x [M,K] f16, hi/lo [N,K] uint8 planes -> y [M,N] f16.
+    FP16 mode rebuilds (hi << 8) | lo; FP8 mode uses hi as E5M2 and
+    quantises x per token to E4M3 (lo unused)."""
+    if x.dtype != torch.float16 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float16 tensor")
+    M, K = x.shape
+    N = hi.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float16, device=x.device)
+    need = nestedfp_linear_workspace_size(M, N, K, mode)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.pgf8_nestedfp_linear_ex(_ptr(x), M, K, _ptr(hi), _ptr(lo) if lo is not None else None, N, mode,
+                                       _ptr(y), _ptr(workspace), wbytes, _opts(path, split_k, tile_n),
+                                       _stream(stream)), "nestedfp_linear")
+    return y
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error status."""
+    return int(lib.pgf8_device_status(_stream(stream)))
+
+
+def version() -> int:
+    return int(lib.pgf8_version())

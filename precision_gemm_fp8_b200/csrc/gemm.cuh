@@ -1,0 +1,565 @@
+// tcgen05 GEMM for the FP8 linear layer and the NestedFP linear layer.
+//
+//   y[m,n] = epilogue( sum_k X[m,k] * W[n,k] )
+//
+// X: activations [M,K], W: weights [N,K], both K-contiguous ("C++ and FP8"
+// §3.3, the "tn" E4M3 x E4M3 -> f32 GEMM with bf16 output).  One kernel
+// template covers the three operand kinds:
+//   kE4M3     X E4M3, W E4M3, y = bf16(acc * sa[m] * sw[n])           (FP8 linear)
+//   kNested8  X E4M3, W = hi plane read as E5M2, y = f16(acc * sa[m])  (NestedFP FP8 mode)
+//   kNested16 X FP16, W = (hi << 8) | lo rebuilt in shared memory, y = f16(acc)
+//             (NestedFP FP16 mode; "NestedFP" §2.1-2.2)
+// and two orientations:
+//   SWAP = false ("tiled"):  MMA A = 128 token rows,  MMA B = BN weight rows,
+//                            accumulator lane = token, column = output channel;
+//   SWAP = true  ("skinny"): MMA A = 128 weight rows, MMA B = BN token rows
+//                            (BN >= M, zero-filled), lane = output channel,
+//                            column = token.  Used for decode-sized M, where the
+//                            layer streams weights from HBM.
+//
+// Structure (one output tile per CTA, 192 threads):
+//   warp 0      TMA producer: STAGES-deep ring of (A tile, B tile), 128 bytes
+//               of K per stage, 128-byte swizzle, mbarrier completion.
+//   warp 1      allocates the tensor-memory accumulator and issues
+//               tcgen05.mma (one thread), committing each stage back to the
+//               producer and the finished tile to the epilogue.
+//   warps 2-5   kNested16 only: rebuild the FP16 weight tile in place from the
+//               hi/lo byte planes (byte permutes into the swizzled K-major
+//               FP16 layout), then hand it to the MMA thread.
+//               All kinds: epilogue — tcgen05.ld of the accumulator, scaling,
+//               rounding, 16- or 2-byte stores.
+// Split-K: with SPLIT, the CTAs of one thread-block cluster (along z) each
+// accumulate a slice of K; partial tiles are exchanged through distributed
+// shared memory and summed in cluster-rank order (deterministic), each CTA
+// finishing an equal share of the tile.
+//
+// Every wait is bounded (kWaitLimitNs).  A thread that gives up raises the
+// CTA's abort flag and the device error word; the other roles stop at their
+// next wait, in-flight copies and MMAs are drained (bounded again), the
+// accumulator is freed and the CTA exits through the same barriers.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+
+namespace pgf8 {
+
+enum OpKind : int { kE4M3 = 0, kNested8 = 1, kNested16 = 2 };
+
+constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;   // 1 s
+constexpr unsigned kErrTimeout = 1u;
+
+__device__ unsigned int g_device_error;
+
+struct GemmParams {
+    int M, N, K;         // elements
+    int kblocks;         // ceil(K * elem_bytes / 128)
+    int splits;          // CTAs per cluster along z (1 = no split)
+    int prefetch_w;      // 1: weight tiles may be loaded before the grid dependency resolves
+    const float *sa;     // [M] (kE4M3, kNested8)
+    const float *sw;     // [N] (kE4M3)
+    void *y;             // [M, N] bf16 (kE4M3) or f16
+};
+
+template <bool SWAP_, int BN_, int STAGES_, int KIND_, bool SPLIT_> struct GemmCfg {
+    static constexpr bool SWAP = SWAP_;
+    static constexpr int BN = BN_;
+    static constexpr int STAGES = STAGES_;
+    static constexpr int KIND = KIND_;
+    static constexpr bool SPLIT = SPLIT_;
+    static constexpr int kThreads = 192;
+    static constexpr int kTileA = 128 * 128;                  // 128 rows x 128 bytes
+    static constexpr int kTileB = BN * 128;
+    static constexpr int kStage = kTileA + kTileB;
+    static constexpr int kRowsW = SWAP ? 128 : BN;            // weight rows per tile
+    static constexpr int kRowsX = SWAP ? BN : 128;            // token rows per tile
+    static constexpr int kTmemCols = BN < 32 ? 32 : BN;
+    // split-K partial tile in shared memory (reuses the stage ring):
+    //   SWAP: column-major [BN][128] f32;  tiled: row-major [128][BN + 4] f32
+    static constexpr int kRedBytes = SWAP ? BN * 128 * 4 : 128 * (BN + 4) * 4;
+    static constexpr int kRingBytes = STAGES * kStage;
+    static constexpr int kDataBytes = kRingBytes > kRedBytes ? kRingBytes : kRedBytes;
+    static constexpr int kBarOffset = kDataBytes;
+    static constexpr int kSmemBytes = kDataBytes + 1024 /*barriers*/ + 1024 /*alignment slack*/;
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128 must be a multiple of 16 in [16,256]");
+    static_assert((BN & (BN - 1)) == 0 || BN % 32 == 0, "BN");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+};
+
+struct SharedCtl {
+    uint64_t full[16];
+    uint64_t empty[16];
+    uint64_t conv[16];
+    uint64_t tmem_full;
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// Bounded wait on an mbarrier phase.  Returns false (and raises the abort
+// flag and the device error word) after kWaitLimitNs, or when another role
+// of the CTA has already raised the abort flag.
+__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t spin = 1;; ++spin) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if ((spin & 63u) == 0) {
+            if (*abort)
+                return false;
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                *abort = 1;
+                atomicOr(&g_device_error, kErrTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+// Wait used only while draining after an abort: bounded, never raises.
+__device__ __forceinline__ void wait_drain(uint64_t *bar, uint32_t parity)
+{
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > kWaitLimitNs)
+            return;
+    }
+}
+
+// Rebuild FP16 weights in place: the stage region holds the hi plane
+// [rows][64 B] followed by the lo plane [rows][64 B] (no swizzle); it is
+// rewritten as FP16 [rows][128 B] in the 128-byte-swizzled K-major layout
+// (16-byte chunk j of row r stored at chunk j ^ (r % 8)).  Half e of a chunk
+// is (hi[e] << 8) | lo[e]; in little-endian bytes: lo[e], hi[e].
+template <int ROWS>
+__device__ __forceinline__ void rebuild_fp16_tile(uint8_t *tile, int tid /*0..127*/)
+{
+    constexpr int kItems = ROWS * 8 / 128;   // 16-byte output chunks per thread
+    uint2 h[kItems], l[kItems];
+#pragma unroll
+    for (int u = 0; u < kItems; ++u) {
+        const int i = tid + 128 * u;         // chunk index: row i/8, chunk i%8
+        h[u] = *reinterpret_cast<const uint2 *>(tile + i * 8);
+        l[u] = *reinterpret_cast<const uint2 *>(tile + ROWS * 64 + i * 8);
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll
+    for (int u = 0; u < kItems; ++u) {
+        const int i = tid + 128 * u;
+        const int r = i >> 3, j = i & 7;
+        uint4 o;
+        o.x = __byte_perm(l[u].x, h[u].x, 0x5140);
+        o.y = __byte_perm(l[u].x, h[u].x, 0x7362);
+        o.z = __byte_perm(l[u].y, h[u].y, 0x5140);
+        o.w = __byte_perm(l[u].y, h[u].y, 0x7362);
+        *reinterpret_cast<uint4 *>(tile + r * 128 + ((j ^ (r & 7)) << 4)) = o;
+    }
+}
+
+template <int KIND> __device__ __forceinline__ void store_out(void *y, int64_t idx, float v);
+template <> __device__ __forceinline__ void store_out<kE4M3>(void *y, int64_t idx, float v)
+{
+    reinterpret_cast<__nv_bfloat16 *>(y)[idx] = __float2bfloat16_rn(v);
+}
+template <> __device__ __forceinline__ void store_out<kNested8>(void *y, int64_t idx, float v)
+{
+    reinterpret_cast<__half *>(y)[idx] = __float2half_rn(v);
+}
+template <> __device__ __forceinline__ void store_out<kNested16>(void *y, int64_t idx, float v)
+{
+    reinterpret_cast<__half *>(y)[idx] = __float2half_rn(v);
+}
+
+// Pack two floats into two 16-bit outputs (low half = a).
+template <int KIND> __device__ __forceinline__ uint32_t pack2(float a, float b)
+{
+    if constexpr (KIND == kE4M3) {
+        __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
+        return *reinterpret_cast<uint32_t *>(&t);
+    } else {
+        __half2 t = __floats2half2_rn(a, b);
+        return *reinterpret_cast<uint32_t *>(&t);
+    }
+}
+
+template <class C>
+__global__ void __launch_bounds__(192, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                const __grid_constant__ CUtensorMap tmW2, const GemmParams p)
+{
+    constexpr bool SWAP = C::SWAP;
+    constexpr int BN = C::BN;
+    constexpr int STAGES = C::STAGES;
+    constexpr int KIND = C::KIND;
+    constexpr bool NEST16 = (KIND == kNested16);
+    constexpr uint32_t kIdesc =
+        make_idesc(128, BN, /*A fmt*/ (SWAP && KIND == kNested8) ? 1 : 0, /*B fmt*/ (!SWAP && KIND == kNested8) ? 1 : 0);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    SharedCtl *ctl = reinterpret_cast<SharedCtl *>(smem + C::kBarOffset);
+    volatile int *abort_flag = &ctl->abort;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int tile_a = blockIdx.x;   // A-side tile (128 rows)
+    const int tile_b = blockIdx.y;   // B-side tile (BN rows)
+    const int split = C::SPLIT ? static_cast<int>(blockIdx.z) : 0;
+    const int kb0 = C::SPLIT ? (split * p.kblocks) / p.splits : 0;
+    const int kb1 = C::SPLIT ? ((split + 1) * p.kblocks) / p.splits : p.kblocks;
+    const int row0_w = SWAP ? tile_a * 128 : tile_b * BN;   // first weight row of the tile
+    const int row0_x = SWAP ? tile_b * BN : tile_a * 128;   // first token row of the tile
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->empty[s], 1);
+            mbar_init(&ctl->conv[s], 128);
+        }
+        mbar_init(&ctl->tmem_full, 1);
+        mbar_init(&ctl->drain, 1);
+        ctl->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmX);
+        tma_prefetch_desc(&tmW);
+        if (NEST16)
+            tma_prefetch_desc(&tmW2);
+    }
+    if (warp == 1) {
+        tmem_alloc(&ctl->tmem_base, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl->tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            // weights are streamed once in the skinny orientation (evict first);
+            // activation tiles are re-read by every CTA (evict last)
+            const uint64_t pol_w = SWAP ? policy_evict_first() : policy_evict_last();
+            const uint64_t pol_x = policy_evict_last();
+            constexpr int kXStep = NEST16 ? 64 : 128;   // K elements per stage
+            bool waited = false;
+            if (!p.prefetch_w) {
+                grid_dependency_wait();
+                waited = true;
+            }
+            int s = 0;
+            uint32_t ph = 0;
+            uint32_t issued_mask = 0, issued_ph = 0;   // per stage: loaded at least once / parity of last load
+            int pending = 0;                            // stages with weights but no activations yet
+            for (int kb = kb0; kb < kb1; ++kb) {
+                if (!wait_bounded(&ctl->empty[s], ph ^ 1u, abort_flag))
+                    break;
+                uint8_t *st = smem + s * C::kStage;
+                uint8_t *w_tile = SWAP ? st : st + C::kTileA;
+                mbar_arrive_expect_tx(&ctl->full[s], C::kStage);
+                if constexpr (NEST16) {
+                    // hi and lo planes, 64 bytes (= 64 weights) of K each
+                    tma_load_2d_hint(w_tile, &tmW, &ctl->full[s], kb * 64, row0_w, pol_w);
+                    tma_load_2d_hint(w_tile + C::kRowsW * 64, &tmW2, &ctl->full[s], kb * 64, row0_w, pol_w);
+                } else {
+                    tma_load_2d_hint(w_tile, &tmW, &ctl->full[s], kb * 128, row0_w, pol_w);
+                }
+                issued_mask |= 1u << s;
+                issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
+                if (waited) {
+                    uint8_t *x_tile = SWAP ? st + C::kTileA : st;
+                    tma_load_2d_hint(x_tile, &tmX, &ctl->full[s], kb * kXStep, row0_x, pol_x);
+                } else if (++pending == STAGES || kb + 1 == kb1) {
+                    // the first pass of weight tiles went out before the
+                    // dependency resolved; activations only after it
+                    grid_dependency_wait();
+                    waited = true;
+                    for (int j = 0; j < pending; ++j) {
+                        const int kbj = kb - pending + 1 + j;
+                        const int sj = (s - pending + 1 + j + STAGES) % STAGES;
+                        uint8_t *stj = smem + sj * C::kStage;
+                        uint8_t *x_tile = SWAP ? stj + C::kTileA : stj;
+                        tma_load_2d_hint(x_tile, &tmX, &ctl->full[sj], kbj * kXStep, row0_x, pol_x);
+                    }
+                    pending = 0;
+                }
+                if (++s == STAGES) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+            if (!waited)
+                grid_dependency_wait();
+            if (*abort_flag) {
+                // drain: the last load of every used stage lands (bounded) before
+                // the CTA may exit; older loads were consumed already
+                for (int j = 0; j < STAGES; ++j)
+                    if (issued_mask & (1u << j))
+                        wait_drain(&ctl->full[j], (issued_ph >> j) & 1u);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        grid_dependency_wait();
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int kb = kb0; kb < kb1; ++kb) {
+                if (!wait_bounded(&ctl->full[s], ph, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                if constexpr (NEST16) {
+                    if (!wait_bounded(&ctl->conv[s], ph, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                tc_fence_after();
+                const uint32_t a_addr = smem_u32(smem + s * C::kStage);
+                const uint32_t b_addr = a_addr + C::kTileA;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {   // 4 MMAs x 32 bytes of K
+                    const uint64_t ad = sdesc_sw128(a_addr + k * 32);
+                    const uint64_t bd = sdesc_sw128(b_addr + k * 32);
+                    const uint32_t acc = (kb > kb0 || k > 0) ? 1u : 0u;
+                    if constexpr (NEST16)
+                        umma_f16(tmem, ad, bd, kIdesc, acc);
+                    else
+                        umma_f8f6f4(tmem, ad, bd, kIdesc, acc);
+                }
+                umma_commit(&ctl->empty[s]);
+                if (++s == STAGES) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+            if (ok) {
+                umma_commit(&ctl->tmem_full);
+            } else {
+                umma_commit(&ctl->drain);
+                wait_drain(&ctl->drain, 0);
+            }
+        }
+        __syncwarp();
+    } else {
+        grid_dependency_wait();
+        // ------------------------------------------------------------ FP16 rebuild
+        if constexpr (NEST16) {
+            const int tt = static_cast<int>(threadIdx.x) - 64;   // 0..127
+            int s = 0;
+            uint32_t ph = 0;
+            for (int kb = kb0; kb < kb1; ++kb) {
+                if (!wait_bounded(&ctl->full[s], ph, abort_flag))
+                    break;
+                uint8_t *tile = smem + s * C::kStage + (SWAP ? 0 : C::kTileA);
+                rebuild_fp16_tile<C::kRowsW>(tile, tt);
+                fence_proxy_async_smem();
+                mbar_arrive(&ctl->conv[s]);
+                if (++s == STAGES) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+        }
+    }
+
+    // ---------------------------------------------------------------- epilogue
+    // All 6 warps reach this point; warps 2-5 own the accumulator rows.
+    const bool epi = warp >= 2;
+    bool have_acc = false;
+    if (epi) {
+        have_acc = wait_bounded(&ctl->tmem_full, 0, abort_flag);
+        have_acc = __all_sync(0xffffffffu, have_acc);
+        tc_fence_after();
+    }
+    const int et = static_cast<int>(threadIdx.x) - 64;   // epilogue thread index 0..127
+    const int q = warp & 3;                     // TMEM lane quadrant of this warp
+    const int r = q * 32 + lane;                // accumulator row (lane)
+    const uint32_t t_row = tmem + (static_cast<uint32_t>(q * 32) << 16);
+
+    if constexpr (!C::SPLIT) {
+        if (epi && have_acc) {
+            if constexpr (SWAP) {
+                // lane = output channel n, column = token m
+                const int n = row0_w + r;
+                float swn = 1.0f;
+                if constexpr (KIND == kE4M3)
+                    swn = (n < p.N) ? p.sw[n] : 0.0f;
+#pragma unroll 1
+                for (int c0 = 0; c0 < BN; c0 += 16) {
+                    if (row0_x + c0 >= p.M)
+                        break;                  // warp-uniform
+                    uint32_t v[16];
+                    tmem_ld_32x32b_x16(t_row + c0, v);
+                    tmem_ld_wait();
+                    if (n < p.N) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int m = row0_x + c0 + j;
+                            if (m < p.M) {
+                                float a = __uint_as_float(v[j]);
+                                if constexpr (KIND != kNested16)
+                                    a = a * p.sa[m];
+                                if constexpr (KIND == kE4M3)
+                                    a = a * swn;
+                                store_out<KIND>(p.y, static_cast<int64_t>(m) * p.N + n, a);
+                            }
+                        }
+                    }
+                }
+            } else {
+                // lane = token m, column = output channel n
+                const int m = row0_x + r;
+                float sam = 1.0f;
+                if constexpr (KIND != kNested16)
+                    sam = (m < p.M) ? p.sa[m] : 0.0f;
+#pragma unroll 1
+                for (int c0 = 0; c0 < BN; c0 += 16) {
+                    const int n0 = row0_w + c0;
+                    if (n0 >= p.N)
+                        break;                  // warp-uniform; N % 16 == 0
+                    uint32_t v[16];
+                    tmem_ld_32x32b_x16(t_row + c0, v);
+                    tmem_ld_wait();
+                    if (m < p.M) {
+                        uint32_t o[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            float a0 = __uint_as_float(v[2 * j]), a1 = __uint_as_float(v[2 * j + 1]);
+                            if constexpr (KIND != kNested16) {
+                                a0 = a0 * sam;
+                                a1 = a1 * sam;
+                            }
+                            if constexpr (KIND == kE4M3) {
+                                a0 = a0 * __ldg(p.sw + n0 + 2 * j);
+                                a1 = a1 * __ldg(p.sw + n0 + 2 * j + 1);
+                            }
+                            o[j] = pack2<KIND>(a0, a1);
+                        }
+                        uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.y) +
+                                                               static_cast<int64_t>(m) * p.N + n0);
+                        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+                        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+                    }
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ split-K
+        // 1. each CTA stores its partial tile into its own (now idle) ring
+        float *red = reinterpret_cast<float *>(smem);
+        if (epi) {
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+                uint32_t v[16];
+                if (have_acc) {
+                    tmem_ld_32x32b_x16(t_row + c0, v);
+                    tmem_ld_wait();
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        v[j] = 0u;
+                }
+                if constexpr (SWAP) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        red[(c0 + j) * 128 + r] = __uint_as_float(v[j]);
+                } else {
+                    float4 *dst = reinterpret_cast<float4 *>(red + r * (BN + 4) + c0);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                             __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+                }
+            }
+        }
+        __syncwarp();
+        cluster_sync_all();
+        // 2. each CTA finishes 1/splits of the tile, summing the partials of
+        //    all CTAs of the cluster in rank order
+        const uint32_t red_addr = smem_u32(red);
+        const int S = p.splits;
+        const int rank = static_cast<int>(cluster_ctarank());
+        if (epi) {
+            // groups of 4 consecutive floats: SWAP: (token c, channels r..r+3);
+            // tiled: (token r, channels c..c+3)
+            constexpr int kGroups = 128 * BN / 4;
+            const int g0 = (rank * kGroups) / S, g1 = ((rank + 1) * kGroups) / S;
+            for (int g = g0 + et; g < g1; g += 128) {
+                int m, n;
+                uint32_t off;
+                if constexpr (SWAP) {
+                    const int c = g / 32, rr = (g % 32) * 4;
+                    m = row0_x + c;
+                    n = row0_w + rr;
+                    off = static_cast<uint32_t>((c * 128 + rr) * 4);
+                } else {
+                    const int rr = g / (BN / 4), c = (g % (BN / 4)) * 4;
+                    m = row0_x + rr;
+                    n = row0_w + c;
+                    off = static_cast<uint32_t>((rr * (BN + 4) + c) * 4);
+                }
+                if (m >= p.M || n >= p.N)
+                    continue;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int z = 0; z < S; ++z) {
+                    const float4 t = ld_shared_cluster_v4(map_shared_rank(red_addr + off, static_cast<uint32_t>(z)));
+                    acc.x += t.x;
+                    acc.y += t.y;
+                    acc.z += t.z;
+                    acc.w += t.w;
+                }
+                float a[4] = {acc.x, acc.y, acc.z, acc.w};
+                if constexpr (SWAP) {
+                    // 4 channels n..n+3 of token m
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        if constexpr (KIND != kNested16)
+                            a[j] = a[j] * p.sa[m];
+                        if constexpr (KIND == kE4M3)
+                            a[j] = a[j] * __ldg(p.sw + n + j);
+                    }
+                } else {
+                    float sam = 1.0f;
+                    if constexpr (KIND != kNested16)
+                        sam = p.sa[m];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        if constexpr (KIND != kNested16)
+                            a[j] = a[j] * sam;
+                        if constexpr (KIND == kE4M3)
+                            a[j] = a[j] * __ldg(p.sw + n + j);
+                    }
+                }
+                uint2 o;
+                o.x = pack2<KIND>(a[0], a[1]);
+                o.y = pack2<KIND>(a[2], a[3]);
+                *reinterpret_cast<uint2 *>(reinterpret_cast<uint16_t *>(p.y) + static_cast<int64_t>(m) * p.N + n) = o;
+            }
+        }
+        __syncwarp();
+        cluster_sync_all();   // no CTA leaves while its partial may still be read
+    }
+
+    // ---------------------------------------------------------------- teardown
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+} // namespace pgf8

@@ -1,0 +1,514 @@
+// C-ABI entry points of libpgf8: argument checks, kernel choice, tensor-map
+// encoding and launches.  The operations are specified in include/pgf8.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "pgf8.h"
+#include "gemm.cuh"
+#include "quantize.cuh"
+
+namespace pgf8 {
+
+static thread_local int tl_last_cuda_error = 0;
+
+static pgf8_status cuda_fail(cudaError_t e)
+{
+    tl_last_cuda_error = static_cast<int>(e);
+    return PGF8_ERR_CUDA;
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+static size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ------------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D row-major [rows, cols] tensor; box = box_cols x box_rows; element
+// size from dtype.  Out-of-range elements of a box read as zero.
+static bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem_bytes, uint64_t rows,
+                     uint64_t cols, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elem_bytes)};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ GEMM launch
+struct GemmLaunch {
+    int kind;          // OpKind
+    const void *x;     // E4M3 codes or FP16 activations [M, K]
+    const void *w;     // E4M3 codes or hi plane [N, K]
+    const void *w2;    // lo plane (kNested16)
+    const float *sa, *sw;
+    void *y;
+    int M, N, K;
+    int pdl;           // launch with programmatic stream serialization
+    int prefetch_w;    // weights may be read before the dependency resolves
+    pgf8_linear_opts opts;
+    cudaStream_t stream;
+};
+
+template <class C> static pgf8_status launch_cfg(const GemmLaunch &L, int splits)
+{
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    });
+    if (attr_err != cudaSuccess)
+        return cuda_fail(attr_err);
+
+    const bool nest16 = (C::KIND == kNested16);
+    CUtensorMap tmX, tmW, tmW2;
+    std::memset(&tmW2, 0, sizeof(tmW2));
+    bool ok;
+    if (nest16) {
+        ok = make_map(&tmX, L.x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, L.M, L.K, 64, C::kRowsX,
+                      CU_TENSOR_MAP_SWIZZLE_128B) &&
+             make_map(&tmW, L.w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.N, L.K, 64, C::kRowsW,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) &&
+             make_map(&tmW2, L.w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.N, L.K, 64, C::kRowsW,
+                      CU_TENSOR_MAP_SWIZZLE_NONE);
+    } else {
+        ok = make_map(&tmX, L.x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.M, L.K, 128, C::kRowsX,
+                      CU_TENSOR_MAP_SWIZZLE_128B) &&
+             make_map(&tmW, L.w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.N, L.K, 128, C::kRowsW,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+        tmW2 = tmW;
+    }
+    if (!ok)
+        return PGF8_ERR_UNSUPPORTED;
+
+    GemmParams p;
+    p.M = L.M;
+    p.N = L.N;
+    p.K = L.K;
+    p.kblocks = static_cast<int>((static_cast<int64_t>(L.K) * (nest16 ? 2 : 1) + 127) / 128);
+    p.splits = splits;
+    p.prefetch_w = L.prefetch_w;
+    p.sa = L.sa;
+    p.sw = L.sw;
+    p.y = L.y;
+
+    const int rows_a = C::SWAP ? L.N : L.M;   // A side: 128-row tiles
+    const int rows_b = C::SWAP ? L.M : L.N;   // B side: BN-row tiles
+    dim3 grid((rows_a + 127) / 128, (rows_b + C::BN - 1) / C::BN, splits);
+
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(C::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = L.stream;
+    cudaLaunchAttribute attrs[2];
+    int na = 0;
+    if (C::SPLIT) {
+        attrs[na].id = cudaLaunchAttributeClusterDimension;
+        attrs[na].val.clusterDim.x = 1;
+        attrs[na].val.clusterDim.y = 1;
+        attrs[na].val.clusterDim.z = static_cast<unsigned>(splits);
+        ++na;
+    }
+    if (L.pdl) {
+        attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attrs[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.attrs = attrs;
+    cfg.numAttrs = na;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel<C>, tmX, tmW, tmW2, p);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    return PGF8_OK;
+}
+
+template <int KIND, bool SWAP, int BN, int STAGES>
+static pgf8_status launch_split_or_not(const GemmLaunch &L, int splits)
+{
+    if (splits > 1)
+        return launch_cfg<GemmCfg<SWAP, BN, STAGES, KIND, true>>(L, splits);
+    return launch_cfg<GemmCfg<SWAP, BN, STAGES, KIND, false>>(L, 1);
+}
+
+static int num_sms()
+{
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms <= 0)
+            sms = 148;
+    }
+    return sms;
+}
+
+template <int KIND> static pgf8_status launch_gemm(const GemmLaunch &L)
+{
+    // argument checks first: nothing below may touch the device before they pass
+    const int elem = (KIND == kNested16) ? 2 : 1;
+    const int kblocks = static_cast<int>((static_cast<int64_t>(L.K) * elem + 127) / 128);
+    int path = L.opts.path;
+    int bn = L.opts.tile_n;
+    int splits = L.opts.split_k;
+    if (path == PGF8_PATH_AUTO)
+        path = (L.M <= 128) ? PGF8_PATH_SKINNY : PGF8_PATH_TILED;
+    if (path != PGF8_PATH_SKINNY && path != PGF8_PATH_TILED)
+        return PGF8_ERR_INVALID_ARG;
+    if (splits < 0 || splits > 8)
+        return PGF8_ERR_INVALID_ARG;
+    if (path == PGF8_PATH_SKINNY) {
+        if (L.M > 128)
+            return PGF8_ERR_UNSUPPORTED;
+        if (bn == 0)
+            bn = L.M <= 16 ? 16 : L.M <= 32 ? 32 : L.M <= 64 ? 64 : 128;
+        if (bn < L.M || (bn != 16 && bn != 32 && bn != 64 && bn != 128))
+            return PGF8_ERR_INVALID_ARG;
+    } else if (bn != 0 && bn != 128 && bn != 256) {
+        return PGF8_ERR_INVALID_ARG;
+    }
+
+    const int sms = (splits == 0 || bn == 0) ? num_sms() : 148;
+    if (path == PGF8_PATH_SKINNY) {
+        const int tiles = (L.N + 127) / 128;
+        if (splits == 0) {
+            // enough CTAs to cover every SM at least once; no more splits
+            // than needed (each split adds a partial-tile exchange)
+            splits = 1;
+            while (splits < 8 && tiles * splits < sms)
+                ++splits;
+        }
+        if (splits > kblocks)
+            splits = kblocks;
+        switch (bn) {
+        case 16: return launch_split_or_not<KIND, true, 16, 6>(L, splits);
+        case 32: return launch_split_or_not<KIND, true, 32, 8>(L, splits);
+        case 64: return launch_split_or_not<KIND, true, 64, 8>(L, splits);
+        default: return launch_split_or_not<KIND, true, 128, 6>(L, splits);
+        }
+    }
+    const int mt = (L.M + 127) / 128;
+    if (bn == 0)
+        bn = (mt * ((L.N + 255) / 256) >= sms) ? 256 : 128;
+    if (splits == 0) {
+        const int tiles = mt * ((L.N + bn - 1) / bn);
+        splits = 1;
+        while (splits < 4 && tiles * (splits + 1) <= sms)
+            ++splits;
+    }
+    if (splits > kblocks)
+        splits = kblocks;
+    if (bn == 256)
+        return launch_split_or_not<KIND, false, 256, 4>(L, splits);
+    return launch_split_or_not<KIND, false, 128, 6>(L, splits);
+}
+
+static pgf8_status check_dims(int64_t M, int64_t N, int64_t K)
+{
+    if (M < 1 || N < 16 || K < 16 || M > (1ll << 30) || N > (1ll << 30) || K > (1ll << 30))
+        return PGF8_ERR_INVALID_ARG;
+    if (K % 16 != 0 || N % 16 != 0)
+        return PGF8_ERR_ALIGNMENT;
+    return PGF8_OK;
+}
+
+static pgf8_linear_opts opts_or_default(const pgf8_linear_opts *o)
+{
+    pgf8_linear_opts d;
+    std::memset(&d, 0, sizeof(d));
+    if (o)
+        d = *o;
+    return d;
+}
+
+static pgf8_status quantize_launch(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
+                                   uint8_t *q, float *scales, int mode, cudaStream_t st)
+{
+    if (rows == 0)
+        return PGF8_OK;
+    dim3 grid(static_cast<unsigned>(rows));
+    if (xdt == PGF8_F32)
+        quantize_rows_kernel<float><<<grid, kQuantThreads, 0, st>>>(static_cast<const float *>(x), rows, cols, ldx,
+                                                                     q, scales, mode);
+    else
+        quantize_rows_kernel<__half><<<grid, kQuantThreads, 0, st>>>(static_cast<const __half *>(x), rows, cols,
+                                                                      ldx, q, scales, mode);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    return PGF8_OK;
+}
+
+static pgf8_status check_quantize_args(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
+                                       const uint8_t *q, const float *scales, int mode)
+{
+    if (!x || !q || !scales || rows < 0 || cols < 16 || ldx < cols || rows > (1ll << 31) - 1)
+        return PGF8_ERR_INVALID_ARG;
+    if (xdt != PGF8_F32 && xdt != PGF8_F16)
+        return PGF8_ERR_UNSUPPORTED;
+    if (mode != PGF8_SCALE_DYNAMIC && mode != PGF8_SCALE_STATIC)
+        return PGF8_ERR_INVALID_ARG;
+    const int eb = xdt == PGF8_F32 ? 4 : 2;
+    if (cols % 16 != 0 || (ldx * eb) % 16 != 0 || !aligned16(x) || !aligned16(q) || !aligned4(scales))
+        return PGF8_ERR_ALIGNMENT;
+    return PGF8_OK;
+}
+
+} // namespace pgf8
+
+using namespace pgf8;
+
+extern "C" {
+
+pgf8_status pgf8_fp8_quantize_rows(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
+                                   uint8_t *q, float *scales, pgf8_scale_mode mode, void *stream)
+{
+    pgf8_status st = check_quantize_args(x, xdt, rows, cols, ldx, q, scales, mode);
+    if (st != PGF8_OK)
+        return st;
+    return quantize_launch(x, xdt, rows, cols, ldx, q, scales, static_cast<int>(mode),
+                           static_cast<cudaStream_t>(stream));
+}
+
+size_t pgf8_fp8_linear_workspace_size(int64_t, int64_t, int64_t) { return 0; }
+
+pgf8_status pgf8_fp8_linear_ex(const uint8_t *aq, const float *sa, int64_t M, int64_t K, const uint8_t *wq,
+                               const float *sw, int64_t N, void *y, void *, size_t, const pgf8_linear_opts *opts,
+                               void *stream)
+{
+    pgf8_status st = check_dims(M, N, K);
+    if (st != PGF8_OK)
+        return st;
+    if (!aq || !sa || !wq || !sw || !y)
+        return PGF8_ERR_INVALID_ARG;
+    if (!aligned16(aq) || !aligned16(wq) || !aligned16(y) || !aligned4(sa) || !aligned4(sw))
+        return PGF8_ERR_ALIGNMENT;
+    GemmLaunch L;
+    L.kind = kE4M3;
+    L.x = aq;
+    L.w = wq;
+    L.w2 = nullptr;
+    L.sa = sa;
+    L.sw = sw;
+    L.y = y;
+    L.M = static_cast<int>(M);
+    L.N = static_cast<int>(N);
+    L.K = static_cast<int>(K);
+    L.pdl = 1;
+    L.prefetch_w = 0;
+    L.opts = opts_or_default(opts);
+    L.stream = static_cast<cudaStream_t>(stream);
+    return launch_gemm<kE4M3>(L);
+}
+
+pgf8_status pgf8_fp8_linear(const uint8_t *aq, const float *sa, int64_t M, int64_t K, const uint8_t *wq,
+                            const float *sw, int64_t N, void *y, void *workspace, size_t workspace_bytes,
+                            void *stream)
+{
+    return pgf8_fp8_linear_ex(aq, sa, M, K, wq, sw, N, y, workspace, workspace_bytes, nullptr, stream);
+}
+
+size_t pgf8_fp8_linear_dynamic_scales_offset(int64_t M, int64_t K)
+{
+    if (M < 0 || K < 0)
+        return 0;
+    return round_up(static_cast<size_t>(M) * static_cast<size_t>(K), 256);
+}
+
+size_t pgf8_fp8_linear_dynamic_workspace_size(int64_t M, int64_t, int64_t K)
+{
+    if (M < 0 || K < 0)
+        return 0;
+    return pgf8_fp8_linear_dynamic_scales_offset(M, K) + round_up(static_cast<size_t>(M) * 4, 256);
+}
+
+static pgf8_status linear_dynamic_impl(const void *x, pgf8_dtype xdt, int64_t M, int64_t K, int64_t ldx,
+                                       const void *w, const void *w2, const float *sw, int64_t N, void *y,
+                                       void *workspace, size_t workspace_bytes, const pgf8_linear_opts *opts,
+                                       void *stream, int kind)
+{
+    pgf8_status st = check_dims(M, N, K);
+    if (st != PGF8_OK)
+        return st;
+    if (!workspace || !w || !y || (kind == kE4M3 && !sw))
+        return PGF8_ERR_INVALID_ARG;
+    if (workspace_bytes < pgf8_fp8_linear_dynamic_workspace_size(M, N, K))
+        return PGF8_ERR_INVALID_ARG;
+    if (!aligned16(workspace) || !aligned16(w) || !aligned16(y) || (sw && !aligned4(sw)))
+        return PGF8_ERR_ALIGNMENT;
+    uint8_t *aq = static_cast<uint8_t *>(workspace);
+    float *sa = reinterpret_cast<float *>(aq + pgf8_fp8_linear_dynamic_scales_offset(M, K));
+    st = check_quantize_args(x, xdt, M, K, ldx, aq, sa, PGF8_SCALE_DYNAMIC);
+    if (st != PGF8_OK)
+        return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    st = quantize_launch(x, xdt, M, K, ldx, aq, sa, 0, cs);
+    if (st != PGF8_OK)
+        return st;
+    GemmLaunch L;
+    L.kind = kind;
+    L.x = aq;
+    L.w = w;
+    L.w2 = w2;
+    L.sa = sa;
+    L.sw = sw;
+    L.y = y;
+    L.M = static_cast<int>(M);
+    L.N = static_cast<int>(N);
+    L.K = static_cast<int>(K);
+    L.pdl = 1;
+    L.prefetch_w = 1;   // the quantisation kernel writes only aq / sa
+    L.opts = opts_or_default(opts);
+    L.stream = cs;
+    if (kind == kNested8)
+        return launch_gemm<kNested8>(L);
+    return launch_gemm<kE4M3>(L);
+}
+
+pgf8_status pgf8_fp8_linear_dynamic(const void *x, pgf8_dtype xdt, int64_t M, int64_t K, int64_t ldx,
+                                    const uint8_t *wq, const float *sw, int64_t N, void *y, void *workspace,
+                                    size_t workspace_bytes, const pgf8_linear_opts *opts, void *stream)
+{
+    return linear_dynamic_impl(x, xdt, M, K, ldx, wq, nullptr, sw, N, y, workspace, workspace_bytes, opts, stream,
+                               kE4M3);
+}
+
+pgf8_status pgf8_nestedfp_split(const void *w, int64_t N, int64_t K, uint8_t *hi, uint8_t *lo, void *stream)
+{
+    if (!w || !hi || !lo || N < 0 || K < 0)
+        return PGF8_ERR_INVALID_ARG;
+    const int64_t count = N * K;
+    if (count % 8 != 0 || !aligned16(w) || !aligned16(hi) || !aligned16(lo))
+        return PGF8_ERR_ALIGNMENT;
+    if (count == 0)
+        return PGF8_OK;
+    const int64_t n8 = count / 8;
+    const int64_t blocks_needed = (n8 + 255) / 256;
+    const unsigned grid = static_cast<unsigned>(blocks_needed < 148 * 16 ? blocks_needed : 148 * 16);
+    nestedfp_split_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4 *>(w), n8, reinterpret_cast<uint2 *>(hi), reinterpret_cast<uint2 *>(lo));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    return PGF8_OK;
+}
+
+size_t pgf8_nestedfp_linear_workspace_size(int64_t M, int64_t N, int64_t K, pgf8_nested_mode mode)
+{
+    if (mode == PGF8_NESTED_FP8)
+        return pgf8_fp8_linear_dynamic_workspace_size(M, N, K);
+    return 0;
+}
+
+pgf8_status pgf8_nestedfp_linear_ex(const void *x, int64_t M, int64_t K, const uint8_t *hi, const uint8_t *lo,
+                                    int64_t N, pgf8_nested_mode mode, void *y, void *workspace,
+                                    size_t workspace_bytes, const pgf8_linear_opts *opts, void *stream)
+{
+    if (mode == PGF8_NESTED_FP8)
+        return linear_dynamic_impl(x, PGF8_F16, M, K, K, hi, nullptr, nullptr, N, y, workspace, workspace_bytes,
+                                   opts, stream, kNested8);
+    if (mode != PGF8_NESTED_FP16)
+        return PGF8_ERR_INVALID_ARG;
+    pgf8_status st = check_dims(M, N, K);
+    if (st != PGF8_OK)
+        return st;
+    if (!x || !hi || !lo || !y)
+        return PGF8_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(hi) || !aligned16(lo) || !aligned16(y))
+        return PGF8_ERR_ALIGNMENT;
+    GemmLaunch L;
+    L.kind = kNested16;
+    L.x = x;
+    L.w = hi;
+    L.w2 = lo;
+    L.sa = nullptr;
+    L.sw = nullptr;
+    L.y = y;
+    L.M = static_cast<int>(M);
+    L.N = static_cast<int>(N);
+    L.K = static_cast<int>(K);
+    L.pdl = 1;
+    L.prefetch_w = 0;
+    L.opts = opts_or_default(opts);
+    L.stream = static_cast<cudaStream_t>(stream);
+    return launch_gemm<kNested16>(L);
+}
+
+pgf8_status pgf8_nestedfp_linear(const void *x, int64_t M, int64_t K, const uint8_t *hi, const uint8_t *lo,
+                                 int64_t N, pgf8_nested_mode mode, void *y, void *workspace, size_t workspace_bytes,
+                                 void *stream)
+{
+    return pgf8_nestedfp_linear_ex(x, M, K, hi, lo, N, mode, y, workspace, workspace_bytes, nullptr, stream);
+}
+
+pgf8_status pgf8_last_cuda_error(int *cuda_err)
+{
+    if (!cuda_err)
+        return PGF8_ERR_INVALID_ARG;
+    *cuda_err = tl_last_cuda_error;
+    return PGF8_OK;
+}
+
+pgf8_status pgf8_device_status(void *stream)
+{
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    unsigned int v = 0;
+    e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v));
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    if (v != 0) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+        if (e != cudaSuccess)
+            return cuda_fail(e);
+        return PGF8_ERR_TIMEOUT;
+    }
+    return PGF8_OK;
+}
+
+const char *pgf8_status_str(pgf8_status s)
+{
+    switch (s) {
+    case PGF8_OK: return "ok";
+    case PGF8_ERR_INVALID_ARG: return "invalid argument";
+    case PGF8_ERR_ALIGNMENT: return "alignment or divisibility requirement violated";
+    case PGF8_ERR_UNSUPPORTED: return "unsupported configuration";
+    case PGF8_ERR_CUDA: return "CUDA error";
+    case PGF8_ERR_TIMEOUT: return "device-side bounded wait expired";
+    }
+    return "unknown status";
+}
+
+int pgf8_version(void) { return 100; }
+
+} // extern "C"

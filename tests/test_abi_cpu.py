@@ -1,0 +1,112 @@
+"""The C-ABI library builds, loads and exports every declared symbol, and its
+host-side argument checks reject bad calls before anything touches a GPU
+(CPU only: no call here reaches a CUDA runtime function)."""
+import ctypes
+import subprocess
+
+import pytest
+
+import precision_gemm_fp8_b200 as pg
+
+
+def test_every_declared_symbol_is_exported():
+    names = pg.header_symbols()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(pg.lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", pg.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+
+
+def test_status_strings_and_version():
+    for s in range(6):
+        assert pg.lib.pgf8_status_str(s)
+    assert pg.lib.pgf8_status_str(99) == b"unknown status"
+    assert pg.version() >= 100
+
+
+def test_workspace_sizes():
+    assert pg.lib.pgf8_fp8_linear_workspace_size(16, 512, 512) == 0
+    off = pg.lib.pgf8_fp8_linear_dynamic_scales_offset(3, 4096)
+    assert off % 256 == 0 and off >= 3 * 4096
+    ws = pg.lib.pgf8_fp8_linear_dynamic_workspace_size(3, 4096, 4096)
+    assert ws >= off + 12 and ws % 256 == 0
+    assert pg.nestedfp_linear_workspace_size(8, 4096, 4096, pg.NESTED_FP16) == 0
+    assert pg.nestedfp_linear_workspace_size(8, 4096, 4096, pg.NESTED_FP8) == \
+        pg.lib.pgf8_fp8_linear_dynamic_workspace_size(8, 4096, 4096)
+
+
+def test_last_cuda_error_starts_clear():
+    e = ctypes.c_int(-1)
+    assert pg.lib.pgf8_last_cuda_error(ctypes.byref(e)) == pg.OK
+    assert e.value == 0
+    assert pg.lib.pgf8_last_cuda_error(None) == pg.ERR_INVALID_ARG
+
+
+A16 = 0x10000      # fake, 16-byte aligned addresses: argument checks fail before use
+B16 = 0x20000
+C16 = 0x30000
+D16 = 0x40000
+MIS = 0x10008      # 8-byte aligned only
+
+
+@pytest.mark.parametrize("M,N,K,expect", [
+    (0, 512, 512, pg.ERR_INVALID_ARG),      # M >= 1
+    (16, 8, 512, pg.ERR_INVALID_ARG),       # N >= 16
+    (16, 512, 8, pg.ERR_INVALID_ARG),       # K >= 16
+    (16, 520, 512, pg.ERR_ALIGNMENT),       # N % 16
+    (16, 512, 520, pg.ERR_ALIGNMENT),       # K % 16
+])
+def test_fp8_linear_rejects_bad_dims(M, N, K, expect):
+    st = pg.lib.pgf8_fp8_linear(A16, B16, M, K, C16, D16, N, A16, None, 0, None)
+    assert st == expect
+
+
+def test_fp8_linear_rejects_null_and_misaligned():
+    assert pg.lib.pgf8_fp8_linear(None, B16, 16, 512, C16, D16, 512, A16, None, 0, None) == pg.ERR_INVALID_ARG
+    assert pg.lib.pgf8_fp8_linear(A16, B16, 16, 512, C16, D16, 512, None, None, 0, None) == pg.ERR_INVALID_ARG
+    assert pg.lib.pgf8_fp8_linear(MIS, B16, 16, 512, C16, D16, 512, A16, None, 0, None) == pg.ERR_ALIGNMENT
+    assert pg.lib.pgf8_fp8_linear(A16, B16, 16, 512, MIS, D16, 512, A16, None, 0, None) == pg.ERR_ALIGNMENT
+    assert pg.lib.pgf8_fp8_linear(A16, B16 + 2, 16, 512, C16, D16, 512, A16, None, 0, None) == pg.ERR_ALIGNMENT
+
+
+def test_fp8_linear_rejects_bad_options():
+    bad = [pg.LinearOpts(7, 0, 0, 0), pg.LinearOpts(pg.PATH_SKINNY, 9, 0, 0),
+           pg.LinearOpts(pg.PATH_SKINNY, 0, 48, 0), pg.LinearOpts(pg.PATH_TILED, 0, 64, 0),
+           pg.LinearOpts(pg.PATH_SKINNY, 0, 16, 0)]
+    Ms = [16, 16, 16, 16, 17]   # the last: tile_n 16 cannot hold 17 tokens
+    for o, M in zip(bad, Ms):
+        st = pg.lib.pgf8_fp8_linear_ex(A16, B16, M, 512, C16, D16, 512, A16, None, 0, ctypes.byref(o), None)
+        assert st in (pg.ERR_INVALID_ARG, pg.ERR_UNSUPPORTED), (o.path, o.split_k, o.tile_n, st)
+    big = pg.LinearOpts(pg.PATH_SKINNY, 0, 0, 0)
+    assert pg.lib.pgf8_fp8_linear_ex(A16, B16, 129, 512, C16, D16, 512, A16, None, 0, ctypes.byref(big),
+                                     None) == pg.ERR_UNSUPPORTED
+
+
+def test_quantize_rejects_bad_args():
+    q = pg.lib.pgf8_fp8_quantize_rows
+    assert q(None, pg.F32, 4, 64, 64, B16, C16, 0, None) == pg.ERR_INVALID_ARG
+    assert q(A16, pg.BF16, 4, 64, 64, B16, C16, 0, None) == pg.ERR_UNSUPPORTED
+    assert q(A16, pg.F32, 4, 60, 64, B16, C16, 0, None) == pg.ERR_ALIGNMENT      # cols % 16
+    assert q(A16, pg.F32, 4, 8, 64, B16, C16, 0, None) == pg.ERR_INVALID_ARG      # cols >= 16
+    assert q(A16, pg.F32, 4, 64, 32, B16, C16, 0, None) == pg.ERR_INVALID_ARG    # ldx < cols
+    assert q(A16, pg.F32, 4, 64, 66, B16, C16, 0, None) == pg.ERR_ALIGNMENT      # row stride not 16 B
+    assert q(MIS, pg.F32, 4, 64, 64, B16, C16, 0, None) == pg.ERR_ALIGNMENT
+    assert q(A16, pg.F32, 4, 64, 64, B16, C16 + 2, 0, None) == pg.ERR_ALIGNMENT
+    assert q(A16, pg.F32, 4, 64, 64, B16, C16, 5, None) == pg.ERR_INVALID_ARG
+
+
+def test_dynamic_and_nested_reject_bad_args():
+    d = pg.lib.pgf8_fp8_linear_dynamic
+    small_ws = 16
+    assert d(A16, pg.F32, 4, 512, 512, B16, C16, 512, D16, A16, small_ws, None, None) == pg.ERR_INVALID_ARG
+    assert d(A16, pg.F32, 4, 512, 512, B16, C16, 512, D16, None, 1 << 20, None, None) == pg.ERR_INVALID_ARG
+    n = pg.lib.pgf8_nestedfp_linear
+    assert n(A16, 4, 512, B16, None, 512, pg.NESTED_FP16, D16, None, 0, None) == pg.ERR_INVALID_ARG
+    assert n(A16, 4, 512, B16, C16, 512, 7, D16, None, 0, None) == pg.ERR_INVALID_ARG
+    assert n(A16, 4, 512, B16, None, 512, pg.NESTED_FP8, D16, None, 0, None) == pg.ERR_INVALID_ARG
+    s = pg.lib.pgf8_nestedfp_split
+    assert s(None, 16, 16, B16, C16, None) == pg.ERR_INVALID_ARG
+    assert s(A16, 3, 5, B16, C16, None) == pg.ERR_ALIGNMENT

@@ -1,0 +1,116 @@
+"""GPU parity of the NestedFP linear layer in both modes against the oracle
+(FP16 mode: weights rebuilt from (hi << 8) | lo; FP8 mode: hi read as E5M2,
+activations per-token E4M3), within the layer's stated bound."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from _parity import E4, E5, assert_within, fp8_row_max, linear_bound
+
+pg = pytest.importorskip("precision_gemm_fp8_b200")
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _to(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+
+def _ref16(x16, hi, lo):
+    ref = oracle.nestedfp_linear_fp16(x16, hi, lo)
+    w = ((hi.astype(np.uint16) << 8) | lo.astype(np.uint16)).view(np.float16).astype(np.float64)
+    a_hat = np.abs(x16.astype(np.float64)).max(axis=1)
+    w_hat = np.abs(w).max(axis=1)
+    return ref, linear_bound(ref, x16.shape[1], a_hat, w_hat)
+
+
+def _ref8(x16, hi):
+    ref, aq, sa = oracle.nestedfp_linear_fp8(x16, hi)
+    w_hat = np.abs(E5[hi]).max(axis=1)
+    return ref, linear_bound(ref, x16.shape[1], fp8_row_max(aq, sa), w_hat), aq, sa
+
+
+def _run(x16, hi, lo, mode, **kw):
+    y = pg.nestedfp_linear(_to(x16), _to(hi), _to(lo) if lo is not None else None, mode=mode, **kw)
+    torch.cuda.synchronize()
+    assert pg.device_status() == pg.OK
+    return y.float().cpu().numpy()
+
+
+RAGGED = [(1, 16, 16), (5, 48, 144), (16, 272, 528), (17, 144, 1040), (128, 256, 256), (130, 272, 400),
+          (257, 528, 192)]
+
+
+@pytest.mark.parametrize("M,N,K", RAGGED)
+def test_nested_fp16_ragged(M, N, K):
+    g = np.random.default_rng(M * 31 + N * 7 + K)
+    x16 = synthetic.activations("normal_f16", M, K, g)
+    w16 = synthetic.weights_f16(N, K, 0.02, g)
+    hi, lo = oracle.nestedfp_split(w16)
+    ref, bound = _ref16(x16, hi, lo)
+    configs = [{"path": pg.PATH_TILED}, {"path": pg.PATH_TILED, "split_k": 2}, {"path": pg.PATH_TILED, "tile_n": 256}]
+    if M <= 128:
+        configs += [{"path": pg.PATH_SKINNY}, {"path": pg.PATH_SKINNY, "split_k": 3}]
+    for kw in configs:
+        assert_within(_run(x16, hi, lo, pg.NESTED_FP16, **kw), ref, bound, f"fp16 M{M} N{N} K{K} {kw}")
+
+
+@pytest.mark.parametrize("M,N,K", RAGGED)
+def test_nested_fp8_ragged(M, N, K):
+    g = np.random.default_rng(M * 37 + N * 11 + K)
+    x16 = synthetic.activations("normal_f16", M, K, g)
+    w16 = synthetic.weights_f16(N, K, 0.02, g)
+    hi, _ = oracle.nestedfp_split(w16)
+    ref, bound, _, _ = _ref8(x16, hi)
+    configs = [{"path": pg.PATH_TILED}, {"path": pg.PATH_TILED, "split_k": 2}]
+    if M <= 128:
+        configs += [{"path": pg.PATH_SKINNY}, {"path": pg.PATH_SKINNY, "split_k": 4}]
+    for kw in configs:
+        assert_within(_run(x16, hi, None, pg.NESTED_FP8, **kw), ref, bound, f"fp8 M{M} N{N} K{K} {kw}")
+
+
+def test_nested_fp16_identity_weights():
+    """W = identity (FP16 1.0 = 0x3C00 -> hi 0x3C, lo 0x00) plus a subnormal
+    off-diagonal carried only by the lo plane: pins the hi/lo interleave and
+    the swizzled layout of the rebuild (any mis-placed byte breaks the bound)."""
+    K = 256
+    g = np.random.default_rng(3)
+    x16 = synthetic.activations("normal_f16", 40, K, g)
+    w = np.zeros((K, K), dtype=np.float16)
+    w[np.arange(K), np.arange(K)] = 1.0
+    w[np.arange(K), (np.arange(K) + 1) % K] = np.float16(2.0 ** -20)   # exercises lo bits (subnormal)
+    hi, lo = oracle.nestedfp_split(w)
+    ref, bound = _ref16(x16, hi, lo)
+    for kw in ({"path": pg.PATH_TILED}, {"path": pg.PATH_SKINNY}):
+        y = _run(x16, hi, lo, pg.NESTED_FP16, **kw)
+        assert_within(y, ref, bound, str(kw))
+
+
+@pytest.mark.parametrize("shape_idx", [0, 1])
+@pytest.mark.parametrize("m_idx", [0, 1, 2, 3])
+def test_nested7b_full_size_both_modes(shape_idx, m_idx):
+    """Both modes on the same stored planes at the workload's sizes, checked
+    on sampled rows and columns."""
+    x16 = synthetic.acts("nested7b", shape_idx, m_idx)
+    w16 = synthetic.weights("nested7b", shape_idx)
+    M, K = x16.shape
+    N = w16.shape[0]
+    hi_g, lo_g = pg.nestedfp_split(_to(w16))
+    xt = _to(x16)
+    y16 = pg.nestedfp_linear(xt, hi_g, lo_g, mode=pg.NESTED_FP16)
+    y8 = pg.nestedfp_linear(xt, hi_g, None, mode=pg.NESTED_FP8)
+    torch.cuda.synchronize()
+    assert pg.device_status() == pg.OK
+    rng = np.random.default_rng(1)
+    ns = np.sort(rng.choice(N, 256, replace=False))
+    ms = np.sort(rng.choice(M, min(M, 12), replace=False))
+    hi, lo = oracle.nestedfp_split(w16[ns])
+    np.testing.assert_array_equal(hi_g.cpu().numpy()[ns], hi)
+    np.testing.assert_array_equal(lo_g.cpu().numpy()[ns], lo)
+    ref, bound = _ref16(x16[ms], hi, lo)
+    assert_within(y16.float().cpu().numpy()[np.ix_(ms, ns)], ref, bound, f"fp16 full M={M}")
+    ref8, bound8, _, _ = _ref8(x16[ms], hi)
+    assert_within(y8.float().cpu().numpy()[np.ix_(ms, ns)], ref8, bound8, f"fp8 full M={M}")
