@@ -1,0 +1,591 @@
+"""Benchmark of the FP8 linear layer hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode7b|prefill7b|nested7b|llama70b|small]
+
+A step is one pass of the hot path over one batch of synthetic inputs: for
+every (M, shape) layer of the workload, dynamic per-token E4M3 quantisation
+of the activations followed by the FP8 GEMM with fused dequantisation
+(weights were quantised per output channel once, at set-up, with the same
+kernel).  The default workload is the Llama-7B decode linears (QKV
+4096->12288, O 4096->4096, gate+up 4096->22016, down 11008->4096 at
+M = 1, 4, 8); every layer reads its own weight copy, so one step streams
+606 MB of FP8 weights, more than the 126 MB L2, and no weight is L2-resident
+when it is read.
+
+Timing: the K timed steps are replayed from a CUDA graph (captured from the
+library's own C-ABI calls) between a barrier + synchronize on both sides,
+CUDA events on the launching stream, max over ranks.  Per-GEMM durations
+for the roofline come from event pairs captured around every GEMM launch of
+the last replayed steps.  `e2e` repeats the metric through the public entry
+point (fp8_linear_dynamic) with the activations copied from pinned host
+memory and the outputs copied back inside the timed region.  `cpu_baseline`
+times the CPU oracle on a bounded sample of the same workload.
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+METRIC = None
+try:
+    with open(os.path.join(ROOT, "BASELINE.json")) as _f:
+        METRIC = json.load(_f)["metric"]
+except Exception:
+    METRIC = "FP8 linear TFLOPS & weight GB/s vs B200 roofline, 7B/70B shapes, M=1–4096"
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+WORKLOAD_TEXT = {
+    "decode7b": "Llama-7B decode linears: QKV 4096->12288, O 4096->4096, gate+up 4096->22016, "
+                "down 11008->4096 at M=1,4,8 tokens; dynamic per-token E4M3 activations "
+                "(N(0,1), 0.5% x30 outliers), static per-channel E4M3 weights (N(0,0.02)), bf16 out",
+    "prefill7b": "Llama-7B prefill linears: same four shapes at M=512,1024,2048; Student-t(4)/sqrt2 "
+                 "activations; bf16 out",
+    "llama70b": "Llama-70B linears: QKV 8192->10240, O 8192->8192, gate+up 8192->57344, down 28672->8192 "
+                "at M=1..4096; Student-t(3) activations; bf16 out",
+    "small": "single FP8 linear 16x512x512",
+    "nested7b": "NestedFP 7B: 4096->12288 and 11008->4096 at M=1,16,128,1024, FP16 and FP8 modes on the "
+                "same hi/lo planes; fp16 out",
+}
+
+
+def _load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- layers
+class Layer:
+    """One (M, shape, weight copy) layer of a workload."""
+
+    def __init__(self, kind, M, K, N, shape_idx, m_idx, copy):
+        self.kind, self.M, self.K, self.N = kind, M, K, N
+        self.shape_idx, self.m_idx, self.copy = shape_idx, m_idx, copy
+
+    @property
+    def flops(self):
+        return 2.0 * self.M * self.N * self.K
+
+    @property
+    def weight_bytes(self):
+        return self.N * self.K * (2 if self.kind == "nested16" else 1)
+
+    @property
+    def gemm_bytes(self):
+        """Algorithmic bytes of one GEMM launch: weights once, activations once,
+        scales, output once."""
+        if self.kind == "fp8":
+            return self.N * self.K + self.M * self.K + 4 * self.M + 4 * self.N + 2 * self.M * self.N
+        if self.kind == "nested8":
+            return self.N * self.K + self.M * self.K + 4 * self.M + 2 * self.M * self.N
+        return 2 * self.N * self.K + 2 * self.M * self.K + 2 * self.M * self.N
+
+
+def workload_layers(name, copies):
+    wl = synthetic.WORKLOADS[name]
+    layers = []
+    if name == "nested7b":
+        for mi, M in enumerate(wl.ms):
+            for si, (K, N, _) in enumerate(wl.shapes):
+                for kind in ("nested16", "nested8"):
+                    layers.append(Layer(kind, M, K, N, si, mi, 0))
+        return layers
+    for mi, M in enumerate(wl.ms):
+        for si, (K, N, _) in enumerate(wl.shapes):
+            layers.append(Layer("fp8", M, K, N, si, mi, mi % copies))
+    return layers
+
+
+def weight_copies(name):
+    # enough distinct weight copies that a step streams more than 3 x L2
+    return {"decode7b": 3, "small": 1}.get(name, 1)
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(prefix="pgf8_clocks_", suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        load = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import precision_gemm_fp8_b200 as pg
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = _load_peaks()
+    name = args.workload
+    copies = weight_copies(name)
+    layers = workload_layers(name, copies)
+    wl = synthetic.WORKLOADS[name]
+
+    # ---- set-up (untimed): weights quantised per channel on the device, activations resident
+    weights = {}
+    for L in layers:
+        key = (L.shape_idx, L.copy, L.kind in ("nested16", "nested8"))
+        if key in weights:
+            continue
+        w = torch.from_numpy(synthetic.weights(name, L.shape_idx, copy=L.copy)).to(dev)
+        if key[2]:
+            weights[key] = pg.nestedfp_split(w)
+        else:
+            weights[key] = pg.fp8_quantize_rows(w)
+        del w
+    acts_host, acts, outs, qbufs = [], [], [], []
+    for L in layers:
+        x = synthetic.acts(name, L.shape_idx, L.m_idx)
+        xh = torch.from_numpy(x).pin_memory()
+        acts_host.append(xh)
+        acts.append(xh.to(dev))
+        out_dt = torch.float16 if L.kind.startswith("nested") else torch.bfloat16
+        outs.append(torch.empty((L.M, L.N), dtype=out_dt, device=dev))
+        if L.kind == "fp8":
+            qbufs.append((torch.empty((L.M, L.K), dtype=torch.uint8, device=dev),
+                          torch.empty((L.M,), dtype=torch.float32, device=dev)))
+        elif L.kind == "nested8":
+            qbufs.append(torch.empty(pg.nestedfp_linear_workspace_size(L.M, L.N, L.K, pg.NESTED_FP8),
+                                     dtype=torch.uint8, device=dev))
+        else:
+            qbufs.append(None)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def enqueue_step(ev_pairs=None):
+        """One step through the C ABI on `stream`; optional event pairs bracket each GEMM."""
+        for i, L in enumerate(layers):
+            W = weights[(L.shape_idx, L.copy, L.kind != "fp8")]
+            if L.kind == "fp8":
+                aq, sa = qbufs[i]
+                pg.fp8_quantize_rows(acts[i], aq, sa, stream=stream)
+                if ev_pairs is not None:
+                    ev_pairs[i][0].record(stream)
+                pg.fp8_linear(aq, sa, W[0], W[1], y=outs[i], stream=stream)
+                if ev_pairs is not None:
+                    ev_pairs[i][1].record(stream)
+            else:
+                mode = pg.NESTED_FP16 if L.kind == "nested16" else pg.NESTED_FP8
+                if ev_pairs is not None:
+                    ev_pairs[i][0].record(stream)
+                pg.nestedfp_linear(acts[i], W[0], W[1] if mode == pg.NESTED_FP16 else None, mode=mode,
+                                   y=outs[i], workspace=qbufs[i], stream=stream)
+                if ev_pairs is not None:
+                    ev_pairs[i][1].record(stream)
+
+    launches_per_step = sum(2 if L.kind in ("fp8", "nested8") else 1 for L in layers)
+
+    # ---- graphs: R steps with per-GEMM events, replayed K / R times
+    K, W = args.steps, args.warmup
+    R = max(1, min(10, K))
+    while K % R:
+        R -= 1
+    evs = [[(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+            for _ in layers] for _ in range(R)]
+    with torch.cuda.stream(stream):
+        enqueue_step()          # load modules / first-call set-up outside capture
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for r in range(R):
+            enqueue_step(evs[r])
+    for _ in range(W):
+        graph.replay()
+    torch.cuda.synchronize()
+    if pg.device_status(stream) != pg.OK:
+        raise RuntimeError("device error word raised during warm-up")
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(K // R):
+        graph.replay()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    ms_total = t0.elapsed_time(t1)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    st = pg.device_status(stream)
+    if st != pg.OK:
+        raise RuntimeError(f"device error word raised in the timed region: {st}")
+
+    # per-GEMM durations (ms) of the last R replayed steps
+    gemm_ms = np.array([[evs[r][i][0].elapsed_time(evs[r][i][1]) for i in range(len(layers))] for r in range(R)])
+    per_layer_ms = gemm_ms.mean(axis=0)
+
+    ms_step = ms_total / K
+    wbytes = sum(L.weight_bytes for L in layers)
+    flops = sum(L.flops for L in layers)
+    gbs = wbytes / (ms_step * 1e-3) / 1e9
+    tflops = flops / (ms_step * 1e-3) / 1e12
+
+    # roofline of the dominant kernel (the GEMM)
+    gemm_bytes = sum(L.gemm_bytes for L in layers)
+    gemm_flops = sum(L.flops for L in layers)
+    gemm_time_s = per_layer_ms.sum() * 1e-3
+    memory_bound = name in ("decode7b", "small")
+    if memory_bound:
+        achieved = gemm_bytes / gemm_time_s / 1e9
+        peak = float(peaks["hbm_gbs"])
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": None,
+                "peak_source": f"{peak_src} HBM copy bandwidth"}
+    else:
+        achieved = gemm_flops / gemm_time_s / 1e12
+        peak = 2.0 * float(peaks["bf16_tflops"])
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": None,
+                "peak_source": f"{peak_src} bf16 burst x 2 (FP8 nominal ratio)"}
+    roof["kernel"] = "pgf8::gemm_kernel"
+    roof["launches_timed"] = int(R * len(layers))
+
+    per_layer = []
+    for L, t in zip(layers, per_layer_ms):
+        per_layer.append({"kind": L.kind, "M": L.M, "K": L.K, "N": L.N, "us": round(t * 1e3, 2),
+                          "gbs": round(L.gemm_bytes / (t * 1e-3) / 1e9, 1),
+                          "tflops": round(L.flops / (t * 1e-3) / 1e12, 1)})
+
+    # ---- e2e through the public entry point, host buffers, copies inside the timed region
+    e2e = run_e2e(pg, torch, dev, layers, weights, acts_host, outs, args, world, wbytes, flops, memory_bound)
+
+    result = {
+        "metric": METRIC,
+        "value": round((gbs if memory_bound else tflops) * world, 2),
+        "unit": "GB/s" if memory_bound else "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp8e4m3" if name != "nested7b" else "fp16+fp8e4m3/e5m2",
+        "data": "synthetic",
+        "config": {"workload": f"{name}: {WORKLOAD_TEXT[name]}",
+                   "l2": "inputs larger than L2 (%d weight copies; %.0f MB of weights streamed per step)"
+                         % (copies, wbytes / 1e6),
+                   "timing": "CUDA graph of the C-ABI calls, K/R replays of R steps"},
+        "secondary": {"tflops": round(tflops * world, 3), "weight_gbs": round(gbs * world, 1)},
+        "roofline": roof,
+        "e2e": e2e,
+        "gpu_launches": int(launches_per_step * K),
+        "clocks": clocks,
+        "per_layer": per_layer,
+    }
+    return result
+
+
+def run_e2e(pg, torch, dev, layers, weights, acts_host, outs, args, world, wbytes, flops, memory_bound):
+    stream = torch.cuda.Stream(device=dev)
+    out_host = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    xdev = [torch.empty(x.shape, dtype=x.dtype, device=dev) for x in acts_host]
+    ws = []
+    for L in layers:
+        if L.kind == "fp8":
+            ws.append(torch.empty(pg.fp8_linear_dynamic_workspace_size(L.M, L.N, L.K), dtype=torch.uint8,
+                                  device=dev))
+        elif L.kind == "nested8":
+            ws.append(torch.empty(pg.nestedfp_linear_workspace_size(L.M, L.N, L.K, pg.NESTED_FP8),
+                                  dtype=torch.uint8, device=dev))
+        else:
+            ws.append(None)
+
+    def step():
+        with torch.cuda.stream(stream):
+            for i, L in enumerate(layers):
+                xdev[i].copy_(acts_host[i], non_blocking=True)
+                W = weights[(L.shape_idx, L.copy, L.kind != "fp8")]
+                if L.kind == "fp8":
+                    pg.fp8_linear_dynamic(xdev[i], W[0], W[1], y=outs[i], workspace=ws[i], stream=stream)
+                else:
+                    mode = pg.NESTED_FP16 if L.kind == "nested16" else pg.NESTED_FP8
+                    pg.nestedfp_linear(xdev[i], W[0], W[1] if mode == pg.NESTED_FP16 else None, mode=mode,
+                                       y=outs[i], workspace=ws[i], stream=stream)
+                out_host[i].copy_(outs[i], non_blocking=True)
+
+    steps = max(3, min(args.steps, 200))
+    for _ in range(3):
+        step()
+    stream.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    stream.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    h2d = sum(x.numel() * x.element_size() for x in acts_host)
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+    v = (wbytes / (ms * 1e-3) / 1e9) if memory_bound else (flops / (ms * 1e-3) / 1e12)
+    return {"value": round(v * world, 2), "unit": "GB/s" if memory_bound else "TFLOP/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "ms_per_step": round(ms, 5), "entry_point": "fp8_linear_dynamic / nestedfp_linear"}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample(name, cols):
+    """Time the CPU oracle on every layer of one step of the workload: the
+    activations are quantised in full, the binary64 contraction runs on the
+    first `cols` output channels of each layer, and its time is extrapolated
+    linearly to all N channels.  Returns (seconds per full step, description,
+    threads used)."""
+    import oracle
+
+    layers = workload_layers(name, weight_copies(name))
+    total = 0.0
+    for L in layers:
+        x = synthetic.acts(name, L.shape_idx, L.m_idx)
+        ncols = min(cols, L.N)
+        w = synthetic.weights(name, L.shape_idx, copy=L.copy, n_override=ncols)
+        if L.kind == "fp8":
+            wq, sw = oracle.quantize_rows(w)      # offline weight quantisation: not timed
+            t0 = time.perf_counter()
+            aq, sa = oracle.quantize_rows(x)
+            t1 = time.perf_counter()
+            oracle.fp8_linear(aq, sa, wq, sw)
+        elif L.kind == "nested16":
+            hi, lo = oracle.nestedfp_split(w)
+            t0 = t1 = time.perf_counter()
+            oracle.nestedfp_linear_fp16(x, hi, lo)
+        else:
+            hi, _ = oracle.nestedfp_split(w)
+            t0 = t1 = time.perf_counter()
+            oracle.nestedfp_linear_fp8(x, hi)
+        t2 = time.perf_counter()
+        total += (t1 - t0) + (t2 - t1) * (L.N / ncols)
+    desc = (f"all {len(layers)} layers of one step: activations quantised in full, binary64 contraction on "
+            f"the first {cols} output channels of each layer, its time scaled linearly to all N channels")
+    return total, desc, 1
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle, as it stands, on the host cores; each
+    step is a bounded sample of one step of the workload (a number of output
+    channels per layer sized so the whole --steps/--warmup run takes about two
+    minutes), extrapolated to the full step."""
+    name = args.workload
+    layers = workload_layers(name, weight_copies(name))
+    wbytes = sum(L.weight_bytes for L in layers)
+    flops = sum(L.flops for L in layers)
+    memory_bound = name in ("decode7b", "small")
+    # size the per-step sample so the whole run takes about two minutes
+    t_start = time.perf_counter()
+    oracle_sample(name, cols=8)
+    t8 = time.perf_counter() - t_start
+    budget = max(0.02, 120.0 / (args.warmup + args.steps))
+    cols = int(max(1, min(4096, 8 * budget / max(t8, 1e-6))))
+    times = []
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        s, desc, _ = oracle_sample(name, cols=cols)
+        if i >= args.warmup:
+            times.append(s)
+    ms = 1e3 * sum(times) / len(times)
+    v = (wbytes / (ms * 1e-3) / 1e9) if memory_bound else (flops / (ms * 1e-3) / 1e12)
+    unit = "GB/s" if memory_bound else "TFLOP/s"
+    return {
+        "metric": METRIC, "value": v, "unit": unit, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": f"{name}: {WORKLOAD_TEXT[name]}"},
+        "cpu_baseline": {"kind": "oracle", "cores": 1, "sample": desc, "value": v, "unit": unit},
+        "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------- main
+def run_single(args):
+    """One layer, launched eagerly `warmup + steps` times: the small, fixed case
+    the profiler captures (e.g. --single fp8,8,4096,12288 = kind,M,K,N)."""
+    import torch
+    import precision_gemm_fp8_b200 as pg
+
+    kind, M, K, N = args.single.split(",")
+    M, K, N = int(M), int(K), int(N)
+    dev = torch.device("cuda", 0)
+    g = synthetic.rng(99, 0, 0, 0)
+    w = torch.from_numpy(synthetic.weights_f16(N, K, 0.02, g)).to(dev)
+    x = torch.from_numpy(synthetic.activations("normal_outl_0p5pct_x30", M, K, g)).to(dev)
+    opts = dict(path=args.path, split_k=args.split_k, tile_n=args.tile_n)
+    if kind == "fp8":
+        wq, sw = pg.fp8_quantize_rows(w)
+        aq, sa = pg.fp8_quantize_rows(x)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        fn = lambda: pg.fp8_linear(aq, sa, wq, sw, y=y, **opts)  # noqa: E731
+    elif kind == "dyn":
+        wq, sw = pg.fp8_quantize_rows(w)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(pg.fp8_linear_dynamic_workspace_size(M, N, K), dtype=torch.uint8, device=dev)
+        fn = lambda: pg.fp8_linear_dynamic(x, wq, sw, y=y, workspace=ws, **opts)  # noqa: E731
+    else:
+        hi, lo = pg.nestedfp_split(w.half())
+        x16 = x.half()
+        mode = pg.NESTED_FP16 if kind == "nested16" else pg.NESTED_FP8
+        y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        ws = torch.empty(max(1, pg.nestedfp_linear_workspace_size(M, N, K, mode)), dtype=torch.uint8, device=dev)
+        fn = lambda: pg.nestedfp_linear(x16, hi, lo, mode=mode, y=y, workspace=ws, **opts)  # noqa: E731
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        fn()
+    t1.record()
+    torch.cuda.synchronize()
+    if pg.device_status() != pg.OK:
+        raise RuntimeError("device error word raised")
+    us = 1e3 * t0.elapsed_time(t1) / args.steps
+    print(json.dumps({"single": args.single, "us_per_call": round(us, 3), "opts": opts,
+                      "weight_gbs": round(N * K * (2 if kind == "nested16" else 1) / (us * 1e-6) / 1e9, 1),
+                      "tflops": round(2.0 * M * N * K / (us * 1e-6) / 1e12, 2)}), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(synthetic.WORKLOADS), default="decode7b")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--single", default=None, help="kind,M,K,N: time (or profile) one layer eagerly")
+    ap.add_argument("--path", type=int, default=0)
+    ap.add_argument("--split-k", type=int, default=0)
+    ap.add_argument("--tile-n", type=int, default=0)
+    args = ap.parse_args()
+    if args.single:
+        run_single(args)
+        return
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(args.gpus if args.gpus == 1 else 1)))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:      # the other ranks exit without work
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if not args.no_cpu_baseline:
+                s, desc, cores = oracle_sample(args.workload, cols=1024)
+                layers = workload_layers(args.workload, weight_copies(args.workload))
+                wbytes = sum(L.weight_bytes for L in layers)
+                flops = sum(L.flops for L in layers)
+                v = (wbytes / s / 1e9) if res["unit"] == "GB/s" else (flops / s / 1e12)
+                res["cpu_baseline"] = {"value": v, "unit": res["unit"], "cores": cores, "kind": "oracle",
+                                       "sample": desc, "ms_per_step_extrapolated": round(s * 1e3, 1),
+                                       "host_cpus": os.cpu_count()}
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -97,7 +97,8 @@ typedef struct {
  *            saturated to +-448, sign of zero kept.
  * q is [rows, cols] contiguous (uint8 codes, OCP E4M3 "FN" layout).
  * Results are bit-exact with respect to that definition.  Non-finite input
- * values give unspecified codes.
+ * values give unspecified codes.  rows == 0 is a no-op (pointers may then
+ * be NULL).
  * ---------------------------------------------------------------------- */
 pgf8_status pgf8_fp8_quantize_rows(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols,
                                    int64_t ldx, uint8_t *q, float *scales,

@@ -270,7 +270,11 @@ static pgf8_status quantize_launch(const void *x, pgf8_dtype xdt, int64_t rows, 
 static pgf8_status check_quantize_args(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
                                        const uint8_t *q, const float *scales, int mode)
 {
-    if (!x || !q || !scales || rows < 0 || cols < 16 || ldx < cols || rows > (1ll << 31) - 1)
+    if (rows < 0 || cols < 16 || ldx < cols || rows > (1ll << 31) - 1)
+        return PGF8_ERR_INVALID_ARG;
+    if (rows == 0)
+        return PGF8_OK;   // nothing to read or write; pointers may be null
+    if (!x || !q || !scales)
         return PGF8_ERR_INVALID_ARG;
     if (xdt != PGF8_F32 && xdt != PGF8_F16)
         return PGF8_ERR_UNSUPPORTED;

@@ -96,6 +96,7 @@ def test_quantize_rejects_bad_args():
     assert q(MIS, pg.F32, 4, 64, 64, B16, C16, 0, None) == pg.ERR_ALIGNMENT
     assert q(A16, pg.F32, 4, 64, 64, B16, C16 + 2, 0, None) == pg.ERR_ALIGNMENT
     assert q(A16, pg.F32, 4, 64, 64, B16, C16, 5, None) == pg.ERR_INVALID_ARG
+    assert q(None, pg.F32, 0, 64, 64, None, None, 0, None) == pg.OK              # no rows: no-op
 
 
 def test_dynamic_and_nested_reject_bad_args():
