@@ -75,13 +75,25 @@ typedef enum {
     PGF8_PATH_TILED = 2    /* tokens are the 128-row MMA operand (any M) */
 } pgf8_path;
 
+/* Flags of pgf8_linear_opts.flags.
+ *
+ * PGF8_FLAG_OVERLAP_PREVIOUS: launch the call's first kernel with
+ * programmatic stream serialization, so that it and the GEMM's first weight
+ * loads may run while the previous kernel in the stream is still finishing
+ * (the GEMM of the previous layer, typically).  Activations are read, and
+ * outputs and workspace written, only after that kernel has completed; the
+ * weights (wq/sw, or hi/lo) may be read earlier.  Set it only when no kernel
+ * that can still be running writes those weights (weights that are static
+ * during inference satisfy this). */
+#define PGF8_FLAG_OVERLAP_PREVIOUS 1
+
 /* Optional tuning of the linear entry points; a NULL pointer means all
  * defaults.  Fields set to 0 mean "choose automatically". */
 typedef struct {
     int32_t path;      /* pgf8_path */
     int32_t split_k;   /* K split across a thread-block cluster, 1..8 */
     int32_t tile_n;    /* narrow MMA operand rows: 16, 32, 64, 128 (skinny) or 128, 256 (tiled) */
-    int32_t reserved;
+    int32_t flags;     /* PGF8_FLAG_* */
 } pgf8_linear_opts;
 
 /* ------------------------------------------------------------------------

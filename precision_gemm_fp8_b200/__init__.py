@@ -31,11 +31,12 @@ F32, F16, BF16 = 0, 1, 2
 SCALE_DYNAMIC, SCALE_STATIC = 0, 1
 NESTED_FP16, NESTED_FP8 = 0, 1
 PATH_AUTO, PATH_SKINNY, PATH_TILED = 0, 1, 2
+FLAG_OVERLAP_PREVIOUS = 1
 
 
 class LinearOpts(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int32), ("split_k", ctypes.c_int32), ("tile_n", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("flags", ctypes.c_int32)]
 
 
 _vp = ctypes.c_void_p
@@ -106,10 +107,10 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(int(stream))
 
 
-def _opts(path=PATH_AUTO, split_k=0, tile_n=0):
-    if path == PATH_AUTO and split_k == 0 and tile_n == 0:
+def _opts(path=PATH_AUTO, split_k=0, tile_n=0, flags=0):
+    if path == PATH_AUTO and split_k == 0 and tile_n == 0 and flags == 0:
         return None
-    return ctypes.byref(LinearOpts(path, split_k, tile_n, 0))
+    return ctypes.byref(LinearOpts(path, split_k, tile_n, flags))
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -140,14 +141,14 @@ def fp8_quantize_rows(x: torch.Tensor, q: torch.Tensor | None = None, scales: to
     return q, scales
 
 
-def fp8_linear(aq, sa, wq, sw, y=None, path=PATH_AUTO, split_k=0, tile_n=0, stream=None):
+def fp8_linear(aq, sa, wq, sw, y=None, path=PATH_AUTO, split_k=0, tile_n=0, flags=0, stream=None):
     """y [M,N] bf16 = (E4M3 aq [M,K] x E4M3 wq [N,K]^T) * sa[m] * sw[n]."""
     M, K = aq.shape
     N = wq.shape[0]
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=aq.device)
     _check(lib.pgf8_fp8_linear_ex(_ptr(aq), _ptr(sa), M, K, _ptr(wq), _ptr(sw), N, _ptr(y), None, 0,
-                                  _opts(path, split_k, tile_n), _stream(stream)), "fp8_linear")
+                                  _opts(path, split_k, tile_n, flags), _stream(stream)), "fp8_linear")
     return y
 
 
@@ -155,7 +156,8 @@ def fp8_linear_dynamic_workspace_size(M: int, N: int, K: int) -> int:
     return int(lib.pgf8_fp8_linear_dynamic_workspace_size(M, N, K))
 
 
-def fp8_linear_dynamic(x, wq, sw, y=None, workspace=None, path=PATH_AUTO, split_k=0, tile_n=0, stream=None):
+def fp8_linear_dynamic(x, wq, sw, y=None, workspace=None, path=PATH_AUTO, split_k=0, tile_n=0, flags=0,
+                       stream=None):
     """Per-token dynamic quantisation of x [M,K] (f32/f16) followed by the FP8
     linear with weights wq [N,K] / sw [N].  Returns y [M,N] bf16."""
     M, K = x.shape
@@ -169,7 +171,7 @@ def fp8_linear_dynamic(x, wq, sw, y=None, workspace=None, path=PATH_AUTO, split_
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     _check(lib.pgf8_fp8_linear_dynamic(_ptr(x), _dtype_code(x), M, K, x.stride(0), _ptr(wq), _ptr(sw), N, _ptr(y),
                                        _ptr(workspace), workspace.numel() * workspace.element_size(),
-                                       _opts(path, split_k, tile_n), _stream(stream)), "fp8_linear_dynamic")
+                                       _opts(path, split_k, tile_n, flags), _stream(stream)), "fp8_linear_dynamic")
     return y
 
 
@@ -199,7 +201,7 @@ def nestedfp_linear_workspace_size(M: int, N: int, K: int, mode: int) -> int:
 
 
 def nestedfp_linear(x, hi, lo, mode=NESTED_FP16, y=None, workspace=None, path=PATH_AUTO, split_k=0, tile_n=0,
-                    stream=None):
+                    flags=0, stream=None):
     """NestedFP linear: x [M,K] f16, hi/lo [N,K] uint8 planes -> y [M,N] f16.
     FP16 mode rebuilds (hi << 8) | lo; FP8 mode uses hi as E5M2 and
     quantises x per token to E4M3 (lo unused)."""
@@ -214,7 +216,7 @@ def nestedfp_linear(x, hi, lo, mode=NESTED_FP16, y=None, workspace=None, path=PA
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.pgf8_nestedfp_linear_ex(_ptr(x), M, K, _ptr(hi), _ptr(lo) if lo is not None else None, N, mode,
-                                       _ptr(y), _ptr(workspace), wbytes, _opts(path, split_k, tile_n),
+                                       _ptr(y), _ptr(workspace), wbytes, _opts(path, split_k, tile_n, flags),
                                        _stream(stream)), "nestedfp_linear")
     return y
 

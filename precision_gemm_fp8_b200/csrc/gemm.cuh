@@ -201,6 +201,11 @@ __global__ void __launch_bounds__(192, 1)
     constexpr uint32_t kIdesc =
         make_idesc(128, BN, /*A fmt*/ (SWAP && KIND == kNested8) ? 1 : 0, /*B fmt*/ (!SWAP && KIND == kNested8) ? 1 : 0);
 
+    // A dependent kernel launched with programmatic serialization (the next
+    // layer) may be scheduled into free SM slots now; it reads nothing this
+    // grid writes before this grid has completed.
+    grid_launch_dependents();
+
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     SharedCtl *ctl = reinterpret_cast<SharedCtl *>(smem + C::kBarOffset);

@@ -200,11 +200,13 @@ template <int KIND> static pgf8_status launch_gemm(const GemmLaunch &L)
     if (path == PGF8_PATH_SKINNY) {
         const int tiles = (L.N + 127) / 128;
         if (splits == 0) {
-            // enough CTAs to cover every SM at least once; no more splits
-            // than needed (each split adds a partial-tile exchange)
+            // double the split while the grid stays within ~1.3 CTAs per SM
+            // (two CTAs fit on an SM at the narrow tile sizes): more CTAs
+            // than that only add partial-tile exchanges and cluster packing
+            // constraints without adding bytes in flight
             splits = 1;
-            while (splits < 8 && tiles * splits < sms)
-                ++splits;
+            while (splits < 8 && tiles * splits * 2 * 10 <= sms * 13)
+                splits *= 2;
         }
         if (splits > kblocks)
             splits = kblocks;
@@ -250,18 +252,30 @@ static pgf8_linear_opts opts_or_default(const pgf8_linear_opts *o)
 }
 
 static pgf8_status quantize_launch(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
-                                   uint8_t *q, float *scales, int mode, cudaStream_t st)
+                                   uint8_t *q, float *scales, int mode, cudaStream_t st, int pdl,
+                                   int trigger_early)
 {
     if (rows == 0)
         return PGF8_OK;
-    dim3 grid(static_cast<unsigned>(rows));
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(rows));
+    cfg.blockDim = dim3(kQuantThreads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    if (pdl) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    cudaError_t e;
     if (xdt == PGF8_F32)
-        quantize_rows_kernel<float><<<grid, kQuantThreads, 0, st>>>(static_cast<const float *>(x), rows, cols, ldx,
-                                                                     q, scales, mode);
+        e = cudaLaunchKernelEx(&cfg, quantize_rows_kernel<float>, static_cast<const float *>(x), rows, cols, ldx, q,
+                               scales, mode, trigger_early);
     else
-        quantize_rows_kernel<__half><<<grid, kQuantThreads, 0, st>>>(static_cast<const __half *>(x), rows, cols,
-                                                                      ldx, q, scales, mode);
-    cudaError_t e = cudaGetLastError();
+        e = cudaLaunchKernelEx(&cfg, quantize_rows_kernel<__half>, static_cast<const __half *>(x), rows, cols, ldx,
+                               q, scales, mode, trigger_early);
     if (e != cudaSuccess)
         return cuda_fail(e);
     return PGF8_OK;
@@ -298,8 +312,11 @@ pgf8_status pgf8_fp8_quantize_rows(const void *x, pgf8_dtype xdt, int64_t rows, 
     pgf8_status st = check_quantize_args(x, xdt, rows, cols, ldx, q, scales, mode);
     if (st != PGF8_OK)
         return st;
+    // a plain launch that signals no early trigger: a following kernel that
+    // may overlap its predecessor (e.g. a GEMM reading these codes as weights)
+    // cannot start before this one has finished
     return quantize_launch(x, xdt, rows, cols, ldx, q, scales, static_cast<int>(mode),
-                           static_cast<cudaStream_t>(stream));
+                           static_cast<cudaStream_t>(stream), 0, 0);
 }
 
 size_t pgf8_fp8_linear_workspace_size(int64_t, int64_t, int64_t) { return 0; }
@@ -327,8 +344,8 @@ pgf8_status pgf8_fp8_linear_ex(const uint8_t *aq, const float *sa, int64_t M, in
     L.N = static_cast<int>(N);
     L.K = static_cast<int>(K);
     L.pdl = 1;
-    L.prefetch_w = 0;
     L.opts = opts_or_default(opts);
+    L.prefetch_w = (L.opts.flags & PGF8_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
     L.stream = static_cast<cudaStream_t>(stream);
     return launch_gemm<kE4M3>(L);
 }
@@ -374,7 +391,11 @@ static pgf8_status linear_dynamic_impl(const void *x, pgf8_dtype xdt, int64_t M,
     if (st != PGF8_OK)
         return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    st = quantize_launch(x, xdt, M, K, ldx, aq, sa, 0, cs);
+    const pgf8_linear_opts o = opts_or_default(opts);
+    const int overlap = (o.flags & PGF8_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
+    // the quantisation signals its dependent (this call's GEMM) at once: the
+    // GEMM loads its first weight tiles while the activations are quantised
+    st = quantize_launch(x, xdt, M, K, ldx, aq, sa, 0, cs, overlap, 1);
     if (st != PGF8_OK)
         return st;
     GemmLaunch L;
@@ -390,7 +411,7 @@ static pgf8_status linear_dynamic_impl(const void *x, pgf8_dtype xdt, int64_t M,
     L.K = static_cast<int>(K);
     L.pdl = 1;
     L.prefetch_w = 1;   // the quantisation kernel writes only aq / sa
-    L.opts = opts_or_default(opts);
+    L.opts = o;
     L.stream = cs;
     if (kind == kNested8)
         return launch_gemm<kNested8>(L);
@@ -460,8 +481,8 @@ pgf8_status pgf8_nestedfp_linear_ex(const void *x, int64_t M, int64_t K, const u
     L.N = static_cast<int>(N);
     L.K = static_cast<int>(K);
     L.pdl = 1;
-    L.prefetch_w = 0;
     L.opts = opts_or_default(opts);
+    L.prefetch_w = (L.opts.flags & PGF8_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
     L.stream = static_cast<cudaStream_t>(stream);
     return launch_gemm<kNested16>(L);
 }

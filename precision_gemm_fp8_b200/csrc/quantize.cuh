@@ -4,11 +4,11 @@
 // static weight scales) and §6.1 (448 bound); "C++ and FP8" §4.2 (per-token /
 // per-channel).  split: "NestedFP dual-precision inference framework" §2.1.
 //
-// Both are HBM-bound elementwise passes.  quantize: one CTA per row; the
-// row is read once from HBM for the amax (128-bit loads, warp-shuffle max,
-// then a CTA max), and the second, converting pass re-reads it from L2
-// (a row is at most a few hundred KB and was just read).  Bytes per element:
-// 4 (f32) or 2 (f16) in, 1 out.
+// Both are HBM-bound elementwise passes.  quantize: one CTA per row, 128-bit
+// loads, warp-shuffle max then a CTA max for the amax; rows of up to 16384
+// elements are held in registers between the amax and the conversion (one
+// pass over memory), longer rows are re-read from L2 for the conversion.
+// Bytes per element: 4 (f32) or 2 (f16) in, 1 out.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -79,23 +79,80 @@ __device__ __forceinline__ float block_max(float v, float *red)
     return red[0];
 }
 
+// Converts 16 binary32 values (already divided by the scale) to 16 codes.
+__device__ __forceinline__ uint4 encode16(const float (&v)[16], float s)
+{
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t lo = cvt_e4m3x2(__fdiv_rn(v[4 * i + 0], s), __fdiv_rn(v[4 * i + 1], s));
+        const uint32_t hi = cvt_e4m3x2(__fdiv_rn(v[4 * i + 2], s), __fdiv_rn(v[4 * i + 3], s));
+        w[i] = lo | (hi << 16);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Rows of up to kRegChunks * kQuantThreads * 16 elements stay in registers
+// between the amax and the conversion (one pass over global memory);
+// longer rows are re-read (from L2) for the conversion.
+constexpr int kRegChunks = 4;
+
 // One CTA per row.  cols % 16 == 0; x rows 16-byte aligned.
+// trigger_early: let a dependent kernel launched with programmatic stream
+// serialization be scheduled at once (used only when that dependent is the
+// library's own GEMM, which reads q/scales after this grid completes).
 template <typename T>
 __global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(const T *__restrict__ x, int64_t rows,
                                                                       int64_t cols, int64_t ldx,
                                                                       uint8_t *__restrict__ q,
-                                                                      float *__restrict__ scales, int mode)
+                                                                      float *__restrict__ scales, int mode,
+                                                                      int trigger_early)
 {
     __shared__ float red[kQuantThreads / 32];
-    // Let a dependent GEMM launched with programmatic serialization start its
-    // set-up now; it waits for this grid's completion before reading q/scales.
-    grid_launch_dependents();
+    if (trigger_early)
+        grid_launch_dependents();
+    // When launched with programmatic serialization, the previous kernel in
+    // the stream may still run: nothing is read or written before it ends.
+    grid_dependency_wait();
     const int64_t row = blockIdx.x;
     if (row >= rows)
         return;
     const T *xr = x + row * ldx;
     uint8_t *qr = q + row * cols;
     const int64_t nchunk = cols / 16;
+
+    if (nchunk <= static_cast<int64_t>(kRegChunks) * kQuantThreads) {
+        Vec16<T> v[kRegChunks];
+        float amax = 0.0f;
+#pragma unroll
+        for (int u = 0; u < kRegChunks; ++u) {
+            const int64_t c = threadIdx.x + static_cast<int64_t>(u) * kQuantThreads;
+            if (c < nchunk) {
+                v[u].load(xr + c * 16);
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    amax = fmaxf(amax, fabsf(v[u].v[i]));
+            }
+        }
+        float s;
+        if (mode == 0) {
+            amax = block_max(amax, red);
+            s = __fdiv_rn(amax, 448.0f);
+            if (s == 0.0f)
+                s = 1.0f;
+            if (threadIdx.x == 0)
+                scales[row] = s;
+        } else {
+            s = scales[row];
+        }
+#pragma unroll
+        for (int u = 0; u < kRegChunks; ++u) {
+            const int64_t c = threadIdx.x + static_cast<int64_t>(u) * kQuantThreads;
+            if (c < nchunk)
+                *reinterpret_cast<uint4 *>(qr + c * 16) = encode16(v[u].v, s);
+        }
+        return;
+    }
 
     float s;
     if (mode == 0) {
@@ -116,18 +173,10 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(const T *_
     } else {
         s = scales[row];
     }
-
     for (int64_t c = threadIdx.x; c < nchunk; c += kQuantThreads) {
         Vec16<T> v;
         v.load(xr + c * 16);
-        uint32_t w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t lo = cvt_e4m3x2(__fdiv_rn(v.v[4 * i + 0], s), __fdiv_rn(v.v[4 * i + 1], s));
-            const uint32_t hi = cvt_e4m3x2(__fdiv_rn(v.v[4 * i + 2], s), __fdiv_rn(v.v[4 * i + 3], s));
-            w[i] = lo | (hi << 16);
-        }
-        *reinterpret_cast<uint4 *>(qr + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4 *>(qr + c * 16) = encode16(v.v, s);
     }
 }
 

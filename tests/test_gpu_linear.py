@@ -156,3 +156,34 @@ def test_prefill7b_full_size(shape_idx):
 @pytest.mark.parametrize("shape_idx,m_idx", [(0, 0), (1, 4), (2, 7), (3, 9), (1, 12), (3, 5)])
 def test_llama70b_full_size(shape_idx, m_idx):
     _full_size_case("llama70b", shape_idx, m_idx)
+
+
+def test_dynamic_chain_with_overlap_flag_matches_unchained():
+    """Back-to-back dynamic FP8 layers with FLAG_OVERLAP_PREVIOUS reusing one
+    workspace (the next layer's quantisation overwrites codes the previous
+    GEMM reads): results equal those of synchronised calls, bit for bit."""
+    shapes = [(4096, 12288), (4096, 4096), (11008, 4096)]
+    g = np.random.default_rng(21)
+    Ws, Xs = [], []
+    for K, N in shapes:
+        wq, sw = pg.fp8_quantize_rows(_to(synthetic.weights_f16(N, K, 0.02, g)))
+        Ws.append((wq, sw))
+        Xs.append(_to(synthetic.activations("normal_outl_0p5pct_x30", 8, K, g)))
+    ws = torch.empty(max(pg.fp8_linear_dynamic_workspace_size(8, N, K) for K, N in shapes), dtype=torch.uint8,
+                     device=DEV)
+    torch.cuda.synchronize()
+
+    def run(flags, sync):
+        ys = []
+        for (wq, sw), x in zip(Ws, Xs):
+            ys.append(pg.fp8_linear_dynamic(x, wq, sw, workspace=ws, flags=flags))
+            if sync:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        return [y.float().cpu().numpy() for y in ys]
+
+    ref = run(0, True)
+    for _ in range(3):
+        for a, b in zip(run(pg.FLAG_OVERLAP_PREVIOUS, False), ref):
+            np.testing.assert_array_equal(a, b)
+    assert pg.device_status() == pg.OK

@@ -114,3 +114,40 @@ def test_nested7b_full_size_both_modes(shape_idx, m_idx):
     assert_within(y16.float().cpu().numpy()[np.ix_(ms, ns)], ref, bound, f"fp16 full M={M}")
     ref8, bound8, _, _ = _ref8(x16[ms], hi)
     assert_within(y8.float().cpu().numpy()[np.ix_(ms, ns)], ref8, bound8, f"fp8 full M={M}")
+
+
+@pytest.mark.parametrize("mode", ["fp16", "fp8"])
+def test_chained_layers_with_overlap_flag(mode):
+    """Four NestedFP layers where each layer's input is the previous layer's
+    output, enqueued back to back with FLAG_OVERLAP_PREVIOUS (each call may
+    start while the previous layer is finishing).  The results must equal the
+    same chain run with a synchronisation between layers, bit for bit: the
+    overlap may only move weight loads earlier, never activation reads."""
+    g = np.random.default_rng(11)
+    M, D = 8, 1024
+    m = pg.NESTED_FP16 if mode == "fp16" else pg.NESTED_FP8
+    planes = []
+    for _ in range(4):
+        w = synthetic.weights_f16(D, D, 0.03, g)
+        planes.append(pg.nestedfp_split(_to(w)))
+    x0 = _to(synthetic.activations("normal_f16", M, D, g))
+    torch.cuda.synchronize()
+
+    def run(flags, sync):
+        x = x0
+        ys = []
+        for hi, lo in planes:
+            y = pg.nestedfp_linear(x, hi, lo if m == pg.NESTED_FP16 else None, mode=m, flags=flags)
+            if sync:
+                torch.cuda.synchronize()
+            ys.append(y)
+            x = y
+        torch.cuda.synchronize()
+        return [t.cpu().numpy() for t in ys]
+
+    ref = run(0, True)
+    for _ in range(3):
+        got = run(pg.FLAG_OVERLAP_PREVIOUS, False)
+        for a, b in zip(got, ref):
+            np.testing.assert_array_equal(a.view(np.uint16), b.view(np.uint16))
+    assert pg.device_status() == pg.OK
