@@ -9,6 +9,7 @@
 
 #include "pgf8.h"
 #include "gemm.cuh"
+#include "gemm_persistent.cuh"
 #include "quantize.cuh"
 
 namespace pgf8 {
@@ -76,18 +77,12 @@ struct GemmLaunch {
     cudaStream_t stream;
 };
 
-template <class C> static pgf8_status launch_cfg(const GemmLaunch &L, int splits)
+// Tensor maps of the two operands for a kernel configuration C (tile rows
+// C::kRowsX / C::kRowsW, 128 bytes of K per box).
+template <class C> static bool make_operand_maps(const GemmLaunch &L, CUtensorMap &tmX, CUtensorMap &tmW,
+                                                 CUtensorMap &tmW2)
 {
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    });
-    if (attr_err != cudaSuccess)
-        return cuda_fail(attr_err);
-
     const bool nest16 = (C::KIND == kNested16);
-    CUtensorMap tmX, tmW, tmW2;
     std::memset(&tmW2, 0, sizeof(tmW2));
     bool ok;
     if (nest16) {
@@ -104,9 +99,12 @@ template <class C> static pgf8_status launch_cfg(const GemmLaunch &L, int splits
                       CU_TENSOR_MAP_SWIZZLE_128B);
         tmW2 = tmW;
     }
-    if (!ok)
-        return PGF8_ERR_UNSUPPORTED;
+    return ok;
+}
 
+static GemmParams make_params(const GemmLaunch &L, int splits)
+{
+    const bool nest16 = (L.kind == kNested16);
     GemmParams p;
     p.M = L.M;
     p.N = L.N;
@@ -117,6 +115,41 @@ template <class C> static pgf8_status launch_cfg(const GemmLaunch &L, int splits
     p.sa = L.sa;
     p.sw = L.sw;
     p.y = L.y;
+    return p;
+}
+
+static void fill_attrs(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attrs, int cluster_z, int pdl)
+{
+    int na = 0;
+    if (cluster_z > 1) {
+        attrs[na].id = cudaLaunchAttributeClusterDimension;
+        attrs[na].val.clusterDim.x = 1;
+        attrs[na].val.clusterDim.y = 1;
+        attrs[na].val.clusterDim.z = static_cast<unsigned>(cluster_z);
+        ++na;
+    }
+    if (pdl) {
+        attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attrs[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.attrs = attrs;
+    cfg.numAttrs = na;
+}
+
+template <class C> static pgf8_status launch_cfg(const GemmLaunch &L, int splits)
+{
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    });
+    if (attr_err != cudaSuccess)
+        return cuda_fail(attr_err);
+    CUtensorMap tmX, tmW, tmW2;
+    if (!make_operand_maps<C>(L, tmX, tmW, tmW2))
+        return PGF8_ERR_UNSUPPORTED;
+    const GemmParams p = make_params(L, splits);
 
     const int rows_a = C::SWAP ? L.N : L.M;   // A side: 128-row tiles
     const int rows_b = C::SWAP ? L.M : L.N;   // B side: BN-row tiles
@@ -129,22 +162,41 @@ template <class C> static pgf8_status launch_cfg(const GemmLaunch &L, int splits
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = L.stream;
     cudaLaunchAttribute attrs[2];
-    int na = 0;
-    if (C::SPLIT) {
-        attrs[na].id = cudaLaunchAttributeClusterDimension;
-        attrs[na].val.clusterDim.x = 1;
-        attrs[na].val.clusterDim.y = 1;
-        attrs[na].val.clusterDim.z = static_cast<unsigned>(splits);
-        ++na;
-    }
-    if (L.pdl) {
-        attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attrs[na].val.programmaticStreamSerializationAllowed = 1;
-        ++na;
-    }
-    cfg.attrs = attrs;
-    cfg.numAttrs = na;
+    fill_attrs(cfg, attrs, C::SPLIT ? splits : 1, L.pdl);
     cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel<C>, tmX, tmW, tmW2, p);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    return PGF8_OK;
+}
+
+static int num_sms();
+
+// Persistent tiled kernel: one CTA per SM (at most one per tile).
+template <class C> static pgf8_status launch_persistent(const GemmLaunch &L)
+{
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(gemm_persistent_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        C::kSmemBytes);
+    });
+    if (attr_err != cudaSuccess)
+        return cuda_fail(attr_err);
+    CUtensorMap tmX, tmW, tmW2;
+    if (!make_operand_maps<C>(L, tmX, tmW, tmW2))
+        return PGF8_ERR_UNSUPPORTED;
+    const GemmParams p = make_params(L, 1);
+    const int64_t tiles = static_cast<int64_t>((L.M + 127) / 128) * ((L.N + C::BN - 1) / C::BN);
+    const int sms = num_sms();
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles < sms ? tiles : sms), 1, 1);
+    cfg.blockDim = dim3(C::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = L.stream;
+    cudaLaunchAttribute attrs[2];
+    fill_attrs(cfg, attrs, 1, L.pdl);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_persistent_kernel<C>, tmX, tmW, tmW2, p);
     if (e != cudaSuccess)
         return cuda_fail(e);
     return PGF8_OK;
@@ -218,9 +270,17 @@ template <int KIND> static pgf8_status launch_gemm(const GemmLaunch &L)
         }
     }
     const int mt = (L.M + 127) / 128;
+    // fraction of the CTA slots the last wave of a persistent launch keeps busy
+    auto wave_eff = [&](int b) {
+        const int64_t t = static_cast<int64_t>(mt) * ((L.N + b - 1) / b);
+        const int64_t waves = (t + sms - 1) / sms;
+        return static_cast<double>(t) / static_cast<double>(waves * sms);
+    };
     if (bn == 0)
-        bn = (mt * ((L.N + 255) / 256) >= sms) ? 256 : 128;
+        bn = (wave_eff(128) > wave_eff(256) + 0.15) ? 128 : 256;
     if (splits == 0) {
+        // split K across a cluster only when there are too few tiles to
+        // occupy the SMs
         const int tiles = mt * ((L.N + bn - 1) / bn);
         splits = 1;
         while (splits < 4 && tiles * (splits + 1) <= sms)
@@ -228,6 +288,11 @@ template <int KIND> static pgf8_status launch_gemm(const GemmLaunch &L)
     }
     if (splits > kblocks)
         splits = kblocks;
+    if (splits == 1) {
+        if (bn == 256)
+            return launch_persistent<PersistCfg<256, 4, KIND>>(L);
+        return launch_persistent<PersistCfg<128, 6, KIND>>(L);
+    }
     if (bn == 256)
         return launch_split_or_not<KIND, false, 256, 4>(L, splits);
     return launch_split_or_not<KIND, false, 128, 6>(L, splits);
