@@ -208,16 +208,17 @@ def run_ours(args, rank, world, local_rank):
         out_dt = torch.float16 if L.kind.startswith("nested") else torch.bfloat16
         outs.append(torch.empty((L.M, L.N), dtype=out_dt, device=dev))
         if L.kind == "fp8":
-            qbufs.append(torch.empty(pg.fp8_linear_dynamic_workspace_size(L.M, L.N, L.K), dtype=torch.uint8,
+            qbufs.append(torch.zeros(pg.fp8_linear_dynamic_workspace_size(L.M, L.N, L.K), dtype=torch.uint8,
                                      device=dev))
-        elif L.kind == "nested8":
-            qbufs.append(torch.empty(pg.nestedfp_linear_workspace_size(L.M, L.N, L.K, pg.NESTED_FP8),
-                                     dtype=torch.uint8, device=dev))
         else:
-            qbufs.append(None)
+            mode = pg.NESTED_FP8 if L.kind == "nested8" else pg.NESTED_FP16
+            qbufs.append(torch.zeros(max(16, pg.nestedfp_linear_workspace_size(L.M, L.N, L.K, mode)),
+                                     dtype=torch.uint8, device=dev))
     torch.cuda.synchronize()
 
     stream = torch.cuda.Stream(device=dev)
+    sk_ws = torch.zeros(max(16, max(pg.lib.pgf8_fp8_linear_workspace_size(L.M, L.N, L.K) for L in layers)),
+                        dtype=torch.uint8, device=dev)
 
     def enqueue_step(ev_pairs=None):
         """One step through the C ABI on `stream`.
@@ -238,7 +239,7 @@ def run_ours(args, rank, world, local_rank):
                 aq, sa = pg.dynamic_workspace_views(qbufs[i], L.M, L.K)
                 pg.fp8_quantize_rows(acts[i], aq, sa, stream=stream)
                 ev_pairs[i][0].record(stream)
-                pg.fp8_linear(aq, sa, W[0], W[1], y=outs[i], stream=stream)
+                pg.fp8_linear(aq, sa, W[0], W[1], y=outs[i], workspace=sk_ws, stream=stream)
                 ev_pairs[i][1].record(stream)
             else:
                 mode = pg.NESTED_FP16 if L.kind == "nested16" else pg.NESTED_FP8
@@ -377,13 +378,12 @@ def run_e2e(pg, torch, dev, layers, weights, acts_host, outs, args, world, wbyte
     ws = []
     for L in layers:
         if L.kind == "fp8":
-            ws.append(torch.empty(pg.fp8_linear_dynamic_workspace_size(L.M, L.N, L.K), dtype=torch.uint8,
+            ws.append(torch.zeros(pg.fp8_linear_dynamic_workspace_size(L.M, L.N, L.K), dtype=torch.uint8,
                                   device=dev))
-        elif L.kind == "nested8":
-            ws.append(torch.empty(pg.nestedfp_linear_workspace_size(L.M, L.N, L.K, pg.NESTED_FP8),
-                                  dtype=torch.uint8, device=dev))
         else:
-            ws.append(None)
+            mode = pg.NESTED_FP8 if L.kind == "nested8" else pg.NESTED_FP16
+            ws.append(torch.zeros(max(16, pg.nestedfp_linear_workspace_size(L.M, L.N, L.K, mode)),
+                                  dtype=torch.uint8, device=dev))
 
     def step():
         with torch.cuda.stream(stream):
@@ -519,14 +519,14 @@ def run_single(args):
     elif kind == "dyn":
         wq, sw = pg.fp8_quantize_rows(w)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        ws = torch.empty(pg.fp8_linear_dynamic_workspace_size(M, N, K), dtype=torch.uint8, device=dev)
+        ws = torch.zeros(pg.fp8_linear_dynamic_workspace_size(M, N, K), dtype=torch.uint8, device=dev)
         fn = lambda: pg.fp8_linear_dynamic(x, wq, sw, y=y, workspace=ws, **opts)  # noqa: E731
     else:
         hi, lo = pg.nestedfp_split(w.half())
         x16 = x.half()
         mode = pg.NESTED_FP16 if kind == "nested16" else pg.NESTED_FP8
         y = torch.empty((M, N), dtype=torch.float16, device=dev)
-        ws = torch.empty(max(1, pg.nestedfp_linear_workspace_size(M, N, K, mode)), dtype=torch.uint8, device=dev)
+        ws = torch.zeros(max(16, pg.nestedfp_linear_workspace_size(M, N, K, mode)), dtype=torch.uint8, device=dev)
         fn = lambda: pg.nestedfp_linear(x16, hi, lo, mode=mode, y=y, workspace=ws, **opts)  # noqa: E731
     for _ in range(args.warmup):
         fn()

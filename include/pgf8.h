@@ -22,6 +22,15 @@
  *   Memory      All pointers are DEVICE pointers owned by the caller.  The
  *               library never allocates or frees device memory; the size of
  *               any workspace is returned by the matching *_workspace_size().
+ *   Workspace   A workspace must be zero-filled once, before its first use
+ *               (e.g. cudaMemset); every call that completes leaves the words
+ *               it synchronises on zero again, so it can be reused without
+ *               clearing.  After PGF8_ERR_TIMEOUT, zero it again.  One
+ *               workspace serves one call at a time (calls on different
+ *               streams need different workspaces).  For M <= 32 the linear
+ *               entry points use it for the stream-K kernel (flags, partial
+ *               tiles); with a NULL or short workspace they choose a kernel
+ *               that needs none.
  *   Layout      Row-major, last index contiguous: activations x/aq [M, K],
  *               weights w/wq/hi/lo [N, K] (K contiguous, "TN"), outputs
  *               y [M, N].  Row strides equal the row length unless an
@@ -72,7 +81,9 @@ typedef enum {
     PGF8_PATH_AUTO = 0,    /* chosen from M, N, K */
     PGF8_PATH_SKINNY = 1,  /* weight-streaming: weights are the 128-row MMA operand,
                               tokens the narrow one (M <= 128) */
-    PGF8_PATH_TILED = 2    /* tokens are the 128-row MMA operand (any M) */
+    PGF8_PATH_TILED = 2,   /* tokens are the 128-row MMA operand (any M) */
+    PGF8_PATH_STREAMK = 3  /* skinny, stream-K over one CTA per SM (M <= 32; needs the
+                              workspace) */
 } pgf8_path;
 
 /* Flags of pgf8_linear_opts.flags.
@@ -120,8 +131,8 @@ pgf8_status pgf8_fp8_quantize_rows(const void *x, pgf8_dtype xdt, int64_t rows, 
  * FP8 linear with fused dequantisation ("C++ and FP8" §3.3):
  *   y[m,n] = bf16_rn( (sum_k e4m3(aq[m,k]) * e4m3(wq[n,k])) * sa[m] * sw[n] )
  * with FP32 accumulation.  aq [M,K] uint8, sa [M] f32, wq [N,K] uint8,
- * sw [N] f32, y [M,N] bf16.  M >= 1.  workspace may be NULL when
- * pgf8_fp8_linear_workspace_size() returns 0 (it currently always does).
+ * sw [N] f32, y [M,N] bf16.  M >= 1.  workspace: see the conventions above
+ * (pgf8_fp8_linear_workspace_size bytes, nonzero for M <= 32; may be NULL).
  * ---------------------------------------------------------------------- */
 pgf8_status pgf8_fp8_linear(const uint8_t *aq, const float *sa, int64_t M, int64_t K,
                             const uint8_t *wq, const float *sw, int64_t N, void *y_bf16,
@@ -140,10 +151,10 @@ size_t pgf8_fp8_linear_workspace_size(int64_t M, int64_t N, int64_t K);
  * one dependent pair so the GEMM's set-up and first weight loads overlap the
  * quantisation ("7B on an RTX 4060 with FP8" §2.2: activations quantised at
  * run time).  x [M,K] f32 or f16 with row stride ldx.  The workspace
- * (size from pgf8_fp8_linear_dynamic_workspace_size) receives the E4M3
- * activation codes [M,K] at offset 0 and the per-token scales [M] at offset
- * pgf8_fp8_linear_dynamic_scales_offset(M, K); the caller may read both
- * after the call completes.  wq must not be written by work enqueued
+ * (size from pgf8_fp8_linear_dynamic_workspace_size; zero-filled before its
+ * first use) receives the E4M3 activation codes [M,K] at offset 0 and the
+ * per-token scales [M] at offset pgf8_fp8_linear_dynamic_scales_offset(M, K);
+ * the caller may read both after the call completes.  wq must not be written by work enqueued
  * between this call's quantisation and GEMM (nothing is).
  * ---------------------------------------------------------------------- */
 pgf8_status pgf8_fp8_linear_dynamic(const void *x, pgf8_dtype xdt, int64_t M, int64_t K,
@@ -166,7 +177,7 @@ pgf8_status pgf8_nestedfp_split(const void *w_f16, int64_t N, int64_t K, uint8_t
  * NestedFP linear ("NestedFP" §2.1-2.2).  x_f16 [M,K] FP16, y_f16 [M,N] FP16.
  *   PGF8_NESTED_FP16: y = fp16_rn( sum_k x[m,k] * fp16((hi<<8)|lo)[n,k] ),
  *     the weight rebuilt bit-exactly in shared memory inside the GEMM;
- *     FP32 accumulation.  workspace unused (size 0).
+ *     FP32 accumulation.  workspace: as for pgf8_fp8_linear (used for M <= 32).
  *   PGF8_NESTED_FP8: x is quantised per token to E4M3 (as
  *     pgf8_fp8_quantize_rows, DYNAMIC) into the workspace, and
  *     y = fp16_rn( (sum_k e4m3(aq[m,k]) * e5m2(hi[n,k])) * sa[m] ): the upper

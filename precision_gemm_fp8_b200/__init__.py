@@ -30,7 +30,7 @@ OK, ERR_INVALID_ARG, ERR_ALIGNMENT, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = ran
 F32, F16, BF16 = 0, 1, 2
 SCALE_DYNAMIC, SCALE_STATIC = 0, 1
 NESTED_FP16, NESTED_FP8 = 0, 1
-PATH_AUTO, PATH_SKINNY, PATH_TILED = 0, 1, 2
+PATH_AUTO, PATH_SKINNY, PATH_TILED, PATH_STREAMK = 0, 1, 2, 3
 FLAG_OVERLAP_PREVIOUS = 1
 
 
@@ -113,6 +113,29 @@ def _opts(path=PATH_AUTO, split_k=0, tile_n=0, flags=0):
     return ctypes.byref(LinearOpts(path, split_k, tile_n, flags))
 
 
+_ws_cache: dict = {}
+
+
+def default_workspace(device, nbytes: int) -> torch.Tensor | None:
+    """A zero-filled workspace of at least `nbytes`, cached per device and
+    shared by every call that is not given its own.  The library leaves its
+    synchronisation words zero after each completed call, so the buffer is
+    reused as is; calls running concurrently on several streams must each be
+    given their own (zero-filled) workspace instead."""
+    if nbytes <= 0:
+        return None
+    dev = torch.device(device)
+    t = _ws_cache.get(dev)
+    if t is None or t.numel() < nbytes:
+        t = torch.zeros(max(nbytes, 1 << 22), dtype=torch.uint8, device=dev)
+        _ws_cache[dev] = t
+    return t
+
+
+def _nbytes(t):
+    return 0 if t is None else t.numel() * t.element_size()
+
+
 def _dtype_code(t: torch.Tensor) -> int:
     if t.dtype == torch.float32:
         return F32
@@ -141,14 +164,19 @@ def fp8_quantize_rows(x: torch.Tensor, q: torch.Tensor | None = None, scales: to
     return q, scales
 
 
-def fp8_linear(aq, sa, wq, sw, y=None, path=PATH_AUTO, split_k=0, tile_n=0, flags=0, stream=None):
-    """y [M,N] bf16 = (E4M3 aq [M,K] x E4M3 wq [N,K]^T) * sa[m] * sw[n]."""
+def fp8_linear(aq, sa, wq, sw, y=None, workspace=None, path=PATH_AUTO, split_k=0, tile_n=0, flags=0,
+               stream=None):
+    """y [M,N] bf16 = (E4M3 aq [M,K] x E4M3 wq [N,K]^T) * sa[m] * sw[n].
+    workspace: zero-filled device buffer (default: the per-device shared one)."""
     M, K = aq.shape
     N = wq.shape[0]
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=aq.device)
-    _check(lib.pgf8_fp8_linear_ex(_ptr(aq), _ptr(sa), M, K, _ptr(wq), _ptr(sw), N, _ptr(y), None, 0,
-                                  _opts(path, split_k, tile_n, flags), _stream(stream)), "fp8_linear")
+    if workspace is None:
+        workspace = default_workspace(aq.device, int(lib.pgf8_fp8_linear_workspace_size(M, N, K)))
+    _check(lib.pgf8_fp8_linear_ex(_ptr(aq), _ptr(sa), M, K, _ptr(wq), _ptr(sw), N, _ptr(y), _ptr(workspace),
+                                  _nbytes(workspace), _opts(path, split_k, tile_n, flags), _stream(stream)),
+           "fp8_linear")
     return y
 
 
@@ -159,7 +187,8 @@ def fp8_linear_dynamic_workspace_size(M: int, N: int, K: int) -> int:
 def fp8_linear_dynamic(x, wq, sw, y=None, workspace=None, path=PATH_AUTO, split_k=0, tile_n=0, flags=0,
                        stream=None):
     """Per-token dynamic quantisation of x [M,K] (f32/f16) followed by the FP8
-    linear with weights wq [N,K] / sw [N].  Returns y [M,N] bf16."""
+    linear with weights wq [N,K] / sw [N].  Returns y [M,N] bf16.  A given
+    workspace must be zero-filled before its first use."""
     M, K = x.shape
     N = wq.shape[0]
     if x.stride(1) != 1:
@@ -168,7 +197,7 @@ def fp8_linear_dynamic(x, wq, sw, y=None, workspace=None, path=PATH_AUTO, split_
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     need = fp8_linear_dynamic_workspace_size(M, N, K)
     if workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+        workspace = default_workspace(x.device, need)
     _check(lib.pgf8_fp8_linear_dynamic(_ptr(x), _dtype_code(x), M, K, x.stride(0), _ptr(wq), _ptr(sw), N, _ptr(y),
                                        _ptr(workspace), workspace.numel() * workspace.element_size(),
                                        _opts(path, split_k, tile_n, flags), _stream(stream)), "fp8_linear_dynamic")
@@ -212,9 +241,9 @@ def nestedfp_linear(x, hi, lo, mode=NESTED_FP16, y=None, workspace=None, path=PA
     if y is None:
         y = torch.empty((M, N), dtype=torch.float16, device=x.device)
     need = nestedfp_linear_workspace_size(M, N, K, mode)
-    if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
-    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if workspace is None:
+        workspace = default_workspace(x.device, need)
+    wbytes = _nbytes(workspace)
     _check(lib.pgf8_nestedfp_linear_ex(_ptr(x), M, K, _ptr(hi), _ptr(lo) if lo is not None else None, N, mode,
                                        _ptr(y), _ptr(workspace), wbytes, _opts(path, split_k, tile_n, flags),
                                        _stream(stream)), "nestedfp_linear")

@@ -10,6 +10,7 @@
 #include "pgf8.h"
 #include "gemm.cuh"
 #include "gemm_persistent.cuh"
+#include "gemm_streamk.cuh"
 #include "quantize.cuh"
 
 namespace pgf8 {
@@ -75,6 +76,8 @@ struct GemmLaunch {
     int prefetch_w;    // weights may be read before the dependency resolves
     pgf8_linear_opts opts;
     cudaStream_t stream;
+    void *ws;          // stream-K region of the workspace (flags, then partial slots), or null
+    size_t ws_bytes;
 };
 
 // Tensor maps of the two operands for a kernel configuration C (tile rows
@@ -202,6 +205,43 @@ template <class C> static pgf8_status launch_persistent(const GemmLaunch &L)
     return PGF8_OK;
 }
 
+// Stream-K skinny kernel: one CTA per SM, equal shares of the weight stream.
+template <class C> static pgf8_status launch_streamk(const GemmLaunch &L)
+{
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(gemm_streamk_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        C::kSmemBytes);
+    });
+    if (attr_err != cudaSuccess)
+        return cuda_fail(attr_err);
+    CUtensorMap tmX, tmW, tmW2;
+    if (!make_operand_maps<C>(L, tmX, tmW, tmW2))
+        return PGF8_ERR_UNSUPPORTED;
+    const GemmParams p = make_params(L, 1);
+    StreamKParams q;
+    q.units = static_cast<int64_t>((L.N + 127) / 128) * p.kblocks;
+    q.flags = static_cast<unsigned *>(L.ws);
+    q.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(L.ws) + kStreamKFlagBytes);
+    int sms = num_sms();
+    if (sms > kStreamKMaxCtas)
+        sms = kStreamKMaxCtas;
+    const int64_t grid = q.units < sms ? q.units : sms;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(C::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = L.stream;
+    cudaLaunchAttribute attrs[2];
+    fill_attrs(cfg, attrs, 1, L.pdl);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_streamk_kernel<C>, tmX, tmW, tmW2, p, q);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    return PGF8_OK;
+}
+
 template <int KIND, bool SWAP, int BN, int STAGES>
 static pgf8_status launch_split_or_not(const GemmLaunch &L, int splits)
 {
@@ -231,8 +271,21 @@ template <int KIND> static pgf8_status launch_gemm(const GemmLaunch &L)
     int path = L.opts.path;
     int bn = L.opts.tile_n;
     int splits = L.opts.split_k;
+    const int sk_bn = L.M <= 16 ? 16 : 32;
+    const bool sk_ws = L.M <= 32 && L.ws != nullptr && L.ws_bytes >= streamk_workspace_bytes(sk_bn);
     if (path == PGF8_PATH_AUTO)
-        path = (L.M <= 128) ? PGF8_PATH_SKINNY : PGF8_PATH_TILED;
+        path = (L.M <= 32 && sk_ws && splits == 0 && bn == 0) ? PGF8_PATH_STREAMK
+               : (L.M <= 128)                                 ? PGF8_PATH_SKINNY
+                                                              : PGF8_PATH_TILED;
+    if (path == PGF8_PATH_STREAMK) {
+        if (L.M > 32)
+            return PGF8_ERR_UNSUPPORTED;
+        if (!sk_ws)
+            return PGF8_ERR_INVALID_ARG;
+        if (sk_bn == 16)
+            return launch_streamk<StreamKCfg<16, 6, KIND>>(L);
+        return launch_streamk<StreamKCfg<32, 5, KIND>>(L);
+    }
     if (path != PGF8_PATH_SKINNY && path != PGF8_PATH_TILED)
         return PGF8_ERR_INVALID_ARG;
     if (splits < 0 || splits > 8)
@@ -276,16 +329,16 @@ template <int KIND> static pgf8_status launch_gemm(const GemmLaunch &L)
         const int64_t waves = (t + sms - 1) / sms;
         return static_cast<double>(t) / static_cast<double>(waves * sms);
     };
+    // Tile choice (measured on B200 over the 7B prefill shapes): 128 x 256
+    // tiles in the persistent kernel whenever they give at least half a wave;
+    // with fewer tiles, a two-way cluster split of K for long K, else the
+    // narrower 128 x 128 tile.
+    const int64_t tiles256 = static_cast<int64_t>(mt) * ((L.N + 255) / 256);
+    const bool few = tiles256 * 2 < sms;
     if (bn == 0)
-        bn = (wave_eff(128) > wave_eff(256) + 0.15) ? 128 : 256;
-    if (splits == 0) {
-        // split K across a cluster only when there are too few tiles to
-        // occupy the SMs
-        const int tiles = mt * ((L.N + bn - 1) / bn);
-        splits = 1;
-        while (splits < 4 && tiles * (splits + 1) <= sms)
-            ++splits;
-    }
+        bn = (few && kblocks < 64) ? 128 : (wave_eff(128) > wave_eff(256) + 0.15 ? 128 : 256);
+    if (splits == 0)
+        splits = (few && bn == 256) ? 2 : 1;
     if (splits > kblocks)
         splits = kblocks;
     if (splits == 1) {
@@ -384,20 +437,25 @@ pgf8_status pgf8_fp8_quantize_rows(const void *x, pgf8_dtype xdt, int64_t rows, 
                            static_cast<cudaStream_t>(stream), 0, 0);
 }
 
-size_t pgf8_fp8_linear_workspace_size(int64_t, int64_t, int64_t) { return 0; }
+static size_t streamk_bytes_for(int64_t M) { return M >= 1 && M <= 32 ? streamk_workspace_bytes(M <= 16 ? 16 : 32) : 0; }
+
+size_t pgf8_fp8_linear_workspace_size(int64_t M, int64_t, int64_t) { return streamk_bytes_for(M); }
 
 pgf8_status pgf8_fp8_linear_ex(const uint8_t *aq, const float *sa, int64_t M, int64_t K, const uint8_t *wq,
-                               const float *sw, int64_t N, void *y, void *, size_t, const pgf8_linear_opts *opts,
-                               void *stream)
+                               const float *sw, int64_t N, void *y, void *workspace, size_t workspace_bytes,
+                               const pgf8_linear_opts *opts, void *stream)
 {
     pgf8_status st = check_dims(M, N, K);
     if (st != PGF8_OK)
         return st;
     if (!aq || !sa || !wq || !sw || !y)
         return PGF8_ERR_INVALID_ARG;
-    if (!aligned16(aq) || !aligned16(wq) || !aligned16(y) || !aligned4(sa) || !aligned4(sw))
+    if (!aligned16(aq) || !aligned16(wq) || !aligned16(y) || !aligned4(sa) || !aligned4(sw) ||
+        !aligned16(workspace))
         return PGF8_ERR_ALIGNMENT;
     GemmLaunch L;
+    L.ws = workspace;
+    L.ws_bytes = workspace ? workspace_bytes : 0;
     L.kind = kE4M3;
     L.x = aq;
     L.w = wq;
@@ -429,11 +487,17 @@ size_t pgf8_fp8_linear_dynamic_scales_offset(int64_t M, int64_t K)
     return round_up(static_cast<size_t>(M) * static_cast<size_t>(K), 256);
 }
 
+// Dynamic workspace: codes [M, K] | scales [M] | stream-K region (M <= 32).
+static size_t dynamic_streamk_offset(int64_t M, int64_t K)
+{
+    return pgf8_fp8_linear_dynamic_scales_offset(M, K) + round_up(static_cast<size_t>(M) * 4, 256);
+}
+
 size_t pgf8_fp8_linear_dynamic_workspace_size(int64_t M, int64_t, int64_t K)
 {
     if (M < 0 || K < 0)
         return 0;
-    return pgf8_fp8_linear_dynamic_scales_offset(M, K) + round_up(static_cast<size_t>(M) * 4, 256);
+    return dynamic_streamk_offset(M, K) + streamk_bytes_for(M);
 }
 
 static pgf8_status linear_dynamic_impl(const void *x, pgf8_dtype xdt, int64_t M, int64_t K, int64_t ldx,
@@ -464,6 +528,8 @@ static pgf8_status linear_dynamic_impl(const void *x, pgf8_dtype xdt, int64_t M,
     if (st != PGF8_OK)
         return st;
     GemmLaunch L;
+    L.ws = static_cast<uint8_t *>(workspace) + dynamic_streamk_offset(M, K);
+    L.ws_bytes = workspace_bytes - dynamic_streamk_offset(M, K);
     L.kind = kind;
     L.x = aq;
     L.w = w;
@@ -515,7 +581,7 @@ size_t pgf8_nestedfp_linear_workspace_size(int64_t M, int64_t N, int64_t K, pgf8
 {
     if (mode == PGF8_NESTED_FP8)
         return pgf8_fp8_linear_dynamic_workspace_size(M, N, K);
-    return 0;
+    return streamk_bytes_for(M);
 }
 
 pgf8_status pgf8_nestedfp_linear_ex(const void *x, int64_t M, int64_t K, const uint8_t *hi, const uint8_t *lo,
@@ -532,9 +598,11 @@ pgf8_status pgf8_nestedfp_linear_ex(const void *x, int64_t M, int64_t K, const u
         return st;
     if (!x || !hi || !lo || !y)
         return PGF8_ERR_INVALID_ARG;
-    if (!aligned16(x) || !aligned16(hi) || !aligned16(lo) || !aligned16(y))
+    if (!aligned16(x) || !aligned16(hi) || !aligned16(lo) || !aligned16(y) || !aligned16(workspace))
         return PGF8_ERR_ALIGNMENT;
     GemmLaunch L;
+    L.ws = workspace;
+    L.ws_bytes = workspace ? workspace_bytes : 0;
     L.kind = kNested16;
     L.x = x;
     L.w = hi;

@@ -28,12 +28,17 @@ def test_status_strings_and_version():
 
 
 def test_workspace_sizes():
-    assert pg.lib.pgf8_fp8_linear_workspace_size(16, 512, 512) == 0
+    # stream-K flags + partial slots for M <= 32, nothing above
+    assert pg.lib.pgf8_fp8_linear_workspace_size(16, 512, 512) >= 1024 + 256 * 16 * 128 * 4
+    assert pg.lib.pgf8_fp8_linear_workspace_size(32, 512, 512) >= 1024 + 256 * 32 * 128 * 4
+    assert pg.lib.pgf8_fp8_linear_workspace_size(33, 512, 512) == 0
     off = pg.lib.pgf8_fp8_linear_dynamic_scales_offset(3, 4096)
     assert off % 256 == 0 and off >= 3 * 4096
     ws = pg.lib.pgf8_fp8_linear_dynamic_workspace_size(3, 4096, 4096)
     assert ws >= off + 12 and ws % 256 == 0
-    assert pg.nestedfp_linear_workspace_size(8, 4096, 4096, pg.NESTED_FP16) == 0
+    assert pg.nestedfp_linear_workspace_size(64, 4096, 4096, pg.NESTED_FP16) == 0
+    assert pg.nestedfp_linear_workspace_size(8, 4096, 4096, pg.NESTED_FP16) == \
+        pg.lib.pgf8_fp8_linear_workspace_size(8, 4096, 4096)
     assert pg.nestedfp_linear_workspace_size(8, 4096, 4096, pg.NESTED_FP8) == \
         pg.lib.pgf8_fp8_linear_dynamic_workspace_size(8, 4096, 4096)
 
@@ -111,3 +116,19 @@ def test_dynamic_and_nested_reject_bad_args():
     s = pg.lib.pgf8_nestedfp_split
     assert s(None, 16, 16, B16, C16, None) == pg.ERR_INVALID_ARG
     assert s(A16, 3, 5, B16, C16, None) == pg.ERR_ALIGNMENT
+
+
+def test_streamk_path_argument_checks():
+    o = pg.LinearOpts(pg.PATH_STREAMK, 0, 0, 0)
+    # no workspace: rejected before launch
+    assert pg.lib.pgf8_fp8_linear_ex(A16, B16, 8, 512, C16, D16, 512, A16, None, 0, ctypes.byref(o),
+                                     None) == pg.ERR_INVALID_ARG
+    # workspace too small
+    assert pg.lib.pgf8_fp8_linear_ex(A16, B16, 8, 512, C16, D16, 512, A16, D16, 4096, ctypes.byref(o),
+                                     None) == pg.ERR_INVALID_ARG
+    # M > 32 is not served by the stream-K kernel
+    assert pg.lib.pgf8_fp8_linear_ex(A16, B16, 33, 512, C16, D16, 512, A16, D16, 1 << 24, ctypes.byref(o),
+                                     None) == pg.ERR_UNSUPPORTED
+    # misaligned workspace
+    assert pg.lib.pgf8_fp8_linear_ex(A16, B16, 8, 512, C16, D16, 512, A16, D16 + 8, 1 << 24, ctypes.byref(o),
+                                     None) == pg.ERR_ALIGNMENT

@@ -102,7 +102,7 @@ def test_dynamic_entry_point_matches_two_step():
     wt = _to(w)
     wq, sw = pg.fp8_quantize_rows(wt)
     xt = _to(x)
-    ws = torch.empty(pg.fp8_linear_dynamic_workspace_size(x.shape[0], w.shape[0], x.shape[1]),
+    ws = torch.zeros(pg.fp8_linear_dynamic_workspace_size(x.shape[0], w.shape[0], x.shape[1]),
                      dtype=torch.uint8, device=DEV)
     y = pg.fp8_linear_dynamic(xt, wq, sw, workspace=ws)
     torch.cuda.synchronize()
@@ -169,7 +169,7 @@ def test_dynamic_chain_with_overlap_flag_matches_unchained():
         wq, sw = pg.fp8_quantize_rows(_to(synthetic.weights_f16(N, K, 0.02, g)))
         Ws.append((wq, sw))
         Xs.append(_to(synthetic.activations("normal_outl_0p5pct_x30", 8, K, g)))
-    ws = torch.empty(max(pg.fp8_linear_dynamic_workspace_size(8, N, K) for K, N in shapes), dtype=torch.uint8,
+    ws = torch.zeros(max(pg.fp8_linear_dynamic_workspace_size(8, N, K) for K, N in shapes), dtype=torch.uint8,
                      device=DEV)
     torch.cuda.synchronize()
 
@@ -187,3 +187,26 @@ def test_dynamic_chain_with_overlap_flag_matches_unchained():
         for a, b in zip(run(pg.FLAG_OVERLAP_PREVIOUS, False), ref):
             np.testing.assert_array_equal(a, b)
     assert pg.device_status() == pg.OK
+
+
+STREAMK = [  # M <= 32; grids from 1 to 148 CTAs, tiles shared by up to 64 CTAs
+    (1, 16, 16), (1, 128, 8192), (3, 272, 1040), (16, 528, 4096), (17, 400, 2000), (32, 4096, 512),
+    (8, 12288, 4096), (5, 256, 11008),
+]
+
+
+@pytest.mark.parametrize("M,N,K", STREAMK)
+def test_streamk_against_oracle_and_flags_cleared(M, N, K):
+    g = np.random.default_rng(M * 7 + N * 13 + K)
+    x = synthetic.activations("normal_outl_0p5pct_x30", M, K, g)
+    w = synthetic.weights_f16(N, K, 0.02, g)
+    aq, sa, wq, sw, ref, bound = _oracle_case(x, w)
+    ws = torch.zeros(int(pg.lib.pgf8_fp8_linear_workspace_size(M, N, K)), dtype=torch.uint8, device=DEV)
+    outs = []
+    for _ in range(3):   # the flags must come back to zero for the next call
+        y = _run_linear(aq, sa, wq, sw, workspace=ws, path=pg.PATH_STREAMK)
+        assert ws[:1024].count_nonzero().item() == 0
+        assert_within(y, ref, bound, f"stream-K M{M} N{N} K{K}")
+        outs.append(y)
+    for y in outs[1:]:
+        np.testing.assert_array_equal(y, outs[0])

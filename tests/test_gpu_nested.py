@@ -151,3 +151,22 @@ def test_chained_layers_with_overlap_flag(mode):
         for a, b in zip(got, ref):
             np.testing.assert_array_equal(a.view(np.uint16), b.view(np.uint16))
     assert pg.device_status() == pg.OK
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 128, 4096), (16, 528, 1040), (30, 272, 2048)])
+@pytest.mark.parametrize("mode", ["fp16", "fp8"])
+def test_nested_streamk(M, N, K, mode):
+    g = np.random.default_rng(M + N + K)
+    x16 = synthetic.activations("normal_f16", M, K, g)
+    w16 = synthetic.weights_f16(N, K, 0.02, g)
+    hi, lo = oracle.nestedfp_split(w16)
+    if mode == "fp16":
+        ref, bound = _ref16(x16, hi, lo)
+        m = pg.NESTED_FP16
+    else:
+        ref, bound, _, _ = _ref8(x16, hi)
+        m = pg.NESTED_FP8
+    ws = torch.zeros(pg.nestedfp_linear_workspace_size(M, N, K, m), dtype=torch.uint8, device=DEV)
+    for _ in range(2):
+        y = _run(x16, hi, lo if m == pg.NESTED_FP16 else None, m, workspace=ws, path=pg.PATH_STREAMK)
+        assert_within(y, ref, bound, f"{mode} stream-K M{M} N{N} K{K}")
