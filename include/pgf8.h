@@ -152,9 +152,11 @@ size_t pgf8_fp8_linear_workspace_size(int64_t M, int64_t N, int64_t K);
  * quantisation ("7B on an RTX 4060 with FP8" §2.2: activations quantised at
  * run time).  x [M,K] f32 or f16 with row stride ldx.  The workspace
  * (size from pgf8_fp8_linear_dynamic_workspace_size; zero-filled before its
- * first use) receives the E4M3 activation codes [M,K] at offset 0 and the
- * per-token scales [M] at offset pgf8_fp8_linear_dynamic_scales_offset(M, K);
- * the caller may read both after the call completes.  wq must not be written by work enqueued
+ * first use) receives the E4M3 activation codes [M,K] at byte offset
+ * pgf8_fp8_linear_dynamic_codes_offset(M, K) and the per-token scales [M] at
+ * pgf8_fp8_linear_dynamic_scales_offset(M, K); the caller may read both after
+ * the call completes.  Its first 1024 bytes are synchronisation words for
+ * every shape, so one workspace can serve layers of different shapes.  wq must not be written by work enqueued
  * between this call's quantisation and GEMM (nothing is).
  * ---------------------------------------------------------------------- */
 pgf8_status pgf8_fp8_linear_dynamic(const void *x, pgf8_dtype xdt, int64_t M, int64_t K,
@@ -163,6 +165,7 @@ pgf8_status pgf8_fp8_linear_dynamic(const void *x, pgf8_dtype xdt, int64_t M, in
                                     const pgf8_linear_opts *opts, void *stream);
 
 size_t pgf8_fp8_linear_dynamic_workspace_size(int64_t M, int64_t N, int64_t K);
+size_t pgf8_fp8_linear_dynamic_codes_offset(int64_t M, int64_t K);
 size_t pgf8_fp8_linear_dynamic_scales_offset(int64_t M, int64_t K);
 
 /* ------------------------------------------------------------------------

@@ -6,7 +6,7 @@ This module is the Python binding of ``libpgf8.so`` (the C ABI declared in
 buffers (PyTorch is used for device memory and streams), every computation
 runs in the library's CUDA kernels, and there is no other code path.  If the
 library has not been built the import fails; build it with
-``python -m precision_gemm_fp8_b200.build``.
+``python precision_gemm_fp8_b200/build.py``.
 """
 from __future__ import annotations
 
@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_PKG, "libpgf8.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "pgf8.h")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m precision_gemm_fp8_b200.build` "
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python precision_gemm_fp8_b200/build.py` "
                       "(the CUDA library is the only implementation)")
 
 lib = ctypes.CDLL(LIB_PATH)
@@ -52,6 +52,7 @@ _SIGS = {
     "pgf8_fp8_linear_workspace_size": ([_i64, _i64, _i64], _sz),
     "pgf8_fp8_linear_dynamic": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _sz, _optp, _vp], _i32),
     "pgf8_fp8_linear_dynamic_workspace_size": ([_i64, _i64, _i64], _sz),
+    "pgf8_fp8_linear_dynamic_codes_offset": ([_i64, _i64], _sz),
     "pgf8_fp8_linear_dynamic_scales_offset": ([_i64, _i64], _sz),
     "pgf8_nestedfp_split": ([_vp, _i64, _i64, _vp, _vp, _vp], _i32),
     "pgf8_nestedfp_linear": ([_vp, _i64, _i64, _vp, _vp, _i64, _i32, _vp, _vp, _sz, _vp], _i32),
@@ -206,8 +207,9 @@ def fp8_linear_dynamic(x, wq, sw, y=None, workspace=None, path=PATH_AUTO, split_
 
 def dynamic_workspace_views(workspace: torch.Tensor, M: int, K: int):
     """(aq [M,K] uint8, sa [M] f32) views of a dynamic-linear workspace."""
+    c0 = int(lib.pgf8_fp8_linear_dynamic_codes_offset(M, K))
     off = int(lib.pgf8_fp8_linear_dynamic_scales_offset(M, K))
-    aq = workspace[:M * K].view(M, K)
+    aq = workspace[c0:c0 + M * K].view(M, K)
     sa = workspace[off:off + 4 * M].view(torch.float32)
     return aq, sa
 

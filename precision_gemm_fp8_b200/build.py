@@ -1,6 +1,7 @@
 """Build libpgf8.so (the CUDA kernels + C ABI) in-tree for sm_100a.
 
-Usage: python -m precision_gemm_fp8_b200.build [--force] [--verbose-ptxas]
+Usage: python precision_gemm_fp8_b200/build.py [--force] [--verbose-ptxas]
+(run it by path: importing the package loads the library this script builds)
 """
 from __future__ import annotations
 

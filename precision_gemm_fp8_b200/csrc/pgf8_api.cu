@@ -480,24 +480,28 @@ pgf8_status pgf8_fp8_linear(const uint8_t *aq, const float *sa, int64_t M, int64
     return pgf8_fp8_linear_ex(aq, sa, M, K, wq, sw, N, y, workspace, workspace_bytes, nullptr, stream);
 }
 
+// Dynamic workspace layout: stream-K flag words (always, so they are never
+// overwritten by codes when one workspace serves layers of different shapes)
+// | stream-K partial slots (M <= 32) | codes [M, K] | scales [M].
+size_t pgf8_fp8_linear_dynamic_codes_offset(int64_t M, int64_t K)
+{
+    if (M < 0 || K < 0)
+        return 0;
+    return M >= 1 && M <= 32 ? streamk_bytes_for(M) : kStreamKFlagBytes;
+}
+
 size_t pgf8_fp8_linear_dynamic_scales_offset(int64_t M, int64_t K)
 {
     if (M < 0 || K < 0)
         return 0;
-    return round_up(static_cast<size_t>(M) * static_cast<size_t>(K), 256);
-}
-
-// Dynamic workspace: codes [M, K] | scales [M] | stream-K region (M <= 32).
-static size_t dynamic_streamk_offset(int64_t M, int64_t K)
-{
-    return pgf8_fp8_linear_dynamic_scales_offset(M, K) + round_up(static_cast<size_t>(M) * 4, 256);
+    return pgf8_fp8_linear_dynamic_codes_offset(M, K) + round_up(static_cast<size_t>(M) * static_cast<size_t>(K), 256);
 }
 
 size_t pgf8_fp8_linear_dynamic_workspace_size(int64_t M, int64_t, int64_t K)
 {
     if (M < 0 || K < 0)
         return 0;
-    return dynamic_streamk_offset(M, K) + streamk_bytes_for(M);
+    return pgf8_fp8_linear_dynamic_scales_offset(M, K) + round_up(static_cast<size_t>(M) * 4, 256);
 }
 
 static pgf8_status linear_dynamic_impl(const void *x, pgf8_dtype xdt, int64_t M, int64_t K, int64_t ldx,
@@ -514,8 +518,9 @@ static pgf8_status linear_dynamic_impl(const void *x, pgf8_dtype xdt, int64_t M,
         return PGF8_ERR_INVALID_ARG;
     if (!aligned16(workspace) || !aligned16(w) || !aligned16(y) || (sw && !aligned4(sw)))
         return PGF8_ERR_ALIGNMENT;
-    uint8_t *aq = static_cast<uint8_t *>(workspace);
-    float *sa = reinterpret_cast<float *>(aq + pgf8_fp8_linear_dynamic_scales_offset(M, K));
+    uint8_t *aq = static_cast<uint8_t *>(workspace) + pgf8_fp8_linear_dynamic_codes_offset(M, K);
+    float *sa = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                          pgf8_fp8_linear_dynamic_scales_offset(M, K));
     st = check_quantize_args(x, xdt, M, K, ldx, aq, sa, PGF8_SCALE_DYNAMIC);
     if (st != PGF8_OK)
         return st;
@@ -528,8 +533,8 @@ static pgf8_status linear_dynamic_impl(const void *x, pgf8_dtype xdt, int64_t M,
     if (st != PGF8_OK)
         return st;
     GemmLaunch L;
-    L.ws = static_cast<uint8_t *>(workspace) + dynamic_streamk_offset(M, K);
-    L.ws_bytes = workspace_bytes - dynamic_streamk_offset(M, K);
+    L.ws = workspace;   // the stream-K region is at offset 0
+    L.ws_bytes = pgf8_fp8_linear_dynamic_codes_offset(M, K);
     L.kind = kind;
     L.x = aq;
     L.w = w;

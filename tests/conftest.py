@@ -28,3 +28,19 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def _build_native():
+    """Build the CUDA library (and the oracle) before collection when they are
+    missing or older than their sources; the build script is loaded by path."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("pgf8_build",
+                                                  os.path.join(ROOT, "precision_gemm_fp8_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+    import oracle
+    oracle.build()
+
+
+_build_native()

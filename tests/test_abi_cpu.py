@@ -32,10 +32,13 @@ def test_workspace_sizes():
     assert pg.lib.pgf8_fp8_linear_workspace_size(16, 512, 512) >= 1024 + 256 * 16 * 128 * 4
     assert pg.lib.pgf8_fp8_linear_workspace_size(32, 512, 512) >= 1024 + 256 * 32 * 128 * 4
     assert pg.lib.pgf8_fp8_linear_workspace_size(33, 512, 512) == 0
-    off = pg.lib.pgf8_fp8_linear_dynamic_scales_offset(3, 4096)
-    assert off % 256 == 0 and off >= 3 * 4096
-    ws = pg.lib.pgf8_fp8_linear_dynamic_workspace_size(3, 4096, 4096)
-    assert ws >= off + 12 and ws % 256 == 0
+    for M in (3, 40):
+        c0 = pg.lib.pgf8_fp8_linear_dynamic_codes_offset(M, 4096)
+        off = pg.lib.pgf8_fp8_linear_dynamic_scales_offset(M, 4096)
+        assert c0 >= 1024 and c0 % 256 == 0          # synchronisation words first, for every shape
+        assert off % 256 == 0 and off >= c0 + M * 4096
+        ws = pg.lib.pgf8_fp8_linear_dynamic_workspace_size(M, 4096, 4096)
+        assert ws >= off + 4 * M and ws % 256 == 0
     assert pg.nestedfp_linear_workspace_size(64, 4096, 4096, pg.NESTED_FP16) == 0
     assert pg.nestedfp_linear_workspace_size(8, 4096, 4096, pg.NESTED_FP16) == \
         pg.lib.pgf8_fp8_linear_workspace_size(8, 4096, 4096)
