@@ -306,6 +306,32 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         const int qd = warp & 3;
         const int r = qd * 32 + lane;
         const uint32_t t_row = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+        // Output of one accumulator row of tile t (this thread: channel n).
+        auto store_row = [&](int t, const float (&a)[BN]) {
+            const int n = t * 128 + r;
+            if (n < p.N) {
+                float swn = 1.0f;
+                if constexpr (KIND == kE4M3)
+                    swn = p.sw[n];
+#pragma unroll
+                for (int j = 0; j < BN; ++j) {
+                    if (j < p.M) {
+                        float v = a[j];
+                        if constexpr (KIND != kNested16)
+                            v = v * p.sa[j];
+                        if constexpr (KIND == kE4M3)
+                            v = v * swn;
+                        store_out<KIND>(p.y, static_cast<int64_t>(j) * p.N + n, v);
+                    }
+                }
+            }
+        };
+        // The first segment may finish a tile started by preceding CTAs; its
+        // values wait in registers until the end, so that this CTA publishes
+        // its own partial (its last segment) first and no CTA ever waits on a
+        // CTA that is itself waiting.
+        float first[BN];
+        int deferred_tile = -1;
         int i = 0;
         for (int64_t u = u0; u < u1; ++i) {
             const int t = static_cast<int>(u / kbt);
@@ -333,7 +359,6 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             if (lane == 0)
                 mbar_arrive(&ctl->acc_empty[buf]);   // accumulator values are in registers now
 
-            const int n = t * 128 + r;
             if (!tile_done) {
                 // a partial of a shared tile: always this CTA's last segment
                 float *slot = q.partials + static_cast<size_t>(c) * BN * 128;
@@ -344,51 +369,44 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                 asm volatile("bar.sync 2, 128;" ::: "memory");
                 if (r == 0)
                     st_release_u32(q.flags + c, 1u);
+            } else if (kb_first > 0) {
+                // finishes a shared tile: always this CTA's first segment
+#pragma unroll
+                for (int j = 0; j < BN; ++j)
+                    first[j] = a[j];
+                deferred_tile = t;
             } else {
-                if (kb_first > 0) {
-                    // finish a shared tile: add the preceding CTAs' partials in order
-                    const int c_first = sk_owner(static_cast<int64_t>(t) * kbt, q.units, G);
-                    float sum[BN];
-#pragma unroll
-                    for (int j = 0; j < BN; ++j)
-                        sum[j] = 0.0f;
-                    bool got = true;
-                    for (int cc = c_first; cc < c; ++cc) {
-                        if (!wait_flag(q.flags + cc, abort_flag)) {
-                            got = false;
-                            break;
-                        }
-                        const float *slot = q.partials + static_cast<size_t>(cc) * BN * 128;
-#pragma unroll
-                        for (int j = 0; j < BN; ++j)
-                            sum[j] += __ldcg(slot + j * 128 + r);
-                    }
-#pragma unroll
-                    for (int j = 0; j < BN; ++j)
-                        a[j] = sum[j] + a[j];
-                    asm volatile("bar.sync 2, 128;" ::: "memory");
-                    if (got && r == 0)
-                        for (int cc = c_first; cc < c; ++cc)
-                            q.flags[cc] = 0u;
-                }
-                if (n < p.N) {
-                    float swn = 1.0f;
-                    if constexpr (KIND == kE4M3)
-                        swn = p.sw[n];
-#pragma unroll
-                    for (int j = 0; j < BN; ++j) {
-                        if (j < p.M) {
-                            float v = a[j];
-                            if constexpr (KIND != kNested16)
-                                v = v * p.sa[j];
-                            if constexpr (KIND == kE4M3)
-                                v = v * swn;
-                            store_out<KIND>(p.y, static_cast<int64_t>(j) * p.N + n, v);
-                        }
-                    }
-                }
+                store_row(t, a);
             }
             u = seg_end;
+        }
+        if (deferred_tile >= 0) {
+            // add the preceding CTAs' partials in CTA order, then this CTA's own
+            const int t = deferred_tile;
+            const int c_first = sk_owner(static_cast<int64_t>(t) * kbt, q.units, G);
+            float sum[BN];
+#pragma unroll
+            for (int j = 0; j < BN; ++j)
+                sum[j] = 0.0f;
+            bool got = true;
+            for (int cc = c_first; cc < c; ++cc) {
+                if (!wait_flag(q.flags + cc, abort_flag)) {
+                    got = false;
+                    break;
+                }
+                const float *slot = q.partials + static_cast<size_t>(cc) * BN * 128;
+#pragma unroll
+                for (int j = 0; j < BN; ++j)
+                    sum[j] += __ldcg(slot + j * 128 + r);
+            }
+#pragma unroll
+            for (int j = 0; j < BN; ++j)
+                sum[j] = sum[j] + first[j];
+            asm volatile("bar.sync 2, 128;" ::: "memory");
+            if (got && r == 0)
+                for (int cc = c_first; cc < c; ++cc)
+                    q.flags[cc] = 0u;
+            store_row(t, sum);
         }
     } else {
         // ------------------------------------------------------------ FP16 rebuild
