@@ -27,10 +27,11 @@
  *               it synchronises on zero again, so it can be reused without
  *               clearing.  After PGF8_ERR_TIMEOUT, zero it again.  One
  *               workspace serves one call at a time (calls on different
- *               streams need different workspaces).  For M <= 32 the linear
- *               entry points use it for the stream-K kernel (flags, partial
- *               tiles); with a NULL or short workspace they choose a kernel
- *               that needs none.
+ *               streams need different workspaces).  For M <= 32 the
+ *               stream-K kernel (PGF8_PATH_STREAMK, chosen only on request)
+ *               keeps its flags and partial tiles there; the kernels chosen
+ *               by PGF8_PATH_AUTO need none beyond the dynamic entry points'
+ *               activation codes and scales.
  *   Layout      Row-major, last index contiguous: activations x/aq [M, K],
  *               weights w/wq/hi/lo [N, K] (K contiguous, "TN"), outputs
  *               y [M, N].  Row strides equal the row length unless an

@@ -13,6 +13,17 @@
 #include "gemm_streamk.cuh"
 #include "quantize.cuh"
 
+// Pipeline depths and stream-K occupancy (compile-time tuning constants).
+#ifndef PGF8_SKINNY16_STAGES
+#define PGF8_SKINNY16_STAGES 6
+#endif
+#ifndef PGF8_STREAMK16_STAGES
+#define PGF8_STREAMK16_STAGES 6
+#endif
+#ifndef PGF8_STREAMK_CTAS_PER_SM
+#define PGF8_STREAMK_CTAS_PER_SM 1
+#endif
+
 namespace pgf8 {
 
 static thread_local int tl_last_cuda_error = 0;
@@ -224,10 +235,10 @@ template <class C> static pgf8_status launch_streamk(const GemmLaunch &L)
     q.units = static_cast<int64_t>((L.N + 127) / 128) * p.kblocks;
     q.flags = static_cast<unsigned *>(L.ws);
     q.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(L.ws) + kStreamKFlagBytes);
-    int sms = num_sms();
-    if (sms > kStreamKMaxCtas)
-        sms = kStreamKMaxCtas;
-    const int64_t grid = q.units < sms ? q.units : sms;
+    int slots = num_sms() * PGF8_STREAMK_CTAS_PER_SM;
+    if (slots > kStreamKMaxCtas)
+        slots = kStreamKMaxCtas;
+    const int64_t grid = q.units < slots ? q.units : slots;
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
@@ -273,17 +284,18 @@ template <int KIND> static pgf8_status launch_gemm(const GemmLaunch &L)
     int splits = L.opts.split_k;
     const int sk_bn = L.M <= 16 ? 16 : 32;
     const bool sk_ws = L.M <= 32 && L.ws != nullptr && L.ws_bytes >= streamk_workspace_bytes(sk_bn);
+    // AUTO never picks stream-K: on B200 the cluster split-K kernel streams
+    // the decode shapes faster (its partial tiles stay in distributed shared
+    // memory instead of a global fix-up); stream-K is selected explicitly.
     if (path == PGF8_PATH_AUTO)
-        path = (L.M <= 32 && sk_ws && splits == 0 && bn == 0) ? PGF8_PATH_STREAMK
-               : (L.M <= 128)                                 ? PGF8_PATH_SKINNY
-                                                              : PGF8_PATH_TILED;
+        path = (L.M <= 128) ? PGF8_PATH_SKINNY : PGF8_PATH_TILED;
     if (path == PGF8_PATH_STREAMK) {
         if (L.M > 32)
             return PGF8_ERR_UNSUPPORTED;
         if (!sk_ws)
             return PGF8_ERR_INVALID_ARG;
         if (sk_bn == 16)
-            return launch_streamk<StreamKCfg<16, 6, KIND>>(L);
+            return launch_streamk<StreamKCfg<16, PGF8_STREAMK16_STAGES, KIND>>(L);
         return launch_streamk<StreamKCfg<32, 5, KIND>>(L);
     }
     if (path != PGF8_PATH_SKINNY && path != PGF8_PATH_TILED)
@@ -316,7 +328,7 @@ template <int KIND> static pgf8_status launch_gemm(const GemmLaunch &L)
         if (splits > kblocks)
             splits = kblocks;
         switch (bn) {
-        case 16: return launch_split_or_not<KIND, true, 16, 6>(L, splits);
+        case 16: return launch_split_or_not<KIND, true, 16, PGF8_SKINNY16_STAGES>(L, splits);
         case 32: return launch_split_or_not<KIND, true, 32, 8>(L, splits);
         case 64: return launch_split_or_not<KIND, true, 64, 8>(L, splits);
         default: return launch_split_or_not<KIND, true, 128, 6>(L, splits);
