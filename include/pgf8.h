@@ -68,7 +68,8 @@ typedef enum {
     PGF8_ERR_ALIGNMENT = 2,
     PGF8_ERR_UNSUPPORTED = 3,
     PGF8_ERR_CUDA = 4,
-    PGF8_ERR_TIMEOUT = 5
+    PGF8_ERR_TIMEOUT = 5,
+    PGF8_ERR_TOO_LARGE = 6
 } pgf8_status;
 
 typedef enum { PGF8_F32 = 0, PGF8_F16 = 1, PGF8_BF16 = 2 } pgf8_dtype;
@@ -200,6 +201,40 @@ pgf8_status pgf8_nestedfp_linear_ex(const void *x_f16, int64_t M, int64_t K, con
 
 size_t pgf8_nestedfp_linear_workspace_size(int64_t M, int64_t N, int64_t K,
                                            pgf8_nested_mode mode);
+
+/* ------------------------------------------------------------------------
+ * Allocation-free dynamic FP8 linear.  The pages have no counterpart of this
+ * entry point; it exists for callers that cannot hand the library a
+ * workspace: a host program that links only this C library and has no
+ * device allocator of its own, or an inference runtime whose device memory
+ * is planned once before serving and which must not allocate on the request
+ * path.
+ *
+ * It computes exactly what pgf8_fp8_linear_dynamic computes (same kernels,
+ * same results), but keeps the activation codes and scales in a fixed array
+ * inside the library (PGF8_NOALLOC_SCRATCH_BYTES, 8 MiB, held by every GPU
+ * that loads the library until the process exits).  The caller still passes
+ * x, wq, sw and y.  Nothing is allocated and no allocating routine is
+ * called.
+ *   Limit   pgf8_fp8_linear_dynamic_workspace_size(M, N, K) must not exceed
+ *           PGF8_NOALLOC_SCRATCH_BYTES, else PGF8_ERR_TOO_LARGE is returned
+ *           before anything is enqueued (e.g. M = 16 allows K up to ~350k;
+ *           M = 1024 allows K up to ~8k).
+ *   Set-up  The first call on each device, with that device current, looks
+ *           up the array's device address (cudaGetSymbolAddress); make that
+ *           first call before any stream capture begins.
+ *   Sharing Every call uses the same array and it keeps the last call's
+ *           codes and scales.  Nothing in it needs clearing (each call
+ *           writes the codes and scales before its GEMM reads them), but
+ *           calls whose work overlaps on the GPU (different streams, or
+ *           different host threads on one device) race on the array: order
+ *           them on one stream.
+ * ---------------------------------------------------------------------- */
+#define PGF8_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+pgf8_status pgf8_fp8_linear_dynamic_noalloc(const void *x, pgf8_dtype xdt, int64_t M, int64_t K,
+                                            int64_t ldx, const uint8_t *wq, const float *sw,
+                                            int64_t N, void *y_bf16, void *stream);
 
 /* ------------------------------------------------------------------------
  * Diagnostics.

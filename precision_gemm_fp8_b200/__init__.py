@@ -26,7 +26,8 @@ if not os.path.exists(LIB_PATH):
 
 lib = ctypes.CDLL(LIB_PATH)
 
-OK, ERR_INVALID_ARG, ERR_ALIGNMENT, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = range(6)
+OK, ERR_INVALID_ARG, ERR_ALIGNMENT, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_TOO_LARGE = range(7)
+NOALLOC_SCRATCH_BYTES = 8 << 20
 F32, F16, BF16 = 0, 1, 2
 SCALE_DYNAMIC, SCALE_STATIC = 0, 1
 NESTED_FP16, NESTED_FP8 = 0, 1
@@ -58,6 +59,7 @@ _SIGS = {
     "pgf8_nestedfp_linear": ([_vp, _i64, _i64, _vp, _vp, _i64, _i32, _vp, _vp, _sz, _vp], _i32),
     "pgf8_nestedfp_linear_ex": ([_vp, _i64, _i64, _vp, _vp, _i64, _i32, _vp, _vp, _sz, _optp, _vp], _i32),
     "pgf8_nestedfp_linear_workspace_size": ([_i64, _i64, _i64, _i32], _sz),
+    "pgf8_fp8_linear_dynamic_noalloc": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _i64, _vp, _vp], _i32),
     "pgf8_last_cuda_error": ([ctypes.POINTER(ctypes.c_int)], _i32),
     "pgf8_device_status": ([_vp], _i32),
     "pgf8_status_str": ([_i32], ctypes.c_char_p),
@@ -202,6 +204,23 @@ def fp8_linear_dynamic(x, wq, sw, y=None, workspace=None, path=PATH_AUTO, split_
     _check(lib.pgf8_fp8_linear_dynamic(_ptr(x), _dtype_code(x), M, K, x.stride(0), _ptr(wq), _ptr(sw), N, _ptr(y),
                                        _ptr(workspace), workspace.numel() * workspace.element_size(),
                                        _opts(path, split_k, tile_n, flags), _stream(stream)), "fp8_linear_dynamic")
+    return y
+
+
+def fp8_linear_dynamic_noalloc(x, wq, sw, y=None, stream=None):
+    """fp8_linear_dynamic without a workspace, for callers that cannot allocate
+    one: the codes and scales live in the library's fixed 8 MiB device array
+    (shared by all calls on a device; keep such calls on one stream).  Raises
+    Pgf8Error(ERR_TOO_LARGE) when the problem does not fit.  (Allocating y
+    here is this wrapper's convenience; pass y to allocate nothing.)"""
+    M, K = x.shape
+    N = wq.shape[0]
+    if x.stride(1) != 1:
+        raise ValueError("x rows must be contiguous")
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _check(lib.pgf8_fp8_linear_dynamic_noalloc(_ptr(x), _dtype_code(x), M, K, x.stride(0), _ptr(wq), _ptr(sw), N,
+                                               _ptr(y), _stream(stream)), "fp8_linear_dynamic_noalloc")
     return y
 
 

@@ -680,10 +680,66 @@ const char *pgf8_status_str(pgf8_status s)
     case PGF8_ERR_UNSUPPORTED: return "unsupported configuration";
     case PGF8_ERR_CUDA: return "CUDA error";
     case PGF8_ERR_TIMEOUT: return "device-side bounded wait expired";
+    case PGF8_ERR_TOO_LARGE: return "problem exceeds the fixed scratch array of the allocation-free entry point";
     }
     return "unknown status";
 }
 
 int pgf8_version(void) { return 100; }
+
+} // extern "C"
+
+// ------------------------------------------------------------------ allocation-free entry point
+// The scratch of pgf8_fp8_linear_dynamic_noalloc: a fixed array in device
+// memory (zero-filled at module load like any static storage).  In host code
+// its name is only a host-side stand-in, so its device address is looked up
+// once per device with cudaGetSymbolAddress and passed to the kernels.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[PGF8_NOALLOC_SCRATCH_BYTES];
+
+namespace pgf8 {
+constexpr int kMaxDevices = 64;
+static std::mutex g_noalloc_mutex;
+static void *g_noalloc_addr[kMaxDevices];
+
+// Device address of the scratch array on the current device (set-up on the
+// first call per device, with that device current).
+static pgf8_status noalloc_scratch(void **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices)
+        return PGF8_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess)
+            return cuda_fail(e);
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return PGF8_OK;
+}
+} // namespace pgf8
+
+extern "C" {
+
+pgf8_status pgf8_fp8_linear_dynamic_noalloc(const void *x, pgf8_dtype xdt, int64_t M, int64_t K, int64_t ldx,
+                                            const uint8_t *wq, const float *sw, int64_t N, void *y, void *stream)
+{
+    pgf8_status st = check_dims(M, N, K);
+    if (st != PGF8_OK)
+        return st;
+    const size_t need = pgf8_fp8_linear_dynamic_workspace_size(M, N, K);
+    if (need > PGF8_NOALLOC_SCRATCH_BYTES)
+        return PGF8_ERR_TOO_LARGE;
+    void *scratch = nullptr;
+    st = noalloc_scratch(&scratch);
+    if (st != PGF8_OK)
+        return st;
+    return pgf8_fp8_linear_dynamic(x, xdt, M, K, ldx, wq, sw, N, y, scratch, need, nullptr, stream);
+}
 
 } // extern "C"
