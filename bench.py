@@ -174,6 +174,59 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+# ----------------------------------------------------------------------------- profiled traffic
+def kernel_sources_hash() -> str:
+    """Short hash of the CUDA sources: profiled counters only describe the
+    kernels they were taken on."""
+    import hashlib
+    csrc = os.path.join(ROOT, "precision_gemm_fp8_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(hashlib.sha256(fh.read()).hexdigest().encode() + b"  " + f.encode() + b"\n")
+    return h.hexdigest()[:12]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes (read + write) per launch of the profiled GEMM of this
+    workload, from profiles/gemm_traffic.txt, scaled to the workload's average
+    launch by algorithmic bytes; None when the kernels changed since the
+    capture."""
+    path = os.path.join(ROOT, "profiles", "gemm_traffic.txt")
+    try:
+        with open(path) as f:
+            for line in f:
+                parts = line.split()
+                if len(parts) >= 5 and not line.startswith("#") and parts[0] == workload:
+                    src_hash, traffic, algo = parts[1], float(parts[2]), float(parts[3])
+                    if src_hash != kernel_sources_hash():
+                        return None, "kernels changed since the ncu capture"
+                    return traffic, (f"ncu capture of {parts[4]}: DRAM read+write {traffic:.0f} B per launch vs "
+                                     f"{algo:.0f} algorithmic B ({traffic / algo:.3f}x)")
+    except OSError:
+        pass
+    return None, "no capture recorded"
+
+
+# ----------------------------------------------------------------------------- ranks
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest value of x over all ranks (timings are reported as the
+    slowest rank's); a no-op for a single process."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, max_seconds: float) -> float:
+    """Whole-job throughput: every rank processed units_per_rank units (weak
+    scaling, independent replicas), the job took the slowest rank's time."""
+    return units_per_rank * world / max_seconds
+
+
 # ----------------------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -237,6 +290,7 @@ def run_ours(args, rank, world, local_rank):
                                           flags=pg.FLAG_OVERLAP_PREVIOUS, stream=stream)
                     continue
                 aq, sa = pg.dynamic_workspace_views(qbufs[i], L.M, L.K)
+                ev_pairs[i][2].record(stream)
                 pg.fp8_quantize_rows(acts[i], aq, sa, stream=stream)
                 ev_pairs[i][0].record(stream)
                 pg.fp8_linear(aq, sa, W[0], W[1], y=outs[i], workspace=sk_ws, stream=stream)
@@ -258,8 +312,7 @@ def run_ours(args, rank, world, local_rank):
     R = max(1, min(10, K))
     while K % R:
         R -= 1
-    evs = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
-           for _ in layers]
+    evs = [tuple(torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)) for _ in layers]
     with torch.cuda.stream(stream):
         enqueue_step()          # load modules / first-call set-up outside capture
         enqueue_step(evs)
@@ -294,24 +347,21 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
-    ms_total = t0.elapsed_time(t1)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(t0.elapsed_time(t1), world, dev)
     st = pg.device_status(stream)
     if st != pg.OK:
         raise RuntimeError(f"device error word raised in the timed region: {st}")
 
     # per-GEMM durations (ms) from the event-bracketed step of the last replay
     per_layer_ms = np.array([evs[i][0].elapsed_time(evs[i][1]) for i in range(len(layers))])
+    quant_ms = np.array([evs[i][2].elapsed_time(evs[i][0]) if L.kind == "fp8" else 0.0
+                         for i, L in enumerate(layers)])
 
     ms_step = ms_total / K
     wbytes = sum(L.weight_bytes for L in layers)
     flops = sum(L.flops for L in layers)
-    gbs = wbytes / (ms_step * 1e-3) / 1e9
-    tflops = flops / (ms_step * 1e-3) / 1e12
+    gbs = job_throughput(wbytes / 1e9, world, ms_step * 1e-3)        # whole job, all ranks
+    tflops = job_throughput(flops / 1e12, world, ms_step * 1e-3)
 
     # roofline of the dominant kernel (the GEMM)
     gemm_bytes = sum(L.gemm_bytes for L in layers)
@@ -332,7 +382,12 @@ def run_ours(args, rank, world, local_rank):
                 "peak_source": f"{peak_src} bf16 burst x 2 (FP8 nominal ratio)"}
     roof["kernel"] = "pgf8::gemm_kernel"
     roof["launches_timed"] = int(len(layers))
-    roof["gemm_share_of_step"] = round(float(per_layer_ms.sum()) / ms_step, 3)
+    # share of the GEMM among this step's kernels, each timed alone (the
+    # figure to compare with the ncu launch list, which also serialises)
+    roof["gemm_share_of_kernel_time"] = round(float(per_layer_ms.sum()) /
+                                              float(per_layer_ms.sum() + quant_ms.sum()), 3)
+    roof["gemm_isolated_sum_over_chained_step"] = round(float(per_layer_ms.sum()) / ms_step, 3)
+    roof["traffic"], roof["traffic_note"] = profiled_traffic(name)
 
     per_layer = []
     for L, t in zip(layers, per_layer_ms):
@@ -345,7 +400,7 @@ def run_ours(args, rank, world, local_rank):
 
     result = {
         "metric": METRIC,
-        "value": round((gbs if memory_bound else tflops) * world, 2),
+        "value": round(gbs if memory_bound else tflops, 2),
         "unit": "GB/s" if memory_bound else "TFLOP/s",
         "n_gpus": world,
         "steps": K,
@@ -361,7 +416,7 @@ def run_ours(args, rank, world, local_rank):
                          % (copies, wbytes / 1e6),
                    "timing": "CUDA graph of the C-ABI calls (R-1 chained steps + 1 event-bracketed step), "
                              "replayed K/R times, R=%d" % R},
-        "secondary": {"tflops": round(tflops * world, 3), "weight_gbs": round(gbs * world, 1)},
+        "secondary": {"tflops": round(tflops, 3), "weight_gbs": round(gbs, 1)},
         "roofline": roof,
         "e2e": e2e,
         "gpu_launches": int(launches_per_step * K),
@@ -412,16 +467,11 @@ def run_e2e(pg, torch, dev, layers, weights, acts_host, outs, args, world, wbyte
         step()
     t1.record(stream)
     stream.synchronize()
-    ms = t0.elapsed_time(t1) / steps
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, world, dev)
     h2d = sum(x.numel() * x.element_size() for x in acts_host)
     d2h = sum(o.numel() * o.element_size() for o in outs)
-    v = (wbytes / (ms * 1e-3) / 1e9) if memory_bound else (flops / (ms * 1e-3) / 1e12)
-    return {"value": round(v * world, 2), "unit": "GB/s" if memory_bound else "TFLOP/s",
+    v = job_throughput(wbytes / 1e9 if memory_bound else flops / 1e12, world, ms * 1e-3)
+    return {"value": round(v, 2), "unit": "GB/s" if memory_bound else "TFLOP/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
             "ms_per_step": round(ms, 5), "entry_point": "fp8_linear_dynamic / nestedfp_linear"}
 
