@@ -84,8 +84,10 @@ typedef enum {
     PGF8_PATH_SKINNY = 1,  /* weight-streaming: weights are the 128-row MMA operand,
                               tokens the narrow one (M <= 128) */
     PGF8_PATH_TILED = 2,   /* tokens are the 128-row MMA operand (any M) */
-    PGF8_PATH_STREAMK = 3  /* skinny, stream-K over one CTA per SM (M <= 32; needs the
+    PGF8_PATH_STREAMK = 3, /* skinny, stream-K over one CTA per SM (M <= 32; needs the
                               workspace) */
+    PGF8_PATH_TILED_PAIR = 4 /* tiled on SM pairs (cta_group::2), 256 x 256 tiles; FP8
+                              operand kinds only */
 } pgf8_path;
 
 /* Flags of pgf8_linear_opts.flags.

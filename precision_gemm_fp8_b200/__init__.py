@@ -31,7 +31,7 @@ NOALLOC_SCRATCH_BYTES = 8 << 20
 F32, F16, BF16 = 0, 1, 2
 SCALE_DYNAMIC, SCALE_STATIC = 0, 1
 NESTED_FP16, NESTED_FP8 = 0, 1
-PATH_AUTO, PATH_SKINNY, PATH_TILED, PATH_STREAMK = 0, 1, 2, 3
+PATH_AUTO, PATH_SKINNY, PATH_TILED, PATH_STREAMK, PATH_TILED_PAIR = 0, 1, 2, 3, 4
 FLAG_OVERLAP_PREVIOUS = 1
 
 

@@ -1,0 +1,361 @@
+// Persistent tcgen05 GEMM on CTA pairs (cta_group::2) for the tiled
+// orientation of the FP8 linear layer ("C++ and FP8" §3.3) and NestedFP FP8
+// mode ("NestedFP" §2.2): 256 x 256 output tiles, one tile per pair of SMs.
+//
+// The two CTAs of a cluster each load half of the tile's operands into their
+// own shared memory (rows m0 + 128*rank of the activations, rows n0 + 128*rank
+// of the weights); one thread of the even CTA issues tcgen05.mma.cta_group::2
+// (M = 256, N = 256), which reads both CTAs' shared memory and accumulates
+// rows m0.. into the even CTA's tensor memory and rows m0+128.. into the odd
+// CTA's.  Per CTA and k-block that is 32 KB of operands for a 128 x 256 slice
+// of the output, two thirds of what the one-CTA 128 x 256 tile moves, which
+// leaves room for a 6-deep ring.
+//
+// Synchronisation (all mbarriers; every wait bounded):
+//   full[s]      even CTA only: both CTAs' TMA loads complete on it (the
+//                cta_group::2 form of the load addresses the even CTA's
+//                barrier); the even producer posts the expected bytes of both.
+//   empty[s]     per CTA: the MMA's commit arrives on the even CTA's; the
+//                even producer, after seeing it, arrives on the odd CTA's.
+//   acc_full[b]  per CTA: the MMA's commit arrives on the even CTA's; an even
+//                epilogue thread, after seeing it, arrives on the odd CTA's.
+//   acc_empty[b] even CTA only: the 4 epilogue warps of both CTAs arrive.
+#pragma once
+
+#include "gemm.cuh"
+
+namespace pgf8 {
+
+template <int STAGES_, int KIND_> struct PairCfg {
+    static constexpr int BN = 256;                 // N of the pair's tile (MMA N)
+    static constexpr int STAGES = STAGES_;
+    static constexpr int KIND = KIND_;
+    static constexpr int kThreads = 192;
+    static constexpr int kTileA = 128 * 128;      // this CTA's 128 activation rows
+    static constexpr int kTileB = 128 * 128;      // this CTA's 128 weight rows
+    static constexpr int kStage = kTileA + kTileB;
+    static constexpr int kRowsX = 128;
+    static constexpr int kRowsW = 128;
+    static constexpr int kTmemCols = 2 * BN;      // two accumulator buffers
+    static constexpr int kRingBytes = STAGES * kStage;
+    static constexpr int kBarOffset = kRingBytes;
+    static constexpr int kSmemBytes = kRingBytes + 1024 + 1024;
+    static_assert(KIND == kE4M3 || KIND == kNested8, "FP8 operand kinds only");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+};
+
+struct PairCtl {
+    uint64_t full[16];
+    uint64_t empty[16];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void umma_f8f6f4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive (once) on `bar` of this CTA when every cta_group::2 tcgen05
+// operation issued so far by this thread has completed.
+__device__ __forceinline__ void umma_commit_pair(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+// TMA load into this CTA's shared memory whose completion is counted on the
+// even CTA's barrier at the same offset (cta_group::2 form).
+__device__ __forceinline__ void tma_load_2d_pair(void *smem_dst, const CUtensorMap *tm, uint64_t *bar, int x, int y,
+                                                 uint64_t policy)
+{
+    const uint32_t bar_even = smem_u32(bar) & 0xFEFFFFFFu;   // clear the pair-rank bit of the address
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar_even), "r"(x), "r"(y), "l"(policy)
+        : "memory");
+}
+
+// Plain arrive on the barrier at the same offset in CTA `rank` of the cluster.
+__device__ __forceinline__ void mbar_arrive_remote(uint64_t *bar, uint32_t rank)
+{
+    asm volatile(
+        "{\n\t.reg .b32 ra;\n\t"
+        "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
+        "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}\n" ::"r"(smem_u32(bar)),
+        "r"(rank)
+        : "memory");
+}
+
+// Bounded wait with cluster-scope acquire (for barriers arrived on from the
+// other CTA of the pair).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool wait_bounded_cluster(uint64_t *bar, uint32_t parity, volatile int *abort)
+{
+    if (mbar_try_wait_cluster(bar, parity))
+        return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t spin = 1;; ++spin) {
+        if (mbar_try_wait_cluster(bar, parity))
+            return true;
+        if ((spin & 63u) == 0) {
+            if (*abort)
+                return false;
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                *abort = 1;
+                atomicOr(&g_device_error, kErrTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                     const __grid_constant__ CUtensorMap tmW2, const GemmParams p)
+{
+    constexpr int BN = C::BN;
+    constexpr int STAGES = C::STAGES;
+    constexpr int KIND = C::KIND;
+    constexpr uint32_t kIdesc = make_idesc(256, BN, 0, KIND == kNested8 ? 1 : 0);
+    (void)tmW2;
+
+    grid_launch_dependents();
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    PairCtl *ctl = reinterpret_cast<PairCtl *>(smem + C::kBarOffset);
+    volatile int *abort_flag = &ctl->abort;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();           // 0: issues the MMA, 1: its partner
+    const bool lead = (rank == 0);
+    const int pair = static_cast<int>(blockIdx.x >> 1);
+    const int npairs = static_cast<int>(gridDim.x >> 1);
+    const int m_tiles = (p.M + 255) / 256;
+    const int n_tiles = (p.N + BN - 1) / BN;
+    const int total = m_tiles * n_tiles;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl->acc_full[b], 1);
+            mbar_init(&ctl->acc_empty[b], 8);   // 4 epilogue warps in each CTA
+        }
+        mbar_init(&ctl->drain, 1);
+        ctl->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmX);
+        tma_prefetch_desc(&tmW);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(&ctl->tmem_base, C::kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();                 // both CTAs' barriers exist before any remote arrive
+    tc_fence_after();
+    const uint32_t tmem = ctl->tmem_base;
+    grid_dependency_wait();
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producers (both CTAs)
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_last();
+            int s = 0;
+            uint32_t ph = 0;
+            uint32_t issued_mask = 0, issued_ph = 0;
+            bool ok = true;
+            int64_t it = 0;
+            for (int t = pair; ok && t < total; t += npairs) {
+                const int row_x = (t % m_tiles) * 256 + static_cast<int>(rank) * 128;
+                const int row_w = (t / m_tiles) * BN + static_cast<int>(rank) * 128;
+                for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
+                    if (!wait_bounded_cluster(&ctl->empty[s], ph ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    // the even CTA passes each real completion of its empty
+                    // barrier on to the odd CTA's
+                    if (lead && it >= STAGES)
+                        mbar_arrive_remote(&ctl->empty[s], 1u);
+                    uint8_t *st = smem + s * C::kStage;
+                    if (lead)
+                        mbar_arrive_expect_tx(&ctl->full[s], 2 * C::kStage);
+                    tma_load_2d_pair(st, &tmX, &ctl->full[s], kb * 128, row_x, pol);
+                    tma_load_2d_pair(st + C::kTileA, &tmW, &ctl->full[s], kb * 128, row_w, pol);
+                    issued_mask |= 1u << s;
+                    issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            if (*abort_flag && lead) {
+                for (int j = 0; j < STAGES; ++j)
+                    if (issued_mask & (1u << j))
+                        wait_drain(&ctl->full[j], (issued_ph >> j) & 1u);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (even CTA)
+        if (lead && lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            int i = 0;
+            for (int t = pair; ok && t < total; t += npairs, ++i) {
+                const int buf = i & 1;
+                const uint32_t use = static_cast<uint32_t>(i >> 1);
+                if (!wait_bounded_cluster(&ctl->acc_empty[buf], (use & 1u) ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d = tmem + static_cast<uint32_t>(buf * BN);
+                for (int kb = 0; kb < p.kblocks; ++kb) {
+                    if (!wait_bounded(&ctl->full[s], ph, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + s * C::kStage);
+                    const uint32_t b_addr = a_addr + C::kTileA;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t ad = sdesc_sw128(a_addr + k * 32);
+                        const uint64_t bd = sdesc_sw128(b_addr + k * 32);
+                        umma_f8f6f4_pair(d, ad, bd, kIdesc, (kb > 0 || k > 0) ? 1u : 0u);
+                    }
+                    umma_commit_pair(&ctl->empty[s]);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (ok)
+                    umma_commit_pair(&ctl->acc_full[buf]);
+            }
+            if (!ok) {
+                umma_commit_pair(&ctl->drain);
+                wait_drain(&ctl->drain, 0);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        const uint32_t t_row = tmem + (static_cast<uint32_t>(q * 32) << 16);
+        int i = 0;
+        for (int t = pair; t < total; t += npairs, ++i) {
+            const int buf = i & 1;
+            const uint32_t use = static_cast<uint32_t>(i >> 1);
+            bool ok = wait_bounded_cluster(&ctl->acc_full[buf], use & 1u, abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok)
+                break;
+            if (lead && warp == 2 && lane == 0)
+                mbar_arrive_remote(&ctl->acc_full[buf], 1u);   // pass the completion on to the odd CTA
+            tc_fence_after();
+            const int m = (t % m_tiles) * 256 + static_cast<int>(rank) * 128 + r;
+            const int n_base = (t / m_tiles) * BN;
+            float sam = (m < p.M) ? p.sa[m] : 0.0f;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+                const int n0 = n_base + c0;
+                if (n0 >= p.N)
+                    break;                      // warp-uniform; N % 16 == 0
+                uint32_t v[16];
+                tmem_ld_32x32b_x16(t_row + static_cast<uint32_t>(buf * BN + c0), v);
+                tmem_ld_wait();
+                if (m < p.M) {
+                    uint32_t o[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        float a0 = __uint_as_float(v[2 * j]) * sam, a1 = __uint_as_float(v[2 * j + 1]) * sam;
+                        if constexpr (KIND == kE4M3) {
+                            a0 = a0 * __ldg(p.sw + n0 + 2 * j);
+                            a1 = a1 * __ldg(p.sw + n0 + 2 * j + 1);
+                        }
+                        o[j] = pack2<KIND>(a0, a1);
+                    }
+                    uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.y) +
+                                                           static_cast<int64_t>(m) * p.N + n0);
+                    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+                    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (lead)
+                    mbar_arrive(&ctl->acc_empty[buf]);
+                else
+                    mbar_arrive_remote(&ctl->acc_empty[buf], 0u);
+            }
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();                 // no CTA leaves while its partner may still signal it
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, C::kTmemCols);
+    }
+}
+
+} // namespace pgf8

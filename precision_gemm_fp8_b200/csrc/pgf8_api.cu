@@ -11,6 +11,7 @@
 #include "gemm.cuh"
 #include "gemm_persistent.cuh"
 #include "gemm_streamk.cuh"
+#include "gemm_2sm.cuh"
 #include "quantize.cuh"
 
 // Pipeline depths and stream-K occupancy (compile-time tuning constants).
@@ -132,12 +133,13 @@ static GemmParams make_params(const GemmLaunch &L, int splits)
     return p;
 }
 
-static void fill_attrs(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attrs, int cluster_z, int pdl)
+static void fill_attrs(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attrs, int cluster_z, int pdl,
+                       int cluster_x = 1)
 {
     int na = 0;
-    if (cluster_z > 1) {
+    if (cluster_z > 1 || cluster_x > 1) {
         attrs[na].id = cudaLaunchAttributeClusterDimension;
-        attrs[na].val.clusterDim.x = 1;
+        attrs[na].val.clusterDim.x = static_cast<unsigned>(cluster_x);
         attrs[na].val.clusterDim.y = 1;
         attrs[na].val.clusterDim.z = static_cast<unsigned>(cluster_z);
         ++na;
@@ -211,6 +213,38 @@ template <class C> static pgf8_status launch_persistent(const GemmLaunch &L)
     cudaLaunchAttribute attrs[2];
     fill_attrs(cfg, attrs, 1, L.pdl);
     cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_persistent_kernel<C>, tmX, tmW, tmW2, p);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    return PGF8_OK;
+}
+
+// Pair kernel: clusters of 2 CTAs, one 256 x 256 tile per pair at a time.
+template <class C> static pgf8_status launch_pair(const GemmLaunch &L)
+{
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(gemm_pair_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        C::kSmemBytes);
+    });
+    if (attr_err != cudaSuccess)
+        return cuda_fail(attr_err);
+    CUtensorMap tmX, tmW, tmW2;
+    if (!make_operand_maps<C>(L, tmX, tmW, tmW2))
+        return PGF8_ERR_UNSUPPORTED;
+    const GemmParams p = make_params(L, 1);
+    const int64_t tiles = static_cast<int64_t>((L.M + 255) / 256) * ((L.N + 255) / 256);
+    const int pairs_max = num_sms() / 2;
+    const int64_t pairs = tiles < pairs_max ? tiles : pairs_max;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+    cfg.blockDim = dim3(C::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = L.stream;
+    cudaLaunchAttribute attrs[2];
+    fill_attrs(cfg, attrs, 1, L.pdl, 2);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<C>, tmX, tmW, tmW2, p);
     if (e != cudaSuccess)
         return cuda_fail(e);
     return PGF8_OK;
@@ -297,6 +331,12 @@ template <int KIND> static pgf8_status launch_gemm(const GemmLaunch &L)
         if (sk_bn == 16)
             return launch_streamk<StreamKCfg<16, PGF8_STREAMK16_STAGES, KIND>>(L);
         return launch_streamk<StreamKCfg<32, 5, KIND>>(L);
+    }
+    if (path == PGF8_PATH_TILED_PAIR) {
+        if (KIND == kNested16)
+            return PGF8_ERR_UNSUPPORTED;
+        if constexpr (KIND != kNested16)
+            return launch_pair<PairCfg<6, KIND>>(L);
     }
     if (path != PGF8_PATH_SKINNY && path != PGF8_PATH_TILED)
         return PGF8_ERR_INVALID_ARG;

@@ -38,9 +38,23 @@ def test_small_workload_full_check():
     """16 x 512 x 512: every output, both kernel families."""
     x, w = synthetic.case("small", 0, 0)
     aq, sa, wq, sw, ref, bound = _oracle_case(x, w)
-    for kw in ({}, {"path": pg.PATH_TILED}, {"path": pg.PATH_SKINNY, "split_k": 4}):
+    for kw in ({}, {"path": pg.PATH_TILED}, {"path": pg.PATH_SKINNY, "split_k": 4}, {"path": pg.PATH_TILED_PAIR}):
         y = _run_linear(aq, sa, wq, sw, **kw)
         assert_within(y, ref, bound, f"small {kw}")
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 256, 128), (512, 768, 1024), (300, 528, 400), (1000, 1040, 2000),
+                                   (2048, 4096, 4096)])
+def test_pair_kernel_against_oracle(M, N, K):
+    """256 x 256 tiles on SM pairs: several tiles per pair (persistent loop),
+    ragged M / N / K tails."""
+    g = np.random.default_rng(M + 7 * N + 13 * K)
+    x = synthetic.activations("student_t4_unit", M, K, g)
+    w = synthetic.weights_f16(N, K, 0.02, g)
+    aq, sa, wq, sw, ref, bound = _oracle_case(x, w)
+    for _ in range(2):
+        y = _run_linear(aq, sa, wq, sw, path=pg.PATH_TILED_PAIR)
+        assert_within(y, ref, bound, f"pair M{M} N{N} K{K}")
 
 
 RAGGED = [  # M, N, K: several tiles plus ragged tails in every dimension
@@ -56,7 +70,7 @@ def test_ragged_shapes_all_paths(M, N, K):
     w = synthetic.weights_f16(N, K, 0.02, g)
     aq, sa, wq, sw, ref, bound = _oracle_case(x, w)
     configs = [{"path": pg.PATH_TILED, "split_k": 1}, {"path": pg.PATH_TILED, "split_k": 3},
-               {"path": pg.PATH_TILED, "tile_n": 256}, {}]
+               {"path": pg.PATH_TILED, "tile_n": 256}, {"path": pg.PATH_TILED_PAIR}, {}]
     if M <= 128:
         configs += [{"path": pg.PATH_SKINNY, "split_k": 1}, {"path": pg.PATH_SKINNY, "split_k": 2},
                     {"path": pg.PATH_SKINNY, "split_k": 8}, {"path": pg.PATH_SKINNY, "tile_n": 128}]

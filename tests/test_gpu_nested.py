@@ -65,7 +65,7 @@ def test_nested_fp8_ragged(M, N, K):
     w16 = synthetic.weights_f16(N, K, 0.02, g)
     hi, _ = oracle.nestedfp_split(w16)
     ref, bound, _, _ = _ref8(x16, hi)
-    configs = [{"path": pg.PATH_TILED}, {"path": pg.PATH_TILED, "split_k": 2}]
+    configs = [{"path": pg.PATH_TILED}, {"path": pg.PATH_TILED, "split_k": 2}, {"path": pg.PATH_TILED_PAIR}]
     if M <= 128:
         configs += [{"path": pg.PATH_SKINNY}, {"path": pg.PATH_SKINNY, "split_k": 4}]
     for kw in configs:
