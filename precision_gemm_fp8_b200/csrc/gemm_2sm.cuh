@@ -15,10 +15,11 @@
 //   full[s]      even CTA only: both CTAs' TMA loads complete on it (the
 //                cta_group::2 form of the load addresses the even CTA's
 //                barrier); the even producer posts the expected bytes of both.
-//   empty[s]     per CTA: the MMA's commit arrives on the even CTA's; the
-//                even producer, after seeing it, arrives on the odd CTA's.
-//   acc_full[b]  per CTA: the MMA's commit arrives on the even CTA's; an even
-//                epilogue thread, after seeing it, arrives on the odd CTA's.
+//   empty[s]     per CTA: the MMA's commit arrives on the barrier at this
+//                offset in both CTAs at once (tcgen05.commit with a CTA mask;
+//                relaying it through a thread of the even CTA measured 2x
+//                slower).
+//   acc_full[b]  per CTA: the same two-CTA commit.
 //   acc_empty[b] even CTA only: the 4 epilogue warps of both CTAs arrive.
 #pragma once
 
@@ -101,6 +102,18 @@ __device__ __forceinline__ void tma_load_2d_pair(void *smem_dst, const CUtensorM
         "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
         " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(smem_dst)),
         "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar_even), "r"(x), "r"(y), "l"(policy)
+        : "memory");
+}
+
+// Arrive (once) on `bar` at the same offset in both CTAs of the pair when
+// every cta_group::2 tcgen05 operation issued so far by this thread has
+// completed.  (A completion signal sent to two CTAs' barriers; no data moves.)
+__device__ __forceinline__ void umma_commit_pair_both(uint64_t *bar)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(static_cast<uint16_t>(3))
         : "memory");
 }
 
@@ -214,19 +227,16 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             uint32_t ph = 0;
             uint32_t issued_mask = 0, issued_ph = 0;
             bool ok = true;
-            int64_t it = 0;
-            for (int t = pair; ok && t < total; t += npairs) {
+                    for (int t = pair; ok && t < total; t += npairs) {
                 const int row_x = (t % m_tiles) * 256 + static_cast<int>(rank) * 128;
                 const int row_w = (t / m_tiles) * BN + static_cast<int>(rank) * 128;
-                for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
+                for (int kb = 0; kb < p.kblocks; ++kb) {
                     if (!wait_bounded_cluster(&ctl->empty[s], ph ^ 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
                     // the even CTA passes each real completion of its empty
                     // barrier on to the odd CTA's
-                    if (lead && it >= STAGES)
-                        mbar_arrive_remote(&ctl->empty[s], 1u);
                     uint8_t *st = smem + s * C::kStage;
                     if (lead)
                         mbar_arrive_expect_tx(&ctl->full[s], 2 * C::kStage);
@@ -277,14 +287,14 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                         const uint64_t bd = sdesc_sw128(b_addr + k * 32);
                         umma_f8f6f4_pair(d, ad, bd, kIdesc, (kb > 0 || k > 0) ? 1u : 0u);
                     }
-                    umma_commit_pair(&ctl->empty[s]);
+                    umma_commit_pair_both(&ctl->empty[s]);
                     if (++s == STAGES) {
                         s = 0;
                         ph ^= 1u;
                     }
                 }
                 if (ok)
-                    umma_commit_pair(&ctl->acc_full[buf]);
+                    umma_commit_pair_both(&ctl->acc_full[buf]);
             }
             if (!ok) {
                 umma_commit_pair(&ctl->drain);
@@ -305,8 +315,6 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             ok = __all_sync(0xffffffffu, ok);
             if (!ok)
                 break;
-            if (lead && warp == 2 && lane == 0)
-                mbar_arrive_remote(&ctl->acc_full[buf], 1u);   // pass the completion on to the odd CTA
             tc_fence_after();
             const int m = (t % m_tiles) * 256 + static_cast<int>(rank) * 128 + r;
             const int n_base = (t / m_tiles) * BN;

@@ -234,15 +234,33 @@ template <class C> static pgf8_status launch_pair(const GemmLaunch &L)
         return PGF8_ERR_UNSUPPORTED;
     const GemmParams p = make_params(L, 1);
     const int64_t tiles = static_cast<int64_t>((L.M + 255) / 256) * ((L.N + 255) / 256);
-    const int pairs_max = num_sms() / 2;
-    const int64_t pairs = tiles < pairs_max ? tiles : pairs_max;
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
     cfg.blockDim = dim3(C::kThreads, 1, 1);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = L.stream;
     cudaLaunchAttribute attrs[2];
+    // A persistent grid must not hold more pairs than can run at once (a
+    // pair needs two SMs of one GPC): ask the occupancy calculator.
+    static int pairs_fit = 0;
+    if (pairs_fit == 0) {
+        cudaLaunchConfig_t q = cfg;
+        q.gridDim = dim3(2 * num_sms(), 1, 1);
+        cudaLaunchAttribute qa[1];
+        qa[0].id = cudaLaunchAttributeClusterDimension;
+        qa[0].val.clusterDim.x = 2;
+        qa[0].val.clusterDim.y = 1;
+        qa[0].val.clusterDim.z = 1;
+        q.attrs = qa;
+        q.numAttrs = 1;
+        int n = 0;
+        cudaError_t e = cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<C>, &q);
+        if (e != cudaSuccess)
+            return cuda_fail(e);
+        pairs_fit = n > 0 ? n : 1;
+    }
+    const int64_t pairs = tiles < pairs_fit ? tiles : pairs_fit;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
     fill_attrs(cfg, attrs, 1, L.pdl, 2);
     cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<C>, tmX, tmW, tmW2, p);
     if (e != cudaSuccess)
