@@ -392,6 +392,13 @@ template <int KIND> static pgf8_status launch_gemm(const GemmLaunch &L)
         default: return launch_split_or_not<KIND, true, 128, 6>(L, splits);
         }
     }
+    // FP8 operands with at least about one wave of 256 x 256 tiles (74 SM
+    // pairs): the pair kernel (measured faster there on every 7B / 70B shape)
+    if constexpr (KIND != kNested16) {
+        const int64_t tiles_pair = static_cast<int64_t>((L.M + 255) / 256) * ((L.N + 255) / 256);
+        if (L.opts.path == PGF8_PATH_AUTO && bn == 0 && splits == 0 && tiles_pair >= 80)
+            return launch_pair<PairCfg<6, KIND>>(L);
+    }
     const int mt = (L.M + 127) / 128;
     // fraction of the CTA slots the last wave of a persistent launch keeps busy
     auto wave_eff = [&](int b) {
