@@ -83,7 +83,7 @@ template <bool SWAP_, int BN_, int STAGES_, int KIND_, bool SPLIT_> struct GemmC
     static constexpr int kRingBytes = STAGES * kStage;
     static constexpr int kDataBytes = kRingBytes > kRedBytes ? kRingBytes : kRedBytes;
     static constexpr int kBarOffset = kDataBytes;
-    static constexpr int kSmemBytes = kDataBytes + 1024 /*barriers*/ + 1024 /*alignment slack*/;
+    static constexpr int kSmemBytes = kDataBytes + 1024 /*control block*/ + 1024 /*alignment slack*/;
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128 must be a multiple of 16 in [16,256]");
     static_assert((BN & (BN - 1)) == 0 || BN % 32 == 0, "BN");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
@@ -95,8 +95,11 @@ struct SharedCtl {
     uint64_t conv[16];
     uint64_t tmem_full;
     uint64_t drain;
+    uint64_t ring_free;     // split-K push: the cluster leader's ring may receive partials
+    uint64_t red_full;      // split-K push (leader): every other CTA's partial has arrived
     uint32_t tmem_base;
     int abort;
+    float sa_s[128];        // per-token scales of the tile's tokens, loaded at kernel start
 };
 
 // Bounded wait on an mbarrier phase.  Returns false (and raises the abort
@@ -188,6 +191,56 @@ template <int KIND> __device__ __forceinline__ uint32_t pack2(float a, float b)
     }
 }
 
+// Bounded wait with cluster-scope acquire (barriers arrived on from another
+// CTA of the cluster).
+__device__ __forceinline__ bool wait_bounded_acq_cluster(uint64_t *bar, uint32_t parity, volatile int *abort)
+{
+    auto try_once = [&]() {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        return ok != 0;
+    };
+    if (try_once())
+        return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t spin = 1;; ++spin) {
+        if (try_once())
+            return true;
+        if ((spin & 63u) == 0) {
+            if (*abort)
+                return false;
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                *abort = 1;
+                atomicOr(&g_device_error, kErrTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+// Arrive, with cluster-scope release, on the barrier at the same offset in
+// CTA `rank` of the cluster.
+__device__ __forceinline__ void mbar_arrive_cluster(uint64_t *bar, uint32_t rank)
+{
+    asm volatile(
+        "{\n\t.reg .b32 ra;\n\t"
+        "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
+        "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}\n" ::"r"(smem_u32(bar)),
+        "r"(rank)
+        : "memory");
+}
+
+__device__ __forceinline__ void st_shared_cluster_f32(uint32_t addr, float v)
+{
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
 template <class C>
 __global__ void __launch_bounds__(192, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
@@ -200,6 +253,11 @@ __global__ void __launch_bounds__(192, 1)
     constexpr bool NEST16 = (KIND == kNested16);
     constexpr uint32_t kIdesc =
         make_idesc(128, BN, /*A fmt*/ (SWAP && KIND == kNested8) ? 1 : 0, /*B fmt*/ (!SWAP && KIND == kNested8) ? 1 : 0);
+    constexpr int kXStep = NEST16 ? 64 : 128;   // K elements per stage
+    // split-K partials are pushed into the cluster leader's ring when the
+    // other CTAs' partial tiles fit there (skinny tiles), else reduced
+    // symmetrically through distributed shared memory
+    constexpr int kPartialBytes = BN * 128 * 4;
 
     // A dependent kernel launched with programmatic serialization (the next
     // layer) may be scheduled into free SM slots now; it reads nothing this
@@ -220,6 +278,59 @@ __global__ void __launch_bounds__(192, 1)
     const int kb1 = C::SPLIT ? ((split + 1) * p.kblocks) / p.splits : p.kblocks;
     const int row0_w = SWAP ? tile_a * 128 : tile_b * BN;   // first weight row of the tile
     const int row0_x = SWAP ? tile_b * BN : tile_a * 128;   // first token row of the tile
+    const bool push = SWAP && C::SPLIT && (p.splits - 1) * kPartialBytes <= C::kRingBytes;
+
+    // Producer state (thread 0): the first pass of the ring is issued before
+    // the CTA-wide synchronisation, so its loads overlap the set-up.
+    int ps = 0;
+    uint32_t pph = 0;
+    uint32_t issued_mask = 0, issued_ph = 0;   // per stage: loaded at least once / parity of last load
+    int pending = 0;                            // stages with weights but no activations yet
+    bool waited = false;
+    int pkb = kb0;
+    uint64_t pol_w = 0, pol_x = 0;
+
+    auto issue_w = [&](int kb, int st_idx) {
+        uint8_t *st = smem + st_idx * C::kStage;
+        uint8_t *w_tile = SWAP ? st : st + C::kTileA;
+        mbar_arrive_expect_tx(&ctl->full[st_idx], C::kStage);
+        if constexpr (NEST16) {
+            // hi and lo planes, 64 bytes (= 64 weights) of K each
+            tma_load_2d_hint(w_tile, &tmW, &ctl->full[st_idx], kb * 64, row0_w, pol_w);
+            tma_load_2d_hint(w_tile + C::kRowsW * 64, &tmW2, &ctl->full[st_idx], kb * 64, row0_w, pol_w);
+        } else {
+            tma_load_2d_hint(w_tile, &tmW, &ctl->full[st_idx], kb * 128, row0_w, pol_w);
+        }
+    };
+    auto issue_x = [&](int kb, int st_idx) {
+        uint8_t *st = smem + st_idx * C::kStage;
+        uint8_t *x_tile = SWAP ? st + C::kTileA : st;
+        tma_load_2d_hint(x_tile, &tmX, &ctl->full[st_idx], kb * kXStep, row0_x, pol_x);
+    };
+    // activations of the `pending` stages issued last (ending at k-block
+    // kb_end - 1, stage s_end - 1), once the grid dependency has resolved
+    auto flush_pending = [&](int kb_end, int s_end) {
+        grid_dependency_wait();
+        waited = true;
+        for (int j = 0; j < pending; ++j)
+            issue_x(kb_end - pending + j, (s_end - pending + j + STAGES) % STAGES);
+        pending = 0;
+    };
+    // one k-block into stage ps (its empty barrier already passed)
+    auto issue_stage = [&](int kb) {
+        issue_w(kb, ps);
+        issued_mask |= 1u << ps;
+        issued_ph = (issued_ph & ~(1u << ps)) | (pph << ps);
+        if (++ps == STAGES) {
+            ps = 0;
+            pph ^= 1u;
+        }
+        if (waited) {
+            issue_x(kb, (ps + STAGES - 1) % STAGES);
+        } else if (++pending == STAGES) {
+            flush_pending(kb + 1, ps);
+        }
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -229,78 +340,58 @@ __global__ void __launch_bounds__(192, 1)
         }
         mbar_init(&ctl->tmem_full, 1);
         mbar_init(&ctl->drain, 1);
+        mbar_init(&ctl->ring_free, 1);
+        mbar_init(&ctl->red_full, 128 * (p.splits > 1 ? p.splits - 1 : 1));
         ctl->abort = 0;
         fence_mbar_init();
-    }
-    if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmX);
         tma_prefetch_desc(&tmW);
         if (NEST16)
             tma_prefetch_desc(&tmW2);
+        // weights are streamed once in the skinny orientation (evict first);
+        // activation tiles are re-read by every CTA (evict last)
+        pol_w = SWAP ? policy_evict_first() : policy_evict_last();
+        pol_x = policy_evict_last();
+        if (!p.prefetch_w) {
+            grid_dependency_wait();
+            waited = true;
+        }
+        const int pre = (kb1 - kb0) < STAGES ? (kb1 - kb0) : STAGES;
+        for (int j = 0; j < pre; ++j)     // fresh ring: no empty-barrier waits
+            issue_stage(kb0 + j);
+        pkb = kb0 + pre;
     }
     if (warp == 1) {
         tmem_alloc(&ctl->tmem_base, C::kTmemCols);
         tmem_relinquish();
     }
+    if (warp >= 2) {
+        // scales of this tile's tokens, read once (after the dependency, as
+        // they may come from the previous kernel)
+        grid_dependency_wait();
+        const int et = static_cast<int>(threadIdx.x) - 64;
+        if constexpr (SWAP && KIND != kNested16) {
+            if (et < BN)
+                ctl->sa_s[et] = (row0_x + et < p.M) ? p.sa[row0_x + et] : 0.0f;
+        }
+    }
     tc_fence_before();
     __syncthreads();
+    if constexpr (C::SPLIT)
+        cluster_sync_all();      // every CTA's barriers exist before any remote arrive
     tc_fence_after();
     const uint32_t tmem = ctl->tmem_base;
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            // weights are streamed once in the skinny orientation (evict first);
-            // activation tiles are re-read by every CTA (evict last)
-            const uint64_t pol_w = SWAP ? policy_evict_first() : policy_evict_last();
-            const uint64_t pol_x = policy_evict_last();
-            constexpr int kXStep = NEST16 ? 64 : 128;   // K elements per stage
-            bool waited = false;
-            if (!p.prefetch_w) {
-                grid_dependency_wait();
-                waited = true;
-            }
-            int s = 0;
-            uint32_t ph = 0;
-            uint32_t issued_mask = 0, issued_ph = 0;   // per stage: loaded at least once / parity of last load
-            int pending = 0;                            // stages with weights but no activations yet
-            for (int kb = kb0; kb < kb1; ++kb) {
-                if (!wait_bounded(&ctl->empty[s], ph ^ 1u, abort_flag))
+            for (int kb = pkb; kb < kb1; ++kb) {
+                if (!wait_bounded(&ctl->empty[ps], pph ^ 1u, abort_flag))
                     break;
-                uint8_t *st = smem + s * C::kStage;
-                uint8_t *w_tile = SWAP ? st : st + C::kTileA;
-                mbar_arrive_expect_tx(&ctl->full[s], C::kStage);
-                if constexpr (NEST16) {
-                    // hi and lo planes, 64 bytes (= 64 weights) of K each
-                    tma_load_2d_hint(w_tile, &tmW, &ctl->full[s], kb * 64, row0_w, pol_w);
-                    tma_load_2d_hint(w_tile + C::kRowsW * 64, &tmW2, &ctl->full[s], kb * 64, row0_w, pol_w);
-                } else {
-                    tma_load_2d_hint(w_tile, &tmW, &ctl->full[s], kb * 128, row0_w, pol_w);
-                }
-                issued_mask |= 1u << s;
-                issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
-                if (waited) {
-                    uint8_t *x_tile = SWAP ? st + C::kTileA : st;
-                    tma_load_2d_hint(x_tile, &tmX, &ctl->full[s], kb * kXStep, row0_x, pol_x);
-                } else if (++pending == STAGES || kb + 1 == kb1) {
-                    // the first pass of weight tiles went out before the
-                    // dependency resolved; activations only after it
-                    grid_dependency_wait();
-                    waited = true;
-                    for (int j = 0; j < pending; ++j) {
-                        const int kbj = kb - pending + 1 + j;
-                        const int sj = (s - pending + 1 + j + STAGES) % STAGES;
-                        uint8_t *stj = smem + sj * C::kStage;
-                        uint8_t *x_tile = SWAP ? stj + C::kTileA : stj;
-                        tma_load_2d_hint(x_tile, &tmX, &ctl->full[sj], kbj * kXStep, row0_x, pol_x);
-                    }
-                    pending = 0;
-                }
-                if (++s == STAGES) {
-                    s = 0;
-                    ph ^= 1u;
-                }
+                issue_stage(kb);
             }
+            if (pending > 0)
+                flush_pending(kb1, ps);
             if (!waited)
                 grid_dependency_wait();
             if (*abort_flag) {
@@ -358,7 +449,6 @@ __global__ void __launch_bounds__(192, 1)
         }
         __syncwarp();
     } else {
-        grid_dependency_wait();
         // ------------------------------------------------------------ FP16 rebuild
         if constexpr (NEST16) {
             const int tt = static_cast<int>(threadIdx.x) - 64;   // 0..127
@@ -393,14 +483,31 @@ __global__ void __launch_bounds__(192, 1)
     const int r = q * 32 + lane;                // accumulator row (lane)
     const uint32_t t_row = tmem + (static_cast<uint32_t>(q * 32) << 16);
 
+    // skinny output of one accumulator row: channel n, tokens row0_x + j
+    auto store_skinny_row = [&](const float *a, int ncols) {
+        const int n = row0_w + r;
+        if (n >= p.N)
+            return;
+        float swn = 1.0f;
+        if constexpr (KIND == kE4M3)
+            swn = p.sw[n];
+        for (int j = 0; j < ncols; ++j) {
+            const int m = row0_x + j;
+            if (m < p.M) {
+                float v = a[j];
+                if constexpr (KIND != kNested16)
+                    v = v * ctl->sa_s[j];
+                if constexpr (KIND == kE4M3)
+                    v = v * swn;
+                store_out<KIND>(p.y, static_cast<int64_t>(m) * p.N + n, v);
+            }
+        }
+    };
+
     if constexpr (!C::SPLIT) {
         if (epi && have_acc) {
             if constexpr (SWAP) {
                 // lane = output channel n, column = token m
-                const int n = row0_w + r;
-                float swn = 1.0f;
-                if constexpr (KIND == kE4M3)
-                    swn = (n < p.N) ? p.sw[n] : 0.0f;
 #pragma unroll 1
                 for (int c0 = 0; c0 < BN; c0 += 16) {
                     if (row0_x + c0 >= p.M)
@@ -408,17 +515,25 @@ __global__ void __launch_bounds__(192, 1)
                     uint32_t v[16];
                     tmem_ld_32x32b_x16(t_row + c0, v);
                     tmem_ld_wait();
+                    float a[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        a[j] = __uint_as_float(v[j]);
+                    const int n = row0_w + r;
                     if (n < p.N) {
+                        float swn = 1.0f;
+                        if constexpr (KIND == kE4M3)
+                            swn = p.sw[n];
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const int m = row0_x + c0 + j;
                             if (m < p.M) {
-                                float a = __uint_as_float(v[j]);
+                                float x = a[j];
                                 if constexpr (KIND != kNested16)
-                                    a = a * p.sa[m];
+                                    x = x * ctl->sa_s[c0 + j];
                                 if constexpr (KIND == kE4M3)
-                                    a = a * swn;
-                                store_out<KIND>(p.y, static_cast<int64_t>(m) * p.N + n, a);
+                                    x = x * swn;
+                                store_out<KIND>(p.y, static_cast<int64_t>(m) * p.N + n, x);
                             }
                         }
                     }
@@ -460,8 +575,87 @@ __global__ void __launch_bounds__(192, 1)
                 }
             }
         }
+    } else if (push) {
+        // ------------------------------------------------------------ split-K, pushed to the leader
+        // The CTAs of rank 1.. write their f32 partial tile into the leader's
+        // (idle) ring, slot rank-1, column-major [BN][128], and arrive on its
+        // red_full barrier; the leader adds the slots in rank order to its own
+        // partial and writes the outputs.  Tokens of the tile: BN <= 32 here
+        // is not assumed; columns are processed 16 at a time.
+        const uint32_t rank = cluster_ctarank();
+        const int S = p.splits;
+        float *red = reinterpret_cast<float *>(smem);
+        if (rank == 0) {
+            // the ring is idle once this CTA's MMAs are done: let the others push
+            if (threadIdx.x == 0) {
+                // (have_acc of the epilogue warps implies the MMAs finished;
+                // thread 0 waits on the same barrier)
+                if (wait_bounded(&ctl->tmem_full, 0, abort_flag))
+                    for (int z = 1; z < S; ++z)
+                        mbar_arrive_cluster(&ctl->ring_free, static_cast<uint32_t>(z));
+            }
+            if (epi) {
+                const bool got = have_acc && wait_bounded_acq_cluster(&ctl->red_full, 0, abort_flag);
+#pragma unroll 1
+                for (int c0 = 0; c0 < BN; c0 += 16) {
+                    if (row0_x + c0 >= p.M)
+                        break;                  // warp-uniform
+                    uint32_t v[16];
+                    tmem_ld_32x32b_x16(t_row + c0, v);
+                    tmem_ld_wait();
+                    float a[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        a[j] = __uint_as_float(v[j]);
+                    if (got) {
+                        for (int z = 1; z < S; ++z) {
+                            const float *slot = red + static_cast<size_t>(z - 1) * (BN * 128);
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                a[j] += slot[(c0 + j) * 128 + r];
+                        }
+                    }
+                    const int n = row0_w + r;
+                    if (n < p.N) {
+                        float swn = 1.0f;
+                        if constexpr (KIND == kE4M3)
+                            swn = p.sw[n];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int m = row0_x + c0 + j;
+                            if (m < p.M) {
+                                float x = a[j];
+                                if constexpr (KIND != kNested16)
+                                    x = x * ctl->sa_s[c0 + j];
+                                if constexpr (KIND == kE4M3)
+                                    x = x * swn;
+                                store_out<KIND>(p.y, static_cast<int64_t>(m) * p.N + n, x);
+                            }
+                        }
+                    }
+                }
+            }
+        } else if (epi) {
+            const bool go = have_acc && wait_bounded_acq_cluster(&ctl->ring_free, 0, abort_flag);
+            const uint32_t slot = map_shared_rank(smem_u32(red + static_cast<size_t>(rank - 1) * (BN * 128)), 0u);
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+                if (row0_x + c0 >= p.M)
+                    break;                      // warp-uniform; the leader reads no further
+                uint32_t v[16];
+                tmem_ld_32x32b_x16(t_row + c0, v);
+                tmem_ld_wait();
+                if (go) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        st_shared_cluster_f32(slot + static_cast<uint32_t>(((c0 + j) * 128 + r) * 4),
+                                              __uint_as_float(v[j]));
+                }
+            }
+            mbar_arrive_cluster(&ctl->red_full, 0u);   // release: the stores above come first
+        }
     } else {
-        // ------------------------------------------------------------ split-K
+        // ------------------------------------------------------------ split-K, symmetric
         // 1. each CTA stores its partial tile into its own (now idle) ring
         float *red = reinterpret_cast<float *>(smem);
         if (epi) {
@@ -526,26 +720,15 @@ __global__ void __launch_bounds__(192, 1)
                     acc.w += t.w;
                 }
                 float a[4] = {acc.x, acc.y, acc.z, acc.w};
-                if constexpr (SWAP) {
-                    // 4 channels n..n+3 of token m
+                float sam = 1.0f;
+                if constexpr (KIND != kNested16)
+                    sam = p.sa[m];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        if constexpr (KIND != kNested16)
-                            a[j] = a[j] * p.sa[m];
-                        if constexpr (KIND == kE4M3)
-                            a[j] = a[j] * __ldg(p.sw + n + j);
-                    }
-                } else {
-                    float sam = 1.0f;
+                for (int j = 0; j < 4; ++j) {
                     if constexpr (KIND != kNested16)
-                        sam = p.sa[m];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        if constexpr (KIND != kNested16)
-                            a[j] = a[j] * sam;
-                        if constexpr (KIND == kE4M3)
-                            a[j] = a[j] * __ldg(p.sw + n + j);
-                    }
+                        a[j] = a[j] * sam;
+                    if constexpr (KIND == kE4M3)
+                        a[j] = a[j] * __ldg(p.sw + n + j);
                 }
                 uint2 o;
                 o.x = pack2<KIND>(a[0], a[1]);
@@ -556,6 +739,7 @@ __global__ void __launch_bounds__(192, 1)
         __syncwarp();
         cluster_sync_all();   // no CTA leaves while its partial may still be read
     }
+    (void)store_skinny_row;
 
     // ---------------------------------------------------------------- teardown
     __syncwarp();
