@@ -341,7 +341,7 @@ __global__ void __launch_bounds__(192, 1)
         mbar_init(&ctl->tmem_full, 1);
         mbar_init(&ctl->drain, 1);
         mbar_init(&ctl->ring_free, 1);
-        mbar_init(&ctl->red_full, 128 * (p.splits > 1 ? p.splits - 1 : 1));
+        mbar_init(&ctl->red_full, p.splits > 1 ? p.splits - 1 : 1);   // one arrival per pushing CTA
         ctl->abort = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmX);
@@ -652,7 +652,12 @@ __global__ void __launch_bounds__(192, 1)
                                               __uint_as_float(v[j]));
                 }
             }
-            mbar_arrive_cluster(&ctl->red_full, 0u);   // release: the stores above come first
+            // each thread's remote stores are ordered before the barrier; one
+            // release-arrive per CTA then publishes all of them to the leader
+            asm volatile("fence.acq_rel.cluster;" ::: "memory");
+            asm volatile("bar.sync 2, 128;" ::: "memory");
+            if (et == 0)
+                mbar_arrive_cluster(&ctl->red_full, 0u);
         }
     } else {
         // ------------------------------------------------------------ split-K, symmetric
