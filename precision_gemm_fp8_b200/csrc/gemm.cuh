@@ -95,8 +95,6 @@ struct SharedCtl {
     uint64_t conv[16];
     uint64_t tmem_full;
     uint64_t drain;
-    uint64_t ring_free;     // split-K push: the cluster leader's ring may receive partials
-    uint64_t red_full;      // split-K push (leader): every other CTA's partial has arrived
     uint32_t tmem_base;
     int abort;
     float sa_s[128];        // per-token scales of the tile's tokens, loaded at kernel start
@@ -191,56 +189,6 @@ template <int KIND> __device__ __forceinline__ uint32_t pack2(float a, float b)
     }
 }
 
-// Bounded wait with cluster-scope acquire (barriers arrived on from another
-// CTA of the cluster).
-__device__ __forceinline__ bool wait_bounded_acq_cluster(uint64_t *bar, uint32_t parity, volatile int *abort)
-{
-    auto try_once = [&]() {
-        uint32_t ok;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}\n"
-            : "=r"(ok)
-            : "r"(smem_u32(bar)), "r"(parity)
-            : "memory");
-        return ok != 0;
-    };
-    if (try_once())
-        return true;
-    const uint64_t t0 = global_timer_ns();
-    for (uint32_t spin = 1;; ++spin) {
-        if (try_once())
-            return true;
-        if ((spin & 63u) == 0) {
-            if (*abort)
-                return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs) {
-                *abort = 1;
-                atomicOr(&g_device_error, kErrTimeout);
-                return false;
-            }
-        }
-    }
-}
-
-// Arrive, with cluster-scope release, on the barrier at the same offset in
-// CTA `rank` of the cluster.
-__device__ __forceinline__ void mbar_arrive_cluster(uint64_t *bar, uint32_t rank)
-{
-    asm volatile(
-        "{\n\t.reg .b32 ra;\n\t"
-        "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
-        "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}\n" ::"r"(smem_u32(bar)),
-        "r"(rank)
-        : "memory");
-}
-
-__device__ __forceinline__ void st_shared_cluster_f32(uint32_t addr, float v)
-{
-    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-
 template <class C>
 __global__ void __launch_bounds__(192, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
@@ -254,10 +202,6 @@ __global__ void __launch_bounds__(192, 1)
     constexpr uint32_t kIdesc =
         make_idesc(128, BN, /*A fmt*/ (SWAP && KIND == kNested8) ? 1 : 0, /*B fmt*/ (!SWAP && KIND == kNested8) ? 1 : 0);
     constexpr int kXStep = NEST16 ? 64 : 128;   // K elements per stage
-    // split-K partials are pushed into the cluster leader's ring when the
-    // other CTAs' partial tiles fit there (skinny tiles), else reduced
-    // symmetrically through distributed shared memory
-    constexpr int kPartialBytes = BN * 128 * 4;
 
     // A dependent kernel launched with programmatic serialization (the next
     // layer) may be scheduled into free SM slots now; it reads nothing this
@@ -278,7 +222,6 @@ __global__ void __launch_bounds__(192, 1)
     const int kb1 = C::SPLIT ? ((split + 1) * p.kblocks) / p.splits : p.kblocks;
     const int row0_w = SWAP ? tile_a * 128 : tile_b * BN;   // first weight row of the tile
     const int row0_x = SWAP ? tile_b * BN : tile_a * 128;   // first token row of the tile
-    const bool push = SWAP && C::SPLIT && (p.splits - 1) * kPartialBytes <= C::kRingBytes;
 
     // Producer state (thread 0): the first pass of the ring is issued before
     // the CTA-wide synchronisation, so its loads overlap the set-up.
@@ -340,8 +283,6 @@ __global__ void __launch_bounds__(192, 1)
         }
         mbar_init(&ctl->tmem_full, 1);
         mbar_init(&ctl->drain, 1);
-        mbar_init(&ctl->ring_free, 1);
-        mbar_init(&ctl->red_full, p.splits > 1 ? p.splits - 1 : 1);   // one arrival per pushing CTA
         ctl->abort = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmX);
@@ -377,8 +318,6 @@ __global__ void __launch_bounds__(192, 1)
     }
     tc_fence_before();
     __syncthreads();
-    if constexpr (C::SPLIT)
-        cluster_sync_all();      // every CTA's barriers exist before any remote arrive
     tc_fence_after();
     const uint32_t tmem = ctl->tmem_base;
 
@@ -575,90 +514,6 @@ __global__ void __launch_bounds__(192, 1)
                 }
             }
         }
-    } else if (push) {
-        // ------------------------------------------------------------ split-K, pushed to the leader
-        // The CTAs of rank 1.. write their f32 partial tile into the leader's
-        // (idle) ring, slot rank-1, column-major [BN][128], and arrive on its
-        // red_full barrier; the leader adds the slots in rank order to its own
-        // partial and writes the outputs.  Tokens of the tile: BN <= 32 here
-        // is not assumed; columns are processed 16 at a time.
-        const uint32_t rank = cluster_ctarank();
-        const int S = p.splits;
-        float *red = reinterpret_cast<float *>(smem);
-        if (rank == 0) {
-            // the ring is idle once this CTA's MMAs are done: let the others push
-            if (threadIdx.x == 0) {
-                // (have_acc of the epilogue warps implies the MMAs finished;
-                // thread 0 waits on the same barrier)
-                if (wait_bounded(&ctl->tmem_full, 0, abort_flag))
-                    for (int z = 1; z < S; ++z)
-                        mbar_arrive_cluster(&ctl->ring_free, static_cast<uint32_t>(z));
-            }
-            if (epi) {
-                const bool got = have_acc && wait_bounded_acq_cluster(&ctl->red_full, 0, abort_flag);
-#pragma unroll 1
-                for (int c0 = 0; c0 < BN; c0 += 16) {
-                    if (row0_x + c0 >= p.M)
-                        break;                  // warp-uniform
-                    uint32_t v[16];
-                    tmem_ld_32x32b_x16(t_row + c0, v);
-                    tmem_ld_wait();
-                    float a[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        a[j] = __uint_as_float(v[j]);
-                    if (got) {
-                        for (int z = 1; z < S; ++z) {
-                            const float *slot = red + static_cast<size_t>(z - 1) * (BN * 128);
-#pragma unroll
-                            for (int j = 0; j < 16; ++j)
-                                a[j] += slot[(c0 + j) * 128 + r];
-                        }
-                    }
-                    const int n = row0_w + r;
-                    if (n < p.N) {
-                        float swn = 1.0f;
-                        if constexpr (KIND == kE4M3)
-                            swn = p.sw[n];
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int m = row0_x + c0 + j;
-                            if (m < p.M) {
-                                float x = a[j];
-                                if constexpr (KIND != kNested16)
-                                    x = x * ctl->sa_s[c0 + j];
-                                if constexpr (KIND == kE4M3)
-                                    x = x * swn;
-                                store_out<KIND>(p.y, static_cast<int64_t>(m) * p.N + n, x);
-                            }
-                        }
-                    }
-                }
-            }
-        } else if (epi) {
-            const bool go = have_acc && wait_bounded_acq_cluster(&ctl->ring_free, 0, abort_flag);
-            const uint32_t slot = map_shared_rank(smem_u32(red + static_cast<size_t>(rank - 1) * (BN * 128)), 0u);
-#pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 16) {
-                if (row0_x + c0 >= p.M)
-                    break;                      // warp-uniform; the leader reads no further
-                uint32_t v[16];
-                tmem_ld_32x32b_x16(t_row + c0, v);
-                tmem_ld_wait();
-                if (go) {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        st_shared_cluster_f32(slot + static_cast<uint32_t>(((c0 + j) * 128 + r) * 4),
-                                              __uint_as_float(v[j]));
-                }
-            }
-            // each thread's remote stores are ordered before the barrier; one
-            // release-arrive per CTA then publishes all of them to the leader
-            asm volatile("fence.acq_rel.cluster;" ::: "memory");
-            asm volatile("bar.sync 2, 128;" ::: "memory");
-            if (et == 0)
-                mbar_arrive_cluster(&ctl->red_full, 0u);
-        }
     } else {
         // ------------------------------------------------------------ split-K, symmetric
         // 1. each CTA stores its partial tile into its own (now idle) ring
@@ -716,13 +571,22 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 if (m >= p.M || n >= p.N)
                     continue;
+                // all partials are requested before any is added (the remote
+                // loads overlap); the sum runs in rank order
+                float4 t[8];
+#pragma unroll
+                for (int z = 0; z < 8; ++z)
+                    if (z < S)
+                        t[z] = ld_shared_cluster_v4_relaxed(map_shared_rank(red_addr + off, static_cast<uint32_t>(z)));
                 float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int z = 0; z < S; ++z) {
-                    const float4 t = ld_shared_cluster_v4(map_shared_rank(red_addr + off, static_cast<uint32_t>(z)));
-                    acc.x += t.x;
-                    acc.y += t.y;
-                    acc.z += t.z;
-                    acc.w += t.w;
+#pragma unroll
+                for (int z = 0; z < 8; ++z) {
+                    if (z < S) {
+                        acc.x += t[z].x;
+                        acc.y += t[z].y;
+                        acc.z += t[z].z;
+                        acc.w += t[z].w;
+                    }
                 }
                 float a[4] = {acc.x, acc.y, acc.z, acc.w};
                 float sam = 1.0f;

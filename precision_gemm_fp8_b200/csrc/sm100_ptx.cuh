@@ -240,6 +240,17 @@ __device__ __forceinline__ uint32_t map_shared_rank(uint32_t saddr, uint32_t ran
     return r;
 }
 
+// Same load without a compiler memory barrier, so that several of them can
+// be in flight at once; callers order them with the cluster barrier.
+__device__ __forceinline__ float4 ld_shared_cluster_v4_relaxed(uint32_t addr)
+{
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
 __device__ __forceinline__ float4 ld_shared_cluster_v4(uint32_t addr)
 {
     float4 v;
