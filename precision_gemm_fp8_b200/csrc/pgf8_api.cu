@@ -375,12 +375,12 @@ template <int KIND> static pgf8_status launch_gemm(const GemmLaunch &L)
     if (path == PGF8_PATH_SKINNY) {
         const int tiles = (L.N + 127) / 128;
         if (splits == 0) {
-            // double the split while the grid stays within ~1.3 CTAs per SM
-            // (two CTAs fit on an SM at the narrow tile sizes): more CTAs
-            // than that only add partial-tile exchanges and cluster packing
-            // constraints without adding bytes in flight
+            // the largest power-of-two split that keeps the grid within ~1.75
+            // CTAs per SM (measured on B200 over the 7B and 70B decode
+            // shapes: 64 weight tiles -> 4, 80-96 -> 2, >= 172 -> 1); beyond
+            // that the extra CTAs wait for a second wave
             splits = 1;
-            while (splits < 8 && tiles * splits * 2 * 10 <= sms * 13)
+            while (splits < 8 && tiles * splits * 2 * 4 <= sms * 7)
                 splits *= 2;
         }
         if (splits > kblocks)
