@@ -27,17 +27,20 @@
 
 namespace pgf8 {
 
-template <int STAGES_, int KIND_> struct PairCfg {
-    static constexpr int BN = 256;                 // N of the pair's tile (MMA N)
+template <int BN_, int STAGES_, int KIND_> struct PairCfg {
+    static constexpr int BN = BN_;                 // N of the pair's tile (MMA N)
     static constexpr int STAGES = STAGES_;
     static constexpr int KIND = KIND_;
     static constexpr int kThreads = 192;
     static constexpr int kTileA = 128 * 128;      // this CTA's 128 activation rows
-    static constexpr int kTileB = 128 * 128;      // this CTA's 128 weight rows
+    static constexpr int kTileB = (BN / 2) * 128; // this CTA's BN/2 weight rows
     static constexpr int kStage = kTileA + kTileB;
     static constexpr int kRowsX = 128;
-    static constexpr int kRowsW = 128;
-    static constexpr int kTmemCols = 2 * BN;      // two accumulator buffers
+    static constexpr int kRowsW = BN / 2;
+    // two accumulator buffers of BN columns, allocated as a power of two
+    static constexpr int kTmemCols = (2 * BN <= 256) ? 256 : 512;
+    static_assert(BN == 128 || BN == 192 || BN == 256, "pair tile width");
+    static_assert((kStage % 1024) == 0, "stage alignment");
     static constexpr int kRingBytes = STAGES * kStage;
     static constexpr int kBarOffset = kRingBytes;
     static constexpr int kSmemBytes = kRingBytes + 1024 + 1024;
@@ -229,7 +232,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             bool ok = true;
                     for (int t = pair; ok && t < total; t += npairs) {
                 const int row_x = (t % m_tiles) * 256 + static_cast<int>(rank) * 128;
-                const int row_w = (t / m_tiles) * BN + static_cast<int>(rank) * 128;
+                const int row_w = (t / m_tiles) * BN + static_cast<int>(rank) * (BN / 2);
                 for (int kb = 0; kb < p.kblocks; ++kb) {
                     if (!wait_bounded_cluster(&ctl->empty[s], ph ^ 1u, abort_flag)) {
                         ok = false;

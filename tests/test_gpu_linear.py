@@ -59,9 +59,10 @@ def test_pair_kernel_against_oracle(M, N, K):
     ns = np.arange(N) if M * N * K <= 2e9 else np.sort(rng.choice(N, 256, replace=False))
     ref = oracle.fp8_linear(aq[ms], sa[ms], wq[ns], sw[ns])
     bound = linear_bound(ref, K, fp8_row_max(aq[ms], sa[ms]), fp8_row_max(wq[ns], sw[ns]))
-    for _ in range(2):
-        y = _run_linear(aq, sa, wq, sw, path=pg.PATH_TILED_PAIR)
-        assert_within(y[np.ix_(ms, ns)], ref, bound, f"pair M{M} N{N} K{K}")
+    for tile_n in (0, 128, 192, 256):
+        for _ in range(2):
+            y = _run_linear(aq, sa, wq, sw, path=pg.PATH_TILED_PAIR, tile_n=tile_n)
+            assert_within(y[np.ix_(ms, ns)], ref, bound, f"pair{tile_n} M{M} N{N} K{K}")
 
 
 RAGGED = [  # M, N, K: several tiles plus ragged tails in every dimension
