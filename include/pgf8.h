@@ -170,6 +170,34 @@ pgf8_status pgf8_fp8_linear_dynamic(const void *x, pgf8_dtype xdt, int64_t M, in
 
 size_t pgf8_fp8_linear_dynamic_workspace_size(int64_t M, int64_t N, int64_t K);
 size_t pgf8_fp8_linear_dynamic_codes_offset(int64_t M, int64_t K);
+
+/* One layer of pgf8_fp8_linear_dynamic_many: the arguments of
+ * pgf8_fp8_linear_dynamic. */
+typedef struct {
+    const void *x;           /* [M, K] f32 or f16, row stride ldx */
+    int32_t xdt;             /* pgf8_dtype */
+    int32_t reserved;
+    int64_t M, K, ldx, N;
+    const uint8_t *wq;       /* [N, K] E4M3 codes */
+    const float *sw;         /* [N] */
+    void *y;                 /* [M, N] bf16 */
+    void *workspace;         /* pgf8_fp8_linear_dynamic_workspace_size(M, N, K) bytes */
+    size_t workspace_bytes;
+} pgf8_fp8_layer;
+
+/* ------------------------------------------------------------------------
+ * A sequence of dynamic FP8 linear layers enqueued by one call, in order, on
+ * `stream` (a decoder step's linears, say).  Every layer is checked before
+ * anything is enqueued; the first invalid one makes the call return its
+ * status and enqueue nothing.  Layer i+1 is launched with
+ * PGF8_FLAG_OVERLAP_PREVIOUS (it may start loading its weights while layer i
+ * finishes), so no layer's weights may alias another layer's x, y or
+ * workspace; the first layer uses the flags given in opts.  Each layer may
+ * read the previous layer's y as its x (the overlap never moves an
+ * activation read ahead of the kernel that writes it).
+ * ---------------------------------------------------------------------- */
+pgf8_status pgf8_fp8_linear_dynamic_many(const pgf8_fp8_layer *layers, int64_t count,
+                                         const pgf8_linear_opts *opts, void *stream);
 size_t pgf8_fp8_linear_dynamic_scales_offset(int64_t M, int64_t K);
 
 /* ------------------------------------------------------------------------
@@ -246,11 +274,18 @@ pgf8_status pgf8_fp8_linear_dynamic_noalloc(const void *x, pgf8_dtype xdt, int64
  *   device error word of the current device: PGF8_ERR_TIMEOUT if a kernel
  *   gave up a bounded wait since the last check, PGF8_ERR_CUDA if the
  *   synchronisation itself failed, else PGF8_OK.
+ * pgf8_selftest_bounded_wait: enqueues a one-thread kernel that waits on a
+ *   barrier phase nothing ever completes, with a bound of limit_ns
+ *   (1e3..2e9) instead of the library's 1 s.  The wait gives up, raises the
+ *   device error word and the kernel returns: the next pgf8_device_status()
+ *   on that stream reports PGF8_ERR_TIMEOUT and clears it.  For checking the
+ *   failure path without hanging or faulting the GPU.
  * pgf8_status_str: static description of a status code.
  * pgf8_version: library version as major*10000 + minor*100 + patch.
  * ---------------------------------------------------------------------- */
 pgf8_status pgf8_last_cuda_error(int *cuda_err);
 pgf8_status pgf8_device_status(void *stream);
+pgf8_status pgf8_selftest_bounded_wait(int64_t limit_ns, void *stream);
 const char *pgf8_status_str(pgf8_status status);
 int pgf8_version(void);
 

@@ -40,6 +40,13 @@ class LinearOpts(ctypes.Structure):
                 ("flags", ctypes.c_int32)]
 
 
+class Fp8Layer(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("xdt", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("M", ctypes.c_int64), ("K", ctypes.c_int64), ("ldx", ctypes.c_int64), ("N", ctypes.c_int64),
+                ("wq", ctypes.c_void_p), ("sw", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+
+
 _vp = ctypes.c_void_p
 _i64 = ctypes.c_int64
 _sz = ctypes.c_size_t
@@ -54,6 +61,7 @@ _SIGS = {
     "pgf8_fp8_linear_dynamic": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _sz, _optp, _vp], _i32),
     "pgf8_fp8_linear_dynamic_workspace_size": ([_i64, _i64, _i64], _sz),
     "pgf8_fp8_linear_dynamic_codes_offset": ([_i64, _i64], _sz),
+    "pgf8_fp8_linear_dynamic_many": ([ctypes.POINTER(Fp8Layer), _i64, _optp, _vp], _i32),
     "pgf8_fp8_linear_dynamic_scales_offset": ([_i64, _i64], _sz),
     "pgf8_nestedfp_split": ([_vp, _i64, _i64, _vp, _vp, _vp], _i32),
     "pgf8_nestedfp_linear": ([_vp, _i64, _i64, _vp, _vp, _i64, _i32, _vp, _vp, _sz, _vp], _i32),
@@ -62,6 +70,7 @@ _SIGS = {
     "pgf8_fp8_linear_dynamic_noalloc": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _i64, _vp, _vp], _i32),
     "pgf8_last_cuda_error": ([ctypes.POINTER(ctypes.c_int)], _i32),
     "pgf8_device_status": ([_vp], _i32),
+    "pgf8_selftest_bounded_wait": ([_i64, _vp], _i32),
     "pgf8_status_str": ([_i32], ctypes.c_char_p),
     "pgf8_version": ([], _i32),
 }
@@ -222,6 +231,27 @@ def fp8_linear_dynamic_noalloc(x, wq, sw, y=None, stream=None):
     _check(lib.pgf8_fp8_linear_dynamic_noalloc(_ptr(x), _dtype_code(x), M, K, x.stride(0), _ptr(wq), _ptr(sw), N,
                                                _ptr(y), _stream(stream)), "fp8_linear_dynamic_noalloc")
     return y
+
+
+class LayerSequence:
+    """A fixed sequence of dynamic FP8 layers (device tensors bound once), run
+    by one call of pgf8_fp8_linear_dynamic_many.  Each entry is a tuple
+    (x, wq, sw, y, workspace); workspaces must be zero-filled before first use."""
+
+    def __init__(self, layers):
+        self._keep = list(layers)
+        arr = (Fp8Layer * len(self._keep))()
+        for i, (x, wq, sw, y, ws) in enumerate(self._keep):
+            if x.stride(1) != 1:
+                raise ValueError("x rows must be contiguous")
+            arr[i] = Fp8Layer(x.data_ptr(), _dtype_code(x), 0, x.shape[0], x.shape[1], x.stride(0), wq.shape[0],
+                              wq.data_ptr(), sw.data_ptr(), y.data_ptr(), ws.data_ptr(), _nbytes(ws))
+        self._arr = arr
+        self.count = len(self._keep)
+
+    def run(self, flags=0, stream=None):
+        _check(lib.pgf8_fp8_linear_dynamic_many(self._arr, self.count, _opts(flags=flags), _stream(stream)),
+               "fp8_linear_dynamic_many")
 
 
 def dynamic_workspace_views(workspace: torch.Tensor, M: int, K: int):

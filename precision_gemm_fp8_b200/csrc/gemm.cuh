@@ -101,9 +101,10 @@ struct SharedCtl {
 };
 
 // Bounded wait on an mbarrier phase.  Returns false (and raises the abort
-// flag and the device error word) after kWaitLimitNs, or when another role
-// of the CTA has already raised the abort flag.
-__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort)
+// flag and the device error word) after limit_ns, or when another role of
+// the CTA has already raised the abort flag.
+__device__ __forceinline__ bool wait_bounded_for(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                                 uint64_t limit_ns)
 {
     if (mbar_try_wait(bar, parity))
         return true;
@@ -114,13 +115,35 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, vol
         if ((spin & 63u) == 0) {
             if (*abort)
                 return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs) {
+            if (global_timer_ns() - t0 > limit_ns) {
                 *abort = 1;
                 atomicOr(&g_device_error, kErrTimeout);
                 return false;
             }
         }
     }
+}
+
+__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort)
+{
+    return wait_bounded_for(bar, parity, abort, kWaitLimitNs);
+}
+
+// Self-test of the bounded wait: one thread waits on a barrier phase that
+// nothing ever completes; the wait gives up after limit_ns, raises the
+// device error word, and the kernel returns normally.
+__global__ void selftest_bounded_wait_kernel(uint64_t limit_ns)
+{
+    __shared__ uint64_t bar;
+    __shared__ int abort;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0)
+        (void)wait_bounded_for(&bar, 0, &abort, limit_ns);
 }
 
 // Wait used only while draining after an abort: bounded, never raises.

@@ -268,31 +268,6 @@ template <class C> static pgf8_status launch_pair(const GemmLaunch &L)
     return PGF8_OK;
 }
 
-// Pair tile width: the one whose last round of tiles keeps the most SM
-// pairs busy, a narrower tile counting 4 % (192) or 10 % (128) less
-// efficient per tile (more operand bytes per flop).
-static int pair_tile_width(int M, int N)
-{
-    const int pairs = num_sms() / 2;
-    const int mt = (M + 255) / 256;
-    int best = 256;
-    double best_score = 0.0;
-    const int widths[3] = {256, 192, 128};
-    const double per_tile[3] = {1.0, 0.96, 0.90};
-    for (int i = 0; i < 3; ++i) {
-        const int64_t t = static_cast<int64_t>(mt) * ((N + widths[i] - 1) / widths[i]);
-        const int64_t rounds = (t + pairs - 1) / pairs;
-        const double useful = static_cast<double>(M) * N;   // same for every width
-        const double covered = static_cast<double>(rounds) * pairs * 256.0 * widths[i];
-        const double score = per_tile[i] * useful / covered;
-        if (score > best_score + 1e-9) {
-            best_score = score;
-            best = widths[i];
-        }
-    }
-    return best;
-}
-
 template <int KIND> static pgf8_status launch_pair_bn(const GemmLaunch &L, int bn)
 {
     if constexpr (KIND == kNested16) {
@@ -394,7 +369,7 @@ template <int KIND> static pgf8_status launch_gemm(const GemmLaunch &L)
         if (bn != 0 && bn != 128 && bn != 192 && bn != 256)
             return PGF8_ERR_INVALID_ARG;
         if constexpr (KIND != kNested16)
-            return launch_pair_bn<KIND>(L, bn == 0 ? pair_tile_width(L.M, L.N) : bn);
+            return launch_pair_bn<KIND>(L, bn == 0 ? 256 : bn);
     }
     if (path != PGF8_PATH_SKINNY && path != PGF8_PATH_TILED)
         return PGF8_ERR_INVALID_ARG;
@@ -436,8 +411,11 @@ template <int KIND> static pgf8_status launch_gemm(const GemmLaunch &L)
     // pairs): the pair kernel (measured faster there on every 7B / 70B shape)
     if constexpr (KIND != kNested16) {
         const int64_t tiles_pair = static_cast<int64_t>((L.M + 255) / 256) * ((L.N + 255) / 256);
+        // (the 192 / 128 widths fill the last round better but measured slower
+        // per tile than 256 on nearly every 7B / 70B shape; they stay
+        // selectable through tile_n)
         if (L.opts.path == PGF8_PATH_AUTO && bn == 0 && splits == 0 && tiles_pair >= 80)
-            return launch_pair_bn<KIND>(L, pair_tile_width(L.M, L.N));
+            return launch_pair_bn<KIND>(L, 256);
     }
     const int mt = (L.M + 127) / 128;
     // fraction of the CTA slots the last wave of a persistent launch keeps busy
@@ -621,10 +599,10 @@ size_t pgf8_fp8_linear_dynamic_workspace_size(int64_t M, int64_t, int64_t K)
     return pgf8_fp8_linear_dynamic_scales_offset(M, K) + round_up(static_cast<size_t>(M) * 4, 256);
 }
 
-static pgf8_status linear_dynamic_impl(const void *x, pgf8_dtype xdt, int64_t M, int64_t K, int64_t ldx,
-                                       const void *w, const void *w2, const float *sw, int64_t N, void *y,
-                                       void *workspace, size_t workspace_bytes, const pgf8_linear_opts *opts,
-                                       void *stream, int kind)
+// Argument checks of a dynamic linear call (nothing is enqueued).
+static pgf8_status check_linear_dynamic(const void *x, pgf8_dtype xdt, int64_t M, int64_t K, int64_t ldx,
+                                       const void *w, const float *sw, int64_t N, void *y, void *workspace,
+                                       size_t workspace_bytes, int kind)
 {
     pgf8_status st = check_dims(M, N, K);
     if (st != PGF8_OK)
@@ -638,9 +616,20 @@ static pgf8_status linear_dynamic_impl(const void *x, pgf8_dtype xdt, int64_t M,
     uint8_t *aq = static_cast<uint8_t *>(workspace) + pgf8_fp8_linear_dynamic_codes_offset(M, K);
     float *sa = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
                                           pgf8_fp8_linear_dynamic_scales_offset(M, K));
-    st = check_quantize_args(x, xdt, M, K, ldx, aq, sa, PGF8_SCALE_DYNAMIC);
+    return check_quantize_args(x, xdt, M, K, ldx, aq, sa, PGF8_SCALE_DYNAMIC);
+}
+
+static pgf8_status linear_dynamic_impl(const void *x, pgf8_dtype xdt, int64_t M, int64_t K, int64_t ldx,
+                                       const void *w, const void *w2, const float *sw, int64_t N, void *y,
+                                       void *workspace, size_t workspace_bytes, const pgf8_linear_opts *opts,
+                                       void *stream, int kind)
+{
+    pgf8_status st = check_linear_dynamic(x, xdt, M, K, ldx, w, sw, N, y, workspace, workspace_bytes, kind);
     if (st != PGF8_OK)
         return st;
+    uint8_t *aq = static_cast<uint8_t *>(workspace) + pgf8_fp8_linear_dynamic_codes_offset(M, K);
+    float *sa = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                          pgf8_fp8_linear_dynamic_scales_offset(M, K));
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const pgf8_linear_opts o = opts_or_default(opts);
     const int overlap = (o.flags & PGF8_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
@@ -677,6 +666,31 @@ pgf8_status pgf8_fp8_linear_dynamic(const void *x, pgf8_dtype xdt, int64_t M, in
 {
     return linear_dynamic_impl(x, xdt, M, K, ldx, wq, nullptr, sw, N, y, workspace, workspace_bytes, opts, stream,
                                kE4M3);
+}
+
+pgf8_status pgf8_fp8_linear_dynamic_many(const pgf8_fp8_layer *layers, int64_t count, const pgf8_linear_opts *opts,
+                                         void *stream)
+{
+    if (count < 0 || (count > 0 && !layers))
+        return PGF8_ERR_INVALID_ARG;
+    for (int64_t i = 0; i < count; ++i) {
+        const pgf8_fp8_layer &l = layers[i];
+        pgf8_status st = check_linear_dynamic(l.x, static_cast<pgf8_dtype>(l.xdt), l.M, l.K, l.ldx, l.wq, l.sw, l.N,
+                                              l.y, l.workspace, l.workspace_bytes, kE4M3);
+        if (st != PGF8_OK)
+            return st;
+    }
+    pgf8_linear_opts o = opts_or_default(opts);
+    for (int64_t i = 0; i < count; ++i) {
+        const pgf8_fp8_layer &l = layers[i];
+        if (i > 0)
+            o.flags |= PGF8_FLAG_OVERLAP_PREVIOUS;
+        pgf8_status st = linear_dynamic_impl(l.x, static_cast<pgf8_dtype>(l.xdt), l.M, l.K, l.ldx, l.wq, nullptr,
+                                             l.sw, l.N, l.y, l.workspace, l.workspace_bytes, &o, stream, kE4M3);
+        if (st != PGF8_OK)
+            return st;
+    }
+    return PGF8_OK;
 }
 
 pgf8_status pgf8_nestedfp_split(const void *w, int64_t N, int64_t K, uint8_t *hi, uint8_t *lo, void *stream)
@@ -754,6 +768,18 @@ pgf8_status pgf8_last_cuda_error(int *cuda_err)
     if (!cuda_err)
         return PGF8_ERR_INVALID_ARG;
     *cuda_err = tl_last_cuda_error;
+    return PGF8_OK;
+}
+
+pgf8_status pgf8_selftest_bounded_wait(int64_t limit_ns, void *stream)
+{
+    if (limit_ns < 1000 || limit_ns > 2000000000ll)
+        return PGF8_ERR_INVALID_ARG;
+    selftest_bounded_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint64_t>(limit_ns));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return cuda_fail(e);
     return PGF8_OK;
 }
 

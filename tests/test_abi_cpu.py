@@ -135,3 +135,14 @@ def test_streamk_path_argument_checks():
     # misaligned workspace
     assert pg.lib.pgf8_fp8_linear_ex(A16, B16, 8, 512, C16, D16, 512, A16, D16 + 8, 1 << 24, ctypes.byref(o),
                                      None) == pg.ERR_ALIGNMENT
+
+
+def test_dynamic_many_checks_every_layer_first():
+    good = pg.Fp8Layer(A16, pg.F32, 0, 4, 512, 512, 512, B16, C16, D16, A16, 1 << 24)
+    bad = pg.Fp8Layer(A16, pg.F32, 0, 4, 520, 520, 512, B16, C16, D16, A16, 1 << 24)   # K % 16
+    arr = (pg.Fp8Layer * 3)(good, bad, good)
+    # the invalid second layer is reported before anything (including layer 1) is enqueued
+    assert pg.lib.pgf8_fp8_linear_dynamic_many(arr, 3, None, None) == pg.ERR_ALIGNMENT
+    assert pg.lib.pgf8_fp8_linear_dynamic_many(None, 2, None, None) == pg.ERR_INVALID_ARG
+    assert pg.lib.pgf8_fp8_linear_dynamic_many(None, 0, None, None) == pg.OK
+    assert pg.lib.pgf8_fp8_linear_dynamic_many(arr, -1, None, None) == pg.ERR_INVALID_ARG

@@ -232,3 +232,33 @@ def test_streamk_against_oracle_and_flags_cleared(M, N, K):
         outs.append(y)
     for y in outs[1:]:
         np.testing.assert_array_equal(y, outs[0])
+
+
+def test_dynamic_many_matches_single_calls():
+    """pgf8_fp8_linear_dynamic_many runs the same kernels as one
+    fp8_linear_dynamic call per layer: outputs bit-identical, and they stay
+    within the bound of the oracle."""
+    shapes = [(1, 4096, 12288), (4, 4096, 4096), (8, 11008, 4096), (300, 512, 1024)]
+    g = np.random.default_rng(31)
+    seq, singles, refs = [], [], []
+    for M, K, N in shapes:
+        x = synthetic.activations("normal_outl_0p5pct_x30", M, K, g)
+        w = synthetic.weights_f16(N, K, 0.02, g)
+        xt = _to(x)
+        wq, sw = pg.fp8_quantize_rows(_to(w))
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
+        ws = torch.zeros(pg.fp8_linear_dynamic_workspace_size(M, N, K), dtype=torch.uint8, device=DEV)
+        seq.append((xt, wq, sw, y, ws))
+        ws2 = torch.zeros_like(ws)
+        singles.append(pg.fp8_linear_dynamic(xt, wq, sw, workspace=ws2))
+        refs.append((x, w))
+    pg.LayerSequence(seq).run()
+    torch.cuda.synchronize()
+    assert pg.device_status() == pg.OK
+    for (xt, wq, sw, y, ws), y1, (x, w) in zip(seq, singles, refs):
+        np.testing.assert_array_equal(y.float().cpu().numpy(), y1.float().cpu().numpy())
+        aq, sa = oracle.quantize_rows(x[:8])
+        wq0, sw0 = oracle.quantize_rows(w[:64])
+        ref = oracle.fp8_linear(aq, sa, wq0, sw0)
+        bound = linear_bound(ref, x.shape[1], fp8_row_max(aq, sa), fp8_row_max(wq0, sw0))
+        assert_within(y.float().cpu().numpy()[:8, :64], ref, bound, f"many {x.shape}")
