@@ -270,6 +270,9 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
 
     stream = torch.cuda.Stream(device=dev)
+    # dynamic layers quantise with their own kernel first (the two-kernel
+    # form); with --fused-quant inside the GEMM where the kernel allows it
+    xflags = pg.FLAG_FUSED_QUANT if args.fused_quant else 0
     sk_ws = torch.zeros(max(16, max(pg.lib.pgf8_fp8_linear_workspace_size(L.M, L.N, L.K) for L in layers)),
                         dtype=torch.uint8, device=dev)
 
@@ -287,7 +290,7 @@ def run_ours(args, rank, world, local_rank):
             if L.kind == "fp8":
                 if ev_pairs is None:
                     pg.fp8_linear_dynamic(acts[i], W[0], W[1], y=outs[i], workspace=qbufs[i],
-                                          flags=pg.FLAG_OVERLAP_PREVIOUS, stream=stream)
+                                          flags=pg.FLAG_OVERLAP_PREVIOUS | xflags, stream=stream)
                     continue
                 aq, sa = pg.dynamic_workspace_views(qbufs[i], L.M, L.K)
                 ev_pairs[i][2].record(stream)
@@ -301,7 +304,8 @@ def run_ours(args, rank, world, local_rank):
                     ev_pairs[i][0].record(stream)
                 pg.nestedfp_linear(acts[i], W[0], W[1] if mode == pg.NESTED_FP16 else None, mode=mode,
                                    y=outs[i], workspace=qbufs[i],
-                                   flags=0 if ev_pairs is not None else pg.FLAG_OVERLAP_PREVIOUS, stream=stream)
+                                   flags=xflags if ev_pairs is not None else pg.FLAG_OVERLAP_PREVIOUS | xflags,
+                                   stream=stream)
                 if ev_pairs is not None:
                     ev_pairs[i][1].record(stream)
 
@@ -422,7 +426,10 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "inputs larger than L2 (%d weight copies; %.0f MB of weights streamed per step)"
                          % (copies, wbytes / 1e6),
                    "timing": "CUDA graph of the C-ABI calls (R-1 chained steps + 1 event-bracketed step), "
-                             "replayed K/R times, R=%d" % R},
+                             "replayed K/R times, R=%d" % R,
+                   "quantisation": "inside the skinny GEMM where each CTA's activation slice fits its "
+                                   "registers, else its own kernel" if args.fused_quant
+                   else "own kernel before each GEMM"},
         "secondary": {"tflops": round(tflops, 3), "weight_gbs": round(gbs, 1)},
         "roofline": roof,
         "e2e": e2e,
@@ -476,14 +483,14 @@ def run_e2e(pg, torch, dev, layers, weights, acts_host, outs, args, world, wbyte
         with torch.cuda.stream(stream):
             x_dev.copy_(x_host, non_blocking=True)
             if seq is not None:
-                seq.run(stream=stream)
+                seq.run(flags=pg.FLAG_FUSED_QUANT if args.fused_quant else 0, stream=stream)
             else:
                 for i, L in enumerate(layers):
                     W = weights[(L.shape_idx, L.copy, True)]
                     mode = pg.NESTED_FP16 if L.kind == "nested16" else pg.NESTED_FP8
+                    fl = (pg.FLAG_OVERLAP_PREVIOUS if i else 0) | (pg.FLAG_FUSED_QUANT if args.fused_quant else 0)
                     pg.nestedfp_linear(x_views[i], W[0], W[1] if mode == pg.NESTED_FP16 else None, mode=mode,
-                                       y=y_views[i], workspace=ws[i], flags=pg.FLAG_OVERLAP_PREVIOUS if i else 0,
-                                       stream=stream)
+                                       y=y_views[i], workspace=ws[i], flags=fl, stream=stream)
             y_host.copy_(y_dev, non_blocking=True)
 
     steps = max(3, min(args.steps, 200))
@@ -638,6 +645,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(synthetic.WORKLOADS), default="decode7b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fused-quant", action="store_true",
+                    help="quantise dynamic activations inside the skinny GEMM where its kernel allows it")
     ap.add_argument("--single", default=None, help="kind,M,K,N: time (or profile) one layer eagerly")
     ap.add_argument("--path", type=int, default=0)
     ap.add_argument("--split-k", type=int, default=0)

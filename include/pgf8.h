@@ -102,6 +102,18 @@ typedef enum {
  * during inference satisfy this). */
 #define PGF8_FLAG_OVERLAP_PREVIOUS 1
 
+/* PGF8_FLAG_FUSED_QUANT (dynamic entry points only): quantise the
+ * activations inside the GEMM instead of running the per-token quantisation
+ * as its own kernel first.  Applies where a dynamic call has M <= 32 on the
+ * skinny path (path AUTO or SKINNY, tile_n 0, 16 or 32) and each CTA's
+ * activation slice (M rows of its K-split) fits its registers (at most 8192
+ * f32 or 16384 f16 elements); elsewhere the flag changes nothing.  One
+ * kernel instead of two, with the same codes, scales and outputs, bit for
+ * bit.  Not the default: on B200 the two-kernel form measured faster in
+ * chained decode steps (its quantisation kernel hides the GEMM's weight
+ * prefetch behind the previous layer). */
+#define PGF8_FLAG_FUSED_QUANT 2
+
 /* Optional tuning of the linear entry points; a NULL pointer means all
  * defaults.  Fields set to 0 mean "choose automatically". */
 typedef struct {
@@ -170,6 +182,17 @@ pgf8_status pgf8_fp8_linear_dynamic(const void *x, pgf8_dtype xdt, int64_t M, in
 
 size_t pgf8_fp8_linear_dynamic_workspace_size(int64_t M, int64_t N, int64_t K);
 size_t pgf8_fp8_linear_dynamic_codes_offset(int64_t M, int64_t K);
+
+/* Which kernels a dynamic FP8 linear call with these arguments would run
+ * (host only: nothing is enqueued, no device memory is touched).  *fused =
+ * 1 when the GEMM quantises the activations itself (PGF8_FLAG_FUSED_QUANT
+ * set and applicable), else 0.  *split_k = the K-split of the skinny GEMM
+ * (1..8), or 0 when the call takes a tiled kernel.  Returns
+ * PGF8_ERR_INVALID_ARG / ALIGNMENT / UNSUPPORTED for arguments the call
+ * itself would reject on shape or dtype grounds.  The pages have no
+ * counterpart: this is a query of this library's kernel choice. */
+pgf8_status pgf8_fp8_linear_dynamic_plan(int64_t M, int64_t N, int64_t K, pgf8_dtype xdt,
+                                         const pgf8_linear_opts *opts, int32_t *fused, int32_t *split_k);
 
 /* One layer of pgf8_fp8_linear_dynamic_many: the arguments of
  * pgf8_fp8_linear_dynamic. */
@@ -280,12 +303,26 @@ pgf8_status pgf8_fp8_linear_dynamic_noalloc(const void *x, pgf8_dtype xdt, int64
  *   device error word and the kernel returns: the next pgf8_device_status()
  *   on that stream reports PGF8_ERR_TIMEOUT and clears it.  For checking the
  *   failure path without hanging or faulting the GPU.
+ * pgf8_selftest_row_division: checks the division the quantisation uses
+ *   (x / s rounded to nearest-even binary32, one divisor per row, by an
+ *   FMA remainder correction) against the device's IEEE division over EVERY
+ *   finite binary32 x with |x| <= 512 s, for each of the `count` divisors in
+ *   divisors[] (device, f32, count 1..64).  mismatches[] (device, 2 * count
+ *   uint64, zero-filled by the caller) receives per divisor i:
+ *   [2i] quotients that differ bitwise where |x| >= 2^-11 s, and [2i+1]
+ *   E4M3 codes (RN, saturating) that differ anywhere in the domain.  Below
+ *   2^-11 s the quotient may differ in its last bits (subnormal remainders)
+ *   while its code is zero either way.  About 2^32 divisions per divisor
+ *   (milliseconds each).  The pages define the quotient only as the rounded
+ *   division; this self-test has no counterpart there.
  * pgf8_status_str: static description of a status code.
  * pgf8_version: library version as major*10000 + minor*100 + patch.
  * ---------------------------------------------------------------------- */
 pgf8_status pgf8_last_cuda_error(int *cuda_err);
 pgf8_status pgf8_device_status(void *stream);
 pgf8_status pgf8_selftest_bounded_wait(int64_t limit_ns, void *stream);
+pgf8_status pgf8_selftest_row_division(const float *divisors, int32_t count,
+                                       unsigned long long *mismatches, void *stream);
 const char *pgf8_status_str(pgf8_status status);
 int pgf8_version(void);
 

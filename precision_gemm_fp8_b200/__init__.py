@@ -33,6 +33,7 @@ SCALE_DYNAMIC, SCALE_STATIC = 0, 1
 NESTED_FP16, NESTED_FP8 = 0, 1
 PATH_AUTO, PATH_SKINNY, PATH_TILED, PATH_STREAMK, PATH_TILED_PAIR = 0, 1, 2, 3, 4
 FLAG_OVERLAP_PREVIOUS = 1
+FLAG_FUSED_QUANT = 2
 
 
 class LinearOpts(ctypes.Structure):
@@ -71,6 +72,8 @@ _SIGS = {
     "pgf8_last_cuda_error": ([ctypes.POINTER(ctypes.c_int)], _i32),
     "pgf8_device_status": ([_vp], _i32),
     "pgf8_selftest_bounded_wait": ([_i64, _vp], _i32),
+    "pgf8_selftest_row_division": ([_vp, _i32, _vp, _vp], _i32),
+    "pgf8_fp8_linear_dynamic_plan": ([_i64, _i64, _i64, _i32, _vp, _vp, _vp], _i32),
     "pgf8_status_str": ([_i32], ctypes.c_char_p),
     "pgf8_version": ([], _i32),
 }
@@ -216,6 +219,21 @@ def fp8_linear_dynamic(x, wq, sw, y=None, workspace=None, path=PATH_AUTO, split_
     return y
 
 
+def fp8_linear_dynamic_plan(M: int, N: int, K: int, x_dtype=torch.float32, path=PATH_AUTO, split_k=0, tile_n=0,
+                            flags=0):
+    """(fused, split_k) the dynamic FP8 linear would use for these arguments:
+    fused True when the GEMM quantises the activations itself; split_k the
+    skinny GEMM's K-split (0 for a tiled kernel)."""
+    code = {torch.float32: F32, torch.float16: F16}.get(x_dtype)
+    if code is None:
+        raise TypeError(f"unsupported activation dtype {x_dtype}")
+    fused, split = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(lib.pgf8_fp8_linear_dynamic_plan(M, N, K, code, _opts(path, split_k, tile_n, flags),
+                                            ctypes.addressof(fused), ctypes.addressof(split)),
+           "fp8_linear_dynamic_plan")
+    return bool(fused.value), int(split.value)
+
+
 def fp8_linear_dynamic_noalloc(x, wq, sw, y=None, stream=None):
     """fp8_linear_dynamic without a workspace, for callers that cannot allocate
     one: the codes and scales live in the library's fixed 8 MiB device array
@@ -299,6 +317,19 @@ def nestedfp_linear(x, hi, lo, mode=NESTED_FP16, y=None, workspace=None, path=PA
                                        _ptr(y), _ptr(workspace), wbytes, _opts(path, split_k, tile_n, flags),
                                        _stream(stream)), "nestedfp_linear")
     return y
+
+
+def selftest_row_division(divisors: torch.Tensor, stream=None):
+    """[count, 2] int64 mismatch counts of the quantisation's division against
+    the device's IEEE division over every binary32 x with |x| <= 512 s:
+    column 0 quotients (where |x| >= 2^-11 s), column 1 E4M3 codes (see
+    pgf8_selftest_row_division)."""
+    if divisors.dtype != torch.float32 or not divisors.is_contiguous():
+        raise ValueError("divisors must be a contiguous float32 tensor")
+    counts = torch.zeros((divisors.numel(), 2), dtype=torch.int64, device=divisors.device)
+    _check(lib.pgf8_selftest_row_division(_ptr(divisors), divisors.numel(), _ptr(counts), _stream(stream)),
+           "selftest_row_division")
+    return counts
 
 
 def device_status(stream=None) -> int:

@@ -28,6 +28,20 @@
 //               FP16 layout), then hand it to the MMA thread.
 //               All kinds: epilogue — tcgen05.ld of the accumulator, scaling,
 //               rounding, 16- or 2-byte stores.
+// Quantised activations (XQ, skinny FP8 kinds, M <= BN <= 32, the CTA's
+// activation slice small enough for registers): the kernel reads the f32 /
+// f16 activations itself instead of E4M3 codes made by a separate pass
+// ("7B on an RTX 4060 with FP8" §2.2 dynamic per-token scale, computed
+// here).  Warps 2-5 load the CTA's K-slice of the M rows into registers and
+// take each token's amax over it; the CTAs of a split-K cluster combine
+// their partial maxima through distributed shared memory; the registers are
+// then converted (x / s rounded to E4M3, saturating, exactly as the
+// quantisation kernel does) and written into the B tiles of the weight
+// stages, which the MMA thread waits for like a TMA load.  The weights need
+// no dependency wait, so with programmatic launch they stream while the
+// previous kernel finishes.  CTAs of weight tile 0 also write the codes (and
+// one CTA the scales) to global memory, so the caller sees the same side
+// outputs as with the separate pass.
 // Split-K: with SPLIT, the CTAs of one thread-block cluster (along z) each
 // accumulate a slice of K; partial tiles are exchanged through distributed
 // shared memory and summed in cluster-rank order (deterministic), each CTA
@@ -43,6 +57,7 @@
 #include <cuda_fp16.h>
 #include <cstdint>
 
+#include "quantize.cuh"
 #include "sm100_ptx.cuh"
 
 namespace pgf8 {
@@ -62,10 +77,62 @@ struct GemmParams {
     const float *sa;     // [M] (kE4M3, kNested8)
     const float *sw;     // [N] (kE4M3)
     void *y;             // [M, N] bf16 (kE4M3) or f16
+    // XQ kernels only
+    const void *x;       // activations [M, K] f32 or f16, row stride ldx elements
+    int64_t ldx;
+    uint8_t *q_out;      // [M, K] E4M3 codes written by the CTAs of weight tile 0, or null
+    float *sa_out;       // [M] scales written by one CTA, or null
 };
 
-template <bool SWAP_, int BN_, int STAGES_, int KIND_, bool SPLIT_> struct GemmCfg {
+// 16 consecutive activations of one row as loaded (XQ = 1: f32, 2: f16).
+template <int XQ> struct XRaw;
+template <> struct XRaw<1> {
+    static constexpr int kElemBytes = 4;
+    uint4 w[4];
+    __device__ __forceinline__ void load(const uint8_t *p)
+    {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            w[i] = __ldg(reinterpret_cast<const uint4 *>(p) + i);
+    }
+    __device__ __forceinline__ void to_float(float (&v)[16]) const
+    {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[4 * i + 0] = __uint_as_float(w[i].x);
+            v[4 * i + 1] = __uint_as_float(w[i].y);
+            v[4 * i + 2] = __uint_as_float(w[i].z);
+            v[4 * i + 3] = __uint_as_float(w[i].w);
+        }
+    }
+};
+template <> struct XRaw<2> {
+    static constexpr int kElemBytes = 2;
+    uint4 w[2];
+    __device__ __forceinline__ void load(const uint8_t *p)
+    {
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+            w[i] = __ldg(reinterpret_cast<const uint4 *>(p) + i);
+    }
+    __device__ __forceinline__ void to_float(float (&v)[16]) const
+    {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const uint32_t t[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&t[j]));   // exact
+                v[8 * i + 2 * j] = f.x;
+                v[8 * i + 2 * j + 1] = f.y;
+            }
+        }
+    }
+};
+
+template <bool SWAP_, int BN_, int STAGES_, int KIND_, bool SPLIT_, int XQ_ = 0> struct GemmCfg {
     static constexpr bool SWAP = SWAP_;
+    static constexpr int XQ = XQ_;   // 0: X read as E4M3 codes by TMA; 1 / 2: f32 / f16 activations quantised in the kernel
     static constexpr int BN = BN_;
     static constexpr int STAGES = STAGES_;
     static constexpr int KIND = KIND_;
@@ -87,12 +154,14 @@ template <bool SWAP_, int BN_, int STAGES_, int KIND_, bool SPLIT_> struct GemmC
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128 must be a multiple of 16 in [16,256]");
     static_assert((BN & (BN - 1)) == 0 || BN % 32 == 0, "BN");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+    static_assert(XQ == 0 || (SWAP && KIND != kNested16 && BN <= 32), "in-kernel quantisation: skinny FP8, M <= 32");
+    static_assert(STAGES <= 8 && kStage % 1024 == 0, "ring");
 };
 
 struct SharedCtl {
-    uint64_t full[16];
-    uint64_t empty[16];
-    uint64_t conv[16];
+    uint64_t full[8];
+    uint64_t empty[8];
+    uint64_t conv[8];
     uint64_t tmem_full;
     uint64_t drain;
     uint32_t tmem_base;
@@ -212,6 +281,174 @@ template <int KIND> __device__ __forceinline__ uint32_t pack2(float a, float b)
     }
 }
 
+// XQ helpers.
+// Partial amax of one batch of 16-element chunks (row[u] < 0: no chunk):
+// f32 max of |x| (NaN ignored, as the quantisation kernel), segmented warp
+// max, shared atomic max on the bits (non-negative floats order like their
+// bit patterns).
+template <int XQ, int U>
+__device__ __forceinline__ void xq_batch_amax(const XRaw<XQ> (&raw)[U], const int (&row)[U], uint32_t *xq_amax,
+                                              int lane)
+{
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        float mx = 0.0f;
+        if (row[u] >= 0) {
+            float v[16];
+            raw[u].to_float(v);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                mx = fmaxf(mx, fabsf(v[i]));
+        }
+        const unsigned grp = __match_any_sync(0xffffffffu, row[u]);
+        const unsigned mb = __reduce_max_sync(grp, __float_as_uint(mx));
+        if (row[u] >= 0 && lane == __ffs(grp) - 1)
+            atomicMax(&xq_amax[row[u]], mb);
+    }
+}
+
+// Per-token scales from the slice maxima: with split-K the cluster barrier
+// publishes every CTA's maxima and each CTA reads all of them, so all derive
+// the same s = amax / 448 (1 when the row is zero) — the "7B on an RTX 4060
+// with FP8" §2.2 / §6.1 dynamic scale — into ctl->sa_s (and, from one CTA,
+// p.sa_out).  Called by all 128 threads of warps 2-5.
+template <class C>
+__device__ __forceinline__ void xq_scales(const GemmParams &p, SharedCtl *ctl, uint32_t *xq_amax, int et, int tile_a,
+                                          int split)
+{
+    if constexpr (C::SPLIT) {
+        cluster_arrive_release();
+        cluster_wait_acquire();
+    } else {
+        bar_sync_warps2to5();
+    }
+    if (et < p.M) {
+        uint32_t b = xq_amax[et];
+        if constexpr (C::SPLIT) {
+            const uint32_t a = smem_u32(&xq_amax[et]);
+            for (int z = 0; z < p.splits; ++z) {
+                const uint32_t o = ld_shared_cluster_u32(map_shared_rank(a, static_cast<uint32_t>(z)));
+                b = o > b ? o : b;
+            }
+        }
+        float sc = __fdiv_rn(__uint_as_float(b), 448.0f);
+        if (sc == 0.0f)
+            sc = 1.0f;
+        ctl->sa_s[et] = sc;
+        if (p.sa_out && tile_a == 0 && split == 0)
+            p.sa_out[et] = sc;
+    }
+    bar_sync_warps2to5();
+}
+
+// XQ: warps 2-5 quantise the CTA's activation slice (M rows x k-blocks
+// [kb0, kb1)), which fits one batch of the amax pass (at most 128 x U chunks
+// of 16 elements) and so stays in registers: amax, scales, then the chunks are converted to codes
+// in registers and written into the B tiles of the weight stages as they
+// free up.  No activation is loaded after pass 1.  The B tiles are zeroed
+// once (rows >= M are never written); in a ragged last k-block the chunks
+// past K are zeroed again.  Loop exits are agreed by all 128 threads
+// (barrier with AND).
+template <class C>
+__device__ __forceinline__ void quantize_x_resident(const GemmParams &p, uint8_t *smem, SharedCtl *ctl,
+                                                    uint32_t *xq_amax, volatile int *abort_flag, int kb0, int kb1,
+                                                    int tile_a, int split)
+{
+    constexpr int XQ = C::XQ;
+    constexpr int EB = XRaw<XQ>::kElemBytes;
+    constexpr int U = XQ == 1 ? 4 : 8;
+    const int et = static_cast<int>(threadIdx.x) - 64;   // 0..127
+    const int lane = et & 31;
+    const uint8_t *xb = static_cast<const uint8_t *>(p.x);
+    const int64_t row_bytes = p.ldx * EB;
+
+    // B tiles start zero (rows >= M are never written)
+    for (int i = et; i < C::STAGES * C::kTileB / 16; i += 128) {
+        const int st = i / (C::kTileB / 16), rest = i % (C::kTileB / 16);
+        *reinterpret_cast<uint4 *>(smem + st * C::kStage + C::kTileA + rest * 16) = make_uint4(0u, 0u, 0u, 0u);
+    }
+
+    // nothing of x may be read before the kernel that writes it has completed
+    grid_dependency_wait();
+
+    // ---- 1. the slice, one batch: chunk it = u * 128 + et -> row m, chunk c
+    const int kbeg = kb0 * 128;
+    const int kend = (kb1 * 128 < p.K) ? kb1 * 128 : p.K;
+    const int nch = (kend - kbeg) >> 4;
+    const int items = p.M * nch;            // <= 128 * U (checked by the host)
+    XRaw<XQ> raw[U];
+    int row[U], chunk[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int it = u * 128 + et;
+        row[u] = -1;
+        chunk[u] = 0;
+        if (it < items) {
+            const int m = it / nch;
+            const int c = it - m * nch;
+            row[u] = m;
+            chunk[u] = c;
+            raw[u].load(xb + m * row_bytes + static_cast<int64_t>(kbeg + c * 16) * EB);
+        }
+    }
+    xq_batch_amax<XQ, U>(raw, row, xq_amax, lane);
+
+    // ---- 2. scales
+    xq_scales<C>(p, ctl, xq_amax, et, tile_a, split);
+
+    // ---- 3. codes in registers, then into the weight stages
+    uint4 code[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        code[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (row[u] >= 0) {
+            float v[16];
+            raw[u].to_float(v);
+            code[u] = encode16(v, RowDivisor(ctl->sa_s[row[u]]));
+        }
+    }
+    const bool write_codes = p.q_out != nullptr && tile_a == 0;
+    int s = 0;
+    uint32_t ph = 0;
+    for (int kb = kb0; kb < kb1; ++kb) {
+        const int n = kb - kb0;
+        bool ok = true;
+        if (n >= C::STAGES)
+            ok = wait_bounded(&ctl->empty[s], ph ^ 1u, abort_flag);
+        if (!bar_and_warps2to5(ok))
+            break;
+        uint8_t *bt = smem + s * C::kStage + C::kTileA;
+        if (kb == kb1 - 1 && kend < kb1 * 128) {
+            // ragged K: the stage's chunks past K still hold an earlier
+            // k-block's codes; zero them (a stale NaN code times a zero-filled
+            // weight would poison the accumulator)
+            for (int i = et; i < p.M * 8; i += 128) {
+                const int r = i >> 3, j = i & 7;
+                if (kb * 128 + 16 * j >= kend)
+                    *reinterpret_cast<uint4 *>(bt + r * 128 + ((j ^ (r & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (row[u] >= 0 && (chunk[u] >> 3) == n) {
+                const int r = row[u], j = chunk[u] & 7;
+                if (write_codes)
+                    *reinterpret_cast<uint4 *>(p.q_out + static_cast<int64_t>(r) * p.K + kbeg + chunk[u] * 16) =
+                        code[u];
+                *reinterpret_cast<uint4 *>(bt + r * 128 + ((j ^ (r & 7)) << 4)) = code[u];
+            }
+        }
+        fence_proxy_async_smem();   // each writer, before the MMA (async proxy) reads
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&ctl->conv[s]);
+        if (++s == C::STAGES) {
+            s = 0;
+            ph ^= 1u;
+        }
+    }
+}
+
 template <class C>
 __global__ void __launch_bounds__(192, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
@@ -222,6 +459,7 @@ __global__ void __launch_bounds__(192, 1)
     constexpr int STAGES = C::STAGES;
     constexpr int KIND = C::KIND;
     constexpr bool NEST16 = (KIND == kNested16);
+    constexpr int XQ = C::XQ;
     constexpr uint32_t kIdesc =
         make_idesc(128, BN, /*A fmt*/ (SWAP && KIND == kNested8) ? 1 : 0, /*B fmt*/ (!SWAP && KIND == kNested8) ? 1 : 0);
     constexpr int kXStep = NEST16 ? 64 : 128;   // K elements per stage
@@ -245,6 +483,7 @@ __global__ void __launch_bounds__(192, 1)
     const int kb1 = C::SPLIT ? ((split + 1) * p.kblocks) / p.splits : p.kblocks;
     const int row0_w = SWAP ? tile_a * 128 : tile_b * BN;   // first weight row of the tile
     const int row0_x = SWAP ? tile_b * BN : tile_a * 128;   // first token row of the tile
+    __shared__ uint32_t xq_amax[XQ ? 32 : 1];   // XQ: bits of the per-token amax (non-negative floats)
 
     // Producer state (thread 0): the first pass of the ring is issued before
     // the CTA-wide synchronisation, so its loads overlap the set-up.
@@ -259,7 +498,7 @@ __global__ void __launch_bounds__(192, 1)
     auto issue_w = [&](int kb, int st_idx) {
         uint8_t *st = smem + st_idx * C::kStage;
         uint8_t *w_tile = SWAP ? st : st + C::kTileA;
-        mbar_arrive_expect_tx(&ctl->full[st_idx], C::kStage);
+        mbar_arrive_expect_tx(&ctl->full[st_idx], XQ ? C::kTileA : C::kStage);
         if constexpr (NEST16) {
             // hi and lo planes, 64 bytes (= 64 weights) of K each
             tma_load_2d_hint(w_tile, &tmW, &ctl->full[st_idx], kb * 64, row0_w, pol_w);
@@ -291,10 +530,12 @@ __global__ void __launch_bounds__(192, 1)
             ps = 0;
             pph ^= 1u;
         }
-        if (waited) {
-            issue_x(kb, (ps + STAGES - 1) % STAGES);
-        } else if (++pending == STAGES) {
-            flush_pending(kb + 1, ps);
+        if constexpr (!XQ) {   // XQ: warps 2-5 load and convert the activations
+            if (waited) {
+                issue_x(kb, (ps + STAGES - 1) % STAGES);
+            } else if (++pending == STAGES) {
+                flush_pending(kb + 1, ps);
+            }
         }
     };
 
@@ -302,13 +543,18 @@ __global__ void __launch_bounds__(192, 1)
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&ctl->full[s], 1);
             mbar_init(&ctl->empty[s], 1);
-            mbar_init(&ctl->conv[s], 128);
+            mbar_init(&ctl->conv[s], 4);    // one arrival per warp of warps 2-5
         }
         mbar_init(&ctl->tmem_full, 1);
         mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
+        if constexpr (XQ) {
+            for (int m = 0; m < 32; ++m)
+                xq_amax[m] = 0u;
+        }
         fence_mbar_init();
-        tma_prefetch_desc(&tmX);
+        if (!XQ)
+            tma_prefetch_desc(&tmX);
         tma_prefetch_desc(&tmW);
         if (NEST16)
             tma_prefetch_desc(&tmW2);
@@ -329,7 +575,7 @@ __global__ void __launch_bounds__(192, 1)
         tmem_alloc(&ctl->tmem_base, C::kTmemCols);
         tmem_relinquish();
     }
-    if (warp >= 2) {
+    if (warp >= 2 && !XQ) {
         // scales of this tile's tokens, read once (after the dependency, as
         // they may come from the previous kernel)
         grid_dependency_wait();
@@ -343,6 +589,13 @@ __global__ void __launch_bounds__(192, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctl->tmem_base;
+    // XQ with split-K: every thread of the cluster takes part in one barrier
+    // phase that publishes the partial maxima; the producer and MMA warps
+    // arrive now and wait after their loops
+    if constexpr (XQ && C::SPLIT) {
+        if (warp < 2)
+            cluster_arrive_relaxed();
+    }
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -377,7 +630,7 @@ __global__ void __launch_bounds__(192, 1)
                     ok = false;
                     break;
                 }
-                if constexpr (NEST16) {
+                if constexpr (NEST16 || XQ) {
                     if (!wait_bounded(&ctl->conv[s], ph, abort_flag)) {
                         ok = false;
                         break;
@@ -421,14 +674,22 @@ __global__ void __launch_bounds__(192, 1)
                     break;
                 uint8_t *tile = smem + s * C::kStage + (SWAP ? 0 : C::kTileA);
                 rebuild_fp16_tile<C::kRowsW>(tile, tt);
-                fence_proxy_async_smem();
-                mbar_arrive(&ctl->conv[s]);
+                fence_proxy_async_smem();   // each writer, before the MMA (async proxy) reads
+                __syncwarp();
+                if ((threadIdx.x & 31) == 0)
+                    mbar_arrive(&ctl->conv[s]);
                 if (++s == STAGES) {
                     s = 0;
                     ph ^= 1u;
                 }
             }
+        } else if constexpr (XQ) {
+            quantize_x_resident<C>(p, smem, ctl, xq_amax, abort_flag, kb0, kb1, tile_a, split);
         }
+    }
+    if constexpr (XQ && C::SPLIT) {
+        if (warp < 2)
+            cluster_wait_acquire();
     }
 
     // ---------------------------------------------------------------- epilogue
@@ -613,7 +874,9 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 float a[4] = {acc.x, acc.y, acc.z, acc.w};
                 float sam = 1.0f;
-                if constexpr (KIND != kNested16)
+                if constexpr (XQ)
+                    sam = ctl->sa_s[m - row0_x];
+                else if constexpr (KIND != kNested16)
                     sam = p.sa[m];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {

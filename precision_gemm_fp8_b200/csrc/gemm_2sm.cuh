@@ -31,6 +31,7 @@ template <int BN_, int STAGES_, int KIND_> struct PairCfg {
     static constexpr int BN = BN_;                 // N of the pair's tile (MMA N)
     static constexpr int STAGES = STAGES_;
     static constexpr int KIND = KIND_;
+    static constexpr int XQ = 0;   // activations arrive as E4M3 codes
     static constexpr int kThreads = 192;
     static constexpr int kTileA = 128 * 128;      // this CTA's 128 activation rows
     static constexpr int kTileB = (BN / 2) * 128; // this CTA's BN/2 weight rows

@@ -25,6 +25,7 @@ template <int BN_, int STAGES_, int KIND_> struct PersistCfg {
     static constexpr int BN = BN_;
     static constexpr int STAGES = STAGES_;
     static constexpr int KIND = KIND_;
+    static constexpr int XQ = 0;   // activations arrive as E4M3 codes
     static constexpr bool SWAP = false;
     static constexpr bool NEST16 = (KIND == kNested16);
     static constexpr int kThreads = NEST16 ? 320 : 192;
@@ -83,7 +84,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&ctl->full[s], 1);
             mbar_init(&ctl->empty[s], 1);
-            mbar_init(&ctl->conv[s], 128);
+            mbar_init(&ctl->conv[s], 4);    // one arrival per rebuild warp
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->acc_full[b], 1);
@@ -271,8 +272,10 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                         break;
                     }
                     rebuild_fp16_tile<BN>(smem + s * C::kStage + C::kTileA, tt);
-                    fence_proxy_async_smem();
-                    mbar_arrive(&ctl->conv[s]);
+                    fence_proxy_async_smem();   // each writer, before the MMA (async proxy) reads
+                    __syncwarp();
+                    if ((threadIdx.x & 31) == 0)
+                        mbar_arrive(&ctl->conv[s]);
                     if (++s == STAGES) {
                         s = 0;
                         ph ^= 1u;

@@ -18,6 +18,14 @@
 #ifndef PGF8_SKINNY16_STAGES
 #define PGF8_SKINNY16_STAGES 6
 #endif
+// In-GEMM quantisation of dynamic activations is used up to this many tokens
+// and this many K-splits (beyond: the quantisation kernel, then the GEMM).
+#ifndef PGF8_FUSED_MAX_M
+#define PGF8_FUSED_MAX_M 32
+#endif
+#ifndef PGF8_FUSED_MAX_SPLITS
+#define PGF8_FUSED_MAX_SPLITS 8
+#endif
 #ifndef PGF8_STREAMK16_STAGES
 #define PGF8_STREAMK16_STAGES 6
 #endif
@@ -61,13 +69,14 @@ static EncodeTiledFn encode_fn()
 // 2-D row-major [rows, cols] tensor; box = box_cols x box_rows; element
 // size from dtype.  Out-of-range elements of a box read as zero.
 static bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem_bytes, uint64_t rows,
-                     uint64_t cols, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw)
+                     uint64_t cols, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw,
+                     uint64_t row_stride_elems = 0)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn)
         return false;
     cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elem_bytes)};
+    cuuint64_t strides[1] = {(row_stride_elems ? row_stride_elems : cols) * static_cast<uint64_t>(elem_bytes)};
     cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
@@ -90,6 +99,11 @@ struct GemmLaunch {
     cudaStream_t stream;
     void *ws;          // stream-K region of the workspace (flags, then partial slots), or null
     size_t ws_bytes;
+    // in-kernel quantisation (XQ kernels): raw activations and side outputs
+    const void *xraw = nullptr;
+    int64_t ldx = 0;
+    uint8_t *q_out = nullptr;
+    float *sa_out = nullptr;
 };
 
 // Tensor maps of the two operands for a kernel configuration C (tile rows
@@ -100,7 +114,13 @@ template <class C> static bool make_operand_maps(const GemmLaunch &L, CUtensorMa
     const bool nest16 = (C::KIND == kNested16);
     std::memset(&tmW2, 0, sizeof(tmW2));
     bool ok;
-    if (nest16) {
+    if constexpr (C::XQ != 0) {
+        // the kernel loads the activations itself; only the weight map is used
+        std::memset(&tmX, 0, sizeof(tmX));
+        ok = make_map(&tmW, L.w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.N, L.K, 128, C::kRowsW,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+        tmW2 = tmW;
+    } else if (nest16) {
         ok = make_map(&tmX, L.x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, L.M, L.K, 64, C::kRowsX,
                       CU_TENSOR_MAP_SWIZZLE_128B) &&
              make_map(&tmW, L.w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.N, L.K, 64, C::kRowsW,
@@ -130,6 +150,10 @@ static GemmParams make_params(const GemmLaunch &L, int splits)
     p.sa = L.sa;
     p.sw = L.sw;
     p.y = L.y;
+    p.x = L.xraw;
+    p.ldx = L.ldx;
+    p.q_out = L.q_out;
+    p.sa_out = L.sa_out;
     return p;
 }
 
@@ -159,6 +183,12 @@ template <class C> static pgf8_status launch_cfg(const GemmLaunch &L, int splits
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
         attr_err = cudaFuncSetAttribute(gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        // the largest shared-memory carveout: the default sizes the SM's
+        // L1 / shared split for one CTA, which leaves the skinny kernels
+        // (about 110 KB each) at one CTA per SM
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(gemm_kernel<C>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                            cudaSharedmemCarveoutMaxShared);
     });
     if (attr_err != cudaSuccess)
         return cuda_fail(attr_err);
@@ -318,12 +348,12 @@ template <class C> static pgf8_status launch_streamk(const GemmLaunch &L)
     return PGF8_OK;
 }
 
-template <int KIND, bool SWAP, int BN, int STAGES>
+template <int KIND, bool SWAP, int BN, int STAGES, int XQ = 0>
 static pgf8_status launch_split_or_not(const GemmLaunch &L, int splits)
 {
     if (splits > 1)
-        return launch_cfg<GemmCfg<SWAP, BN, STAGES, KIND, true>>(L, splits);
-    return launch_cfg<GemmCfg<SWAP, BN, STAGES, KIND, false>>(L, 1);
+        return launch_cfg<GemmCfg<SWAP, BN, STAGES, KIND, true, XQ>>(L, splits);
+    return launch_cfg<GemmCfg<SWAP, BN, STAGES, KIND, false, XQ>>(L, 1);
 }
 
 static int num_sms()
@@ -337,6 +367,72 @@ static int num_sms()
             sms = 148;
     }
     return sms;
+}
+
+// The largest power-of-two split that keeps a skinny grid within ~1.75 CTAs
+// per SM (measured on B200 over the 7B and 70B decode shapes: 64 weight
+// tiles -> 4, 80-96 -> 2, >= 172 -> 1); beyond that the extra CTAs wait for
+// a second wave.
+static int skinny_auto_splits(int tiles, int sms)
+{
+    int splits = 1;
+    while (splits < 8 && tiles * splits * 2 * 4 <= sms * 7)
+        splits *= 2;
+    return splits;
+}
+
+template <int KIND, int BN, int STAGES, int XQ> static pgf8_status launch_xq_cfg(const GemmLaunch &L, int splits)
+{
+    // two CTAs per SM: 228 KB per SM, 1 KB reserved per CTA, 128 bytes static
+    static_assert(GemmCfg<true, BN, STAGES, KIND, true, XQ>::kSmemBytes + 128 + 1024 <= 228 * 1024 / 2,
+                  "fused-quantisation configuration exceeds half an SM's shared memory");
+    if (splits > 1)
+        return launch_cfg<GemmCfg<true, BN, STAGES, KIND, true, XQ>>(L, splits);
+    return launch_cfg<GemmCfg<true, BN, STAGES, KIND, false, XQ>>(L, 1);
+}
+
+// Split and tile of the skinny GEMM that quantises its activations itself,
+// and whether it applies: each CTA holds its whole activation slice (M rows
+// x its K-slice) in the registers of 128 threads, at most 4 chunks of 16
+// f32 or 8 of 16 f16 per thread.  L.opts.path is AUTO or SKINNY, tile_n 0 /
+// 16 / 32 (>= M), split_k 0..8 (checked by the caller).
+static bool xq_plan(const GemmLaunch &L, int xq, int &bn, int &splits)
+{
+    const int kblocks = (L.K + 127) / 128;
+    bn = L.opts.tile_n != 0 ? L.opts.tile_n : (L.M <= 16 ? 16 : 32);
+    splits = L.opts.split_k != 0 ? L.opts.split_k : skinny_auto_splits((L.N + 127) / 128, num_sms());
+    if (splits > kblocks)
+        splits = kblocks;
+    const int slice_kb = (kblocks + splits - 1) / splits;
+    const int64_t chunks = static_cast<int64_t>(L.M) * slice_kb * 8;
+    return chunks <= 128 * (xq == 1 ? 4 : 8) && L.M <= PGF8_FUSED_MAX_M && splits <= PGF8_FUSED_MAX_SPLITS;
+}
+
+// Whether a dynamic call with these (checked) arguments quantises inside the
+// GEMM, and with which tile width and split.
+static bool fused_quant_plan(int64_t M, int64_t N, int64_t K, pgf8_dtype xdt, const pgf8_linear_opts &o, int &bn,
+                             int &splits)
+{
+    const bool eligible = (o.flags & PGF8_FLAG_FUSED_QUANT) && M <= 32 &&
+                          (o.path == PGF8_PATH_AUTO || o.path == PGF8_PATH_SKINNY) &&
+                          (o.tile_n == 0 || ((o.tile_n == 16 || o.tile_n == 32) && o.tile_n >= M)) &&
+                          o.split_k >= 0 && o.split_k <= 8;
+    if (!eligible)
+        return false;
+    GemmLaunch P;
+    P.M = static_cast<int>(M);
+    P.N = static_cast<int>(N);
+    P.K = static_cast<int>(K);
+    P.opts = o;
+    return xq_plan(P, xdt == PGF8_F32 ? 1 : 2, bn, splits);
+}
+
+template <int KIND, int XQ> static pgf8_status launch_gemm_xq(const GemmLaunch &L, int bn, int splits)
+{
+    // the skinny kernel's stage counts (both fit two CTAs per SM)
+    if (bn == 16)
+        return launch_xq_cfg<KIND, 16, 6, XQ>(L, splits);
+    return launch_xq_cfg<KIND, 32, 5, XQ>(L, splits);
 }
 
 template <int KIND> static pgf8_status launch_gemm(const GemmLaunch &L)
@@ -389,15 +485,8 @@ template <int KIND> static pgf8_status launch_gemm(const GemmLaunch &L)
     const int sms = (splits == 0 || bn == 0) ? num_sms() : 148;
     if (path == PGF8_PATH_SKINNY) {
         const int tiles = (L.N + 127) / 128;
-        if (splits == 0) {
-            // the largest power-of-two split that keeps the grid within ~1.75
-            // CTAs per SM (measured on B200 over the 7B and 70B decode
-            // shapes: 64 weight tiles -> 4, 80-96 -> 2, >= 172 -> 1); beyond
-            // that the extra CTAs wait for a second wave
-            splits = 1;
-            while (splits < 8 && tiles * splits * 2 * 4 <= sms * 7)
-                splits *= 2;
-        }
+        if (splits == 0)
+            splits = skinny_auto_splits(tiles, sms);
         if (splits > kblocks)
             splits = kblocks;
         switch (bn) {
@@ -633,6 +722,36 @@ static pgf8_status linear_dynamic_impl(const void *x, pgf8_dtype xdt, int64_t M,
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const pgf8_linear_opts o = opts_or_default(opts);
     const int overlap = (o.flags & PGF8_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
+    int xq_bn = 0, xq_splits = 0;
+    if (fused_quant_plan(M, N, K, xdt, o, xq_bn, xq_splits)) {
+        // one kernel: the GEMM quantises the activations of its K-slice itself
+        // and writes the codes and scales to the workspace as a side output
+        GemmLaunch L;
+        L.ws = nullptr;
+        L.ws_bytes = 0;
+        L.kind = kind;
+        L.x = nullptr;
+        L.w = w;
+        L.w2 = nullptr;
+        L.sa = sa;
+        L.sw = sw;
+        L.y = y;
+        L.M = static_cast<int>(M);
+        L.N = static_cast<int>(N);
+        L.K = static_cast<int>(K);
+        L.pdl = overlap;
+        L.prefetch_w = 1;   // weights never wait for the previous kernel (see PGF8_FLAG_OVERLAP_PREVIOUS)
+        L.opts = o;
+        L.stream = cs;
+        L.xraw = x;
+        L.ldx = ldx;
+        L.q_out = aq;
+        L.sa_out = sa;
+        if (kind == kNested8)   // NestedFP activations are f16
+            return launch_gemm_xq<kNested8, 2>(L, xq_bn, xq_splits);
+        return xdt == PGF8_F32 ? launch_gemm_xq<kE4M3, 1>(L, xq_bn, xq_splits)
+                               : launch_gemm_xq<kE4M3, 2>(L, xq_bn, xq_splits);
+    }
     // the quantisation signals its dependent (this call's GEMM) at once: the
     // GEMM loads its first weight tiles while the activations are quantised
     st = quantize_launch(x, xdt, M, K, ldx, aq, sa, 0, cs, overlap, 1);
@@ -666,6 +785,34 @@ pgf8_status pgf8_fp8_linear_dynamic(const void *x, pgf8_dtype xdt, int64_t M, in
 {
     return linear_dynamic_impl(x, xdt, M, K, ldx, wq, nullptr, sw, N, y, workspace, workspace_bytes, opts, stream,
                                kE4M3);
+}
+
+pgf8_status pgf8_fp8_linear_dynamic_plan(int64_t M, int64_t N, int64_t K, pgf8_dtype xdt,
+                                         const pgf8_linear_opts *opts, int32_t *fused, int32_t *split_k)
+{
+    if (!fused || !split_k)
+        return PGF8_ERR_INVALID_ARG;
+    pgf8_status st = check_dims(M, N, K);
+    if (st != PGF8_OK)
+        return st;
+    if (xdt != PGF8_F32 && xdt != PGF8_F16)
+        return PGF8_ERR_UNSUPPORTED;
+    const pgf8_linear_opts o = opts_or_default(opts);
+    *fused = 0;
+    *split_k = 0;
+    int bn = 0, splits = 0;
+    if (fused_quant_plan(M, N, K, xdt, o, bn, splits)) {
+        *fused = 1;
+        *split_k = splits;
+        return PGF8_OK;
+    }
+    const bool skinny = (o.path == PGF8_PATH_AUTO && M <= 128) || o.path == PGF8_PATH_SKINNY;
+    if (skinny && M <= 128) {
+        const int kblocks = static_cast<int>((K + 127) / 128);
+        int sp = o.split_k != 0 ? o.split_k : skinny_auto_splits(static_cast<int>((N + 127) / 128), num_sms());
+        *split_k = sp > kblocks ? kblocks : sp;
+    }
+    return PGF8_OK;
 }
 
 pgf8_status pgf8_fp8_linear_dynamic_many(const pgf8_fp8_layer *layers, int64_t count, const pgf8_linear_opts *opts,
@@ -777,6 +924,21 @@ pgf8_status pgf8_selftest_bounded_wait(int64_t limit_ns, void *stream)
         return PGF8_ERR_INVALID_ARG;
     selftest_bounded_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<uint64_t>(limit_ns));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    return PGF8_OK;
+}
+
+pgf8_status pgf8_selftest_row_division(const float *divisors, int32_t count, unsigned long long *mismatches,
+                                       void *stream)
+{
+    if (!divisors || !mismatches || count < 1 || count > 64)
+        return PGF8_ERR_INVALID_ARG;
+    if (!aligned4(divisors) || (reinterpret_cast<uintptr_t>(mismatches) & 7u) != 0)
+        return PGF8_ERR_ALIGNMENT;
+    dim3 grid(static_cast<unsigned>(num_sms() * 8), static_cast<unsigned>(count));
+    selftest_row_division_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(divisors, count, mismatches);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return cuda_fail(e);

@@ -79,17 +79,124 @@ __device__ __forceinline__ float block_max(float v, float *red)
     return red[0];
 }
 
-// Converts 16 binary32 values (already divided by the scale) to 16 codes.
-__device__ __forceinline__ uint4 encode16(const float (&v)[16], float s)
+// x / s correctly rounded (binary32, nearest-even) for many x and one
+// divisor s — the quotient the quantisation rounds to E4M3.
+//
+// Method: Markstein's FMA division (P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
+// 1990; "Markstein's theorem" in Muller et al., Handbook of Floating-Point
+// Arithmetic).  With y = RN(1/s) (correctly rounded reciprocal, once per
+// divisor) and a = |x|:
+//   q0 = RN(a y)                 within (2u + u^2) |a/s|, u = 2^-24
+//   r0 = RN(a - s q0)            (fma)
+//   q1 = RN(q0 + r0 y)           error ~4u^2 |a/s| before rounding: faithful
+//   r1 = a - s q1                exact (fma): the remainder of a faithful
+//                                quotient is representable barring underflow
+//   q2 = RN(q1 + r1 y) = RN(a/s) by Markstein's theorem (y within half an ulp
+//                                of 1/s, q1 faithful, r1 exact)
+// and the sign of x is put back (so -0 gives -0).  The steps need no
+// overflow and no underflow of the remainders: that holds for
+// 2^-60 <= s <= 2^96 and |x / s| <= 512 (the quantisation divides values of
+// magnitude at most amax by s = RN(amax / 448)); quotients so small that
+// the remainders underflow are below 2^-11 and round to a zero code either
+// way.  Other divisors, and non-finite x, take the IEEE division itself.
+// Checked exhaustively against __fdiv_rn over all binary32 x with
+// |x| <= 512 s for a set of divisors (pgf8_selftest_row_division): equal
+// quotients wherever |x / s| >= 2^-11, equal E4M3 codes everywhere.
+struct RowDivisor {
+    float s, y;
+    bool fast;
+    RowDivisor() = default;
+    __device__ __forceinline__ explicit RowDivisor(float s_)
+    {
+        s = s_;
+        y = __frcp_rn(s_);
+        fast = s_ >= 0x1p-60f && s_ <= 0x1p96f;
+    }
+    // the FMA sequence alone (caller checked `fast` and that x is finite)
+    __device__ __forceinline__ float div_fast(float x) const
+    {
+        const float a = fabsf(x);
+        const float q0 = __fmul_rn(a, y);
+        const float r0 = __fmaf_rn(-s, q0, a);
+        const float q1 = __fmaf_rn(r0, y, q0);
+        const float r1 = __fmaf_rn(-s, q1, a);
+        const float q2 = __fmaf_rn(r1, y, q1);
+        return copysignf(q2, x);
+    }
+    __device__ __forceinline__ float div(float x) const
+    {
+        if (!fast || !isfinite(x))
+            return __fdiv_rn(x, s);
+        return div_fast(x);
+    }
+};
+
+// Converts N (8 or 16) binary32 values to N codes: E4M3(RN(v / s)),
+// saturating.  One branch for the whole group (divisor in range and every
+// value finite), so the N division chains interleave.
+template <int N>
+__device__ __forceinline__ void encode_codes(const float (&v)[N], const RowDivisor &d, uint32_t (&w)[N / 4])
 {
-    uint32_t w[4];
+    uint32_t inf_nan = 0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t lo = cvt_e4m3x2(__fdiv_rn(v[4 * i + 0], s), __fdiv_rn(v[4 * i + 1], s));
-        const uint32_t hi = cvt_e4m3x2(__fdiv_rn(v[4 * i + 2], s), __fdiv_rn(v[4 * i + 3], s));
+    for (int i = 0; i < N; ++i)
+        inf_nan |= static_cast<uint32_t>((__float_as_uint(v[i]) & 0x7F800000u) == 0x7F800000u);
+    float q[N];
+    if (d.fast && !inf_nan) {
+#pragma unroll
+        for (int i = 0; i < N; ++i)
+            q[i] = d.div_fast(v[i]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < N; ++i)
+            q[i] = d.div(v[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i) {
+        const uint32_t lo = cvt_e4m3x2(q[4 * i + 0], q[4 * i + 1]);
+        const uint32_t hi = cvt_e4m3x2(q[4 * i + 2], q[4 * i + 3]);
         w[i] = lo | (hi << 16);
     }
+}
+
+__device__ __forceinline__ uint4 encode16(const float (&v)[16], const RowDivisor &d)
+{
+    uint32_t w[4];
+    encode_codes<16>(v, d, w);
     return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Self-test of RowDivisor: for each divisor s, every finite binary32 x with
+// |x| <= 512 s (enumerated by bit pattern) is divided both ways.  Counted
+// per divisor: [2i] quotients that differ where |x| >= 2^-11 s (the
+// quotients the E4M3 rounding can tell apart), [2i+1] E4M3 codes that differ
+// anywhere in the domain.
+__global__ void __launch_bounds__(256) selftest_row_division_kernel(const float *__restrict__ divisors, int count,
+                                                                    unsigned long long *__restrict__ mismatches)
+{
+    const int di = blockIdx.y;
+    if (di >= count)
+        return;
+    const RowDivisor d(divisors[di]);
+    const float lim = 512.0f * d.s;
+    const float small = 0x1p-11f * d.s;
+    unsigned long long bad_q = 0, bad_code = 0;
+    const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+    for (uint64_t b = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < (1ull << 32); b += stride) {
+        const float x = __uint_as_float(static_cast<uint32_t>(b));
+        if (!(fabsf(x) <= lim))
+            continue;
+        const float q = d.div(x), ref = __fdiv_rn(x, d.s);
+        if (fabsf(x) >= small && __float_as_uint(q) != __float_as_uint(ref))
+            ++bad_q;
+        if (cvt_e4m3x2(q, 0.0f) != cvt_e4m3x2(ref, 0.0f))
+            ++bad_code;
+    }
+    if (bad_q)
+        atomicAdd(&mismatches[2 * di], bad_q);
+    if (bad_code)
+        atomicAdd(&mismatches[2 * di + 1], bad_code);
 }
 
 // Rows of up to kRegChunks * kQuantThreads * 16 elements stay in registers
@@ -145,11 +252,12 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(const T *_
         } else {
             s = scales[row];
         }
+        const RowDivisor d(s);
 #pragma unroll
         for (int u = 0; u < kRegChunks; ++u) {
             const int64_t c = threadIdx.x + static_cast<int64_t>(u) * kQuantThreads;
             if (c < nchunk)
-                *reinterpret_cast<uint4 *>(qr + c * 16) = encode16(v[u].v, s);
+                *reinterpret_cast<uint4 *>(qr + c * 16) = encode16(v[u].v, d);
         }
         return;
     }
@@ -173,10 +281,11 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(const T *_
     } else {
         s = scales[row];
     }
+    const RowDivisor d(s);
     for (int64_t c = threadIdx.x; c < nchunk; c += kQuantThreads) {
         Vec16<T> v;
         v.load(xr + c * 16);
-        *reinterpret_cast<uint4 *>(qr + c * 16) = encode16(v.v, s);
+        *reinterpret_cast<uint4 *>(qr + c * 16) = encode16(v.v, d);
     }
 }
 

@@ -233,6 +233,52 @@ __device__ __forceinline__ void cluster_sync_all()
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// Split phases of the cluster barrier, for threads that arrive at different
+// points of the kernel (each thread alternates arrive and wait).
+__device__ __forceinline__ void cluster_arrive_relaxed()
+{
+    asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_arrive_release()
+{
+    asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait_acquire()
+{
+    asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+// Named barrier 1 over the 128 threads of warps 2-5.
+__device__ __forceinline__ void bar_sync_warps2to5()
+{
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+// The same barrier, returning the AND of `v` over the 128 threads (so that
+// all of them take the same branch afterwards).
+__device__ __forceinline__ bool bar_and_warps2to5(bool v)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, 1, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}\n"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(v))
+        : "memory");
+    return r != 0;
+}
+
 __device__ __forceinline__ uint32_t map_shared_rank(uint32_t saddr, uint32_t rank)
 {
     uint32_t r;

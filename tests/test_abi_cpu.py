@@ -146,3 +146,27 @@ def test_dynamic_many_checks_every_layer_first():
     assert pg.lib.pgf8_fp8_linear_dynamic_many(None, 2, None, None) == pg.ERR_INVALID_ARG
     assert pg.lib.pgf8_fp8_linear_dynamic_many(None, 0, None, None) == pg.OK
     assert pg.lib.pgf8_fp8_linear_dynamic_many(arr, -1, None, None) == pg.ERR_INVALID_ARG
+
+
+def test_selftest_row_division_argument_checks():
+    f = pg.lib.pgf8_selftest_row_division
+    buf = (ctypes.c_uint64 * 4)()
+    assert f(None, 1, ctypes.addressof(buf), None) == pg.ERR_INVALID_ARG
+    assert f(ctypes.addressof(buf), 0, ctypes.addressof(buf), None) == pg.ERR_INVALID_ARG
+    assert f(ctypes.addressof(buf), 65, ctypes.addressof(buf), None) == pg.ERR_INVALID_ARG
+    assert f(ctypes.addressof(buf), 1, None, None) == pg.ERR_INVALID_ARG
+    assert f(ctypes.addressof(buf) + 1, 1, ctypes.addressof(buf), None) == pg.ERR_ALIGNMENT
+    assert f(ctypes.addressof(buf), 1, ctypes.addressof(buf) + 4, None) == pg.ERR_ALIGNMENT
+
+
+def test_dynamic_plan_is_host_only_and_follows_the_flag():
+    # decode-sized M on the skinny path: split chosen, fused only when asked for
+    fused, split = pg.fp8_linear_dynamic_plan(1, 4096, 4096, flags=pg.FLAG_FUSED_QUANT)
+    assert fused and 1 <= split <= 8
+    assert pg.fp8_linear_dynamic_plan(1, 4096, 4096) == (False, split)
+    # a slice too long for the registers (f32: 4 x 16 per thread): two-kernel form
+    assert pg.fp8_linear_dynamic_plan(8, 22016, 4096, flags=pg.FLAG_FUSED_QUANT)[0] is False
+    # prefill-sized M: tiled kernels, no split reported
+    assert pg.fp8_linear_dynamic_plan(2048, 4096, 4096, flags=pg.FLAG_FUSED_QUANT) == (False, 0)
+    with pytest.raises(pg.Pgf8Error):
+        pg.fp8_linear_dynamic_plan(1, 4096, 4000 + 8)   # K % 16 != 0
