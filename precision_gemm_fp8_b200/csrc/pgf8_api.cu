@@ -18,6 +18,10 @@
 #ifndef PGF8_SKINNY16_STAGES
 #define PGF8_SKINNY16_STAGES 6
 #endif
+// Skinny split-K grids are kept within this many CTAs per SM, times 4.
+#ifndef PGF8_SKINNY_CTAS_PER_SM_X4
+#define PGF8_SKINNY_CTAS_PER_SM_X4 7
+#endif
 // In-GEMM quantisation of dynamic activations is used up to this many tokens
 // and this many K-splits (beyond: the quantisation kernel, then the GEMM).
 #ifndef PGF8_FUSED_MAX_M
@@ -376,7 +380,7 @@ static int num_sms()
 static int skinny_auto_splits(int tiles, int sms)
 {
     int splits = 1;
-    while (splits < 8 && tiles * splits * 2 * 4 <= sms * 7)
+    while (splits < 8 && tiles * splits * 2 * 4 <= sms * PGF8_SKINNY_CTAS_PER_SM_X4)
         splits *= 2;
     return splits;
 }
