@@ -74,6 +74,13 @@ def _load():
         lib.orc_nestedfp_linear_fp16.argtypes = [u16p, i64, i64, u8p, u8p, i64, f64p]
         lib.orc_nestedfp_linear_fp16.restype = None
         lib.orc_nestedfp_linear_fp8.argtypes = [u16p, i64, i64, u8p, i64, f64p, u8p, f32p, f32p]
+        lib.orc_amax_accumulate_f32.argtypes = [f32p, i64, i64, i64, f32p]
+        lib.orc_amax_accumulate_f32.restype = ctypes.c_int
+        lib.orc_quantize_tensor_f32.argtypes = [f32p, i64, i64, i64, ctypes.c_float, u8p, f32p]
+        lib.orc_quantize_tensor_f32.restype = ctypes.c_int
+        lib.orc_delayed_step_f32.argtypes = [f32p, i64, i64, i64, u8p, f32p, ctypes.c_int32,
+                                             ctypes.POINTER(ctypes.c_int32), f32p, f32p]
+        lib.orc_delayed_step_f32.restype = ctypes.c_int
         lib.orc_nestedfp_linear_fp8.restype = ctypes.c_int
         _lib = lib
         return lib
@@ -237,3 +244,63 @@ def nestedfp_linear_fp8(x16: np.ndarray, hi: np.ndarray):
                                      _ptr(sa, ctypes.c_float), _ptr(tmp, ctypes.c_float))
     _check(st)
     return ref, aq, sa
+
+
+# ---------------------------------------------------------------- per-tensor scaling
+def _as_f32_2d(x: np.ndarray) -> np.ndarray:
+    """float32 copy of a 2-D float32 / float16 array (float16 widens exactly)."""
+    x = np.asarray(x)
+    if x.ndim != 2 or x.dtype not in (np.float32, np.float16):
+        raise ValueError("x must be a 2-D float32 or float16 array")
+    return np.ascontiguousarray(x, dtype=np.float32)
+
+
+def amax_accumulate(x: np.ndarray, amax: float = 0.0) -> float:
+    """max(amax, max |x|) — the MINMAX calibration statistic of a tensor."""
+    lib = _load()
+    x = _as_f32_2d(x)
+    a = np.array([amax], dtype=np.float32)
+    _check(lib.orc_amax_accumulate_f32(_ptr(x, ctypes.c_float), x.shape[0], x.shape[1], x.shape[1],
+                                       _ptr(a, ctypes.c_float)))
+    return float(a[0])
+
+
+def quantize_tensor(x: np.ndarray, amax: float):
+    """Static per-tensor quantisation with the scale of a calibrated amax.
+    Returns (codes uint8 [R,C], scale f32)."""
+    lib = _load()
+    x = _as_f32_2d(x)
+    q = np.empty(x.shape, dtype=np.uint8)
+    s = np.zeros(1, dtype=np.float32)
+    _check(lib.orc_quantize_tensor_f32(_ptr(x, ctypes.c_float), x.shape[0], x.shape[1], x.shape[1],
+                                       np.float32(amax), _ptr(q, ctypes.c_uint8), _ptr(s, ctypes.c_float)))
+    return q, np.float32(s[0])
+
+
+class DelayedScaling:
+    """Delayed per-tensor scaling over an amax history of length H: each
+    step quantises with the scale carried from the previous step, then
+    records its amax and carries max(history) / 448."""
+
+    def __init__(self, history_len: int, initial_scale: float = 1.0):
+        if history_len < 1:
+            raise ValueError("history_len must be >= 1")
+        self.history = np.zeros(history_len, dtype=np.float32)
+        self.pos = 0
+        self.scale = np.float32(initial_scale)
+
+    def step(self, x: np.ndarray):
+        """Returns (codes uint8 [R,C], the scale they were made with)."""
+        lib = _load()
+        x = _as_f32_2d(x)
+        q = np.empty(x.shape, dtype=np.uint8)
+        pos = ctypes.c_int32(self.pos)
+        sc = np.array([self.scale], dtype=np.float32)
+        used = np.zeros(1, dtype=np.float32)
+        _check(lib.orc_delayed_step_f32(_ptr(x, ctypes.c_float), x.shape[0], x.shape[1], x.shape[1],
+                                        _ptr(q, ctypes.c_uint8), _ptr(self.history, ctypes.c_float),
+                                        len(self.history), ctypes.byref(pos), _ptr(sc, ctypes.c_float),
+                                        _ptr(used, ctypes.c_float)))
+        self.pos = pos.value
+        self.scale = np.float32(sc[0])
+        return q, np.float32(used[0])

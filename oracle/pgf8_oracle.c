@@ -317,3 +317,99 @@ int orc_nestedfp_linear_fp8(const uint16_t *x, int64_t M, int64_t K,
         }
     return ORC_OK;
 }
+
+/* ------------------------------------------------------------------ */
+/* Per-tensor scaling variants.                                        */
+/*                                                                     */
+/* [CPP-FP8] §5.1 names MINMAX calibration (the scale follows the      */
+/* largest magnitude seen over representative calibration data);       */
+/* [FP8-4060] §6.1 asks for an amax history of length >= 1024 and a    */
+/* scale below 448.  Readings (the pages give no formulas):            */
+/*   amax of a tensor   = max |x| over all its elements (exact);       */
+/*   per-tensor scale   s = fl32(amax / 448), 1 when that is 0 (as the */
+/*                      per-row rule);                                 */
+/*   delayed scaling    step t quantises with the scale carried in     */
+/*                      from step t-1; then history[pos] = amax(x_t),  */
+/*                      pos = (pos + 1) mod H, and the carried scale   */
+/*                      becomes fl32(max(history) / 448) (1 when 0).   */
+/* Values above 448 s saturate to the largest finite code (satfinite). */
+/* Non-finite inputs are an error here (the pages define no result).   */
+/* ------------------------------------------------------------------ */
+
+/* *amax = max(*amax, max |x|) over a rows x cols block (row stride ldx). */
+int orc_amax_accumulate_f32(const float *x, int64_t rows, int64_t cols, int64_t ldx, float *amax)
+{
+    if (rows < 0 || cols < 0 || ldx < cols || !amax || !(*amax >= 0.0f))
+        return ORC_ERR_ARG;
+    float m = *amax;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t k = 0; k < cols; ++k) {
+            float a = fabsf(x[r * ldx + k]);
+            if (!isfinite(a))
+                return ORC_ERR_NONFINITE;
+            if (a > m)
+                m = a;
+        }
+    }
+    *amax = m;
+    return ORC_OK;
+}
+
+/* The per-tensor scale of an amax (reading above). */
+static float scale_of_amax(float amax)
+{
+    float s = amax / 448.0f;
+    if (s == 0.0f)
+        s = 1.0f;
+    return s;
+}
+
+/* Static per-tensor quantisation with the scale of a calibrated amax:
+ * every row uses s = scale_of_amax(amax); s is written to *s_out. */
+int orc_quantize_tensor_f32(const float *x, int64_t rows, int64_t cols, int64_t ldx, float amax, uint8_t *q,
+                            float *s_out)
+{
+    if (rows < 0 || cols < 0 || ldx < cols || !(amax >= 0.0f) || !isfinite(amax))
+        return ORC_ERR_ARG;
+    float s = scale_of_amax(amax);
+    for (int64_t r = 0; r < rows; ++r) {
+        float sr = s;
+        int st = quantize_one_row(x + r * ldx, cols, q + r * cols, &sr, 1);
+        if (st != ORC_OK)
+            return st;
+    }
+    *s_out = s;
+    return ORC_OK;
+}
+
+/* One step of delayed scaling (reading above).  history: H >= 1 amaxes,
+ * *pos in [0, H), *scale the carried scale (> 0, finite).  q receives the
+ * codes of this step; *step_scale the scale they were made with. */
+int orc_delayed_step_f32(const float *x, int64_t rows, int64_t cols, int64_t ldx, uint8_t *q, float *history,
+                         int32_t H, int32_t *pos, float *scale, float *step_scale)
+{
+    if (rows < 0 || cols < 0 || ldx < cols || H < 1 || !pos || *pos < 0 || *pos >= H || !scale)
+        return ORC_ERR_ARG;
+    float s = *scale;
+    if (!(s > 0.0f) || !isfinite(s))
+        return ORC_ERR_BADSCALE;
+    for (int64_t r = 0; r < rows; ++r) {
+        float sr = s;
+        int st = quantize_one_row(x + r * ldx, cols, q + r * cols, &sr, 1);
+        if (st != ORC_OK)
+            return st;
+    }
+    float a = 0.0f;
+    int st = orc_amax_accumulate_f32(x, rows, cols, ldx, &a);
+    if (st != ORC_OK)
+        return st;
+    *step_scale = s;
+    history[*pos] = a;
+    *pos = (*pos + 1) % H;
+    float hmax = 0.0f;
+    for (int32_t i = 0; i < H; ++i)
+        if (history[i] > hmax)
+            hmax = history[i];
+    *scale = scale_of_amax(hmax);
+    return ORC_OK;
+}
