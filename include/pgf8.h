@@ -162,6 +162,49 @@ pgf8_status pgf8_fp8_linear_ex(const uint8_t *aq, const float *sa, int64_t M, in
 size_t pgf8_fp8_linear_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /* ------------------------------------------------------------------------
+ * Per-tensor activation scaling ("C++ and FP8" §5.1: MINMAX calibration,
+ * the scale follows the largest magnitude seen over calibration data;
+ * "7B on an RTX 4060 with FP8" §6.1: delayed scaling over an amax history
+ * of length >= 1024, scale below 448).  Readings: amax = max |x| over the
+ * tensor (NaN ignored); scale = RN(amax / 448) in binary32, 1 when 0; codes
+ * = E4M3(RN(x / scale)), saturating.  The codes and per-row scales feed
+ * pgf8_fp8_linear as they are (every row carries the tensor's scale).
+ * x [rows, cols] f32 or f16, row stride ldx; q [rows, cols] contiguous;
+ * alignment as for pgf8_fp8_quantize_rows; rows == 0 does nothing.
+ *
+ * pgf8_fp8_amax_accumulate: *amax = max(*amax, amax(x)) (device scalar,
+ *   start from +0.0; calibration over several batches accumulates).
+ * pgf8_fp8_quantize_tensor: static per-tensor quantisation with the scale
+ *   of a calibrated amax (device scalar); scales [rows] (may be NULL)
+ *   receives that scale.
+ * pgf8_delayed_state_init: history [history_len] (device) zeroed, the
+ *   state (device, 16-byte aligned) set to quantise its first step with
+ *   initial_scale (> 0).  history_len 1..2^24 (the pages ask >= 1024).
+ * pgf8_fp8_quantize_delayed: one step: quantises x with the state's
+ *   carried scale (written to scales [rows] if not NULL), then records
+ *   amax(x) in history at the state's slot, advances the slot (mod
+ *   history_len) and carries RN(max(history) / 448) (1 when 0) to the next
+ *   step.  One kernel; the state is updated by the last CTA to finish, so
+ *   steps on one state must be stream-ordered (one stream, or events).
+ * ---------------------------------------------------------------------- */
+typedef struct {
+    float scale;          /* the scale the next step quantises with */
+    uint32_t amax_bits;   /* internal: running amax of a step in flight */
+    int32_t pos;          /* next history slot */
+    uint32_t done;        /* internal: CTAs of a step in flight that finished */
+} pgf8_delayed_state;
+
+pgf8_status pgf8_fp8_amax_accumulate(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
+                                     float *amax, void *stream);
+pgf8_status pgf8_fp8_quantize_tensor(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
+                                     const float *amax, uint8_t *q, float *scales, void *stream);
+pgf8_status pgf8_delayed_state_init(pgf8_delayed_state *state, float *history, int32_t history_len,
+                                    float initial_scale, void *stream);
+pgf8_status pgf8_fp8_quantize_delayed(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
+                                      uint8_t *q, float *scales, float *history, int32_t history_len,
+                                      pgf8_delayed_state *state, void *stream);
+
+/* ------------------------------------------------------------------------
  * Dynamic-activation FP8 linear: per-token quantisation of x (as
  * pgf8_fp8_quantize_rows, DYNAMIC) followed by pgf8_fp8_linear, enqueued as
  * one dependent pair so the GEMM's set-up and first weight loads overlap the

@@ -56,6 +56,10 @@ _optp = ctypes.POINTER(LinearOpts)
 
 _SIGS = {
     "pgf8_fp8_quantize_rows": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _i32, _vp], _i32),
+    "pgf8_fp8_amax_accumulate": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp], _i32),
+    "pgf8_fp8_quantize_tensor": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _vp], _i32),
+    "pgf8_delayed_state_init": ([_vp, _vp, _i32, ctypes.c_float, _vp], _i32),
+    "pgf8_fp8_quantize_delayed": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _i32, _vp, _vp], _i32),
     "pgf8_fp8_linear": ([_vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _sz, _vp], _i32),
     "pgf8_fp8_linear_ex": ([_vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _sz, _optp, _vp], _i32),
     "pgf8_fp8_linear_workspace_size": ([_i64, _i64, _i64], _sz),
@@ -177,6 +181,70 @@ def fp8_quantize_rows(x: torch.Tensor, q: torch.Tensor | None = None, scales: to
     _check(lib.pgf8_fp8_quantize_rows(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(q), _ptr(scales),
                                       mode, _stream(stream)), "fp8_quantize_rows")
     return q, scales
+
+
+def fp8_amax_accumulate(x: torch.Tensor, amax: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """amax = max(amax, max |x|) as a device float32 [1] tensor (a new zero
+    one when not given): the MINMAX calibration statistic, accumulated over
+    calibration batches."""
+    rows, cols = x.shape
+    if x.stride(1) != 1:
+        raise ValueError("x rows must be contiguous")
+    if amax is None:
+        amax = torch.zeros(1, dtype=torch.float32, device=x.device)
+    _check(lib.pgf8_fp8_amax_accumulate(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(amax),
+                                        _stream(stream)), "fp8_amax_accumulate")
+    return amax
+
+
+def fp8_quantize_tensor(x: torch.Tensor, amax: torch.Tensor, q: torch.Tensor | None = None,
+                        scales: torch.Tensor | None = None, stream=None):
+    """Static per-tensor quantisation with the scale of a calibrated amax
+    (device float32 [1]).  Returns (q uint8 [rows, cols], scales f32 [rows],
+    every row holding the tensor's scale)."""
+    rows, cols = x.shape
+    if x.stride(1) != 1:
+        raise ValueError("x rows must be contiguous")
+    if q is None:
+        q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(rows, dtype=torch.float32, device=x.device)
+    _check(lib.pgf8_fp8_quantize_tensor(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(amax), _ptr(q),
+                                        _ptr(scales), _stream(stream)), "fp8_quantize_tensor")
+    return q, scales
+
+
+class DelayedScaling:
+    """Delayed per-tensor scaling of one activation tensor: a device amax
+    history of ``history_len`` entries and the carried scale.  Each
+    ``step(x)`` quantises x with the carried scale, records amax(x) and
+    carries RN(max(history) / 448) to the next step (one kernel)."""
+
+    def __init__(self, history_len: int = 1024, initial_scale: float = 1.0, device="cuda", stream=None):
+        self.history_len = int(history_len)
+        self.history = torch.empty(self.history_len, dtype=torch.float32, device=device)
+        self.state = torch.empty(4, dtype=torch.int32, device=device)   # pgf8_delayed_state, 16 bytes
+        _check(lib.pgf8_delayed_state_init(_ptr(self.state), _ptr(self.history), self.history_len,
+                                           float(initial_scale), _stream(stream)), "delayed_state_init")
+
+    def step(self, x: torch.Tensor, q: torch.Tensor | None = None, scales: torch.Tensor | None = None, stream=None):
+        """Returns (q uint8 [rows, cols], scales f32 [rows]: the step's scale)."""
+        rows, cols = x.shape
+        if x.stride(1) != 1:
+            raise ValueError("x rows must be contiguous")
+        if q is None:
+            q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+        if scales is None:
+            scales = torch.empty(rows, dtype=torch.float32, device=x.device)
+        _check(lib.pgf8_fp8_quantize_delayed(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(q),
+                                             _ptr(scales), _ptr(self.history), self.history_len, _ptr(self.state),
+                                             _stream(stream)), "fp8_quantize_delayed")
+        return q, scales
+
+    def carried(self):
+        """(carried scale, next history slot), read back (synchronises)."""
+        st = self.state.cpu()
+        return float(st[0:1].view(torch.float32).item()), int(st[2].item())
 
 
 def fp8_linear(aq, sa, wq, sw, y=None, workspace=None, path=PATH_AUTO, split_k=0, tile_n=0, flags=0,

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cmath>
 #include <cstring>
 #include <mutex>
 
@@ -606,11 +607,121 @@ static pgf8_status check_quantize_args(const void *x, pgf8_dtype xdt, int64_t ro
     return PGF8_OK;
 }
 
+// Checks of the per-tensor scaling calls: x and (when given) q as for the
+// per-row quantisation; scales may be null.
+static pgf8_status check_tensor_args(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
+                                     const uint8_t *q, bool need_q, const float *scales)
+{
+    if (rows < 0 || cols < 16 || ldx < cols || rows > (1ll << 31) - 1)
+        return PGF8_ERR_INVALID_ARG;
+    if (rows == 0)
+        return PGF8_OK;
+    if (!x || (need_q && !q))
+        return PGF8_ERR_INVALID_ARG;
+    if (xdt != PGF8_F32 && xdt != PGF8_F16)
+        return PGF8_ERR_UNSUPPORTED;
+    const int eb = xdt == PGF8_F32 ? 4 : 2;
+    if (cols % 16 != 0 || (ldx * eb) % 16 != 0 || !aligned16(x) || (q && !aligned16(q)) ||
+        (scales && !aligned4(scales)))
+        return PGF8_ERR_ALIGNMENT;
+    return PGF8_OK;
+}
+
+template <typename T, typename... Args>
+static pgf8_status launch_simple(void (*kernel)(Args...), unsigned grid, cudaStream_t st, Args... args)
+{
+    kernel<<<grid, kQuantThreads, 0, st>>>(args...);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? PGF8_OK : cuda_fail(e);
+}
+
 } // namespace pgf8
 
 using namespace pgf8;
 
 extern "C" {
+
+pgf8_status pgf8_fp8_amax_accumulate(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
+                                     float *amax, void *stream)
+{
+    pgf8_status st = check_tensor_args(x, xdt, rows, cols, ldx, nullptr, false, nullptr);
+    if (st != PGF8_OK)
+        return st;
+    if (!amax)
+        return PGF8_ERR_INVALID_ARG;
+    if (!aligned4(amax))
+        return PGF8_ERR_ALIGNMENT;
+    if (rows == 0)
+        return PGF8_OK;
+    const int64_t chunks = rows * (cols / 16);
+    const int64_t want = (chunks + kQuantThreads - 1) / kQuantThreads;
+    const unsigned grid = static_cast<unsigned>(want < num_sms() * 4 ? want : num_sms() * 4);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    unsigned *bits = reinterpret_cast<unsigned *>(amax);
+    if (xdt == PGF8_F32)
+        return launch_simple<float>(amax_accumulate_kernel<float>, grid, cs, static_cast<const float *>(x), rows,
+                                    cols, ldx, bits);
+    return launch_simple<__half>(amax_accumulate_kernel<__half>, grid, cs, static_cast<const __half *>(x), rows, cols,
+                                 ldx, bits);
+}
+
+pgf8_status pgf8_fp8_quantize_tensor(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
+                                     const float *amax, uint8_t *q, float *scales, void *stream)
+{
+    pgf8_status st = check_tensor_args(x, xdt, rows, cols, ldx, q, true, scales);
+    if (st != PGF8_OK)
+        return st;
+    if (rows == 0)
+        return PGF8_OK;
+    if (!amax)
+        return PGF8_ERR_INVALID_ARG;
+    if (!aligned4(amax))
+        return PGF8_ERR_ALIGNMENT;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const unsigned grid = static_cast<unsigned>(rows);
+    if (xdt == PGF8_F32)
+        return launch_simple<float>(quantize_tensor_kernel<float>, grid, cs, static_cast<const float *>(x), cols, ldx,
+                                    amax, q, scales);
+    return launch_simple<__half>(quantize_tensor_kernel<__half>, grid, cs, static_cast<const __half *>(x), cols, ldx,
+                                 amax, q, scales);
+}
+
+pgf8_status pgf8_delayed_state_init(pgf8_delayed_state *state, float *history, int32_t history_len,
+                                    float initial_scale, void *stream)
+{
+    if (!state || !history || history_len < 1 || history_len > (1 << 24) || !(initial_scale > 0.0f) ||
+        !std::isfinite(initial_scale))
+        return PGF8_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(state) & 15u) != 0 || !aligned4(history))
+        return PGF8_ERR_ALIGNMENT;
+    const unsigned grid = static_cast<unsigned>((history_len + kQuantThreads - 1) / kQuantThreads);
+    return launch_simple<float>(delayed_init_kernel, grid < 1024u ? grid : 1024u, static_cast<cudaStream_t>(stream),
+                                history, static_cast<int>(history_len), reinterpret_cast<DelayedState *>(state),
+                                initial_scale);
+}
+
+pgf8_status pgf8_fp8_quantize_delayed(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
+                                      uint8_t *q, float *scales, float *history, int32_t history_len,
+                                      pgf8_delayed_state *state, void *stream)
+{
+    pgf8_status st = check_tensor_args(x, xdt, rows, cols, ldx, q, true, scales);
+    if (st != PGF8_OK)
+        return st;
+    if (!state || !history || history_len < 1 || history_len > (1 << 24))
+        return PGF8_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(state) & 15u) != 0 || !aligned4(history))
+        return PGF8_ERR_ALIGNMENT;
+    if (rows == 0)
+        return PGF8_OK;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const unsigned grid = static_cast<unsigned>(rows);
+    DelayedState *ds = reinterpret_cast<DelayedState *>(state);
+    if (xdt == PGF8_F32)
+        return launch_simple<float>(quantize_delayed_kernel<float>, grid, cs, static_cast<const float *>(x), cols,
+                                    ldx, q, scales, history, static_cast<int>(history_len), ds);
+    return launch_simple<__half>(quantize_delayed_kernel<__half>, grid, cs, static_cast<const __half *>(x), cols, ldx,
+                                 q, scales, history, static_cast<int>(history_len), ds);
+}
 
 pgf8_status pgf8_fp8_quantize_rows(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
                                    uint8_t *q, float *scales, pgf8_scale_mode mode, void *stream)

@@ -289,6 +289,147 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(const T *_
     }
 }
 
+// ------------------------------------------------------------------ per-tensor scaling
+// "C++ and FP8" §5.1 (MINMAX calibration: the scale follows the largest
+// magnitude over calibration data) and "7B on an RTX 4060 with FP8" §6.1
+// (delayed scaling over an amax history of length >= 1024, scale below
+// 448).  amax = max |x| over the tensor (NaN ignored, as the per-row
+// quantisation); scale = RN(amax / 448), 1 when 0.  A delayed step
+// quantises with the scale carried from the previous step, then records its
+// amax in a ring of H and carries RN(max(history) / 448).
+
+// Device layout of pgf8_delayed_state (16 bytes).
+struct DelayedState {
+    float scale;          // the scale the next step quantises with
+    unsigned amax_bits;   // running amax of the step in flight (bits of a non-negative float)
+    int pos;              // next history slot
+    unsigned done;        // CTAs of the step in flight that have finished
+};
+
+__device__ __forceinline__ float per_tensor_scale(float amax)
+{
+    const float s = __fdiv_rn(amax, 448.0f);
+    return s == 0.0f ? 1.0f : s;
+}
+
+// *amax = max(*amax, max |x|): grid-stride over 16-element chunks, warp max,
+// one atomic max per warp on the bits (non-negative floats, +0 start).
+template <typename T>
+__global__ void __launch_bounds__(kQuantThreads) amax_accumulate_kernel(const T *__restrict__ x, int64_t rows,
+                                                                        int64_t cols, int64_t ldx,
+                                                                        unsigned *__restrict__ amax_bits)
+{
+    const int64_t nch = cols / 16, total = rows * nch;
+    float m = 0.0f;
+    for (int64_t c = blockIdx.x * static_cast<int64_t>(kQuantThreads) + threadIdx.x; c < total;
+         c += static_cast<int64_t>(gridDim.x) * kQuantThreads) {
+        const int64_t r = c / nch, k = (c - r * nch) * 16;
+        Vec16<T> v;
+        v.load(x + r * ldx + k);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            m = fmaxf(m, fabsf(v.v[i]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0 && m > 0.0f)
+        atomicMax(amax_bits, __float_as_uint(m));
+}
+
+// Quantises one row with a given per-tensor scale; returns the row's amax
+// (block-wide, valid in every thread).
+template <typename T>
+__device__ __forceinline__ float quantize_row_with_scale(const T *xr, int64_t cols, uint8_t *qr, float s, float *red)
+{
+    const RowDivisor d(s);
+    float m = 0.0f;
+    for (int64_t c = threadIdx.x; c < cols / 16; c += kQuantThreads) {
+        Vec16<T> v;
+        v.load(xr + c * 16);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            m = fmaxf(m, fabsf(v.v[i]));
+        *reinterpret_cast<uint4 *>(qr + c * 16) = encode16(v.v, d);
+    }
+    return block_max(m, red);
+}
+
+// Static per-tensor quantisation with the scale of a calibrated amax; one
+// CTA per row.
+template <typename T>
+__global__ void __launch_bounds__(kQuantThreads) quantize_tensor_kernel(const T *__restrict__ x, int64_t cols,
+                                                                        int64_t ldx, const float *__restrict__ amax,
+                                                                        uint8_t *__restrict__ q,
+                                                                        float *__restrict__ scales)
+{
+    __shared__ float red[kQuantThreads / 32];
+    const int64_t row = blockIdx.x;
+    const float s = per_tensor_scale(*amax);
+    (void)quantize_row_with_scale(x + row * ldx, cols, q + row * cols, s, red);
+    if (scales && threadIdx.x == 0)
+        scales[row] = s;
+}
+
+// One delayed-scaling step; one CTA per row.  Every CTA quantises with the
+// carried scale (read before it signs off), folds its row amax into the
+// state, and signs off on a counter after a fence; the CTA that signs off
+// last records the step's amax in the history, carries the new scale and
+// resets the counters for the next step.  No CTA waits for another.
+template <typename T>
+__global__ void __launch_bounds__(kQuantThreads) quantize_delayed_kernel(const T *__restrict__ x, int64_t cols,
+                                                                         int64_t ldx, uint8_t *__restrict__ q,
+                                                                         float *__restrict__ scales,
+                                                                         float *__restrict__ history, int H,
+                                                                         DelayedState *st)
+{
+    __shared__ float red[kQuantThreads / 32];
+    __shared__ int last;
+    const int64_t row = blockIdx.x;
+    const float s = st->scale;
+    const float m = quantize_row_with_scale(x + row * ldx, cols, q + row * cols, s, red);
+    if (threadIdx.x == 0) {
+        if (scales)
+            scales[row] = s;
+        if (m > 0.0f)
+            atomicMax(&st->amax_bits, __float_as_uint(m));
+        __threadfence();
+        last = atomicAdd(&st->done, 1u) == gridDim.x - 1;
+    }
+    __syncthreads();
+    if (!last)
+        return;
+    __threadfence();
+    const float amax = __uint_as_float(atomicAdd(&st->amax_bits, 0u));
+    const int pos = st->pos;
+    float hm = 0.0f;
+    for (int i = threadIdx.x; i < H; i += kQuantThreads)
+        hm = fmaxf(hm, i == pos ? amax : history[i]);
+    hm = block_max(hm, red);
+    if (threadIdx.x == 0) {
+        history[pos] = amax;
+        st->pos = pos + 1 == H ? 0 : pos + 1;
+        st->scale = per_tensor_scale(hm);
+        st->amax_bits = 0u;
+        st->done = 0u;
+    }
+}
+
+// Fresh delayed-scaling state: history zero, first step at slot 0 with the
+// given scale.
+__global__ void __launch_bounds__(kQuantThreads) delayed_init_kernel(float *__restrict__ history, int H,
+                                                                     DelayedState *st, float initial_scale)
+{
+    for (int i = blockIdx.x * kQuantThreads + threadIdx.x; i < H; i += gridDim.x * kQuantThreads)
+        history[i] = 0.0f;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        st->scale = initial_scale;
+        st->amax_bits = 0u;
+        st->pos = 0;
+        st->done = 0u;
+    }
+}
+
 // NestedFP split: 8 FP16 bit patterns per thread per step (16 bytes in, 8 + 8 out).
 __global__ void __launch_bounds__(256) nestedfp_split_kernel(const uint4 *__restrict__ w, int64_t n8,
                                                              uint2 *__restrict__ hi, uint2 *__restrict__ lo)

@@ -170,3 +170,29 @@ def test_dynamic_plan_is_host_only_and_follows_the_flag():
     assert pg.fp8_linear_dynamic_plan(2048, 4096, 4096, flags=pg.FLAG_FUSED_QUANT) == (False, 0)
     with pytest.raises(pg.Pgf8Error):
         pg.fp8_linear_dynamic_plan(1, 4096, 4000 + 8)   # K % 16 != 0
+
+
+def test_per_tensor_scaling_argument_checks():
+    buf = (ctypes.c_uint8 * 4096)()
+    a = ctypes.addressof(buf)
+    a16 = (a + 15) // 16 * 16
+    amax = pg.lib.pgf8_fp8_amax_accumulate
+    assert amax(a16, pg.F32, 0, 16, 16, a16, None) == pg.OK            # empty: nothing enqueued
+    assert amax(a16, pg.F32, 2, 15, 16, a16, None) == pg.ERR_INVALID_ARG
+    assert amax(a16, pg.F32, 2, 16, 16, None, None) == pg.ERR_INVALID_ARG
+    assert amax(a16 + 4, pg.F32, 2, 16, 16, a16, None) == pg.ERR_ALIGNMENT
+    assert amax(a16, pg.BF16, 2, 16, 16, a16, None) == pg.ERR_UNSUPPORTED
+    qt = pg.lib.pgf8_fp8_quantize_tensor
+    assert qt(a16, pg.F32, 2, 16, 16, a16, None, None, None) == pg.ERR_INVALID_ARG      # no q
+    assert qt(a16, pg.F32, 2, 16, 16, None, a16, None, None) == pg.ERR_INVALID_ARG      # no amax
+    assert qt(a16, pg.F32, 2, 16, 16, a16, a16 + 8, None, None) == pg.ERR_ALIGNMENT
+    init = pg.lib.pgf8_delayed_state_init
+    assert init(a16, a16, 0, 1.0, None) == pg.ERR_INVALID_ARG
+    assert init(a16, a16, 1024, 0.0, None) == pg.ERR_INVALID_ARG
+    assert init(a16, a16, 1024, float("inf"), None) == pg.ERR_INVALID_ARG
+    assert init(a16 + 4, a16, 1024, 1.0, None) == pg.ERR_ALIGNMENT
+    qd = pg.lib.pgf8_fp8_quantize_delayed
+    assert qd(a16, pg.F32, 2, 16, 16, a16, None, a16, 0, a16, None) == pg.ERR_INVALID_ARG
+    assert qd(a16, pg.F32, 2, 16, 16, a16, None, a16, 1024, None, None) == pg.ERR_INVALID_ARG
+    assert qd(a16, pg.F32, 2, 16, 16, a16, None, a16, 1024, a16 + 8, None) == pg.ERR_ALIGNMENT
+    assert qd(a16, pg.F32, 0, 16, 16, a16, None, a16, 1024, a16, None) == pg.OK          # empty step
