@@ -275,6 +275,26 @@ def run_ours(args, rank, world, local_rank):
     xflags = pg.FLAG_FUSED_QUANT if args.fused_quant else 0
     sk_ws = torch.zeros(max(16, max(pg.lib.pgf8_fp8_linear_workspace_size(L.M, L.N, L.K) for L in layers)),
                         dtype=torch.uint8, device=dev)
+    # per-tensor activation scaling instead of per-token dynamic (--scaling):
+    # one delayed-scaling history or one calibrated amax per layer
+    per_tensor = {}
+    if args.scaling != "dynamic":
+        for i, L in enumerate(layers):
+            if L.kind != "fp8":
+                continue
+            if args.scaling == "delayed":
+                per_tensor[i] = pg.DelayedScaling(1024, device=dev)
+            else:
+                per_tensor[i] = pg.fp8_amax_accumulate(acts[i])   # MINMAX calibration on the layer's input
+        torch.cuda.synchronize()
+
+    def quantise_per_tensor(i, L, flags=0):
+        aq, sa = pg.dynamic_workspace_views(qbufs[i], L.M, L.K)
+        if args.scaling == "delayed":
+            per_tensor[i].step(acts[i], aq, sa, flags=flags, stream=stream)
+        else:
+            pg.fp8_quantize_tensor(acts[i], per_tensor[i], aq, sa, flags=flags, stream=stream)
+        return aq, sa
 
     def enqueue_step(ev_pairs=None):
         """One step through the C ABI on `stream`.
@@ -288,13 +308,21 @@ def run_ours(args, rank, world, local_rank):
         for i, L in enumerate(layers):
             W = weights[(L.shape_idx, L.copy, L.kind != "fp8")]
             if L.kind == "fp8":
-                if ev_pairs is None:
+                if ev_pairs is None and not per_tensor:
                     pg.fp8_linear_dynamic(acts[i], W[0], W[1], y=outs[i], workspace=qbufs[i],
                                           flags=pg.FLAG_OVERLAP_PREVIOUS | xflags, stream=stream)
                     continue
-                aq, sa = pg.dynamic_workspace_views(qbufs[i], L.M, L.K)
+                if ev_pairs is None:
+                    aq, sa = quantise_per_tensor(i, L, pg.FLAG_OVERLAP_PREVIOUS)
+                    pg.fp8_linear(aq, sa, W[0], W[1], y=outs[i], workspace=sk_ws, flags=pg.FLAG_OVERLAP_PREVIOUS,
+                                  stream=stream)
+                    continue
                 ev_pairs[i][2].record(stream)
-                pg.fp8_quantize_rows(acts[i], aq, sa, stream=stream)
+                if per_tensor:
+                    aq, sa = quantise_per_tensor(i, L)
+                else:
+                    aq, sa = pg.dynamic_workspace_views(qbufs[i], L.M, L.K)
+                    pg.fp8_quantize_rows(acts[i], aq, sa, stream=stream)
                 ev_pairs[i][0].record(stream)
                 pg.fp8_linear(aq, sa, W[0], W[1], y=outs[i], workspace=sk_ws, stream=stream)
                 ev_pairs[i][1].record(stream)
@@ -429,7 +457,10 @@ def run_ours(args, rank, world, local_rank):
                              "replayed K/R times, R=%d" % R,
                    "quantisation": "inside the skinny GEMM where each CTA's activation slice fits its "
                                    "registers, else its own kernel" if args.fused_quant
-                   else "own kernel before each GEMM"},
+                   else "own kernel before each GEMM",
+                   "activation_scaling": {"dynamic": "per token, dynamic",
+                                          "delayed": "per tensor, delayed (amax history of 1024 per layer)",
+                                          "static": "per tensor, MINMAX-calibrated amax"}[args.scaling]},
         "secondary": {"tflops": round(tflops, 3), "weight_gbs": round(gbs, 1)},
         "roofline": roof,
         "e2e": e2e,
@@ -474,7 +505,13 @@ def run_e2e(pg, torch, dev, layers, weights, acts_host, outs, args, world, wbyte
                                   dtype=torch.uint8, device=dev))
     all_fp8 = all(L.kind == "fp8" for L in layers)
     seq = None
-    if all_fp8:
+    per_tensor = {}
+    if all_fp8 and args.scaling != "dynamic":
+        for i, L in enumerate(layers):
+            per_tensor[i] = (pg.DelayedScaling(1024, device=dev) if args.scaling == "delayed"
+                             else pg.fp8_amax_accumulate(x_views[i].copy_(acts_host[i].to(dev))))
+        torch.cuda.synchronize()
+    elif all_fp8:
         seq = pg.LayerSequence([(x_views[i], weights[(L.shape_idx, L.copy, False)][0],
                                  weights[(L.shape_idx, L.copy, False)][1], y_views[i], ws[i])
                                 for i, L in enumerate(layers)])
@@ -484,6 +521,17 @@ def run_e2e(pg, torch, dev, layers, weights, acts_host, outs, args, world, wbyte
             x_dev.copy_(x_host, non_blocking=True)
             if seq is not None:
                 seq.run(flags=pg.FLAG_FUSED_QUANT if args.fused_quant else 0, stream=stream)
+            elif per_tensor:
+                for i, L in enumerate(layers):
+                    W = weights[(L.shape_idx, L.copy, False)]
+                    aq, sa = pg.dynamic_workspace_views(ws[i], L.M, L.K)
+                    fl = pg.FLAG_OVERLAP_PREVIOUS if i else 0
+                    if args.scaling == "delayed":
+                        per_tensor[i].step(x_views[i], aq, sa, flags=fl, stream=stream)
+                    else:
+                        pg.fp8_quantize_tensor(x_views[i], per_tensor[i], aq, sa, flags=fl, stream=stream)
+                    pg.fp8_linear(aq, sa, W[0], W[1], y=y_views[i], workspace=ws[i],
+                                  flags=pg.FLAG_OVERLAP_PREVIOUS, stream=stream)
             else:
                 for i, L in enumerate(layers):
                     W = weights[(L.shape_idx, L.copy, True)]
@@ -514,7 +562,10 @@ def run_e2e(pg, torch, dev, layers, weights, acts_host, outs, args, world, wbyte
     return {"value": round(v, 2), "unit": "GB/s" if memory_bound else "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(ms, 5),
-            "entry_point": "pgf8_fp8_linear_dynamic_many" if all_fp8 else "pgf8_nestedfp_linear"}
+            "entry_point": ("pgf8_nestedfp_linear" if not all_fp8 else "pgf8_fp8_linear_dynamic_many"
+                            if args.scaling == "dynamic" else
+                            {"delayed": "pgf8_fp8_quantize_delayed", "static": "pgf8_fp8_quantize_tensor"}[args.scaling]
+                            + " + pgf8_fp8_linear per layer")}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -645,6 +696,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(synthetic.WORKLOADS), default="decode7b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--scaling", choices=["dynamic", "delayed", "static"], default="dynamic",
+                    help="activation scales of the FP8 layers: per-token dynamic (default), per-tensor delayed "
+                         "(amax history of 1024) or per-tensor static (MINMAX-calibrated)")
     ap.add_argument("--fused-quant", action="store_true",
                     help="quantise dynamic activations inside the skinny GEMM where its kernel allows it")
     ap.add_argument("--single", default=None, help="kind,M,K,N: time (or profile) one layer eagerly")

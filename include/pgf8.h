@@ -170,7 +170,8 @@ size_t pgf8_fp8_linear_workspace_size(int64_t M, int64_t N, int64_t K);
  * = E4M3(RN(x / scale)), saturating.  The codes and per-row scales feed
  * pgf8_fp8_linear as they are (every row carries the tensor's scale).
  * x [rows, cols] f32 or f16, row stride ldx; q [rows, cols] contiguous;
- * alignment as for pgf8_fp8_quantize_rows; rows == 0 does nothing.
+ * alignment as for pgf8_fp8_quantize_rows; rows == 0 does nothing (except
+ * for a delayed step, which needs at least one row).
  *
  * pgf8_fp8_amax_accumulate: *amax = max(*amax, amax(x)) (device scalar,
  *   start from +0.0; calibration over several batches accumulates).
@@ -178,31 +179,38 @@ size_t pgf8_fp8_linear_workspace_size(int64_t M, int64_t N, int64_t K);
  *   of a calibrated amax (device scalar); scales [rows] (may be NULL)
  *   receives that scale.
  * pgf8_delayed_state_init: history [history_len] (device) zeroed, the
- *   state (device, 16-byte aligned) set to quantise its first step with
+ *   state (device, 16-byte aligned) set to quantise step 0 with
  *   initial_scale (> 0).  history_len 1..2^24 (the pages ask >= 1024).
- * pgf8_fp8_quantize_delayed: one step: quantises x with the state's
- *   carried scale (written to scales [rows] if not NULL), then records
- *   amax(x) in history at the state's slot, advances the slot (mod
- *   history_len) and carries RN(max(history) / 448) (1 when 0) to the next
- *   step.  One kernel; the state is updated by the last CTA to finish, so
- *   steps on one state must be stream-ordered (one stream, or events).
+ * pgf8_fp8_quantize_delayed: step `step` (0, 1, 2, ... : the caller counts
+ *   the calls made on this state) quantises x (rows >= 1) with the scale
+ *   carried out of the previous step, RN(max of the last history_len
+ *   amaxes / 448) (1 when 0; step 0: initial_scale), written to scales
+ *   [rows] if not NULL; x's amax is recorded for the steps that follow.
+ *   One kernel, no CTA waits for another: step t derives its scale from the
+ *   history ring (amaxes up to step t-2) and the amax of step t-1, which is
+ *   still pending in state.pending[(t-1) % 3] (one CTA then files it into
+ *   slot (t-1) mod history_len).  Steps on one state must be stream-ordered
+ *   and numbered consecutively.
+ * flags (quantize_tensor, quantize_delayed): PGF8_FLAG_OVERLAP_PREVIOUS
+ *   launches the kernel with programmatic stream serialization, as for the
+ *   linear entry points: it reads and writes nothing before the previous
+ *   kernel in the stream has completed, and a GEMM launched the same way
+ *   after it may start loading its weights while it runs.
  * ---------------------------------------------------------------------- */
 typedef struct {
-    float scale;          /* the scale the next step quantises with */
-    uint32_t amax_bits;   /* internal: running amax of a step in flight */
-    int32_t pos;          /* next history slot */
-    uint32_t done;        /* internal: CTAs of a step in flight that finished */
+    float initial_scale;  /* the scale of step 0 */
+    uint32_t pending[3];  /* amax of step t, accumulated in pending[t % 3] (bits of a float >= 0) */
 } pgf8_delayed_state;
 
 pgf8_status pgf8_fp8_amax_accumulate(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
                                      float *amax, void *stream);
 pgf8_status pgf8_fp8_quantize_tensor(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
-                                     const float *amax, uint8_t *q, float *scales, void *stream);
+                                     const float *amax, uint8_t *q, float *scales, int32_t flags, void *stream);
 pgf8_status pgf8_delayed_state_init(pgf8_delayed_state *state, float *history, int32_t history_len,
                                     float initial_scale, void *stream);
 pgf8_status pgf8_fp8_quantize_delayed(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
                                       uint8_t *q, float *scales, float *history, int32_t history_len,
-                                      pgf8_delayed_state *state, void *stream);
+                                      pgf8_delayed_state *state, int64_t step, int32_t flags, void *stream);
 
 /* ------------------------------------------------------------------------
  * Dynamic-activation FP8 linear: per-token quantisation of x (as

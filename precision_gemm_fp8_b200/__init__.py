@@ -57,9 +57,9 @@ _optp = ctypes.POINTER(LinearOpts)
 _SIGS = {
     "pgf8_fp8_quantize_rows": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _i32, _vp], _i32),
     "pgf8_fp8_amax_accumulate": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp], _i32),
-    "pgf8_fp8_quantize_tensor": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _vp], _i32),
+    "pgf8_fp8_quantize_tensor": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _i32, _vp], _i32),
     "pgf8_delayed_state_init": ([_vp, _vp, _i32, ctypes.c_float, _vp], _i32),
-    "pgf8_fp8_quantize_delayed": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _i32, _vp, _vp], _i32),
+    "pgf8_fp8_quantize_delayed": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _i32, _vp, _i64, _i32, _vp], _i32),
     "pgf8_fp8_linear": ([_vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _sz, _vp], _i32),
     "pgf8_fp8_linear_ex": ([_vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _sz, _optp, _vp], _i32),
     "pgf8_fp8_linear_workspace_size": ([_i64, _i64, _i64], _sz),
@@ -198,7 +198,7 @@ def fp8_amax_accumulate(x: torch.Tensor, amax: torch.Tensor | None = None, strea
 
 
 def fp8_quantize_tensor(x: torch.Tensor, amax: torch.Tensor, q: torch.Tensor | None = None,
-                        scales: torch.Tensor | None = None, stream=None):
+                        scales: torch.Tensor | None = None, flags: int = 0, stream=None):
     """Static per-tensor quantisation with the scale of a calibrated amax
     (device float32 [1]).  Returns (q uint8 [rows, cols], scales f32 [rows],
     every row holding the tensor's scale)."""
@@ -210,24 +210,28 @@ def fp8_quantize_tensor(x: torch.Tensor, amax: torch.Tensor, q: torch.Tensor | N
     if scales is None:
         scales = torch.empty(rows, dtype=torch.float32, device=x.device)
     _check(lib.pgf8_fp8_quantize_tensor(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(amax), _ptr(q),
-                                        _ptr(scales), _stream(stream)), "fp8_quantize_tensor")
+                                        _ptr(scales), flags, _stream(stream)), "fp8_quantize_tensor")
     return q, scales
 
 
 class DelayedScaling:
     """Delayed per-tensor scaling of one activation tensor: a device amax
-    history of ``history_len`` entries and the carried scale.  Each
-    ``step(x)`` quantises x with the carried scale, records amax(x) and
-    carries RN(max(history) / 448) to the next step (one kernel)."""
+    history of ``history_len`` entries and the pending amax of the last
+    step.  Each ``step(x)`` quantises x with the scale carried out of the
+    previous step, RN(max of the last history_len amaxes / 448), and records
+    amax(x) (one kernel)."""
 
     def __init__(self, history_len: int = 1024, initial_scale: float = 1.0, device="cuda", stream=None):
         self.history_len = int(history_len)
         self.history = torch.empty(self.history_len, dtype=torch.float32, device=device)
         self.state = torch.empty(4, dtype=torch.int32, device=device)   # pgf8_delayed_state, 16 bytes
+        self.steps = 0
+        self.initial_scale = float(initial_scale)
         _check(lib.pgf8_delayed_state_init(_ptr(self.state), _ptr(self.history), self.history_len,
-                                           float(initial_scale), _stream(stream)), "delayed_state_init")
+                                           self.initial_scale, _stream(stream)), "delayed_state_init")
 
-    def step(self, x: torch.Tensor, q: torch.Tensor | None = None, scales: torch.Tensor | None = None, stream=None):
+    def step(self, x: torch.Tensor, q: torch.Tensor | None = None, scales: torch.Tensor | None = None, flags: int = 0,
+             stream=None):
         """Returns (q uint8 [rows, cols], scales f32 [rows]: the step's scale)."""
         rows, cols = x.shape
         if x.stride(1) != 1:
@@ -238,13 +242,21 @@ class DelayedScaling:
             scales = torch.empty(rows, dtype=torch.float32, device=x.device)
         _check(lib.pgf8_fp8_quantize_delayed(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(q),
                                              _ptr(scales), _ptr(self.history), self.history_len, _ptr(self.state),
-                                             _stream(stream)), "fp8_quantize_delayed")
+                                             self.steps, flags, _stream(stream)), "fp8_quantize_delayed")
+        self.steps += 1
         return q, scales
 
-    def carried(self):
-        """(carried scale, next history slot), read back (synchronises)."""
-        st = self.state.cpu()
-        return float(st[0:1].view(torch.float32).item()), int(st[2].item())
+    def window(self):
+        """The last history_len amaxes as the ring holds them after the steps
+        so far (the newest, still pending on the device, filed in its slot);
+        read back (synchronises)."""
+        import numpy as _np
+        h = self.history.cpu().numpy().copy()
+        if self.steps:
+            t = self.steps - 1
+            pend = self.state.cpu().numpy().view(_np.uint32)[1 + t % 3]
+            h[t % self.history_len] = _np.array([pend], dtype=_np.uint32).view(_np.float32)[0]
+        return h
 
 
 def fp8_linear(aq, sa, wq, sw, y=None, workspace=None, path=PATH_AUTO, split_k=0, tile_n=0, flags=0,

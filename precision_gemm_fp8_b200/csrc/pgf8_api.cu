@@ -635,6 +635,27 @@ static pgf8_status launch_simple(void (*kernel)(Args...), unsigned grid, cudaStr
     return e == cudaSuccess ? PGF8_OK : cuda_fail(e);
 }
 
+// The same, optionally with programmatic stream serialization (the kernel
+// waits on the grid dependency before its first read).
+template <typename... Args>
+static pgf8_status launch_quant(void (*kernel)(Args...), unsigned grid, cudaStream_t st, int pdl, Args... args)
+{
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kQuantThreads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    if (pdl) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+    return e == cudaSuccess ? PGF8_OK : cuda_fail(e);
+}
+
 } // namespace pgf8
 
 using namespace pgf8;
@@ -666,7 +687,7 @@ pgf8_status pgf8_fp8_amax_accumulate(const void *x, pgf8_dtype xdt, int64_t rows
 }
 
 pgf8_status pgf8_fp8_quantize_tensor(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
-                                     const float *amax, uint8_t *q, float *scales, void *stream)
+                                     const float *amax, uint8_t *q, float *scales, int32_t flags, void *stream)
 {
     pgf8_status st = check_tensor_args(x, xdt, rows, cols, ldx, q, true, scales);
     if (st != PGF8_OK)
@@ -679,11 +700,12 @@ pgf8_status pgf8_fp8_quantize_tensor(const void *x, pgf8_dtype xdt, int64_t rows
         return PGF8_ERR_ALIGNMENT;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const unsigned grid = static_cast<unsigned>(rows);
+    const int pdl = (flags & PGF8_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
     if (xdt == PGF8_F32)
-        return launch_simple<float>(quantize_tensor_kernel<float>, grid, cs, static_cast<const float *>(x), cols, ldx,
-                                    amax, q, scales);
-    return launch_simple<__half>(quantize_tensor_kernel<__half>, grid, cs, static_cast<const __half *>(x), cols, ldx,
-                                 amax, q, scales);
+        return launch_quant(quantize_tensor_kernel<float>, grid, cs, pdl, static_cast<const float *>(x), cols, ldx,
+                            amax, q, scales);
+    return launch_quant(quantize_tensor_kernel<__half>, grid, cs, pdl, static_cast<const __half *>(x), cols, ldx,
+                        amax, q, scales);
 }
 
 pgf8_status pgf8_delayed_state_init(pgf8_delayed_state *state, float *history, int32_t history_len,
@@ -702,25 +724,26 @@ pgf8_status pgf8_delayed_state_init(pgf8_delayed_state *state, float *history, i
 
 pgf8_status pgf8_fp8_quantize_delayed(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
                                       uint8_t *q, float *scales, float *history, int32_t history_len,
-                                      pgf8_delayed_state *state, void *stream)
+                                      pgf8_delayed_state *state, int64_t step, int32_t flags, void *stream)
 {
     pgf8_status st = check_tensor_args(x, xdt, rows, cols, ldx, q, true, scales);
     if (st != PGF8_OK)
         return st;
-    if (!state || !history || history_len < 1 || history_len > (1 << 24))
+    if (!state || !history || history_len < 1 || history_len > (1 << 24) || step < 0)
         return PGF8_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(state) & 15u) != 0 || !aligned4(history))
         return PGF8_ERR_ALIGNMENT;
     if (rows == 0)
-        return PGF8_OK;
+        return PGF8_ERR_INVALID_ARG;   // a step needs its amax: at least one row
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const unsigned grid = static_cast<unsigned>(rows);
     DelayedState *ds = reinterpret_cast<DelayedState *>(state);
+    const int pdl = (flags & PGF8_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
     if (xdt == PGF8_F32)
-        return launch_simple<float>(quantize_delayed_kernel<float>, grid, cs, static_cast<const float *>(x), cols,
-                                    ldx, q, scales, history, static_cast<int>(history_len), ds);
-    return launch_simple<__half>(quantize_delayed_kernel<__half>, grid, cs, static_cast<const __half *>(x), cols, ldx,
-                                 q, scales, history, static_cast<int>(history_len), ds);
+        return launch_quant(quantize_delayed_kernel<float>, grid, cs, pdl, static_cast<const float *>(x), cols, ldx,
+                            q, scales, history, static_cast<int>(history_len), ds, step);
+    return launch_quant(quantize_delayed_kernel<__half>, grid, cs, pdl, static_cast<const __half *>(x), cols, ldx, q,
+                        scales, history, static_cast<int>(history_len), ds, step);
 }
 
 pgf8_status pgf8_fp8_quantize_rows(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,

@@ -295,15 +295,13 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(const T *_
 // (delayed scaling over an amax history of length >= 1024, scale below
 // 448).  amax = max |x| over the tensor (NaN ignored, as the per-row
 // quantisation); scale = RN(amax / 448), 1 when 0.  A delayed step
-// quantises with the scale carried from the previous step, then records its
-// amax in a ring of H and carries RN(max(history) / 448).
+// quantises with the scale carried from the previous step: RN(max of the
+// last H amaxes / 448).
 
 // Device layout of pgf8_delayed_state (16 bytes).
 struct DelayedState {
-    float scale;          // the scale the next step quantises with
-    unsigned amax_bits;   // running amax of the step in flight (bits of a non-negative float)
-    int pos;              // next history slot
-    unsigned done;        // CTAs of the step in flight that have finished
+    float initial_scale;   // the scale of step 0
+    unsigned pending[3];   // amax of step t accumulates in pending[t % 3] (bits of a non-negative float)
 };
 
 __device__ __forceinline__ float per_tensor_scale(float amax)
@@ -337,22 +335,52 @@ __global__ void __launch_bounds__(kQuantThreads) amax_accumulate_kernel(const T 
         atomicMax(amax_bits, __float_as_uint(m));
 }
 
-// Quantises one row with a given per-tensor scale; returns the row's amax
-// (block-wide, valid in every thread).
-template <typename T>
-__device__ __forceinline__ float quantize_row_with_scale(const T *xr, int64_t cols, uint8_t *qr, float s, float *red)
+// Quantises one row with a per-tensor scale that get_scale() produces (a
+// read of device state, possibly a CTA-wide reduction); returns the row's
+// amax (block-wide, valid in every thread).  Rows of up to kRegChunks x 256
+// chunks are loaded into registers before get_scale() runs, so the row's
+// load latency overlaps the scale's; longer rows are streamed after it.
+template <typename T, typename GetScale>
+__device__ __forceinline__ float quantize_row_scaled(const T *xr, int64_t cols, uint8_t *qr, float *red,
+                                                     GetScale get_scale, float &s_out)
 {
-    const RowDivisor d(s);
-    float m = 0.0f;
-    for (int64_t c = threadIdx.x; c < cols / 16; c += kQuantThreads) {
-        Vec16<T> v;
-        v.load(xr + c * 16);
+    const int64_t nchunk = cols / 16;
+    float a = 0.0f;
+    if (nchunk <= static_cast<int64_t>(kRegChunks) * kQuantThreads) {
+        Vec16<T> v[kRegChunks];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-            m = fmaxf(m, fabsf(v.v[i]));
-        *reinterpret_cast<uint4 *>(qr + c * 16) = encode16(v.v, d);
+        for (int u = 0; u < kRegChunks; ++u) {
+            const int64_t c = threadIdx.x + static_cast<int64_t>(u) * kQuantThreads;
+            if (c < nchunk)
+                v[u].load(xr + c * 16);
+        }
+        const float s = get_scale();
+        s_out = s;
+        const RowDivisor d(s);
+#pragma unroll
+        for (int u = 0; u < kRegChunks; ++u) {
+            const int64_t c = threadIdx.x + static_cast<int64_t>(u) * kQuantThreads;
+            if (c < nchunk) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    a = fmaxf(a, fabsf(v[u].v[i]));
+                *reinterpret_cast<uint4 *>(qr + c * 16) = encode16(v[u].v, d);
+            }
+        }
+    } else {
+        const float s = get_scale();
+        s_out = s;
+        const RowDivisor d(s);
+        for (int64_t c = threadIdx.x; c < nchunk; c += kQuantThreads) {
+            Vec16<T> v;
+            v.load(xr + c * 16);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                a = fmaxf(a, fabsf(v.v[i]));
+            *reinterpret_cast<uint4 *>(qr + c * 16) = encode16(v.v, d);
+        }
     }
-    return block_max(m, red);
+    return block_max(a, red);
 }
 
 // Static per-tensor quantisation with the scale of a calibrated amax; one
@@ -364,58 +392,68 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_tensor_kernel(const T 
                                                                         float *__restrict__ scales)
 {
     __shared__ float red[kQuantThreads / 32];
+    // a dependent GEMM launched with programmatic serialization may load its
+    // weights now; it reads q / scales only after this grid has completed
+    grid_launch_dependents();
+    // launched with programmatic serialization, the previous kernel may still
+    // run: nothing is read or written before it has completed
+    grid_dependency_wait();
     const int64_t row = blockIdx.x;
-    const float s = per_tensor_scale(*amax);
-    (void)quantize_row_with_scale(x + row * ldx, cols, q + row * cols, s, red);
+    float s;
+    (void)quantize_row_scaled(x + row * ldx, cols, q + row * cols, red, [&] { return per_tensor_scale(*amax); }, s);
     if (scales && threadIdx.x == 0)
         scales[row] = s;
 }
 
-// One delayed-scaling step; one CTA per row.  Every CTA quantises with the
-// carried scale (read before it signs off), folds its row amax into the
-// state, and signs off on a counter after a fence; the CTA that signs off
-// last records the step's amax in the history, carries the new scale and
-// resets the counters for the next step.  No CTA waits for another.
+// Step t of delayed scaling; one CTA per row.  The scale of step t is the
+// scale carried out of step t-1: max over the last H amaxes (steps t-H ..
+// t-1) / 448.  The history ring holds the amaxes up to step t-2; step t-1's
+// amax is still pending (accumulated by its CTAs), so every CTA takes
+//   max(history without slot (t-1) mod H, pending[(t-1) % 3])
+// (that slot held step t-1-H, which leaves the window), and CTA 0 files the
+// pending amax into the slot and clears the buffer step t+1 accumulates
+// into.  Each CTA then quantises its row and folds the row amax into
+// pending[t % 3].  Nothing waits on another CTA and nothing runs after the
+// quantisation; step t = 0 uses the initial scale.
 template <typename T>
 __global__ void __launch_bounds__(kQuantThreads) quantize_delayed_kernel(const T *__restrict__ x, int64_t cols,
                                                                          int64_t ldx, uint8_t *__restrict__ q,
                                                                          float *__restrict__ scales,
                                                                          float *__restrict__ history, int H,
-                                                                         DelayedState *st)
+                                                                         DelayedState *st, int64_t t)
 {
     __shared__ float red[kQuantThreads / 32];
-    __shared__ int last;
+    grid_launch_dependents();   // as in quantize_tensor_kernel
+    grid_dependency_wait();
     const int64_t row = blockIdx.x;
-    const float s = st->scale;
-    const float m = quantize_row_with_scale(x + row * ldx, cols, q + row * cols, s, red);
+    auto carried_scale = [&]() -> float {
+        if (t == 0)
+            return st->initial_scale;
+        const int slot = static_cast<int>((t - 1) % H);
+        const float prev = __uint_as_float(st->pending[(t - 1) % 3]);
+        float m = prev;
+        for (int i = threadIdx.x; i < H; i += kQuantThreads)
+            if (i != slot)
+                m = fmaxf(m, history[i]);
+        const float sc = per_tensor_scale(block_max(m, red));
+        __syncthreads();   // red is reused by the row's amax
+        if (blockIdx.x == 0 && threadIdx.x == 0)
+            history[slot] = prev;
+        return sc;
+    };
+    if (blockIdx.x == 0 && threadIdx.x == 0)
+        st->pending[(t + 1) % 3] = 0u;
+    float s;
+    const float m = quantize_row_scaled(x + row * ldx, cols, q + row * cols, red, carried_scale, s);
     if (threadIdx.x == 0) {
         if (scales)
             scales[row] = s;
         if (m > 0.0f)
-            atomicMax(&st->amax_bits, __float_as_uint(m));
-        __threadfence();
-        last = atomicAdd(&st->done, 1u) == gridDim.x - 1;
-    }
-    __syncthreads();
-    if (!last)
-        return;
-    __threadfence();
-    const float amax = __uint_as_float(atomicAdd(&st->amax_bits, 0u));
-    const int pos = st->pos;
-    float hm = 0.0f;
-    for (int i = threadIdx.x; i < H; i += kQuantThreads)
-        hm = fmaxf(hm, i == pos ? amax : history[i]);
-    hm = block_max(hm, red);
-    if (threadIdx.x == 0) {
-        history[pos] = amax;
-        st->pos = pos + 1 == H ? 0 : pos + 1;
-        st->scale = per_tensor_scale(hm);
-        st->amax_bits = 0u;
-        st->done = 0u;
+            atomicMax(&st->pending[t % 3], __float_as_uint(m));
     }
 }
 
-// Fresh delayed-scaling state: history zero, first step at slot 0 with the
+// Fresh delayed-scaling state: history zero, nothing pending, step 0 at the
 // given scale.
 __global__ void __launch_bounds__(kQuantThreads) delayed_init_kernel(float *__restrict__ history, int H,
                                                                      DelayedState *st, float initial_scale)
@@ -423,10 +461,8 @@ __global__ void __launch_bounds__(kQuantThreads) delayed_init_kernel(float *__re
     for (int i = blockIdx.x * kQuantThreads + threadIdx.x; i < H; i += gridDim.x * kQuantThreads)
         history[i] = 0.0f;
     if (blockIdx.x == 0 && threadIdx.x == 0) {
-        st->scale = initial_scale;
-        st->amax_bits = 0u;
-        st->pos = 0;
-        st->done = 0u;
+        st->initial_scale = initial_scale;
+        st->pending[0] = st->pending[1] = st->pending[2] = 0u;
     }
 }
 

@@ -183,16 +183,17 @@ def test_per_tensor_scaling_argument_checks():
     assert amax(a16 + 4, pg.F32, 2, 16, 16, a16, None) == pg.ERR_ALIGNMENT
     assert amax(a16, pg.BF16, 2, 16, 16, a16, None) == pg.ERR_UNSUPPORTED
     qt = pg.lib.pgf8_fp8_quantize_tensor
-    assert qt(a16, pg.F32, 2, 16, 16, a16, None, None, None) == pg.ERR_INVALID_ARG      # no q
-    assert qt(a16, pg.F32, 2, 16, 16, None, a16, None, None) == pg.ERR_INVALID_ARG      # no amax
-    assert qt(a16, pg.F32, 2, 16, 16, a16, a16 + 8, None, None) == pg.ERR_ALIGNMENT
+    assert qt(a16, pg.F32, 2, 16, 16, a16, None, None, 0, None) == pg.ERR_INVALID_ARG      # no q
+    assert qt(a16, pg.F32, 2, 16, 16, None, a16, None, 0, None) == pg.ERR_INVALID_ARG      # no amax
+    assert qt(a16, pg.F32, 2, 16, 16, a16, a16 + 8, None, 0, None) == pg.ERR_ALIGNMENT
     init = pg.lib.pgf8_delayed_state_init
     assert init(a16, a16, 0, 1.0, None) == pg.ERR_INVALID_ARG
     assert init(a16, a16, 1024, 0.0, None) == pg.ERR_INVALID_ARG
     assert init(a16, a16, 1024, float("inf"), None) == pg.ERR_INVALID_ARG
     assert init(a16 + 4, a16, 1024, 1.0, None) == pg.ERR_ALIGNMENT
     qd = pg.lib.pgf8_fp8_quantize_delayed
-    assert qd(a16, pg.F32, 2, 16, 16, a16, None, a16, 0, a16, None) == pg.ERR_INVALID_ARG
-    assert qd(a16, pg.F32, 2, 16, 16, a16, None, a16, 1024, None, None) == pg.ERR_INVALID_ARG
-    assert qd(a16, pg.F32, 2, 16, 16, a16, None, a16, 1024, a16 + 8, None) == pg.ERR_ALIGNMENT
-    assert qd(a16, pg.F32, 0, 16, 16, a16, None, a16, 1024, a16, None) == pg.OK          # empty step
+    assert qd(a16, pg.F32, 2, 16, 16, a16, None, a16, 0, a16, 0, 0, None) == pg.ERR_INVALID_ARG
+    assert qd(a16, pg.F32, 2, 16, 16, a16, None, a16, 1024, None, 0, 0, None) == pg.ERR_INVALID_ARG
+    assert qd(a16, pg.F32, 2, 16, 16, a16, None, a16, 1024, a16 + 8, 0, 0, None) == pg.ERR_ALIGNMENT
+    assert qd(a16, pg.F32, 0, 16, 16, a16, None, a16, 1024, a16, 0, 0, None) == pg.ERR_INVALID_ARG   # a step needs rows
+    assert qd(a16, pg.F32, 2, 16, 16, a16, None, a16, 1024, a16, -1, 0, None) == pg.ERR_INVALID_ARG  # step < 0
