@@ -81,6 +81,10 @@ def _load():
         lib.orc_delayed_step_f32.argtypes = [f32p, i64, i64, i64, u8p, f32p, ctypes.c_int32,
                                              ctypes.POINTER(ctypes.c_int32), f32p, f32p]
         lib.orc_delayed_step_f32.restype = ctypes.c_int
+        lib.orc_norm_rows.argtypes = [f32p, i64, i64, i64, f32p, f32p, ctypes.c_double, f64p]
+        lib.orc_norm_rows.restype = ctypes.c_int
+        lib.orc_silu_mul.argtypes = [f64p, f64p, i64, f64p]
+        lib.orc_silu_mul.restype = None
         lib.orc_nestedfp_linear_fp8.restype = ctypes.c_int
         _lib = lib
         return lib
@@ -304,3 +308,29 @@ class DelayedScaling:
         self.pos = pos.value
         self.scale = np.float32(sc[0])
         return q, np.float32(used[0])
+
+
+# ---------------------------------------------------------------- normalisation / gated activation
+def norm_rows(x: np.ndarray, gamma: np.ndarray, beta: np.ndarray | None = None, eps: float = 1e-5) -> np.ndarray:
+    """LayerNorm (beta given) or RMSNorm (beta None) of each row, binary64."""
+    lib = _load()
+    x = _as_f32_2d(x)
+    R, C = x.shape
+    gamma = np.ascontiguousarray(gamma, dtype=np.float32)
+    y = np.empty((R, C), dtype=np.float64)
+    bp = None if beta is None else _ptr(np.ascontiguousarray(beta, dtype=np.float32), ctypes.c_float)
+    _check(lib.orc_norm_rows(_ptr(x, ctypes.c_float), R, C, C, _ptr(gamma, ctypes.c_float), bp, float(eps),
+                             _ptr(y, ctypes.c_double)))
+    return y
+
+
+def silu_mul(g: np.ndarray, u: np.ndarray) -> np.ndarray:
+    """g / (1 + exp(-g)) * u elementwise, binary64 (inputs widened exactly)."""
+    lib = _load()
+    g = np.ascontiguousarray(g, dtype=np.float64)
+    u = np.ascontiguousarray(u, dtype=np.float64)
+    if g.shape != u.shape:
+        raise ValueError("g and u must have the same shape")
+    h = np.empty(g.shape, dtype=np.float64)
+    lib.orc_silu_mul(_ptr(g, ctypes.c_double), _ptr(u, ctypes.c_double), g.size, _ptr(h, ctypes.c_double))
+    return h

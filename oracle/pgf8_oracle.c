@@ -413,3 +413,57 @@ int orc_delayed_step_f32(const float *x, int64_t rows, int64_t cols, int64_t ldx
     *scale = scale_of_amax(hmax);
     return ORC_OK;
 }
+
+/* ------------------------------------------------------------------ */
+/* Normalisation and gated activation ahead of the quantisation.       */
+/*                                                                     */
+/* [FP8-4060] "computation graph restructuring" §2.1 fuses LayerNorm   */
+/* with the QKV projection's input; its feature list pairs LayerNorm   */
+/* with the activation.  The pages print no formula.  Readings (the    */
+/* textbook definitions), evaluated in binary64:                       */
+/*   LayerNorm  y = (x - mean) / sqrt(var + eps) * gamma + beta,       */
+/*              mean = sum x / K, var = sum (x - mean)^2 / K;          */
+/*   RMSNorm    y = x / sqrt(sum x^2 / K + eps) * gamma  (beta absent);*/
+/*   SiLU gate  h = g / (1 + exp(-g)) * u.                             */
+/* ------------------------------------------------------------------ */
+
+/* y [rows, cols] binary64 from x (row stride ldx); beta == NULL selects
+ * RMSNorm. */
+int orc_norm_rows(const float *x, int64_t rows, int64_t cols, int64_t ldx, const float *gamma, const float *beta,
+                  double eps, double *y)
+{
+    if (rows < 0 || cols < 1 || ldx < cols || !gamma || !(eps >= 0.0))
+        return ORC_ERR_ARG;
+    for (int64_t r = 0; r < rows; ++r) {
+        const float *xr = x + r * ldx;
+        for (int64_t k = 0; k < cols; ++k)
+            if (!isfinite(xr[k]))
+                return ORC_ERR_NONFINITE;
+        double mean = 0.0;
+        if (beta) {
+            for (int64_t k = 0; k < cols; ++k)
+                mean += (double)xr[k];
+            mean /= (double)cols;
+        }
+        double ss = 0.0;
+        for (int64_t k = 0; k < cols; ++k) {
+            double d = (double)xr[k] - mean;
+            ss += d * d;
+        }
+        double inv = 1.0 / sqrt(ss / (double)cols + eps);
+        for (int64_t k = 0; k < cols; ++k) {
+            double v = ((double)xr[k] - mean) * inv * (double)gamma[k];
+            if (beta)
+                v += (double)beta[k];
+            y[r * cols + k] = v;
+        }
+    }
+    return ORC_OK;
+}
+
+/* h[i] = g[i] / (1 + exp(-g[i])) * u[i] in binary64. */
+void orc_silu_mul(const double *g, const double *u, int64_t count, double *h)
+{
+    for (int64_t i = 0; i < count; ++i)
+        h[i] = g[i] / (1.0 + exp(-g[i])) * u[i];
+}
