@@ -162,6 +162,34 @@ pgf8_status pgf8_fp8_linear_ex(const uint8_t *aq, const float *sa, int64_t M, in
 size_t pgf8_fp8_linear_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /* ------------------------------------------------------------------------
+ * Normalisation or gate fused with the per-token quantisation ("7B on an
+ * RTX 4060 with FP8", computation graph §2.1: LayerNorm fused with the QKV
+ * projection's input).  The normalised / gated values never go to memory;
+ * the codes and per-token scales feed pgf8_fp8_linear.  The values are
+ * computed in binary32 (textbook definitions below), then quantised as in
+ * pgf8_fp8_quantize_rows (DYNAMIC).  The pages print no formula and no
+ * numerics for these steps; the binary32 rounding of the values depends on
+ * the kernel's reduction order and on expf.
+ *
+ * pgf8_fp8_norm_quantize: x [rows, cols] f32 or f16 (row stride ldx),
+ *   gamma [cols] f32, beta [cols] f32 or NULL.  With beta: LayerNorm
+ *   y = (x - mean) * rsqrt(var + eps) * gamma + beta (biased variance);
+ *   without: RMSNorm y = x * rsqrt(mean(x^2) + eps) * gamma.  eps >= 0.
+ *   cols % 16 == 0 and cols <= 16384 (a row is held in registers; else
+ *   PGF8_ERR_UNSUPPORTED).  q [rows, cols], scales [rows].
+ * pgf8_fp8_silu_mul_quantize: gu [rows, 2*inter] bf16 or f32 (row stride
+ *   ldg >= 2*inter), the gate+up projection's output: gate = columns
+ *   [0, inter), up = [inter, 2*inter).  h = gate / (1 + exp(-gate)) * up is
+ *   quantised into q [rows, inter], scales [rows].  inter % 16 == 0.
+ * flags: PGF8_FLAG_OVERLAP_PREVIOUS as for the per-tensor calls.
+ * ---------------------------------------------------------------------- */
+pgf8_status pgf8_fp8_norm_quantize(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
+                                   const float *gamma, const float *beta, float eps, uint8_t *q, float *scales,
+                                   int32_t flags, void *stream);
+pgf8_status pgf8_fp8_silu_mul_quantize(const void *gu, pgf8_dtype gdt, int64_t rows, int64_t inter, int64_t ldg,
+                                       uint8_t *q, float *scales, int32_t flags, void *stream);
+
+/* ------------------------------------------------------------------------
  * Per-tensor activation scaling ("C++ and FP8" §5.1: MINMAX calibration,
  * the scale follows the largest magnitude seen over calibration data;
  * "7B on an RTX 4060 with FP8" §6.1: delayed scaling over an amax history

@@ -57,6 +57,8 @@ _optp = ctypes.POINTER(LinearOpts)
 _SIGS = {
     "pgf8_fp8_quantize_rows": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _i32, _vp], _i32),
     "pgf8_fp8_amax_accumulate": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp], _i32),
+    "pgf8_fp8_norm_quantize": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, ctypes.c_float, _vp, _vp, _i32, _vp], _i32),
+    "pgf8_fp8_silu_mul_quantize": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _i32, _vp], _i32),
     "pgf8_fp8_quantize_tensor": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _i32, _vp], _i32),
     "pgf8_delayed_state_init": ([_vp, _vp, _i32, ctypes.c_float, _vp], _i32),
     "pgf8_fp8_quantize_delayed": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _i32, _vp, _i64, _i32, _vp], _i32),
@@ -180,6 +182,45 @@ def fp8_quantize_rows(x: torch.Tensor, q: torch.Tensor | None = None, scales: to
         scales = torch.empty(rows, dtype=torch.float32, device=x.device)
     _check(lib.pgf8_fp8_quantize_rows(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(q), _ptr(scales),
                                       mode, _stream(stream)), "fp8_quantize_rows")
+    return q, scales
+
+
+def fp8_norm_quantize(x: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor | None = None, eps: float = 1e-5,
+                      q: torch.Tensor | None = None, scales: torch.Tensor | None = None, flags: int = 0, stream=None):
+    """LayerNorm (beta given) or RMSNorm (beta None) of each row of x [rows,
+    cols] (f32/f16), quantised per token to E4M3.  Returns (q uint8 [rows,
+    cols], scales f32 [rows])."""
+    rows, cols = x.shape
+    if x.stride(1) != 1:
+        raise ValueError("x rows must be contiguous")
+    if q is None:
+        q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(rows, dtype=torch.float32, device=x.device)
+    _check(lib.pgf8_fp8_norm_quantize(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(gamma),
+                                      None if beta is None else _ptr(beta), float(eps), _ptr(q), _ptr(scales), flags,
+                                      _stream(stream)), "fp8_norm_quantize")
+    return q, scales
+
+
+def fp8_silu_mul_quantize(gu: torch.Tensor, q: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                          flags: int = 0, stream=None):
+    """silu(gate) * up of the gate+up output gu [rows, 2I] (bf16 or f32; gate
+    = first I columns), quantised per token to E4M3.  Returns (q uint8
+    [rows, I], scales f32 [rows])."""
+    rows, two_i = gu.shape
+    if gu.stride(1) != 1 or two_i % 2:
+        raise ValueError("gu rows must be contiguous with an even width")
+    inter = two_i // 2
+    code = {torch.bfloat16: BF16, torch.float32: F32}.get(gu.dtype)
+    if code is None:
+        raise TypeError(f"unsupported gate/up dtype {gu.dtype}")
+    if q is None:
+        q = torch.empty((rows, inter), dtype=torch.uint8, device=gu.device)
+    if scales is None:
+        scales = torch.empty(rows, dtype=torch.float32, device=gu.device)
+    _check(lib.pgf8_fp8_silu_mul_quantize(_ptr(gu), code, rows, inter, gu.stride(0), _ptr(q), _ptr(scales), flags,
+                                          _stream(stream)), "fp8_silu_mul_quantize")
     return q, scales
 
 

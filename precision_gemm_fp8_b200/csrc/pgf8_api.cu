@@ -746,6 +746,55 @@ pgf8_status pgf8_fp8_quantize_delayed(const void *x, pgf8_dtype xdt, int64_t row
                         scales, history, static_cast<int>(history_len), ds, step);
 }
 
+pgf8_status pgf8_fp8_norm_quantize(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
+                                   const float *gamma, const float *beta, float eps, uint8_t *q, float *scales,
+                                   int32_t flags, void *stream)
+{
+    pgf8_status st = check_quantize_args(x, xdt, rows, cols, ldx, q, scales, PGF8_SCALE_DYNAMIC);
+    if (st != PGF8_OK)
+        return st;
+    if (rows == 0)
+        return PGF8_OK;
+    if (!gamma || !(eps >= 0.0f) || !std::isfinite(eps))
+        return PGF8_ERR_INVALID_ARG;
+    if (!aligned4(gamma) || (beta && !aligned4(beta)))
+        return PGF8_ERR_ALIGNMENT;
+    if (cols > static_cast<int64_t>(kRegChunks) * kQuantThreads * 16)
+        return PGF8_ERR_UNSUPPORTED;   // the row is held in registers
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const int pdl = (flags & PGF8_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
+    const unsigned grid = static_cast<unsigned>(rows);
+    if (xdt == PGF8_F32)
+        return launch_quant(norm_quantize_kernel<float>, grid, cs, pdl, static_cast<const float *>(x), cols, ldx,
+                            gamma, beta, eps, q, scales);
+    return launch_quant(norm_quantize_kernel<__half>, grid, cs, pdl, static_cast<const __half *>(x), cols, ldx,
+                        gamma, beta, eps, q, scales);
+}
+
+pgf8_status pgf8_fp8_silu_mul_quantize(const void *gu, pgf8_dtype gdt, int64_t rows, int64_t inter, int64_t ldg,
+                                       uint8_t *q, float *scales, int32_t flags, void *stream)
+{
+    if (rows < 0 || inter < 16 || ldg < 2 * inter || rows > (1ll << 31) - 1)
+        return PGF8_ERR_INVALID_ARG;
+    if (rows == 0)
+        return PGF8_OK;
+    if (!gu || !q || !scales)
+        return PGF8_ERR_INVALID_ARG;
+    if (gdt != PGF8_BF16 && gdt != PGF8_F32)
+        return PGF8_ERR_UNSUPPORTED;
+    const int eb = gdt == PGF8_F32 ? 4 : 2;
+    if (inter % 16 != 0 || (ldg * eb) % 16 != 0 || !aligned16(gu) || !aligned16(q) || !aligned4(scales))
+        return PGF8_ERR_ALIGNMENT;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const int pdl = (flags & PGF8_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
+    const unsigned grid = static_cast<unsigned>(rows);
+    if (gdt == PGF8_F32)
+        return launch_quant(silu_mul_quantize_kernel<float>, grid, cs, pdl, static_cast<const float *>(gu), inter,
+                            ldg, q, scales);
+    return launch_quant(silu_mul_quantize_kernel<__nv_bfloat16>, grid, cs, pdl,
+                        static_cast<const __nv_bfloat16 *>(gu), inter, ldg, q, scales);
+}
+
 pgf8_status pgf8_fp8_quantize_rows(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
                                    uint8_t *q, float *scales, pgf8_scale_mode mode, void *stream)
 {

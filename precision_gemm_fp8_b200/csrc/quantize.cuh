@@ -11,6 +11,7 @@
 // Bytes per element: 4 (f32) or 2 (f16) in, 1 out.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cstdint>
 
@@ -464,6 +465,228 @@ __global__ void __launch_bounds__(kQuantThreads) delayed_init_kernel(float *__re
         st->initial_scale = initial_scale;
         st->pending[0] = st->pending[1] = st->pending[2] = 0u;
     }
+}
+
+// ------------------------------------------------------------------ norm / gate + quantisation
+// "7B on an RTX 4060 with FP8", computation graph §2.1: LayerNorm fused with
+// the QKV projection's input.  Here the normalisation (LayerNorm, or
+// RMSNorm for the Llama shapes) runs in the quantisation kernel that feeds
+// the projection, and the SiLU gate in the one that feeds the down
+// projection, so neither intermediate goes to memory:
+//   LayerNorm y = (x - mean) * rsqrt(var + eps) * gamma + beta  (biased var)
+//   RMSNorm   y = x * rsqrt(mean(x^2) + eps) * gamma
+//   gate      h = g / (1 + exp(-g)) * u
+// in binary32, then per-token E4M3 as quantize_rows (amax, RN(amax/448),
+// RN(y/s) saturating).
+
+template <> struct Vec16<__nv_bfloat16> {
+    float v[16];
+    __device__ __forceinline__ void load(const __nv_bfloat16 *p)
+    {
+        const uint4 *q = reinterpret_cast<const uint4 *>(p);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            uint4 t = __ldg(q + i);
+            uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                // bf16 -> f32 is exact: the bf16 bits are the f32's upper half
+                v[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+                v[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+            }
+        }
+    }
+};
+
+__device__ __forceinline__ float block_sum(float v, float *red)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __syncthreads();   // red may still be read by a previous reduction
+    if (lane == 0)
+        red[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        v = lane < (kQuantThreads / 32) ? red[lane] : 0.0f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0)
+            red[0] = v;
+    }
+    __syncthreads();
+    return red[0];
+}
+
+// Encodes the row held in registers (y values), writes codes and the scale.
+__device__ __forceinline__ void quantize_held_row(Vec16<float> (&y)[kRegChunks], int64_t nchunk, uint8_t *qr,
+                                                  float *scale_out, float *red)
+{
+    float a = 0.0f;
+#pragma unroll
+    for (int u = 0; u < kRegChunks; ++u) {
+        const int64_t c = threadIdx.x + static_cast<int64_t>(u) * kQuantThreads;
+        if (c < nchunk) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                a = fmaxf(a, fabsf(y[u].v[i]));
+        }
+    }
+    __syncthreads();   // red may still be read by a previous reduction
+    a = block_max(a, red);
+    float s = __fdiv_rn(a, 448.0f);
+    if (s == 0.0f)
+        s = 1.0f;
+    const RowDivisor d(s);
+#pragma unroll
+    for (int u = 0; u < kRegChunks; ++u) {
+        const int64_t c = threadIdx.x + static_cast<int64_t>(u) * kQuantThreads;
+        if (c < nchunk)
+            *reinterpret_cast<uint4 *>(qr + c * 16) = encode16(y[u].v, d);
+    }
+    if (threadIdx.x == 0)
+        *scale_out = s;
+}
+
+// One CTA per row; rows of up to kRegChunks x 256 x 16 elements (held in
+// registers).  beta == nullptr: RMSNorm.
+template <typename T>
+__global__ void __launch_bounds__(kQuantThreads) norm_quantize_kernel(const T *__restrict__ x, int64_t cols,
+                                                                      int64_t ldx, const float *__restrict__ gamma,
+                                                                      const float *__restrict__ beta, float eps,
+                                                                      uint8_t *__restrict__ q,
+                                                                      float *__restrict__ scales)
+{
+    __shared__ float red[kQuantThreads / 32];
+    grid_launch_dependents();   // a dependent GEMM reads q / scales only after this grid completes
+    grid_dependency_wait();
+    const int64_t row = blockIdx.x;
+    const T *xr = x + row * ldx;
+    const int64_t nchunk = cols / 16;
+    Vec16<float> v[kRegChunks];
+#pragma unroll
+    for (int u = 0; u < kRegChunks; ++u) {
+        const int64_t c = threadIdx.x + static_cast<int64_t>(u) * kQuantThreads;
+        if (c < nchunk) {
+            Vec16<T> t;
+            t.load(xr + c * 16);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                v[u].v[i] = t.v[i];
+        }
+    }
+    const float inv_n = 1.0f / static_cast<float>(cols);
+    float mean = 0.0f;
+    if (beta) {
+        float sum = 0.0f;
+#pragma unroll
+        for (int u = 0; u < kRegChunks; ++u) {
+            const int64_t c = threadIdx.x + static_cast<int64_t>(u) * kQuantThreads;
+            if (c < nchunk) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    sum += v[u].v[i];
+            }
+        }
+        mean = block_sum(sum, red) * inv_n;
+    }
+    float ss = 0.0f;
+#pragma unroll
+    for (int u = 0; u < kRegChunks; ++u) {
+        const int64_t c = threadIdx.x + static_cast<int64_t>(u) * kQuantThreads;
+        if (c < nchunk) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float d = v[u].v[i] - mean;
+                ss = fmaf(d, d, ss);
+            }
+        }
+    }
+    const float rstd = __frsqrt_rn(block_sum(ss, red) * inv_n + eps);
+#pragma unroll
+    for (int u = 0; u < kRegChunks; ++u) {
+        const int64_t c = threadIdx.x + static_cast<int64_t>(u) * kQuantThreads;
+        if (c < nchunk) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int64_t k = c * 16 + i;
+                float y = (v[u].v[i] - mean) * rstd * __ldg(gamma + k);
+                if (beta)
+                    y += __ldg(beta + k);
+                v[u].v[i] = y;
+            }
+        }
+    }
+    quantize_held_row(v, nchunk, q + row * cols, scales + row, red);
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u)
+{
+    return __fdiv_rn(g, 1.0f + expf(-g)) * u;
+}
+
+// One CTA per row of the gate+up output gu [rows, 2I] (gate = columns
+// [0, I), up = [I, 2I)); h [rows, I] is quantised.  Rows of up to
+// kRegChunks x 256 x 16 elements are held in registers; longer rows are
+// computed twice (amax pass, then the codes), identically.
+template <typename T>
+__global__ void __launch_bounds__(kQuantThreads) silu_mul_quantize_kernel(const T *__restrict__ gu, int64_t inter,
+                                                                          int64_t ldg, uint8_t *__restrict__ q,
+                                                                          float *__restrict__ scales)
+{
+    __shared__ float red[kQuantThreads / 32];
+    grid_launch_dependents();
+    grid_dependency_wait();
+    const int64_t row = blockIdx.x;
+    const T *gr = gu + row * ldg;
+    const T *ur = gr + inter;
+    uint8_t *qr = q + row * inter;
+    const int64_t nchunk = inter / 16;
+    if (nchunk <= static_cast<int64_t>(kRegChunks) * kQuantThreads) {
+        Vec16<float> h[kRegChunks];
+#pragma unroll
+        for (int u = 0; u < kRegChunks; ++u) {
+            const int64_t c = threadIdx.x + static_cast<int64_t>(u) * kQuantThreads;
+            if (c < nchunk) {
+                Vec16<T> g, up;
+                g.load(gr + c * 16);
+                up.load(ur + c * 16);
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    h[u].v[i] = silu_mul(g.v[i], up.v[i]);
+            }
+        }
+        quantize_held_row(h, nchunk, qr, scales + row, red);
+        return;
+    }
+    float a = 0.0f;
+    for (int64_t c = threadIdx.x; c < nchunk; c += kQuantThreads) {
+        Vec16<T> g, up;
+        g.load(gr + c * 16);
+        up.load(ur + c * 16);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            a = fmaxf(a, fabsf(silu_mul(g.v[i], up.v[i])));
+    }
+    a = block_max(a, red);
+    float s = __fdiv_rn(a, 448.0f);
+    if (s == 0.0f)
+        s = 1.0f;
+    const RowDivisor d(s);
+    for (int64_t c = threadIdx.x; c < nchunk; c += kQuantThreads) {
+        Vec16<T> g, up;
+        g.load(gr + c * 16);
+        up.load(ur + c * 16);
+        float hv[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            hv[i] = silu_mul(g.v[i], up.v[i]);
+        *reinterpret_cast<uint4 *>(qr + c * 16) = encode16(hv, d);
+    }
+    if (threadIdx.x == 0)
+        scales[row] = s;
 }
 
 // NestedFP split: 8 FP16 bit patterns per thread per step (16 bytes in, 8 + 8 out).
