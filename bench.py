@@ -288,6 +288,29 @@ def run_ours(args, rank, world, local_rank):
                 per_tensor[i] = pg.fp8_amax_accumulate(acts[i])   # MINMAX calibration on the layer's input
         torch.cuda.synchronize()
 
+    # --chain: the decoder layer's own producers of each GEMM input: RMSNorm
+    # fused with the quantisation ahead of QKV and gate+up, the SiLU gate
+    # over the gate+up output fused with the quantisation ahead of down (O
+    # keeps its dynamic quantisation: its input is the attention output)
+    gammas = {}
+    if args.chain:
+        if any(L.kind != "fp8" for L in layers) or len(wl.shapes) != 4:
+            raise SystemExit("--chain needs a workload of QKV, O, gate+up, down FP8 layers")
+        g = torch.Generator().manual_seed(7)
+        for i, L in enumerate(layers):
+            if L.shape_idx in (0, 2):
+                gammas[i] = (0.5 + torch.rand(L.K, generator=g)).to(dev)
+
+    def quantise_chain(i, L, flags):
+        aq, sa = pg.dynamic_workspace_views(qbufs[i], L.M, L.K)
+        if L.shape_idx in (0, 2):
+            pg.fp8_norm_quantize(acts[i], gammas[i], None, 1e-6, aq, sa, flags=flags, stream=stream)
+        elif L.shape_idx == 3:
+            pg.fp8_silu_mul_quantize(outs[i - 1], aq, sa, flags=flags, stream=stream)
+        else:
+            pg.fp8_quantize_rows(acts[i], aq, sa, stream=stream)
+        return aq, sa
+
     def quantise_per_tensor(i, L, flags=0):
         aq, sa = pg.dynamic_workspace_views(qbufs[i], L.M, L.K)
         if args.scaling == "delayed":
@@ -307,6 +330,22 @@ def run_ours(args, rank, world, local_rank):
         isolation; these are the durations the roofline uses)."""
         for i, L in enumerate(layers):
             W = weights[(L.shape_idx, L.copy, L.kind != "fp8")]
+            if L.kind == "fp8" and args.chain:
+                if ev_pairs is None and L.shape_idx == 1:   # O: the dynamic pair, overlapped
+                    pg.fp8_linear_dynamic(acts[i], W[0], W[1], y=outs[i], workspace=qbufs[i],
+                                          flags=pg.FLAG_OVERLAP_PREVIOUS, stream=stream)
+                    continue
+                if ev_pairs is None:
+                    aq, sa = quantise_chain(i, L, pg.FLAG_OVERLAP_PREVIOUS)
+                    pg.fp8_linear(aq, sa, W[0], W[1], y=outs[i], workspace=sk_ws, flags=pg.FLAG_OVERLAP_PREVIOUS,
+                                  stream=stream)
+                    continue
+                ev_pairs[i][2].record(stream)
+                aq, sa = quantise_chain(i, L, 0)
+                ev_pairs[i][0].record(stream)
+                pg.fp8_linear(aq, sa, W[0], W[1], y=outs[i], workspace=sk_ws, stream=stream)
+                ev_pairs[i][1].record(stream)
+                continue
             if L.kind == "fp8":
                 if ev_pairs is None and not per_tensor:
                     pg.fp8_linear_dynamic(acts[i], W[0], W[1], y=outs[i], workspace=qbufs[i],
@@ -458,6 +497,8 @@ def run_ours(args, rank, world, local_rank):
                    "quantisation": "inside the skinny GEMM where each CTA's activation slice fits its "
                                    "registers, else its own kernel" if args.fused_quant
                    else "own kernel before each GEMM",
+                   "chain": ("decoder layer: RMSNorm+quantise -> QKV; quantise -> O; RMSNorm+quantise -> "
+                             "gate+up; SiLU gate+quantise of the gate+up output -> down") if args.chain else None,
                    "activation_scaling": {"dynamic": "per token, dynamic",
                                           "delayed": "per tensor, delayed (amax history of 1024 per layer)",
                                           "static": "per tensor, MINMAX-calibrated amax"}[args.scaling]},
@@ -506,7 +547,13 @@ def run_e2e(pg, torch, dev, layers, weights, acts_host, outs, args, world, wbyte
     all_fp8 = all(L.kind == "fp8" for L in layers)
     seq = None
     per_tensor = {}
-    if all_fp8 and args.scaling != "dynamic":
+    gammas = {}
+    if all_fp8 and args.chain:
+        g = torch.Generator().manual_seed(7)
+        for i, L in enumerate(layers):
+            if L.shape_idx in (0, 2):
+                gammas[i] = (0.5 + torch.rand(L.K, generator=g)).to(dev)
+    elif all_fp8 and args.scaling != "dynamic":
         for i, L in enumerate(layers):
             per_tensor[i] = (pg.DelayedScaling(1024, device=dev) if args.scaling == "delayed"
                              else pg.fp8_amax_accumulate(x_views[i].copy_(acts_host[i].to(dev))))
@@ -521,6 +568,21 @@ def run_e2e(pg, torch, dev, layers, weights, acts_host, outs, args, world, wbyte
             x_dev.copy_(x_host, non_blocking=True)
             if seq is not None:
                 seq.run(flags=pg.FLAG_FUSED_QUANT if args.fused_quant else 0, stream=stream)
+            elif gammas:
+                for i, L in enumerate(layers):
+                    W = weights[(L.shape_idx, L.copy, False)]
+                    aq, sa = pg.dynamic_workspace_views(ws[i], L.M, L.K)
+                    fl = pg.FLAG_OVERLAP_PREVIOUS if i else 0
+                    if L.shape_idx == 1:
+                        pg.fp8_linear_dynamic(x_views[i], W[0], W[1], y=y_views[i], workspace=ws[i], flags=fl,
+                                              stream=stream)
+                        continue
+                    if L.shape_idx in (0, 2):
+                        pg.fp8_norm_quantize(x_views[i], gammas[i], None, 1e-6, aq, sa, flags=fl, stream=stream)
+                    else:
+                        pg.fp8_silu_mul_quantize(y_views[i - 1], aq, sa, flags=fl, stream=stream)
+                    pg.fp8_linear(aq, sa, W[0], W[1], y=y_views[i], workspace=ws[i],
+                                  flags=pg.FLAG_OVERLAP_PREVIOUS, stream=stream)
             elif per_tensor:
                 for i, L in enumerate(layers):
                     W = weights[(L.shape_idx, L.copy, False)]
@@ -562,7 +624,9 @@ def run_e2e(pg, torch, dev, layers, weights, acts_host, outs, args, world, wbyte
     return {"value": round(v, 2), "unit": "GB/s" if memory_bound else "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(ms, 5),
-            "entry_point": ("pgf8_nestedfp_linear" if not all_fp8 else "pgf8_fp8_linear_dynamic_many"
+            "entry_point": ("pgf8_nestedfp_linear" if not all_fp8 else
+                            "pgf8_fp8_norm_quantize / pgf8_fp8_silu_mul_quantize / pgf8_fp8_quantize_rows + "
+                            "pgf8_fp8_linear per layer" if args.chain else "pgf8_fp8_linear_dynamic_many"
                             if args.scaling == "dynamic" else
                             {"delayed": "pgf8_fp8_quantize_delayed", "static": "pgf8_fp8_quantize_tensor"}[args.scaling]
                             + " + pgf8_fp8_linear per layer")}
@@ -699,6 +763,9 @@ def main():
     ap.add_argument("--scaling", choices=["dynamic", "delayed", "static"], default="dynamic",
                     help="activation scales of the FP8 layers: per-token dynamic (default), per-tensor delayed "
                          "(amax history of 1024) or per-tensor static (MINMAX-calibrated)")
+    ap.add_argument("--chain", action="store_true",
+                    help="feed each GEMM from its decoder-layer producer: RMSNorm fused with the quantisation ahead "
+                         "of QKV and gate+up, the SiLU gate of the gate+up output ahead of down")
     ap.add_argument("--fused-quant", action="store_true",
                     help="quantise dynamic activations inside the skinny GEMM where its kernel allows it")
     ap.add_argument("--single", default=None, help="kind,M,K,N: time (or profile) one layer eagerly")
