@@ -773,6 +773,9 @@ def main():
     ap.add_argument("--split-k", type=int, default=0)
     ap.add_argument("--tile-n", type=int, default=0)
     args = ap.parse_args()
+    if args.chain and (args.scaling != "dynamic" or args.fused_quant):
+        ap.error("--chain measures the decoder-layer producers with per-token scales; it takes neither "
+                 "--scaling nor --fused-quant")
     if args.single:
         run_single(args)
         return
