@@ -85,6 +85,14 @@ def _load():
         lib.orc_norm_rows.restype = ctypes.c_int
         lib.orc_silu_mul.argtypes = [f64p, f64p, i64, f64p]
         lib.orc_silu_mul.restype = None
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        lib.orc_kv_calibrate_scales.argtypes = [f32p, i64, i64, i64, f32p]
+        lib.orc_kv_calibrate_scales.restype = ctypes.c_int
+        lib.orc_kv_write_paged.argtypes = [f32p, i64, i64, i64, i64, f32p, i64, i32p, i64, u8p]
+        lib.orc_kv_write_paged.restype = ctypes.c_int
+        lib.orc_attention_paged.argtypes = [f64p, i64, i64, i64, u8p, u8p, f32p, f32p, i64, i64, i32p, i64, i64,
+                                            f64p, f64p]
+        lib.orc_attention_paged.restype = ctypes.c_int
         lib.orc_nestedfp_linear_fp8.restype = ctypes.c_int
         _lib = lib
         return lib
@@ -334,3 +342,60 @@ def silu_mul(g: np.ndarray, u: np.ndarray) -> np.ndarray:
     h = np.empty(g.shape, dtype=np.float64)
     lib.orc_silu_mul(_ptr(g, ctypes.c_double), _ptr(u, ctypes.c_double), g.size, _ptr(h, ctypes.c_double))
     return h
+
+
+# ---------------------------------------------------------------- FP8 KV cache
+def kv_calibrate_scales(kv: np.ndarray) -> np.ndarray:
+    """Per-KV-head MINMAX scales of kv [T, H, D]: fl32(max |kv[:, h, :]| / 448), 1 when 0."""
+    lib = _load()
+    kv = np.ascontiguousarray(kv, dtype=np.float32)
+    T, H, D = kv.shape
+    s = np.empty(H, dtype=np.float32)
+    _check(lib.orc_kv_calibrate_scales(_ptr(kv, ctypes.c_float), T, H, D, _ptr(s, ctypes.c_float)))
+    return s
+
+
+class PagedKV:
+    """An FP8 (E4M3) paged cache [num_blocks, H, B, D] with per-head scales
+    and a block table (logical block -> physical block)."""
+
+    def __init__(self, num_blocks: int, heads: int, head_dim: int, block_size: int, scales: np.ndarray,
+                 block_table: np.ndarray):
+        self.cache = np.zeros((num_blocks, heads, block_size, head_dim), dtype=np.uint8)
+        self.scales = np.ascontiguousarray(scales, dtype=np.float32)
+        self.block_table = np.ascontiguousarray(block_table, dtype=np.int32)
+        self.B, self.H, self.D = block_size, heads, head_dim
+
+    def write(self, kv: np.ndarray, t0: int):
+        """Quantise kv [T, H, D] into positions t0 .. t0 + T - 1."""
+        lib = _load()
+        kv = np.ascontiguousarray(kv, dtype=np.float32)
+        T = kv.shape[0]
+        if (t0 + T + self.B - 1) // self.B > len(self.block_table):
+            raise ValueError("block table too short")
+        _check(lib.orc_kv_write_paged(_ptr(kv, ctypes.c_float), t0, T, self.H, self.D, _ptr(self.scales, ctypes.c_float),
+                                      self.B, self.block_table.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                      self.cache.shape[0], _ptr(self.cache, ctypes.c_uint8)))
+
+    def gather(self, ctx: int) -> np.ndarray:
+        """Codes of positions 0 .. ctx - 1 as [ctx, H, D] (logical order)."""
+        idx = np.arange(ctx)
+        return self.cache[self.block_table[idx // self.B], :, idx % self.B, :]
+
+
+def attention_paged(q: np.ndarray, k: PagedKV, v: PagedKV, ctx: int) -> np.ndarray:
+    """Causal attention of q [Tq, Hq, D] at positions ctx - Tq .. ctx - 1
+    over the dequantised paged K / V caches (binary64)."""
+    lib = _load()
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    Tq, Hq, D = q.shape
+    if not (np.array_equal(k.block_table, v.block_table) and k.B == v.B and k.H == v.H and k.D == D == v.D):
+        raise ValueError("K and V caches must share block size, table and shape")
+    out = np.empty((Tq, Hq, D), dtype=np.float64)
+    scratch = np.empty(max(ctx, 1), dtype=np.float64)
+    bt = k.block_table.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    _check(lib.orc_attention_paged(_ptr(q, ctypes.c_double), Tq, Hq, D, _ptr(k.cache, ctypes.c_uint8),
+                                   _ptr(v.cache, ctypes.c_uint8), _ptr(k.scales, ctypes.c_float),
+                                   _ptr(v.scales, ctypes.c_float), k.H, k.B, bt, k.cache.shape[0], ctx,
+                                   _ptr(out, ctypes.c_double), _ptr(scratch, ctypes.c_double)))
+    return out

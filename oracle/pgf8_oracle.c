@@ -467,3 +467,121 @@ void orc_silu_mul(const double *g, const double *u, int64_t count, double *h)
     for (int64_t i = 0; i < count; ++i)
         h[i] = g[i] / (1.0 + exp(-g[i])) * u[i];
 }
+
+/* ------------------------------------------------------------------ */
+/* FP8 KV cache.                                                       */
+/*                                                                     */
+/* [FP8-4060] stores K/V in FP8 (half the cache: 96 -> 48 MB at 1024   */
+/* tokens, ~1 % conversion cost); [CPP-FP8] §3.2 pages the cache in    */
+/* blocks of 16 tokens handed out by a central allocator and keeps the */
+/* blocks in FP8, §3.3 computes context attention in the FP8 dataflow  */
+/* (kv_cache_dtype fp8).  No formula or scale granularity is printed.  */
+/* Readings:                                                           */
+/*   scales     one per KV head, MINMAX over calibration data:         */
+/*              s_h = fl32(max |k[., h, .]| / 448), 1 when 0;          */
+/*   codes      E4M3_satfinite_RNE(fl32(k / s_h)), as the rows above;  */
+/*   layout     cache[block][kv_head][slot][d], slot = token % B, the  */
+/*              block of a token from a block table (token / B -> id); */
+/*   attention  per query head h (KV head h / G with G = Hq / Hkv):    */
+/*              out = sum_t softmax_t(q . k_t / sqrt(D)) v_t over the  */
+/*              dequantised cache, keys t <= the query's position,     */
+/*              evaluated in binary64 (q unquantised).                 */
+/* ------------------------------------------------------------------ */
+
+/* s[h] for kv [T, H, D] binary32 (contiguous). */
+int orc_kv_calibrate_scales(const float *kv, int64_t T, int64_t H, int64_t D, float *s)
+{
+    if (T < 0 || H < 1 || D < 1)
+        return ORC_ERR_ARG;
+    for (int64_t h = 0; h < H; ++h) {
+        float amax = 0.0f;
+        for (int64_t t = 0; t < T; ++t)
+            for (int64_t d = 0; d < D; ++d) {
+                float a = fabsf(kv[(t * H + h) * D + d]);
+                if (!isfinite(a))
+                    return ORC_ERR_NONFINITE;
+                if (a > amax)
+                    amax = a;
+            }
+        s[h] = scale_of_amax(amax);
+    }
+    return ORC_OK;
+}
+
+/* Writes tokens [t0, t0 + T) of kv [T, H, D] into the paged cache
+ * [num_blocks, H, B, D] through block_table (logical block -> physical). */
+int orc_kv_write_paged(const float *kv, int64_t t0, int64_t T, int64_t H, int64_t D, const float *s, int64_t B,
+                       const int32_t *block_table, int64_t num_blocks, uint8_t *cache)
+{
+    if (t0 < 0 || T < 0 || H < 1 || D < 1 || B < 1)
+        return ORC_ERR_ARG;
+    for (int64_t t = 0; t < T; ++t) {
+        int64_t pos = t0 + t;
+        int64_t blk = block_table[pos / B];
+        if (blk < 0 || blk >= num_blocks)
+            return ORC_ERR_ARG;
+        int64_t slot = pos % B;
+        for (int64_t h = 0; h < H; ++h) {
+            if (!(s[h] > 0.0f) || !isfinite(s[h]))
+                return ORC_ERR_BADSCALE;
+            for (int64_t d = 0; d < D; ++d) {
+                float x = kv[(t * H + h) * D + d];
+                if (!isfinite(x))
+                    return ORC_ERR_NONFINITE;
+                float q = x / s[h];
+                cache[((blk * H + h) * B + slot) * D + d] = orc_e4m3_encode(q);
+            }
+        }
+    }
+    return ORC_OK;
+}
+
+/* Attention of Tq queries q [Tq, Hq, D] (binary64) at positions
+ * ctx - Tq .. ctx - 1 over the first ctx tokens of the paged K / V caches
+ * [num_blocks, Hkv, B, D]; causal: query i sees positions <= ctx - Tq + i.
+ * out [Tq, Hq, D] binary64. */
+int orc_attention_paged(const double *q, int64_t Tq, int64_t Hq, int64_t D, const uint8_t *kcache,
+                        const uint8_t *vcache, const float *sk, const float *sv, int64_t Hkv, int64_t B,
+                        const int32_t *block_table, int64_t num_blocks, int64_t ctx, double *out, double *scratch)
+{
+    if (Tq < 1 || Hq < 1 || D < 1 || Hkv < 1 || Hq % Hkv != 0 || B < 1 || ctx < Tq)
+        return ORC_ERR_ARG;
+    const int64_t G = Hq / Hkv;
+    const double inv = 1.0 / sqrt((double)D);
+    for (int64_t i = 0; i < Tq; ++i) {
+        const int64_t last = ctx - Tq + i;   /* causal: keys 0 .. last */
+        for (int64_t h = 0; h < Hq; ++h) {
+            const int64_t hk = h / G;
+            const double *qv = q + (i * Hq + h) * D;
+            double mx = -INFINITY;
+            for (int64_t t = 0; t <= last; ++t) {
+                int64_t blk = block_table[t / B];
+                if (blk < 0 || blk >= num_blocks)
+                    return ORC_ERR_ARG;
+                const uint8_t *kr = kcache + ((blk * Hkv + hk) * B + t % B) * D;
+                double dot = 0.0;
+                for (int64_t d = 0; d < D; ++d)
+                    dot += qv[d] * orc_e4m3_decode(kr[d]) * (double)sk[hk];
+                scratch[t] = dot * inv;
+                if (scratch[t] > mx)
+                    mx = scratch[t];
+            }
+            double den = 0.0;
+            for (int64_t t = 0; t <= last; ++t) {
+                scratch[t] = exp(scratch[t] - mx);
+                den += scratch[t];
+            }
+            double *o = out + (i * Hq + h) * D;
+            for (int64_t d = 0; d < D; ++d)
+                o[d] = 0.0;
+            for (int64_t t = 0; t <= last; ++t) {
+                int64_t blk = block_table[t / B];
+                const uint8_t *vr = vcache + ((blk * Hkv + hk) * B + t % B) * D;
+                const double p = scratch[t] / den;
+                for (int64_t d = 0; d < D; ++d)
+                    o[d] += p * orc_e4m3_decode(vr[d]) * (double)sv[hk];
+            }
+        }
+    }
+    return ORC_OK;
+}
