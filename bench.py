@@ -175,13 +175,20 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- profiled traffic
+# The GEMM kernels' sources (and the helpers they include): what a DRAM
+# traffic record describes.  The record also names the kernel configuration
+# it was taken on.
+GEMM_SOURCES = ("gemm.cuh", "gemm_2sm.cuh", "gemm_persistent.cuh", "gemm_streamk.cuh", "quantize.cuh",
+                "sm100_ptx.cuh")
+
+
 def kernel_sources_hash() -> str:
-    """Short hash of the CUDA sources: profiled counters only describe the
-    kernels they were taken on."""
+    """Short hash of the GEMM kernels' CUDA sources: profiled counters only
+    describe the kernels they were taken on."""
     import hashlib
     csrc = os.path.join(ROOT, "precision_gemm_fp8_b200", "csrc")
     h = hashlib.sha256()
-    for f in sorted(os.listdir(csrc)):
+    for f in GEMM_SOURCES:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(hashlib.sha256(fh.read()).hexdigest().encode() + b"  " + f.encode() + b"\n")
     return h.hexdigest()[:12]

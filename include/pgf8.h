@@ -162,6 +162,29 @@ pgf8_status pgf8_fp8_linear_ex(const uint8_t *aq, const float *sa, int64_t M, in
 size_t pgf8_fp8_linear_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /* ------------------------------------------------------------------------
+ * FP8 paged KV cache ("7B on an RTX 4060 with FP8": K/V stored in FP8;
+ * "C++ and FP8" §3.2: a paged cache of token blocks kept in FP8).
+ *
+ * pgf8_fp8_kv_write_paged: writes `tokens` K (or V) rows of
+ *   kv [tokens, heads, head_dim] (f32, f16 or bf16; token stride ldkv
+ *   elements, so a slice of the QKV projection's output can be passed as
+ *   it is) at positions first_pos .. first_pos + tokens - 1 into
+ *   cache [num_blocks, heads, block_size, head_dim] (E4M3 codes): position
+ *   p goes to block block_table[p / block_size], slot p % block_size.
+ *   Codes E4M3(RN(x / scales[h])), saturating (scales [heads] f32, one per
+ *   KV head, > 0).  The block table (device int32 [table_len]) must cover
+ *   the positions (else PGF8_ERR_INVALID_ARG before any launch); entries
+ *   outside [0, num_blocks) are skipped and counted per token into
+ *   *bad_blocks (device int32, may be NULL): nothing is written outside the
+ *   cache.  head_dim % 16 == 0; kv, cache 16-byte aligned.  flags:
+ *   PGF8_FLAG_OVERLAP_PREVIOUS as for the quantisation calls.
+ * ---------------------------------------------------------------------- */
+pgf8_status pgf8_fp8_kv_write_paged(const void *kv, pgf8_dtype dt, int64_t tokens, int64_t heads, int64_t head_dim,
+                                    int64_t ldkv, const float *scales, int64_t first_pos, int64_t block_size,
+                                    const int32_t *block_table, int64_t table_len, int64_t num_blocks,
+                                    uint8_t *cache, int32_t *bad_blocks, int32_t flags, void *stream);
+
+/* ------------------------------------------------------------------------
  * Normalisation or gate fused with the per-token quantisation ("7B on an
  * RTX 4060 with FP8", computation graph §2.1: LayerNorm fused with the QKV
  * projection's input).  The normalised / gated values never go to memory;

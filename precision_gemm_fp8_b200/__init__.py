@@ -57,6 +57,8 @@ _optp = ctypes.POINTER(LinearOpts)
 _SIGS = {
     "pgf8_fp8_quantize_rows": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _i32, _vp], _i32),
     "pgf8_fp8_amax_accumulate": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp], _i32),
+    "pgf8_fp8_kv_write_paged": ([_vp, _i32, _i64, _i64, _i64, _i64, _vp, _i64, _i64, _vp, _i64, _i64, _vp, _vp, _i32,
+                                 _vp], _i32),
     "pgf8_fp8_norm_quantize": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, ctypes.c_float, _vp, _vp, _i32, _vp], _i32),
     "pgf8_fp8_silu_mul_quantize": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _i32, _vp], _i32),
     "pgf8_fp8_quantize_tensor": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _i32, _vp], _i32),
@@ -183,6 +185,29 @@ def fp8_quantize_rows(x: torch.Tensor, q: torch.Tensor | None = None, scales: to
     _check(lib.pgf8_fp8_quantize_rows(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(q), _ptr(scales),
                                       mode, _stream(stream)), "fp8_quantize_rows")
     return q, scales
+
+
+def fp8_kv_write_paged(kv: torch.Tensor, scales: torch.Tensor, cache: torch.Tensor, block_table: torch.Tensor,
+                       first_pos: int, bad_blocks: torch.Tensor | None = None, flags: int = 0, stream=None):
+    """Quantise kv [tokens, heads, head_dim] (f32 / f16 / bf16; token rows may
+    be strided) into the paged E4M3 cache [num_blocks, heads, block_size,
+    head_dim] at positions first_pos.. through block_table (int32)."""
+    tokens, heads, head_dim = kv.shape
+    if kv.stride(2) != 1 or kv.stride(1) != head_dim:
+        raise ValueError("kv heads must be contiguous within a token")
+    code = {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}.get(kv.dtype)
+    if code is None:
+        raise TypeError(f"unsupported kv dtype {kv.dtype}")
+    num_blocks, ch, block_size, cd = cache.shape
+    if (ch, cd) != (heads, head_dim) or cache.dtype != torch.uint8 or not cache.is_contiguous():
+        raise ValueError("cache must be a contiguous uint8 [num_blocks, heads, block_size, head_dim] tensor")
+    if block_table.dtype != torch.int32 or not block_table.is_contiguous():
+        raise ValueError("block_table must be a contiguous int32 tensor")
+    _check(lib.pgf8_fp8_kv_write_paged(_ptr(kv), code, tokens, heads, head_dim, kv.stride(0), _ptr(scales), first_pos,
+                                       block_size, _ptr(block_table), block_table.numel(), num_blocks, _ptr(cache),
+                                       None if bad_blocks is None else _ptr(bad_blocks), flags, _stream(stream)),
+           "fp8_kv_write_paged")
+    return cache
 
 
 def fp8_norm_quantize(x: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor | None = None, eps: float = 1e-5,

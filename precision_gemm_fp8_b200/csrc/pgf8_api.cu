@@ -10,6 +10,7 @@
 
 #include "pgf8.h"
 #include "gemm.cuh"
+#include "kvcache.cuh"
 #include "gemm_persistent.cuh"
 #include "gemm_streamk.cuh"
 #include "gemm_2sm.cuh"
@@ -793,6 +794,44 @@ pgf8_status pgf8_fp8_silu_mul_quantize(const void *gu, pgf8_dtype gdt, int64_t r
                             ldg, q, scales);
     return launch_quant(silu_mul_quantize_kernel<__nv_bfloat16>, grid, cs, pdl,
                         static_cast<const __nv_bfloat16 *>(gu), inter, ldg, q, scales);
+}
+
+pgf8_status pgf8_fp8_kv_write_paged(const void *kv, pgf8_dtype dt, int64_t tokens, int64_t heads, int64_t head_dim,
+                                    int64_t ldkv, const float *scales, int64_t first_pos, int64_t block_size,
+                                    const int32_t *block_table, int64_t table_len, int64_t num_blocks,
+                                    uint8_t *cache, int32_t *bad_blocks, int32_t flags, void *stream)
+{
+    if (tokens < 0 || heads < 1 || head_dim < 16 || block_size < 1 || first_pos < 0 || num_blocks < 1 ||
+        table_len < 1 || ldkv < heads * head_dim || tokens > (1ll << 40))
+        return PGF8_ERR_INVALID_ARG;
+    if (tokens == 0)
+        return PGF8_OK;
+    if (!kv || !scales || !block_table || !cache)
+        return PGF8_ERR_INVALID_ARG;
+    if ((first_pos + tokens - 1) / block_size >= table_len)
+        return PGF8_ERR_INVALID_ARG;   // positions beyond the block table
+    if (dt != PGF8_F32 && dt != PGF8_F16 && dt != PGF8_BF16)
+        return PGF8_ERR_UNSUPPORTED;
+    const int eb = dt == PGF8_F32 ? 4 : 2;
+    if (head_dim % 16 != 0 || (ldkv * eb) % 16 != 0 || !aligned16(kv) || !aligned16(cache) || !aligned4(scales) ||
+        !aligned4(block_table) || (bad_blocks && !aligned4(bad_blocks)))
+        return PGF8_ERR_ALIGNMENT;
+    const int64_t items = tokens * heads * (head_dim / 16);
+    const int64_t want = (items + kQuantThreads - 1) / kQuantThreads;
+    const unsigned grid = static_cast<unsigned>(want < num_sms() * 8 ? want : num_sms() * 8);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const int pdl = (flags & PGF8_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
+    if (dt == PGF8_F32)
+        return launch_quant(kv_write_paged_kernel<float>, grid, cs, pdl, static_cast<const float *>(kv), tokens,
+                            heads, head_dim, ldkv, scales, first_pos, block_size, block_table, num_blocks, cache,
+                            bad_blocks);
+    if (dt == PGF8_F16)
+        return launch_quant(kv_write_paged_kernel<__half>, grid, cs, pdl, static_cast<const __half *>(kv), tokens,
+                            heads, head_dim, ldkv, scales, first_pos, block_size, block_table, num_blocks, cache,
+                            bad_blocks);
+    return launch_quant(kv_write_paged_kernel<__nv_bfloat16>, grid, cs, pdl, static_cast<const __nv_bfloat16 *>(kv),
+                        tokens, heads, head_dim, ldkv, scales, first_pos, block_size, block_table, num_blocks, cache,
+                        bad_blocks);
 }
 
 pgf8_status pgf8_fp8_quantize_rows(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,

@@ -197,3 +197,18 @@ def test_per_tensor_scaling_argument_checks():
     assert qd(a16, pg.F32, 2, 16, 16, a16, None, a16, 1024, a16 + 8, 0, 0, None) == pg.ERR_ALIGNMENT
     assert qd(a16, pg.F32, 0, 16, 16, a16, None, a16, 1024, a16, 0, 0, None) == pg.ERR_INVALID_ARG   # a step needs rows
     assert qd(a16, pg.F32, 2, 16, 16, a16, None, a16, 1024, a16, -1, 0, None) == pg.ERR_INVALID_ARG  # step < 0
+
+
+def test_kv_write_paged_argument_checks():
+    buf = (ctypes.c_uint8 * 8192)()
+    a16 = (ctypes.addressof(buf) + 15) // 16 * 16
+    f = pg.lib.pgf8_fp8_kv_write_paged
+    # (kv, dt, tokens, heads, head_dim, ldkv, scales, first_pos, block_size, table, table_len, num_blocks, cache, bad, flags, stream)
+    assert f(a16, pg.F32, 0, 2, 64, 128, a16, 0, 16, a16, 1, 1, a16, None, 0, None) == pg.OK           # nothing to write
+    assert f(a16, pg.F32, 20, 2, 64, 128, a16, 0, 16, a16, 1, 2, a16, None, 0, None) == pg.ERR_INVALID_ARG  # table too short
+    assert f(a16, pg.F32, 4, 2, 8, 16, a16, 0, 16, a16, 1, 1, a16, None, 0, None) == pg.ERR_INVALID_ARG    # head_dim < 16
+    assert f(a16, pg.F32, 4, 2, 64, 100, a16, 0, 16, a16, 1, 1, a16, None, 0, None) == pg.ERR_INVALID_ARG  # ldkv < H*D
+    assert f(a16, pg.F32, 4, 2, 40, 80, a16, 0, 16, a16, 1, 1, a16, None, 0, None) == pg.ERR_ALIGNMENT    # D % 16
+    assert f(a16 + 4, pg.F32, 4, 2, 64, 128, a16, 0, 16, a16, 1, 1, a16, None, 0, None) == pg.ERR_ALIGNMENT
+    assert f(a16, 7, 4, 2, 64, 128, a16, 0, 16, a16, 1, 1, a16, None, 0, None) == pg.ERR_UNSUPPORTED
+    assert f(a16, pg.F32, 4, 2, 64, 128, None, 0, 16, a16, 1, 1, a16, None, 0, None) == pg.ERR_INVALID_ARG
