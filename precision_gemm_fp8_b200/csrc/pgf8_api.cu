@@ -628,16 +628,9 @@ static pgf8_status check_tensor_args(const void *x, pgf8_dtype xdt, int64_t rows
     return PGF8_OK;
 }
 
-template <typename T, typename... Args>
-static pgf8_status launch_simple(void (*kernel)(Args...), unsigned grid, cudaStream_t st, Args... args)
-{
-    kernel<<<grid, kQuantThreads, 0, st>>>(args...);
-    cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? PGF8_OK : cuda_fail(e);
-}
-
-// The same, optionally with programmatic stream serialization (the kernel
-// waits on the grid dependency before its first read).
+// Launches a 256-thread quantisation-family kernel, optionally with
+// programmatic stream serialization (the kernel waits on the grid
+// dependency before its first read).
 template <typename... Args>
 static pgf8_status launch_quant(void (*kernel)(Args...), unsigned grid, cudaStream_t st, int pdl, Args... args)
 {
@@ -681,10 +674,10 @@ pgf8_status pgf8_fp8_amax_accumulate(const void *x, pgf8_dtype xdt, int64_t rows
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     unsigned *bits = reinterpret_cast<unsigned *>(amax);
     if (xdt == PGF8_F32)
-        return launch_simple<float>(amax_accumulate_kernel<float>, grid, cs, static_cast<const float *>(x), rows,
-                                    cols, ldx, bits);
-    return launch_simple<__half>(amax_accumulate_kernel<__half>, grid, cs, static_cast<const __half *>(x), rows, cols,
-                                 ldx, bits);
+        return launch_quant(amax_accumulate_kernel<float>, grid, cs, 0, static_cast<const float *>(x), rows, cols,
+                            ldx, bits);
+    return launch_quant(amax_accumulate_kernel<__half>, grid, cs, 0, static_cast<const __half *>(x), rows, cols, ldx,
+                        bits);
 }
 
 pgf8_status pgf8_fp8_quantize_tensor(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
@@ -718,9 +711,9 @@ pgf8_status pgf8_delayed_state_init(pgf8_delayed_state *state, float *history, i
     if ((reinterpret_cast<uintptr_t>(state) & 15u) != 0 || !aligned4(history))
         return PGF8_ERR_ALIGNMENT;
     const unsigned grid = static_cast<unsigned>((history_len + kQuantThreads - 1) / kQuantThreads);
-    return launch_simple<float>(delayed_init_kernel, grid < 1024u ? grid : 1024u, static_cast<cudaStream_t>(stream),
-                                history, static_cast<int>(history_len), reinterpret_cast<DelayedState *>(state),
-                                initial_scale);
+    return launch_quant(delayed_init_kernel, grid < 1024u ? grid : 1024u, static_cast<cudaStream_t>(stream), 0,
+                        history, static_cast<int>(history_len), reinterpret_cast<DelayedState *>(state),
+                        initial_scale);
 }
 
 pgf8_status pgf8_fp8_quantize_delayed(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
