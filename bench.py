@@ -759,6 +759,63 @@ def run_single(args):
                       "tflops": round(2.0 * M * N * K / (us * 1e-6) / 1e12, 2)}), flush=True)
 
 
+def run_attention(args):
+    """Decode attention over the FP8 paged cache, launched eagerly `warmup +
+    steps` times (e.g. --attention 64,64,8,128,4096 = seqs, query heads, KV
+    heads, head_dim, context: a 70B-shaped decode batch).  Caches of
+    N(0,1) K / V written by the cache writer with per-head scales 4.5/448,
+    blocks of 16 positions scattered by a seeded permutation; the caches
+    (2 x seqs x context x KV heads x head_dim bytes) exceed L2 at the
+    intended sizes, so every call streams them from HBM."""
+    import torch
+    import precision_gemm_fp8_b200 as pg
+
+    seqs, hq, hkv, d, ctx = (int(v) for v in args.attention.split(","))
+    B = 16
+    dev = torch.device("cuda", 0)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234)
+    nblk = (ctx + B - 1) // B
+    num_blocks = seqs * nblk
+    tables = torch.randperm(num_blocks, generator=gen, device=dev).to(torch.int32).view(seqs, nblk)
+    kc = torch.zeros((num_blocks, hkv, B, d), dtype=torch.uint8, device=dev)
+    vc = torch.zeros_like(kc)
+    sk = torch.full((hkv,), 4.5 / 448.0, dtype=torch.float32, device=dev)
+    sv = sk.clone()
+    for s in range(seqs):
+        for cache, sc in ((kc, sk), (vc, sv)):
+            kv = torch.randn((ctx, hkv, d), generator=gen, device=dev)
+            pg.fp8_kv_write_paged(kv, sc, cache, tables[s].contiguous(), 0)
+    q = torch.randn((seqs, hq, d), generator=gen, device=dev)
+    lens = torch.full((seqs,), ctx, dtype=torch.int32, device=dev)
+    out = torch.empty((seqs, hq, d), dtype=torch.float32, device=dev)
+    nsplit, chunk = pg.fp8_attention_decode_plan(seqs, hq, hkv, d, ctx, args.split_k)
+    ws_bytes = pg.lib.pgf8_fp8_attention_decode_workspace_size(seqs, hq, hkv, d, ctx, args.split_k)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    fn = lambda: pg.fp8_attention_decode_paged(q, kc, vc, sk, sv, tables, lens, ctx, out=out,  # noqa: E731
+                                               splits=args.split_k, workspace=ws)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        fn()
+    t1.record()
+    torch.cuda.synchronize()
+    if pg.device_status() != pg.OK:
+        raise RuntimeError("device error word raised")
+    us = 1e3 * t0.elapsed_time(t1) / args.steps
+    kv_bytes = 2 * seqs * ctx * hkv * d
+    alg = kv_bytes + seqs * hq * d * 8 + seqs * nblk * 4
+    peaks, src = _load_peaks()
+    gbs = alg / (us * 1e-6) / 1e9
+    print(json.dumps({"attention": args.attention, "us_per_call": round(us, 3), "nsplit": nsplit, "chunk": chunk,
+                      "algorithmic_bytes": alg, "kv_bytes": kv_bytes, "gbs": round(gbs, 1),
+                      "frac_hbm": round(gbs / float(peaks["hbm_gbs"]), 3), "peak_source": src}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -776,6 +833,9 @@ def main():
     ap.add_argument("--fused-quant", action="store_true",
                     help="quantise dynamic activations inside the skinny GEMM where its kernel allows it")
     ap.add_argument("--single", default=None, help="kind,M,K,N: time (or profile) one layer eagerly")
+    ap.add_argument("--attention", default=None,
+                    help="seqs,q_heads,kv_heads,head_dim,context: time (or profile) the FP8 paged decode attention "
+                         "eagerly (--split-k caps its context chunks)")
     ap.add_argument("--path", type=int, default=0)
     ap.add_argument("--split-k", type=int, default=0)
     ap.add_argument("--tile-n", type=int, default=0)
@@ -785,6 +845,9 @@ def main():
                  "--scaling nor --fused-quant")
     if args.single:
         run_single(args)
+        return
+    if args.attention:
+        run_attention(args)
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -185,6 +185,69 @@ pgf8_status pgf8_fp8_kv_write_paged(const void *kv, pgf8_dtype dt, int64_t token
                                     uint8_t *cache, int32_t *bad_blocks, int32_t flags, void *stream);
 
 /* ------------------------------------------------------------------------
+ * Decode attention over the FP8 paged KV cache ("7B on an RTX 4060 with
+ * FP8": K/V held in FP8 and dequantised on use; "C++ and FP8" §3.2 paged
+ * cache of 16-token blocks, §3.3 attention in the FP8 dataflow).
+ *
+ * One query row per sequence: the token being generated, at position
+ * ctx - 1, which sees cached positions 0 .. ctx - 1 (ctx = context_lens[s]).
+ * For query head h over KV head hk = h / (q_heads / kv_heads):
+ *   score_t = (q[s,h,:] . dec(K_t)) * k_scales[hk] / sqrt(head_dim)
+ *   out[s,h,:] = (sum_t softmax(score)_t * dec(V_t)) * v_scales[hk]
+ * with dec the E4M3 value of a code and K_t / V_t the cache rows of
+ * position t: block block_tables[s * table_stride + t / block_size], slot
+ * t % block_size.  Computed in binary32 (q widened, scores and softmax in
+ * binary32 with exp2f, outputs rounded once to out_dt); ctx == 0 gives 0.
+ *
+ * q:    [seqs, q_heads, head_dim], f32 / f16 / bf16, sequence stride ldq
+ *       elements (a slice of the QKV projection output can be passed).
+ * cache: the K and V caches [num_blocks, kv_heads, block_size, head_dim]
+ *       (as written by pgf8_fp8_kv_write_paged), their per-head scales.
+ *       head_dim 64, 128 or 256; block_size a multiple of 16; q_heads a
+ *       multiple of kv_heads.
+ * block_tables: device int32 [seqs, table_stride]; context_lens: device
+ *       int32 [seqs].  max_context (host) bounds every context length and
+ *       must fit the table (max_context <= table_stride * block_size); a
+ *       longer (or negative) length is clamped to it and counted.
+ * out:  [seqs, q_heads, head_dim], out_dt, sequence stride ldo elements.
+ * splits: 0 chooses the number of context chunks from the grid
+ *       (pgf8_fp8_attention_decode_plan reports it); > 0 caps it.  With more
+ *       than one chunk a second kernel merges the chunks in chunk order,
+ *       through `workspace` (pgf8_fp8_attention_decode_workspace_size bytes
+ *       for the same arguments, 4-byte aligned; may be NULL when that is 0).
+ * errors: device int32 or NULL.  Block-table entries outside
+ *       [0, num_blocks) are counted (once per 16 positions) and those
+ *       positions left out; clamped context lengths are counted once per
+ *       sequence.  Nothing outside the cache is read.
+ * Alignment: caches 16 bytes; q and out their element size; scales, tables,
+ * lengths and errors 4 bytes.  flags: PGF8_FLAG_OVERLAP_PREVIOUS.
+ * seqs == 0 is a no-op.  Results do not depend on scheduling.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+    const uint8_t *k_cache;   /* [num_blocks, kv_heads, block_size, head_dim] E4M3 codes */
+    const uint8_t *v_cache;   /* same shape */
+    const float *k_scales;    /* [kv_heads] */
+    const float *v_scales;    /* [kv_heads] */
+    int64_t num_blocks;
+    int64_t kv_heads;
+    int64_t block_size;
+    int64_t head_dim;
+} pgf8_paged_kv_cache;
+
+pgf8_status pgf8_fp8_attention_decode_plan(int64_t seqs, int64_t q_heads, int64_t kv_heads, int64_t head_dim,
+                                           int64_t max_context, int64_t splits, int64_t *nsplit, int64_t *chunk);
+
+size_t pgf8_fp8_attention_decode_workspace_size(int64_t seqs, int64_t q_heads, int64_t kv_heads, int64_t head_dim,
+                                                int64_t max_context, int64_t splits);
+
+pgf8_status pgf8_fp8_attention_decode_paged(const void *q, pgf8_dtype q_dt, int64_t seqs, int64_t q_heads,
+                                            int64_t ldq, const pgf8_paged_kv_cache *cache,
+                                            const int32_t *block_tables, int64_t table_stride,
+                                            const int32_t *context_lens, int64_t max_context, void *out,
+                                            pgf8_dtype out_dt, int64_t ldo, int64_t splits, void *workspace,
+                                            size_t workspace_bytes, int32_t *errors, int32_t flags, void *stream);
+
+/* ------------------------------------------------------------------------
  * Normalisation or gate fused with the per-token quantisation ("7B on an
  * RTX 4060 with FP8", computation graph §2.1: LayerNorm fused with the QKV
  * projection's input).  The normalised / gated values never go to memory;

@@ -41,6 +41,12 @@ class LinearOpts(ctypes.Structure):
                 ("flags", ctypes.c_int32)]
 
 
+class PagedKVCache(ctypes.Structure):
+    _fields_ = [("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p), ("k_scales", ctypes.c_void_p),
+                ("v_scales", ctypes.c_void_p), ("num_blocks", ctypes.c_int64), ("kv_heads", ctypes.c_int64),
+                ("block_size", ctypes.c_int64), ("head_dim", ctypes.c_int64)]
+
+
 class Fp8Layer(ctypes.Structure):
     _fields_ = [("x", ctypes.c_void_p), ("xdt", ctypes.c_int32), ("reserved", ctypes.c_int32),
                 ("M", ctypes.c_int64), ("K", ctypes.c_int64), ("ldx", ctypes.c_int64), ("N", ctypes.c_int64),
@@ -59,6 +65,10 @@ _SIGS = {
     "pgf8_fp8_amax_accumulate": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp], _i32),
     "pgf8_fp8_kv_write_paged": ([_vp, _i32, _i64, _i64, _i64, _i64, _vp, _i64, _i64, _vp, _i64, _i64, _vp, _vp, _i32,
                                  _vp], _i32),
+    "pgf8_fp8_attention_decode_plan": ([_i64, _i64, _i64, _i64, _i64, _i64, _vp, _vp], _i32),
+    "pgf8_fp8_attention_decode_workspace_size": ([_i64, _i64, _i64, _i64, _i64, _i64], _sz),
+    "pgf8_fp8_attention_decode_paged": ([_vp, _i32, _i64, _i64, _i64, ctypes.POINTER(PagedKVCache), _vp, _i64, _vp,
+                                         _i64, _vp, _i32, _i64, _i64, _vp, _sz, _vp, _i32, _vp], _i32),
     "pgf8_fp8_norm_quantize": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, ctypes.c_float, _vp, _vp, _i32, _vp], _i32),
     "pgf8_fp8_silu_mul_quantize": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _i32, _vp], _i32),
     "pgf8_fp8_quantize_tensor": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _i32, _vp], _i32),
@@ -208,6 +218,58 @@ def fp8_kv_write_paged(kv: torch.Tensor, scales: torch.Tensor, cache: torch.Tens
                                        None if bad_blocks is None else _ptr(bad_blocks), flags, _stream(stream)),
            "fp8_kv_write_paged")
     return cache
+
+
+def fp8_attention_decode_plan(seqs: int, q_heads: int, kv_heads: int, head_dim: int, max_context: int,
+                              splits: int = 0) -> tuple[int, int]:
+    """(number of context chunks, positions per chunk) the decode attention
+    uses for these sizes (host only)."""
+    ns, ch = ctypes.c_int64(0), ctypes.c_int64(0)
+    _check(lib.pgf8_fp8_attention_decode_plan(seqs, q_heads, kv_heads, head_dim, max_context, splits,
+                                              ctypes.byref(ns), ctypes.byref(ch)), "fp8_attention_decode_plan")
+    return ns.value, ch.value
+
+
+def fp8_attention_decode_paged(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                               k_scales: torch.Tensor, v_scales: torch.Tensor, block_tables: torch.Tensor,
+                               context_lens: torch.Tensor, max_context: int, out: torch.Tensor | None = None,
+                               out_dtype: torch.dtype = torch.float32, splits: int = 0,
+                               workspace: torch.Tensor | None = None, errors: torch.Tensor | None = None,
+                               flags: int = 0, stream=None) -> torch.Tensor:
+    """Decode attention of q [seqs, q_heads, head_dim] (one query per
+    sequence, at its last position) over the paged E4M3 K / V caches
+    [num_blocks, kv_heads, block_size, head_dim] with per-KV-head scales,
+    block_tables int32 [seqs, table_stride], context_lens int32 [seqs].
+    Returns out [seqs, q_heads, head_dim]."""
+    seqs, q_heads, head_dim = q.shape
+    if q.stride(2) != 1 or q.stride(1) != head_dim:
+        raise ValueError("q heads must be contiguous within a sequence")
+    num_blocks, kv_heads, block_size, cd = k_cache.shape
+    for c in (k_cache, v_cache):
+        if c.shape != k_cache.shape or c.dtype != torch.uint8 or not c.is_contiguous() or cd != head_dim:
+            raise ValueError("caches must be contiguous uint8 [num_blocks, kv_heads, block_size, head_dim] tensors")
+    if block_tables.dtype != torch.int32 or block_tables.dim() != 2 or block_tables.stride(1) != 1:
+        raise ValueError("block_tables must be an int32 [seqs, table_stride] tensor with contiguous rows")
+    if context_lens.dtype != torch.int32 or not context_lens.is_contiguous():
+        raise ValueError("context_lens must be a contiguous int32 tensor")
+    if out is None:
+        out = torch.empty((seqs, q_heads, head_dim), dtype=out_dtype, device=q.device)
+    if out.stride(2) != 1 or out.stride(1) != head_dim:
+        raise ValueError("out heads must be contiguous within a sequence")
+    codes = {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}
+    if q.dtype not in codes or out.dtype not in codes:
+        raise TypeError("q and out must be float32, float16 or bfloat16")
+    need = lib.pgf8_fp8_attention_decode_workspace_size(seqs, q_heads, kv_heads, head_dim, max_context, splits)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    cache = PagedKVCache(_ptr(k_cache), _ptr(v_cache), _ptr(k_scales), _ptr(v_scales), num_blocks, kv_heads,
+                         block_size, head_dim)
+    _check(lib.pgf8_fp8_attention_decode_paged(
+        _ptr(q), codes[q.dtype], seqs, q_heads, q.stride(0), ctypes.byref(cache), _ptr(block_tables),
+        block_tables.stride(0), _ptr(context_lens), max_context, _ptr(out), codes[out.dtype], out.stride(0), splits,
+        _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
+        None if errors is None else _ptr(errors), flags, _stream(stream)), "fp8_attention_decode_paged")
+    return out
 
 
 def fp8_norm_quantize(x: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor | None = None, eps: float = 1e-5,

@@ -11,6 +11,7 @@
 #include "pgf8.h"
 #include "gemm.cuh"
 #include "kvcache.cuh"
+#include "attention.cuh"
 #include "gemm_persistent.cuh"
 #include "gemm_streamk.cuh"
 #include "gemm_2sm.cuh"
@@ -628,16 +629,16 @@ static pgf8_status check_tensor_args(const void *x, pgf8_dtype xdt, int64_t rows
     return PGF8_OK;
 }
 
-// Launches a 256-thread quantisation-family kernel, optionally with
-// programmatic stream serialization (the kernel waits on the grid
-// dependency before its first read).
+// Launches a kernel, optionally with programmatic stream serialization
+// (the kernel waits on the grid dependency before its first read).
 template <typename... Args>
-static pgf8_status launch_quant(void (*kernel)(Args...), unsigned grid, cudaStream_t st, int pdl, Args... args)
+static pgf8_status launch_grid(void (*kernel)(Args...), dim3 grid, dim3 block, cudaStream_t st, int pdl,
+                               Args... args)
 {
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kQuantThreads);
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     if (pdl) {
@@ -648,6 +649,104 @@ static pgf8_status launch_quant(void (*kernel)(Args...), unsigned grid, cudaStre
     }
     cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
     return e == cudaSuccess ? PGF8_OK : cuda_fail(e);
+}
+
+// A 256-thread quantisation-family kernel on a 1-D grid.
+template <typename... Args>
+static pgf8_status launch_quant(void (*kernel)(Args...), unsigned grid, cudaStream_t st, int pdl, Args... args)
+{
+    return launch_grid(kernel, dim3(grid), dim3(kQuantThreads), st, pdl, args...);
+}
+
+// ------------------------------------------------------------------ decode attention plan
+// Query heads per CTA: the largest of 8, 4, 2, 1 that divides the group
+// size Hq / Hkv (the heads of one CTA share every K / V load).
+static int attn_heads_per_cta(int64_t G)
+{
+    for (int gt = 8; gt > 1; gt >>= 1)
+        if (G % gt == 0)
+            return gt;
+    return 1;
+}
+
+constexpr int64_t kAttnCtasPerSm = 4;     // CTAs per SM the automatic split aims for
+constexpr int64_t kAttnMinChunk = 256;    // positions per split at least (automatic split)
+
+struct AttnPlan {
+    int64_t nsplit, chunk;
+    int gt, groups;
+};
+
+// Splits the context [0, max_ctx) into nsplit chunks of `chunk` positions.
+// Automatic (splits == 0): enough chunks for ~kAttnCtasPerSm CTAs per SM,
+// no chunk under kAttnMinChunk positions, chunks a multiple of 64 (whole
+// 16-position steps for each of the 4 warps).  Forced: at most `splits`
+// chunks, a multiple of 16 positions.
+static AttnPlan attn_plan(int64_t seqs, int64_t Hq, int64_t Hkv, int64_t max_ctx, int64_t splits)
+{
+    AttnPlan p;
+    p.gt = attn_heads_per_cta(Hq / Hkv);
+    p.groups = static_cast<int>(Hq / Hkv / p.gt);
+    if (max_ctx <= kAttnStep) {
+        p.nsplit = 1;
+        p.chunk = kAttnStep;
+        return p;
+    }
+    int64_t ns;
+    if (splits > 0) {
+        const int64_t steps = (max_ctx + kAttnStep - 1) / kAttnStep;
+        ns = splits < steps ? splits : steps;
+    } else {
+        const int64_t ctas = seqs * Hkv * p.groups;
+        const int64_t target = static_cast<int64_t>(num_sms()) * kAttnCtasPerSm;
+        const int64_t cap = max_ctx / kAttnMinChunk;   // every chunk >= kAttnMinChunk positions
+        ns = (target + ctas - 1) / ctas;
+        if (ns > cap)
+            ns = cap;
+        if (ns < 1)
+            ns = 1;
+    }
+    const int64_t gran = splits > 0 ? kAttnStep : kAttnStep * kAttnWarps;
+    const int64_t per = (max_ctx + ns - 1) / ns;
+    p.chunk = (per + gran - 1) / gran * gran;
+    p.nsplit = (max_ctx + p.chunk - 1) / p.chunk;
+    return p;
+}
+
+static size_t attn_workspace_bytes(int64_t seqs, int64_t Hq, int64_t D, const AttnPlan &p)
+{
+    return p.nsplit > 1 ? static_cast<size_t>(seqs * Hq * p.nsplit * (D + 2)) * sizeof(float) : 0;
+}
+
+static bool attn_shape_ok(int64_t seqs, int64_t Hq, int64_t Hkv, int64_t D, int64_t max_ctx)
+{
+    return seqs >= 0 && seqs <= 65535 && Hkv >= 1 && Hq >= Hkv && Hq % Hkv == 0 && Hq <= 65535 &&
+           (D == 64 || D == 128 || D == 256) && max_ctx >= 0 && max_ctx <= (1ll << 30);
+}
+
+template <int D, int GT>
+static pgf8_status launch_attn_gt(const AttnDecodeArgs &a, int64_t seqs, cudaStream_t st, int pdl)
+{
+    const dim3 grid(static_cast<unsigned>(a.nsplit), static_cast<unsigned>(a.Hkv * a.groups),
+                    static_cast<unsigned>(seqs));
+    return launch_grid(attn_decode_paged_kernel<D, GT>, grid, dim3(kAttnThreads), st, pdl, a);
+}
+
+template <int D>
+static pgf8_status launch_attn(const AttnDecodeArgs &a, int gt, int64_t seqs, cudaStream_t st, int pdl)
+{
+    pgf8_status r;
+    switch (gt) {
+    case 8: r = launch_attn_gt<D, 8>(a, seqs, st, pdl); break;
+    case 4: r = launch_attn_gt<D, 4>(a, seqs, st, pdl); break;
+    case 2: r = launch_attn_gt<D, 2>(a, seqs, st, pdl); break;
+    default: r = launch_attn_gt<D, 1>(a, seqs, st, pdl); break;
+    }
+    if (r != PGF8_OK || a.nsplit == 1)
+        return r;
+    // the merge overlaps the chunk kernel's tail and waits for its results
+    return launch_grid(attn_decode_combine_kernel<D>, dim3(static_cast<unsigned>(seqs * a.Hq)), dim3(D), st, 1,
+                       static_cast<const float *>(a.part), a.nsplit, a.Hq, a.Hkv, a.sv, a.out, a.ldo, a.odt);
 }
 
 } // namespace pgf8
@@ -825,6 +924,97 @@ pgf8_status pgf8_fp8_kv_write_paged(const void *kv, pgf8_dtype dt, int64_t token
     return launch_quant(kv_write_paged_kernel<__nv_bfloat16>, grid, cs, pdl, static_cast<const __nv_bfloat16 *>(kv),
                         tokens, heads, head_dim, ldkv, scales, first_pos, block_size, block_table, num_blocks, cache,
                         bad_blocks);
+}
+
+pgf8_status pgf8_fp8_attention_decode_plan(int64_t seqs, int64_t q_heads, int64_t kv_heads, int64_t head_dim,
+                                           int64_t max_context, int64_t splits, int64_t *nsplit, int64_t *chunk)
+{
+    if (!attn_shape_ok(seqs, q_heads, kv_heads, head_dim, max_context) || splits < 0)
+        return PGF8_ERR_INVALID_ARG;
+    const AttnPlan p = attn_plan(seqs, q_heads, kv_heads, max_context, splits);
+    if (nsplit)
+        *nsplit = p.nsplit;
+    if (chunk)
+        *chunk = p.chunk;
+    return PGF8_OK;
+}
+
+size_t pgf8_fp8_attention_decode_workspace_size(int64_t seqs, int64_t q_heads, int64_t kv_heads, int64_t head_dim,
+                                                int64_t max_context, int64_t splits)
+{
+    if (!attn_shape_ok(seqs, q_heads, kv_heads, head_dim, max_context) || splits < 0)
+        return 0;
+    return attn_workspace_bytes(seqs, q_heads, head_dim, attn_plan(seqs, q_heads, kv_heads, max_context, splits));
+}
+
+pgf8_status pgf8_fp8_attention_decode_paged(const void *q, pgf8_dtype q_dt, int64_t seqs, int64_t q_heads,
+                                            int64_t ldq, const pgf8_paged_kv_cache *cache,
+                                            const int32_t *block_tables, int64_t table_stride,
+                                            const int32_t *context_lens, int64_t max_context, void *out,
+                                            pgf8_dtype out_dt, int64_t ldo, int64_t splits, void *workspace,
+                                            size_t workspace_bytes, int32_t *errors, int32_t flags, void *stream)
+{
+    if (!cache)
+        return PGF8_ERR_INVALID_ARG;
+    const int64_t Hkv = cache->kv_heads, D = cache->head_dim, B = cache->block_size;
+    if (!attn_shape_ok(seqs, q_heads, Hkv, D, max_context) || splits < 0 || cache->num_blocks < 1 || B < 16 ||
+        B % 16 != 0 || ldq < q_heads * D || ldo < q_heads * D || table_stride < 1 ||
+        max_context > table_stride * B || seqs * q_heads > 0x7fffffffll)
+        return PGF8_ERR_INVALID_ARG;
+    if (seqs == 0)
+        return PGF8_OK;
+    if (!q || !out || !cache->k_cache || !cache->v_cache || !cache->k_scales || !cache->v_scales || !block_tables ||
+        !context_lens)
+        return PGF8_ERR_INVALID_ARG;
+    const bool qok = q_dt == PGF8_F32 || q_dt == PGF8_F16 || q_dt == PGF8_BF16;
+    const bool ook = out_dt == PGF8_F32 || out_dt == PGF8_F16 || out_dt == PGF8_BF16;
+    if (!qok || !ook)
+        return PGF8_ERR_UNSUPPORTED;
+    const uintptr_t qa = q_dt == PGF8_F32 ? 3u : 1u, oa = out_dt == PGF8_F32 ? 3u : 1u;
+    if (!aligned16(cache->k_cache) || !aligned16(cache->v_cache) || !aligned4(cache->k_scales) ||
+        !aligned4(cache->v_scales) || !aligned4(block_tables) || !aligned4(context_lens) ||
+        (errors && !aligned4(errors)) || (reinterpret_cast<uintptr_t>(q) & qa) ||
+        (reinterpret_cast<uintptr_t>(out) & oa))
+        return PGF8_ERR_ALIGNMENT;
+    const AttnPlan p = attn_plan(seqs, q_heads, Hkv, max_context, splits);
+    const size_t need = attn_workspace_bytes(seqs, q_heads, D, p);
+    if (need > 0 && (!workspace || workspace_bytes < need))
+        return PGF8_ERR_INVALID_ARG;
+    if (need > 0 && !aligned4(workspace))
+        return PGF8_ERR_ALIGNMENT;
+
+    AttnDecodeArgs a;
+    a.q = q;
+    a.ldq = ldq;
+    a.qdt = static_cast<int>(q_dt);
+    a.kc = cache->k_cache;
+    a.vc = cache->v_cache;
+    a.sk = cache->k_scales;
+    a.sv = cache->v_scales;
+    a.tables = block_tables;
+    a.table_stride = table_stride;
+    a.ctx_lens = context_lens;
+    a.num_blocks = cache->num_blocks;
+    a.Hkv = Hkv;
+    a.Hq = q_heads;
+    a.B = B;
+    a.max_ctx = max_context;
+    a.chunk = p.chunk;
+    a.nsplit = static_cast<int>(p.nsplit);
+    a.groups = p.groups;
+    a.qscale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));   // log2(e) / sqrt(D)
+    a.out = out;
+    a.ldo = ldo;
+    a.odt = static_cast<int>(out_dt);
+    a.part = static_cast<float *>(workspace);
+    a.errors = errors;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const int pdl = (flags & PGF8_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
+    if (D == 64)
+        return launch_attn<64>(a, p.gt, seqs, cs, pdl);
+    if (D == 128)
+        return launch_attn<128>(a, p.gt, seqs, cs, pdl);
+    return launch_attn<256>(a, p.gt, seqs, cs, pdl);
 }
 
 pgf8_status pgf8_fp8_quantize_rows(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,

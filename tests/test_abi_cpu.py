@@ -212,3 +212,74 @@ def test_kv_write_paged_argument_checks():
     assert f(a16 + 4, pg.F32, 4, 2, 64, 128, a16, 0, 16, a16, 1, 1, a16, None, 0, None) == pg.ERR_ALIGNMENT
     assert f(a16, 7, 4, 2, 64, 128, a16, 0, 16, a16, 1, 1, a16, None, 0, None) == pg.ERR_UNSUPPORTED
     assert f(a16, pg.F32, 4, 2, 64, 128, None, 0, 16, a16, 1, 1, a16, None, 0, None) == pg.ERR_INVALID_ARG
+
+
+def test_attention_decode_plan_covers_the_context():
+    # automatic split: chunks of whole warp steps (64 positions), none empty
+    for seqs, hq, hkv, ctx in [(8, 32, 32, 4096), (8, 64, 8, 4096), (1, 32, 32, 100000), (64, 64, 8, 1024),
+                               (1, 8, 1, 17), (3, 12, 4, 333)]:
+        ns, ch = pg.fp8_attention_decode_plan(seqs, hq, hkv, 128, ctx)
+        assert ch % 64 == 0 and ns >= 1
+        assert ns * ch >= ctx > (ns - 1) * ch
+        if ns > 1:
+            assert ch >= 256
+        ws = pg.lib.pgf8_fp8_attention_decode_workspace_size(seqs, hq, hkv, 128, ctx, 0)
+        assert ws == (seqs * hq * ns * 130 * 4 if ns > 1 else 0)
+    # a small batch is split for the grid, a large one is not
+    assert pg.fp8_attention_decode_plan(1, 32, 32, 128, 4096)[0] > 1
+    assert pg.fp8_attention_decode_plan(256, 32, 32, 128, 4096)[0] == 1
+    # forced: at most the requested chunks, multiples of 16 positions
+    for ctx, splits in [(100, 3), (4096, 7), (40, 9), (16, 4), (0, 2)]:
+        ns, ch = pg.fp8_attention_decode_plan(2, 8, 8, 64, ctx, splits)
+        assert 1 <= ns <= splits and ch % 16 == 0
+        assert ns * ch >= ctx and (ns == 1 or (ns - 1) * ch < ctx)
+    assert pg.fp8_attention_decode_plan(2, 8, 8, 64, 100, 3) == (3, 48)
+    with pytest.raises(pg.Pgf8Error):
+        pg.fp8_attention_decode_plan(2, 12, 8, 128, 64)     # q_heads not a multiple of kv_heads
+    with pytest.raises(pg.Pgf8Error):
+        pg.fp8_attention_decode_plan(2, 8, 8, 96, 64)      # head_dim not 64 / 128 / 256
+
+
+def test_attention_decode_argument_checks():
+    buf = (ctypes.c_uint8 * 16384)()
+    a16 = (ctypes.addressof(buf) + 15) // 16 * 16
+    f = pg.lib.pgf8_fp8_attention_decode_paged
+
+    def cache(**kw):
+        c = dict(k_cache=a16, v_cache=a16, k_scales=a16, v_scales=a16, num_blocks=4, kv_heads=2, block_size=16,
+                 head_dim=64)
+        c.update(kw)
+        return ctypes.byref(pg.PagedKVCache(**c))
+
+    def call(c=None, seqs=2, hq=4, ldq=256, q=a16, qdt=pg.F32, table_stride=2, max_ctx=32, out=a16, odt=pg.F32,
+             ldo=256, splits=1, ws=None, wsb=0, errors=None):
+        # (q, q_dt, seqs, q_heads, ldq, cache, tables, table_stride, ctx_lens, max_context, out, out_dt, ldo,
+        #  splits, workspace, workspace_bytes, errors, flags, stream)
+        return f(q, qdt, seqs, hq, ldq, cache() if c is None else c, a16, table_stride, a16, max_ctx, out, odt, ldo,
+                 splits, ws, wsb, errors, 0, None)
+
+    assert call(seqs=0) == pg.OK                                      # nothing to do
+    assert f(a16, pg.F32, 2, 4, 256, None, a16, 2, a16, 32, a16, pg.F32, 256, 1, None, 0, None, 0, None) \
+        == pg.ERR_INVALID_ARG                                         # no cache
+    assert call(c=cache(head_dim=96), ldq=384, ldo=384) == pg.ERR_INVALID_ARG
+    assert call(c=cache(block_size=8)) == pg.ERR_INVALID_ARG          # block_size % 16
+    assert call(c=cache(kv_heads=3)) == pg.ERR_INVALID_ARG            # q_heads % kv_heads
+    assert call(c=cache(num_blocks=0)) == pg.ERR_INVALID_ARG
+    assert call(max_ctx=33) == pg.ERR_INVALID_ARG                     # past the table (2 x 16)
+    assert call(ldq=200) == pg.ERR_INVALID_ARG                        # ldq < q_heads * head_dim
+    assert call(ldo=200) == pg.ERR_INVALID_ARG
+    assert call(splits=-1) == pg.ERR_INVALID_ARG
+    assert call(q=None) == pg.ERR_INVALID_ARG
+    assert call(c=cache(v_scales=None)) == pg.ERR_INVALID_ARG
+    assert call(qdt=5) == pg.ERR_UNSUPPORTED
+    assert call(odt=5) == pg.ERR_UNSUPPORTED
+    assert call(c=cache(k_cache=a16 + 8)) == pg.ERR_ALIGNMENT
+    assert call(q=a16 + 2) == pg.ERR_ALIGNMENT                        # f32 query
+    assert call(out=a16 + 1, odt=pg.BF16) == pg.ERR_ALIGNMENT
+    assert call(errors=a16 + 2) == pg.ERR_ALIGNMENT
+    # two chunks need the merge workspace
+    need = pg.lib.pgf8_fp8_attention_decode_workspace_size(2, 4, 2, 64, 32, 2)
+    assert need == 2 * 4 * 2 * 66 * 4
+    assert call(splits=2) == pg.ERR_INVALID_ARG
+    assert call(splits=2, ws=a16, wsb=need - 4) == pg.ERR_INVALID_ARG
+    assert call(splits=2, ws=a16 + 2, wsb=need) == pg.ERR_ALIGNMENT
