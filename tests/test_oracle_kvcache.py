@@ -108,3 +108,35 @@ def test_argument_errors():
     K.write(kv, 0)
     with pytest.raises(oracle.OracleError):
         oracle.attention_paged(np.ones((1, 3, 8)), K, K, 4)  # 3 query heads over 2 KV heads
+
+
+def test_attention_equals_the_library_routine():
+    """torch's scaled_dot_product_attention (binary64, default scale 1/sqrt(D))
+    on the dequantised cache: pins the temperature, the key scale, the
+    softmax and the causal alignment (a full prompt: query i sees 0..i)."""
+    import torch
+    import torch.nn.functional as F
+    g = np.random.default_rng(4)
+    T, Hkv, D, G = 45, 2, 32, 2
+    kk = (g.standard_normal((T, Hkv, D)) * 3).astype(np.float32)
+    vv = g.standard_normal((T, Hkv, D)).astype(np.float32)
+    K, V = _caches(kk, vv, np.array([2, 0, 1], np.int32), 3)
+    kd = torch.from_numpy(np.repeat(_deq(K, T), G, axis=1)).permute(1, 0, 2)   # [Hq, T, D]
+    vd = torch.from_numpy(np.repeat(_deq(V, T), G, axis=1)).permute(1, 0, 2)
+    # decode: one query at the last position sees every key
+    q1 = g.standard_normal((1, Hkv * G, D))
+    ref1 = F.scaled_dot_product_attention(torch.from_numpy(q1).permute(1, 0, 2), kd, vd)
+    np.testing.assert_allclose(oracle.attention_paged(q1, K, V, T), ref1.permute(1, 0, 2).numpy(),
+                               rtol=1e-12, atol=1e-13)
+    # context: T queries over T keys, causal
+    qc = g.standard_normal((T, Hkv * G, D))
+    refc = F.scaled_dot_product_attention(torch.from_numpy(qc).permute(1, 0, 2), kd, vd, is_causal=True)
+    np.testing.assert_allclose(oracle.attention_paged(qc, K, V, T), refc.permute(1, 0, 2).numpy(),
+                               rtol=1e-12, atol=1e-13)
+    # the last Tq queries of a longer context (bottom-right causal alignment): explicit mask
+    Tq = 5
+    qt = qc[-Tq:]
+    mask = torch.from_numpy(np.arange(T)[None, :] <= (T - Tq + np.arange(Tq))[:, None])
+    reft = F.scaled_dot_product_attention(torch.from_numpy(qt).permute(1, 0, 2), kd, vd, attn_mask=mask)
+    np.testing.assert_allclose(oracle.attention_paged(qt, K, V, T), reft.permute(1, 0, 2).numpy(),
+                               rtol=1e-12, atol=1e-13)
