@@ -62,3 +62,25 @@ def test_silu_mul_closed_forms():
     assert abs((h[4] - h[5]) - 2.5) < 1e-15                    # silu(x) - silu(-x) = x
     u = np.array([3.0, -2.0, 0.5, 7.0, 0.0, -1.0])
     np.testing.assert_allclose(oracle.silu_mul(x, u), h * u, rtol=1e-15, atol=0)
+
+
+def test_norms_and_gate_equal_the_library_routines():
+    """torch's binary64 layer_norm, rms_norm and silu on the same (widened)
+    inputs: pins eps placement in both norms with gamma and beta applied."""
+    import torch
+    import torch.nn.functional as F
+    g = np.random.default_rng(3)
+    x = (g.standard_normal((6, 80)) * 2 + 0.5).astype(F32)
+    x[0] *= F32(1e-3)                                          # a row where eps matters
+    gamma = g.uniform(0.5, 2, 80).astype(F32)
+    beta = g.standard_normal(80).astype(F32)
+    xt, gt, bt = (torch.from_numpy(a.astype(np.float64)) for a in (x, gamma, beta))
+    for eps in (1e-5, 1e-6, 0.25):
+        np.testing.assert_allclose(oracle.norm_rows(x, gamma, beta, eps),
+                                   F.layer_norm(xt, (80,), gt, bt, eps).numpy(), rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(oracle.norm_rows(x, gamma, None, eps),
+                                   F.rms_norm(xt, (80,), gt, eps).numpy(), rtol=1e-12, atol=1e-13)
+    gg = g.standard_normal(200) * 6
+    uu = g.standard_normal(200)
+    np.testing.assert_allclose(oracle.silu_mul(gg, uu), (F.silu(torch.from_numpy(gg)) * torch.from_numpy(uu)).numpy(),
+                               rtol=1e-14, atol=1e-300)
