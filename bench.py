@@ -816,6 +816,65 @@ def run_attention(args):
                       "frac_hbm": round(gbs / float(peaks["hbm_gbs"]), 3), "peak_source": src}), flush=True)
 
 
+def run_attention_context(args):
+    """Context attention over the FP8 paged cache, launched eagerly `warmup +
+    steps` times (e.g. --attention-context 4,32,32,2048 = seqs, query heads,
+    KV heads, prompt length: 7B-shaped prefill, each sequence's prompt is its
+    whole context).  Queries N(0,1) quantised per (token, head) row by the
+    row quantiser before the timed region; caches as for --attention.
+    FLOPs counted: 4 * 128 * sum over query rows of the keys they see (the
+    causal half of Q K^T and P V), per query head."""
+    import torch
+    import precision_gemm_fp8_b200 as pg
+
+    seqs, hq, hkv, qlen = (int(v) for v in args.attention_context.split(","))
+    d, B, ctx = 128, 16, qlen
+    dev = torch.device("cuda", 0)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4321)
+    nblk = (ctx + B - 1) // B
+    num_blocks = seqs * nblk
+    tables = torch.randperm(num_blocks, generator=gen, device=dev).to(torch.int32).view(seqs, nblk)
+    kc = torch.zeros((num_blocks, hkv, B, d), dtype=torch.uint8, device=dev)
+    vc = torch.zeros_like(kc)
+    sk = torch.full((hkv,), 4.5 / 448.0, dtype=torch.float32, device=dev)
+    sv = sk.clone()
+    for s in range(seqs):
+        for cache, sc in ((kc, sk), (vc, sv)):
+            kv = torch.randn((ctx, hkv, d), generator=gen, device=dev)
+            pg.fp8_kv_write_paged(kv, sc, cache, tables[s].contiguous(), 0)
+    total_q = seqs * qlen
+    q = torch.randn((total_q * hq, d), generator=gen, device=dev)
+    qc, qs = pg.fp8_quantize_rows(q)
+    qc = qc.view(total_q, hq, d)
+    q_start = torch.arange(0, total_q + 1, qlen, dtype=torch.int32, device=dev)
+    lens = torch.full((seqs,), ctx, dtype=torch.int32, device=dev)
+    out = torch.empty((total_q, hq, d), dtype=torch.bfloat16, device=dev)
+    fn = lambda: pg.fp8_attention_context_paged(qc, qs, q_start, lens, kc, vc, sk, sv, tables, ctx, qlen,  # noqa: E731
+                                                out=out)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        fn()
+    t1.record()
+    torch.cuda.synchronize()
+    if pg.device_status() != pg.OK:
+        raise RuntimeError("device error word raised")
+    us = 1e3 * t0.elapsed_time(t1) / args.steps
+    seen = qlen * (qlen + 1) // 2          # keys seen, summed over the query rows of one sequence
+    flops = 4.0 * d * seen * hq * seqs
+    peaks, src = _load_peaks()
+    fp8_peak = 2.0 * float(peaks["bf16_tflops"])
+    tf = flops / (us * 1e-6) / 1e12
+    print(json.dumps({"attention_context": args.attention_context, "us_per_call": round(us, 3),
+                      "flops": flops, "tflops": round(tf, 1), "frac_fp8_burst": round(tf / fp8_peak, 3),
+                      "fp8_peak_tflops": fp8_peak, "peak_source": src}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -836,6 +895,9 @@ def main():
     ap.add_argument("--attention", default=None,
                     help="seqs,q_heads,kv_heads,head_dim,context: time (or profile) the FP8 paged decode attention "
                          "eagerly (--split-k caps its context chunks)")
+    ap.add_argument("--attention-context", default=None,
+                    help="seqs,q_heads,kv_heads,prompt_len: time (or profile) the FP8 paged context attention "
+                         "eagerly (head_dim 128, causal prompts)")
     ap.add_argument("--path", type=int, default=0)
     ap.add_argument("--split-k", type=int, default=0)
     ap.add_argument("--tile-n", type=int, default=0)
@@ -848,6 +910,9 @@ def main():
         return
     if args.attention:
         run_attention(args)
+        return
+    if args.attention_context:
+        run_attention_context(args)
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -248,6 +248,45 @@ pgf8_status pgf8_fp8_attention_decode_paged(const void *q, pgf8_dtype q_dt, int6
                                             size_t workspace_bytes, int32_t *errors, int32_t flags, void *stream);
 
 /* ------------------------------------------------------------------------
+ * Context (prefill) attention over the FP8 paged KV cache on the tensor
+ * cores ("C++ and FP8" §3.3: context attention in the FP8 dataflow; §3.2:
+ * paged FP8 cache).  The queries of sequence s are the q_len(s) =
+ * q_start[s+1] - q_start[s] tokens q_start[s] .. q_start[s+1] - 1 of the
+ * packed query batch, at positions ctx - q_len .. ctx - 1 (ctx =
+ * context_lens[s] >= q_len; the cache must already hold positions
+ * 0 .. ctx - 1, the new ones included).  Query i sees positions
+ * 0 .. ctx - q_len + i (causal); query head h reads KV head
+ * h / (q_heads / kv_heads).
+ *
+ * The query enters as E4M3 codes with one scale per (token, head) row:
+ * q_codes [total_q, q_heads, 128] and q_scales [total_q * q_heads], as
+ * pgf8_fp8_quantize_rows (DYNAMIC) writes them for q viewed as
+ * [total_q * q_heads, 128].  Both products run E4M3 x E4M3 with binary32
+ * accumulation: scores S = q_codes . k_codes * sq * sk / sqrt(128); softmax
+ * in binary32 (exp2f); the probabilities relative to the running row
+ * maximum are rounded to E4M3 after scaling by 2^8 (the only rounding
+ * beyond binary32: at most 2^-4 relative, or 2^-18 absolute below 2^-14);
+ * out = (sum_t P_t . v_codes_t) * 2^-8 * sv / sum_t p_t, rounded once to
+ * out_dt.
+ *
+ * head_dim must be 128 (else PGF8_ERR_UNSUPPORTED); block_size a multiple
+ * of 16; num_blocks * kv_heads * block_size < 2^31 - 1.  max_q_len (host)
+ * bounds every q_len: the grid covers it.  out [total_q, q_heads, 128],
+ * token stride ldo elements.  errors (device int32 or NULL) counts
+ * out-of-range block-table entries (those positions are left out), q_len
+ * beyond max_q_len (the tail rows are not written) and sequences with
+ * ctx < q_len or ctx > max_context (not written).  Alignment: q_codes and
+ * the caches 16 bytes; q_scales, q_start, tables, lengths, errors 4 bytes;
+ * out its element size.  seqs, total_q or max_q_len == 0: no-op.
+ * ---------------------------------------------------------------------- */
+pgf8_status pgf8_fp8_attention_context_paged(const uint8_t *q_codes, const float *q_scales,
+                                             const int32_t *q_start, int64_t seqs, int64_t total_q,
+                                             int64_t max_q_len, int64_t q_heads, const pgf8_paged_kv_cache *cache,
+                                             const int32_t *block_tables, int64_t table_stride,
+                                             const int32_t *context_lens, int64_t max_context, void *out,
+                                             pgf8_dtype out_dt, int64_t ldo, int32_t *errors, void *stream);
+
+/* ------------------------------------------------------------------------
  * Normalisation or gate fused with the per-token quantisation ("7B on an
  * RTX 4060 with FP8", computation graph §2.1: LayerNorm fused with the QKV
  * projection's input).  The normalised / gated values never go to memory;

@@ -69,6 +69,8 @@ _SIGS = {
     "pgf8_fp8_attention_decode_workspace_size": ([_i64, _i64, _i64, _i64, _i64, _i64], _sz),
     "pgf8_fp8_attention_decode_paged": ([_vp, _i32, _i64, _i64, _i64, ctypes.POINTER(PagedKVCache), _vp, _i64, _vp,
                                          _i64, _vp, _i32, _i64, _i64, _vp, _sz, _vp, _i32, _vp], _i32),
+    "pgf8_fp8_attention_context_paged": ([_vp, _vp, _vp, _i64, _i64, _i64, _i64, ctypes.POINTER(PagedKVCache),
+                                          _vp, _i64, _vp, _i64, _vp, _i32, _i64, _vp, _vp], _i32),
     "pgf8_fp8_norm_quantize": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, ctypes.c_float, _vp, _vp, _i32, _vp], _i32),
     "pgf8_fp8_silu_mul_quantize": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _i32, _vp], _i32),
     "pgf8_fp8_quantize_tensor": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _i32, _vp], _i32),
@@ -269,6 +271,47 @@ def fp8_attention_decode_paged(q: torch.Tensor, k_cache: torch.Tensor, v_cache: 
         block_tables.stride(0), _ptr(context_lens), max_context, _ptr(out), codes[out.dtype], out.stride(0), splits,
         _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
         None if errors is None else _ptr(errors), flags, _stream(stream)), "fp8_attention_decode_paged")
+    return out
+
+
+def fp8_attention_context_paged(q_codes: torch.Tensor, q_scales: torch.Tensor, q_start: torch.Tensor,
+                                context_lens: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                                k_scales: torch.Tensor, v_scales: torch.Tensor, block_tables: torch.Tensor,
+                                max_context: int, max_q_len: int, out: torch.Tensor | None = None,
+                                out_dtype: torch.dtype = torch.bfloat16, errors: torch.Tensor | None = None,
+                                stream=None) -> torch.Tensor:
+    """Causal context attention of the packed queries (E4M3 codes q_codes
+    [total_q, q_heads, 128] with per-(token, head) scales q_scales
+    [total_q * q_heads], as fp8_quantize_rows writes them) over the paged
+    E4M3 K / V caches; sequence s owns query tokens q_start[s] ..
+    q_start[s+1] - 1 (int32 [seqs + 1]), the last positions of its
+    context_lens[s] cached ones.  Returns out [total_q, q_heads, 128]."""
+    total_q, q_heads, head_dim = q_codes.shape
+    if q_codes.dtype != torch.uint8 or not q_codes.is_contiguous():
+        raise ValueError("q_codes must be a contiguous uint8 [total_q, q_heads, head_dim] tensor")
+    num_blocks, kv_heads, block_size, cd = k_cache.shape
+    for c in (k_cache, v_cache):
+        if c.shape != k_cache.shape or c.dtype != torch.uint8 or not c.is_contiguous() or cd != head_dim:
+            raise ValueError("caches must be contiguous uint8 [num_blocks, kv_heads, block_size, head_dim] tensors")
+    if block_tables.dtype != torch.int32 or block_tables.dim() != 2 or block_tables.stride(1) != 1:
+        raise ValueError("block_tables must be an int32 [seqs, table_stride] tensor with contiguous rows")
+    for t in (q_start, context_lens):
+        if t.dtype != torch.int32 or not t.is_contiguous():
+            raise ValueError("q_start and context_lens must be contiguous int32 tensors")
+    seqs = context_lens.numel()
+    if q_start.numel() != seqs + 1:
+        raise ValueError("q_start must hold seqs + 1 offsets")
+    if out is None:
+        out = torch.empty((total_q, q_heads, head_dim), dtype=out_dtype, device=q_codes.device)
+    codes = {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}
+    if out.dtype not in codes or out.stride(2) != 1 or out.stride(1) != head_dim:
+        raise ValueError("out must be float32 / float16 / bfloat16 with heads contiguous within a token")
+    cache = PagedKVCache(_ptr(k_cache), _ptr(v_cache), _ptr(k_scales), _ptr(v_scales), num_blocks, kv_heads,
+                         block_size, head_dim)
+    _check(lib.pgf8_fp8_attention_context_paged(
+        _ptr(q_codes), _ptr(q_scales), _ptr(q_start), seqs, total_q, max_q_len, q_heads, ctypes.byref(cache),
+        _ptr(block_tables), block_tables.stride(0), _ptr(context_lens), max_context, _ptr(out), codes[out.dtype],
+        out.stride(0), None if errors is None else _ptr(errors), _stream(stream)), "fp8_attention_context_paged")
     return out
 
 

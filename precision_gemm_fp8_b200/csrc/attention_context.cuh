@@ -1,0 +1,404 @@
+// Context (prefill) attention over the FP8 (E4M3) paged KV cache on the
+// 5th-generation tensor cores.
+//
+// "C++ and FP8" §3.3: the context attention runs in the FP8 dataflow; §3.2:
+// the K / V cache is paged in blocks of 16 tokens kept in FP8.  This
+// library's reading: the queries of a sequence are its last q_len positions
+// ctx - q_len .. ctx - 1 (a prompt, or a prompt continued after a cached
+// prefix), query i sees positions 0 .. ctx - q_len + i (causal), grouped
+// query heads.  Both products are E4M3 x E4M3 -> f32 on the tensor cores:
+//   S = Q_codes . K_codes^T              (Q quantised per (token, head) row
+//                                         beforehand by the row quantiser)
+//   P = E4M3(2^8 . exp2(S . sq . sk . log2(e)/sqrt(D) - m))   (online softmax)
+//   O = P . V_codes . 2^-8 . sv / l
+// l sums the unrounded probabilities.  head_dim 128.
+//
+// One CTA per (128-query tile, query head, sequence), 192 threads:
+//   warp 0      TMA: the Q tile once, then per 128-key tile eight 16-row
+//               pieces of K and of V straight from the paged cache (a piece
+//               past the context, or of an out-of-range block, is read at a
+//               row past the cache's end and arrives as zeros);
+//   warp 1      TMEM (512 columns: S double buffer, PV double buffer) and
+//               the MMA issue: S_j = Q K_j^T, then PV_{j-1} = P_{j-1} V_{j-1}
+//               (V as an MN-major operand: the cache rows are d-contiguous);
+//   warps 2-5   one query row per thread: scores from TMEM (two passes),
+//               causal and validity masks, online softmax in base 2, P codes
+//               written into shared memory in the 128-byte-swizzled K-major
+//               layout, PV_{j-1} added into registers one tile late (so the
+//               PV MMA overlaps the next softmax), final 1/l and scales.
+// Every wait is bounded: a wait that gives up raises the CTA's abort flag
+// and the device error word; in-flight copies and MMAs are drained before
+// the CTA frees its TMEM and exits.
+#pragma once
+
+#include "attention.cuh"
+#include "gemm.cuh"
+
+namespace pgf8 {
+
+constexpr int kCtxStages = 3;                   // K / V ring depth (128 keys per stage)
+constexpr int kCtxTile = 16384;                  // 128 rows x 128 bytes
+constexpr int kCtxQ = 0;
+constexpr int kCtxK = kCtxQ + kCtxTile;
+constexpr int kCtxV = kCtxK + kCtxStages * kCtxTile;
+constexpr int kCtxP = kCtxV + kCtxStages * kCtxTile;
+constexpr int kCtxCtl = kCtxP + 2 * kCtxTile;
+constexpr int kCtxSmemBytes = kCtxCtl + 1024 /*control*/ + 1024 /*alignment slack*/;
+constexpr uint32_t kCtxTmemCols = 512;
+static_assert(kCtxSmemBytes <= 227 * 1024, "shared memory");
+
+struct AttnCtxCtl {
+    uint64_t q_full;
+    uint64_t kv_full[kCtxStages];
+    uint64_t kv_empty[kCtxStages];
+    uint64_t s_full[2], s_free[2];   // S buffer b: MMA -> softmax, softmax -> MMA
+    uint64_t p_full[2];              // P buffer b written (softmax -> MMA)
+    uint64_t o_full[2], o_free[2];   // PV buffer b: MMA -> softmax, softmax -> MMA
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+static_assert(sizeof(AttnCtxCtl) <= 1024, "control block");
+
+struct AttnCtxParams {
+    const float *q_scales;       // [total_q * Hq]: row (token, head) = token * Hq + head
+    const int32_t *q_start;      // [seqs + 1] first query token of each sequence
+    const int32_t *ctx_lens;     // [seqs]
+    const int32_t *tables;       // [seqs][table_stride]
+    int64_t table_stride;
+    const float *sk, *sv;        // [Hkv]
+    int Hq, Hkv, B;
+    int64_t num_blocks;
+    int cache_rows;              // num_blocks * Hkv * B: a row coordinate past the cache (zeros)
+    int max_ctx;
+    void *out;                   // [total_q][Hq][128], token stride ldo elements
+    int64_t ldo;
+    int odt;
+    int32_t *errors;
+};
+
+// Shared-memory descriptor of an MN-major operand tile in the 128-byte
+// swizzled canonical layout: rows of 128 bytes along MN (one swizzle atom
+// wide: MN = 128 for 8-bit types), K rows at 128 bytes, 8-row groups at
+// 1024 bytes (stride byte offset).  The leading byte offset (distance
+// between 128-element MN atoms) is not used with a single atom.
+__device__ __forceinline__ uint64_t sdesc_sw128_mn(uint32_t saddr)
+{
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>(kCtxTile >> 4) << 16;
+    d |= static_cast<uint64_t>(1024 >> 4) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(2) << 61;
+    return d;
+}
+
+// Cache row of the 16-position piece starting at `key` for KV head hk, or
+// cache_rows (a zero piece) when the piece lies past the context or its
+// block-table entry is out of range.
+__device__ __forceinline__ int ctx_piece_row(const AttnCtxParams &p, int64_t s, int hk, int key, int ctx)
+{
+    if (key >= ctx)
+        return p.cache_rows;
+    const int64_t blk = p.tables[s * p.table_stride + key / p.B];
+    if (blk < 0 || blk >= p.num_blocks)
+        return p.cache_rows;
+    return static_cast<int>((blk * p.Hkv + hk) * p.B + key % p.B);
+}
+
+__global__ void __launch_bounds__(192, 1) attn_context_kernel(const __grid_constant__ CUtensorMap tmQ,
+                                                              const __grid_constant__ CUtensorMap tmK,
+                                                              const __grid_constant__ CUtensorMap tmV,
+                                                              const AttnCtxParams p)
+{
+    constexpr uint32_t kIdescS = make_idesc(128, 128, 0, 0);                  // Q (K-major) x K (K-major)
+    constexpr uint32_t kIdescPV = make_idesc(128, 128, 0, 0) | (1u << 16);    // P (K-major) x V (MN-major)
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int qt = blockIdx.x, h = blockIdx.y;
+    const int64_t s = blockIdx.z;
+    const int hk = h / (p.Hq / p.Hkv);
+    const int q0 = p.q_start[s];
+    const int q_len = p.q_start[s + 1] - q0;
+    const int ctx = p.ctx_lens[s];
+    if (q_len <= qt * 128)
+        return;                                          // CTA-uniform: no tile here
+    if (q_len < 0 || ctx < q_len || ctx > p.max_ctx) {
+        if (threadIdx.x == 0 && qt == 0 && h == 0 && p.errors)
+            atomicAdd(p.errors, 1);
+        return;                                          // an invalid sequence is not written
+    }
+    if (qt == 0 && h == 0 && threadIdx.x == 0 && p.errors && q_len > static_cast<int>(gridDim.x) * 128)
+        atomicAdd(p.errors, 1);                          // longer than the grid covers: the tail is not written
+    const int nrows = q_len - qt * 128 < 128 ? q_len - qt * 128 : 128;
+    const int pos0 = ctx - q_len + qt * 128;            // position of the tile's first query
+    const int nkt = (pos0 + nrows - 1) / 128 + 1;        // key tiles 0 .. nkt - 1
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    AttnCtxCtl *ctl = reinterpret_cast<AttnCtxCtl *>(smem + kCtxCtl);
+    volatile int *abort_flag = &ctl->abort;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&ctl->q_full, 1);
+        for (int i = 0; i < kCtxStages; ++i) {
+            mbar_init(&ctl->kv_full[i], 1);
+            mbar_init(&ctl->kv_empty[i], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl->s_full[b], 1);
+            mbar_init(&ctl->s_free[b], 4);    // one arrival per softmax warp
+            mbar_init(&ctl->p_full[b], 4);
+            mbar_init(&ctl->o_full[b], 1);
+            mbar_init(&ctl->o_free[b], 4);
+        }
+        mbar_init(&ctl->drain, 1);
+        ctl->abort = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+    }
+    if (warp == 1) {
+        tmem_alloc(&ctl->tmem_base, kCtxTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl->tmem_base;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            uint32_t issued_mask = 0, issued_ph = 0;   // per stage: loaded at least once / parity of last load
+            mbar_arrive_expect_tx(&ctl->q_full, kCtxTile);
+            tma_load_2d(smem + kCtxQ, &tmQ, &ctl->q_full, h * 128, q0 + qt * 128);
+            for (int j = 0; j < nkt; ++j) {
+                const int st = j % kCtxStages;
+                const uint32_t ph = static_cast<uint32_t>(j / kCtxStages) & 1u;
+                if (!wait_bounded(&ctl->kv_empty[st], ph ^ 1u, abort_flag))
+                    break;
+                mbar_arrive_expect_tx(&ctl->kv_full[st], 2 * kCtxTile);
+                for (int i = 0; i < 8; ++i) {
+                    const int row = ctx_piece_row(p, s, hk, j * 128 + i * 16, ctx);
+                    tma_load_2d(smem + kCtxK + st * kCtxTile + i * 2048, &tmK, &ctl->kv_full[st], 0, row);
+                    tma_load_2d(smem + kCtxV + st * kCtxTile + i * 2048, &tmV, &ctl->kv_full[st], 0, row);
+                }
+                issued_mask |= 1u << st;
+                issued_ph = (issued_ph & ~(1u << st)) | (ph << st);
+            }
+            if (*abort_flag) {
+                wait_drain(&ctl->q_full, 0);
+                for (int i = 0; i < kCtxStages; ++i)
+                    if (issued_mask & (1u << i))
+                        wait_drain(&ctl->kv_full[i], (issued_ph >> i) & 1u);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            bool ok = wait_bounded(&ctl->q_full, 0, abort_flag);
+            const uint32_t q_addr = smem_u32(smem + kCtxQ);
+            auto issue_pv = [&](int i) -> bool {
+                const int b = i & 1, k = i >> 1, st = i % kCtxStages;
+                if (!wait_bounded(&ctl->p_full[b], static_cast<uint32_t>(k) & 1u, abort_flag))
+                    return false;
+                if (k >= 1 && !wait_bounded(&ctl->o_free[b], static_cast<uint32_t>(k - 1) & 1u, abort_flag))
+                    return false;
+                tc_fence_after();
+                const uint32_t p_addr = smem_u32(smem + kCtxP + b * kCtxTile);
+                const uint32_t v_addr = smem_u32(smem + kCtxV + st * kCtxTile);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)   // 4 x 32 keys
+                    umma_f8f6f4(tmem + 256 + b * 128, sdesc_sw128(p_addr + kk * 32),
+                                sdesc_sw128_mn(v_addr + kk * 32 * 128), kIdescPV, kk > 0 ? 1u : 0u);
+                umma_commit(&ctl->o_full[b]);
+                umma_commit(&ctl->kv_empty[st]);
+                return true;
+            };
+            for (int j = 0; ok && j < nkt; ++j) {
+                const int st = j % kCtxStages, b = j & 1, k = j >> 1;
+                if (!wait_bounded(&ctl->kv_full[st], static_cast<uint32_t>(j / kCtxStages) & 1u, abort_flag) ||
+                    (k >= 1 && !wait_bounded(&ctl->s_free[b], static_cast<uint32_t>(k - 1) & 1u, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t k_addr = smem_u32(smem + kCtxK + st * kCtxTile);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)   // 4 x 32 bytes of head_dim
+                    umma_f8f6f4(tmem + b * 128, sdesc_sw128(q_addr + kk * 32), sdesc_sw128(k_addr + kk * 32),
+                                kIdescS, kk > 0 ? 1u : 0u);
+                umma_commit(&ctl->s_full[b]);
+                if (j >= 1 && !issue_pv(j - 1))
+                    ok = false;
+            }
+            if (ok)
+                ok = issue_pv(nkt - 1);
+            if (!ok) {
+                umma_commit(&ctl->drain);
+                wait_drain(&ctl->drain, 0);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------------- softmax (one query row per thread)
+        const int qd = warp & 3;                          // TMEM lane quadrant of this warp
+        const int r = qd * 32 + lane;                     // query row of the tile
+        const int et = static_cast<int>(threadIdx.x) - 64;
+        const bool row_ok = r < nrows;
+        const int pos = pos0 + r;
+        const uint32_t t_lane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+        const float scale = row_ok ? p.q_scales[(static_cast<int64_t>(q0) + qt * 128 + r) * p.Hq + h] * p.sk[hk] *
+                                         (1.4426950408889634f * 0.08838834764831845f)   // log2(e) / sqrt(128)
+                                   : 0.0f;
+        float m = -INFINITY, l = 0.0f, alpha_prev = 0.0f;
+        float o[128];
+#pragma unroll
+        for (int d = 0; d < 128; ++d)
+            o[d] = 0.0f;
+        bool ok = true;
+
+        // O += PV_i (relative to the maximum after tile i), rescaling by alpha
+        auto accumulate = [&](int i, float alpha) -> bool {
+            const int b = i & 1, k = i >> 1;
+            bool w = wait_bounded(&ctl->o_full[b], static_cast<uint32_t>(k) & 1u, abort_flag);
+            w = __all_sync(0xffffffffu, w);
+            if (!w)
+                return false;
+            tc_fence_after();
+#pragma unroll
+            for (int c0 = 0; c0 < 128; c0 += 16) {
+                uint32_t v[16];
+                tmem_ld_32x32b_x16(t_lane + 256 + b * 128 + c0, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    o[c0 + e] = fmaf(o[c0 + e], alpha, __uint_as_float(v[e]));
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&ctl->o_free[b]);
+            return true;
+        };
+
+        for (int j = 0; j < nkt; ++j) {
+            const int b = j & 1, k = j >> 1, st = j % kCtxStages;
+            // validity of the tile's eight 16-key pieces (block-table entries)
+            uint32_t piece_ok = 0;
+            for (int i = 0; i < 8; ++i) {
+                const int key = j * 128 + i * 16;
+                if (key >= ctx)
+                    continue;
+                const int64_t blk = p.tables[s * p.table_stride + key / p.B];
+                if (blk >= 0 && blk < p.num_blocks)
+                    piece_ok |= 1u << i;
+                else if (et == 0 && h == 0 && p.errors)
+                    atomicAdd(p.errors, 1);
+            }
+            bool w = wait_bounded(&ctl->s_full[b], static_cast<uint32_t>(k) & 1u, abort_flag);
+            w = __all_sync(0xffffffffu, w);
+            if (!w) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t t_s = t_lane + b * 128;
+            // pass 1: the row maximum of the valid scores
+            float mx = -INFINITY;
+#pragma unroll 1
+            for (int c0 = 0; c0 < 128; c0 += 16) {
+                uint32_t v[16];
+                tmem_ld_32x32b_x16(t_s + c0, v);
+                tmem_ld_wait();
+                const bool pok = (piece_ok >> (c0 >> 4)) & 1u;
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int key = j * 128 + c0 + e;
+                    const float sc = __uint_as_float(v[e]) * scale;
+                    mx = (pok && row_ok && key <= pos) ? fmaxf(mx, sc) : mx;
+                }
+            }
+            const float mn = fmaxf(m, mx);
+            const float alpha = m == -INFINITY ? 0.0f : exp2f(m - mn);
+            // pass 2: probabilities, their codes (x 2^8) into P buffer b, the row sum
+            float rs = 0.0f;
+            uint8_t *prow = smem + kCtxP + b * kCtxTile + r * 128;
+#pragma unroll 1
+            for (int c0 = 0; c0 < 128; c0 += 16) {
+                uint32_t v[16];
+                tmem_ld_32x32b_x16(t_s + c0, v);
+                tmem_ld_wait();
+                const bool pok = (piece_ok >> (c0 >> 4)) & 1u;
+                float pr[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int key = j * 128 + c0 + e;
+                    const bool valid = pok && row_ok && key <= pos;
+                    pr[e] = valid ? exp2f(__uint_as_float(v[e]) * scale - mn) : 0.0f;
+                    rs += pr[e];
+                }
+                uint32_t wv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    wv[u] = static_cast<uint32_t>(cvt_e4m3x2(pr[4 * u] * 256.0f, pr[4 * u + 1] * 256.0f)) |
+                            (static_cast<uint32_t>(cvt_e4m3x2(pr[4 * u + 2] * 256.0f, pr[4 * u + 3] * 256.0f)) << 16);
+                *reinterpret_cast<uint4 *>(prow + (((c0 >> 4) ^ (r & 7)) << 4)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&ctl->s_free[b]);
+            // V rows past the context inside the piece that holds position ctx
+            // come from the cache as they are: clear them, since a zero
+            // probability times a NaN code would still be NaN
+            const int cut = ctx - j * 128;
+            if (cut > 0 && cut < 128 && (cut & 15) != 0 && ((piece_ok >> (cut >> 4)) & 1u)) {
+                bool wk = wait_bounded(&ctl->kv_full[st], static_cast<uint32_t>(j / kCtxStages) & 1u, abort_flag);
+                wk = __all_sync(0xffffffffu, wk);
+                if (!wk) {
+                    ok = false;
+                    break;
+                }
+                const int row = cut + (et >> 3);          // 16 rows x 8 chunks cover the rest of the piece
+                if (et < 128 && row < ((cut >> 4) + 1) * 16)
+                    *reinterpret_cast<uint4 *>(smem + kCtxV + st * kCtxTile + row * 128 + (et & 7) * 16) =
+                        make_uint4(0u, 0u, 0u, 0u);
+            }
+            fence_proxy_async_smem();   // P codes (and cleared V rows) before the MMA reads them
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&ctl->p_full[b]);
+            m = mn;
+            l = fmaf(l, alpha, rs);
+            if (j >= 1 && !accumulate(j - 1, alpha_prev)) {
+                ok = false;
+                break;
+            }
+            alpha_prev = alpha;
+        }
+        if (ok)
+            ok = accumulate(nkt - 1, alpha_prev);
+        if (ok && row_ok) {
+            const float f = l > 0.0f ? p.sv[hk] * 0.00390625f / l : 0.0f;   // 2^-8 undoes the P code scale
+            const int64_t base = (static_cast<int64_t>(q0) + qt * 128 + r) * p.ldo + static_cast<int64_t>(h) * 128;
+#pragma unroll
+            for (int d = 0; d < 128; ++d)
+                store_elem(p.out, base + d, p.odt, o[d] * f);
+        }
+    }
+
+    // -------------------------------------------------------------------- teardown
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kCtxTmemCols);
+    }
+}
+
+} // namespace pgf8

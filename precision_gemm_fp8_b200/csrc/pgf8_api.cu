@@ -12,6 +12,7 @@
 #include "gemm.cuh"
 #include "kvcache.cuh"
 #include "attention.cuh"
+#include "attention_context.cuh"
 #include "gemm_persistent.cuh"
 #include "gemm_streamk.cuh"
 #include "gemm_2sm.cuh"
@@ -1015,6 +1016,84 @@ pgf8_status pgf8_fp8_attention_decode_paged(const void *q, pgf8_dtype q_dt, int6
     if (D == 128)
         return launch_attn<128>(a, p.gt, seqs, cs, pdl);
     return launch_attn<256>(a, p.gt, seqs, cs, pdl);
+}
+
+pgf8_status pgf8_fp8_attention_context_paged(const uint8_t *q_codes, const float *q_scales,
+                                             const int32_t *q_start, int64_t seqs, int64_t total_q,
+                                             int64_t max_q_len, int64_t q_heads, const pgf8_paged_kv_cache *cache,
+                                             const int32_t *block_tables, int64_t table_stride,
+                                             const int32_t *context_lens, int64_t max_context, void *out,
+                                             pgf8_dtype out_dt, int64_t ldo, int32_t *errors, void *stream)
+{
+    if (!cache)
+        return PGF8_ERR_INVALID_ARG;
+    const int64_t Hkv = cache->kv_heads, D = cache->head_dim, B = cache->block_size;
+    if (seqs < 0 || seqs > 65535 || total_q < 0 || total_q >= (1ll << 31) || max_q_len < 0 || Hkv < 1 ||
+        q_heads < Hkv || q_heads % Hkv != 0 || q_heads > 65535 || B < 16 || B % 16 != 0 || cache->num_blocks < 1 ||
+        max_context < 0 || table_stride < 1 || max_context > table_stride * B || max_context >= (1ll << 31) ||
+        ldo < q_heads * 128 || cache->num_blocks * Hkv * B >= (1ll << 31) - 1)
+        return PGF8_ERR_INVALID_ARG;
+    if (D != 128)
+        return PGF8_ERR_UNSUPPORTED;
+    if (seqs == 0 || total_q == 0 || max_q_len == 0)
+        return PGF8_OK;
+    if (!q_codes || !q_scales || !q_start || !out || !cache->k_cache || !cache->v_cache || !cache->k_scales ||
+        !cache->v_scales || !block_tables || !context_lens)
+        return PGF8_ERR_INVALID_ARG;
+    if (out_dt != PGF8_F32 && out_dt != PGF8_F16 && out_dt != PGF8_BF16)
+        return PGF8_ERR_UNSUPPORTED;
+    const uintptr_t oa = out_dt == PGF8_F32 ? 3u : 1u;
+    if (!aligned16(q_codes) || !aligned16(cache->k_cache) || !aligned16(cache->v_cache) || !aligned4(q_scales) ||
+        !aligned4(q_start) || !aligned4(cache->k_scales) || !aligned4(cache->v_scales) || !aligned4(block_tables) ||
+        !aligned4(context_lens) || (errors && !aligned4(errors)) || (reinterpret_cast<uintptr_t>(out) & oa))
+        return PGF8_ERR_ALIGNMENT;
+
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(attn_context_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        kCtxSmemBytes);
+    });
+    if (attr_err != cudaSuccess)
+        return cuda_fail(attr_err);
+    const uint64_t cache_rows = static_cast<uint64_t>(cache->num_blocks * Hkv * B);
+    CUtensorMap tmQ, tmK, tmV;
+    if (!make_map(&tmQ, q_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(total_q),
+                  static_cast<uint64_t>(q_heads * 128), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tmK, cache->k_cache, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, cache_rows, 128, 128, 16,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tmV, cache->v_cache, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, cache_rows, 128, 128, 16,
+                  CU_TENSOR_MAP_SWIZZLE_128B))
+        return PGF8_ERR_UNSUPPORTED;
+
+    AttnCtxParams a;
+    a.q_scales = q_scales;
+    a.q_start = q_start;
+    a.ctx_lens = context_lens;
+    a.tables = block_tables;
+    a.table_stride = table_stride;
+    a.sk = cache->k_scales;
+    a.sv = cache->v_scales;
+    a.Hq = static_cast<int>(q_heads);
+    a.Hkv = static_cast<int>(Hkv);
+    a.B = static_cast<int>(B);
+    a.num_blocks = cache->num_blocks;
+    a.cache_rows = static_cast<int>(cache_rows);
+    a.max_ctx = static_cast<int>(max_context);
+    a.out = out;
+    a.ldo = ldo;
+    a.odt = static_cast<int>(out_dt);
+    a.errors = errors;
+
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>((max_q_len + 127) / 128), static_cast<unsigned>(q_heads),
+                       static_cast<unsigned>(seqs));
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = kCtxSmemBytes;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, attn_context_kernel, tmQ, tmK, tmV, a);
+    return e == cudaSuccess ? PGF8_OK : cuda_fail(e);
 }
 
 pgf8_status pgf8_fp8_quantize_rows(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,

@@ -283,3 +283,39 @@ def test_attention_decode_argument_checks():
     assert call(splits=2) == pg.ERR_INVALID_ARG
     assert call(splits=2, ws=a16, wsb=need - 4) == pg.ERR_INVALID_ARG
     assert call(splits=2, ws=a16 + 2, wsb=need) == pg.ERR_ALIGNMENT
+
+
+def test_attention_context_argument_checks():
+    buf = (ctypes.c_uint8 * 16384)()
+    a16 = (ctypes.addressof(buf) + 15) // 16 * 16
+    f = pg.lib.pgf8_fp8_attention_context_paged
+
+    def cache(**kw):
+        c = dict(k_cache=a16, v_cache=a16, k_scales=a16, v_scales=a16, num_blocks=4, kv_heads=2, block_size=16,
+                 head_dim=128)
+        c.update(kw)
+        return ctypes.byref(pg.PagedKVCache(**c))
+
+    def call(c=None, qc=a16, seqs=2, total_q=40, max_q_len=20, hq=4, table_stride=2, max_ctx=32, out=a16,
+             odt=pg.BF16, ldo=512, errors=None):
+        # (q_codes, q_scales, q_start, seqs, total_q, max_q_len, q_heads, cache, tables, table_stride,
+        #  ctx_lens, max_context, out, out_dt, ldo, errors, stream)
+        return f(qc, a16, a16, seqs, total_q, max_q_len, hq, cache() if c is None else c, a16, table_stride, a16,
+                 max_ctx, out, odt, ldo, errors, None)
+
+    assert call(seqs=0) == pg.OK and call(total_q=0) == pg.OK and call(max_q_len=0) == pg.OK   # nothing to do
+    assert f(a16, a16, a16, 2, 40, 20, 4, None, a16, 2, a16, 32, a16, pg.BF16, 512, None, None) == pg.ERR_INVALID_ARG
+    assert call(c=cache(head_dim=64)) == pg.ERR_UNSUPPORTED           # head_dim 128 only
+    assert call(c=cache(block_size=24)) == pg.ERR_INVALID_ARG         # block_size % 16
+    assert call(c=cache(kv_heads=3)) == pg.ERR_INVALID_ARG            # q_heads % kv_heads
+    assert call(max_ctx=33) == pg.ERR_INVALID_ARG                     # past the table (2 x 16)
+    assert call(ldo=500) == pg.ERR_INVALID_ARG                        # ldo < q_heads * 128
+    assert call(seqs=70000) == pg.ERR_INVALID_ARG
+    assert call(c=cache(num_blocks=1 << 27)) == pg.ERR_INVALID_ARG    # cache rows past 2^31
+    assert call(qc=None) == pg.ERR_INVALID_ARG
+    assert call(c=cache(k_scales=None)) == pg.ERR_INVALID_ARG
+    assert call(odt=9) == pg.ERR_UNSUPPORTED
+    assert call(qc=a16 + 8) == pg.ERR_ALIGNMENT                       # TMA base
+    assert call(c=cache(v_cache=a16 + 4)) == pg.ERR_ALIGNMENT
+    assert call(out=a16 + 1) == pg.ERR_ALIGNMENT
+    assert call(errors=a16 + 1) == pg.ERR_ALIGNMENT
