@@ -816,6 +816,49 @@ def run_attention(args):
                       "frac_hbm": round(gbs / float(peaks["hbm_gbs"]), 3), "peak_source": src}), flush=True)
 
 
+def run_kv_write(args):
+    """The FP8 paged KV-cache writer, launched eagerly `warmup + steps` times
+    (e.g. --kv-write 2048,32,128 = tokens, KV heads, head_dim: one 7B
+    prefill's K).  The K rows are a bf16 slice of a QKV-projection-shaped
+    output [tokens, (32 + 2 * heads) * head_dim] read in place; positions
+    0 .. tokens - 1 through a seeded permutation of blocks of 16."""
+    import torch
+    import precision_gemm_fp8_b200 as pg
+
+    tokens, heads, d = (int(v) for v in args.kv_write.split(","))
+    B = 16
+    dev = torch.device("cuda", 0)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(99)
+    width = (32 + 2 * heads) * d
+    qkv = torch.randn((tokens, width), generator=gen, device=dev).to(torch.bfloat16)
+    k = torch.as_strided(qkv, (tokens, heads, d), (width, d, 1), 32 * d)
+    nblk = (tokens + B - 1) // B
+    table = torch.randperm(nblk, generator=gen, device=dev).to(torch.int32)
+    cache = torch.zeros((nblk, heads, B, d), dtype=torch.uint8, device=dev)
+    scales = torch.full((heads,), 4.5 / 448.0, dtype=torch.float32, device=dev)
+    fn = lambda: pg.fp8_kv_write_paged(k, scales, cache, table, 0)  # noqa: E731
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        fn()
+    t1.record()
+    torch.cuda.synchronize()
+    if pg.device_status() != pg.OK:
+        raise RuntimeError("device error word raised")
+    us = 1e3 * t0.elapsed_time(t1) / args.steps
+    alg = tokens * heads * d * 3 + nblk * 4      # bf16 in, E4M3 out, the table
+    peaks, src = _load_peaks()
+    gbs = alg / (us * 1e-6) / 1e9
+    print(json.dumps({"kv_write": args.kv_write, "us_per_call": round(us, 3), "algorithmic_bytes": alg,
+                      "gbs": round(gbs, 1), "frac_hbm": round(gbs / float(peaks["hbm_gbs"]), 3),
+                      "peak_source": src, "l2_note": "inputs below L2 size are timed warm"}), flush=True)
+
+
 def run_attention_context(args):
     """Context attention over the FP8 paged cache, launched eagerly `warmup +
     steps` times (e.g. --attention-context 4,32,32,2048 = seqs, query heads,
@@ -898,6 +941,8 @@ def main():
     ap.add_argument("--attention-context", default=None,
                     help="seqs,q_heads,kv_heads,prompt_len: time (or profile) the FP8 paged context attention "
                          "eagerly (head_dim 128, causal prompts)")
+    ap.add_argument("--kv-write", default=None,
+                    help="tokens,kv_heads,head_dim: time (or profile) the FP8 paged KV-cache writer eagerly")
     ap.add_argument("--path", type=int, default=0)
     ap.add_argument("--split-k", type=int, default=0)
     ap.add_argument("--tile-n", type=int, default=0)
@@ -913,6 +958,9 @@ def main():
         return
     if args.attention_context:
         run_attention_context(args)
+        return
+    if args.kv_write:
+        run_kv_write(args)
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
