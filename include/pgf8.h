@@ -275,7 +275,8 @@ pgf8_status pgf8_fp8_attention_decode_paged(const void *q, pgf8_dtype q_dt, int6
  * token stride ldo elements.  errors (device int32 or NULL) counts
  * out-of-range block-table entries (those positions are left out), q_len
  * beyond max_q_len (the tail rows are not written) and sequences with
- * ctx < q_len or ctx > max_context (not written).  Alignment: q_codes and
+ * ctx < q_len, ctx > max_context or query tokens outside [0, total_q)
+ * (not written).  Alignment: q_codes and
  * the caches 16 bytes; q_scales, q_start, tables, lengths, errors 4 bytes;
  * out its element size.  seqs, total_q or max_q_len == 0: no-op.
  * ---------------------------------------------------------------------- */

@@ -254,6 +254,12 @@ def fp8_attention_decode_paged(q: torch.Tensor, k_cache: torch.Tensor, v_cache: 
         raise ValueError("block_tables must be an int32 [seqs, table_stride] tensor with contiguous rows")
     if context_lens.dtype != torch.int32 or not context_lens.is_contiguous():
         raise ValueError("context_lens must be a contiguous int32 tensor")
+    if context_lens.numel() != seqs or block_tables.shape[0] < seqs:
+        raise ValueError("context_lens needs one entry and block_tables one row per sequence")
+    if k_scales.numel() < kv_heads or v_scales.numel() < kv_heads:
+        raise ValueError("k_scales and v_scales need one entry per KV head")
+    if max_context > block_tables.shape[1] * block_size:
+        raise ValueError("max_context is longer than the block tables cover")
     if out is None:
         out = torch.empty((seqs, q_heads, head_dim), dtype=out_dtype, device=q.device)
     if out.stride(2) != 1 or out.stride(1) != head_dim:
@@ -301,6 +307,14 @@ def fp8_attention_context_paged(q_codes: torch.Tensor, q_scales: torch.Tensor, q
     seqs = context_lens.numel()
     if q_start.numel() != seqs + 1:
         raise ValueError("q_start must hold seqs + 1 offsets")
+    if q_scales.numel() < total_q * q_heads:
+        raise ValueError("q_scales needs one scale per (token, head) row")
+    if block_tables.shape[0] < seqs:
+        raise ValueError("block_tables needs one row per sequence")
+    if k_scales.numel() < kv_heads or v_scales.numel() < kv_heads:
+        raise ValueError("k_scales and v_scales need one entry per KV head")
+    if max_context > block_tables.shape[1] * block_size:
+        raise ValueError("max_context is longer than the block tables cover")
     if out is None:
         out = torch.empty((total_q, q_heads, head_dim), dtype=out_dtype, device=q_codes.device)
     codes = {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}

@@ -71,6 +71,7 @@ struct AttnCtxParams {
     int64_t num_blocks;
     int cache_rows;              // num_blocks * Hkv * B: a row coordinate past the cache (zeros)
     int max_ctx;
+    int total_q;                 // query tokens in the batch: q_start must stay within it
     void *out;                   // [total_q][Hq][128], token stride ldo elements
     int64_t ldo;
     int odt;
@@ -123,7 +124,7 @@ __global__ void __launch_bounds__(192, 1) attn_context_kernel(const __grid_const
     const int ctx = p.ctx_lens[s];
     if (q_len <= qt * 128)
         return;                                          // CTA-uniform: no tile here
-    if (q_len < 0 || ctx < q_len || ctx > p.max_ctx) {
+    if (q_len < 0 || q0 < 0 || q0 + q_len > p.total_q || ctx < q_len || ctx > p.max_ctx) {
         if (threadIdx.x == 0 && qt == 0 && h == 0 && p.errors)
             atomicAdd(p.errors, 1);
         return;                                          // an invalid sequence is not written

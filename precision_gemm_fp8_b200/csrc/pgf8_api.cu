@@ -1080,6 +1080,7 @@ pgf8_status pgf8_fp8_attention_context_paged(const uint8_t *q_codes, const float
     a.num_blocks = cache->num_blocks;
     a.cache_rows = static_cast<int>(cache_rows);
     a.max_ctx = static_cast<int>(max_context);
+    a.total_q = static_cast<int>(total_q);
     a.out = out;
     a.ldo = ldo;
     a.odt = static_cast<int>(out_dt);
