@@ -319,3 +319,58 @@ def test_attention_context_argument_checks():
     assert call(c=cache(v_cache=a16 + 4)) == pg.ERR_ALIGNMENT
     assert call(out=a16 + 1) == pg.ERR_ALIGNMENT
     assert call(errors=a16 + 1) == pg.ERR_ALIGNMENT
+
+
+def test_attention_bindings_check_shapes_before_any_pointer():
+    """The attention bindings reject inconsistent tensors with their own
+    messages before a pointer is taken (CPU tensors: nothing is launched)."""
+    import torch
+    u8 = lambda *s: torch.zeros(s, dtype=torch.uint8)       # noqa: E731
+    i32 = lambda *s: torch.zeros(s, dtype=torch.int32)      # noqa: E731
+    f32 = lambda *s: torch.zeros(s, dtype=torch.float32)    # noqa: E731
+    q = f32(2, 4, 64)
+    kc, vc = u8(4, 2, 16, 64), u8(4, 2, 16, 64)
+    ok = dict(k_scales=f32(2), v_scales=f32(2), block_tables=i32(2, 2), context_lens=i32(2), max_context=32)
+
+    def dec(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return pg.fp8_attention_decode_paged(q, kc, vc, **a)
+
+    with pytest.raises(ValueError, match="caches must be"):
+        pg.fp8_attention_decode_paged(q, kc, u8(4, 2, 16, 32), **ok)
+    with pytest.raises(ValueError, match="one entry and block_tables one row"):
+        dec(context_lens=i32(3))
+    with pytest.raises(ValueError, match="one entry per KV head"):
+        dec(v_scales=f32(1))
+    with pytest.raises(ValueError, match="longer than the block tables"):
+        dec(max_context=33)
+    with pytest.raises(ValueError, match="int32"):
+        dec(block_tables=torch.zeros((2, 2), dtype=torch.int64))
+    with pytest.raises(ValueError, match="device tensors"):
+        dec()                                                # consistent: only the device check remains
+
+    qc, qs = u8(40, 4, 128), f32(160)
+    kc2, vc2 = u8(4, 2, 16, 128), u8(4, 2, 16, 128)
+    okc = dict(k_scales=f32(2), v_scales=f32(2), block_tables=i32(2, 2), max_context=32, max_q_len=20)
+
+    def ctx(**kw):
+        a = dict(okc)
+        a.update(kw)
+        qsc = a.pop("q_scales", qs)
+        qst = a.pop("q_start", i32(3))
+        lens = a.pop("context_lens", i32(2))
+        return pg.fp8_attention_context_paged(qc, qsc, qst, lens, kc2, vc2, **a)
+
+    with pytest.raises(ValueError, match="seqs \\+ 1 offsets"):
+        ctx(q_start=i32(2))
+    with pytest.raises(ValueError, match="one scale per"):
+        ctx(q_scales=f32(100))
+    with pytest.raises(ValueError, match="one row per sequence"):
+        ctx(block_tables=i32(1, 2))
+    with pytest.raises(ValueError, match="one entry per KV head"):
+        ctx(k_scales=f32(1))
+    with pytest.raises(ValueError, match="longer than the block tables"):
+        ctx(max_context=40)
+    with pytest.raises(ValueError, match="device tensors"):
+        ctx()
