@@ -1467,7 +1467,7 @@ const char *pgf8_status_str(pgf8_status s)
     return "unknown status";
 }
 
-int pgf8_version(void) { return 100; }
+int pgf8_version(void) { return 200; }   // 0.2.0: per-tensor scaling, norm / gate fusion, FP8 KV cache and attention
 
 } // extern "C"
 
