@@ -147,3 +147,26 @@ def test_bad_entries_and_lengths_are_counted():
     assert errors.item() == 1
     ref2 = _reference(c2, qc2, qs2)
     assert np.abs(o2[:128].cpu().numpy() - ref2[:128]).max() <= 2.0 ** -14 * _vmax(c2)
+
+
+def test_one_hot_values_expose_each_key_probability():
+    """V row t = e_(t mod 128) (code 0x38 = 1.0): output column d is the
+    probability mass of the keys t = d (mod 128).  With exact power-of-two
+    probabilities this checks the P layout (swizzle) and the MN-major V
+    operand column by column; a wrong layout shows up as a permutation."""
+    seqs, Hq, Hkv, B, D = 1, 1, 1, 16, 128
+    q_len, ctx = 1, 256                            # one query at the last position sees all 256 keys
+    c = _case(seqs, Hq, Hkv, B, [q_len], [ctx], seed=9, exact=True)
+    vc = c["vc"]
+    vc[:] = 0
+    for t in range(ctx):
+        blk = c["tables"][0, t // B]
+        vc[blk, 0, t % B, t % 128] = 0x38
+    c["sv"] = np.ones(1, np.float32)
+    for K, V in c["refs"]:
+        V.scales = c["sv"]
+    out, qc, qs = _run(c)
+    ref = _reference(c, qc, qs)
+    got = out.cpu().numpy()[0, 0].astype(np.float64)
+    np.testing.assert_allclose(got, ref[0, 0], rtol=0, atol=2.0 ** -14)
+    assert abs(got.sum() - 1.0) < 1e-5            # the probabilities of all keys add up to 1
