@@ -82,12 +82,14 @@ struct AttnCtxParams {
 // swizzled canonical layout: rows of 128 bytes along MN (one swizzle atom
 // wide: MN = 128 for 8-bit types), K rows at 128 bytes, 8-row groups at
 // 1024 bytes (stride byte offset).  The leading byte offset (distance
-// between 128-element MN atoms) is not used with a single atom.
+// between 128-element MN atoms) is not applied with a single atom; it is
+// set to the same 1024 bytes, so that no reading of the two fields can
+// address past the tile.
 __device__ __forceinline__ uint64_t sdesc_sw128_mn(uint32_t saddr)
 {
     uint64_t d = 0;
     d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
-    d |= static_cast<uint64_t>(kCtxTile >> 4) << 16;
+    d |= static_cast<uint64_t>(1024 >> 4) << 16;
     d |= static_cast<uint64_t>(1024 >> 4) << 32;
     d |= static_cast<uint64_t>(1) << 46;
     d |= static_cast<uint64_t>(2) << 61;
