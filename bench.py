@@ -792,8 +792,9 @@ def run_attention(args):
     nsplit, chunk = pg.fp8_attention_decode_plan(seqs, hq, hkv, d, ctx, args.split_k)
     ws_bytes = pg.lib.pgf8_fp8_attention_decode_workspace_size(seqs, hq, hkv, d, ctx, args.split_k)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    flags = pg.FLAG_ATTN_MMA if args.attn_mma else 0
     fn = lambda: pg.fp8_attention_decode_paged(q, kc, vc, sk, sv, tables, lens, ctx, out=out,  # noqa: E731
-                                               splits=args.split_k, workspace=ws)
+                                               splits=args.split_k, workspace=ws, flags=flags)
     for _ in range(args.warmup):
         fn()
     torch.cuda.synchronize()
@@ -811,7 +812,8 @@ def run_attention(args):
     alg = kv_bytes + seqs * hq * d * 8 + seqs * nblk * 4
     peaks, src = _load_peaks()
     gbs = alg / (us * 1e-6) / 1e9
-    print(json.dumps({"attention": args.attention, "us_per_call": round(us, 3), "nsplit": nsplit, "chunk": chunk,
+    print(json.dumps({"attention": args.attention, "tensor_cores": bool(args.attn_mma), "us_per_call": round(us, 3),
+                      "nsplit": nsplit, "chunk": chunk,
                       "algorithmic_bytes": alg, "kv_bytes": kv_bytes, "gbs": round(gbs, 1),
                       "frac_hbm": round(gbs / float(peaks["hbm_gbs"]), 3), "peak_source": src}), flush=True)
 
@@ -938,6 +940,8 @@ def main():
     ap.add_argument("--attention", default=None,
                     help="seqs,q_heads,kv_heads,head_dim,context: time (or profile) the FP8 paged decode attention "
                          "eagerly (--split-k caps its context chunks)")
+    ap.add_argument("--attn-mma", action="store_true",
+                    help="with --attention: both products on the tensor cores (PGF8_FLAG_ATTN_MMA)")
     ap.add_argument("--attention-context", default=None,
                     help="seqs,q_heads,kv_heads,prompt_len: time (or profile) the FP8 paged context attention "
                          "eagerly (head_dim 128, causal prompts)")

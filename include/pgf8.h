@@ -114,6 +114,14 @@ typedef enum {
  * prefetch behind the previous layer). */
 #define PGF8_FLAG_FUSED_QUANT 2
 
+/* PGF8_FLAG_ATTN_MMA (pgf8_fp8_attention_decode_paged only): run both
+ * products on the tensor cores (mma.sync, binary16 operands, binary32
+ * accumulation), up to 8 query heads of one KV head per CTA.  The query and
+ * the probabilities are rounded to binary16 on the way (relative 2^-11);
+ * K / V codes widen exactly.  Without the flag the CUDA-core kernel keeps
+ * them in binary32. */
+#define PGF8_FLAG_ATTN_MMA 4
+
 /* Optional tuning of the linear entry points; a NULL pointer means all
  * defaults.  Fields set to 0 mean "choose automatically". */
 typedef struct {
@@ -220,8 +228,9 @@ pgf8_status pgf8_fp8_kv_write_paged(const void *kv, pgf8_dtype dt, int64_t token
  *       positions left out; clamped context lengths are counted once per
  *       sequence.  Nothing outside the cache is read.
  * Alignment: caches 16 bytes; q and out their element size; scales, tables,
- * lengths and errors 4 bytes.  flags: PGF8_FLAG_OVERLAP_PREVIOUS.
- * seqs == 0 is a no-op.  Results do not depend on scheduling.
+ * lengths and errors 4 bytes.  flags: PGF8_FLAG_OVERLAP_PREVIOUS,
+ * PGF8_FLAG_ATTN_MMA.  seqs == 0 is a no-op.  Results do not depend on
+ * scheduling.
  * ---------------------------------------------------------------------- */
 typedef struct {
     const uint8_t *k_cache;   /* [num_blocks, kv_heads, block_size, head_dim] E4M3 codes */

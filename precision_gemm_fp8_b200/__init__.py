@@ -34,6 +34,7 @@ NESTED_FP16, NESTED_FP8 = 0, 1
 PATH_AUTO, PATH_SKINNY, PATH_TILED, PATH_STREAMK, PATH_TILED_PAIR = 0, 1, 2, 3, 4
 FLAG_OVERLAP_PREVIOUS = 1
 FLAG_FUSED_QUANT = 2
+FLAG_ATTN_MMA = 4
 
 
 class LinearOpts(ctypes.Structure):

@@ -9,10 +9,12 @@
 // the context, output sum p * v * s_v.
 //
 // HBM-bound: a decoded token costs 2·D bytes of K and V codes against about
-// 4·G·D flops for the G query heads that share its KV head, so the kernel
-// streams the cache with 128-bit (K) and coalesced (V) loads on the CUDA
-// cores; there is no contraction here wide enough for the tensor cores to
-// pay.  The context is split into chunks ("flash-decoding"): one CTA per
+// 4·G·D flops for the G query heads that share its KV head.  The first
+// kernel streams the cache with 128-bit (K) and coalesced (V) loads on the
+// CUDA cores, which keep up with HBM for one or two heads per KV head; the
+// second (attn_decode_mma_kernel, on request) puts both products on the
+// tensor cores with the heads as the MMA's N dimension, for larger groups.
+// The context is split into chunks ("flash-decoding"): one CTA per
 // (chunk, KV head, group of GT query heads, sequence) keeps each SM busy
 // when the batch is small.  Each CTA reduces its chunk to a running maximum
 // m, a sum l and an unnormalised output o per query head (online softmax,
@@ -362,6 +364,272 @@ __global__ void __launch_bounds__(D) attn_decode_combine_kernel(const float *__r
         }
     }
     store_elem(out, s * ldo + h * D + d, odt, L > 0.0f ? O / L * sv[h / (Hq / Hkv)] : 0.0f);
+}
+
+// ---------------------------------------------------------------------------
+// The same decode attention with both products on the tensor cores
+// (mma.sync m16n8k16, binary16 operands, binary32 accumulation), for query
+// heads that share a KV head: the up to 8 heads of a CTA are the MMA's N
+// dimension, so one K / V load serves all of them in one instruction.
+//   scores^T [16 positions x 8 heads] = K [16 x D] . Q^T [D x 8]
+//   O^T [D x 8 heads] += V^T [D x 16 positions] . P^T [16 x 8]
+// K and V codes widen exactly to binary16 (cvt from E4M3 pairs); q and the
+// probabilities are rounded to binary16.  The contraction index of each
+// product is permuted (the sum does not depend on its order) so that every
+// thread loads whole 16-byte pieces of the rows it needs: for QK, thread
+// (g = lane / 4, t4 = lane % 4) holds bytes [D/4 t4, D/4 t4 + D/4) of
+// positions g and g + 8, k-step j taking bytes 4j .. 4j + 3 of that piece;
+// for PV it holds bytes [D/8 g, D/8 g + D/8) of positions 4 t4 .. 4 t4 + 3,
+// output block b taking dims D/8 g + 2b (MMA row g) and D/8 g + 2b + 1
+// (row g + 8).  The probabilities move from the score layout (positions
+// g, g + 8; heads 2 t4, 2 t4 + 1) to the operand layout (heads g;
+// positions 4 t4 .. 4 t4 + 3) through 256 bytes of shared memory per warp.
+// Grid, chunks, masks, merge and outputs as attn_decode_paged_kernel.
+
+__device__ __forceinline__ uint32_t e4m3x2_to_h2bits(uint32_t two)
+{
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xFFFFu), __NV_E4M3);
+    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
+__device__ __forceinline__ uint32_t f32x2_to_h2bits(float lo, float hi)
+{
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// D(16x8, f32) += A(16x16, f16, row) . B(16x8, f16, col)
+__device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1)
+{
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                 "{%8, %9}, {%0, %1, %2, %3};"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// N / 4 32-bit words of one row piece, loaded as 16-byte (or 8-byte) words.
+template <int NBYTES> struct RowPiece {
+    static constexpr int kWords = NBYTES / 4;
+    uint32_t w[kWords];
+    __device__ __forceinline__ void load(const uint8_t *p)
+    {
+        if constexpr (NBYTES == 8) {
+            const uint2 t = __ldg(reinterpret_cast<const uint2 *>(p));
+            w[0] = t.x;
+            w[1] = t.y;
+        } else {
+#pragma unroll
+            for (int i = 0; i < NBYTES / 16; ++i) {
+                const uint4 t = __ldg(reinterpret_cast<const uint4 *>(p) + i);
+                w[4 * i + 0] = t.x;
+                w[4 * i + 1] = t.y;
+                w[4 * i + 2] = t.z;
+                w[4 * i + 3] = t.w;
+            }
+        }
+    }
+    __device__ __forceinline__ void zero()
+    {
+#pragma unroll
+        for (int i = 0; i < kWords; ++i)
+            w[i] = 0u;
+    }
+};
+
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads) attn_decode_mma_kernel(const AttnDecodeArgs a)
+{
+    static_assert(D == 64 || D == 128 || D == 256, "head_dim 64, 128 or 256");
+    constexpr int KSTEPS = D / 16;   // k-steps of the QK product
+    constexpr int KSEG = D / 4;      // bytes of a K row per thread
+    constexpr int VSEG = D / 8;      // bytes of a V row per thread
+    constexpr int DB = D / 16;       // 16-row blocks of the PV product
+
+    __shared__ __align__(16) __half ps[kAttnWarps][8][kAttnStep];   // probabilities [head][position]
+    __shared__ float red_m[kAttnWarps][8], red_l[kAttnWarps][8];
+    __shared__ __align__(16) float red_o[kAttnWarps][8][D];
+
+    grid_launch_dependents();
+    grid_dependency_wait();   // q from the QKV projection, the cache from its writer
+
+    const int sp = blockIdx.x;
+    const int G = static_cast<int>(a.Hq / a.Hkv);
+    const int64_t hk = blockIdx.y / a.groups;
+    const int gi = static_cast<int>(blockIdx.y % a.groups);
+    const int nh = G - gi * 8 < 8 ? G - gi * 8 : 8;   // query heads of this CTA
+    const int64_t h0 = hk * G + gi * 8;
+    const int64_t s = blockIdx.z;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t4 = lane & 3;
+
+    // Q^T operand of every k-step: head g (zero for the padding heads)
+    uint32_t qb[KSTEPS][2];
+#pragma unroll
+    for (int j = 0; j < KSTEPS; ++j) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int d = KSEG * t4 + 4 * j + 2 * e;
+            float x0 = 0.0f, x1 = 0.0f;
+            if (g < nh) {
+                const int64_t base = s * a.ldq + (h0 + g) * D + d;
+                x0 = load_elem(a.q, base, a.qdt);
+                x1 = load_elem(a.q, base + 1, a.qdt);
+            }
+            qb[j][e] = f32x2_to_h2bits(x0, x1);
+        }
+    }
+
+    int64_t ctx = a.ctx_lens[s];
+    if (ctx < 0 || ctx > a.max_ctx) {
+        if (a.errors && threadIdx.x == 0 && sp == 0 && blockIdx.y == 0)
+            atomicAdd(a.errors, 1);
+        ctx = ctx < 0 ? 0 : a.max_ctx;
+    }
+    const int64_t t_begin = static_cast<int64_t>(sp) * a.chunk;
+    const int64_t t_end = t_begin + a.chunk < ctx ? t_begin + a.chunk : ctx;
+    const float scale = a.sk[hk] * a.qscale;   // base-2 units
+
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.0f, 0.0f};   // heads 2 t4, 2 t4 + 1
+    float o[DB][4];
+#pragma unroll
+    for (int b = 0; b < DB; ++b)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            o[b][i] = 0.0f;
+
+    for (int64_t base = t_begin + kAttnStep * w; base < t_end; base += kAttnStep * kAttnWarps) {
+        const int nvalid = t_end - base < kAttnStep ? static_cast<int>(t_end - base) : kAttnStep;
+        const int64_t blk = a.tables[s * a.table_stride + base / a.B];
+        if (blk < 0 || blk >= a.num_blocks) {   // warp-uniform
+            if (a.errors && lane == 0 && blockIdx.y == 0)
+                atomicAdd(a.errors, 1);
+            continue;
+        }
+        const int64_t row0 = (blk * a.Hkv + hk) * a.B + base % a.B;
+
+        // every load of the step first; rows past the context read as zeros
+        RowPiece<KSEG> k0, k1;
+        if (g < nvalid)
+            k0.load(a.kc + (row0 + g) * D + KSEG * t4);
+        else
+            k0.zero();
+        if (g + 8 < nvalid)
+            k1.load(a.kc + (row0 + g + 8) * D + KSEG * t4);
+        else
+            k1.zero();
+        RowPiece<VSEG> v[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            if (4 * t4 + r < nvalid)
+                v[r].load(a.vc + (row0 + 4 * t4 + r) * D + VSEG * g);
+            else
+                v[r].zero();
+        }
+
+        // scores^T = K . Q^T
+        float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int j = 0; j < KSTEPS; ++j)
+            mma_16816(c, e4m3x2_to_h2bits(k0.w[j]), e4m3x2_to_h2bits(k1.w[j]), e4m3x2_to_h2bits(k0.w[j] >> 16),
+                      e4m3x2_to_h2bits(k1.w[j] >> 16), qb[j][0], qb[j][1]);
+
+        // online softmax; c[0], c[1]: position g, heads 2 t4, 2 t4 + 1; c[2], c[3]: position g + 8
+        const bool v0 = g < nvalid, v1 = g + 8 < nvalid;
+        float pr[4];
+        float alpha[2];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const float s0 = v0 ? c[hh] * scale : -INFINITY;
+            const float s1 = v1 ? c[2 + hh] * scale : -INFINITY;
+            float mx = fmaxf(s0, s1);
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1)
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            const float mn = fmaxf(m[hh], mx);   // finite: position `base` is valid
+            alpha[hh] = m[hh] == -INFINITY ? 0.0f : exp2f(m[hh] - mn);
+            pr[hh] = v0 ? exp2f(s0 - mn) : 0.0f;
+            pr[2 + hh] = v1 ? exp2f(s1 - mn) : 0.0f;
+            float psum = pr[hh] + pr[2 + hh];
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1)
+                psum += __shfl_xor_sync(0xffffffffu, psum, off);
+            l[hh] = l[hh] * alpha[hh] + psum;
+            m[hh] = mn;
+        }
+#pragma unroll
+        for (int b = 0; b < DB; ++b) {
+            o[b][0] *= alpha[0];
+            o[b][1] *= alpha[1];
+            o[b][2] *= alpha[0];
+            o[b][3] *= alpha[1];
+        }
+        ps[w][2 * t4][g] = __float2half_rn(pr[0]);
+        ps[w][2 * t4 + 1][g] = __float2half_rn(pr[1]);
+        ps[w][2 * t4][g + 8] = __float2half_rn(pr[2]);
+        ps[w][2 * t4 + 1][g + 8] = __float2half_rn(pr[3]);
+        __syncwarp();
+        const uint2 pb = *reinterpret_cast<const uint2 *>(&ps[w][g][4 * t4]);   // positions 4 t4 .. 4 t4 + 3
+
+        // O^T += V^T . P^T
+#pragma unroll
+        for (int b = 0; b < DB; ++b) {
+            const int wi = b >> 1, sh = 2 * (b & 1);
+            // bytes (row r byte sh, row r+1 byte sh, row r byte sh+1, row r+1 byte sh+1)
+            const uint32_t sel = static_cast<uint32_t>(sh | ((4 + sh) << 4) | ((sh + 1) << 8) | ((5 + sh) << 12));
+            const uint32_t x01 = __byte_perm(v[0].w[wi], v[1].w[wi], sel);
+            const uint32_t x23 = __byte_perm(v[2].w[wi], v[3].w[wi], sel);
+            mma_16816(o[b], e4m3x2_to_h2bits(x01), e4m3x2_to_h2bits(x01 >> 16), e4m3x2_to_h2bits(x23),
+                      e4m3x2_to_h2bits(x23 >> 16), pb.x, pb.y);
+        }
+        __syncwarp();   // ps is rewritten by the next step
+    }
+
+    // merge the warps' partial softmax states
+    if (g == 0) {
+        red_m[w][2 * t4] = m[0];
+        red_m[w][2 * t4 + 1] = m[1];
+        red_l[w][2 * t4] = l[0];
+        red_l[w][2 * t4 + 1] = l[1];
+    }
+#pragma unroll
+    for (int b = 0; b < DB; ++b) {
+        const int d = VSEG * g + 2 * b;
+        red_o[w][2 * t4][d] = o[b][0];
+        red_o[w][2 * t4 + 1][d] = o[b][1];
+        red_o[w][2 * t4][d + 1] = o[b][2];
+        red_o[w][2 * t4 + 1][d + 1] = o[b][3];
+    }
+    __syncthreads();
+
+    const float vscale = a.sv[hk];
+    for (int e = threadIdx.x; e < nh * D; e += kAttnThreads) {
+        const int hh = e / D, d = e % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int ww = 0; ww < kAttnWarps; ++ww)
+            M = fmaxf(M, red_m[ww][hh]);
+        float L = 0.0f, O = 0.0f;
+#pragma unroll
+        for (int ww = 0; ww < kAttnWarps; ++ww) {
+            if (red_m[ww][hh] != -INFINITY) {
+                const float f = exp2f(red_m[ww][hh] - M);
+                L = fmaf(red_l[ww][hh], f, L);
+                O = fmaf(red_o[ww][hh][d], f, O);
+            }
+        }
+        const int64_t h = h0 + hh;
+        if (a.nsplit == 1) {
+            store_elem(a.out, s * a.ldo + h * D + d, a.odt, L > 0.0f ? O / L * vscale : 0.0f);
+        } else {
+            float *pp = a.part + ((s * a.Hq + h) * a.nsplit + sp) * (D + 2);
+            pp[d] = O;
+            if (d == 0) {
+                pp[D] = M;
+                pp[D + 1] = L;
+            }
+        }
+    }
 }
 
 } // namespace pgf8

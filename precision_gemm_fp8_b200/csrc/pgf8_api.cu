@@ -734,14 +734,23 @@ static pgf8_status launch_attn_gt(const AttnDecodeArgs &a, int64_t seqs, cudaStr
 }
 
 template <int D>
-static pgf8_status launch_attn(const AttnDecodeArgs &a, int gt, int64_t seqs, cudaStream_t st, int pdl)
+static pgf8_status launch_attn(const AttnDecodeArgs &a, int gt, bool mma, int64_t seqs, cudaStream_t st, int pdl)
 {
     pgf8_status r;
-    switch (gt) {
-    case 8: r = launch_attn_gt<D, 8>(a, seqs, st, pdl); break;
-    case 4: r = launch_attn_gt<D, 4>(a, seqs, st, pdl); break;
-    case 2: r = launch_attn_gt<D, 2>(a, seqs, st, pdl); break;
-    default: r = launch_attn_gt<D, 1>(a, seqs, st, pdl); break;
+    if (mma) {
+        // up to 8 query heads of one KV head per CTA: the MMA's N dimension
+        AttnDecodeArgs am = a;
+        am.groups = static_cast<int>((a.Hq / a.Hkv + 7) / 8);
+        const dim3 grid(static_cast<unsigned>(a.nsplit), static_cast<unsigned>(a.Hkv * am.groups),
+                        static_cast<unsigned>(seqs));
+        r = launch_grid(attn_decode_mma_kernel<D>, grid, dim3(kAttnThreads), st, pdl, am);
+    } else {
+        switch (gt) {
+        case 8: r = launch_attn_gt<D, 8>(a, seqs, st, pdl); break;
+        case 4: r = launch_attn_gt<D, 4>(a, seqs, st, pdl); break;
+        case 2: r = launch_attn_gt<D, 2>(a, seqs, st, pdl); break;
+        default: r = launch_attn_gt<D, 1>(a, seqs, st, pdl); break;
+        }
     }
     if (r != PGF8_OK || a.nsplit == 1)
         return r;
@@ -1011,11 +1020,12 @@ pgf8_status pgf8_fp8_attention_decode_paged(const void *q, pgf8_dtype q_dt, int6
     a.errors = errors;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const int pdl = (flags & PGF8_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
+    const bool mma = (flags & PGF8_FLAG_ATTN_MMA) != 0;
     if (D == 64)
-        return launch_attn<64>(a, p.gt, seqs, cs, pdl);
+        return launch_attn<64>(a, p.gt, mma, seqs, cs, pdl);
     if (D == 128)
-        return launch_attn<128>(a, p.gt, seqs, cs, pdl);
-    return launch_attn<256>(a, p.gt, seqs, cs, pdl);
+        return launch_attn<128>(a, p.gt, mma, seqs, cs, pdl);
+    return launch_attn<256>(a, p.gt, mma, seqs, cs, pdl);
 }
 
 pgf8_status pgf8_fp8_attention_context_paged(const uint8_t *q_codes, const float *q_scales,

@@ -6,15 +6,19 @@ GPU parity of the FP8 paged decode attention against the oracle ("7B on
 an RTX 4060 with FP8": K/V held in FP8; "C++ and FP8" §3.2 paged cache of
 16-token blocks, §3.3 attention in the FP8 dataflow).
 
-The kernel works in binary32 on the dequantised cache; the oracle in
-binary64 on the same codes and the same (binary32) queries.  Bound per
+The CUDA-core kernel works in binary32 on the dequantised cache; the oracle
+in binary64 on the same codes and the same (binary32) queries.  Bound per
 output element d of a (sequence, head), from the binary32 steps:
   logit error (base 2)  D_t <= (D + 4) 2^-24 sum_d |q_d k_td| s_k log2(e)/sqrt(D)
   weight error          |dp_t / p_t| <= 2 ln2 max_t D_t + 2^-21 (two exp2f)
   sums over T positions (T + 16) 2^-24 (sequential accumulation per warp)
   |out - ref| <= (2 (2 ln2 D + 2^-21) + (T + 16) 2^-24) max_t |v_td s_v|
                  + rounding of the output (2^-24, 2^-11 or 2^-8 of |ref|),
-taken twice for margin."""
+taken twice for margin.  The tensor-core kernel (PGF8_FLAG_ATTN_MMA) also
+rounds q and the probabilities to binary16 (2^-11 relative, 2^-25 absolute
+below the normal range) and accumulates on the tensor cores: its logit term
+gains 2^-11 sum_d |q_d k_td| (and 2^-22 per addition), its weights 2^-11 plus
+2^-25 T absolute."""
 import math
 
 import numpy as np
@@ -35,7 +39,7 @@ def _to(a):
     return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
 
 
-def _tolerance(q, K, V, ctx, out_dtype):
+def _tolerance(q, K, V, ctx, out_dtype, mma=False):
     """Per-element bound [Hq, D] for one sequence (see the module docstring)."""
     Hq, D = q.shape
     Hkv = K.H
@@ -45,9 +49,12 @@ def _tolerance(q, K, V, ctx, out_dtype):
     tol = np.empty((Hq, D))
     for h in range(Hq):
         hk = h // G
-        dl = (D + 4) * 2.0 ** -24 * np.abs(kd[:, hk, :] * q[h][None, :]).sum(axis=1).max() * \
+        rel = (2.0 ** -11 + (D + 4) * 2.0 ** -22) if mma else (D + 4) * 2.0 ** -24
+        dl = rel * np.abs(kd[:, hk, :] * q[h][None, :]).sum(axis=1).max() * \
             K.scales[hk] * math.log2(math.e) / math.sqrt(D)
         eps = 2 * (2 * math.log(2) * dl + 2.0 ** -21) + (ctx + 16) * 2.0 ** -24
+        if mma:
+            eps += 2.0 ** -11 + 2.0 ** -25 * ctx + (ctx + 16) * 2.0 ** -22
         tol[h] = 2 * eps * np.abs(vd[:, hk, :]).max(axis=0)
     return tol, OUT_ULP[out_dtype]
 
@@ -77,14 +84,14 @@ def _build(seqs, Hkv, D, B, ctxs, seed, kv_scale=1.0):
     return dict(kc=kc, vc=vc, sk=sk, sv=sv, tables=tables, refs=refs, max_ctx=max_ctx)
 
 
-def _run(c, q_dev, ctxs, out_dtype=torch.float32, splits=0, max_ctx=None, errors=None):
+def _run(c, q_dev, ctxs, out_dtype=torch.float32, splits=0, max_ctx=None, errors=None, mma=False):
     return pg.fp8_attention_decode_paged(q_dev, _to(c["kc"]), _to(c["vc"]), _to(c["sk"]), _to(c["sv"]),
                                          _to(c["tables"]), _to(np.array(ctxs, np.int32)),
                                          c["max_ctx"] if max_ctx is None else max_ctx, out_dtype=out_dtype,
-                                         splits=splits, errors=errors)
+                                         splits=splits, errors=errors, flags=pg.FLAG_ATTN_MMA if mma else 0)
 
 
-def _check(c, q, out, ctxs, out_dtype):
+def _check(c, q, out, ctxs, out_dtype, mma=False):
     got = out.to(torch.float32).cpu().numpy().astype(np.float64)
     for s, ctx in enumerate(ctxs):
         if ctx == 0:
@@ -92,12 +99,13 @@ def _check(c, q, out, ctxs, out_dtype):
             continue
         K, V = c["refs"][s]
         ref = oracle.attention_paged(q[s:s + 1].astype(np.float64), K, V, ctx)[0]
-        tol, ulp = _tolerance(q[s], K, V, ctx, out_dtype)
+        tol, ulp = _tolerance(q[s], K, V, ctx, out_dtype, mma)
         err = np.abs(got[s] - ref)
         bad = err > tol + ulp * np.abs(ref)
         assert not bad.any(), (s, ctx, float(err.max()), float(tol.max()))
 
 
+@pytest.mark.parametrize("mma", [False, True])
 @pytest.mark.parametrize("seqs,Hq,Hkv,D,B,ctxs,splits", [
     (3, 8, 8, 128, 16, [1, 77, 300], 0),          # MHA, ragged
     (3, 8, 8, 128, 16, [1, 77, 300], 1),          # one chunk: no merge kernel
@@ -106,13 +114,26 @@ def _check(c, q, out, ctxs, out_dtype):
     (2, 8, 2, 256, 16, [250, 31], 0),             # head_dim 256, 4 per KV head
     (4, 4, 4, 64, 16, [0, 15, 16, 17], 2),        # empty and block-edge contexts
 ])
-def test_decode_attention_matches_the_oracle(seqs, Hq, Hkv, D, B, ctxs, splits):
+def test_decode_attention_matches_the_oracle(seqs, Hq, Hkv, D, B, ctxs, splits, mma):
     c = _build(seqs, Hkv, D, B, ctxs, seed=seqs * 100 + Hq + D)
     q = np.random.default_rng(D).standard_normal((seqs, Hq, D)).astype(np.float32)
-    out = _run(c, _to(q), ctxs, splits=splits)
+    out = _run(c, _to(q), ctxs, splits=splits, mma=mma)
     torch.cuda.synchronize()
     assert pg.device_status() == pg.OK
-    _check(c, q, out, ctxs, torch.float32)
+    _check(c, q, out, ctxs, torch.float32, mma)
+
+
+@pytest.mark.parametrize("G", [1, 3, 8, 16])
+def test_tensor_core_path_across_group_sizes(G):
+    """Padding heads (G not a multiple of 8) and several CTAs per KV head (G = 16)."""
+    seqs, Hkv, D = 2, 2, 128
+    ctxs = [333, 64]
+    c = _build(seqs, Hkv, D, 16, ctxs, seed=50 + G)
+    q = np.random.default_rng(G).standard_normal((seqs, Hkv * G, D)).astype(np.float32)
+    out = _run(c, _to(q), ctxs, mma=True)
+    torch.cuda.synchronize()
+    assert pg.device_status() == pg.OK
+    _check(c, q, out, ctxs, torch.float32, mma=True)
 
 
 @pytest.mark.parametrize("qdt,odt", [(torch.float16, torch.bfloat16), (torch.bfloat16, torch.float16),
