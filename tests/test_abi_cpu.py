@@ -374,3 +374,19 @@ def test_attention_bindings_check_shapes_before_any_pointer():
         ctx(max_context=40)
     with pytest.raises(ValueError, match="device tensors"):
         ctx()
+
+
+def test_binding_constants_match_the_header():
+    """Every enum value and flag the binding names equals the header's."""
+    import re
+    text = open(pg.HEADER_PATH).read()
+    values = {m.group(1): int(m.group(2)) for m in re.finditer(r"\b(PGF8_[A-Z0-9_]+)\s*=\s*(\d+)", text)}
+    values.update({m.group(1): int(m.group(2)) for m in re.finditer(r"#define\s+(PGF8_FLAG_\w+)\s+(\d+)", text)})
+    names = ["OK", "ERR_INVALID_ARG", "ERR_ALIGNMENT", "ERR_UNSUPPORTED", "ERR_CUDA", "ERR_TIMEOUT", "ERR_TOO_LARGE",
+             "F32", "F16", "BF16", "SCALE_DYNAMIC", "SCALE_STATIC", "NESTED_FP16", "NESTED_FP8", "PATH_AUTO",
+             "PATH_SKINNY", "PATH_TILED", "PATH_STREAMK", "PATH_TILED_PAIR", "FLAG_OVERLAP_PREVIOUS",
+             "FLAG_FUSED_QUANT", "FLAG_ATTN_MMA"]
+    for n in names:
+        assert getattr(pg, n) == values["PGF8_" + n], n
+    flags = [values[k] for k in values if k.startswith("PGF8_FLAG_")]
+    assert len(set(flags)) == len(flags) and all(f & (f - 1) == 0 for f in flags)   # distinct single bits
