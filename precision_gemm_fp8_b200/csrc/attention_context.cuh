@@ -75,8 +75,45 @@ struct AttnCtxParams {
     void *out;                   // [total_q][Hq][128], token stride ldo elements
     int64_t ldo;
     int odt;
+    int vec_out;                 // out and its token stride allow 16-byte stores
     int32_t *errors;
 };
+
+// One query row of the output (128 values, already scaled) into `dst`:
+// 16-byte stores when allowed, else element by element.
+__device__ __forceinline__ void store_row128(void *out, int64_t base, int odt, bool vec, const float (&o)[128], float f)
+{
+    if (!vec) {
+#pragma unroll
+        for (int d = 0; d < 128; ++d)
+            store_elem(out, base + d, odt, o[d] * f);
+        return;
+    }
+    if (odt == 0) {
+        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(out) + base);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            dst[i] = make_float4(o[4 * i] * f, o[4 * i + 1] * f, o[4 * i + 2] * f, o[4 * i + 3] * f);
+        return;
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(out) + base);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        uint32_t w[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const float lo = o[8 * i + 2 * u] * f, hi = o[8 * i + 2 * u + 1] * f;
+            if (odt == 1) {
+                const __half2 hv = __floats2half2_rn(lo, hi);
+                w[u] = *reinterpret_cast<const uint32_t *>(&hv);
+            } else {
+                const __nv_bfloat162 bv = __floats2bfloat162_rn(lo, hi);
+                w[u] = *reinterpret_cast<const uint32_t *>(&bv);
+            }
+        }
+        dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
 
 // Shared-memory descriptor of an MN-major operand tile in the 128-byte
 // swizzled canonical layout: rows of 128 bytes along MN (one swizzle atom
@@ -388,9 +425,7 @@ __global__ void __launch_bounds__(192, 1) attn_context_kernel(const __grid_const
         if (ok && row_ok) {
             const float f = l > 0.0f ? p.sv[hk] * 0.00390625f / l : 0.0f;   // 2^-8 undoes the P code scale
             const int64_t base = (static_cast<int64_t>(q0) + qt * 128 + r) * p.ldo + static_cast<int64_t>(h) * 128;
-#pragma unroll
-            for (int d = 0; d < 128; ++d)
-                store_elem(p.out, base + d, p.odt, o[d] * f);
+            store_row128(p.out, base, p.odt, p.vec_out != 0, o, f);
         }
     }
 

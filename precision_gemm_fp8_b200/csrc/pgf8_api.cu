@@ -1094,6 +1094,7 @@ pgf8_status pgf8_fp8_attention_context_paged(const uint8_t *q_codes, const float
     a.out = out;
     a.ldo = ldo;
     a.odt = static_cast<int>(out_dt);
+    a.vec_out = aligned16(out) && (ldo * (out_dt == PGF8_F32 ? 4 : 2)) % 16 == 0;
     a.errors = errors;
 
     cudaLaunchConfig_t cfg;

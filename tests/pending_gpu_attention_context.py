@@ -170,3 +170,25 @@ def test_one_hot_values_expose_each_key_probability():
     got = out.cpu().numpy()[0, 0].astype(np.float64)
     np.testing.assert_allclose(got, ref[0, 0], rtol=0, atol=2.0 ** -14)
     assert abs(got.sum() - 1.0) < 1e-5            # the probabilities of all keys add up to 1
+
+
+def test_strided_output_rows():
+    """Output rows with a padded token stride: 16-byte-aligned strides take the
+    packed stores, others the element stores; both land in place."""
+    c = _case(1, 2, 1, 16, [140], [140], seed=11, exact=True)
+    total_q, Hq, D = c["q"].shape
+    qc_dev, qs_dev = pg.fp8_quantize_rows(_to(c["q"]).view(total_q * Hq, D))
+    ref = _reference(c, qc_dev.view(total_q, Hq, D).cpu().numpy(), qs_dev.cpu().numpy())
+    for pad, dt in ((8, torch.bfloat16), (2, torch.bfloat16), (1, torch.float32)):
+        wide = torch.full((total_q, Hq * D + pad), float("nan"), dtype=dt, device=DEV)
+        out = torch.as_strided(wide, (total_q, Hq, D), (Hq * D + pad, D, 1))
+        pg.fp8_attention_context_paged(qc_dev.view(total_q, Hq, D), qs_dev, _to(c["q_start"]),
+                                       _to(np.array(c["ctxs"], np.int32)), _to(c["kc"]), _to(c["vc"]),
+                                       _to(c["sk"]), _to(c["sv"]), _to(c["tables"]), c["max_ctx"], c["max_q_len"],
+                                       out=out)
+        torch.cuda.synchronize()
+        assert pg.device_status() == pg.OK
+        ulp = 2.0 ** -8 if dt == torch.bfloat16 else 2.0 ** -24
+        got = out.to(torch.float32).cpu().numpy()
+        assert (np.abs(got - ref) <= 2.0 ** -14 * _vmax(c) + ulp * np.abs(ref)).all()
+        assert torch.isnan(wide[:, Hq * D:].to(torch.float32)).all()     # the padding is untouched
