@@ -13,7 +13,7 @@
 //   O = P . V_codes . 2^-8 . sv / l
 // l sums the unrounded probabilities.  head_dim 128.
 //
-// One CTA per (128-query tile, query head, sequence), 192 threads:
+// One CTA per (128-query tile, query head, sequence), heaviest tiles first, 192 threads:
 //   warp 0      TMA: the Q tile once, then per 128-key tile eight 16-row
 //               pieces of K and of V straight from the paged cache (a piece
 //               past the context, or of an out-of-range block, is read at a
@@ -155,7 +155,11 @@ __global__ void __launch_bounds__(192, 1) attn_context_kernel(const __grid_const
     constexpr uint32_t kIdescPV = make_idesc(128, 128, 0, 0) | (1u << 16);    // P (K-major) x V (MN-major)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qt = blockIdx.x, h = blockIdx.y;
+    // grid.x = query tiles x heads, heaviest (last) tiles of every head
+    // first: causal tiles differ in length, and the short ones fill in last
+    const int nqt = static_cast<int>(gridDim.x) / p.Hq;
+    const int h = static_cast<int>(blockIdx.x) % p.Hq;
+    const int qt = nqt - 1 - static_cast<int>(blockIdx.x) / p.Hq;
     const int64_t s = blockIdx.z;
     const int hk = h / (p.Hq / p.Hkv);
     const int q0 = p.q_start[s];
@@ -168,7 +172,7 @@ __global__ void __launch_bounds__(192, 1) attn_context_kernel(const __grid_const
             atomicAdd(p.errors, 1);
         return;                                          // an invalid sequence is not written
     }
-    if (qt == 0 && h == 0 && threadIdx.x == 0 && p.errors && q_len > static_cast<int>(gridDim.x) * 128)
+    if (qt == 0 && h == 0 && threadIdx.x == 0 && p.errors && q_len > nqt * 128)
         atomicAdd(p.errors, 1);                          // longer than the grid covers: the tail is not written
     const int nrows = q_len - qt * 128 < 128 ? q_len - qt * 128 : 128;
     const int pos0 = ctx - q_len + qt * 128;            // position of the tile's first query

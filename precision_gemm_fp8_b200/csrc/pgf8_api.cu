@@ -1038,7 +1038,8 @@ pgf8_status pgf8_fp8_attention_context_paged(const uint8_t *q_codes, const float
     if (!cache)
         return PGF8_ERR_INVALID_ARG;
     const int64_t Hkv = cache->kv_heads, D = cache->head_dim, B = cache->block_size;
-    if (seqs < 0 || seqs > 65535 || total_q < 0 || total_q >= (1ll << 31) || max_q_len < 0 || Hkv < 1 ||
+    if (seqs < 0 || seqs > 65535 || total_q < 0 || total_q >= (1ll << 31) || max_q_len < 0 ||
+        max_q_len >= (1ll << 31) || (max_q_len + 127) / 128 * q_heads >= (1ll << 31) || Hkv < 1 ||
         q_heads < Hkv || q_heads % Hkv != 0 || q_heads > 65535 || B < 16 || B % 16 != 0 || cache->num_blocks < 1 ||
         max_context < 0 || table_stride < 1 || max_context > table_stride * B || max_context >= (1ll << 31) ||
         ldo < q_heads * 128 || cache->num_blocks * Hkv * B >= (1ll << 31) - 1)
@@ -1099,8 +1100,7 @@ pgf8_status pgf8_fp8_attention_context_paged(const uint8_t *q_codes, const float
 
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3(static_cast<unsigned>((max_q_len + 127) / 128), static_cast<unsigned>(q_heads),
-                       static_cast<unsigned>(seqs));
+    cfg.gridDim = dim3(static_cast<unsigned>((max_q_len + 127) / 128 * q_heads), 1, static_cast<unsigned>(seqs));
     cfg.blockDim = dim3(192);
     cfg.dynamicSmemBytes = kCtxSmemBytes;
     cfg.stream = static_cast<cudaStream_t>(stream);
