@@ -165,13 +165,13 @@ __global__ void __launch_bounds__(192, 1) attn_context_kernel(const __grid_const
     const int q0 = p.q_start[s];
     const int q_len = p.q_start[s + 1] - q0;
     const int ctx = p.ctx_lens[s];
-    if (q_len <= qt * 128)
-        return;                                          // CTA-uniform: no tile here
     if (q_len < 0 || q0 < 0 || q0 + q_len > p.total_q || ctx < q_len || ctx > p.max_ctx) {
         if (threadIdx.x == 0 && qt == 0 && h == 0 && p.errors)
             atomicAdd(p.errors, 1);
         return;                                          // an invalid sequence is not written
     }
+    if (q_len <= qt * 128)
+        return;                                          // CTA-uniform: no tile here
     if (qt == 0 && h == 0 && threadIdx.x == 0 && p.errors && q_len > nqt * 128)
         atomicAdd(p.errors, 1);                          // longer than the grid covers: the tail is not written
     const int nrows = q_len - qt * 128 < 128 ? q_len - qt * 128 : 128;
