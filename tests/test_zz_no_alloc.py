@@ -4,10 +4,14 @@ It serves callers that cannot hand the library a workspace (a host program
 that links only the C library and has no device allocator, or a runtime that
 plans all device memory before serving and forbids allocating on the request
 path).  Its codes and scales live in the library's fixed device array, which
-every call shares and which keeps the previous call's contents, so the test
-makes two calls in a row with different inputs and checks each one against
-the workspace-taking entry point within the layer's stated bound.  The file
-sorts last so a run that stops at the first failure has run everything else.
+every call shares and which keeps the previous call's contents.  It runs the
+same kernels as the workspace-taking entry point, so the test makes two calls
+in a row with different inputs and different token counts (M = 8, then 64:
+the scales move inside the shared array between the two), and checks each
+output bit for bit against the workspace-taking entry point, whose codes and
+scales it checks bit for bit against the oracle, and the output against the
+oracle's binary64 layer within the stated bound.  The file sorts last so a
+run that stops at the first failure has run everything else.
 """
 import ctypes
 
@@ -36,11 +40,11 @@ def _call_noalloc(x, wq, sw, y):
 def test_noalloc_matches_workspace_entry_point_twice():
     torch.cuda.set_device(0)
     g = np.random.default_rng(2024)
-    M, K, N = 8, 4096, 4096
+    K, N = 4096, 4096
     w = synthetic.weights_f16(N, K, 0.02, g)
     wq, sw = pg.fp8_quantize_rows(torch.from_numpy(w).to(DEV))
     wq0, sw0 = oracle.quantize_rows(w)
-    for call in range(2):                       # two calls in a row share the fixed array
+    for call, M in enumerate((8, 64)):          # two calls in a row share the fixed array
         x = synthetic.activations("normal_outl_0p5pct_x30", M, K, g)
         xt = torch.from_numpy(x).to(DEV)
         y_na = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
@@ -49,10 +53,14 @@ def test_noalloc_matches_workspace_entry_point_twice():
         y_ws = pg.fp8_linear_dynamic(xt, wq, sw, workspace=ws)
         torch.cuda.synchronize()
         assert pg.device_status() == pg.OK
+        assert torch.equal(y_na.view(torch.int16), y_ws.view(torch.int16)), f"call {call}: outputs differ"
         aq0, sa0 = oracle.quantize_rows(x)
-        ref = y_ws.float().cpu().numpy().astype(np.float64)
+        aq, sa = pg.dynamic_workspace_views(ws, M, K)
+        assert np.array_equal(aq.cpu().numpy(), aq0), f"call {call}: codes differ from the oracle"
+        assert np.array_equal(sa.cpu().numpy().view(np.uint32), sa0.view(np.uint32)), f"call {call}: scales"
+        ref = oracle.fp8_linear(aq0, sa0, wq0, sw0)
         bound = linear_bound(ref, K, fp8_row_max(aq0, sa0), fp8_row_max(wq0, sw0))
-        assert_within(y_na.float().cpu().numpy(), ref, bound, f"no-alloc call {call}")
+        assert_within(y_na.float().cpu().numpy(), ref, bound, f"no-alloc call {call} (M={M})")
 
 
 def test_noalloc_rejects_problems_beyond_the_array():
