@@ -438,6 +438,44 @@ pgf8_status pgf8_fp8_linear_dynamic_many(const pgf8_fp8_layer *layers, int64_t c
 size_t pgf8_fp8_linear_dynamic_scales_offset(int64_t M, int64_t K);
 
 /* ------------------------------------------------------------------------
+ * A group of INDEPENDENT dynamic FP8 linear layers (no layer reads another
+ * layer's output: the linears of several sequences or of one decoder step
+ * measured as a batch, the separate Q, K, V or gate and up projections)
+ * enqueued by one call on `stream`.  Each layer computes exactly what
+ * pgf8_fp8_linear_dynamic computes ("7B on an RTX 4060 with FP8" §2.2
+ * per-token dynamic scale, §6.1 scale = amax / 448; "C++ and FP8" §3.3
+ * E4M3 x E4M3 -> f32 -> bf16): its codes and scales in its own workspace
+ * are bit-identical to that call's, its outputs are within the same bound
+ * (the f32 summation order differs).
+ *
+ * Layers with M <= 128 are quantised by one launch and then streamed by one
+ * persistent grouped kernel (one CTA per SM, each SM streaming an equal
+ * share of all those layers' weights, up to 32 layers per launch pair);
+ * larger layers run one dynamic call each afterwards.  Decode-sized layers
+ * are bound by their weight stream ("7B token speed on consumer GPUs" §1),
+ * and one stream for the whole group pays the start and the end of a
+ * launch once instead of once per layer.
+ *
+ * group_workspace: pgf8_fp8_linear_group_workspace_size(max M over the
+ * layers) bytes of device memory, 16-byte aligned, zero-filled once before
+ * its first use; every completed call leaves its flag words zero again, so
+ * it is reused without clearing.  Calls that use one group workspace must
+ * not overlap on the GPU.  May be null when no layer has M <= 128.
+ * Errors: any layer's own argument errors (nothing is enqueued);
+ * PGF8_ERR_INVALID_ARG when an output or workspace of one layer overlaps
+ * an input, output or workspace of another (or its own input), or the
+ * group workspace is missing or too small; PGF8_ERR_ALIGNMENT for an
+ * unaligned group workspace.  Deterministic for a fixed group of shapes on
+ * a fixed device.  PGF8_FLAG_OVERLAP_PREVIOUS in opts applies to the first
+ * launch.  The pages have no grouped form: this is how this library
+ * streams a step's decode linears on B200.
+ * ---------------------------------------------------------------------- */
+pgf8_status pgf8_fp8_linear_dynamic_group(const pgf8_fp8_layer *layers, int64_t count,
+                                          void *group_workspace, size_t group_workspace_bytes,
+                                          const pgf8_linear_opts *opts, void *stream);
+size_t pgf8_fp8_linear_group_workspace_size(int64_t max_m);
+
+/* ------------------------------------------------------------------------
  * NestedFP byte-plane split ("NestedFP" §2.1): for each FP16 weight bit
  * pattern b of w_f16 [N,K]: hi[n,k] = b >> 8 (sign, 5 exponent bits, top 2
  * mantissa bits), lo[n,k] = b & 0xFF.  Bit-exact; (hi << 8) | lo == b.

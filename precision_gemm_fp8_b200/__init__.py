@@ -85,6 +85,8 @@ _SIGS = {
     "pgf8_fp8_linear_dynamic_codes_offset": ([_i64, _i64], _sz),
     "pgf8_fp8_linear_dynamic_many": ([ctypes.POINTER(Fp8Layer), _i64, _optp, _vp], _i32),
     "pgf8_fp8_linear_dynamic_scales_offset": ([_i64, _i64], _sz),
+    "pgf8_fp8_linear_dynamic_group": ([ctypes.POINTER(Fp8Layer), _i64, _vp, _sz, _optp, _vp], _i32),
+    "pgf8_fp8_linear_group_workspace_size": ([_i64], _sz),
     "pgf8_nestedfp_split": ([_vp, _i64, _i64, _vp, _vp, _vp], _i32),
     "pgf8_nestedfp_linear": ([_vp, _i64, _i64, _vp, _vp, _i64, _i32, _vp, _vp, _sz, _vp], _i32),
     "pgf8_nestedfp_linear_ex": ([_vp, _i64, _i64, _vp, _vp, _i64, _i32, _vp, _vp, _sz, _optp, _vp], _i32),
@@ -536,6 +538,34 @@ class LayerSequence:
     def run(self, flags=0, stream=None):
         _check(lib.pgf8_fp8_linear_dynamic_many(self._arr, self.count, _opts(flags=flags), _stream(stream)),
                "fp8_linear_dynamic_many")
+
+
+class LayerGroup(LayerSequence):
+    """A fixed group of INDEPENDENT dynamic FP8 layers (no layer reads another
+    layer's output), run by one call of pgf8_fp8_linear_dynamic_group: the
+    layers with M <= 128 stream their weights through one grouped kernel.
+    Entries as LayerSequence; the group workspace is allocated (zero-filled)
+    here unless given."""
+
+    def __init__(self, layers, group_workspace=None):
+        super().__init__(layers)
+        max_m = max((x.shape[0] for (x, _, _, _, _) in self._keep), default=0)
+        need = group_workspace_size(max_m)
+        if group_workspace is None:
+            dev = self._keep[0][0].device if self._keep else "cuda"
+            group_workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
+        elif _nbytes(group_workspace) < need:
+            raise ValueError(f"group workspace needs {need} bytes")
+        self.group_workspace = group_workspace
+
+    def run(self, flags=0, stream=None):
+        _check(lib.pgf8_fp8_linear_dynamic_group(self._arr, self.count, _ptr(self.group_workspace),
+                                                 _nbytes(self.group_workspace), _opts(flags=flags), _stream(stream)),
+               "fp8_linear_dynamic_group")
+
+
+def group_workspace_size(max_m: int) -> int:
+    return int(lib.pgf8_fp8_linear_group_workspace_size(max_m))
 
 
 def dynamic_workspace_views(workspace: torch.Tensor, M: int, K: int):

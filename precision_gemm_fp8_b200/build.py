@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpgf8.so")
 SOURCES = ["pgf8_api.cu"]
-DEPS = ["pgf8_api.cu", "gemm.cuh", "gemm_persistent.cuh", "gemm_streamk.cuh", "gemm_2sm.cuh", "quantize.cuh", "sm100_ptx.cuh",
+DEPS = ["pgf8_api.cu", "gemm.cuh", "gemm_persistent.cuh", "gemm_streamk.cuh", "gemm_2sm.cuh", "gemm_group.cuh", "quantize.cuh", "sm100_ptx.cuh",
         "kvcache.cuh", "attention.cuh", "attention_context.cuh"]
 
 

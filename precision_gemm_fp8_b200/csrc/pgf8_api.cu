@@ -16,6 +16,7 @@
 #include "gemm_persistent.cuh"
 #include "gemm_streamk.cuh"
 #include "gemm_2sm.cuh"
+#include "gemm_group.cuh"
 #include "quantize.cuh"
 
 // Pipeline depths and stream-K occupancy (compile-time tuning constants).
@@ -37,6 +38,11 @@
 #ifndef PGF8_STREAMK16_STAGES
 #define PGF8_STREAMK16_STAGES 6
 #endif
+// Layers of a grouped call with at most this many tokens run in the grouped
+// weight-streaming kernel; larger ones take the per-layer kernels.
+#ifndef PGF8_GROUP_MAX_M
+#define PGF8_GROUP_MAX_M 128
+#endif
 #ifndef PGF8_STREAMK_CTAS_PER_SM
 #define PGF8_STREAMK_CTAS_PER_SM 1
 #endif
@@ -54,6 +60,45 @@ static pgf8_status cuda_fail(cudaError_t e)
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 static bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 static size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ------------------------------------------------------------------ per-device set-up
+// Kernel attributes (dynamic shared-memory limit, carveout), occupancy
+// answers and SM counts belong to one device: a process that drives several
+// GPUs sets and queries them once for each device, on the first launch with
+// that device current.  Ordinals past kSetupDevices are set up on every call.
+constexpr int kSetupDevices = 64;
+
+struct PerDeviceSetup {
+    std::mutex mu;
+    bool done[kSetupDevices] = {};
+    cudaError_t err[kSetupDevices] = {};
+    int value[kSetupDevices] = {};
+};
+
+// Runs `fn` (returning cudaError_t, writing an int) once per device and
+// returns its cached status; `*value` receives the cached int.
+template <class Fn> static cudaError_t setup_once_per_device(PerDeviceSetup &st, Fn fn, int *value = nullptr)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev < 0 || dev >= kSetupDevices) {
+        int v = 0;
+        e = fn(dev, &v);
+        if (value)
+            *value = v;
+        return e;
+    }
+    std::lock_guard<std::mutex> lock(st.mu);
+    if (!st.done[dev]) {
+        st.err[dev] = fn(dev, &st.value[dev]);
+        st.done[dev] = true;
+    }
+    if (value)
+        *value = st.value[dev];
+    return st.err[dev];
+}
 
 // ------------------------------------------------------------------ tensor maps
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -187,16 +232,17 @@ static void fill_attrs(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attrs, int 
 
 template <class C> static pgf8_status launch_cfg(const GemmLaunch &L, int splits)
 {
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    static PerDeviceSetup setup;
+    const cudaError_t attr_err = setup_once_per_device(setup, [](int, int *) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::kSmemBytes);
         // the largest shared-memory carveout: the default sizes the SM's
         // L1 / shared split for one CTA, which leaves the skinny kernels
         // (about 110 KB each) at one CTA per SM
-        if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(gemm_kernel<C>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                            cudaSharedmemCarveoutMaxShared);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gemm_kernel<C>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     cudaSharedmemCarveoutMaxShared);
+        return e;
     });
     if (attr_err != cudaSuccess)
         return cuda_fail(attr_err);
@@ -228,11 +274,9 @@ static int num_sms();
 // Persistent tiled kernel: one CTA per SM (at most one per tile).
 template <class C> static pgf8_status launch_persistent(const GemmLaunch &L)
 {
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(gemm_persistent_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        C::kSmemBytes);
+    static PerDeviceSetup setup;
+    const cudaError_t attr_err = setup_once_per_device(setup, [](int, int *) {
+        return cudaFuncSetAttribute(gemm_persistent_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     });
     if (attr_err != cudaSuccess)
         return cuda_fail(attr_err);
@@ -259,11 +303,9 @@ template <class C> static pgf8_status launch_persistent(const GemmLaunch &L)
 // Pair kernel: clusters of 2 CTAs, one 256 x 256 tile per pair at a time.
 template <class C> static pgf8_status launch_pair(const GemmLaunch &L)
 {
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(gemm_pair_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        C::kSmemBytes);
+    static PerDeviceSetup setup;
+    const cudaError_t attr_err = setup_once_per_device(setup, [](int, int *) {
+        return cudaFuncSetAttribute(gemm_pair_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     });
     if (attr_err != cudaSuccess)
         return cuda_fail(attr_err);
@@ -280,8 +322,9 @@ template <class C> static pgf8_status launch_pair(const GemmLaunch &L)
     cudaLaunchAttribute attrs[2];
     // A persistent grid must not hold more pairs than can run at once (a
     // pair needs two SMs of one GPC): ask the occupancy calculator.
-    static int pairs_fit = 0;
-    if (pairs_fit == 0) {
+    static PerDeviceSetup fit_setup;
+    int pairs_fit = 1;
+    const cudaError_t fit_err = setup_once_per_device(fit_setup, [&cfg](int, int *v) {
         cudaLaunchConfig_t q = cfg;
         q.gridDim = dim3(2 * num_sms(), 1, 1);
         cudaLaunchAttribute qa[1];
@@ -292,11 +335,12 @@ template <class C> static pgf8_status launch_pair(const GemmLaunch &L)
         q.attrs = qa;
         q.numAttrs = 1;
         int n = 0;
-        cudaError_t e = cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<C>, &q);
-        if (e != cudaSuccess)
-            return cuda_fail(e);
-        pairs_fit = n > 0 ? n : 1;
-    }
+        const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<C>, &q);
+        *v = n > 0 ? n : 1;
+        return e;
+    }, &pairs_fit);
+    if (fit_err != cudaSuccess)
+        return cuda_fail(fit_err);
     const int64_t pairs = tiles < pairs_fit ? tiles : pairs_fit;
     cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
     fill_attrs(cfg, attrs, 1, L.pdl, 2);
@@ -322,11 +366,9 @@ template <int KIND> static pgf8_status launch_pair_bn(const GemmLaunch &L, int b
 // Stream-K skinny kernel: one CTA per SM, equal shares of the weight stream.
 template <class C> static pgf8_status launch_streamk(const GemmLaunch &L)
 {
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(gemm_streamk_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        C::kSmemBytes);
+    static PerDeviceSetup setup;
+    const cudaError_t attr_err = setup_once_per_device(setup, [](int, int *) {
+        return cudaFuncSetAttribute(gemm_streamk_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     });
     if (attr_err != cudaSuccess)
         return cuda_fail(attr_err);
@@ -366,15 +408,15 @@ static pgf8_status launch_split_or_not(const GemmLaunch &L, int splits)
 
 static int num_sms()
 {
-    static int sms = 0;
-    if (sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (sms <= 0)
-            sms = 148;
-    }
-    return sms;
+    static PerDeviceSetup setup;
+    int sms = 0;
+    setup_once_per_device(setup, [](int dev, int *v) {
+        int n = 0;
+        const cudaError_t e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        *v = (e == cudaSuccess && n > 0) ? n : 148;
+        return cudaSuccess;
+    }, &sms);
+    return sms > 0 ? sms : 148;
 }
 
 // The largest power-of-two split that keeps a skinny grid within ~1.75 CTAs
@@ -1059,11 +1101,9 @@ pgf8_status pgf8_fp8_attention_context_paged(const uint8_t *q_codes, const float
         !aligned4(context_lens) || (errors && !aligned4(errors)) || (reinterpret_cast<uintptr_t>(out) & oa))
         return PGF8_ERR_ALIGNMENT;
 
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(attn_context_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        kCtxSmemBytes);
+    static PerDeviceSetup setup;
+    const cudaError_t attr_err = setup_once_per_device(setup, [](int, int *) {
+        return cudaFuncSetAttribute(attn_context_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kCtxSmemBytes);
     });
     if (attr_err != cudaSuccess)
         return cuda_fail(attr_err);
@@ -1336,6 +1376,218 @@ pgf8_status pgf8_fp8_linear_dynamic_many(const pgf8_fp8_layer *layers, int64_t c
                                              l.sw, l.N, l.y, l.workspace, l.workspace_bytes, &o, stream, kE4M3);
         if (st != PGF8_OK)
             return st;
+    }
+    return PGF8_OK;
+}
+
+} // extern "C"
+
+namespace pgf8 {
+
+static int group_bn(int64_t M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128; }
+
+static bool ranges_overlap(const void *a, size_t na, const void *b, size_t nb)
+{
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return na > 0 && nb > 0 && a0 < b0 + nb && b0 < a0 + na;
+}
+
+// Bytes of a layer's activations [M, K] at row stride ldx.
+static size_t x_span(const pgf8_fp8_layer &l)
+{
+    const size_t eb = l.xdt == PGF8_F32 ? 4 : 2;
+    return (static_cast<size_t>(l.M - 1) * static_cast<size_t>(l.ldx) + static_cast<size_t>(l.K)) * eb;
+}
+
+template <class C> static pgf8_status launch_group_cfg(const GroupParams &p, int grid, cudaStream_t st)
+{
+    static PerDeviceSetup setup;
+    const cudaError_t attr_err = setup_once_per_device(setup, [](int, int *) {
+        return cudaFuncSetAttribute(gemm_group_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    });
+    if (attr_err != cudaSuccess)
+        return cuda_fail(attr_err);
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(C::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attrs[1];
+    attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attrs;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_group_kernel<C>, p);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    return PGF8_OK;
+}
+
+// One grouped launch pair for up to kGroupMaxLayers small-M layers: the
+// per-token quantisation of all of them, then the grouped GEMM, which
+// streams its first ring of weights while the quantisation runs.
+static pgf8_status group_chunk(const pgf8_fp8_layer *const *ls, int n, void *group_ws, int first_pdl,
+                               cudaStream_t cs)
+{
+    QuantGroupParams qp;
+    std::memset(&qp, 0, sizeof(qp));
+    GroupParams gp;   // about 10 KB: passed by value as the kernel's parameter block
+    std::memset(&gp, 0, sizeof(gp));
+    int64_t rows = 0, units = 0;
+    int bnmax = 16;
+    for (int i = 0; i < n; ++i) {
+        const pgf8_fp8_layer &l = *ls[i];
+        uint8_t *aq = static_cast<uint8_t *>(l.workspace) + pgf8_fp8_linear_dynamic_codes_offset(l.M, l.K);
+        float *sa = reinterpret_cast<float *>(static_cast<uint8_t *>(l.workspace) +
+                                              pgf8_fp8_linear_dynamic_scales_offset(l.M, l.K));
+        QuantGroupLayer &q = qp.L[i];
+        q.x = l.x;
+        q.ldx = l.ldx;
+        q.cols = l.K;
+        q.row0 = rows;
+        q.rows = l.M;
+        q.q = aq;
+        q.scales = sa;
+        q.xdt = l.xdt == PGF8_F32 ? 0 : 1;
+        rows += l.M;
+
+        const int bn = group_bn(l.M);
+        bnmax = bn > bnmax ? bn : bnmax;
+        GroupLayer &g = gp.L[i];
+        g.unit0 = units;
+        g.M = static_cast<int>(l.M);
+        g.N = static_cast<int>(l.N);
+        g.K = static_cast<int>(l.K);
+        g.kblocks = static_cast<int>((l.K + 127) / 128);
+        g.bn = bn;
+        g.sa = sa;
+        g.sw = l.sw;
+        g.y = l.y;
+        units += static_cast<int64_t>((l.N + 127) / 128) * g.kblocks;
+        if (!make_map(&gp.tmW[i], l.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(l.N),
+                      static_cast<uint64_t>(l.K), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&gp.tmX[i], aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(l.M),
+                      static_cast<uint64_t>(l.K), 128, static_cast<uint32_t>(bn), CU_TENSOR_MAP_SWIZZLE_128B))
+            return PGF8_ERR_UNSUPPORTED;
+    }
+    qp.nlayers = n;
+    gp.nlayers = n;
+    gp.prefetch_w = 1;   // the quantisation kernel writes only codes and scales
+    gp.units = units;
+    gp.flags = static_cast<unsigned *>(group_ws);
+    gp.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(group_ws) + kGroupFlagBytes);
+
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(rows));
+    cfg.blockDim = dim3(kQuantThreads);
+    cfg.stream = cs;
+    cudaLaunchAttribute attr[1];
+    if (first_pdl) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    cudaError_t e = cudaLaunchKernelEx(&cfg, quantize_group_kernel, qp);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+
+    int grid = num_sms();
+    if (grid > kGroupMaxCtas)
+        grid = kGroupMaxCtas;
+    if (static_cast<int64_t>(grid) > units)
+        grid = static_cast<int>(units);
+    switch (bnmax) {
+    case 16:
+        return launch_group_cfg<GroupCfg<16, 12>>(gp, grid, cs);
+    case 32:
+        return launch_group_cfg<GroupCfg<32, 11>>(gp, grid, cs);
+    case 64:
+        return launch_group_cfg<GroupCfg<64, 9>>(gp, grid, cs);
+    default:
+        return launch_group_cfg<GroupCfg<128, 6>>(gp, grid, cs);
+    }
+}
+
+} // namespace pgf8
+
+extern "C" {
+
+size_t pgf8_fp8_linear_group_workspace_size(int64_t max_m)
+{
+    if (max_m < 1)
+        return kGroupFlagBytes;
+    return group_workspace_bytes(group_bn(max_m < PGF8_GROUP_MAX_M ? max_m : PGF8_GROUP_MAX_M));
+}
+
+pgf8_status pgf8_fp8_linear_dynamic_group(const pgf8_fp8_layer *layers, int64_t count, void *group_workspace,
+                                          size_t group_workspace_bytes, const pgf8_linear_opts *opts, void *stream)
+{
+    if (count < 0 || (count > 0 && !layers))
+        return PGF8_ERR_INVALID_ARG;
+    int64_t max_small = 0;
+    for (int64_t i = 0; i < count; ++i) {
+        const pgf8_fp8_layer &l = layers[i];
+        pgf8_status st = check_linear_dynamic(l.x, static_cast<pgf8_dtype>(l.xdt), l.M, l.K, l.ldx, l.wq, l.sw, l.N,
+                                              l.y, l.workspace, l.workspace_bytes, kE4M3);
+        if (st != PGF8_OK)
+            return st;
+        if (l.M <= PGF8_GROUP_MAX_M && l.M > max_small)
+            max_small = l.M;
+    }
+    // independent layers only: no layer writes (y, workspace) what another
+    // layer reads or writes
+    for (int64_t i = 0; i < count; ++i) {
+        const pgf8_fp8_layer &a = layers[i];
+        const size_t ya = static_cast<size_t>(a.M) * static_cast<size_t>(a.N) * 2;
+        for (int64_t j = 0; j < count; ++j) {
+            const pgf8_fp8_layer &b = layers[j];
+            if (ranges_overlap(a.y, ya, b.x, x_span(b)) ||
+                ranges_overlap(a.workspace, a.workspace_bytes, b.x, x_span(b)))
+                return PGF8_ERR_INVALID_ARG;
+            if (i != j && (ranges_overlap(a.y, ya, b.y, static_cast<size_t>(b.M) * static_cast<size_t>(b.N) * 2) ||
+                           ranges_overlap(a.workspace, a.workspace_bytes, b.workspace, b.workspace_bytes) ||
+                           ranges_overlap(a.y, ya, b.workspace, b.workspace_bytes)))
+                return PGF8_ERR_INVALID_ARG;
+        }
+    }
+    if (max_small > 0) {
+        if (!group_workspace || group_workspace_bytes < pgf8_fp8_linear_group_workspace_size(max_small))
+            return PGF8_ERR_INVALID_ARG;
+        if (!aligned16(group_workspace))
+            return PGF8_ERR_ALIGNMENT;
+    }
+    pgf8_linear_opts o = opts_or_default(opts);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    int pdl = (o.flags & PGF8_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
+    // small layers: grouped, kGroupMaxLayers per launch pair, in call order
+    const pgf8_fp8_layer *chunk[kGroupMaxLayers];
+    int n = 0;
+    for (int64_t i = 0; i <= count; ++i) {
+        if (i < count && layers[i].M <= PGF8_GROUP_MAX_M)
+            chunk[n++] = &layers[i];
+        if (n == kGroupMaxLayers || (i == count && n > 0)) {
+            pgf8_status st = group_chunk(chunk, n, group_workspace, pdl, cs);
+            if (st != PGF8_OK)
+                return st;
+            n = 0;
+            pdl = 1;
+        }
+    }
+    // large layers: one dynamic call each, overlapping the previous one
+    for (int64_t i = 0; i < count; ++i) {
+        const pgf8_fp8_layer &l = layers[i];
+        if (l.M <= PGF8_GROUP_MAX_M)
+            continue;
+        if (pdl)
+            o.flags |= PGF8_FLAG_OVERLAP_PREVIOUS;
+        pgf8_status st = linear_dynamic_impl(l.x, static_cast<pgf8_dtype>(l.xdt), l.M, l.K, l.ldx, l.wq, nullptr,
+                                             l.sw, l.N, l.y, l.workspace, l.workspace_bytes, &o, stream, kE4M3);
+        if (st != PGF8_OK)
+            return st;
+        pdl = 1;
     }
     return PGF8_OK;
 }

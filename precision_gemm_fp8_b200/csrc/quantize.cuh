@@ -205,28 +205,14 @@ __global__ void __launch_bounds__(256) selftest_row_division_kernel(const float 
 // longer rows are re-read (from L2) for the conversion.
 constexpr int kRegChunks = 4;
 
-// One CTA per row.  cols % 16 == 0; x rows 16-byte aligned.
-// trigger_early: let a dependent kernel launched with programmatic stream
-// serialization be scheduled at once (used only when that dependent is the
-// library's own GEMM, which reads q/scales after this grid completes).
+// One row quantised by one CTA of kQuantThreads threads (every thread of
+// the CTA calls it).  cols % 16 == 0; the row 16-byte aligned.  mode 0:
+// dynamic (*srow = fl32(amax / 448), 1 for an all-zero row); mode 1: the
+// scale is read from *srow.
 template <typename T>
-__global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(const T *__restrict__ x, int64_t rows,
-                                                                      int64_t cols, int64_t ldx,
-                                                                      uint8_t *__restrict__ q,
-                                                                      float *__restrict__ scales, int mode,
-                                                                      int trigger_early)
+__device__ __forceinline__ void quantize_one_row(const T *__restrict__ xr, int64_t cols, uint8_t *__restrict__ qr,
+                                                 float *srow, int mode, float *red)
 {
-    __shared__ float red[kQuantThreads / 32];
-    if (trigger_early)
-        grid_launch_dependents();
-    // When launched with programmatic serialization, the previous kernel in
-    // the stream may still run: nothing is read or written before it ends.
-    grid_dependency_wait();
-    const int64_t row = blockIdx.x;
-    if (row >= rows)
-        return;
-    const T *xr = x + row * ldx;
-    uint8_t *qr = q + row * cols;
     const int64_t nchunk = cols / 16;
 
     if (nchunk <= static_cast<int64_t>(kRegChunks) * kQuantThreads) {
@@ -249,9 +235,9 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(const T *_
             if (s == 0.0f)
                 s = 1.0f;
             if (threadIdx.x == 0)
-                scales[row] = s;
+                *srow = s;
         } else {
-            s = scales[row];
+            s = *srow;
         }
         const RowDivisor d(s);
 #pragma unroll
@@ -278,9 +264,9 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(const T *_
         if (s == 0.0f)
             s = 1.0f;
         if (threadIdx.x == 0)
-            scales[row] = s;
+            *srow = s;
     } else {
-        s = scales[row];
+        s = *srow;
     }
     const RowDivisor d(s);
     for (int64_t c = threadIdx.x; c < nchunk; c += kQuantThreads) {
@@ -288,6 +274,69 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(const T *_
         v.load(xr + c * 16);
         *reinterpret_cast<uint4 *>(qr + c * 16) = encode16(v.v, d);
     }
+}
+
+// One CTA per row.  cols % 16 == 0; x rows 16-byte aligned.
+// trigger_early: let a dependent kernel launched with programmatic stream
+// serialization be scheduled at once (used only when that dependent is the
+// library's own GEMM, which reads q/scales after this grid completes).
+template <typename T>
+__global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(const T *__restrict__ x, int64_t rows,
+                                                                      int64_t cols, int64_t ldx,
+                                                                      uint8_t *__restrict__ q,
+                                                                      float *__restrict__ scales, int mode,
+                                                                      int trigger_early)
+{
+    __shared__ float red[kQuantThreads / 32];
+    if (trigger_early)
+        grid_launch_dependents();
+    // When launched with programmatic serialization, the previous kernel in
+    // the stream may still run: nothing is read or written before it ends.
+    grid_dependency_wait();
+    const int64_t row = blockIdx.x;
+    if (row >= rows)
+        return;
+    quantize_one_row<T>(x + row * ldx, cols, q + row * cols, scales + row, mode, red);
+}
+
+// Dynamic per-token quantisation of the activations of several independent
+// layers in one launch: one CTA per row over all the layers' rows (layer l
+// owns rows [row0, row0 + rows) of the grid), each row exactly as
+// quantize_rows_kernel computes it.
+constexpr int kQuantGroupMaxLayers = 64;
+
+struct QuantGroupLayer {
+    const void *x;       // [rows, cols] f32 or f16, row stride ldx elements
+    int64_t ldx, cols, row0, rows;
+    uint8_t *q;          // [rows, cols] codes
+    float *scales;       // [rows]
+    int xdt;             // 0 f32, 1 f16
+};
+
+struct QuantGroupParams {
+    QuantGroupLayer L[kQuantGroupMaxLayers];
+    int nlayers;
+};
+
+__global__ void __launch_bounds__(kQuantThreads) quantize_group_kernel(const __grid_constant__ QuantGroupParams p)
+{
+    __shared__ float red[kQuantThreads / 32];
+    grid_launch_dependents();   // the dependent is the library's grouped GEMM
+    grid_dependency_wait();
+    const int64_t row = blockIdx.x;
+    int l = 0;
+    while (l + 1 < p.nlayers && p.L[l + 1].row0 <= row)
+        ++l;
+    const QuantGroupLayer &g = p.L[l];
+    const int64_t r = row - g.row0;
+    if (r < 0 || r >= g.rows)
+        return;
+    if (g.xdt == 0)
+        quantize_one_row<float>(static_cast<const float *>(g.x) + r * g.ldx, g.cols, g.q + r * g.cols,
+                                g.scales + r, 0, red);
+    else
+        quantize_one_row<__half>(static_cast<const __half *>(g.x) + r * g.ldx, g.cols, g.q + r * g.cols,
+                                 g.scales + r, 0, red);
 }
 
 // ------------------------------------------------------------------ per-tensor scaling

@@ -148,6 +148,37 @@ def test_dynamic_many_checks_every_layer_first():
     assert pg.lib.pgf8_fp8_linear_dynamic_many(arr, -1, None, None) == pg.ERR_INVALID_ARG
 
 
+def test_dynamic_group_checks_layers_aliasing_and_workspace_first():
+    """pgf8_fp8_linear_dynamic_group: every layer checked, independence (no
+    output or workspace overlapping another layer's buffers) and the group
+    workspace checked, all before anything is enqueued."""
+    f = pg.lib.pgf8_fp8_linear_dynamic_group
+    ws_need = pg.lib.pgf8_fp8_linear_group_workspace_size(4)
+    assert ws_need == pg.lib.pgf8_fp8_linear_group_workspace_size(16) > 1024
+    assert pg.lib.pgf8_fp8_linear_group_workspace_size(128) == pg.lib.pgf8_fp8_linear_group_workspace_size(4096)
+    assert pg.lib.pgf8_fp8_linear_group_workspace_size(0) == 1024
+    base = 1 << 32
+    x0, x1, y0, y1, w0, w1 = (base + i * (1 << 26) for i in range(6))
+    wsp0, wsp1, gws = base + 6 * (1 << 26), base + 7 * (1 << 26), base + 8 * (1 << 26)
+    l0 = pg.Fp8Layer(x0, pg.F32, 0, 4, 512, 512, 512, base + 9 * (1 << 26), C16, y0, wsp0, 1 << 24)
+    l1 = pg.Fp8Layer(x1, pg.F32, 0, 4, 512, 512, 512, base + 10 * (1 << 26), C16, y1, wsp1, 1 << 24)
+    bad = pg.Fp8Layer(x1, pg.F32, 0, 4, 520, 520, 512, base + 10 * (1 << 26), C16, y1, wsp1, 1 << 24)   # K % 16
+    arr = (pg.Fp8Layer * 2)(l0, bad)
+    assert f(arr, 2, gws, ws_need, None, None) == pg.ERR_ALIGNMENT
+    # layer 1 reads layer 0's output: not independent
+    dep = pg.Fp8Layer(y0, pg.F32, 0, 4, 512, 512, 512, base + 10 * (1 << 26), C16, y1, wsp1, 1 << 24)
+    assert f((pg.Fp8Layer * 2)(l0, dep), 2, gws, ws_need, None, None) == pg.ERR_INVALID_ARG
+    # two layers sharing one workspace
+    share = pg.Fp8Layer(x1, pg.F32, 0, 4, 512, 512, 512, base + 10 * (1 << 26), C16, y1, wsp0, 1 << 24)
+    assert f((pg.Fp8Layer * 2)(l0, share), 2, gws, ws_need, None, None) == pg.ERR_INVALID_ARG
+    ok2 = (pg.Fp8Layer * 2)(l0, l1)
+    assert f(ok2, 2, None, 0, None, None) == pg.ERR_INVALID_ARG            # group workspace missing
+    assert f(ok2, 2, gws, ws_need - 16, None, None) == pg.ERR_INVALID_ARG  # too small
+    assert f(ok2, 2, gws + 8, ws_need, None, None) == pg.ERR_ALIGNMENT
+    assert f(None, 2, gws, ws_need, None, None) == pg.ERR_INVALID_ARG
+    assert f(None, 0, None, 0, None, None) == pg.OK
+
+
 def test_selftest_row_division_argument_checks():
     f = pg.lib.pgf8_selftest_row_division
     buf = (ctypes.c_uint64 * 4)()

@@ -1,0 +1,122 @@
+"""GPU parity of the grouped dynamic FP8 linear (pgf8_fp8_linear_dynamic_group):
+every layer's codes and scales bit-exact against the oracle, every output
+within the layer's stated bound |y - ref| <= 2^-8 |ref| + 1e-4 sqrt(K) A_m W_n
+against the oracle's binary64 layer.  The cases cover every token-tile class
+of the grouped kernel (M <= 16, 32, 64, 128) in one group, layers past it
+(M > 128, per-layer kernels), ragged N and K, groups small enough that one
+weight tile is shared by several CTAs and large enough that a CTA walks
+many tiles and crosses layer boundaries, and repeated calls (the flag words
+must be left zero, and the results must repeat bit for bit)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from _parity import assert_within, fp8_row_max, linear_bound
+
+pg = pytest.importorskip("precision_gemm_fp8_b200")
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _make_group(shapes, seed, recipe="student_t3"):
+    g = np.random.default_rng(seed)
+    layers, host = [], []
+    for (M, K, N) in shapes:
+        x = synthetic.activations(recipe, M, K, g)
+        w = synthetic.weights_f16(N, K, 0.02, g)
+        wq, sw = pg.fp8_quantize_rows(torch.from_numpy(w).to(DEV))
+        xt = torch.from_numpy(x).to(DEV)
+        y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+        ws = torch.zeros(pg.fp8_linear_dynamic_workspace_size(M, N, K), dtype=torch.uint8, device=DEV)
+        layers.append((xt, wq, sw, y, ws))
+        host.append((x, w))
+    return layers, host
+
+
+def _check_layer(i, layer, x, w, ns=None):
+    xt, wq_d, sw_d, y, ws = layer
+    M, K = x.shape
+    aq0, sa0 = oracle.quantize_rows(x)
+    aq, sa = pg.dynamic_workspace_views(ws, M, K)
+    assert np.array_equal(aq.cpu().numpy(), aq0), f"layer {i}: codes differ from the oracle"
+    assert np.array_equal(sa.cpu().numpy().view(np.uint32), sa0.view(np.uint32)), f"layer {i}: scales"
+    wsub = w if ns is None else w[ns]
+    wq0, sw0 = oracle.quantize_rows(wsub)
+    ref = oracle.fp8_linear(aq0, sa0, wq0, sw0)
+    bound = linear_bound(ref, K, fp8_row_max(aq0, sa0), fp8_row_max(wq0, sw0))
+    got = y.float().cpu().numpy()
+    if ns is not None:
+        got = got[:, ns]
+    assert_within(got, ref, bound, f"group layer {i} (M={M} K={K} N={w.shape[0]})")
+
+
+MIXED = [  # (M, K, N): all token classes, ragged N and K, one layer past the grouped kernel
+    (1, 512, 528), (4, 272, 400), (8, 1040, 144), (16, 528, 1040), (17, 400, 272), (32, 1008, 656),
+    (33, 144, 912), (64, 656, 528), (65, 272, 1296), (100, 528, 400), (128, 1024, 1024), (160, 400, 528),
+]
+
+
+def test_group_mixed_token_classes():
+    layers, host = _make_group(MIXED, 11)
+    grp = pg.LayerGroup(layers)
+    grp.run()
+    torch.cuda.synchronize()
+    assert pg.device_status() == pg.OK
+    first = [l[3].clone() for l in layers]
+    for i, (layer, (x, w)) in enumerate(zip(layers, host)):
+        _check_layer(i, layer, x, w)
+    # the flags left by the first call are zero: the second call repeats it bit for bit
+    for l in layers:
+        l[3].fill_(float("nan"))
+    grp.run()
+    torch.cuda.synchronize()
+    assert pg.device_status() == pg.OK
+    for i, (l, f) in enumerate(zip(layers, first)):
+        assert torch.equal(l[3].view(torch.int16), f.view(torch.int16)), f"layer {i} differs on the second call"
+    assert not grp.group_workspace[:1024].any(), "flag words not cleared"
+
+
+@pytest.mark.parametrize("shapes", [
+    [(8, 4096, 512)],                       # 4 tiles x 32 k-blocks: tiles shared by many CTAs
+    [(1, 16, 16), (2, 32, 16)],             # fewer units than SMs: one unit per CTA
+    [(8, 11008, 256), (3, 128, 2048)],      # long K; short layer after it
+])
+def test_group_shared_tiles(shapes):
+    layers, host = _make_group(shapes, 5 + len(shapes), recipe="normal_outl_0p5pct_x30")
+    grp = pg.LayerGroup(layers)
+    for _ in range(3):
+        grp.run()
+    torch.cuda.synchronize()
+    assert pg.device_status() == pg.OK
+    for i, (layer, (x, w)) in enumerate(zip(layers, host)):
+        _check_layer(i, layer, x, w)
+    assert not grp.group_workspace[:1024].any()
+
+
+@pytest.mark.slow
+def test_group_decode7b_full_size_sampled():
+    """The decode7b step as one group (12 layers, 606 MB of weights at full
+    size), checked on 384 sampled output channels of every layer."""
+    wl = synthetic.WORKLOADS["decode7b"]
+    layers, host = [], []
+    for mi, M in enumerate(wl.ms):
+        for si, (K, N, _) in enumerate(wl.shapes):
+            x = synthetic.acts("decode7b", si, mi)
+            w = synthetic.weights("decode7b", si, copy=mi)
+            wq, sw = pg.fp8_quantize_rows(torch.from_numpy(w).to(DEV))
+            y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+            ws = torch.zeros(pg.fp8_linear_dynamic_workspace_size(M, N, K), dtype=torch.uint8, device=DEV)
+            layers.append((torch.from_numpy(x).to(DEV), wq, sw, y, ws))
+            host.append((x, w))
+    grp = pg.LayerGroup(layers)
+    grp.run()
+    grp.run()
+    torch.cuda.synchronize()
+    assert pg.device_status() == pg.OK
+    rng = np.random.default_rng(3)
+    for i, (layer, (x, w)) in enumerate(zip(layers, host)):
+        ns = np.sort(rng.choice(w.shape[0], 384, replace=False))
+        _check_layer(i, layer, x, w, ns)
