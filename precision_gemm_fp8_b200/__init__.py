@@ -170,6 +170,18 @@ def default_workspace(device, nbytes: int) -> torch.Tensor | None:
     return t
 
 
+def _lead(t: torch.Tensor) -> int:
+    """Element stride between consecutive entries of the leading dimension.
+    A size-1 leading dimension may carry any stride (torch keeps numpy's 0),
+    so there the rows are taken as packed: the product of the other sizes."""
+    if t.shape[0] > 1:
+        return t.stride(0)
+    n = 1
+    for d in t.shape[1:]:
+        n *= d
+    return max(t.stride(0), n)
+
+
 def _nbytes(t):
     return 0 if t is None else t.numel() * t.element_size()
 
@@ -197,7 +209,7 @@ def fp8_quantize_rows(x: torch.Tensor, q: torch.Tensor | None = None, scales: to
         if mode == SCALE_STATIC:
             raise ValueError("static mode needs scales")
         scales = torch.empty(rows, dtype=torch.float32, device=x.device)
-    _check(lib.pgf8_fp8_quantize_rows(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(q), _ptr(scales),
+    _check(lib.pgf8_fp8_quantize_rows(_ptr(x), _dtype_code(x), rows, cols, _lead(x), _ptr(q), _ptr(scales),
                                       mode, _stream(stream)), "fp8_quantize_rows")
     return q, scales
 
@@ -218,7 +230,7 @@ def fp8_kv_write_paged(kv: torch.Tensor, scales: torch.Tensor, cache: torch.Tens
         raise ValueError("cache must be a contiguous uint8 [num_blocks, heads, block_size, head_dim] tensor")
     if block_table.dtype != torch.int32 or not block_table.is_contiguous():
         raise ValueError("block_table must be a contiguous int32 tensor")
-    _check(lib.pgf8_fp8_kv_write_paged(_ptr(kv), code, tokens, heads, head_dim, kv.stride(0), _ptr(scales), first_pos,
+    _check(lib.pgf8_fp8_kv_write_paged(_ptr(kv), code, tokens, heads, head_dim, _lead(kv), _ptr(scales), first_pos,
                                        block_size, _ptr(block_table), block_table.numel(), num_blocks, _ptr(cache),
                                        None if bad_blocks is None else _ptr(bad_blocks), flags, _stream(stream)),
            "fp8_kv_write_paged")
@@ -276,8 +288,8 @@ def fp8_attention_decode_paged(q: torch.Tensor, k_cache: torch.Tensor, v_cache: 
     cache = PagedKVCache(_ptr(k_cache), _ptr(v_cache), _ptr(k_scales), _ptr(v_scales), num_blocks, kv_heads,
                          block_size, head_dim)
     _check(lib.pgf8_fp8_attention_decode_paged(
-        _ptr(q), codes[q.dtype], seqs, q_heads, q.stride(0), ctypes.byref(cache), _ptr(block_tables),
-        block_tables.stride(0), _ptr(context_lens), max_context, _ptr(out), codes[out.dtype], out.stride(0), splits,
+        _ptr(q), codes[q.dtype], seqs, q_heads, _lead(q), ctypes.byref(cache), _ptr(block_tables),
+        _lead(block_tables), _ptr(context_lens), max_context, _ptr(out), codes[out.dtype], _lead(out), splits,
         _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
         None if errors is None else _ptr(errors), flags, _stream(stream)), "fp8_attention_decode_paged")
     return out
@@ -327,8 +339,8 @@ def fp8_attention_context_paged(q_codes: torch.Tensor, q_scales: torch.Tensor, q
                          block_size, head_dim)
     _check(lib.pgf8_fp8_attention_context_paged(
         _ptr(q_codes), _ptr(q_scales), _ptr(q_start), seqs, total_q, max_q_len, q_heads, ctypes.byref(cache),
-        _ptr(block_tables), block_tables.stride(0), _ptr(context_lens), max_context, _ptr(out), codes[out.dtype],
-        out.stride(0), None if errors is None else _ptr(errors), _stream(stream)), "fp8_attention_context_paged")
+        _ptr(block_tables), _lead(block_tables), _ptr(context_lens), max_context, _ptr(out), codes[out.dtype],
+        _lead(out), None if errors is None else _ptr(errors), _stream(stream)), "fp8_attention_context_paged")
     return out
 
 
@@ -344,7 +356,7 @@ def fp8_norm_quantize(x: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor |
         q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
     if scales is None:
         scales = torch.empty(rows, dtype=torch.float32, device=x.device)
-    _check(lib.pgf8_fp8_norm_quantize(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(gamma),
+    _check(lib.pgf8_fp8_norm_quantize(_ptr(x), _dtype_code(x), rows, cols, _lead(x), _ptr(gamma),
                                       None if beta is None else _ptr(beta), float(eps), _ptr(q), _ptr(scales), flags,
                                       _stream(stream)), "fp8_norm_quantize")
     return q, scales
@@ -366,7 +378,7 @@ def fp8_silu_mul_quantize(gu: torch.Tensor, q: torch.Tensor | None = None, scale
         q = torch.empty((rows, inter), dtype=torch.uint8, device=gu.device)
     if scales is None:
         scales = torch.empty(rows, dtype=torch.float32, device=gu.device)
-    _check(lib.pgf8_fp8_silu_mul_quantize(_ptr(gu), code, rows, inter, gu.stride(0), _ptr(q), _ptr(scales), flags,
+    _check(lib.pgf8_fp8_silu_mul_quantize(_ptr(gu), code, rows, inter, _lead(gu), _ptr(q), _ptr(scales), flags,
                                           _stream(stream)), "fp8_silu_mul_quantize")
     return q, scales
 
@@ -380,7 +392,7 @@ def fp8_amax_accumulate(x: torch.Tensor, amax: torch.Tensor | None = None, strea
         raise ValueError("x rows must be contiguous")
     if amax is None:
         amax = torch.zeros(1, dtype=torch.float32, device=x.device)
-    _check(lib.pgf8_fp8_amax_accumulate(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(amax),
+    _check(lib.pgf8_fp8_amax_accumulate(_ptr(x), _dtype_code(x), rows, cols, _lead(x), _ptr(amax),
                                         _stream(stream)), "fp8_amax_accumulate")
     return amax
 
@@ -397,7 +409,7 @@ def fp8_quantize_tensor(x: torch.Tensor, amax: torch.Tensor, q: torch.Tensor | N
         q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
     if scales is None:
         scales = torch.empty(rows, dtype=torch.float32, device=x.device)
-    _check(lib.pgf8_fp8_quantize_tensor(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(amax), _ptr(q),
+    _check(lib.pgf8_fp8_quantize_tensor(_ptr(x), _dtype_code(x), rows, cols, _lead(x), _ptr(amax), _ptr(q),
                                         _ptr(scales), flags, _stream(stream)), "fp8_quantize_tensor")
     return q, scales
 
@@ -428,7 +440,7 @@ class DelayedScaling:
             q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
         if scales is None:
             scales = torch.empty(rows, dtype=torch.float32, device=x.device)
-        _check(lib.pgf8_fp8_quantize_delayed(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(q),
+        _check(lib.pgf8_fp8_quantize_delayed(_ptr(x), _dtype_code(x), rows, cols, _lead(x), _ptr(q),
                                              _ptr(scales), _ptr(self.history), self.history_len, _ptr(self.state),
                                              self.steps, flags, _stream(stream)), "fp8_quantize_delayed")
         self.steps += 1
@@ -481,7 +493,7 @@ def fp8_linear_dynamic(x, wq, sw, y=None, workspace=None, path=PATH_AUTO, split_
     need = fp8_linear_dynamic_workspace_size(M, N, K)
     if workspace is None:
         workspace = default_workspace(x.device, need)
-    _check(lib.pgf8_fp8_linear_dynamic(_ptr(x), _dtype_code(x), M, K, x.stride(0), _ptr(wq), _ptr(sw), N, _ptr(y),
+    _check(lib.pgf8_fp8_linear_dynamic(_ptr(x), _dtype_code(x), M, K, _lead(x), _ptr(wq), _ptr(sw), N, _ptr(y),
                                        _ptr(workspace), workspace.numel() * workspace.element_size(),
                                        _opts(path, split_k, tile_n, flags), _stream(stream)), "fp8_linear_dynamic")
     return y
@@ -514,7 +526,7 @@ def fp8_linear_dynamic_noalloc(x, wq, sw, y=None, stream=None):
         raise ValueError("x rows must be contiguous")
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    _check(lib.pgf8_fp8_linear_dynamic_noalloc(_ptr(x), _dtype_code(x), M, K, x.stride(0), _ptr(wq), _ptr(sw), N,
+    _check(lib.pgf8_fp8_linear_dynamic_noalloc(_ptr(x), _dtype_code(x), M, K, _lead(x), _ptr(wq), _ptr(sw), N,
                                                _ptr(y), _stream(stream)), "fp8_linear_dynamic_noalloc")
     return y
 
@@ -530,7 +542,7 @@ class LayerSequence:
         for i, (x, wq, sw, y, ws) in enumerate(self._keep):
             if x.stride(1) != 1:
                 raise ValueError("x rows must be contiguous")
-            arr[i] = Fp8Layer(x.data_ptr(), _dtype_code(x), 0, x.shape[0], x.shape[1], x.stride(0), wq.shape[0],
+            arr[i] = Fp8Layer(x.data_ptr(), _dtype_code(x), 0, x.shape[0], x.shape[1], _lead(x), wq.shape[0],
                               wq.data_ptr(), sw.data_ptr(), y.data_ptr(), ws.data_ptr(), _nbytes(ws))
         self._arr = arr
         self.count = len(self._keep)

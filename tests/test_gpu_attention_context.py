@@ -1,8 +1,4 @@
-"""Not collected yet (the file name does not start with test_): the context attention kernel
-has not yet run on a B200.  Once it has passed there, this file becomes
-tests/test_gpu_attention_context.py.
-
-GPU parity of the FP8 context attention over the paged cache ("C++ and
+"""GPU parity of the FP8 context attention over the paged cache ("C++ and
 FP8" §3.2-3.3) against the oracle.
 
 The query is quantised by the row quantiser (bit-exact with the oracle's);

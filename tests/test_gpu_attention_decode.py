@@ -1,8 +1,4 @@
-"""Not collected yet (the file name does not start with test_): the decode attention kernel
-has not yet run on a B200.  Once it has passed there, this file becomes
-tests/test_gpu_attention_decode.py.
-
-GPU parity of the FP8 paged decode attention against the oracle ("7B on
+"""GPU parity of the FP8 paged decode attention against the oracle ("7B on
 an RTX 4060 with FP8": K/V held in FP8; "C++ and FP8" §3.2 paged cache of
 16-token blocks, §3.3 attention in the FP8 dataflow).
 
