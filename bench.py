@@ -1,26 +1,30 @@
 """Benchmark of the FP8 linear layer hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode7b|prefill7b|nested7b|llama70b|small]
+                    [--workload llama70b|decode7b|prefill7b|nested7b|small] [--per-layer]
 
 A step is one pass of the hot path over one batch of synthetic inputs: for
 every (M, shape) layer of the workload, dynamic per-token E4M3 quantisation
 of the activations followed by the FP8 GEMM with fused dequantisation
 (weights were quantised per output channel once, at set-up, with the same
-kernel).  The default workload is the Llama-7B decode linears (QKV
-4096->12288, O 4096->4096, gate+up 4096->22016, down 11008->4096 at
-M = 1, 4, 8); every layer reads its own weight copy, so one step streams
-606 MB of FP8 weights, more than the 126 MB L2, and no weight is L2-resident
-when it is read.
+kernel).  The default workload is the Llama-70B linears (QKV 8192->10240,
+O 8192->8192, gate+up 8192->57344, down 28672->8192) at M = 1, 2, 4, ...,
+4096 tokens: 52 independent layers, 11.1 GB of FP8 weights streamed per step
+(the same weights for every M, 855 MB per M: more than the 126 MB L2, so no
+weight is L2-resident when it is re-read).  One step is one
+pgf8_fp8_linear_dynamic_group call: the M <= 128 layers stream their weights
+through one grouped kernel, the larger ones run the tiled tensor-core GEMMs.
+decode7b, prefill7b and nested7b are timed as secondary steps in the same run.
 
 Timing: the K timed steps are replayed from a CUDA graph (captured from the
 library's own C-ABI calls) between a barrier + synchronize on both sides,
-CUDA events on the launching stream, max over ranks.  Per-GEMM durations
-for the roofline come from event pairs captured around every GEMM launch of
-the last replayed steps.  `e2e` repeats the metric through the public entry
-point (fp8_linear_dynamic) with the activations copied from pinned host
-memory and the outputs copied back inside the timed region.  `cpu_baseline`
-times the CPU oracle on a bounded sample of the same workload.
+CUDA events on the launching stream, max over ranks.  The per-kernel shares
+for the roofline come from a step run with an event between consecutive
+launch groups, scaled to the timed step.  `e2e` repeats the metric through
+the public entry point with the activations copied from pinned host memory
+and the outputs copied back inside the timed region.  `cpu_baseline` times
+the CPU oracle on a bounded sample of the same workload, one thread and all
+host threads.
 
 Prints one JSON line (rank 0).
 """
@@ -178,8 +182,8 @@ class ClockSampler:
 # The GEMM kernels' sources (and the helpers they include): what a DRAM
 # traffic record describes.  The record also names the kernel configuration
 # it was taken on.
-GEMM_SOURCES = ("gemm.cuh", "gemm_2sm.cuh", "gemm_persistent.cuh", "gemm_streamk.cuh", "quantize.cuh",
-                "sm100_ptx.cuh")
+GEMM_SOURCES = ("gemm.cuh", "gemm_2sm.cuh", "gemm_persistent.cuh", "gemm_streamk.cuh", "gemm_group.cuh",
+                "quantize.cuh", "sm100_ptx.cuh")
 
 
 def kernel_sources_hash() -> str:
@@ -235,29 +239,59 @@ def job_throughput(units_per_rank: float, world: int, max_seconds: float) -> flo
 
 
 # ----------------------------------------------------------------------------- our arm
-def run_ours(args, rank, world, local_rank):
-    import torch
-    import precision_gemm_fp8_b200 as pg
+def measure_fp8_peak(torch, dev, seconds=2.0):
+    """Dense E4M3 GEMM throughput of the installed library (torch._scaled_mm,
+    8192^3, bf16 out, per-tensor unit scales): best of 10 single calls
+    (burst) and the mean of back-to-back calls over `seconds` (sustained,
+    power-capped).  Library timing, used only as a reference figure."""
+    n = 8192
+    try:
+        a = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn).t()
+        one = torch.ones((), device=dev, dtype=torch.float32)
+        fn = lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)  # noqa: E731
+        for _ in range(5):
+            fn()
+        torch.cuda.synchronize()
+        best = float("inf")
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        reps = max(10, int(seconds * 1e3 / best))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        e1.synchronize()
+        mean = e0.elapsed_time(e1) / reps
+        flops = 2.0 * n ** 3
+        del a, b
+        return {"burst_tflops": round(flops / (best * 1e-3) / 1e12, 1),
+                "sustained_tflops": round(flops / (mean * 1e-3) / 1e12, 1),
+                "how": f"torch._scaled_mm e4m3 x e4m3 -> bf16, {n}^3: best of 10 (burst), mean of {reps} back to "
+                       f"back (sustained)"}
+    except Exception as e:  # library without FP8 GEMM support: reported, not fatal
+        return {"error": f"{type(e).__name__}: {e}"[:200]}
 
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    peaks, peak_src = _load_peaks()
-    name = args.workload
+
+def setup_workload(pg, torch, dev, name):
+    """Weights quantised per channel (or split into NestedFP planes) on the
+    device, activations resident on the device and pinned on the host,
+    outputs and zero-filled workspaces: everything a step reads or writes."""
     copies = weight_copies(name)
     layers = workload_layers(name, copies)
-    wl = synthetic.WORKLOADS[name]
-
-    # ---- set-up (untimed): weights quantised per channel on the device, activations resident
     weights = {}
     for L in layers:
         key = (L.shape_idx, L.copy, L.kind in ("nested16", "nested8"))
         if key in weights:
             continue
         w = torch.from_numpy(synthetic.weights(name, L.shape_idx, copy=L.copy)).to(dev)
-        if key[2]:
-            weights[key] = pg.nestedfp_split(w)
-        else:
-            weights[key] = pg.fp8_quantize_rows(w)
+        weights[key] = pg.nestedfp_split(w) if key[2] else pg.fp8_quantize_rows(w)
         del w
     acts_host, acts, outs, qbufs = [], [], [], []
     for L in layers:
@@ -275,132 +309,276 @@ def run_ours(args, rank, world, local_rank):
             qbufs.append(torch.zeros(max(16, pg.nestedfp_linear_workspace_size(L.M, L.N, L.K, mode)),
                                      dtype=torch.uint8, device=dev))
     torch.cuda.synchronize()
+    return dict(name=name, copies=copies, layers=layers, weights=weights, acts_host=acts_host, acts=acts,
+                outs=outs, qbufs=qbufs)
 
-    stream = torch.cuda.Stream(device=dev)
-    # dynamic layers quantise with their own kernel first (the two-kernel
-    # form); with --fused-quant inside the GEMM where the kernel allows it
-    xflags = pg.FLAG_FUSED_QUANT if args.fused_quant else 0
-    sk_ws = torch.zeros(max(16, max(pg.lib.pgf8_fp8_linear_workspace_size(L.M, L.N, L.K) for L in layers)),
-                        dtype=torch.uint8, device=dev)
-    # per-tensor activation scaling instead of per-token dynamic (--scaling):
-    # one delayed-scaling history or one calibrated amax per layer
-    per_tensor = {}
-    if args.scaling != "dynamic":
-        for i, L in enumerate(layers):
-            if L.kind != "fp8":
-                continue
-            if args.scaling == "delayed":
-                per_tensor[i] = pg.DelayedScaling(1024, device=dev)
+
+def _wkey(L):
+    return (L.shape_idx, L.copy, L.kind != "fp8")
+
+
+GROUP_MAX_M = 128   # the library's grouped weight-streaming kernel takes layers up to this many tokens
+
+
+class StepRunner:
+    """Enqueues one step of a workload on `stream` through the C ABI.
+
+    Grouped form (FP8 workloads, per-token dynamic scales, the default): one
+    pgf8_fp8_linear_dynamic_group call for every layer of the step.  The
+    per-layer form (--per-layer, and every option that changes the layers'
+    producers) chains one call per layer with PGF8_FLAG_OVERLAP_PREVIOUS.
+
+    The bracketed step (for the roofline) runs the same kernels with an event
+    between consecutive launch groups: the grouped kernel on the M <= 16 layers
+    and on the 17..128 layers, then the quantisation and the GEMM of every
+    larger layer; its intervals are scaled to the timed step."""
+
+    def __init__(self, pg, torch, dev, wl, args, stream):
+        self.pg, self.torch, self.dev, self.wl, self.args, self.stream = pg, torch, dev, wl, args, stream
+        layers = wl["layers"]
+        self.layers = layers
+        self.grouped = (all(L.kind == "fp8" for L in layers) and not args.per_layer and not args.chain
+                        and args.scaling == "dynamic" and not args.fused_quant)
+        self.xflags = pg.FLAG_FUSED_QUANT if args.fused_quant else 0
+        self.sk_ws = torch.zeros(max(16, max(pg.lib.pgf8_fp8_linear_workspace_size(L.M, L.N, L.K) for L in layers)),
+                                 dtype=torch.uint8, device=dev)
+        if self.grouped:
+            ent = lambda i: (wl["acts"][i], *wl["weights"][_wkey(layers[i])], wl["outs"][i], wl["qbufs"][i])  # noqa: E731
+            self.group = pg.LayerGroup([ent(i) for i in range(len(layers))])
+            self.small = [i for i, L in enumerate(layers) if L.M <= 16]
+            self.mid = [i for i, L in enumerate(layers) if 16 < L.M <= GROUP_MAX_M]
+            self.large = [i for i, L in enumerate(layers) if L.M > GROUP_MAX_M]
+            self.sub = {k: pg.LayerGroup([ent(i) for i in idx]) for k, idx in (("small", self.small),
+                                                                                ("mid", self.mid)) if idx}
+        self.per_tensor = {}
+        if not self.grouped and args.scaling != "dynamic":
+            for i, L in enumerate(layers):
+                if L.kind == "fp8":
+                    self.per_tensor[i] = (pg.DelayedScaling(1024, device=dev) if args.scaling == "delayed"
+                                          else pg.fp8_amax_accumulate(wl["acts"][i]))
+            torch.cuda.synchronize()
+        self.gammas = {}
+        if args.chain:
+            if any(L.kind != "fp8" for L in layers) or len(synthetic.WORKLOADS[wl["name"]].shapes) != 4:
+                raise SystemExit("--chain needs a workload of QKV, O, gate+up, down FP8 layers")
+            g = torch.Generator().manual_seed(7)
+            for i, L in enumerate(layers):
+                if L.shape_idx in (0, 2):
+                    self.gammas[i] = (0.5 + torch.rand(L.K, generator=g)).to(dev)
+
+    # -- launches -------------------------------------------------------------------------------------------------
+    def launches_per_step(self):
+        if self.grouped:
+            n = 2 * ((len(self.layers) - len(self.large) + 31) // 32) if len(self.layers) > len(self.large) else 0
+            return n + 2 * len(self.large)
+        return sum(2 if L.kind in ("fp8", "nested8") else 1 for L in self.layers)
+
+    def _quantise(self, i, L, flags):
+        pg, wl, s = self.pg, self.wl, self.stream
+        aq, sa = pg.dynamic_workspace_views(wl["qbufs"][i], L.M, L.K)
+        if self.gammas and L.shape_idx in (0, 2):
+            pg.fp8_norm_quantize(wl["acts"][i], self.gammas[i], None, 1e-6, aq, sa, flags=flags, stream=s)
+        elif self.gammas and L.shape_idx == 3:
+            pg.fp8_silu_mul_quantize(wl["outs"][i - 1], aq, sa, flags=flags, stream=s)
+        elif i in self.per_tensor:
+            if self.args.scaling == "delayed":
+                self.per_tensor[i].step(wl["acts"][i], aq, sa, flags=flags, stream=s)
             else:
-                per_tensor[i] = pg.fp8_amax_accumulate(acts[i])   # MINMAX calibration on the layer's input
-        torch.cuda.synchronize()
-
-    # --chain: the decoder layer's own producers of each GEMM input: RMSNorm
-    # fused with the quantisation ahead of QKV and gate+up, the SiLU gate
-    # over the gate+up output fused with the quantisation ahead of down (O
-    # keeps its dynamic quantisation: its input is the attention output)
-    gammas = {}
-    if args.chain:
-        if any(L.kind != "fp8" for L in layers) or len(wl.shapes) != 4:
-            raise SystemExit("--chain needs a workload of QKV, O, gate+up, down FP8 layers")
-        g = torch.Generator().manual_seed(7)
-        for i, L in enumerate(layers):
-            if L.shape_idx in (0, 2):
-                gammas[i] = (0.5 + torch.rand(L.K, generator=g)).to(dev)
-
-    def quantise_chain(i, L, flags):
-        aq, sa = pg.dynamic_workspace_views(qbufs[i], L.M, L.K)
-        if L.shape_idx in (0, 2):
-            pg.fp8_norm_quantize(acts[i], gammas[i], None, 1e-6, aq, sa, flags=flags, stream=stream)
-        elif L.shape_idx == 3:
-            pg.fp8_silu_mul_quantize(outs[i - 1], aq, sa, flags=flags, stream=stream)
+                pg.fp8_quantize_tensor(wl["acts"][i], self.per_tensor[i], aq, sa, flags=flags, stream=s)
         else:
-            pg.fp8_quantize_rows(acts[i], aq, sa, stream=stream)
+            pg.fp8_quantize_rows(wl["acts"][i], aq, sa, stream=s)
         return aq, sa
 
-    def quantise_per_tensor(i, L, flags=0):
-        aq, sa = pg.dynamic_workspace_views(qbufs[i], L.M, L.K)
-        if args.scaling == "delayed":
-            per_tensor[i].step(acts[i], aq, sa, flags=flags, stream=stream)
-        else:
-            pg.fp8_quantize_tensor(acts[i], per_tensor[i], aq, sa, flags=flags, stream=stream)
-        return aq, sa
-
-    def enqueue_step(ev_pairs=None):
-        """One step through the C ABI on `stream`.
-
-        Without ev_pairs: the layers are chained as in inference — every call
-        carries FLAG_OVERLAP_PREVIOUS, so each layer's quantisation and weight
-        loads overlap the previous layer's tail (programmatic dependent
-        launch).  With ev_pairs: the same kernels through the two-call form,
-        an event pair bracketing every GEMM launch (each GEMM then runs in
-        isolation; these are the durations the roofline uses)."""
-        for i, L in enumerate(layers):
-            W = weights[(L.shape_idx, L.copy, L.kind != "fp8")]
-            if L.kind == "fp8" and args.chain:
-                if ev_pairs is None and L.shape_idx == 1:   # O: the dynamic pair, overlapped
-                    pg.fp8_linear_dynamic(acts[i], W[0], W[1], y=outs[i], workspace=qbufs[i],
-                                          flags=pg.FLAG_OVERLAP_PREVIOUS, stream=stream)
-                    continue
-                if ev_pairs is None:
-                    aq, sa = quantise_chain(i, L, pg.FLAG_OVERLAP_PREVIOUS)
-                    pg.fp8_linear(aq, sa, W[0], W[1], y=outs[i], workspace=sk_ws, flags=pg.FLAG_OVERLAP_PREVIOUS,
-                                  stream=stream)
-                    continue
-                ev_pairs[i][2].record(stream)
-                aq, sa = quantise_chain(i, L, 0)
-                ev_pairs[i][0].record(stream)
-                pg.fp8_linear(aq, sa, W[0], W[1], y=outs[i], workspace=sk_ws, stream=stream)
-                ev_pairs[i][1].record(stream)
-                continue
+    def step(self):
+        """One step as a user runs it (no events)."""
+        pg, wl, s = self.pg, self.wl, self.stream
+        if self.grouped:
+            self.group.run(flags=pg.FLAG_OVERLAP_PREVIOUS, stream=s)
+            return
+        ov = pg.FLAG_OVERLAP_PREVIOUS
+        for i, L in enumerate(self.layers):
+            W = wl["weights"][_wkey(L)]
             if L.kind == "fp8":
-                if ev_pairs is None and not per_tensor:
-                    pg.fp8_linear_dynamic(acts[i], W[0], W[1], y=outs[i], workspace=qbufs[i],
-                                          flags=pg.FLAG_OVERLAP_PREVIOUS | xflags, stream=stream)
+                if not self.gammas and not self.per_tensor:
+                    pg.fp8_linear_dynamic(wl["acts"][i], W[0], W[1], y=wl["outs"][i], workspace=wl["qbufs"][i],
+                                          flags=ov | self.xflags, stream=s)
                     continue
-                if ev_pairs is None:
-                    aq, sa = quantise_per_tensor(i, L, pg.FLAG_OVERLAP_PREVIOUS)
-                    pg.fp8_linear(aq, sa, W[0], W[1], y=outs[i], workspace=sk_ws, flags=pg.FLAG_OVERLAP_PREVIOUS,
-                                  stream=stream)
+                if self.gammas and L.shape_idx == 1:   # O: dynamic pair, overlapped
+                    pg.fp8_linear_dynamic(wl["acts"][i], W[0], W[1], y=wl["outs"][i], workspace=wl["qbufs"][i],
+                                          flags=ov, stream=s)
                     continue
-                ev_pairs[i][2].record(stream)
-                if per_tensor:
-                    aq, sa = quantise_per_tensor(i, L)
-                else:
-                    aq, sa = pg.dynamic_workspace_views(qbufs[i], L.M, L.K)
-                    pg.fp8_quantize_rows(acts[i], aq, sa, stream=stream)
-                ev_pairs[i][0].record(stream)
-                pg.fp8_linear(aq, sa, W[0], W[1], y=outs[i], workspace=sk_ws, stream=stream)
-                ev_pairs[i][1].record(stream)
+                aq, sa = self._quantise(i, L, ov)
+                pg.fp8_linear(aq, sa, W[0], W[1], y=wl["outs"][i], workspace=self.sk_ws, flags=ov, stream=s)
             else:
                 mode = pg.NESTED_FP16 if L.kind == "nested16" else pg.NESTED_FP8
-                if ev_pairs is not None:
-                    ev_pairs[i][0].record(stream)
-                pg.nestedfp_linear(acts[i], W[0], W[1] if mode == pg.NESTED_FP16 else None, mode=mode,
-                                   y=outs[i], workspace=qbufs[i],
-                                   flags=xflags if ev_pairs is not None else pg.FLAG_OVERLAP_PREVIOUS | xflags,
-                                   stream=stream)
-                if ev_pairs is not None:
-                    ev_pairs[i][1].record(stream)
+                pg.nestedfp_linear(wl["acts"][i], W[0], W[1] if mode == pg.NESTED_FP16 else None, mode=mode,
+                                   y=wl["outs"][i], workspace=wl["qbufs"][i], flags=ov | self.xflags, stream=s)
 
-    launches_per_step = sum(2 if L.kind in ("fp8", "nested8") else 1 for L in layers)
+    def bracketed_step(self, marks):
+        """The same kernels with an event recorded before every launch group
+        and one at the end: marks.append((segment, event))."""
+        pg, wl, s, torch = self.pg, self.wl, self.stream, self.torch
 
-    # ---- graph of R steps (R-1 chained, the last with per-GEMM events), replayed K / R times
-    K, W = args.steps, args.warmup
-    R = max(1, min(10, K))
-    while K % R:
+        def mark(seg):
+            e = torch.cuda.Event(enable_timing=True, external=True)
+            e.record(s)
+            marks.append((seg, e))
+
+        if self.grouped:
+            for key, idx in (("small", self.small), ("mid", self.mid)):
+                if idx:
+                    mark(("group", tuple(idx)))
+                    self.sub[key].run(stream=s)
+            for i in self.large:
+                L = self.layers[i]
+                W = wl["weights"][_wkey(L)]
+                mark(("quant", (i,)))
+                aq, sa = self._quantise(i, L, 0)
+                mark(("gemm", (i,)))
+                pg.fp8_linear(aq, sa, W[0], W[1], y=wl["outs"][i], workspace=self.sk_ws, stream=s)
+        else:
+            for i, L in enumerate(self.layers):
+                W = wl["weights"][_wkey(L)]
+                if L.kind == "fp8":
+                    mark(("quant", (i,)))
+                    aq, sa = self._quantise(i, L, 0)
+                    mark(("gemm", (i,)))
+                    pg.fp8_linear(aq, sa, W[0], W[1], y=wl["outs"][i], workspace=self.sk_ws, stream=s)
+                else:
+                    mode = pg.NESTED_FP16 if L.kind == "nested16" else pg.NESTED_FP8
+                    mark(("gemm", (i,)))
+                    pg.nestedfp_linear(wl["acts"][i], W[0], W[1] if mode == pg.NESTED_FP16 else None, mode=mode,
+                                       y=wl["outs"][i], workspace=wl["qbufs"][i], flags=self.xflags, stream=s)
+        mark(("end", ()))
+
+
+def quant_bytes(L):
+    xb = 2 if L.kind.startswith("nested") else 4
+    return L.M * L.K * (xb + 1) + 4 * L.M
+
+
+def analyse_segments(layers, marks, ms_step, peaks, fp8_peak):
+    """Per-segment durations of the bracketed step, scaled so that they sum
+    to the timed step (a kernel's share of the step times the step), the
+    dominant kernel's roofline and the regime checks of the layer's targets:
+    decode (M <= 16) >= 80 % of HBM, M 17..256 >= 75 % of HBM (weight
+    streaming), prefill (M >= 512) >= 60 % of the FP8 tensor peak."""
+    segs = []
+    for (seg, e0), (_, e1) in zip(marks[:-1], marks[1:]):
+        kind, idx = seg
+        segs.append({"kind": kind, "layers": list(idx), "ms": e0.elapsed_time(e1)})
+    total = sum(sg["ms"] for sg in segs)
+    scale = ms_step / total if total > 0 else 1.0
+    hbm = float(peaks["hbm_gbs"])
+    sustained = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    fp8_peak_tf = 2.0 * sustained
+    out = []
+    cls_time, cls_bytes, cls_flops = {}, {}, {}
+    for sg in segs:
+        Ls = [layers[i] for i in sg["layers"]]
+        t_in = sg["ms"] * scale
+        if sg["kind"] == "quant":
+            b = sum(quant_bytes(L) for L in Ls)
+            f = 0.0
+        else:
+            b = sum(L.gemm_bytes for L in Ls)
+            f = sum(L.flops for L in Ls)
+        wb = sum(L.weight_bytes for L in Ls) if sg["kind"] != "quant" else 0
+        cls = sg["kind"]
+        cls_time[cls] = cls_time.get(cls, 0.0) + t_in
+        cls_bytes[cls] = cls_bytes.get(cls, 0.0) + b
+        cls_flops[cls] = cls_flops.get(cls, 0.0) + f
+        out.append({"kind": sg["kind"], "M": sorted({L.M for L in Ls}), "shapes": len(Ls),
+                    "us_bracketed": round(sg["ms"] * 1e3, 2), "us_in_step": round(t_in * 1e3, 2),
+                    "gbs": round(b / (t_in * 1e-3) / 1e9, 1) if t_in > 0 else None,
+                    "weight_gbs": round(wb / (t_in * 1e-3) / 1e9, 1) if (t_in > 0 and wb) else None,
+                    "tflops": round(f / (t_in * 1e-3) / 1e12, 1) if (t_in > 0 and f) else None})
+    def peak_of(L):   # dense tensor peak of the layer's MMA kind (TFLOP/s)
+        return sustained if L.kind == "nested16" else fp8_peak_tf
+
+    dom = max(cls_time, key=cls_time.get)
+    t = cls_time[dom] * 1e-3
+    if dom == "gemm" and any(layers[i].M > 256 for sg in segs if sg["kind"] == "gemm" for i in sg["layers"]):
+        achieved = cls_flops[dom] / t / 1e12
+        dom_layers = [layers[i] for sg in segs if sg["kind"] == dom for i in sg["layers"]]
+        ideal_s = sum(L.flops / (peak_of(L) * 1e12) for L in dom_layers)
+        peak_eff = cls_flops[dom] / ideal_s / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak_eff, 1),
+                "unit": "TFLOP/s", "frac": round(ideal_s / t, 4),
+                "peak_source": "measured bf16 sustained (MEASURED_PEAKS.json) x 2 for E4M3 MMAs (the FP8/bf16 "
+                               "nominal ratio), x 1 for FP16 MMAs; kernels timed inside a long power-capped step"}
+        if fp8_peak and "sustained_tflops" in fp8_peak:
+            roof["frac_of_scaled_mm_fp8_sustained"] = round(achieved / fp8_peak["sustained_tflops"], 4)
+            roof["frac_of_scaled_mm_fp8_burst"] = round(achieved / fp8_peak["burst_tflops"], 4)
+        roof["kernel"] = "pgf8::gemm_pair_kernel / gemm_persistent_kernel (tiled GEMMs of the M > 128 layers)"
+    else:
+        achieved = cls_bytes[dom] / t / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4),
+                "peak_source": "measured HBM copy bandwidth (MEASURED_PEAKS.json)"}
+        roof["kernel"] = ("pgf8::gemm_group_kernel (with its quantisation launch)" if dom == "group"
+                          else "pgf8::gemm_kernel")
+    roof["dominant_class"] = dom
+    roof["kernel_ms_per_step"] = round(cls_time[dom], 5)
+    roof["share_of_step"] = round(cls_time[dom] / ms_step, 4)
+    roof["bracketed_over_timed_step"] = round(total / ms_step, 4)
+    roof["algorithmic_per_step"] = (f"{cls_flops[dom]:.4e} flop" if roof["bound"] == "tensor"
+                                    else f"{cls_bytes[dom]:.4e} B")
+
+    def regime(pred, what):
+        t_s = wbytes = fl = ideal = 0.0
+        for sg in segs:
+            Ls = [layers[i] for i in sg["layers"]]
+            if Ls and all(pred(L.M) for L in Ls):
+                t_s += sg["ms"] * scale * 1e-3
+                if sg["kind"] != "quant":
+                    wbytes += sum(L.weight_bytes for L in Ls)
+                    fl += sum(L.flops for L in Ls)
+                    ideal += sum(L.flops / (peak_of(L) * 1e12) for L in Ls)
+        if t_s == 0:
+            return None
+        if what == "hbm":
+            gbs = wbytes / t_s / 1e9
+            return {"weight_gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4)}
+        tf = fl / t_s / 1e12
+        r = {"tflops": round(tf, 1), "frac_fp8_peak": round(ideal / t_s, 4)}
+        if fp8_peak and "sustained_tflops" in fp8_peak:
+            r["frac_scaled_mm_fp8_sustained"] = round(tf / fp8_peak["sustained_tflops"], 4)
+        return r
+
+    regimes = {}
+    for key, pred, what, target in (("decode_m_le_16", lambda m: m <= 16, "hbm", 0.80),
+                                    ("stream_m_17_256", lambda m: 16 < m <= 256, "hbm", 0.75),
+                                    ("prefill_m_ge_512", lambda m: m >= 512, "tensor", 0.60)):
+        r = regime(pred, what)
+        if r is not None:
+            frac = r["frac_hbm"] if what == "hbm" else r["frac_fp8_peak"]
+            r["target"] = target
+            r["pass"] = bool(frac >= target)
+            regimes[key] = r
+    return roof, regimes, out
+
+
+def time_workload(pg, torch, dev, wl, args, steps, warmup, world, peaks, fp8_peak, clocks=False):
+    """Graph of R steps replayed (steps / R) times between barriers and
+    synchronizes, CUDA events on the launching stream, max over ranks; then
+    one bracketed step for the per-kernel shares."""
+    stream = torch.cuda.Stream(device=dev)
+    runner = StepRunner(pg, torch, dev, wl, args, stream)
+    layers = wl["layers"]
+    R = max(1, min(10, steps))
+    while steps % R:
         R -= 1
-    evs = [tuple(torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)) for _ in layers]
     with torch.cuda.stream(stream):
-        enqueue_step()          # load modules / first-call set-up outside capture
-        enqueue_step(evs)
+        runner.step()                      # first-call set-up outside capture
+        runner.bracketed_step([])
     stream.synchronize()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
-        for r in range(R):
-            enqueue_step(evs if r == R - 1 else None)
+        for _ in range(R):
+            runner.step()
     with torch.cuda.stream(stream):
-        for _ in range(max(1, W // R)):
+        for _ in range(max(1, -(-warmup // R))):
             graph.replay()
     torch.cuda.synchronize()
     if pg.device_status(stream) != pg.OK:
@@ -411,78 +589,74 @@ def run_ours(args, rank, world, local_rank):
             import torch.distributed as dist
             dist.barrier()
 
-    sampler = ClockSampler(local_rank)
-    sampler.start()
+    sampler = ClockSampler(dev.index or 0) if clocks else None
+    if sampler:
+        sampler.start()
     barrier()
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         t0.record(stream)
-        for _ in range(K // R):
+        for _ in range(steps // R):
             graph.replay()
         t1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    clocks = sampler.stop()
+    clk = sampler.stop() if sampler else None
     ms_total = max_over_ranks(t0.elapsed_time(t1), world, dev)
     st = pg.device_status(stream)
     if st != pg.OK:
         raise RuntimeError(f"device error word raised in the timed region: {st}")
+    ms_step = ms_total / steps
 
-    # per-GEMM durations (ms) from the event-bracketed step of the last replay
-    per_layer_ms = np.array([evs[i][0].elapsed_time(evs[i][1]) for i in range(len(layers))])
-    quant_ms = np.array([evs[i][2].elapsed_time(evs[i][0]) if L.kind == "fp8" else 0.0
-                         for i, L in enumerate(layers)])
-
-    ms_step = ms_total / K
+    # bracketed steps (outside the timed region): median of 3 per segment
+    runs = []
+    for _ in range(3):
+        marks = []
+        with torch.cuda.stream(stream):
+            runner.bracketed_step(marks)
+        stream.synchronize()
+        runs.append(marks)
+    # keep the middle run by total bracketed time
+    totals = [r[0][1].elapsed_time(r[-1][1]) for r in runs]
+    marks = runs[sorted(range(3), key=lambda k: totals[k])[1]]
+    roof, regimes, segments = analyse_segments(layers, marks, ms_step, peaks, fp8_peak)
+    del graph
     wbytes = sum(L.weight_bytes for L in layers)
     flops = sum(L.flops for L in layers)
+    return dict(runner=runner, ms_step=ms_step, R=R, wbytes=wbytes, flops=flops, roof=roof, regimes=regimes,
+                segments=segments, clocks=clk, launches=runner.launches_per_step())
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import precision_gemm_fp8_b200 as pg
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = _load_peaks()
+    name = args.workload
+    fp8_peak = measure_fp8_peak(torch, dev) if not args.no_fp8_peak else None
+    wl = setup_workload(pg, torch, dev, name)
+    layers = wl["layers"]
+    K, W = args.steps, args.warmup
+    res = time_workload(pg, torch, dev, wl, args, K, W, world, peaks, fp8_peak, clocks=True)
+    ms_step = res["ms_step"]
+    wbytes, flops = res["wbytes"], res["flops"]
     gbs = job_throughput(wbytes / 1e9, world, ms_step * 1e-3)        # whole job, all ranks
     tflops = job_throughput(flops / 1e12, world, ms_step * 1e-3)
-
-    # roofline of the dominant kernel (the GEMM)
-    gemm_bytes = sum(L.gemm_bytes for L in layers)
-    gemm_flops = sum(L.flops for L in layers)
-    gemm_time_s = per_layer_ms.sum() * 1e-3
     memory_bound = name in ("decode7b", "small")
-    if memory_bound:
-        achieved = gemm_bytes / gemm_time_s / 1e9
-        peak = float(peaks["hbm_gbs"])
-        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": None,
-                "peak_source": f"{peak_src} HBM copy bandwidth"}
-    else:
-        # The GEMMs are timed inside a long, power-capped step: the sustained
-        # bf16 figure is the denominator (x 2, the FP8 / bf16 nominal ratio);
-        # the fraction of the burst figure is reported beside it.
-        achieved = gemm_flops / gemm_time_s / 1e12
-        sustained = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
-        peak = 2.0 * sustained
-        burst = 2.0 * float(peaks["bf16_tflops"])
-        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": None,
-                "peak_source": f"{peak_src} bf16 sustained x 2 (FP8 nominal ratio); kernels timed inside a "
-                               f"long power-capped step",
-                "frac_of_burst_peak": round(achieved / burst, 4), "burst_peak": burst}
-    roof["kernel"] = "pgf8::gemm_kernel"
-    roof["launches_timed"] = int(len(layers))
-    # share of the GEMM among this step's kernels, each timed alone (the
-    # figure to compare with the ncu launch list, which also serialises)
-    roof["gemm_share_of_kernel_time"] = round(float(per_layer_ms.sum()) /
-                                              float(per_layer_ms.sum() + quant_ms.sum()), 3)
-    roof["gemm_isolated_sum_over_chained_step"] = round(float(per_layer_ms.sum()) / ms_step, 3)
+    roof = res["roof"]
     roof["traffic"], roof["traffic_note"] = profiled_traffic(name)
-
-    per_layer = []
-    for L, t in zip(layers, per_layer_ms):
-        per_layer.append({"kind": L.kind, "M": L.M, "K": L.K, "N": L.N, "us": round(t * 1e3, 2),
-                          "gbs": round(L.gemm_bytes / (t * 1e-3) / 1e9, 1),
-                          "tflops": round(L.flops / (t * 1e-3) / 1e12, 1)})
+    if fp8_peak is not None:
+        roof["fp8_scaled_mm_measured"] = fp8_peak
+    roof["peak_file"] = peak_src
 
     # ---- e2e through the public entry point, host buffers, copies inside the timed region
-    e2e = run_e2e(pg, torch, dev, layers, weights, acts_host, outs, args, world, wbytes, flops, memory_bound)
+    e2e = run_e2e(pg, torch, dev, wl, args, world, wbytes, flops, memory_bound)
 
+    grouped = res["runner"].grouped
     result = {
         "metric": METRIC,
         "value": round(gbs if memory_bound else tflops, 2),
@@ -498,36 +672,55 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic",
         "config": {"workload": f"{name}: {WORKLOAD_TEXT[name]}",
                    "l2": "inputs larger than L2 (%d weight copies; %.0f MB of weights streamed per step)"
-                         % (copies, wbytes / 1e6),
-                   "timing": "CUDA graph of the C-ABI calls (R-1 chained steps + 1 event-bracketed step), "
-                             "replayed K/R times, R=%d" % R,
-                   "quantisation": "inside the skinny GEMM where each CTA's activation slice fits its "
-                                   "registers, else its own kernel" if args.fused_quant
-                   else "own kernel before each GEMM",
+                         % (wl["copies"], wbytes / 1e6),
+                   "step": ("one pgf8_fp8_linear_dynamic_group call: the M <= 128 layers quantised by one launch and "
+                            "streamed by one grouped kernel, each larger layer quantised and multiplied by its own "
+                            "kernels" if grouped else
+                            "one call per layer, chained with PGF8_FLAG_OVERLAP_PREVIOUS"),
+                   "timing": "CUDA graph of the C-ABI calls, R=%d steps per replay, replayed K/R times" % res["R"],
+                   "quantisation": ("inside the skinny GEMM where each CTA's activation slice fits its registers"
+                                    if args.fused_quant else "per token, dynamic, own kernel before the GEMM"),
                    "chain": ("decoder layer: RMSNorm+quantise -> QKV; quantise -> O; RMSNorm+quantise -> "
                              "gate+up; SiLU gate+quantise of the gate+up output -> down") if args.chain else None,
                    "activation_scaling": {"dynamic": "per token, dynamic",
                                           "delayed": "per tensor, delayed (amax history of 1024 per layer)",
                                           "static": "per tensor, MINMAX-calibrated amax"}[args.scaling]},
-        "secondary": {"tflops": round(tflops, 3), "weight_gbs": round(gbs, 1)},
+        "secondary": {"tflops": round(tflops, 3), "weight_gbs": round(gbs, 1), "regimes": res["regimes"]},
         "roofline": roof,
         "e2e": e2e,
-        "gpu_launches": int(launches_per_step * K),
-        "clocks": clocks,
-        "per_layer": per_layer,
+        "gpu_launches": int(res["launches"] * K),
+        "clocks": res["clocks"],
+        "segments": res["segments"],
     }
+    del wl, res
+    torch.cuda.empty_cache()
+
+    # ---- the other configurations, each timed as its own step in this run
+    if not args.no_secondary and name == "llama70b":
+        for sec in ("decode7b", "prefill7b", "nested7b"):
+            wl2 = setup_workload(pg, torch, dev, sec)
+            steps2 = {"decode7b": 400, "prefill7b": 60, "nested7b": 60}[sec]
+            r2 = time_workload(pg, torch, dev, wl2, args, steps2, 10, world, peaks, fp8_peak)
+            mb = sec == "decode7b"
+            v = (r2["wbytes"] / 1e9 if mb else r2["flops"] / 1e12) / (r2["ms_step"] * 1e-3) * world
+            result["secondary"][sec] = {
+                "value": round(v, 2), "unit": "GB/s" if mb else "TFLOP/s", "ms_per_step": round(r2["ms_step"], 5),
+                "steps": steps2, "grouped": r2["runner"].grouped, "roofline": r2["roof"], "regimes": r2["regimes"],
+                "segments": r2["segments"]}
+            del wl2, r2
+            torch.cuda.empty_cache()
     return result
 
 
-def run_e2e(pg, torch, dev, layers, weights, acts_host, outs, args, world, wbytes, flops, memory_bound):
+def run_e2e(pg, torch, dev, wl, args, world, wbytes, flops, memory_bound):
     """The metric end to end through the public API with host buffers: every
     step copies all of its activations from one pinned host buffer to the
-    device, runs the layers (one pgf8_fp8_linear_dynamic_many call for the
-    FP8 workloads, one nestedfp_linear call per layer otherwise) and copies
-    all outputs back to one pinned host buffer; the copies are inside the
-    timed region."""
+    device, runs the step (one pgf8_fp8_linear_dynamic_group call for the FP8
+    workloads, one call per layer otherwise) and copies all outputs back to
+    one pinned host buffer; the copies are inside the timed region."""
+    layers, weights, acts_host, outs = wl["layers"], wl["weights"], wl["acts_host"], wl["outs"]
     stream = torch.cuda.Stream(device=dev)
-    # packed activations / outputs (16-byte aligned slices)
+
     def packed(tensors, device):
         offs, total = [], 0
         for t in tensors:
@@ -540,77 +733,21 @@ def run_e2e(pg, torch, dev, layers, weights, acts_host, outs, args, world, wbyte
     for v, a in zip(x_host_views, acts_host):
         v.copy_(a)
     x_dev, x_views = packed(acts_host, dev)
+    x_dev.copy_(x_host)          # calibrated per-tensor scales (--scaling static) read the inputs at set-up
+    torch.cuda.synchronize()
     y_dev, y_views = packed(outs, dev)
     y_host, _ = packed(outs, "cpu")
-    ws = []
-    for L in layers:
-        if L.kind == "fp8":
-            ws.append(torch.zeros(pg.fp8_linear_dynamic_workspace_size(L.M, L.N, L.K), dtype=torch.uint8,
-                                  device=dev))
-        else:
-            mode = pg.NESTED_FP8 if L.kind == "nested8" else pg.NESTED_FP16
-            ws.append(torch.zeros(max(16, pg.nestedfp_linear_workspace_size(L.M, L.N, L.K, mode)),
-                                  dtype=torch.uint8, device=dev))
-    all_fp8 = all(L.kind == "fp8" for L in layers)
-    seq = None
-    per_tensor = {}
-    gammas = {}
-    if all_fp8 and args.chain:
-        g = torch.Generator().manual_seed(7)
-        for i, L in enumerate(layers):
-            if L.shape_idx in (0, 2):
-                gammas[i] = (0.5 + torch.rand(L.K, generator=g)).to(dev)
-    elif all_fp8 and args.scaling != "dynamic":
-        for i, L in enumerate(layers):
-            per_tensor[i] = (pg.DelayedScaling(1024, device=dev) if args.scaling == "delayed"
-                             else pg.fp8_amax_accumulate(x_views[i].copy_(acts_host[i].to(dev))))
-        torch.cuda.synchronize()
-    elif all_fp8:
-        seq = pg.LayerSequence([(x_views[i], weights[(L.shape_idx, L.copy, False)][0],
-                                 weights[(L.shape_idx, L.copy, False)][1], y_views[i], ws[i])
-                                for i, L in enumerate(layers)])
+    ws = [torch.zeros_like(q) for q in wl["qbufs"]]
+    wl_e2e = dict(wl, acts=x_views, outs=y_views, qbufs=ws)
+    runner = StepRunner(pg, torch, dev, wl_e2e, args, stream)
 
     def step():
         with torch.cuda.stream(stream):
             x_dev.copy_(x_host, non_blocking=True)
-            if seq is not None:
-                seq.run(flags=pg.FLAG_FUSED_QUANT if args.fused_quant else 0, stream=stream)
-            elif gammas:
-                for i, L in enumerate(layers):
-                    W = weights[(L.shape_idx, L.copy, False)]
-                    aq, sa = pg.dynamic_workspace_views(ws[i], L.M, L.K)
-                    fl = pg.FLAG_OVERLAP_PREVIOUS if i else 0
-                    if L.shape_idx == 1:
-                        pg.fp8_linear_dynamic(x_views[i], W[0], W[1], y=y_views[i], workspace=ws[i], flags=fl,
-                                              stream=stream)
-                        continue
-                    if L.shape_idx in (0, 2):
-                        pg.fp8_norm_quantize(x_views[i], gammas[i], None, 1e-6, aq, sa, flags=fl, stream=stream)
-                    else:
-                        pg.fp8_silu_mul_quantize(y_views[i - 1], aq, sa, flags=fl, stream=stream)
-                    pg.fp8_linear(aq, sa, W[0], W[1], y=y_views[i], workspace=ws[i],
-                                  flags=pg.FLAG_OVERLAP_PREVIOUS, stream=stream)
-            elif per_tensor:
-                for i, L in enumerate(layers):
-                    W = weights[(L.shape_idx, L.copy, False)]
-                    aq, sa = pg.dynamic_workspace_views(ws[i], L.M, L.K)
-                    fl = pg.FLAG_OVERLAP_PREVIOUS if i else 0
-                    if args.scaling == "delayed":
-                        per_tensor[i].step(x_views[i], aq, sa, flags=fl, stream=stream)
-                    else:
-                        pg.fp8_quantize_tensor(x_views[i], per_tensor[i], aq, sa, flags=fl, stream=stream)
-                    pg.fp8_linear(aq, sa, W[0], W[1], y=y_views[i], workspace=ws[i],
-                                  flags=pg.FLAG_OVERLAP_PREVIOUS, stream=stream)
-            else:
-                for i, L in enumerate(layers):
-                    W = weights[(L.shape_idx, L.copy, True)]
-                    mode = pg.NESTED_FP16 if L.kind == "nested16" else pg.NESTED_FP8
-                    fl = (pg.FLAG_OVERLAP_PREVIOUS if i else 0) | (pg.FLAG_FUSED_QUANT if args.fused_quant else 0)
-                    pg.nestedfp_linear(x_views[i], W[0], W[1] if mode == pg.NESTED_FP16 else None, mode=mode,
-                                       y=y_views[i], workspace=ws[i], flags=fl, stream=stream)
+            runner.step()
             y_host.copy_(y_dev, non_blocking=True)
 
-    steps = max(3, min(args.steps, 200))
+    steps = max(3, min(args.steps, 100))
     for _ in range(3):
         step()
     stream.synchronize()
@@ -625,87 +762,133 @@ def run_e2e(pg, torch, dev, layers, weights, acts_host, outs, args, world, wbyte
     t1.record(stream)
     stream.synchronize()
     ms = max_over_ranks(t0.elapsed_time(t1) / steps, world, dev)
-    h2d = int(x_host.numel())
-    d2h = int(y_host.numel())
     v = job_throughput(wbytes / 1e9 if memory_bound else flops / 1e12, world, ms * 1e-3)
     return {"value": round(v, 2), "unit": "GB/s" if memory_bound else "TFLOP/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "h2d_bytes_per_step": int(x_host.numel()), "d2h_bytes_per_step": int(y_host.numel()), "steps": steps,
             "ms_per_step": round(ms, 5),
-            "entry_point": ("pgf8_nestedfp_linear" if not all_fp8 else
-                            "pgf8_fp8_norm_quantize / pgf8_fp8_silu_mul_quantize / pgf8_fp8_quantize_rows + "
-                            "pgf8_fp8_linear per layer" if args.chain else "pgf8_fp8_linear_dynamic_many"
-                            if args.scaling == "dynamic" else
-                            {"delayed": "pgf8_fp8_quantize_delayed", "static": "pgf8_fp8_quantize_tensor"}[args.scaling]
-                            + " + pgf8_fp8_linear per layer")}
+            "entry_point": ("pgf8_fp8_linear_dynamic_group" if runner.grouped else
+                            "one C-ABI call per layer (pgf8_fp8_linear_dynamic / pgf8_nestedfp_linear / the "
+                            "scaling and producer variants + pgf8_fp8_linear)")}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
-def oracle_sample(name, cols):
-    """Time the CPU oracle on every layer of one step of the workload: the
-    activations are quantised in full, the binary64 contraction runs on the
-    first `cols` output channels of each layer, and its time is extrapolated
-    linearly to all N channels.  Returns (seconds per full step, description,
-    threads used)."""
+ORACLE_SAMPLE = {  # per layer: first `rows` tokens x first `cols` output channels
+    "small": (16, 512), "decode7b": (8, 256), "prefill7b": (16, 48), "nested7b": (16, 96), "llama70b": (16, 64),
+}
+
+
+def oracle_inputs(name, rows=None, cols=None):
+    """Inputs of the bounded oracle sample of one step of the workload (not
+    timed): for every layer, its first `rows` tokens and the weights of its
+    first `cols` output channels, quantised / split as the layer stores them
+    (the weights' offline preparation is not part of the step)."""
     import oracle
 
-    layers = workload_layers(name, weight_copies(name))
-    total = 0.0
-    for L in layers:
-        x = synthetic.acts(name, L.shape_idx, L.m_idx)
-        ncols = min(cols, L.N)
-        w = synthetic.weights(name, L.shape_idx, copy=L.copy, n_override=ncols)
+    r0, c0 = ORACLE_SAMPLE[name]
+    rows, cols = rows or r0, cols or c0
+    items = []
+    for L in workload_layers(name, weight_copies(name)):
+        m = min(rows, L.M)
+        x = synthetic.acts(name, L.shape_idx, L.m_idx, M=m)
+        nc = min(cols, L.N)
+        w = synthetic.weights(name, L.shape_idx, copy=L.copy, n_override=nc)
+        prep = oracle.quantize_rows(w) if L.kind == "fp8" else oracle.nestedfp_split(w)
+        items.append((L, x, prep))
+    desc = (f"all {len(items)} layers of one step, each on its first {rows} tokens (quantised over the full K) x "
+            f"first {cols} output channels; value = work computed / seconds (no extrapolation)")
+    return items, desc
+
+
+def oracle_run(items, threads, pool=None):
+    """Time the CPU oracle, as it stands, on prepared sample inputs: the
+    per-token quantisation and the binary64 contraction of every layer, the
+    output channels split over `threads` host threads (the oracle is a C
+    library called through ctypes, which releases the interpreter lock, so
+    nothing of its arithmetic changes).  Returns (seconds, flops, weight bytes)."""
+    import oracle
+
+    total = flops = wbytes = 0.0
+    for L, x, prep in items:
+        nc = prep[0].shape[0]
+        parts = [p for p in np.array_split(np.arange(nc), threads) if p.size]
+        t0 = time.perf_counter()
         if L.kind == "fp8":
-            wq, sw = oracle.quantize_rows(w)      # offline weight quantisation: not timed
-            t0 = time.perf_counter()
+            wq, sw = prep
             aq, sa = oracle.quantize_rows(x)
-            t1 = time.perf_counter()
-            oracle.fp8_linear(aq, sa, wq, sw)
+            fn = lambda p: oracle.fp8_linear(aq, sa, wq[p[0]:p[-1] + 1], sw[p[0]:p[-1] + 1])  # noqa: E731
         elif L.kind == "nested16":
-            hi, lo = oracle.nestedfp_split(w)
-            t0 = t1 = time.perf_counter()
-            oracle.nestedfp_linear_fp16(x, hi, lo)
+            hi, lo = prep
+            fn = lambda p: oracle.nestedfp_linear_fp16(x, hi[p[0]:p[-1] + 1], lo[p[0]:p[-1] + 1])  # noqa: E731
         else:
-            hi, _ = oracle.nestedfp_split(w)
-            t0 = t1 = time.perf_counter()
-            oracle.nestedfp_linear_fp8(x, hi)
-        t2 = time.perf_counter()
-        total += (t1 - t0) + (t2 - t1) * (L.N / ncols)
-    desc = (f"all {len(layers)} layers of one step: activations quantised in full, binary64 contraction on "
-            f"the first {cols} output channels of each layer, its time scaled linearly to all N channels")
-    return total, desc, 1
+            hi = prep[0]
+            fn = lambda p: oracle.nestedfp_linear_fp8(x, hi[p[0]:p[-1] + 1])  # noqa: E731
+        if pool is not None and len(parts) > 1:
+            list(pool.map(fn, parts))
+        else:
+            fn(np.arange(nc))
+        total += time.perf_counter() - t0
+        flops += 2.0 * x.shape[0] * nc * L.K
+        wbytes += nc * L.K * (2 if L.kind == "nested16" else 1)
+    return total, flops, wbytes
+
+
+def cpu_baseline_entry(name, unit):
+    from concurrent.futures import ThreadPoolExecutor
+
+    threads = os.cpu_count() or 1
+    items, desc = oracle_inputs(name)
+    val = (lambda s, f, b: (b / s / 1e9) if unit == "GB/s" else (f / s / 1e12))
+    with ThreadPoolExecutor(threads) as pool:
+        sn, fn_, bn = oracle_run(items, threads, pool)
+        s1, f1, b1 = oracle_run(items, 1)
+        out = {"value": val(sn, fn_, bn), "unit": unit, "cores": threads, "kind": "oracle", "sample": desc,
+               "sample_seconds": round(sn, 3),
+               "single_thread": {"value": val(s1, f1, b1), "cores": 1, "sample_seconds": round(s1, 3)},
+               "host_cpus": os.cpu_count()}
+        if name in ("llama70b", "decode7b"):
+            # the decode7b step at M = 1 with every output channel of every layer
+            full, _ = oracle_inputs("decode7b", rows=1, cols=1 << 30)
+            full = [it for it in full if it[0].M == 1]
+            t, f, b = oracle_run(full, threads, pool)
+            out["decode7b_m1_full"] = {"weight_gbs": round(b / t / 1e9, 5), "tflops": f / t / 1e12,
+                                       "seconds": round(t, 3), "cores": threads,
+                                       "sample": "decode7b at M = 1: all four layers, every output channel"}
+    return out
 
 
 def run_reference(args):
     """The reference arm: the CPU oracle, as it stands, on the host cores; each
-    step is a bounded sample of one step of the workload (a number of output
-    channels per layer sized so the whole --steps/--warmup run takes about two
-    minutes), extrapolated to the full step."""
+    step is one bounded sample of the workload (every layer on its first
+    tokens x first output channels), sized so the whole --steps/--warmup run
+    takes about two minutes.  value = work computed / time, ms_per_step = the
+    sample's own time."""
+    from concurrent.futures import ThreadPoolExecutor
+
     name = args.workload
-    layers = workload_layers(name, weight_copies(name))
-    wbytes = sum(L.weight_bytes for L in layers)
-    flops = sum(L.flops for L in layers)
     memory_bound = name in ("decode7b", "small")
-    # size the per-step sample so the whole run takes about two minutes
-    t_start = time.perf_counter()
-    oracle_sample(name, cols=8)
-    t8 = time.perf_counter() - t_start
-    budget = max(0.02, 120.0 / (args.warmup + args.steps))
-    cols = int(max(1, min(4096, 8 * budget / max(t8, 1e-6))))
-    times = []
-    desc = ""
-    for i in range(args.warmup + args.steps):
-        s, desc, _ = oracle_sample(name, cols=cols)
-        if i >= args.warmup:
-            times.append(s)
+    threads = os.cpu_count() or 1
+    r0, c0 = ORACLE_SAMPLE[name]
+    with ThreadPoolExecutor(threads) as pool:
+        probe, _ = oracle_inputs(name, rows=r0, cols=max(1, c0 // 8))
+        s, _, _ = oracle_run(probe, threads, pool)
+        budget = max(0.05, 100.0 / (args.warmup + args.steps))
+        cols = int(max(1, min(c0 * 8, max(1, c0 // 8) * budget / max(s, 1e-6))))
+        items, desc = oracle_inputs(name, rows=r0, cols=cols)
+        times, fl, wb = [], 0.0, 0.0
+        for i in range(args.warmup + args.steps):
+            s, f, b = oracle_run(items, threads, pool)
+            if i >= args.warmup:
+                times.append(s)
+                fl, wb = f, b
     ms = 1e3 * sum(times) / len(times)
-    v = (wbytes / (ms * 1e-3) / 1e9) if memory_bound else (flops / (ms * 1e-3) / 1e12)
+    v = (wb / (ms * 1e-3) / 1e9) if memory_bound else (fl / (ms * 1e-3) / 1e12)
     unit = "GB/s" if memory_bound else "TFLOP/s"
     return {
         "metric": METRIC, "value": v, "unit": unit, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic", "impl": "reference",
         "config": {"workload": f"{name}: {WORKLOAD_TEXT[name]}"},
-        "cpu_baseline": {"kind": "oracle", "cores": 1, "sample": desc, "value": v, "unit": unit},
+        "cpu_baseline": {"kind": "oracle", "cores": threads, "sample": desc, "value": v, "unit": unit},
         "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -923,11 +1106,17 @@ def run_attention_context(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
-    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(synthetic.WORKLOADS), default="decode7b")
+    ap.add_argument("--workload", choices=sorted(synthetic.WORKLOADS), default="llama70b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="llama70b: skip timing decode7b, prefill7b and nested7b as secondary steps")
+    ap.add_argument("--no-fp8-peak", action="store_true", help="skip the torch._scaled_mm FP8 reference figure")
+    ap.add_argument("--per-layer", action="store_true",
+                    help="one C-ABI call per layer, chained (the form a dependent layer sequence runs in) instead "
+                         "of one grouped call per step")
     ap.add_argument("--scaling", choices=["dynamic", "delayed", "static"], default="dynamic",
                     help="activation scales of the FP8 layers: per-token dynamic (default), per-tensor delayed "
                          "(amax history of 1024) or per-tensor static (MINMAX-calibrated)")
@@ -990,14 +1179,7 @@ def main():
         res = run_ours(args, rank, world, local_rank)
         if rank == 0:
             if not args.no_cpu_baseline:
-                s, desc, cores = oracle_sample(args.workload, cols=1024)
-                layers = workload_layers(args.workload, weight_copies(args.workload))
-                wbytes = sum(L.weight_bytes for L in layers)
-                flops = sum(L.flops for L in layers)
-                v = (wbytes / s / 1e9) if res["unit"] == "GB/s" else (flops / s / 1e12)
-                res["cpu_baseline"] = {"value": v, "unit": res["unit"], "cores": cores, "kind": "oracle",
-                                       "sample": desc, "ms_per_step_extrapolated": round(s * 1e3, 1),
-                                       "host_cpus": os.cpu_count()}
+                res["cpu_baseline"] = cpu_baseline_entry(args.workload, res["unit"])
             print(json.dumps(res), flush=True)
     finally:
         if world > 1:
