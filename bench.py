@@ -328,10 +328,10 @@ class StepRunner:
     per-layer form (--per-layer, and every option that changes the layers'
     producers) chains one call per layer with PGF8_FLAG_OVERLAP_PREVIOUS.
 
-    The bracketed step (for the roofline) runs the same kernels with an event
-    between consecutive launch groups: the grouped kernel on the M <= 16 layers
-    and on the 17..128 layers, then the quantisation and the GEMM of every
-    larger layer; its intervals are scaled to the timed step."""
+    The bracketed step (for the roofline) runs the same launches with an
+    event between consecutive launch groups: the grouped kernel of each
+    token-tile class (M <= 16, 32, 64, 128), then the quantisation and the
+    GEMM of every larger layer; its intervals are scaled to the timed step."""
 
     def __init__(self, pg, torch, dev, wl, args, stream):
         self.pg, self.torch, self.dev, self.wl, self.args, self.stream = pg, torch, dev, wl, args, stream
@@ -345,11 +345,13 @@ class StepRunner:
         if self.grouped:
             ent = lambda i: (wl["acts"][i], *wl["weights"][_wkey(layers[i])], wl["outs"][i], wl["qbufs"][i])  # noqa: E731
             self.group = pg.LayerGroup([ent(i) for i in range(len(layers))])
-            self.small = [i for i, L in enumerate(layers) if L.M <= 16]
-            self.mid = [i for i, L in enumerate(layers) if 16 < L.M <= GROUP_MAX_M]
+            # the library's launches for a group: one grouped kernel per
+            # token-tile class (M <= 16, 32, 64, 128), then the larger layers
+            self.classes = [[i for i, L in enumerate(layers) if lo < L.M <= hi]
+                            for lo, hi in ((0, 16), (16, 32), (32, 64), (64, GROUP_MAX_M))]
+            self.classes = [c for c in self.classes if c]
             self.large = [i for i, L in enumerate(layers) if L.M > GROUP_MAX_M]
-            self.sub = {k: pg.LayerGroup([ent(i) for i in idx]) for k, idx in (("small", self.small),
-                                                                                ("mid", self.mid)) if idx}
+            self.sub = [pg.LayerGroup([ent(i) for i in idx]) for idx in self.classes]
         self.per_tensor = {}
         if not self.grouped and args.scaling != "dynamic":
             for i, L in enumerate(layers):
@@ -369,8 +371,7 @@ class StepRunner:
     # -- launches -------------------------------------------------------------------------------------------------
     def launches_per_step(self):
         if self.grouped:
-            n = 2 * ((len(self.layers) - len(self.large) + 31) // 32) if len(self.layers) > len(self.large) else 0
-            return n + 2 * len(self.large)
+            return sum(2 * ((len(c) + 31) // 32) for c in self.classes) + 2 * len(self.large)
         return sum(2 if L.kind in ("fp8", "nested8") else 1 for L in self.layers)
 
     def _quantise(self, i, L, flags):
@@ -425,10 +426,9 @@ class StepRunner:
             marks.append((seg, e))
 
         if self.grouped:
-            for key, idx in (("small", self.small), ("mid", self.mid)):
-                if idx:
-                    mark(("group", tuple(idx)))
-                    self.sub[key].run(stream=s)
+            for idx, sub in zip(self.classes, self.sub):
+                mark(("group", tuple(idx)))
+                sub.run(stream=s)
             for i in self.large:
                 L = self.layers[i]
                 W = wl["weights"][_wkey(L)]

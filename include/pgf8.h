@@ -122,6 +122,15 @@ typedef enum {
  * them in binary32. */
 #define PGF8_FLAG_ATTN_MMA 4
 
+/* PGF8_FLAG_STREAM_K_TAIL (FP8 linear entry points, M > 128, pair kernel):
+ * the last full round of 256 x 256 tiles and the ragged tail are split in
+ * equal k-block ranges over every SM pair, partial tiles summed in a fixed
+ * order through the workspace (pgf8_fp8_linear_workspace_size bytes for
+ * M > 128).  Off by default: measured on B200 it is slower than whole
+ * tiles on most 7B / 70B shapes (pairs working on disjoint k-ranges no
+ * longer share weight tiles in L2). */
+#define PGF8_FLAG_STREAM_K_TAIL 8
+
 /* Optional tuning of the linear entry points; a NULL pointer means all
  * defaults.  Fields set to 0 mean "choose automatically". */
 typedef struct {
@@ -450,8 +459,9 @@ size_t pgf8_fp8_linear_dynamic_scales_offset(int64_t M, int64_t K);
  *
  * Layers with M <= 128 are quantised by one launch and then streamed by one
  * persistent grouped kernel (one CTA per SM, each SM streaming an equal
- * share of all those layers' weights, up to 32 layers per launch pair);
- * larger layers run one dynamic call each afterwards.  Decode-sized layers
+ * share of all those layers' weights), one launch pair per token-tile class
+ * (M <= 16, <= 32, <= 64, <= 128) and per 32 layers of a class; larger
+ * layers run one dynamic call each afterwards.  Decode-sized layers
  * are bound by their weight stream ("7B token speed on consumer GPUs" §1),
  * and one stream for the whole group pays the start and the end of a
  * launch once instead of once per layer.
@@ -474,6 +484,50 @@ pgf8_status pgf8_fp8_linear_dynamic_group(const pgf8_fp8_layer *layers, int64_t 
                                           void *group_workspace, size_t group_workspace_bytes,
                                           const pgf8_linear_opts *opts, void *stream);
 size_t pgf8_fp8_linear_group_workspace_size(int64_t max_m);
+
+/* ------------------------------------------------------------------------
+ * Building blocks of a tensor-parallel FP8 linear layer ("C++ and FP8"
+ * §4.2: the --tp_size deployment; §5.2: the partial results of a split
+ * layer summed over NVLink).  A layer split along K (row-parallel) gives
+ * each rank a slice of every token's row, but the per-token scale must
+ * come from the amax over the WHOLE row ("7B on an RTX 4060 with FP8"
+ * §2.2, §6.1), and the partial products must be summed before the single
+ * rounding to bf16.  The sequence per rank is:
+ *   pgf8_fp8_row_amax        amax of each row of this rank's slice
+ *   (all-reduce MAX of the amax over the ranks)
+ *   pgf8_fp8_quantize_rows_amax   codes and scales from the reduced amax:
+ *                            bit-identical to pgf8_fp8_quantize_rows
+ *                            (DYNAMIC) on the full rows
+ *   pgf8_fp8_linear_partial  f32 partial sum of this rank's slice of K,
+ *                            scaled by sa[m] * sw[n] (sw of the full rows)
+ *   (all-reduce SUM of the f32 partials over the ranks)
+ *   pgf8_round_bf16          one rounding of the sum to bf16
+ * A layer split along N (column-parallel) needs none of this: each rank
+ * quantises the whole activation rows and runs pgf8_fp8_linear_dynamic on
+ * its channels.
+ *
+ * pgf8_fp8_row_amax: amax[r] = max_c |x[r, c]| (NaN ignored), x [rows,
+ *   cols] f32 or f16 (row stride ldx elements).  Checks and alignment as
+ *   pgf8_fp8_quantize_rows (no codes).
+ * pgf8_fp8_quantize_rows_amax: amax_scales[r] holds the row's amax on
+ *   input; on output it holds s = fl32(amax / 448) (1 for a zero amax), and
+ *   q[r, c] = E4M3_satfinite_RN(fl32(x[r, c] / s)).
+ * pgf8_fp8_linear_partial: y_f32[m, n] = fl32(sum_k e4m3(aq[m,k])
+ *   e4m3(wq[n,k]) * sa[m] * sw[n]) with f32 accumulation and no rounding
+ *   to 16 bits.  workspace: pgf8_fp8_linear_partial_workspace_size bytes,
+ *   16-byte aligned, zero-filled once (the kernels leave their flag words
+ *   zero).  y_f32 16-byte aligned.  Deterministic for a fixed shape.
+ * pgf8_round_bf16: y[i] = bf16_RN(x[i]); n % 8 == 0, both 16-byte aligned.
+ * ---------------------------------------------------------------------- */
+pgf8_status pgf8_fp8_row_amax(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
+                              float *amax, void *stream);
+pgf8_status pgf8_fp8_quantize_rows_amax(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols,
+                                        int64_t ldx, uint8_t *q, float *amax_scales, void *stream);
+pgf8_status pgf8_fp8_linear_partial(const uint8_t *aq, const float *sa, int64_t M, int64_t K,
+                                    const uint8_t *wq, const float *sw, int64_t N, float *y_f32,
+                                    void *workspace, size_t workspace_bytes, void *stream);
+size_t pgf8_fp8_linear_partial_workspace_size(int64_t M, int64_t N, int64_t K);
+pgf8_status pgf8_round_bf16(const float *x, int64_t n, void *y_bf16, void *stream);
 
 /* ------------------------------------------------------------------------
  * NestedFP byte-plane split ("NestedFP" §2.1): for each FP16 weight bit

@@ -35,6 +35,7 @@ PATH_AUTO, PATH_SKINNY, PATH_TILED, PATH_STREAMK, PATH_TILED_PAIR = 0, 1, 2, 3, 
 FLAG_OVERLAP_PREVIOUS = 1
 FLAG_FUSED_QUANT = 2
 FLAG_ATTN_MMA = 4
+FLAG_STREAM_K_TAIL = 8
 
 
 class LinearOpts(ctypes.Structure):
@@ -87,6 +88,11 @@ _SIGS = {
     "pgf8_fp8_linear_dynamic_scales_offset": ([_i64, _i64], _sz),
     "pgf8_fp8_linear_dynamic_group": ([ctypes.POINTER(Fp8Layer), _i64, _vp, _sz, _optp, _vp], _i32),
     "pgf8_fp8_linear_group_workspace_size": ([_i64], _sz),
+    "pgf8_fp8_row_amax": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp], _i32),
+    "pgf8_fp8_quantize_rows_amax": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _vp], _i32),
+    "pgf8_fp8_linear_partial": ([_vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _sz, _vp], _i32),
+    "pgf8_fp8_linear_partial_workspace_size": ([_i64, _i64, _i64], _sz),
+    "pgf8_round_bf16": ([_vp, _i64, _vp, _vp], _i32),
     "pgf8_nestedfp_split": ([_vp, _i64, _i64, _vp, _vp, _vp], _i32),
     "pgf8_nestedfp_linear": ([_vp, _i64, _i64, _vp, _vp, _i64, _i32, _vp, _vp, _sz, _vp], _i32),
     "pgf8_nestedfp_linear_ex": ([_vp, _i64, _i64, _vp, _vp, _i64, _i32, _vp, _vp, _sz, _optp, _vp], _i32),
@@ -472,6 +478,59 @@ def fp8_linear(aq, sa, wq, sw, y=None, workspace=None, path=PATH_AUTO, split_k=0
     _check(lib.pgf8_fp8_linear_ex(_ptr(aq), _ptr(sa), M, K, _ptr(wq), _ptr(sw), N, _ptr(y), _ptr(workspace),
                                   _nbytes(workspace), _opts(path, split_k, tile_n, flags), _stream(stream)),
            "fp8_linear")
+    return y
+
+
+def fp8_row_amax(x: torch.Tensor, amax: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """amax [rows] f32 = max_c |x[r, c]| of x [rows, cols] (f32 or f16)."""
+    rows, cols = x.shape
+    if x.stride(1) != 1:
+        raise ValueError("x rows must be contiguous")
+    if amax is None:
+        amax = torch.empty(rows, dtype=torch.float32, device=x.device)
+    _check(lib.pgf8_fp8_row_amax(_ptr(x), _dtype_code(x), rows, cols, _lead(x), _ptr(amax), _stream(stream)),
+           "fp8_row_amax")
+    return amax
+
+
+def fp8_quantize_rows_amax(x: torch.Tensor, amax: torch.Tensor, q: torch.Tensor | None = None, stream=None):
+    """Codes and scales of x [rows, cols] from the given per-row amax (taken
+    over the whole rows, of which x may hold a slice).  `amax` is replaced
+    by the scales in place.  Returns (q uint8 [rows, cols], scales = amax)."""
+    rows, cols = x.shape
+    if x.stride(1) != 1:
+        raise ValueError("x rows must be contiguous")
+    if amax.dtype != torch.float32 or amax.numel() != rows or not amax.is_contiguous():
+        raise ValueError("amax must be a contiguous float32 tensor with one entry per row")
+    if q is None:
+        q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    _check(lib.pgf8_fp8_quantize_rows_amax(_ptr(x), _dtype_code(x), rows, cols, _lead(x), _ptr(q), _ptr(amax),
+                                           _stream(stream)), "fp8_quantize_rows_amax")
+    return q, amax
+
+
+def fp8_linear_partial(aq, sa, wq, sw, y=None, workspace=None, stream=None):
+    """y [M,N] f32 = (E4M3 aq [M,K] x E4M3 wq [N,K]^T) * sa[m] * sw[n], summed
+    in f32 and not rounded: one rank's share of a layer split along K."""
+    M, K = aq.shape
+    N = wq.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=aq.device)
+    need = int(lib.pgf8_fp8_linear_partial_workspace_size(M, N, K))
+    if workspace is None:
+        workspace = default_workspace(aq.device, need)
+    _check(lib.pgf8_fp8_linear_partial(_ptr(aq), _ptr(sa), M, K, _ptr(wq), _ptr(sw), N, _ptr(y), _ptr(workspace),
+                                       _nbytes(workspace), _stream(stream)), "fp8_linear_partial")
+    return y
+
+
+def round_bf16(x: torch.Tensor, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y = bf16_RN(x) for a contiguous f32 tensor (numel % 8 == 0)."""
+    if x.dtype != torch.float32 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float32 tensor")
+    if y is None:
+        y = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device)
+    _check(lib.pgf8_round_bf16(_ptr(x), x.numel(), _ptr(y), _stream(stream)), "round_bf16")
     return y
 
 

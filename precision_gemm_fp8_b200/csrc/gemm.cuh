@@ -76,7 +76,8 @@ struct GemmParams {
     int prefetch_w;      // 1: weight tiles may be loaded before the grid dependency resolves
     const float *sa;     // [M] (kE4M3, kNested8)
     const float *sw;     // [N] (kE4M3)
-    void *y;             // [M, N] bf16 (kE4M3) or f16
+    void *y;             // [M, N] bf16 (kE4M3) or f16; f32 when out_f32
+    int out_f32;         // pair kernel, kE4M3: y is f32, the scaled sum before rounding
     // XQ kernels only
     const void *x;       // activations [M, K] f32 or f16, row stride ldx elements
     int64_t ldx;

@@ -21,9 +21,25 @@
 //                slower).
 //   acc_full[b]  per CTA: the same two-CTA commit.
 //   acc_empty[b] even CTA only: the 4 epilogue warps of both CTAs arrive.
+//
+// Wave quantisation: with T tiles on P pairs the last round of a plain
+// persistent walk keeps only T mod P pairs busy.  With a stream-K region
+// (sk.units > 0) the pairs walk the tiles below sk.t0 round-robin as
+// above (whole tiles; neighbouring pairs on neighbouring tiles, so weight
+// and activation tiles are shared in L2), and then split the remaining
+// tiles' (tile, k-block) units into equal contiguous ranges, one per pair.
+// sk.t0 leaves one full round plus the ragged tail to that region, so a
+// tile is split between two or three pairs at most.  Fix-up as in the
+// grouped kernel: a tile shared by several pairs is finished by the pair
+// holding its first k-block (its last segment, accumulator kept in tensor
+// memory); the following pairs store their f32 partial (each CTA its 128
+// rows) into their slot at the start of their range and raise a flag; the
+// finishing CTA adds them in pair order after its own (deterministic),
+// clears the flags and writes the tile.
 #pragma once
 
 #include "gemm.cuh"
+#include "gemm_streamk.cuh"
 
 namespace pgf8 {
 
@@ -49,12 +65,68 @@ template <int BN_, int STAGES_, int KIND_> struct PairCfg {
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
+constexpr int kPairSKMaxCtas = 160;              // partial slots (two per pair) in the workspace
+constexpr size_t kPairSKFlagBytes = 1024;        // 256 flag words: CTA index < kPairSKMaxCtas
+
+__host__ __device__ constexpr size_t pair_sk_workspace_bytes(int bn)
+{
+    return kPairSKFlagBytes + static_cast<size_t>(kPairSKMaxCtas) * 128 * bn * 4;
+}
+
+struct PairSK {
+    int t0;              // first tile of the stream-K region (tiles below: whole, round-robin)
+    int64_t units;       // (tile, k-block) units of the region; 0: no stream-K region
+    unsigned *flags;     // [kPairSKMaxCtas], zero between calls
+    float *partials;     // [kPairSKMaxCtas][BN][128]: this CTA's 128 rows, column-major
+};
+
+// One step of a pair's walk: tile t, k-blocks [kb0, kb1).  The whole tiles
+// of the round-robin part first, then the segments of the pair's range of
+// the stream-K region.
+struct PairWalk {
+    int pair, npairs, t0, kblocks;
+    int64_t units, u0, u1;
+    int t_next;          // next round-robin tile
+    int64_t u;           // next stream-K unit
+
+    __device__ __forceinline__ PairWalk(int pair_, int npairs_, const PairSK &sk, int total, int kblocks_)
+        : pair(pair_), npairs(npairs_), t0(sk.units > 0 ? sk.t0 : total), kblocks(kblocks_), units(sk.units)
+    {
+        u0 = sk.units > 0 ? (static_cast<int64_t>(pair) * sk.units) / npairs : 0;
+        u1 = sk.units > 0 ? (static_cast<int64_t>(pair + 1) * sk.units) / npairs : 0;
+        t_next = pair;
+        u = u0;
+    }
+    // false when the walk is over
+    __device__ __forceinline__ bool next(int &t, int &kb0, int &kb1)
+    {
+        if (t_next < t0) {
+            t = t_next;
+            kb0 = 0;
+            kb1 = kblocks;
+            t_next += npairs;
+            return true;
+        }
+        if (u >= u1)
+            return false;
+        const int local_t = static_cast<int>(u / kblocks);
+        kb0 = static_cast<int>(u % kblocks);
+        const int64_t tile_end = static_cast<int64_t>(local_t + 1) * kblocks;
+        const int64_t seg_end = u1 < tile_end ? u1 : tile_end;
+        kb1 = static_cast<int>(seg_end - static_cast<int64_t>(local_t) * kblocks);
+        t = t0 + local_t;
+        u = seg_end;
+        return true;
+    }
+};
+
 struct PairCtl {
     uint64_t full[16];
     uint64_t empty[16];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t drain;
+    uint64_t fix;        // stream-K region: partial tiles copied into shared memory
     uint32_t tmem_base;
     int abort;
 };
@@ -170,15 +242,13 @@ __device__ __forceinline__ bool wait_bounded_cluster(uint64_t *bar, uint32_t par
 template <class C>
 __global__ void __launch_bounds__(C::kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                     const __grid_constant__ CUtensorMap tmW2, const GemmParams p)
+                     const __grid_constant__ CUtensorMap tmW2, const GemmParams p, const PairSK sk)
 {
     constexpr int BN = C::BN;
     constexpr int STAGES = C::STAGES;
     constexpr int KIND = C::KIND;
     constexpr uint32_t kIdesc = make_idesc(256, BN, 0, KIND == kNested8 ? 1 : 0);
     (void)tmW2;
-
-    grid_launch_dependents();
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -205,6 +275,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             mbar_init(&ctl->acc_empty[b], 8);   // 4 epilogue warps in each CTA
         }
         mbar_init(&ctl->drain, 1);
+        mbar_init(&ctl->fix, 1);
         ctl->abort = 0;
         fence_mbar_init();
     }
@@ -222,6 +293,11 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = ctl->tmem_base;
     grid_dependency_wait();
+    // Dependents may start only now, when everything this grid depends on
+    // has completed: a dependent that does not wait itself (the next
+    // independent layer's quantisation in a grouped call) then still runs
+    // after every kernel before this one.
+    grid_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producers (both CTAs)
@@ -231,10 +307,12 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             uint32_t ph = 0;
             uint32_t issued_mask = 0, issued_ph = 0;
             bool ok = true;
-                    for (int t = pair; ok && t < total; t += npairs) {
+            PairWalk walk(pair, npairs, sk, total, p.kblocks);
+            int t, kb0, kb1;
+            while (ok && walk.next(t, kb0, kb1)) {
                 const int row_x = (t % m_tiles) * 256 + static_cast<int>(rank) * 128;
                 const int row_w = (t / m_tiles) * BN + static_cast<int>(rank) * (BN / 2);
-                for (int kb = 0; kb < p.kblocks; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!wait_bounded_cluster(&ctl->empty[s], ph ^ 1u, abort_flag)) {
                         ok = false;
                         break;
@@ -268,7 +346,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             uint32_t ph = 0;
             bool ok = true;
             int i = 0;
-            for (int t = pair; ok && t < total; t += npairs, ++i) {
+            PairWalk walk(pair, npairs, sk, total, p.kblocks);
+            int t, kb0, kb1;
+            for (; ok && walk.next(t, kb0, kb1); ++i) {
                 const int buf = i & 1;
                 const uint32_t use = static_cast<uint32_t>(i >> 1);
                 if (!wait_bounded_cluster(&ctl->acc_empty[buf], (use & 1u) ^ 1u, abort_flag)) {
@@ -277,7 +357,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                 }
                 tc_fence_after();
                 const uint32_t d = tmem + static_cast<uint32_t>(buf * BN);
-                for (int kb = 0; kb < p.kblocks; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!wait_bounded(&ctl->full[s], ph, abort_flag)) {
                         ok = false;
                         break;
@@ -289,7 +369,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     for (int k = 0; k < 4; ++k) {
                         const uint64_t ad = sdesc_sw128(a_addr + k * 32);
                         const uint64_t bd = sdesc_sw128(b_addr + k * 32);
-                        umma_f8f6f4_pair(d, ad, bd, kIdesc, (kb > 0 || k > 0) ? 1u : 0u);
+                        umma_f8f6f4_pair(d, ad, bd, kIdesc, (kb > kb0 || k > 0) ? 1u : 0u);
                     }
                     umma_commit_pair_both(&ctl->empty[s]);
                     if (++s == STAGES) {
@@ -311,43 +391,50 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         const int q = warp & 3;
         const int r = q * 32 + lane;
         const uint32_t t_row = tmem + (static_cast<uint32_t>(q * 32) << 16);
-        int i = 0;
-        for (int t = pair; t < total; t += npairs, ++i) {
-            const int buf = i & 1;
-            const uint32_t use = static_cast<uint32_t>(i >> 1);
-            bool ok = wait_bounded_cluster(&ctl->acc_full[buf], use & 1u, abort_flag);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok)
-                break;
-            tc_fence_after();
+        const int cta = static_cast<int>(blockIdx.x);
+        // scaled, rounded outputs of accumulator columns c0 .. c0 + 15 of row r of tile t
+        auto store16 = [&](int t, int c0, const float (&a)[16]) {
             const int m = (t % m_tiles) * 256 + static_cast<int>(rank) * 128 + r;
-            const int n_base = (t / m_tiles) * BN;
-            float sam = (m < p.M) ? p.sa[m] : 0.0f;
-#pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 16) {
-                const int n0 = n_base + c0;
-                if (n0 >= p.N)
-                    break;                      // warp-uniform; N % 16 == 0
-                uint32_t v[16];
-                tmem_ld_32x32b_x16(t_row + static_cast<uint32_t>(buf * BN + c0), v);
-                tmem_ld_wait();
-                if (m < p.M) {
-                    uint32_t o[8];
+            const int n0 = (t / m_tiles) * BN + c0;
+            if (m >= p.M || n0 >= p.N)
+                return;
+            const float sam = p.sa[m];
+            if constexpr (KIND == kE4M3) {
+                if (p.out_f32) {
+                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.y) + static_cast<int64_t>(m) * p.N +
+                                                             n0);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        float a0 = __uint_as_float(v[2 * j]) * sam, a1 = __uint_as_float(v[2 * j + 1]) * sam;
-                        if constexpr (KIND == kE4M3) {
-                            a0 = a0 * __ldg(p.sw + n0 + 2 * j);
-                            a1 = a1 * __ldg(p.sw + n0 + 2 * j + 1);
-                        }
-                        o[j] = pack2<KIND>(a0, a1);
-                    }
-                    uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.y) +
-                                                           static_cast<int64_t>(m) * p.N + n0);
-                    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-                    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+                    for (int j = 0; j < 4; ++j)
+                        dst[j] = make_float4(a[4 * j] * sam * __ldg(p.sw + n0 + 4 * j),
+                                             a[4 * j + 1] * sam * __ldg(p.sw + n0 + 4 * j + 1),
+                                             a[4 * j + 2] * sam * __ldg(p.sw + n0 + 4 * j + 2),
+                                             a[4 * j + 3] * sam * __ldg(p.sw + n0 + 4 * j + 3));
+                    return;
                 }
             }
+            uint32_t o[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float a0 = a[2 * j] * sam, a1 = a[2 * j + 1] * sam;
+                if constexpr (KIND == kE4M3) {
+                    a0 = a0 * __ldg(p.sw + n0 + 2 * j);
+                    a1 = a1 * __ldg(p.sw + n0 + 2 * j + 1);
+                }
+                o[j] = pack2<KIND>(a0, a1);
+            }
+            uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.y) + static_cast<int64_t>(m) * p.N + n0);
+            dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+            dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+        };
+        auto load16 = [&](uint32_t col, float (&a)[16]) {
+            uint32_t v[16];
+            tmem_ld_32x32b_x16(t_row + col, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                a[j] = __uint_as_float(v[j]);
+        };
+        auto release = [&](int buf) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -356,6 +443,83 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                 else
                     mbar_arrive_remote(&ctl->acc_empty[buf], 0u);
             }
+        };
+        int fin_t = -1, fin_buf = 0;
+        int i = 0;
+        PairWalk walk(pair, npairs, sk, total, p.kblocks);
+        int t, kb0, kb1;
+        for (; walk.next(t, kb0, kb1); ++i) {
+            const int buf = i & 1;
+            const uint32_t use = static_cast<uint32_t>(i >> 1);
+            bool ok = wait_bounded_cluster(&ctl->acc_full[buf], use & 1u, abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok)
+                break;
+            tc_fence_after();
+            if (kb0 == 0 && kb1 < p.kblocks) {
+                // the start of a tile finished with the following pairs'
+                // partials: always the last segment; kept in tensor memory
+                fin_t = t;
+                fin_buf = buf;
+                continue;
+            }
+            const bool contrib = kb0 > 0;   // always the first segment of the stream-K range
+            float *slot = sk.partials + static_cast<size_t>(cta) * BN * 128;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+                float a[16];
+                if (contrib) {
+                    load16(static_cast<uint32_t>(buf * BN + c0), a);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        __stcg(slot + (c0 + j) * 128 + r, a[j]);
+                } else {
+                    if ((t / m_tiles) * BN + c0 >= p.N)
+                        break;                  // warp-uniform; N % 16 == 0
+                    load16(static_cast<uint32_t>(buf * BN + c0), a);
+                    store16(t, c0, a);
+                }
+            }
+            release(buf);
+            if (contrib) {
+                __threadfence();
+                asm volatile("bar.sync 2, 128;" ::: "memory");
+                if (r == 0)
+                    st_release_u32(sk.flags + cta, 1u);
+            }
+        }
+        if (fin_t >= 0) {
+            // this pair's part, then the following pairs' partials in pair order
+            const int64_t last = static_cast<int64_t>(fin_t - sk.t0 + 1) * p.kblocks - 1;
+            const int p_last = sk_owner(last, sk.units, npairs);
+            bool got = true;
+            if (r == 0)
+                for (int pp = pair + 1; pp <= p_last && got; ++pp)
+                    got = wait_flag_sleep(sk.flags + 2 * pp + static_cast<int>(rank), abort_flag);
+            got = epi_all(got);
+            // the partials, one after another through the idle ring, into
+            // this pair's accumulator (the slots of this rank: every other one)
+            uint32_t fph = 0;
+            if (got && p_last > pair)
+                got = add_partials_into_tmem(t_row, static_cast<uint32_t>(fin_buf * BN), BN,
+                                             sk.partials + static_cast<size_t>(rank) * BN * 128,
+                                             static_cast<size_t>(2) * BN * 128, pair + 1, p_last, smem, &ctl->fix,
+                                             fph, abort_flag, r);
+            if (got) {
+#pragma unroll 1
+                for (int c0 = 0; c0 < BN; c0 += 16) {
+                    if ((fin_t / m_tiles) * BN + c0 >= p.N)
+                        break;
+                    float a[16];
+                    load16(static_cast<uint32_t>(fin_buf * BN + c0), a);
+                    store16(fin_t, c0, a);
+                }
+                asm volatile("bar.sync 2, 128;" ::: "memory");
+                if (r == 0)
+                    for (int pp = pair + 1; pp <= p_last; ++pp)
+                        sk.flags[2 * pp + rank] = 0u;
+            }
+            tc_fence_before();
         }
     }
 

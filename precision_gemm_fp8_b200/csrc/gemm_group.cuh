@@ -72,7 +72,8 @@ struct GroupLayer {
     int bn;              // token rows of the MMA: M rounded up to 16 (<= BNMAX)
     const float *sa;     // [M] per-token scales
     const float *sw;     // [N] per-channel scales
-    void *y;             // [M, N] bf16
+    void *y;             // [M, N] bf16, or f32 when out_f32
+    int out_f32;         // 1: y is f32, the scaled sum before rounding
 };
 
 struct GroupParams {
@@ -143,6 +144,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_group_kernel(const __grid
             mbar_init(&ctl->acc_empty[b], 4);
         }
         mbar_init(&ctl->drain, 1);
+        mbar_init(&ctl->fix, 1);
         ctl->abort = 0;
         fence_mbar_init();
     }
@@ -287,6 +289,14 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_group_kernel(const __grid
             if (n >= g.N)
                 return;
             const float swn = g.sw[n];
+            if (g.out_f32) {
+                float *y = static_cast<float *>(g.y);
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    if (c0 + j < g.M)
+                        y[static_cast<int64_t>(c0 + j) * g.N + n] = a[j] * __ldg(g.sa + c0 + j) * swn;
+                return;
+            }
             __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(g.y);
 #pragma unroll
             for (int j = 0; j < 16; ++j)
@@ -358,20 +368,22 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_group_kernel(const __grid
             const int64_t last = g.unit0 + static_cast<int64_t>(fin_t + 1) * g.kblocks - 1;
             const int c_last = sk_owner(last, p.units, G);
             bool got = true;
-            for (int cc = c + 1; cc <= c_last && got; ++cc)
-                got = wait_flag(p.flags + cc, abort_flag);
+            if (r == 0)
+                for (int cc = c + 1; cc <= c_last && got; ++cc)
+                    got = wait_flag_sleep(p.flags + cc, abort_flag);
             got = epi_all(got);
+            // the partials, one after another through the idle ring, into
+            // this CTA's accumulator
+            uint32_t fph = 0;
+            if (got && c_last > c)
+                got = add_partials_into_tmem(t_row, static_cast<uint32_t>(fin_buf * BNMAX), g.bn, p.partials,
+                                             static_cast<size_t>(BNMAX) * 128, c + 1, c_last, smem, &ctl->fix, fph,
+                                             abort_flag, r);
             if (got) {
 #pragma unroll 1
                 for (int c0 = 0; c0 < g.bn; c0 += 16) {
                     float a[16];
                     load16(static_cast<uint32_t>(fin_buf * BNMAX + c0), a);
-                    for (int cc = c + 1; cc <= c_last; ++cc) {
-                        const float *slot = p.partials + static_cast<size_t>(cc) * BNMAX * 128;
-#pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            a[j] += __ldcg(slot + (c0 + j) * 128 + r);
-                    }
                     store16(g, fin_t, c0, a);
                 }
                 asm volatile("bar.sync 2, 128;" ::: "memory");

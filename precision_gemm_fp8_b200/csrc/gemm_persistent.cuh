@@ -51,6 +51,7 @@ struct PersistCtl {
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t drain;
+    uint64_t fix;        // stream-K kernels: partial tiles copied into shared memory
     uint32_t tmem_base;
     int abort;
 };

@@ -112,6 +112,78 @@ __device__ __forceinline__ bool wait_flag(const unsigned *f, volatile int *abort
     }
 }
 
+// Bounded wait for a flag word, for ONE thread of a CTA, sleeping between
+// polls (64 ns doubling to 1 us): a CTA of spinning threads would flood L2
+// with loads that the TMA loads of the CTAs still computing need.  The
+// caller releases the CTA's other threads with a barrier afterwards.
+__device__ __forceinline__ bool wait_flag_sleep(const unsigned *f, volatile int *abort)
+{
+    if (ld_acquire_u32(f) != 0u)
+        return true;
+    const uint64_t t0 = global_timer_ns();
+    unsigned ns = 64;
+    for (;;) {
+        __nanosleep(ns);
+        if (ld_acquire_u32(f) != 0u)
+            return true;
+        if (ns < 1024)
+            ns <<= 1;
+        if (*abort)
+            return false;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            *abort = 1;
+            atomicOr(&g_device_error, kErrTimeout);
+            return false;
+        }
+    }
+}
+
+// Finishing side of a tile shared by several CTAs: adds the partial tiles
+// of the CTAs cfirst .. clast (slot c at parts + c * slot_floats; column j
+// of accumulator row r at j * 128 + r) in that order into this CTA's
+// accumulator columns [col0, col0 + ncols) of tensor memory, for the 128
+// rows owned by warps 2-5 (thread r; t_row = its warp's lane quadrant).
+// One partial at a time, one thread copies it whole into `stage` (idle
+// shared memory of at least ncols * 512 bytes) with the bulk-copy engine;
+// every thread then adds its row from shared memory into tensor memory.
+// Reading the partials from global memory chunk by chunk instead costs a
+// dependent L2 round trip per 16 columns.  Returns false when a wait gave
+// up.  Called by all 128 threads; uses named barrier 2.
+__device__ __forceinline__ bool add_partials_into_tmem(uint32_t t_row, uint32_t col0, int ncols, const float *parts,
+                                                       size_t slot_floats, int cfirst, int clast, uint8_t *stage,
+                                                       uint64_t *bar, uint32_t &phase, volatile int *abort, int r)
+{
+    const float *st = reinterpret_cast<const float *>(stage);
+    for (int c = cfirst; c <= clast; ++c) {
+        if (r == 0) {
+            fence_proxy_async_smem();   // earlier generic reads of `stage` before the copy overwrites it
+            mbar_arrive_expect_tx(bar, static_cast<uint32_t>(ncols) * 512u);
+            bulk_copy_g2s(stage, parts + static_cast<size_t>(c) * slot_floats, static_cast<uint32_t>(ncols) * 512u,
+                          bar);
+        }
+        bool ok = wait_bounded(bar, phase, abort);
+        phase ^= 1u;
+        if (!epi_all(ok)) {
+            if (r == 0)
+                wait_drain(bar, phase ^ 1u);   // the copy in flight lands before the CTA may exit
+            return false;
+        }
+#pragma unroll 1
+        for (int c0 = 0; c0 < ncols; c0 += 16) {
+            uint32_t v[16];
+            tmem_ld_32x32b_x16(t_row + col0 + static_cast<uint32_t>(c0), v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                v[j] = __float_as_uint(__uint_as_float(v[j]) + st[(c0 + j) * 128 + r]);
+            tmem_st_32x32b_x16(t_row + col0 + static_cast<uint32_t>(c0), v);
+        }
+        tmem_st_wait();
+        asm volatile("bar.sync 2, 128;" ::: "memory");   // every row read before the next copy
+    }
+    return true;
+}
+
 __device__ __forceinline__ int64_t sk_unit_begin(int c, int64_t units, int G)
 {
     return (static_cast<int64_t>(c) * units) / G;
@@ -390,11 +462,11 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             for (int j = 0; j < BN; ++j)
                 sum[j] = 0.0f;
             bool got = true;
-            for (int cc = c_first; cc < c; ++cc) {
-                if (!wait_flag(q.flags + cc, abort_flag)) {
-                    got = false;
-                    break;
-                }
+            if (r == 0)
+                for (int cc = c_first; cc < c && got; ++cc)
+                    got = wait_flag_sleep(q.flags + cc, abort_flag);
+            got = epi_all(got);
+            for (int cc = c_first; got && cc < c; ++cc) {
                 const float *slot = q.partials + static_cast<size_t>(cc) * BN * 128;
 #pragma unroll
                 for (int j = 0; j < BN; ++j)

@@ -155,6 +155,7 @@ struct GemmLaunch {
     // in-kernel quantisation (XQ kernels): raw activations and side outputs
     const void *xraw = nullptr;
     int64_t ldx = 0;
+    int out_f32 = 0;   // pair kernel: f32 outputs
     uint8_t *q_out = nullptr;
     float *sa_out = nullptr;
 };
@@ -203,6 +204,7 @@ static GemmParams make_params(const GemmLaunch &L, int splits)
     p.sa = L.sa;
     p.sw = L.sw;
     p.y = L.y;
+    p.out_f32 = L.out_f32;
     p.x = L.xraw;
     p.ldx = L.ldx;
     p.q_out = L.q_out;
@@ -341,10 +343,25 @@ template <class C> static pgf8_status launch_pair(const GemmLaunch &L)
     }, &pairs_fit);
     if (fit_err != cudaSuccess)
         return cuda_fail(fit_err);
-    const int64_t pairs = tiles < pairs_fit ? tiles : pairs_fit;
+    // Stream-K region (on request, when the workspace holds the partial
+    // slots and the tiles do not fill whole rounds): one full round plus the
+    // ragged tail, split in equal k-block ranges over every pair.
+    PairSK sk;
+    std::memset(&sk, 0, sizeof(sk));
+    int64_t pairs = tiles < pairs_fit ? tiles : pairs_fit;
+    const int64_t sk_pairs = pairs_fit < kPairSKMaxCtas / 2 ? pairs_fit : kPairSKMaxCtas / 2;
+    if ((L.opts.flags & PGF8_FLAG_STREAM_K_TAIL) && L.ws != nullptr && L.ws_bytes >= pair_sk_workspace_bytes(C::BN) &&
+        tiles % sk_pairs != 0 && L.opts.split_k == 0) {
+        const int64_t rounds = tiles / sk_pairs;
+        sk.t0 = static_cast<int>((rounds > 1 ? rounds - 1 : 0) * sk_pairs);
+        sk.units = (tiles - sk.t0) * p.kblocks;
+        sk.flags = static_cast<unsigned *>(L.ws);
+        sk.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(L.ws) + kPairSKFlagBytes);
+        pairs = sk_pairs < sk.units ? sk_pairs : sk.units;
+    }
     cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
     fill_attrs(cfg, attrs, 1, L.pdl, 2);
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<C>, tmX, tmW, tmW2, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<C>, tmX, tmW, tmW2, p, sk);
     if (e != cudaSuccess)
         return cuda_fail(e);
     return PGF8_OK;
@@ -546,14 +563,17 @@ template <int KIND> static pgf8_status launch_gemm(const GemmLaunch &L)
         default: return launch_split_or_not<KIND, true, 128, 6>(L, splits);
         }
     }
-    // FP8 operands with at least about one wave of 256 x 256 tiles (74 SM
-    // pairs): the pair kernel (measured faster there on every 7B / 70B shape)
+    // FP8 operands with at least about half a round of 256 x 256 tiles (74
+    // SM pairs): the pair kernel.  Measured on B200 over every tiled 7B /
+    // 70B shape (M = 256 .. 4096): with 40 or more tiles it is the fastest or
+    // within 3 %; with 32 tiles the one-CTA persistent kernel below is
+    // faster (more SMs busy on 128-row tiles).
     if constexpr (KIND != kNested16) {
         const int64_t tiles_pair = static_cast<int64_t>((L.M + 255) / 256) * ((L.N + 255) / 256);
         // (the 192 / 128 widths fill the last round better but measured slower
         // per tile than 256 on nearly every 7B / 70B shape; they stay
         // selectable through tile_n)
-        if (L.opts.path == PGF8_PATH_AUTO && bn == 0 && splits == 0 && tiles_pair >= 80)
+        if (L.opts.path == PGF8_PATH_AUTO && bn == 0 && splits == 0 && tiles_pair >= 40)
             return launch_pair_bn<KIND>(L, 256);
     }
     const int mt = (L.M + 127) / 128;
@@ -605,8 +625,9 @@ static pgf8_linear_opts opts_or_default(const pgf8_linear_opts *o)
 
 static pgf8_status quantize_launch(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
                                    uint8_t *q, float *scales, int mode, cudaStream_t st, int pdl,
-                                   int trigger_early)
+                                   int trigger_early, int no_wait = 0)
 {
+    const int qflags = (trigger_early ? kQuantTriggerEarly : 0) | (no_wait ? kQuantNoWait : 0);
     if (rows == 0)
         return PGF8_OK;
     cudaLaunchConfig_t cfg;
@@ -621,13 +642,37 @@ static pgf8_status quantize_launch(const void *x, pgf8_dtype xdt, int64_t rows, 
         cfg.attrs = attr;
         cfg.numAttrs = 1;
     }
+    // rows held in registers by the smallest CTA footprint that fits them
+    // (1, 2 or 4 chunks of 16 per thread of 256); longer rows take the
+    // two-pass kernel (measured faster at 28672 than a 512-thread CTA
+    // holding the row)
+    const int64_t nchunk = cols / 16;
     cudaError_t e;
-    if (xdt == PGF8_F32)
-        e = cudaLaunchKernelEx(&cfg, quantize_rows_kernel<float>, static_cast<const float *>(x), rows, cols, ldx, q,
-                               scales, mode, trigger_early);
-    else
-        e = cudaLaunchKernelEx(&cfg, quantize_rows_kernel<__half>, static_cast<const __half *>(x), rows, cols, ldx,
-                               q, scales, mode, trigger_early);
+    auto launch = [&](auto kern, unsigned threads, auto xp) {
+        cfg.blockDim = dim3(threads);
+        return cudaLaunchKernelEx(&cfg, kern, xp, rows, cols, ldx, q, scales, mode, qflags);
+    };
+    const float *xf = static_cast<const float *>(x);
+    const __half *xh = static_cast<const __half *>(x);
+    if (xdt == PGF8_F32) {
+        if (nchunk <= 256)
+            e = launch(quantize_rows_held_kernel<float, 1, 256>, 256, xf);
+        else if (nchunk <= 512)
+            e = launch(quantize_rows_held_kernel<float, 2, 256>, 256, xf);
+        else if (nchunk <= 1024)
+            e = launch(quantize_rows_held_kernel<float, 4, 256>, 256, xf);
+        else
+            e = launch(quantize_rows_kernel<float>, kQuantThreads, xf);
+    } else {
+        if (nchunk <= 256)
+            e = launch(quantize_rows_held_kernel<__half, 1, 256>, 256, xh);
+        else if (nchunk <= 512)
+            e = launch(quantize_rows_held_kernel<__half, 2, 256>, 256, xh);
+        else if (nchunk <= 1024)
+            e = launch(quantize_rows_held_kernel<__half, 4, 256>, 256, xh);
+        else
+            e = launch(quantize_rows_kernel<__half>, kQuantThreads, xh);
+    }
     if (e != cudaSuccess)
         return cuda_fail(e);
     return PGF8_OK;
@@ -1161,9 +1206,45 @@ pgf8_status pgf8_fp8_quantize_rows(const void *x, pgf8_dtype xdt, int64_t rows, 
                            static_cast<cudaStream_t>(stream), 0, 0);
 }
 
+pgf8_status pgf8_fp8_row_amax(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx, float *amax,
+                              void *stream)
+{
+    pgf8_status st = check_tensor_args(x, xdt, rows, cols, ldx, nullptr, false, amax);
+    if (st != PGF8_OK)
+        return st;
+    if (rows > 0 && !amax)
+        return PGF8_ERR_INVALID_ARG;
+    return quantize_launch(x, xdt, rows, cols, ldx, nullptr, amax, kQuantAmaxOnly, static_cast<cudaStream_t>(stream),
+                           0, 0);
+}
+
+pgf8_status pgf8_fp8_quantize_rows_amax(const void *x, pgf8_dtype xdt, int64_t rows, int64_t cols, int64_t ldx,
+                                        uint8_t *q, float *amax_scales, void *stream)
+{
+    pgf8_status st = check_quantize_args(x, xdt, rows, cols, ldx, q, amax_scales, PGF8_SCALE_DYNAMIC);
+    if (st != PGF8_OK)
+        return st;
+    return quantize_launch(x, xdt, rows, cols, ldx, q, amax_scales, kQuantFromAmax,
+                           static_cast<cudaStream_t>(stream), 0, 0);
+}
+
 static size_t streamk_bytes_for(int64_t M) { return M >= 1 && M <= 32 ? streamk_workspace_bytes(M <= 16 ? 16 : 32) : 0; }
 
-size_t pgf8_fp8_linear_workspace_size(int64_t M, int64_t, int64_t) { return streamk_bytes_for(M); }
+// Workspace of an FP8 linear call: the stream-K region of the kernel the
+// call takes (flag words at offset 0 in every layout): skinny stream-K slots
+// for M <= 32, the pair kernel's partial slots for M > 128.
+static_assert(kPairSKFlagBytes == kStreamKFlagBytes, "flag words at the start of every workspace layout");
+
+static size_t linear_ws_bytes(int64_t M)
+{
+    if (M >= 1 && M <= 32)
+        return streamk_bytes_for(M);
+    if (M > 128)
+        return pair_sk_workspace_bytes(256);
+    return 0;
+}
+
+size_t pgf8_fp8_linear_workspace_size(int64_t M, int64_t, int64_t) { return linear_ws_bytes(M); }
 
 pgf8_status pgf8_fp8_linear_ex(const uint8_t *aq, const float *sa, int64_t M, int64_t K, const uint8_t *wq,
                                const float *sw, int64_t N, void *y, void *workspace, size_t workspace_bytes,
@@ -1206,12 +1287,14 @@ pgf8_status pgf8_fp8_linear(const uint8_t *aq, const float *sa, int64_t M, int64
 
 // Dynamic workspace layout: stream-K flag words (always, so they are never
 // overwritten by codes when one workspace serves layers of different shapes)
-// | stream-K partial slots (M <= 32) | codes [M, K] | scales [M].
+// | stream-K partial slots (M <= 32: skinny; M > 128: pair kernel) | codes
+// [M, K] | scales [M].
 size_t pgf8_fp8_linear_dynamic_codes_offset(int64_t M, int64_t K)
 {
     if (M < 0 || K < 0)
         return 0;
-    return M >= 1 && M <= 32 ? streamk_bytes_for(M) : kStreamKFlagBytes;
+    const size_t b = linear_ws_bytes(M);
+    return b > kStreamKFlagBytes ? b : kStreamKFlagBytes;
 }
 
 size_t pgf8_fp8_linear_dynamic_scales_offset(int64_t M, int64_t K)
@@ -1248,10 +1331,13 @@ static pgf8_status check_linear_dynamic(const void *x, pgf8_dtype xdt, int64_t M
     return check_quantize_args(x, xdt, M, K, ldx, aq, sa, PGF8_SCALE_DYNAMIC);
 }
 
+// quant_no_wait: the quantisation does not wait for the previous kernel in
+// the stream (a grouped call's previous independent layer, run by the pair
+// kernel, which signals its dependents only after its own wait).
 static pgf8_status linear_dynamic_impl(const void *x, pgf8_dtype xdt, int64_t M, int64_t K, int64_t ldx,
                                        const void *w, const void *w2, const float *sw, int64_t N, void *y,
                                        void *workspace, size_t workspace_bytes, const pgf8_linear_opts *opts,
-                                       void *stream, int kind)
+                                       void *stream, int kind, bool quant_no_wait = false)
 {
     pgf8_status st = check_linear_dynamic(x, xdt, M, K, ldx, w, sw, N, y, workspace, workspace_bytes, kind);
     if (st != PGF8_OK)
@@ -1294,7 +1380,7 @@ static pgf8_status linear_dynamic_impl(const void *x, pgf8_dtype xdt, int64_t M,
     }
     // the quantisation signals its dependent (this call's GEMM) at once: the
     // GEMM loads its first weight tiles while the activations are quantised
-    st = quantize_launch(x, xdt, M, K, ldx, aq, sa, 0, cs, overlap, 1);
+    st = quantize_launch(x, xdt, M, K, ldx, aq, sa, 0, cs, overlap || quant_no_wait, 1, quant_no_wait ? 1 : 0);
     if (st != PGF8_OK)
         return st;
     GemmLaunch L;
@@ -1424,6 +1510,27 @@ template <class C> static pgf8_status launch_group_cfg(const GroupParams &p, int
     return PGF8_OK;
 }
 
+// The grouped kernel for the layers described in gp (units already set),
+// token tile bnmax, one CTA per SM at most.
+static pgf8_status launch_group(const GroupParams &gp, int bnmax, cudaStream_t cs)
+{
+    int grid = num_sms();
+    if (grid > kGroupMaxCtas)
+        grid = kGroupMaxCtas;
+    if (static_cast<int64_t>(grid) > gp.units)
+        grid = static_cast<int>(gp.units);
+    switch (bnmax) {
+    case 16:
+        return launch_group_cfg<GroupCfg<16, 12>>(gp, grid, cs);
+    case 32:
+        return launch_group_cfg<GroupCfg<32, 11>>(gp, grid, cs);
+    case 64:
+        return launch_group_cfg<GroupCfg<64, 9>>(gp, grid, cs);
+    default:
+        return launch_group_cfg<GroupCfg<128, 6>>(gp, grid, cs);
+    }
+}
+
 // One grouped launch pair for up to kGroupMaxLayers small-M layers: the
 // per-token quantisation of all of them, then the grouped GEMM, which
 // streams its first ring of weights while the quantisation runs.
@@ -1494,21 +1601,7 @@ static pgf8_status group_chunk(const pgf8_fp8_layer *const *ls, int n, void *gro
     if (e != cudaSuccess)
         return cuda_fail(e);
 
-    int grid = num_sms();
-    if (grid > kGroupMaxCtas)
-        grid = kGroupMaxCtas;
-    if (static_cast<int64_t>(grid) > units)
-        grid = static_cast<int>(units);
-    switch (bnmax) {
-    case 16:
-        return launch_group_cfg<GroupCfg<16, 12>>(gp, grid, cs);
-    case 32:
-        return launch_group_cfg<GroupCfg<32, 11>>(gp, grid, cs);
-    case 64:
-        return launch_group_cfg<GroupCfg<64, 9>>(gp, grid, cs);
-    default:
-        return launch_group_cfg<GroupCfg<128, 6>>(gp, grid, cs);
-    }
+    return launch_group(gp, bnmax, cs);
 }
 
 } // namespace pgf8
@@ -1562,21 +1655,32 @@ pgf8_status pgf8_fp8_linear_dynamic_group(const pgf8_fp8_layer *layers, int64_t 
     pgf8_linear_opts o = opts_or_default(opts);
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     int pdl = (o.flags & PGF8_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
-    // small layers: grouped, kGroupMaxLayers per launch pair, in call order
+    // small layers: grouped by token tile (16, 32, 64, 128 rows: each class
+    // gets the deepest weight ring its tile allows), kGroupMaxLayers per
+    // launch pair, in call order within a class
     const pgf8_fp8_layer *chunk[kGroupMaxLayers];
-    int n = 0;
-    for (int64_t i = 0; i <= count; ++i) {
-        if (i < count && layers[i].M <= PGF8_GROUP_MAX_M)
-            chunk[n++] = &layers[i];
-        if (n == kGroupMaxLayers || (i == count && n > 0)) {
-            pgf8_status st = group_chunk(chunk, n, group_workspace, pdl, cs);
-            if (st != PGF8_OK)
-                return st;
-            n = 0;
-            pdl = 1;
+    for (int bn = 16; bn <= 128; bn *= 2) {
+        int n = 0;
+        for (int64_t i = 0; i <= count; ++i) {
+            if (i < count && layers[i].M <= PGF8_GROUP_MAX_M && group_bn(layers[i].M) == bn)
+                chunk[n++] = &layers[i];
+            if (n == kGroupMaxLayers || (i == count && n > 0)) {
+                pgf8_status st = group_chunk(chunk, n, group_workspace, pdl, cs);
+                if (st != PGF8_OK)
+                    return st;
+                n = 0;
+                pdl = 1;
+            }
         }
     }
-    // large layers: one dynamic call each, overlapping the previous one
+    // large layers: one dynamic call each, overlapping the previous one.
+    // Their GEMMs run the pair kernel (FP8, M > 128, the dynamic workspace
+    // holds its stream-K slots, automatic choice), which signals its
+    // dependents only after its own dependency wait; the layers are
+    // independent, so from the second large layer on the quantisation does
+    // not wait for the previous GEMM and runs while it computes.
+    const bool auto_choice = o.path == PGF8_PATH_AUTO && o.tile_n == 0 && o.split_k == 0;
+    bool prev_pair = false;
     for (int64_t i = 0; i < count; ++i) {
         const pgf8_fp8_layer &l = layers[i];
         if (l.M <= PGF8_GROUP_MAX_M)
@@ -1584,11 +1688,102 @@ pgf8_status pgf8_fp8_linear_dynamic_group(const pgf8_fp8_layer *layers, int64_t 
         if (pdl)
             o.flags |= PGF8_FLAG_OVERLAP_PREVIOUS;
         pgf8_status st = linear_dynamic_impl(l.x, static_cast<pgf8_dtype>(l.xdt), l.M, l.K, l.ldx, l.wq, nullptr,
-                                             l.sw, l.N, l.y, l.workspace, l.workspace_bytes, &o, stream, kE4M3);
+                                             l.sw, l.N, l.y, l.workspace, l.workspace_bytes, &o, stream, kE4M3,
+                                             prev_pair);
         if (st != PGF8_OK)
             return st;
         pdl = 1;
+        prev_pair = auto_choice;
     }
+    return PGF8_OK;
+}
+
+size_t pgf8_fp8_linear_partial_workspace_size(int64_t M, int64_t, int64_t)
+{
+    if (M < 1)
+        return 0;
+    return M <= PGF8_GROUP_MAX_M ? group_workspace_bytes(group_bn(M)) : pair_sk_workspace_bytes(256);
+}
+
+pgf8_status pgf8_fp8_linear_partial(const uint8_t *aq, const float *sa, int64_t M, int64_t K, const uint8_t *wq,
+                                    const float *sw, int64_t N, float *y_f32, void *workspace, size_t workspace_bytes,
+                                    void *stream)
+{
+    pgf8_status st = check_dims(M, N, K);
+    if (st != PGF8_OK)
+        return st;
+    if (!aq || !sa || !wq || !sw || !y_f32 || !workspace)
+        return PGF8_ERR_INVALID_ARG;
+    if (workspace_bytes < pgf8_fp8_linear_partial_workspace_size(M, N, K))
+        return PGF8_ERR_INVALID_ARG;
+    if (!aligned16(aq) || !aligned16(wq) || !aligned16(y_f32) || !aligned4(sa) || !aligned4(sw) ||
+        !aligned16(workspace))
+        return PGF8_ERR_ALIGNMENT;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (M <= PGF8_GROUP_MAX_M) {
+        GroupParams gp;
+        std::memset(&gp, 0, sizeof(gp));
+        const int bn = group_bn(M);
+        GroupLayer &g = gp.L[0];
+        g.unit0 = 0;
+        g.M = static_cast<int>(M);
+        g.N = static_cast<int>(N);
+        g.K = static_cast<int>(K);
+        g.kblocks = static_cast<int>((K + 127) / 128);
+        g.bn = bn;
+        g.sa = sa;
+        g.sw = sw;
+        g.y = y_f32;
+        g.out_f32 = 1;
+        if (!make_map(&gp.tmW[0], wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(N),
+                      static_cast<uint64_t>(K), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&gp.tmX[0], aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(M),
+                      static_cast<uint64_t>(K), 128, static_cast<uint32_t>(bn), CU_TENSOR_MAP_SWIZZLE_128B))
+            return PGF8_ERR_UNSUPPORTED;
+        gp.nlayers = 1;
+        gp.prefetch_w = 0;
+        gp.units = static_cast<int64_t>((N + 127) / 128) * g.kblocks;
+        gp.flags = static_cast<unsigned *>(workspace);
+        gp.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + kGroupFlagBytes);
+        return launch_group(gp, bn, cs);
+    }
+    GemmLaunch L;
+    L.ws = workspace;
+    L.ws_bytes = workspace_bytes;
+    L.kind = kE4M3;
+    L.x = aq;
+    L.w = wq;
+    L.w2 = nullptr;
+    L.sa = sa;
+    L.sw = sw;
+    L.y = y_f32;
+    L.M = static_cast<int>(M);
+    L.N = static_cast<int>(N);
+    L.K = static_cast<int>(K);
+    L.pdl = 1;
+    L.prefetch_w = 0;
+    L.opts = opts_or_default(nullptr);
+    L.stream = cs;
+    L.out_f32 = 1;
+    return launch_pair_bn<kE4M3>(L, 256);
+}
+
+pgf8_status pgf8_round_bf16(const float *x, int64_t n, void *y_bf16, void *stream)
+{
+    if (n < 0 || (n > 0 && (!x || !y_bf16)))
+        return PGF8_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y_bf16) || n % 8 != 0)
+        return PGF8_ERR_ALIGNMENT;
+    if (n == 0)
+        return PGF8_OK;
+    const int64_t n8 = n / 8;
+    const int64_t want = (n8 + 255) / 256;
+    const unsigned grid = static_cast<unsigned>(want < 148 * 16 ? want : 148 * 16);
+    round_bf16_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(reinterpret_cast<const float4 *>(x), n8,
+                                                                          static_cast<uint4 *>(y_bf16));
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return cuda_fail(e);
     return PGF8_OK;
 }
 

@@ -59,6 +59,28 @@ template <> struct Vec16<__half> {
     }
 };
 
+// Maximum over the CTA's THREADS threads (red: THREADS / 32 floats).
+template <int THREADS> __device__ __forceinline__ float block_max_n(float v, float *red)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0)
+        red[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        v = lane < (THREADS / 32) ? red[lane] : 0.0f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+        if (lane == 0)
+            red[0] = v;
+    }
+    __syncthreads();
+    return red[0];
+}
+
 __device__ __forceinline__ float block_max(float v, float *red)
 {
 #pragma unroll
@@ -78,6 +100,43 @@ __device__ __forceinline__ float block_max(float v, float *red)
     }
     __syncthreads();
     return red[0];
+}
+
+// Modes of the row quantisers.  0 dynamic: *srow = fl32(amax / 448), 1 for
+// an all-zero row ("7B on an RTX 4060 with FP8" §2.2 per-token scale, §6.1
+// the 448 limit); 1 static: the scale is read from *srow; 2 given amax:
+// *srow holds the row's amax on input (taken over the whole row, e.g.
+// reduced over tensor-parallel ranks that each hold a slice of it) and its
+// scale, computed as in mode 0, on output; 3 amax only: *srow = amax, no
+// codes are written.
+enum : int { kQuantDynamic = 0, kQuantStatic = 1, kQuantFromAmax = 2, kQuantAmaxOnly = 3 };
+
+// The row's scale s from this thread's partial amax (all THREADS threads
+// call it).  Returns false when the row is done (mode 3).
+template <int THREADS>
+__device__ __forceinline__ bool row_scale(float amax, float *srow, int mode, float *red, float &s)
+{
+    if (mode == kQuantStatic) {
+        s = *srow;
+        return true;
+    }
+    if (mode == kQuantFromAmax) {
+        amax = *srow;
+        __syncthreads();   // every thread has read the amax before it is replaced by the scale
+    } else {
+        amax = block_max_n<THREADS>(amax, red);
+        if (mode == kQuantAmaxOnly) {
+            if (threadIdx.x == 0)
+                *srow = amax;
+            return false;
+        }
+    }
+    s = __fdiv_rn(amax, 448.0f);
+    if (s == 0.0f)
+        s = 1.0f;
+    if (threadIdx.x == 0)
+        *srow = s;
+    return true;
 }
 
 // x / s correctly rounded (binary32, nearest-even) for many x and one
@@ -206,9 +265,8 @@ __global__ void __launch_bounds__(256) selftest_row_division_kernel(const float 
 constexpr int kRegChunks = 4;
 
 // One row quantised by one CTA of kQuantThreads threads (every thread of
-// the CTA calls it).  cols % 16 == 0; the row 16-byte aligned.  mode 0:
-// dynamic (*srow = fl32(amax / 448), 1 for an all-zero row); mode 1: the
-// scale is read from *srow.
+// the CTA calls it).  cols % 16 == 0; the row 16-byte aligned.  mode: see
+// row_scale.
 template <typename T>
 __device__ __forceinline__ void quantize_one_row(const T *__restrict__ xr, int64_t cols, uint8_t *__restrict__ qr,
                                                  float *srow, int mode, float *red)
@@ -229,16 +287,8 @@ __device__ __forceinline__ void quantize_one_row(const T *__restrict__ xr, int64
             }
         }
         float s;
-        if (mode == 0) {
-            amax = block_max(amax, red);
-            s = __fdiv_rn(amax, 448.0f);
-            if (s == 0.0f)
-                s = 1.0f;
-            if (threadIdx.x == 0)
-                *srow = s;
-        } else {
-            s = *srow;
-        }
+        if (!row_scale<kQuantThreads>(amax, srow, mode, red, s))
+            return;
         const RowDivisor d(s);
 #pragma unroll
         for (int u = 0; u < kRegChunks; ++u) {
@@ -249,9 +299,8 @@ __device__ __forceinline__ void quantize_one_row(const T *__restrict__ xr, int64
         return;
     }
 
-    float s;
-    if (mode == 0) {
-        float amax = 0.0f;
+    float amax = 0.0f;
+    if (mode == kQuantDynamic || mode == kQuantAmaxOnly) {
         for (int64_t c = threadIdx.x; c < nchunk; c += kQuantThreads) {
             Vec16<T> v;
             v.load(xr + c * 16);
@@ -259,15 +308,10 @@ __device__ __forceinline__ void quantize_one_row(const T *__restrict__ xr, int64
             for (int i = 0; i < 16; ++i)
                 amax = fmaxf(amax, fabsf(v.v[i]));
         }
-        amax = block_max(amax, red);
-        s = __fdiv_rn(amax, 448.0f);
-        if (s == 0.0f)
-            s = 1.0f;
-        if (threadIdx.x == 0)
-            *srow = s;
-    } else {
-        s = *srow;
     }
+    float s;
+    if (!row_scale<kQuantThreads>(amax, srow, mode, red, s))
+        return;
     const RowDivisor d(s);
     for (int64_t c = threadIdx.x; c < nchunk; c += kQuantThreads) {
         Vec16<T> v;
@@ -277,26 +321,81 @@ __device__ __forceinline__ void quantize_one_row(const T *__restrict__ xr, int64
 }
 
 // One CTA per row.  cols % 16 == 0; x rows 16-byte aligned.
-// trigger_early: let a dependent kernel launched with programmatic stream
-// serialization be scheduled at once (used only when that dependent is the
-// library's own GEMM, which reads q/scales after this grid completes).
+// flags: kQuantTriggerEarly lets a dependent launched with programmatic
+// serialization start at once (used when that dependent is the library's
+// own GEMM, which reads q / scales only after this grid completes);
+// kQuantNoWait skips the wait for the previous kernel (used only when that
+// kernel is independent of this one's inputs and signals its dependents
+// after its own wait, so everything before it has completed).
+constexpr int kQuantTriggerEarly = 1;
+constexpr int kQuantNoWait = 2;
+
 template <typename T>
 __global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(const T *__restrict__ x, int64_t rows,
                                                                       int64_t cols, int64_t ldx,
                                                                       uint8_t *__restrict__ q,
                                                                       float *__restrict__ scales, int mode,
-                                                                      int trigger_early)
+                                                                      int flags)
 {
     __shared__ float red[kQuantThreads / 32];
-    if (trigger_early)
+    if (flags & kQuantTriggerEarly)
         grid_launch_dependents();
     // When launched with programmatic serialization, the previous kernel in
     // the stream may still run: nothing is read or written before it ends.
-    grid_dependency_wait();
+    if (!(flags & kQuantNoWait))
+        grid_dependency_wait();
     const int64_t row = blockIdx.x;
     if (row >= rows)
         return;
     quantize_one_row<T>(x + row * ldx, cols, q + row * cols, scales + row, mode, red);
+}
+
+// The same row quantisation with the row held in registers by a CTA of
+// THREADS threads, CH 16-element chunks per thread (rows of at most
+// CH * THREADS * 16 elements): the launch picks the smallest CH (and 512
+// threads for the longest rows), so the CTA holds no more registers than
+// its row needs and more rows are in flight per SM.  Same arithmetic as
+// quantize_one_row, element by element.
+template <typename T, int CH, int THREADS>
+__global__ void __launch_bounds__(THREADS) quantize_rows_held_kernel(const T *__restrict__ x, int64_t rows,
+                                                                     int64_t cols, int64_t ldx,
+                                                                     uint8_t *__restrict__ q,
+                                                                     float *__restrict__ scales, int mode,
+                                                                     int flags)
+{
+    __shared__ float red[THREADS / 32];
+    if (flags & kQuantTriggerEarly)
+        grid_launch_dependents();
+    if (!(flags & kQuantNoWait))
+        grid_dependency_wait();
+    const int64_t row = blockIdx.x;
+    if (row >= rows)
+        return;
+    const T *xr = x + row * ldx;
+    uint8_t *qr = q + row * cols;
+    const int64_t nchunk = cols / 16;
+    Vec16<T> v[CH];
+    float amax = 0.0f;
+#pragma unroll
+    for (int u = 0; u < CH; ++u) {
+        const int64_t c = threadIdx.x + static_cast<int64_t>(u) * THREADS;
+        if (c < nchunk) {
+            v[u].load(xr + c * 16);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                amax = fmaxf(amax, fabsf(v[u].v[i]));
+        }
+    }
+    float s;
+    if (!row_scale<THREADS>(amax, scales + row, mode, red, s))
+        return;
+    const RowDivisor d(s);
+#pragma unroll
+    for (int u = 0; u < CH; ++u) {
+        const int64_t c = threadIdx.x + static_cast<int64_t>(u) * THREADS;
+        if (c < nchunk)
+            *reinterpret_cast<uint4 *>(qr + c * 16) = encode16(v[u].v, d);
+    }
 }
 
 // Dynamic per-token quantisation of the activations of several independent
@@ -739,6 +838,21 @@ __global__ void __launch_bounds__(kQuantThreads) silu_mul_quantize_kernel(const 
 }
 
 // NestedFP split: 8 FP16 bit patterns per thread per step (16 bytes in, 8 + 8 out).
+// y = bf16_rn(x), 8 elements per step (the final rounding of a
+// tensor-parallel layer's f32 sum).
+__global__ void __launch_bounds__(256) round_bf16_kernel(const float4 *__restrict__ x, int64_t n8,
+                                                         uint4 *__restrict__ y)
+{
+    grid_dependency_wait();
+    for (int64_t i = blockIdx.x * 256ll + threadIdx.x; i < n8; i += static_cast<int64_t>(gridDim.x) * 256) {
+        const float4 a = x[2 * i], b = x[2 * i + 1];
+        const __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y), p1 = __floats2bfloat162_rn(a.z, a.w);
+        const __nv_bfloat162 p2 = __floats2bfloat162_rn(b.x, b.y), p3 = __floats2bfloat162_rn(b.z, b.w);
+        y[i] = make_uint4(*reinterpret_cast<const uint32_t *>(&p0), *reinterpret_cast<const uint32_t *>(&p1),
+                          *reinterpret_cast<const uint32_t *>(&p2), *reinterpret_cast<const uint32_t *>(&p3));
+    }
+}
+
 __global__ void __launch_bounds__(256) nestedfp_split_kernel(const uint4 *__restrict__ w, int64_t n8,
                                                              uint2 *__restrict__ hi, uint2 *__restrict__ lo)
 {

@@ -179,6 +179,27 @@ def test_dynamic_group_checks_layers_aliasing_and_workspace_first():
     assert f(None, 0, None, 0, None, None) == pg.OK
 
 
+def test_tensor_parallel_blocks_argument_checks():
+    lib = pg.lib
+    assert lib.pgf8_fp8_row_amax(A16, pg.F32, 4, 512, 512, A16 + 2, None) == pg.ERR_ALIGNMENT
+    assert lib.pgf8_fp8_row_amax(A16, pg.F32, 4, 520, 520, B16, None) == pg.ERR_ALIGNMENT     # cols % 16
+    assert lib.pgf8_fp8_row_amax(A16, pg.F32, 4, 512, 256, B16, None) == pg.ERR_INVALID_ARG   # ldx < cols
+    assert lib.pgf8_fp8_row_amax(A16, pg.F32, 0, 512, 512, None, None) == pg.OK
+    assert lib.pgf8_fp8_quantize_rows_amax(A16, pg.F32, 4, 512, 512, B16 + 8, C16, None) == pg.ERR_ALIGNMENT
+    assert lib.pgf8_fp8_quantize_rows_amax(None, pg.F32, 4, 512, 512, B16, C16, None) == pg.ERR_INVALID_ARG
+    ws = lib.pgf8_fp8_linear_partial_workspace_size(8, 512, 512)
+    assert ws == lib.pgf8_fp8_linear_group_workspace_size(8)
+    assert lib.pgf8_fp8_linear_partial_workspace_size(300, 512, 512) > 16 << 20
+    f = lib.pgf8_fp8_linear_partial
+    assert f(A16, B16, 8, 512, C16, D16, 512, A16, B16, ws - 16, None) == pg.ERR_INVALID_ARG
+    assert f(A16, B16, 8, 512, C16, D16, 512, A16, None, ws, None) == pg.ERR_INVALID_ARG
+    assert f(A16, B16, 8, 512, C16, D16, 512, A16 + 4, B16, ws, None) == pg.ERR_ALIGNMENT
+    assert f(A16, B16, 8, 520, C16, D16, 512, A16, B16, ws, None) == pg.ERR_ALIGNMENT
+    assert lib.pgf8_round_bf16(A16, 12, B16, None) == pg.ERR_ALIGNMENT
+    assert lib.pgf8_round_bf16(None, 16, B16, None) == pg.ERR_INVALID_ARG
+    assert lib.pgf8_round_bf16(None, 0, None, None) == pg.OK
+
+
 def test_selftest_row_division_argument_checks():
     f = pg.lib.pgf8_selftest_row_division
     buf = (ctypes.c_uint64 * 4)()
@@ -416,7 +437,7 @@ def test_binding_constants_match_the_header():
     names = ["OK", "ERR_INVALID_ARG", "ERR_ALIGNMENT", "ERR_UNSUPPORTED", "ERR_CUDA", "ERR_TIMEOUT", "ERR_TOO_LARGE",
              "F32", "F16", "BF16", "SCALE_DYNAMIC", "SCALE_STATIC", "NESTED_FP16", "NESTED_FP8", "PATH_AUTO",
              "PATH_SKINNY", "PATH_TILED", "PATH_STREAMK", "PATH_TILED_PAIR", "FLAG_OVERLAP_PREVIOUS",
-             "FLAG_FUSED_QUANT", "FLAG_ATTN_MMA"]
+             "FLAG_FUSED_QUANT", "FLAG_ATTN_MMA", "FLAG_STREAM_K_TAIL"]
     for n in names:
         assert getattr(pg, n) == values["PGF8_" + n], n
     flags = [values[k] for k in values if k.startswith("PGF8_FLAG_")]

@@ -120,3 +120,26 @@ def test_group_decode7b_full_size_sampled():
     for i, (layer, (x, w)) in enumerate(zip(layers, host)):
         ns = np.sort(rng.choice(w.shape[0], 384, replace=False))
         _check_layer(i, layer, x, w, ns)
+
+
+def test_group_several_large_layers_after_a_producer():
+    """Several layers past the grouped kernel: from the second one on, each
+    layer's quantisation runs while the previous layer's GEMM computes.  The
+    activations are written by a device kernel right before the call (the
+    call's first launch overlaps it), and the last layer's activations are
+    the ones written last: every layer must still see its final inputs."""
+    shapes = [(4, 1024, 528), (200, 1024, 528), (260, 528, 1040), (300, 1008, 272), (33, 400, 144)]
+    layers, host = _make_group(shapes, 23)
+    srcs = [torch.from_numpy(x).to(DEV) for (x, _) in host]
+    for l in layers:
+        l[0].zero_()
+    grp = pg.LayerGroup(layers)
+    stream = torch.cuda.current_stream()
+    for _ in range(2):
+        for l, s in zip(layers, srcs):
+            l[0].copy_(s)                       # the producer kernels, in stream order
+        grp.run(flags=pg.FLAG_OVERLAP_PREVIOUS, stream=stream)
+    torch.cuda.synchronize()
+    assert pg.device_status() == pg.OK
+    for i, (layer, (x, w)) in enumerate(zip(layers, host)):
+        _check_layer(i, layer, x, w)

@@ -262,3 +262,38 @@ def test_dynamic_many_matches_single_calls():
         ref = oracle.fp8_linear(aq, sa, wq0, sw0)
         bound = linear_bound(ref, x.shape[1], fp8_row_max(aq, sa), fp8_row_max(wq0, sw0))
         assert_within(y.float().cpu().numpy()[:8, :64], ref, bound, f"many {x.shape}")
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 528, 400), (1000, 1040, 2000), (512, 10240, 1024), (2048, 4096, 4096),
+                                   (4096, 12288, 256), (256, 8192, 8192)])
+def test_pair_kernel_stream_k_region(M, N, K):
+    """The pair kernel with its stream-K region (the last full round and the
+    ragged tail of tiles split in k-block ranges over every pair, partial
+    tiles summed through the workspace): within the bound against the oracle
+    on sampled rows and columns, the same bits on a repeated call, the flag
+    words left zero; the plain round-robin form (no room for the partials)
+    within the bound as well."""
+    g = np.random.default_rng(M + 3 * N + 5 * K)
+    x = synthetic.activations("student_t3", M, K, g)
+    w = synthetic.weights_f16(N, K, 0.01, g)
+    aq, sa = oracle.quantize_rows(x)
+    wq, sw = oracle.quantize_rows(w)
+    rng = np.random.default_rng(2)
+    big = M * N * K > 2e9
+    ms = np.sort(rng.choice(M, 32, replace=False)) if big else np.arange(M)
+    ns = np.sort(rng.choice(N, 384, replace=False)) if big else np.arange(N)
+    ref = oracle.fp8_linear(aq[ms], sa[ms], wq[ns], sw[ns])
+    bound = linear_bound(ref, K, fp8_row_max(aq[ms], sa[ms]), fp8_row_max(wq[ns], sw[ns]))
+    ws = torch.zeros(pg.lib.pgf8_fp8_linear_workspace_size(M, N, K), dtype=torch.uint8, device=DEV)
+    assert ws.numel() > 16 << 20
+    A, SA, W, SW = _to(aq), _to(sa), _to(wq), _to(sw)
+    y1 = pg.fp8_linear(A, SA, W, SW, workspace=ws, path=pg.PATH_TILED_PAIR, flags=pg.FLAG_STREAM_K_TAIL)
+    y2 = pg.fp8_linear(A, SA, W, SW, workspace=ws, path=pg.PATH_TILED_PAIR, flags=pg.FLAG_STREAM_K_TAIL)
+    y_rr = pg.fp8_linear(A, SA, W, SW, workspace=torch.zeros(1024, dtype=torch.uint8, device=DEV),
+                         path=pg.PATH_TILED_PAIR)
+    torch.cuda.synchronize()
+    assert pg.device_status() == pg.OK
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    assert not ws[:1024].any(), "flag words not cleared"
+    for name, y in (("stream-K", y1), ("round-robin", y_rr)):
+        assert_within(y.float().cpu().numpy()[np.ix_(ms, ns)], ref, bound, f"pair {name} M{M} N{N} K{K}")
