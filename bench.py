@@ -12,8 +12,8 @@ O 8192->8192, gate+up 8192->57344, down 28672->8192) at M = 1, 2, 4, ...,
 4096 tokens: 52 independent layers, 11.1 GB of FP8 weights streamed per step
 (the same weights for every M, 855 MB per M: more than the 126 MB L2, so no
 weight is L2-resident when it is re-read).  One step is one
-pgf8_fp8_linear_dynamic_group call: the M <= 128 layers stream their weights
-through one grouped kernel, the larger ones run the tiled tensor-core GEMMs.
+pgf8_fp8_linear_dynamic_group call: the M <= 256 layers stream their weights
+through the grouped kernel, the larger ones run the tiled tensor-core GEMMs.
 decode7b, prefill7b and nested7b are timed as secondary steps in the same run.
 
 Timing: the K timed steps are replayed from a CUDA graph (captured from the
@@ -317,7 +317,7 @@ def _wkey(L):
     return (L.shape_idx, L.copy, L.kind != "fp8")
 
 
-GROUP_MAX_M = 128   # the library's grouped weight-streaming kernel takes layers up to this many tokens
+GROUP_MAX_M = 256   # the library's grouped weight-streaming kernel takes layers up to this many tokens
 
 
 class StepRunner:
@@ -329,9 +329,10 @@ class StepRunner:
     producers) chains one call per layer with PGF8_FLAG_OVERLAP_PREVIOUS.
 
     The bracketed step (for the roofline) runs the same launches with an
-    event between consecutive launch groups: the grouped kernel of each
-    token-tile class (M <= 16, 32, 64, 128), then the quantisation and the
-    GEMM of every larger layer; its intervals are scaled to the timed step."""
+    event between consecutive launch groups: the grouped kernel on the
+    M <= 128 layers and on the 128 < M <= 256 layers, then the quantisation
+    and the GEMM of every larger layer; its intervals are scaled to the
+    timed step."""
 
     def __init__(self, pg, torch, dev, wl, args, stream):
         self.pg, self.torch, self.dev, self.wl, self.args, self.stream = pg, torch, dev, wl, args, stream
@@ -345,11 +346,13 @@ class StepRunner:
         if self.grouped:
             ent = lambda i: (wl["acts"][i], *wl["weights"][_wkey(layers[i])], wl["outs"][i], wl["qbufs"][i])  # noqa: E731
             self.group = pg.LayerGroup([ent(i) for i in range(len(layers))])
-            # the library's launches for a group: one grouped kernel per
-            # token-tile class (M <= 16, 32, 64, 128), then the larger layers
-            self.classes = [[i for i, L in enumerate(layers) if lo < L.M <= hi]
-                            for lo, hi in ((0, 16), (16, 32), (32, 64), (64, GROUP_MAX_M))]
-            self.classes = [c for c in self.classes if c]
+            # the library's launches for a group: the grouped kernel on the
+            # M <= 128 layers and on the 128 < M <= 256 layers (32 per
+            # launch), then each larger layer
+            self.classes = []
+            for lo, hi in ((0, 128), (128, GROUP_MAX_M)):
+                idx = [i for i, L in enumerate(layers) if lo < L.M <= hi]
+                self.classes += [idx[j:j + 32] for j in range(0, len(idx), 32)]
             self.large = [i for i, L in enumerate(layers) if L.M > GROUP_MAX_M]
             self.sub = [pg.LayerGroup([ent(i) for i in idx]) for idx in self.classes]
         self.per_tensor = {}
@@ -460,9 +463,11 @@ def quant_bytes(L):
 def analyse_segments(layers, marks, ms_step, peaks, fp8_peak):
     """Per-segment durations of the bracketed step, scaled so that they sum
     to the timed step (a kernel's share of the step times the step), the
-    dominant kernel's roofline and the regime checks of the layer's targets:
-    decode (M <= 16) >= 80 % of HBM, M 17..256 >= 75 % of HBM (weight
-    streaming), prefill (M >= 512) >= 60 % of the FP8 tensor peak."""
+    dominant kernel's roofline and the regime checks of the layer's targets,
+    over the segments whose layers all fall in the regime: decode (M <= 16)
+    >= 80 % of HBM; weight streaming (M <= 256, the grouped kernel and the
+    M = 256 layers) >= 75 % of HBM; prefill (M >= 512) >= 60 % of the FP8
+    tensor peak."""
     segs = []
     for (seg, e0), (_, e1) in zip(marks[:-1], marks[1:]):
         kind, idx = seg
@@ -548,7 +553,7 @@ def analyse_segments(layers, marks, ms_step, peaks, fp8_peak):
 
     regimes = {}
     for key, pred, what, target in (("decode_m_le_16", lambda m: m <= 16, "hbm", 0.80),
-                                    ("stream_m_17_256", lambda m: 16 < m <= 256, "hbm", 0.75),
+                                    ("weight_streaming_m_le_256", lambda m: m <= 256, "hbm", 0.75),
                                     ("prefill_m_ge_512", lambda m: m >= 512, "tensor", 0.60)):
         r = regime(pred, what)
         if r is not None:
@@ -707,6 +712,11 @@ def run_ours(args, rank, world, local_rank):
                 "value": round(v, 2), "unit": "GB/s" if mb else "TFLOP/s", "ms_per_step": round(r2["ms_step"], 5),
                 "steps": steps2, "grouped": r2["runner"].grouped, "roofline": r2["roof"], "regimes": r2["regimes"],
                 "segments": r2["segments"]}
+            if sec == "decode7b" and "decode_m_le_16" in r2["regimes"]:
+                # the decode regime as its own step (the 70B step streams its
+                # M <= 16 layers together with the M <= 128 ones)
+                result["secondary"]["regimes"]["decode_m_le_16"] = dict(r2["regimes"]["decode_m_le_16"],
+                                                                        measured_on="decode7b step")
             del wl2, r2
             torch.cuda.empty_cache()
     return result
@@ -714,12 +724,20 @@ def run_ours(args, rank, world, local_rank):
 
 def run_e2e(pg, torch, dev, wl, args, world, wbytes, flops, memory_bound):
     """The metric end to end through the public API with host buffers: every
-    step copies all of its activations from one pinned host buffer to the
+    step copies all of its activations from a pinned host buffer to the
     device, runs the step (one pgf8_fp8_linear_dynamic_group call for the FP8
-    workloads, one call per layer otherwise) and copies all outputs back to
-    one pinned host buffer; the copies are inside the timed region."""
-    layers, weights, acts_host, outs = wl["layers"], wl["weights"], wl["acts_host"], wl["outs"]
-    stream = torch.cuda.Stream(device=dev)
+    workloads, one call per layer otherwise) and copies all of its outputs
+    back to a pinned host buffer; the copies are inside the timed region.
+
+    Steps are pipelined as a server runs them: two device buffer sets, the
+    host-to-device copies on one stream, the kernels on a second and the
+    device-to-host copies on a third, so step k's outputs go back to the host
+    while step k+1's inputs come in and step k+1 computes (PCIe carries both
+    directions at once).  Events order the buffers: a step's inputs are not
+    overwritten before the step that reads them has computed, its outputs not
+    before they have been copied out."""
+    layers, acts_host, outs = wl["layers"], wl["acts_host"], wl["outs"]
+    s_in, s_comp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
 
     def packed(tensors, device):
         offs, total = [], 0
@@ -732,41 +750,58 @@ def run_e2e(pg, torch, dev, wl, args, world, wbytes, flops, memory_bound):
     x_host, x_host_views = packed(acts_host, "cpu")
     for v, a in zip(x_host_views, acts_host):
         v.copy_(a)
-    x_dev, x_views = packed(acts_host, dev)
-    x_dev.copy_(x_host)          # calibrated per-tensor scales (--scaling static) read the inputs at set-up
-    torch.cuda.synchronize()
-    y_dev, y_views = packed(outs, dev)
-    y_host, _ = packed(outs, "cpu")
     ws = [torch.zeros_like(q) for q in wl["qbufs"]]
-    wl_e2e = dict(wl, acts=x_views, outs=y_views, qbufs=ws)
-    runner = StepRunner(pg, torch, dev, wl_e2e, args, stream)
+    bufs = []
+    for _ in range(2):
+        x_dev, x_views = packed(acts_host, dev)
+        x_dev.copy_(x_host)      # calibrated per-tensor scales (--scaling static) read the inputs at set-up
+        y_dev, y_views = packed(outs, dev)
+        y_host, _ = packed(outs, "cpu")
+        torch.cuda.synchronize()
+        runner = StepRunner(pg, torch, dev, dict(wl, acts=x_views, outs=y_views, qbufs=ws), args, s_comp)
+        ev = {k: torch.cuda.Event() for k in ("in", "comp", "out")}
+        bufs.append(dict(x_dev=x_dev, y_dev=y_dev, y_host=y_host, runner=runner, ev=ev, used=False))
 
-    def step():
-        with torch.cuda.stream(stream):
-            x_dev.copy_(x_host, non_blocking=True)
-            runner.step()
-            y_host.copy_(y_dev, non_blocking=True)
+    def step(k):
+        b = bufs[k % 2]
+        if b["used"]:
+            s_in.wait_event(b["ev"]["comp"])       # the previous step on these buffers has read its inputs
+        with torch.cuda.stream(s_in):
+            b["x_dev"].copy_(x_host, non_blocking=True)
+            b["ev"]["in"].record(s_in)
+        s_comp.wait_event(b["ev"]["in"])
+        if b["used"]:
+            s_comp.wait_event(b["ev"]["out"])      # ... and its outputs have been copied out
+        with torch.cuda.stream(s_comp):
+            b["runner"].step()
+            b["ev"]["comp"].record(s_comp)
+        s_out.wait_event(b["ev"]["comp"])
+        with torch.cuda.stream(s_out):
+            b["y_host"].copy_(b["y_dev"], non_blocking=True)
+            b["ev"]["out"].record(s_out)
+        b["used"] = True
 
     steps = max(3, min(args.steps, 100))
-    for _ in range(3):
-        step()
-    stream.synchronize()
+    for k in range(4):
+        step(k)
+    torch.cuda.synchronize()
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(steps):
-        step()
-    t1.record(stream)
-    stream.synchronize()
+    t0.record(s_in)
+    for k in range(steps):
+        step(k)
+    t1.record(s_out)
+    torch.cuda.synchronize()
     ms = max_over_ranks(t0.elapsed_time(t1) / steps, world, dev)
     v = job_throughput(wbytes / 1e9 if memory_bound else flops / 1e12, world, ms * 1e-3)
     return {"value": round(v, 2), "unit": "GB/s" if memory_bound else "TFLOP/s",
-            "h2d_bytes_per_step": int(x_host.numel()), "d2h_bytes_per_step": int(y_host.numel()), "steps": steps,
-            "ms_per_step": round(ms, 5),
-            "entry_point": ("pgf8_fp8_linear_dynamic_group" if runner.grouped else
+            "h2d_bytes_per_step": int(x_host.numel()), "d2h_bytes_per_step": int(bufs[0]["y_host"].numel()),
+            "steps": steps, "ms_per_step": round(ms, 5),
+            "pipeline": "two device buffer sets; H2D, kernels and D2H on three streams ordered by events",
+            "entry_point": ("pgf8_fp8_linear_dynamic_group" if bufs[0]["runner"].grouped else
                             "one C-ABI call per layer (pgf8_fp8_linear_dynamic / pgf8_nestedfp_linear / the "
                             "scaling and producer variants + pgf8_fp8_linear)")}
 

@@ -457,11 +457,11 @@ size_t pgf8_fp8_linear_dynamic_scales_offset(int64_t M, int64_t K);
  * are bit-identical to that call's, its outputs are within the same bound
  * (the f32 summation order differs).
  *
- * Layers with M <= 128 are quantised by one launch and then streamed by one
+ * Layers with M <= 256 are quantised by one launch and then streamed by one
  * persistent grouped kernel (one CTA per SM, each SM streaming an equal
- * share of all those layers' weights), one launch pair per token-tile class
- * (M <= 16, <= 32, <= 64, <= 128) and per 32 layers of a class; larger
- * layers run one dynamic call each afterwards.  Decode-sized layers
+ * share of all those layers' weights, up to 32 layers per launch pair; the
+ * layers with 128 < M <= 256 in a launch pair of their own); larger layers
+ * run one dynamic call each afterwards.  Decode-sized layers
  * are bound by their weight stream ("7B token speed on consumer GPUs" §1),
  * and one stream for the whole group pays the start and the end of a
  * launch once instead of once per layer.
@@ -470,7 +470,7 @@ size_t pgf8_fp8_linear_dynamic_scales_offset(int64_t M, int64_t K);
  * layers) bytes of device memory, 16-byte aligned, zero-filled once before
  * its first use; every completed call leaves its flag words zero again, so
  * it is reused without clearing.  Calls that use one group workspace must
- * not overlap on the GPU.  May be null when no layer has M <= 128.
+ * not overlap on the GPU.  May be null when no layer has M <= 256.
  * Errors: any layer's own argument errors (nothing is enqueued);
  * PGF8_ERR_INVALID_ARG when an output or workspace of one layer overlaps
  * an input, output or workspace of another (or its own input), or the

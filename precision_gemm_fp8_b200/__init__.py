@@ -614,7 +614,7 @@ class LayerSequence:
 class LayerGroup(LayerSequence):
     """A fixed group of INDEPENDENT dynamic FP8 layers (no layer reads another
     layer's output), run by one call of pgf8_fp8_linear_dynamic_group: the
-    layers with M <= 128 stream their weights through one grouped kernel.
+    layers with M <= 256 stream their weights through the grouped kernel.
     Entries as LayerSequence; the group workspace is allocated (zero-filled)
     here unless given."""
 

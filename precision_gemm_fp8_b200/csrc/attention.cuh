@@ -463,7 +463,22 @@ __global__ void __launch_bounds__(kAttnThreads) attn_decode_mma_kernel(const Att
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t4 = lane & 3;
 
-    // Q^T operand of every k-step: head g (zero for the padding heads)
+    // Q^T operand of every k-step: head g (zero for the padding heads).  The
+    // operand is binary16, so a head whose largest |q| reaches 2^14 is
+    // scaled by 2^-e first (exact; q stays below 2^15 < 65504) and its scores
+    // by 2^e after the product.
+    float qmax = 0.0f;
+    if (g < nh) {
+#pragma unroll
+        for (int j = 0; j < KSTEPS; ++j)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                qmax = fmaxf(qmax, fabsf(load_elem(a.q, s * a.ldq + (h0 + g) * D + KSEG * t4 + 4 * j + i, a.qdt)));
+    }
+    qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, 1));
+    qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, 2));   // the 4 lanes of head g
+    const int qexp = qmax >= 16384.0f && qmax <= 3.4e38f ? ilogbf(qmax) - 14 : 0;
+    const float qpre = ldexpf(1.0f, -qexp);
     uint32_t qb[KSTEPS][2];
 #pragma unroll
     for (int j = 0; j < KSTEPS; ++j) {
@@ -473,8 +488,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_decode_mma_kernel(const Att
             float x0 = 0.0f, x1 = 0.0f;
             if (g < nh) {
                 const int64_t base = s * a.ldq + (h0 + g) * D + d;
-                x0 = load_elem(a.q, base, a.qdt);
-                x1 = load_elem(a.q, base + 1, a.qdt);
+                x0 = load_elem(a.q, base, a.qdt) * qpre;
+                x1 = load_elem(a.q, base + 1, a.qdt) * qpre;
             }
             qb[j][e] = f32x2_to_h2bits(x0, x1);
         }
@@ -488,7 +503,10 @@ __global__ void __launch_bounds__(kAttnThreads) attn_decode_mma_kernel(const Att
     }
     const int64_t t_begin = static_cast<int64_t>(sp) * a.chunk;
     const int64_t t_end = t_begin + a.chunk < ctx ? t_begin + a.chunk : ctx;
-    const float scale = a.sk[hk] * a.qscale;   // base-2 units
+    // base-2 units; the scores of heads 2 t4 and 2 t4 + 1 undo their pre-scale
+    const float scale = a.sk[hk] * a.qscale;
+    const float hscale[2] = {scale * ldexpf(1.0f, __shfl_sync(0xffffffffu, qexp, 8 * t4)),
+                             scale * ldexpf(1.0f, __shfl_sync(0xffffffffu, qexp, 8 * t4 + 4))};
 
     float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.0f, 0.0f};   // heads 2 t4, 2 t4 + 1
     float o[DB][4];
@@ -540,8 +558,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_decode_mma_kernel(const Att
         float alpha[2];
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-            const float s0 = v0 ? c[hh] * scale : -INFINITY;
-            const float s1 = v1 ? c[2 + hh] * scale : -INFINITY;
+            const float s0 = v0 ? c[hh] * hscale[hh] : -INFINITY;
+            const float s1 = v1 ? c[2 + hh] * hscale[hh] : -INFINITY;
             float mx = fmaxf(s0, s1);
 #pragma unroll
             for (int off = 4; off < 32; off <<= 1)

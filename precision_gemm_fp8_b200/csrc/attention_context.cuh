@@ -340,8 +340,8 @@ __global__ void __launch_bounds__(192, 1) attn_context_kernel(const __grid_const
                 const int64_t blk = p.tables[s * p.table_stride + key / p.B];
                 if (blk >= 0 && blk < p.num_blocks)
                     piece_ok |= 1u << i;
-                else if (et == 0 && h == 0 && p.errors)
-                    atomicAdd(p.errors, 1);
+                else if (et == 0 && h == 0 && qt == (q_len - 1) / 128 && p.errors)
+                    atomicAdd(p.errors, 1);   // once: the sequence's last query tile visits every key tile
             }
             bool w = wait_bounded(&ctl->s_full[b], static_cast<uint32_t>(k) & 1u, abort_flag);
             w = __all_sync(0xffffffffu, w);

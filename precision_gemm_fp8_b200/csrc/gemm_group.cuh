@@ -55,7 +55,7 @@ template <int BNMAX_, int STAGES_> struct GroupCfg {
     static constexpr int kRingBytes = STAGES * kStage;
     static constexpr int kBarOffset = kRingBytes;
     static constexpr int kSmemBytes = kRingBytes + 1024 + 1024;
-    static_assert(BNMAX == 16 || BNMAX == 32 || BNMAX == 64 || BNMAX == 128, "token tile");
+    static_assert(BNMAX == 16 || BNMAX == 32 || BNMAX == 64 || BNMAX == 128 || BNMAX == 256, "token tile");
     static_assert(STAGES <= 16 && kStage % 1024 == 0, "ring");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };

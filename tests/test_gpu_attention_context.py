@@ -132,7 +132,7 @@ def test_bad_entries_and_lengths_are_counted():
     c["tables"][1, 2] = 10 ** 6                    # positions 32..47 of sequence 1: out of range
     errors = torch.zeros(1, dtype=torch.int32, device=DEV)
     out, qc, qs = _run(c, errors=errors)
-    assert errors.item() >= 1
+    assert errors.item() == 1                      # the one bad entry, counted once
     assert torch.isfinite(out[:40]).all()          # sequence 0 is unaffected
     ref = _reference(c, qc, qs)
     assert np.abs(out[:40].cpu().numpy() - ref[:40]).max() <= 2.0 ** -14 * _vmax(c)

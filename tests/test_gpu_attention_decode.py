@@ -217,3 +217,24 @@ def test_bad_table_entries_and_long_contexts_are_counted():
     ref32 = oracle.attention_paged(q[1:2].astype(np.float64), K, V, 32)[0]
     tol, ulp = _tolerance(q[1], K, V, 32, torch.float32)
     assert (np.abs(out2[1].cpu().numpy() - ref32) <= tol + ulp * np.abs(ref32)).all()
+
+
+@pytest.mark.parametrize("qdt", [torch.float32, torch.bfloat16])
+def test_tensor_core_path_queries_beyond_binary16_range(qdt):
+    """Queries of magnitude up to 2^20 (beyond binary16's 65504): the
+    tensor-core path scales each head's query by a power of two into binary16
+    range and its scores back, so it stays finite and within the bound like
+    the CUDA-core path."""
+    seqs, Hq, Hkv, D, B, ctxs = 2, 8, 2, 128, 16, [200, 77]
+    c = _build(seqs, Hkv, D, B, ctxs, seed=91)
+    g = np.random.default_rng(92)
+    q = g.standard_normal((seqs, Hq, D)).astype(np.float32)
+    q[:, ::2] *= 2.0 ** 20                          # every other head far beyond 65504
+    q[0, 1] *= 2.0 ** 13                            # and one just below
+    qt = _to(q).to(qdt)
+    qref = qt.float().cpu().numpy()
+    for mma in (False, True):
+        out = _run(c, qt, ctxs, mma=mma)
+        torch.cuda.synchronize()
+        assert torch.isfinite(out).all(), f"mma={mma}: non-finite outputs"
+        _check(c, qref, out, ctxs, torch.float32, mma=mma)

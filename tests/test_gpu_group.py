@@ -2,8 +2,8 @@
 every layer's codes and scales bit-exact against the oracle, every output
 within the layer's stated bound |y - ref| <= 2^-8 |ref| + 1e-4 sqrt(K) A_m W_n
 against the oracle's binary64 layer.  The cases cover every token-tile class
-of the grouped kernel (M <= 16, 32, 64, 128) in one group, layers past it
-(M > 128, per-layer kernels), ragged N and K, groups small enough that one
+of the grouped kernel (M <= 16, 32, 64, 128, 256) in one group, layers past it
+(M > 256, per-layer kernels), ragged N and K, groups small enough that one
 weight tile is shared by several CTAs and large enough that a CTA walks
 many tiles and crosses layer boundaries, and repeated calls (the flag words
 must be left zero, and the results must repeat bit for bit)."""
@@ -56,6 +56,7 @@ def _check_layer(i, layer, x, w, ns=None):
 MIXED = [  # (M, K, N): all token classes, ragged N and K, one layer past the grouped kernel
     (1, 512, 528), (4, 272, 400), (8, 1040, 144), (16, 528, 1040), (17, 400, 272), (32, 1008, 656),
     (33, 144, 912), (64, 656, 528), (65, 272, 1296), (100, 528, 400), (128, 1024, 1024), (160, 400, 528),
+    (256, 656, 272), (300, 400, 528),
 ]
 
 
@@ -128,7 +129,8 @@ def test_group_several_large_layers_after_a_producer():
     activations are written by a device kernel right before the call (the
     call's first launch overlaps it), and the last layer's activations are
     the ones written last: every layer must still see its final inputs."""
-    shapes = [(4, 1024, 528), (200, 1024, 528), (260, 528, 1040), (300, 1008, 272), (33, 400, 144)]
+    shapes = [(4, 1024, 528), (200, 1024, 528), (260, 528, 1040), (300, 1008, 272), (33, 400, 144),
+              (400, 656, 400)]
     layers, host = _make_group(shapes, 23)
     srcs = [torch.from_numpy(x).to(DEV) for (x, _) in host]
     for l in layers:
