@@ -338,8 +338,10 @@ class StepRunner:
         self.pg, self.torch, self.dev, self.wl, self.args, self.stream = pg, torch, dev, wl, args, stream
         layers = wl["layers"]
         self.layers = layers
-        self.grouped = (all(L.kind == "fp8" for L in layers) and not args.per_layer and not args.chain
-                        and args.scaling == "dynamic" and not args.fused_quant)
+        plain = not args.per_layer and not args.chain and args.scaling == "dynamic" and not args.fused_quant
+        self.grouped = plain and all(L.kind == "fp8" for L in layers)
+        # NestedFP workloads: one pgf8_nestedfp_linear_group call per mode
+        self.nested_grouped = plain and all(L.kind in ("nested16", "nested8") for L in layers)
         self.xflags = pg.FLAG_FUSED_QUANT if args.fused_quant else 0
         self.sk_ws = torch.zeros(max(16, max(pg.lib.pgf8_fp8_linear_workspace_size(L.M, L.N, L.K) for L in layers)),
                                  dtype=torch.uint8, device=dev)
@@ -355,6 +357,25 @@ class StepRunner:
                 self.classes += [idx[j:j + 32] for j in range(0, len(idx), 32)]
             self.large = [i for i, L in enumerate(layers) if L.M > GROUP_MAX_M]
             self.sub = [pg.LayerGroup([ent(i) for i in idx]) for idx in self.classes]
+        if self.nested_grouped:
+            def nent(i):
+                L = layers[i]
+                hi, lo = wl["weights"][_wkey(L)]
+                n16 = L.kind == "nested16"
+                return (wl["acts"][i], hi, lo if n16 else None, wl["outs"][i], None if n16 else wl["qbufs"][i])
+            self.ngroups, self.nsub, self.nlarge = [], [], []
+            for kind in ("nested16", "nested8"):
+                mode = pg.NESTED_FP16 if kind == "nested16" else pg.NESTED_FP8
+                idx = [i for i, L in enumerate(layers) if L.kind == kind]
+                if not idx:
+                    continue
+                self.ngroups.append(pg.NestedLayerGroup([nent(i) for i in idx], mode=mode))
+                for lo_m, hi_m in ((0, 128), (128, GROUP_MAX_M)):
+                    cls = [i for i in idx if lo_m < layers[i].M <= hi_m]
+                    for j in range(0, len(cls), 32):
+                        self.nsub.append((cls[j:j + 32], pg.NestedLayerGroup([nent(i) for i in cls[j:j + 32]],
+                                                                             mode=mode)))
+                self.nlarge += [i for i in idx if layers[i].M > GROUP_MAX_M]
         self.per_tensor = {}
         if not self.grouped and args.scaling != "dynamic":
             for i, L in enumerate(layers):
@@ -375,6 +396,9 @@ class StepRunner:
     def launches_per_step(self):
         if self.grouped:
             return sum(2 * ((len(c) + 31) // 32) for c in self.classes) + 2 * len(self.large)
+        if self.nested_grouped:
+            per = lambda i: 2 if self.layers[i].kind == "nested8" else 1  # noqa: E731
+            return sum(per(idx[0]) for idx, _ in self.nsub) + sum(per(i) for i in self.nlarge)
         return sum(2 if L.kind in ("fp8", "nested8") else 1 for L in self.layers)
 
     def _quantise(self, i, L, flags):
@@ -398,6 +422,10 @@ class StepRunner:
         pg, wl, s = self.pg, self.wl, self.stream
         if self.grouped:
             self.group.run(flags=pg.FLAG_OVERLAP_PREVIOUS, stream=s)
+            return
+        if self.nested_grouped:
+            for grp in self.ngroups:
+                grp.run(flags=pg.FLAG_OVERLAP_PREVIOUS, stream=s)
             return
         ov = pg.FLAG_OVERLAP_PREVIOUS
         for i, L in enumerate(self.layers):
@@ -439,6 +467,17 @@ class StepRunner:
                 aq, sa = self._quantise(i, L, 0)
                 mark(("gemm", (i,)))
                 pg.fp8_linear(aq, sa, W[0], W[1], y=wl["outs"][i], workspace=self.sk_ws, stream=s)
+        elif self.nested_grouped:
+            for idx, sub in self.nsub:
+                mark(("group", tuple(idx)))
+                sub.run(stream=s)
+            for i in self.nlarge:
+                L = self.layers[i]
+                W = wl["weights"][_wkey(L)]
+                mode = pg.NESTED_FP16 if L.kind == "nested16" else pg.NESTED_FP8
+                mark(("gemm", (i,)))
+                pg.nestedfp_linear(wl["acts"][i], W[0], W[1] if mode == pg.NESTED_FP16 else None, mode=mode,
+                                   y=wl["outs"][i], workspace=wl["qbufs"][i], stream=s)
         else:
             for i, L in enumerate(self.layers):
                 W = wl["weights"][_wkey(L)]
@@ -662,6 +701,7 @@ def run_ours(args, rank, world, local_rank):
     e2e = run_e2e(pg, torch, dev, wl, args, world, wbytes, flops, memory_bound)
 
     grouped = res["runner"].grouped
+    nested_grouped = res["runner"].nested_grouped
     result = {
         "metric": METRIC,
         "value": round(gbs if memory_bound else tflops, 2),
@@ -681,6 +721,8 @@ def run_ours(args, rank, world, local_rank):
                    "step": ("one pgf8_fp8_linear_dynamic_group call: the M <= 128 layers quantised by one launch and "
                             "streamed by one grouped kernel, each larger layer quantised and multiplied by its own "
                             "kernels" if grouped else
+                            "one pgf8_nestedfp_linear_group call per mode: its M <= 128 layers streamed by one "
+                            "grouped kernel, each larger layer by the tiled kernels" if nested_grouped else
                             "one call per layer, chained with PGF8_FLAG_OVERLAP_PREVIOUS"),
                    "timing": "CUDA graph of the C-ABI calls, R=%d steps per replay, replayed K/R times" % res["R"],
                    "quantisation": ("inside the skinny GEMM where each CTA's activation slice fits its registers"
@@ -710,7 +752,8 @@ def run_ours(args, rank, world, local_rank):
             v = (r2["wbytes"] / 1e9 if mb else r2["flops"] / 1e12) / (r2["ms_step"] * 1e-3) * world
             result["secondary"][sec] = {
                 "value": round(v, 2), "unit": "GB/s" if mb else "TFLOP/s", "ms_per_step": round(r2["ms_step"], 5),
-                "steps": steps2, "grouped": r2["runner"].grouped, "roofline": r2["roof"], "regimes": r2["regimes"],
+                "steps": steps2, "grouped": r2["runner"].grouped or r2["runner"].nested_grouped,
+                "roofline": r2["roof"], "regimes": r2["regimes"],
                 "segments": r2["segments"]}
             if sec == "decode7b" and "decode_m_le_16" in r2["regimes"]:
                 # the decode regime as its own step (the 70B step streams its
@@ -802,6 +845,7 @@ def run_e2e(pg, torch, dev, wl, args, world, wbytes, flops, memory_bound):
             "steps": steps, "ms_per_step": round(ms, 5),
             "pipeline": "two device buffer sets; H2D, kernels and D2H on three streams ordered by events",
             "entry_point": ("pgf8_fp8_linear_dynamic_group" if bufs[0]["runner"].grouped else
+                            "pgf8_nestedfp_linear_group" if bufs[0]["runner"].nested_grouped else
                             "one C-ABI call per layer (pgf8_fp8_linear_dynamic / pgf8_nestedfp_linear / the "
                             "scaling and producer variants + pgf8_fp8_linear)")}
 
@@ -952,6 +996,13 @@ def run_single(args):
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         ws = torch.zeros(pg.fp8_linear_dynamic_workspace_size(M, N, K), dtype=torch.uint8, device=dev)
         fn = lambda: pg.fp8_linear_dynamic(x, wq, sw, y=y, workspace=ws, **opts)  # noqa: E731
+    elif kind == "group":
+        # the layer as a grouped call of one (M <= 256: the grouped weight-streaming kernel)
+        wq, sw = pg.fp8_quantize_rows(w)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws = torch.zeros(pg.fp8_linear_dynamic_workspace_size(M, N, K), dtype=torch.uint8, device=dev)
+        grp = pg.LayerGroup([(x, wq, sw, y, ws)])
+        fn = grp.run
     else:
         hi, lo = pg.nestedfp_split(w.half())
         x16 = x.half()
@@ -1160,7 +1211,8 @@ def main():
                          "of QKV and gate+up, the SiLU gate of the gate+up output ahead of down")
     ap.add_argument("--fused-quant", action="store_true",
                     help="quantise dynamic activations inside the skinny GEMM where its kernel allows it")
-    ap.add_argument("--single", default=None, help="kind,M,K,N: time (or profile) one layer eagerly")
+    ap.add_argument("--single", default=None, help="kind,M,K,N: time (or profile) one layer eagerly; kind = fp8 (pre-quantised "
+                         "activations), dyn (dynamic), group (a grouped call of one), nested16, nested8")
     ap.add_argument("--attention", default=None,
                     help="seqs,q_heads,kv_heads,head_dim,context: time (or profile) the FP8 paged decode attention "
                          "eagerly (--split-k caps its context chunks)")

@@ -86,8 +86,8 @@ typedef enum {
     PGF8_PATH_TILED = 2,   /* tokens are the 128-row MMA operand (any M) */
     PGF8_PATH_STREAMK = 3, /* skinny, stream-K over one CTA per SM (M <= 32; needs the
                               workspace) */
-    PGF8_PATH_TILED_PAIR = 4 /* tiled on SM pairs (cta_group::2), 256 x 256 tiles; FP8
-                              operand kinds only */
+    PGF8_PATH_TILED_PAIR = 4 /* tiled on SM pairs (cta_group::2), 256 x 256 tiles (FP8
+                              kinds: tile_n 128 / 192 / 256; NestedFP FP16 mode: 256) */
 } pgf8_path;
 
 /* Flags of pgf8_linear_opts.flags.
@@ -541,12 +541,17 @@ pgf8_status pgf8_nestedfp_split(const void *w_f16, int64_t N, int64_t K, uint8_t
  * NestedFP linear ("NestedFP" §2.1-2.2).  x_f16 [M,K] FP16, y_f16 [M,N] FP16.
  *   PGF8_NESTED_FP16: y = fp16_rn( sum_k x[m,k] * fp16((hi<<8)|lo)[n,k] ),
  *     the weight rebuilt bit-exactly in shared memory inside the GEMM;
- *     FP32 accumulation.  workspace: as for pgf8_fp8_linear (used for M <= 32).
+ *     FP32 accumulation.  workspace: pgf8_nestedfp_linear_workspace_size
+ *     bytes (nonzero for M <= 256: flags and partial slots of the grouped
+ *     kernel, zero-filled once), may be NULL above.
  *   PGF8_NESTED_FP8: x is quantised per token to E4M3 (as
  *     pgf8_fp8_quantize_rows, DYNAMIC) into the workspace, and
  *     y = fp16_rn( (sum_k e4m3(aq[m,k]) * e5m2(hi[n,k])) * sa[m] ): the upper
  *     byte is read as an E5M2 code with unit scale, which is the FP16 weight
  *     with its low 8 bits cleared.  lo is ignored and may be NULL.
+ * With the automatic kernel choice, M <= 256 runs the grouped
+ * weight-streaming kernel on this one layer (every SM streams an equal
+ * share of the weight planes); larger M runs the tiled kernels.
  * ---------------------------------------------------------------------- */
 pgf8_status pgf8_nestedfp_linear(const void *x_f16, int64_t M, int64_t K, const uint8_t *hi,
                                  const uint8_t *lo, int64_t N, pgf8_nested_mode mode,
@@ -560,6 +565,42 @@ pgf8_status pgf8_nestedfp_linear_ex(const void *x_f16, int64_t M, int64_t K, con
 
 size_t pgf8_nestedfp_linear_workspace_size(int64_t M, int64_t N, int64_t K,
                                            pgf8_nested_mode mode);
+
+/* One layer of pgf8_nestedfp_linear_group: the arguments of
+ * pgf8_nestedfp_linear. */
+typedef struct {
+    const void *x_f16;       /* [M, K] FP16, rows K elements apart */
+    const uint8_t *hi;       /* [N, K] upper byte plane */
+    const uint8_t *lo;       /* [N, K] lower byte plane (FP16 mode; ignored in FP8 mode) */
+    void *y_f16;             /* [M, N] FP16 */
+    void *workspace;         /* FP8 mode: pgf8_nestedfp_linear_workspace_size(M, N, K, FP8) bytes
+                                (codes and scales); FP16 mode: unused, may be NULL */
+    size_t workspace_bytes;
+    int64_t M, K, N;
+} pgf8_nested_layer;
+
+/* ------------------------------------------------------------------------
+ * A group of INDEPENDENT NestedFP linear layers in one mode ("NestedFP"
+ * §2.1-2.2; no layer reads another layer's output), enqueued by one call on
+ * `stream`.  Each layer computes exactly what pgf8_nestedfp_linear computes
+ * in that mode (FP8 mode: its codes and scales bit-identical; its outputs
+ * within the same bound, the f32 summation order differs).
+ * Layers with M <= 256 stream their weight planes through the grouped
+ * kernel as pgf8_fp8_linear_dynamic_group does (FP8 mode: one quantisation
+ * launch first; one launch for the layers with M <= 128 and one for
+ * 128 < M <= 256, up to 32 layers each); larger layers run one call each.
+ *   group_workspace: pgf8_fp8_linear_group_workspace_size(max M of the
+ *     layers with M <= 256) bytes, zero-filled once before first use and
+ *     left zero by every call; may be NULL when no layer has M <= 256.
+ *   Every layer is checked before anything is enqueued (as
+ *   pgf8_nestedfp_linear, plus: no layer's y or workspace overlaps any
+ *   layer's x or another layer's y or workspace, else INVALID_ARG).
+ *   PGF8_FLAG_OVERLAP_PREVIOUS in opts applies to the first launch.
+ * ---------------------------------------------------------------------- */
+pgf8_status pgf8_nestedfp_linear_group(const pgf8_nested_layer *layers, int64_t count,
+                                       pgf8_nested_mode mode, void *group_workspace,
+                                       size_t group_workspace_bytes, const pgf8_linear_opts *opts,
+                                       void *stream);
 
 /* ------------------------------------------------------------------------
  * Allocation-free dynamic FP8 linear.  The pages have no counterpart of this

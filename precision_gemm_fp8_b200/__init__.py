@@ -56,6 +56,12 @@ class Fp8Layer(ctypes.Structure):
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
 
 
+class NestedLayer(ctypes.Structure):
+    _fields_ = [("x_f16", ctypes.c_void_p), ("hi", ctypes.c_void_p), ("lo", ctypes.c_void_p),
+                ("y_f16", ctypes.c_void_p), ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+                ("M", ctypes.c_int64), ("K", ctypes.c_int64), ("N", ctypes.c_int64)]
+
+
 _vp = ctypes.c_void_p
 _i64 = ctypes.c_int64
 _sz = ctypes.c_size_t
@@ -96,6 +102,7 @@ _SIGS = {
     "pgf8_nestedfp_split": ([_vp, _i64, _i64, _vp, _vp, _vp], _i32),
     "pgf8_nestedfp_linear": ([_vp, _i64, _i64, _vp, _vp, _i64, _i32, _vp, _vp, _sz, _vp], _i32),
     "pgf8_nestedfp_linear_ex": ([_vp, _i64, _i64, _vp, _vp, _i64, _i32, _vp, _vp, _sz, _optp, _vp], _i32),
+    "pgf8_nestedfp_linear_group": ([ctypes.POINTER(NestedLayer), _i64, _i32, _vp, _sz, _optp, _vp], _i32),
     "pgf8_nestedfp_linear_workspace_size": ([_i64, _i64, _i64, _i32], _sz),
     "pgf8_fp8_linear_dynamic_noalloc": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _i64, _vp, _vp], _i32),
     "pgf8_last_cuda_error": ([ctypes.POINTER(ctypes.c_int)], _i32),
@@ -684,6 +691,42 @@ def nestedfp_linear(x, hi, lo, mode=NESTED_FP16, y=None, workspace=None, path=PA
                                        _ptr(y), _ptr(workspace), wbytes, _opts(path, split_k, tile_n, flags),
                                        _stream(stream)), "nestedfp_linear")
     return y
+
+
+class NestedLayerGroup:
+    """A fixed group of INDEPENDENT NestedFP layers in one mode, run by one
+    call of pgf8_nestedfp_linear_group: the layers with M <= 256 stream their
+    weight planes through the grouped kernel.  Entries are tuples
+    (x [M,K] f16, hi [N,K], lo [N,K] or None, y [M,N] f16, workspace or None);
+    FP8 mode needs each layer's workspace (nestedfp_linear_workspace_size
+    bytes), FP16 mode none.  The group workspace is allocated (zero-filled)
+    here unless given."""
+
+    def __init__(self, layers, mode=NESTED_FP16, group_workspace=None):
+        self._keep = list(layers)
+        self.mode = mode
+        arr = (NestedLayer * len(self._keep))()
+        for i, (x, hi, lo, y, ws) in enumerate(self._keep):
+            if x.dtype != torch.float16 or not x.is_contiguous():
+                raise ValueError("x must be a contiguous float16 tensor")
+            arr[i] = NestedLayer(x.data_ptr(), hi.data_ptr(), lo.data_ptr() if lo is not None else None,
+                                 y.data_ptr(), ws.data_ptr() if ws is not None else None, _nbytes(ws),
+                                 x.shape[0], x.shape[1], hi.shape[0])
+        self._arr = arr
+        self.count = len(self._keep)
+        max_m = max((x.shape[0] for (x, *_rest) in self._keep if x.shape[0] <= 256), default=0)
+        need = group_workspace_size(max_m) if max_m else 0
+        if group_workspace is None:
+            dev = self._keep[0][0].device if self._keep else "cuda"
+            group_workspace = torch.zeros(max(need, 16), dtype=torch.uint8, device=dev)
+        elif _nbytes(group_workspace) < need:
+            raise ValueError(f"group workspace needs {need} bytes")
+        self.group_workspace = group_workspace
+
+    def run(self, flags=0, stream=None):
+        _check(lib.pgf8_nestedfp_linear_group(self._arr, self.count, self.mode, _ptr(self.group_workspace),
+                                              _nbytes(self.group_workspace), _opts(flags=flags), _stream(stream)),
+               "nestedfp_linear_group")
 
 
 def selftest_row_division(divisors: torch.Tensor, stream=None):

@@ -13,7 +13,7 @@
 //   O = P . V_codes . 2^-8 . sv / l
 // l sums the unrounded probabilities.  head_dim 128.
 //
-// One CTA per (128-query tile, query head, sequence), heaviest tiles first, 192 threads:
+// One CTA per (128-query tile, query head, sequence), heaviest tiles first, 320 threads:
 //   warp 0      TMA: the Q tile once, then per 128-key tile eight 16-row
 //               pieces of K and of V straight from the paged cache (a piece
 //               past the context, or of an out-of-range block, is read at a
@@ -21,11 +21,16 @@
 //   warp 1      TMEM (512 columns: S double buffer, PV double buffer) and
 //               the MMA issue: S_j = Q K_j^T, then PV_{j-1} = P_{j-1} V_{j-1}
 //               (V as an MN-major operand: the cache rows are d-contiguous);
-//   warps 2-5   one query row per thread: scores from TMEM (two passes),
-//               causal and validity masks, online softmax in base 2, P codes
+//   warps 2-9   two threads per query row (warps 2-5: keys / head-dim
+//               columns 0-63 of their TMEM lane quadrant, warps 6-9: columns
+//               64-127): scores from TMEM (two passes), causal and validity
+//               masks, online softmax in base 2 (the two halves' maxima
+//               exchanged through shared memory at a named barrier), P codes
 //               written into shared memory in the 128-byte-swizzled K-major
 //               layout, PV_{j-1} added into registers one tile late (so the
 //               PV MMA overlaps the next softmax), final 1/l and scales.
+//               Every barrier of these 8 warps also ANDs their wait results,
+//               so they leave the loop together when one of them gives up.
 // Every wait is bounded: a wait that gives up raises the CTA's abort flag
 // and the device error word; in-flight copies and MMAs are drained before
 // the CTA frees its TMEM and exits.
@@ -43,7 +48,10 @@ constexpr int kCtxK = kCtxQ + kCtxTile;
 constexpr int kCtxV = kCtxK + kCtxStages * kCtxTile;
 constexpr int kCtxP = kCtxV + kCtxStages * kCtxTile;
 constexpr int kCtxCtl = kCtxP + 2 * kCtxTile;
-constexpr int kCtxSmemBytes = kCtxCtl + 1024 /*control*/ + 1024 /*alignment slack*/;
+constexpr int kCtxRed = kCtxCtl + 1024;         // [2 parities][2 halves][128 rows] f32: row-max exchange
+constexpr int kCtxSmemBytes = kCtxRed + 2048 + 1024 /*alignment slack*/;
+constexpr int kCtxThreads = 320;                 // producer, MMA, 8 softmax warps
+constexpr int kCtxSoftmaxThreads = 256;
 constexpr uint32_t kCtxTmemCols = 512;
 static_assert(kCtxSmemBytes <= 227 * 1024, "shared memory");
 
@@ -79,26 +87,27 @@ struct AttnCtxParams {
     int32_t *errors;
 };
 
-// One query row of the output (128 values, already scaled) into `dst`:
+// N values of one query row of the output (scaled by f) into out[base ..]:
 // 16-byte stores when allowed, else element by element.
-__device__ __forceinline__ void store_row128(void *out, int64_t base, int odt, bool vec, const float (&o)[128], float f)
+template <int N>
+__device__ __forceinline__ void store_row(void *out, int64_t base, int odt, bool vec, const float (&o)[N], float f)
 {
     if (!vec) {
 #pragma unroll
-        for (int d = 0; d < 128; ++d)
+        for (int d = 0; d < N; ++d)
             store_elem(out, base + d, odt, o[d] * f);
         return;
     }
     if (odt == 0) {
         float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(out) + base);
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
+        for (int i = 0; i < N / 4; ++i)
             dst[i] = make_float4(o[4 * i] * f, o[4 * i + 1] * f, o[4 * i + 2] * f, o[4 * i + 3] * f);
         return;
     }
     uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(out) + base);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
+    for (int i = 0; i < N / 8; ++i) {
         uint32_t w[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -146,7 +155,23 @@ __device__ __forceinline__ int ctx_piece_row(const AttnCtxParams &p, int64_t s, 
     return static_cast<int>((blk * p.Hkv + hk) * p.B + key % p.B);
 }
 
-__global__ void __launch_bounds__(192, 1) attn_context_kernel(const __grid_constant__ CUtensorMap tmQ,
+// AND of v over the 8 softmax warps (named barrier 1): also the barrier at
+// which they exchange row maxima through shared memory.
+__device__ __forceinline__ bool ctx_softmax_all(bool v)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, 1, 256, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}\n"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(v))
+        : "memory");
+    return r != 0;
+}
+
+__global__ void __launch_bounds__(kCtxThreads, 1) attn_context_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                               const __grid_constant__ CUtensorMap tmK,
                                                               const __grid_constant__ CUtensorMap tmV,
                                                               const AttnCtxParams p)
@@ -191,10 +216,10 @@ __global__ void __launch_bounds__(192, 1) attn_context_kernel(const __grid_const
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->s_full[b], 1);
-            mbar_init(&ctl->s_free[b], 4);    // one arrival per softmax warp
-            mbar_init(&ctl->p_full[b], 4);
+            mbar_init(&ctl->s_free[b], 8);    // one arrival per softmax warp
+            mbar_init(&ctl->p_full[b], 8);
             mbar_init(&ctl->o_full[b], 1);
-            mbar_init(&ctl->o_free[b], 4);
+            mbar_init(&ctl->o_free[b], 8);
         }
         mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
@@ -288,35 +313,37 @@ __global__ void __launch_bounds__(192, 1) attn_context_kernel(const __grid_const
         }
         __syncwarp();
     } else {
-        // ---------------------------------------------------------------- softmax (one query row per thread)
+        // ---------------------------------------------------------------- softmax (two threads per query row)
         const int qd = warp & 3;                          // TMEM lane quadrant of this warp
+        const int half = (warp - 2) >> 2;                 // 0: columns 0-63, 1: columns 64-127
         const int r = qd * 32 + lane;                     // query row of the tile
-        const int et = static_cast<int>(threadIdx.x) - 64;
+        const int et = static_cast<int>(threadIdx.x) - 64;   // 0 .. 255
+        const int c_lo = half * 64;
         const bool row_ok = r < nrows;
         const int pos = pos0 + r;
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+        float *red = reinterpret_cast<float *>(smem + kCtxRed);   // [parity][half][row]
         const float scale = row_ok ? p.q_scales[(static_cast<int64_t>(q0) + qt * 128 + r) * p.Hq + h] * p.sk[hk] *
                                          (1.4426950408889634f * 0.08838834764831845f)   // log2(e) / sqrt(128)
                                    : 0.0f;
-        float m = -INFINITY, l = 0.0f, alpha_prev = 0.0f;
-        float o[128];
+        float m = -INFINITY, l = 0.0f, alpha_prev = 0.0f;   // l: this half's share of the row sum
+        float o[64];                                         // head-dim columns c_lo .. c_lo + 63
 #pragma unroll
-        for (int d = 0; d < 128; ++d)
+        for (int d = 0; d < 64; ++d)
             o[d] = 0.0f;
         bool ok = true;
 
         // O += PV_i (relative to the maximum after tile i), rescaling by alpha
         auto accumulate = [&](int i, float alpha) -> bool {
             const int b = i & 1, k = i >> 1;
-            bool w = wait_bounded(&ctl->o_full[b], static_cast<uint32_t>(k) & 1u, abort_flag);
-            w = __all_sync(0xffffffffu, w);
+            const bool w = ctx_softmax_all(wait_bounded(&ctl->o_full[b], static_cast<uint32_t>(k) & 1u, abort_flag));
             if (!w)
                 return false;
             tc_fence_after();
 #pragma unroll
-            for (int c0 = 0; c0 < 128; c0 += 16) {
+            for (int c0 = 0; c0 < 64; c0 += 16) {
                 uint32_t v[16];
-                tmem_ld_32x32b_x16(t_lane + 256 + b * 128 + c0, v);
+                tmem_ld_32x32b_x16(t_lane + 256 + b * 128 + c_lo + c0, v);
                 tmem_ld_wait();
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
@@ -343,44 +370,49 @@ __global__ void __launch_bounds__(192, 1) attn_context_kernel(const __grid_const
                 else if (et == 0 && h == 0 && qt == (q_len - 1) / 128 && p.errors)
                     atomicAdd(p.errors, 1);   // once: the sequence's last query tile visits every key tile
             }
-            bool w = wait_bounded(&ctl->s_full[b], static_cast<uint32_t>(k) & 1u, abort_flag);
-            w = __all_sync(0xffffffffu, w);
-            if (!w) {
+            const bool w = wait_bounded(&ctl->s_full[b], static_cast<uint32_t>(k) & 1u, abort_flag);
+            const uint32_t t_s = t_lane + b * 128 + c_lo;
+            // pass 1: the maximum of this half's valid scores, exchanged with the other half's
+            float mx = -INFINITY;
+            if (w) {
+                tc_fence_after();
+#pragma unroll 1
+                for (int c0 = 0; c0 < 64; c0 += 16) {
+                    uint32_t v[16];
+                    tmem_ld_32x32b_x16(t_s + c0, v);
+                    tmem_ld_wait();
+                    const bool pok = (piece_ok >> ((c_lo + c0) >> 4)) & 1u;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int key = j * 128 + c_lo + c0 + e;
+                        const float sc = __uint_as_float(v[e]) * scale;
+                        mx = (pok && row_ok && key <= pos) ? fmaxf(mx, sc) : mx;
+                    }
+                }
+            }
+            float *red_j = red + (j & 1) * 256;
+            red_j[half * 128 + r] = mx;
+            if (!ctx_softmax_all(w)) {
                 ok = false;
                 break;
             }
-            tc_fence_after();
-            const uint32_t t_s = t_lane + b * 128;
-            // pass 1: the row maximum of the valid scores
-            float mx = -INFINITY;
-#pragma unroll 1
-            for (int c0 = 0; c0 < 128; c0 += 16) {
-                uint32_t v[16];
-                tmem_ld_32x32b_x16(t_s + c0, v);
-                tmem_ld_wait();
-                const bool pok = (piece_ok >> (c0 >> 4)) & 1u;
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int key = j * 128 + c0 + e;
-                    const float sc = __uint_as_float(v[e]) * scale;
-                    mx = (pok && row_ok && key <= pos) ? fmaxf(mx, sc) : mx;
-                }
-            }
+            mx = fmaxf(mx, red_j[(half ^ 1) * 128 + r]);
             const float mn = fmaxf(m, mx);
             const float alpha = m == -INFINITY ? 0.0f : exp2f(m - mn);
-            // pass 2: probabilities, their codes (x 2^8) into P buffer b, the row sum
+            // pass 2: probabilities, their codes (x 2^8) into P buffer b, this half's row sum
             float rs = 0.0f;
             uint8_t *prow = smem + kCtxP + b * kCtxTile + r * 128;
 #pragma unroll 1
-            for (int c0 = 0; c0 < 128; c0 += 16) {
+            for (int c0 = 0; c0 < 64; c0 += 16) {
                 uint32_t v[16];
                 tmem_ld_32x32b_x16(t_s + c0, v);
                 tmem_ld_wait();
-                const bool pok = (piece_ok >> (c0 >> 4)) & 1u;
+                const int cc = c_lo + c0;
+                const bool pok = (piece_ok >> (cc >> 4)) & 1u;
                 float pr[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const int key = j * 128 + c0 + e;
+                    const int key = j * 128 + cc + e;
                     const bool valid = pok && row_ok && key <= pos;
                     pr[e] = valid ? exp2f(__uint_as_float(v[e]) * scale - mn) : 0.0f;
                     rs += pr[e];
@@ -390,7 +422,7 @@ __global__ void __launch_bounds__(192, 1) attn_context_kernel(const __grid_const
                 for (int u = 0; u < 4; ++u)
                     wv[u] = static_cast<uint32_t>(cvt_e4m3x2(pr[4 * u] * 256.0f, pr[4 * u + 1] * 256.0f)) |
                             (static_cast<uint32_t>(cvt_e4m3x2(pr[4 * u + 2] * 256.0f, pr[4 * u + 3] * 256.0f)) << 16);
-                *reinterpret_cast<uint4 *>(prow + (((c0 >> 4) ^ (r & 7)) << 4)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                *reinterpret_cast<uint4 *>(prow + (((cc >> 4) ^ (r & 7)) << 4)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
             }
             tc_fence_before();
             __syncwarp();
@@ -401,8 +433,8 @@ __global__ void __launch_bounds__(192, 1) attn_context_kernel(const __grid_const
             // probability times a NaN code would still be NaN
             const int cut = ctx - j * 128;
             if (cut > 0 && cut < 128 && (cut & 15) != 0 && ((piece_ok >> (cut >> 4)) & 1u)) {
-                bool wk = wait_bounded(&ctl->kv_full[st], static_cast<uint32_t>(j / kCtxStages) & 1u, abort_flag);
-                wk = __all_sync(0xffffffffu, wk);
+                const bool wk = ctx_softmax_all(
+                    wait_bounded(&ctl->kv_full[st], static_cast<uint32_t>(j / kCtxStages) & 1u, abort_flag));
                 if (!wk) {
                     ok = false;
                     break;
@@ -426,10 +458,18 @@ __global__ void __launch_bounds__(192, 1) attn_context_kernel(const __grid_const
         }
         if (ok)
             ok = accumulate(nkt - 1, alpha_prev);
-        if (ok && row_ok) {
-            const float f = l > 0.0f ? p.sv[hk] * 0.00390625f / l : 0.0f;   // 2^-8 undoes the P code scale
-            const int64_t base = (static_cast<int64_t>(q0) + qt * 128 + r) * p.ldo + static_cast<int64_t>(h) * 128;
-            store_row128(p.out, base, p.odt, p.vec_out != 0, o, f);
+        if (ok) {
+            // the row sum: both halves add the two shares in the same order
+            float *red_l = red + (nkt & 1) * 256;
+            red_l[half * 128 + r] = l;
+            ctx_softmax_all(true);
+            const float lsum = red_l[r] + red_l[128 + r];
+            if (row_ok) {
+                const float f = lsum > 0.0f ? p.sv[hk] * 0.00390625f / lsum : 0.0f;   // 2^-8 undoes the P code scale
+                const int64_t base =
+                    (static_cast<int64_t>(q0) + qt * 128 + r) * p.ldo + static_cast<int64_t>(h) * 128 + c_lo;
+                store_row<64>(p.out, base, p.odt, p.vec_out != 0, o, f);
+            }
         }
     }
 

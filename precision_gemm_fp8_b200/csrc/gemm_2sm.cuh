@@ -47,8 +47,9 @@ template <int BN_, int STAGES_, int KIND_> struct PairCfg {
     static constexpr int BN = BN_;                 // N of the pair's tile (MMA N)
     static constexpr int STAGES = STAGES_;
     static constexpr int KIND = KIND_;
-    static constexpr int XQ = 0;   // activations arrive as E4M3 codes
-    static constexpr int kThreads = 192;
+    static constexpr bool NEST16 = (KIND == kNested16);
+    static constexpr int XQ = 0;   // activations arrive as E4M3 codes (FP16 mode: as f16)
+    static constexpr int kThreads = NEST16 ? 320 : 192;   // FP16 mode: 4 rebuild warps
     static constexpr int kTileA = 128 * 128;      // this CTA's 128 activation rows
     static constexpr int kTileB = (BN / 2) * 128; // this CTA's BN/2 weight rows
     static constexpr int kStage = kTileA + kTileB;
@@ -61,7 +62,7 @@ template <int BN_, int STAGES_, int KIND_> struct PairCfg {
     static constexpr int kRingBytes = STAGES * kStage;
     static constexpr int kBarOffset = kRingBytes;
     static constexpr int kSmemBytes = kRingBytes + 1024 + 1024;
-    static_assert(KIND == kE4M3 || KIND == kNested8, "FP8 operand kinds only");
+    static_assert(!NEST16 || BN == 256, "FP16 mode: 256-wide tiles");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
@@ -123,6 +124,7 @@ struct PairWalk {
 struct PairCtl {
     uint64_t full[16];
     uint64_t empty[16];
+    uint64_t conv[16];   // FP16 mode, even CTA: both CTAs' weight halves rebuilt
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t drain;
@@ -155,6 +157,17 @@ __device__ __forceinline__ void umma_f8f6f4_pair(uint32_t d_tmem, uint64_t adesc
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_f16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
@@ -247,8 +260,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     constexpr int BN = C::BN;
     constexpr int STAGES = C::STAGES;
     constexpr int KIND = C::KIND;
+    constexpr bool NEST16 = C::NEST16;
     constexpr uint32_t kIdesc = make_idesc(256, BN, 0, KIND == kNested8 ? 1 : 0);
-    (void)tmW2;
+    constexpr int kXStep = NEST16 ? 64 : 128;   // activation elements per k-block
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -269,6 +283,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&ctl->full[s], 1);
             mbar_init(&ctl->empty[s], 1);
+            mbar_init(&ctl->conv[s], 8);        // FP16 mode: 4 rebuild warps in each CTA
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->acc_full[b], 1);
@@ -282,6 +297,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmX);
         tma_prefetch_desc(&tmW);
+        if (NEST16)
+            tma_prefetch_desc(&tmW2);
     }
     if (warp == 1) {
         tmem_alloc_pair(&ctl->tmem_base, C::kTmemCols);
@@ -320,10 +337,20 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     // the even CTA passes each real completion of its empty
                     // barrier on to the odd CTA's
                     uint8_t *st = smem + s * C::kStage;
-                    if (lead)
-                        mbar_arrive_expect_tx(&ctl->full[s], 2 * C::kStage);
-                    tma_load_2d_pair(st, &tmX, &ctl->full[s], kb * 128, row_x, pol);
-                    tma_load_2d_pair(st + C::kTileA, &tmW, &ctl->full[s], kb * 128, row_w, pol);
+                    if constexpr (NEST16) {
+                        // each CTA's loads complete on its own barrier: its
+                        // rebuild warps wait for them; the MMA waits for both
+                        // CTAs' rebuilds instead (conv, even CTA)
+                        mbar_arrive_expect_tx(&ctl->full[s], C::kStage);
+                        tma_load_2d_hint(st, &tmX, &ctl->full[s], kb * kXStep, row_x, pol);
+                        tma_load_2d_hint(st + C::kTileA, &tmW, &ctl->full[s], kb * 64, row_w, pol);
+                        tma_load_2d_hint(st + C::kTileA + (BN / 2) * 64, &tmW2, &ctl->full[s], kb * 64, row_w, pol);
+                    } else {
+                        if (lead)
+                            mbar_arrive_expect_tx(&ctl->full[s], 2 * C::kStage);
+                        tma_load_2d_pair(st, &tmX, &ctl->full[s], kb * 128, row_x, pol);
+                        tma_load_2d_pair(st + C::kTileA, &tmW, &ctl->full[s], kb * 128, row_w, pol);
+                    }
                     issued_mask |= 1u << s;
                     issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
                     if (++s == STAGES) {
@@ -332,7 +359,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     }
                 }
             }
-            if (*abort_flag && lead) {
+            if (*abort_flag && (lead || NEST16)) {
                 for (int j = 0; j < STAGES; ++j)
                     if (issued_mask & (1u << j))
                         wait_drain(&ctl->full[j], (issued_ph >> j) & 1u);
@@ -358,7 +385,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                 tc_fence_after();
                 const uint32_t d = tmem + static_cast<uint32_t>(buf * BN);
                 for (int kb = kb0; kb < kb1; ++kb) {
-                    if (!wait_bounded(&ctl->full[s], ph, abort_flag)) {
+                    const bool got = NEST16 ? wait_bounded_cluster(&ctl->conv[s], ph, abort_flag)
+                                            : wait_bounded(&ctl->full[s], ph, abort_flag);
+                    if (!got) {
                         ok = false;
                         break;
                     }
@@ -369,7 +398,10 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     for (int k = 0; k < 4; ++k) {
                         const uint64_t ad = sdesc_sw128(a_addr + k * 32);
                         const uint64_t bd = sdesc_sw128(b_addr + k * 32);
-                        umma_f8f6f4_pair(d, ad, bd, kIdesc, (kb > kb0 || k > 0) ? 1u : 0u);
+                        if constexpr (NEST16)
+                            umma_f16_pair(d, ad, bd, kIdesc, (kb > kb0 || k > 0) ? 1u : 0u);
+                        else
+                            umma_f8f6f4_pair(d, ad, bd, kIdesc, (kb > kb0 || k > 0) ? 1u : 0u);
                     }
                     umma_commit_pair_both(&ctl->empty[s]);
                     if (++s == STAGES) {
@@ -386,6 +418,38 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             }
         }
         __syncwarp();
+    } else if (warp >= 6) {
+        // ------------------------------------------------------------ FP16 rebuild (both CTAs)
+        if constexpr (NEST16) {
+            const int tt = static_cast<int>(threadIdx.x) - 192;   // 0..127
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            PairWalk walk(pair, npairs, sk, total, p.kblocks);
+            int t, kb0, kb1;
+            while (ok && walk.next(t, kb0, kb1)) {
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!wait_bounded(&ctl->full[s], ph, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    // this CTA's 128 weight rows: (hi << 8) | lo in the swizzled K-major FP16 layout
+                    rebuild_fp16_tile<128>(smem + s * C::kStage + C::kTileA, tt);
+                    fence_proxy_async_smem();   // before the MMA (async proxy, issued by the even CTA) reads
+                    __syncwarp();
+                    if (lane == 0) {
+                        if (lead)
+                            mbar_arrive(&ctl->conv[s]);
+                        else
+                            mbar_arrive_remote(&ctl->conv[s], 0u);
+                    }
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+        }
     } else {
         // ------------------------------------------------------------ epilogue (both CTAs)
         const int q = warp & 3;
@@ -398,7 +462,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             const int n0 = (t / m_tiles) * BN + c0;
             if (m >= p.M || n0 >= p.N)
                 return;
-            const float sam = p.sa[m];
+            const float sam = NEST16 ? 1.0f : p.sa[m];
             if constexpr (KIND == kE4M3) {
                 if (p.out_f32) {
                     float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.y) + static_cast<int64_t>(m) * p.N +

@@ -45,10 +45,12 @@ constexpr int kGroupMaxLayers = 32;
 constexpr int kGroupMaxCtas = 256;             // partial slots in the group workspace
 constexpr size_t kGroupFlagBytes = 1024;       // kGroupMaxCtas 32-bit flags
 
-template <int BNMAX_, int STAGES_> struct GroupCfg {
+template <int BNMAX_, int STAGES_, int KIND_ = kE4M3> struct GroupCfg {
     static constexpr int BNMAX = BNMAX_;
     static constexpr int STAGES = STAGES_;
-    static constexpr int kThreads = 192;
+    static constexpr int KIND = KIND_;
+    static constexpr bool NEST16 = (KIND == kNested16);
+    static constexpr int kThreads = NEST16 ? 320 : 192;   // FP16 mode: 4 rebuild warps
     static constexpr int kTileA = 128 * 128;
     static constexpr int kStage = kTileA + BNMAX * 128;
     static constexpr int kTmemCols = (2 * BNMAX) < 32 ? 32 : 2 * BNMAX;
@@ -68,17 +70,19 @@ __host__ __device__ constexpr size_t group_workspace_bytes(int bnmax)
 struct GroupLayer {
     int64_t unit0;       // first unit of the layer in the group's order
     int M, N, K;
-    int kblocks;         // ceil(K / 128)
+    int kblocks;         // ceil(K bytes / 128): K / 64 k-blocks of FP16 activations in FP16 mode
     int bn;              // token rows of the MMA: M rounded up to 16 (<= BNMAX)
-    const float *sa;     // [M] per-token scales
-    const float *sw;     // [N] per-channel scales
-    void *y;             // [M, N] bf16, or f32 when out_f32
+    const float *sa;     // [M] per-token scales (E4M3 and NestedFP FP8 mode)
+    const float *sw;     // [N] per-channel scales (E4M3)
+    void *y;             // [M, N] bf16 (E4M3), f16 (NestedFP), or f32 when out_f32
     int out_f32;         // 1: y is f32, the scaled sum before rounding
 };
 
 struct GroupParams {
-    CUtensorMap tmW[kGroupMaxLayers];   // weights [N, K] codes, box 128 x 128
-    CUtensorMap tmX[kGroupMaxLayers];   // activation codes [M, K], box 128 x bn
+    CUtensorMap tmW[kGroupMaxLayers];   // weights [N, K] codes (NestedFP: the hi plane), box 128 x 128;
+                                        // FP16 mode: hi plane, box 64 bytes x 128, no swizzle
+    CUtensorMap tmW2[kGroupMaxLayers];  // FP16 mode: lo plane, as tmW
+    CUtensorMap tmX[kGroupMaxLayers];   // activation codes [M, K], box 128 x bn (FP16 mode: f16, box 64 x bn)
     GroupLayer L[kGroupMaxLayers];
     int nlayers;
     int prefetch_w;      // weights may be read before the grid dependency resolves
@@ -119,6 +123,9 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_group_kernel(const __grid
 {
     constexpr int BNMAX = C::BNMAX;
     constexpr int STAGES = C::STAGES;
+    constexpr int KIND = C::KIND;
+    constexpr bool NEST16 = C::NEST16;
+    constexpr int kXStep = NEST16 ? 64 : 128;   // activation elements per k-block
 
     grid_launch_dependents();
 
@@ -138,6 +145,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_group_kernel(const __grid
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&ctl->full[s], 1);
             mbar_init(&ctl->empty[s], 1);
+            mbar_init(&ctl->conv[s], 4);    // FP16 mode: one arrival per rebuild warp
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->acc_full[b], 1);
@@ -187,11 +195,17 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_group_kernel(const __grid
                     }
                     uint8_t *st = smem + s * C::kStage;
                     mbar_arrive_expect_tx(&ctl->full[s], bytes);
-                    tma_load_2d_hint(st, &p.tmW[sg.l], &ctl->full[s], kb * 128, sg.t * 128, pol_w);
+                    if constexpr (NEST16) {
+                        // hi and lo planes, 64 bytes (= 64 weights) of K each
+                        tma_load_2d_hint(st, &p.tmW[sg.l], &ctl->full[s], kb * 64, sg.t * 128, pol_w);
+                        tma_load_2d_hint(st + 128 * 64, &p.tmW2[sg.l], &ctl->full[s], kb * 64, sg.t * 128, pol_w);
+                    } else {
+                        tma_load_2d_hint(st, &p.tmW[sg.l], &ctl->full[s], kb * 128, sg.t * 128, pol_w);
+                    }
                     issued_mask |= 1u << s;
                     issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
                     if (waited) {
-                        tma_load_2d_hint(st + C::kTileA, &p.tmX[sg.l], &ctl->full[s], kb * 128, 0, pol_x);
+                        tma_load_2d_hint(st + C::kTileA, &p.tmX[sg.l], &ctl->full[s], kb * kXStep, 0, pol_x);
                     } else {
                         pend_l[pending] = sg.l;
                         pend_kb[pending] = kb;
@@ -203,7 +217,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_group_kernel(const __grid
                             waited = true;
                             for (int j = 0; j < pending; ++j)
                                 tma_load_2d_hint(smem + pend_s[j] * C::kStage + C::kTileA, &p.tmX[pend_l[j]],
-                                                 &ctl->full[pend_s[j]], pend_kb[j] * 128, 0, pol_x);
+                                                 &ctl->full[pend_s[j]], pend_kb[j] * kXStep, 0, pol_x);
                             pending = 0;
                         }
                     }
@@ -218,7 +232,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_group_kernel(const __grid
                 grid_dependency_wait();
             for (int j = 0; j < pending; ++j)
                 tma_load_2d_hint(smem + pend_s[j] * C::kStage + C::kTileA, &p.tmX[pend_l[j]], &ctl->full[pend_s[j]],
-                                 pend_kb[j] * 128, 0, pol_x);
+                                 pend_kb[j] * kXStep, 0, pol_x);
             if (*abort_flag) {
                 for (int j = 0; j < STAGES; ++j)
                     if (issued_mask & (1u << j))
@@ -238,7 +252,8 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_group_kernel(const __grid
             for (int64_t u = u0; ok && u < u1; ++i) {
                 const GroupSeg sg = group_seg(p, u, u1, l_hint);
                 l_hint = sg.l;
-                const uint32_t idesc = make_idesc(128, p.L[sg.l].bn, 0, 0);
+                // weights are operand A: E5M2 in NestedFP FP8 mode; FP16 in FP16 mode (kind::f16)
+                const uint32_t idesc = make_idesc(128, p.L[sg.l].bn, KIND == kNested8 ? 1 : 0, 0);
                 const int buf = i & 1;
                 const uint32_t use = static_cast<uint32_t>(i >> 1);
                 if (!wait_bounded(&ctl->acc_empty[buf], (use & 1u) ^ 1u, abort_flag)) {
@@ -252,13 +267,22 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_group_kernel(const __grid
                         ok = false;
                         break;
                     }
+                    if constexpr (NEST16) {
+                        if (!wait_bounded(&ctl->conv[s], ph, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                    }
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(smem + s * C::kStage);
                     const uint32_t b_addr = a_addr + C::kTileA;
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         const uint32_t acc = (kb > sg.kb0 || k > 0) ? 1u : 0u;
-                        umma_f8f6f4(d, sdesc_sw128(a_addr + k * 32), sdesc_sw128(b_addr + k * 32), idesc, acc);
+                        if constexpr (NEST16)
+                            umma_f16(d, sdesc_sw128(a_addr + k * 32), sdesc_sw128(b_addr + k * 32), idesc, acc);
+                        else
+                            umma_f8f6f4(d, sdesc_sw128(a_addr + k * 32), sdesc_sw128(b_addr + k * 32), idesc, acc);
                     }
                     umma_commit(&ctl->empty[s]);
                     if (++s == STAGES) {
@@ -276,6 +300,35 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_group_kernel(const __grid
             }
         }
         __syncwarp();
+    } else if (warp >= 6) {
+        // ------------------------------------------------------------ FP16 rebuild (FP16 mode)
+        if constexpr (NEST16) {
+            const int tt = static_cast<int>(threadIdx.x) - 192;   // 0..127
+            int s = 0;
+            uint32_t ph = 0;
+            int l_hint = 0;
+            bool ok = true;
+            for (int64_t u = u0; ok && u < u1;) {
+                const GroupSeg sg = group_seg(p, u, u1, l_hint);
+                l_hint = sg.l;
+                for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
+                    if (!wait_bounded(&ctl->full[s], ph, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    rebuild_fp16_tile<128>(smem + s * C::kStage, tt);
+                    fence_proxy_async_smem();   // each writer, before the MMA (async proxy) reads
+                    __syncwarp();
+                    if ((threadIdx.x & 31) == 0)
+                        mbar_arrive(&ctl->conv[s]);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                u = group_seg_end(p, sg);
+            }
+        }
     } else {
         // ------------------------------------------------------------ epilogue
         grid_dependency_wait();   // per-token scales come from the kernel before
@@ -288,21 +341,35 @@ __global__ void __launch_bounds__(C::kThreads, 1) gemm_group_kernel(const __grid
             const int n = t * 128 + r;
             if (n >= g.N)
                 return;
-            const float swn = g.sw[n];
-            if (g.out_f32) {
-                float *y = static_cast<float *>(g.y);
+            if constexpr (KIND == kE4M3) {
+                const float swn = g.sw[n];
+                if (g.out_f32) {
+                    float *y = static_cast<float *>(g.y);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (c0 + j < g.M)
+                            y[static_cast<int64_t>(c0 + j) * g.N + n] = a[j] * __ldg(g.sa + c0 + j) * swn;
+                    return;
+                }
+                __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(g.y);
 #pragma unroll
                 for (int j = 0; j < 16; ++j)
                     if (c0 + j < g.M)
-                        y[static_cast<int64_t>(c0 + j) * g.N + n] = a[j] * __ldg(g.sa + c0 + j) * swn;
-                return;
-            }
-            __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(g.y);
+                        y[static_cast<int64_t>(c0 + j) * g.N + n] =
+                            __float2bfloat16_rn(a[j] * __ldg(g.sa + c0 + j) * swn);
+            } else {
+                // NestedFP: f16 out; FP8 mode scales by the per-token scale
+                __half *y = static_cast<__half *>(g.y);
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-                if (c0 + j < g.M)
-                    y[static_cast<int64_t>(c0 + j) * g.N + n] =
-                        __float2bfloat16_rn(a[j] * __ldg(g.sa + c0 + j) * swn);
+                for (int j = 0; j < 16; ++j) {
+                    if (c0 + j < g.M) {
+                        float v = a[j];
+                        if constexpr (KIND == kNested8)
+                            v = v * __ldg(g.sa + c0 + j);
+                        y[static_cast<int64_t>(c0 + j) * g.N + n] = __float2half_rn(v);
+                    }
+                }
+            }
         };
         auto load16 = [&](uint32_t col, float (&a)[16]) {
             uint32_t v[16];

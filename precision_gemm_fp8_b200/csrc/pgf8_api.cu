@@ -370,7 +370,11 @@ template <class C> static pgf8_status launch_pair(const GemmLaunch &L)
 template <int KIND> static pgf8_status launch_pair_bn(const GemmLaunch &L, int bn)
 {
     if constexpr (KIND == kNested16) {
-        return PGF8_ERR_UNSUPPORTED;
+        // FP16 mode: 256-wide tiles only (6 stages of 16 KB activations +
+        // 16 KB rebuilt weights per CTA)
+        if (bn != 256)
+            return PGF8_ERR_UNSUPPORTED;
+        return launch_pair<PairCfg<256, 6, KIND>>(L);
     } else {
         if (bn == 128)
             return launch_pair<PairCfg<128, 8, KIND>>(L);
@@ -527,12 +531,9 @@ template <int KIND> static pgf8_status launch_gemm(const GemmLaunch &L)
         return launch_streamk<StreamKCfg<32, 5, KIND>>(L);
     }
     if (path == PGF8_PATH_TILED_PAIR) {
-        if (KIND == kNested16)
-            return PGF8_ERR_UNSUPPORTED;
         if (bn != 0 && bn != 128 && bn != 192 && bn != 256)
             return PGF8_ERR_INVALID_ARG;
-        if constexpr (KIND != kNested16)
-            return launch_pair_bn<KIND>(L, bn == 0 ? 256 : bn);
+        return launch_pair_bn<KIND>(L, bn == 0 ? 256 : bn);
     }
     if (path != PGF8_PATH_SKINNY && path != PGF8_PATH_TILED)
         return PGF8_ERR_INVALID_ARG;
@@ -568,6 +569,9 @@ template <int KIND> static pgf8_status launch_gemm(const GemmLaunch &L)
     // 70B shape (M = 256 .. 4096): with 40 or more tiles it is the fastest or
     // within 3 %; with 32 tiles the one-CTA persistent kernel below is
     // faster (more SMs busy on 128-row tiles).
+    // (NestedFP FP16 mode stays on the one-CTA kernels: its pair form
+    // measured 1.6-1.8x slower on B200 at every 7B / 70B shape, M = 512 ..
+    // 4096; it stays selectable through PGF8_PATH_TILED_PAIR)
     if constexpr (KIND != kNested16) {
         const int64_t tiles_pair = static_cast<int64_t>((L.M + 255) / 256) * ((L.N + 255) / 256);
         // (the 192 / 128 widths fill the last round better but measured slower
@@ -1186,7 +1190,7 @@ pgf8_status pgf8_fp8_attention_context_paged(const uint8_t *q_codes, const float
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(static_cast<unsigned>((max_q_len + 127) / 128 * q_heads), 1, static_cast<unsigned>(seqs));
-    cfg.blockDim = dim3(192);
+    cfg.blockDim = dim3(kCtxThreads);
     cfg.dynamicSmemBytes = kCtxSmemBytes;
     cfg.stream = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaLaunchKernelEx(&cfg, attn_context_kernel, tmQ, tmK, tmV, a);
@@ -1233,7 +1237,11 @@ static size_t streamk_bytes_for(int64_t M) { return M >= 1 && M <= 32 ? streamk_
 // Workspace of an FP8 linear call: the stream-K region of the kernel the
 // call takes (flag words at offset 0 in every layout): skinny stream-K slots
 // for M <= 32, the pair kernel's partial slots for M > 128.
-static_assert(kPairSKFlagBytes == kStreamKFlagBytes, "flag words at the start of every workspace layout");
+static_assert(kPairSKFlagBytes == kStreamKFlagBytes && kGroupFlagBytes == kStreamKFlagBytes,
+              "flag words at the start of every workspace layout");
+static_assert(streamk_workspace_bytes(16) == group_workspace_bytes(16) &&
+                  streamk_workspace_bytes(32) == group_workspace_bytes(32),
+              "an M <= 32 workspace holds the grouped kernel's slots");
 
 static size_t linear_ws_bytes(int64_t M)
 {
@@ -1242,6 +1250,16 @@ static size_t linear_ws_bytes(int64_t M)
     if (M > 128)
         return pair_sk_workspace_bytes(256);
     return 0;
+}
+
+// The grouped kernel's flags and partial slots for one layer of M tokens
+// (the NestedFP layers with M <= PGF8_GROUP_MAX_M run it): equal to the
+// skinny stream-K region for M <= 32.
+static size_t group_one_ws_bytes(int64_t M)
+{
+    if (M < 1 || M > PGF8_GROUP_MAX_M)
+        return 0;
+    return group_workspace_bytes(M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256);
 }
 
 size_t pgf8_fp8_linear_workspace_size(int64_t M, int64_t, int64_t) { return linear_ws_bytes(M); }
@@ -1287,7 +1305,8 @@ pgf8_status pgf8_fp8_linear(const uint8_t *aq, const float *sa, int64_t M, int64
 
 // Dynamic workspace layout: stream-K flag words (always, so they are never
 // overwritten by codes when one workspace serves layers of different shapes)
-// | stream-K partial slots (M <= 32: skinny; M > 128: pair kernel) | codes
+// | partial slots (M <= 256: the grouped kernel's for one layer, equal to the
+// skinny stream-K slots for M <= 32; M > 128: the pair kernel's) | codes
 // [M, K] | scales [M].
 size_t pgf8_fp8_linear_dynamic_codes_offset(int64_t M, int64_t K)
 {
@@ -1295,6 +1314,22 @@ size_t pgf8_fp8_linear_dynamic_codes_offset(int64_t M, int64_t K)
         return 0;
     const size_t b = linear_ws_bytes(M);
     return b > kStreamKFlagBytes ? b : kStreamKFlagBytes;
+}
+
+// NestedFP FP8 mode through the grouped kernel (M <= PGF8_GROUP_MAX_M): the
+// grouped kernel's flags and partial slots at offset 0, then the codes and
+// the scales (a larger region than a dynamic FP8 call's, so that the latter
+// keeps its size).
+static size_t nested8_codes_offset(int64_t M)
+{
+    size_t b = linear_ws_bytes(M);
+    b = group_one_ws_bytes(M) > b ? group_one_ws_bytes(M) : b;
+    return b > kStreamKFlagBytes ? b : kStreamKFlagBytes;
+}
+
+static size_t nested8_scales_offset(int64_t M, int64_t K)
+{
+    return nested8_codes_offset(M) + round_up(static_cast<size_t>(M) * static_cast<size_t>(K), 256);
 }
 
 size_t pgf8_fp8_linear_dynamic_scales_offset(int64_t M, int64_t K)
@@ -1512,7 +1547,7 @@ template <class C> static pgf8_status launch_group_cfg(const GroupParams &p, int
 
 // The grouped kernel for the layers described in gp (units already set),
 // token tile bnmax, one CTA per SM at most.
-static pgf8_status launch_group(const GroupParams &gp, int bnmax, cudaStream_t cs)
+template <int KIND = kE4M3> static pgf8_status launch_group(const GroupParams &gp, int bnmax, cudaStream_t cs)
 {
     int grid = num_sms();
     if (grid > kGroupMaxCtas)
@@ -1521,16 +1556,145 @@ static pgf8_status launch_group(const GroupParams &gp, int bnmax, cudaStream_t c
         grid = static_cast<int>(gp.units);
     switch (bnmax) {
     case 16:
-        return launch_group_cfg<GroupCfg<16, 12>>(gp, grid, cs);
+        return launch_group_cfg<GroupCfg<16, 12, KIND>>(gp, grid, cs);
     case 32:
-        return launch_group_cfg<GroupCfg<32, 11>>(gp, grid, cs);
+        return launch_group_cfg<GroupCfg<32, 11, KIND>>(gp, grid, cs);
     case 64:
-        return launch_group_cfg<GroupCfg<64, 9>>(gp, grid, cs);
+        return launch_group_cfg<GroupCfg<64, 9, KIND>>(gp, grid, cs);
     case 128:
-        return launch_group_cfg<GroupCfg<128, 6>>(gp, grid, cs);
+        return launch_group_cfg<GroupCfg<128, 6, KIND>>(gp, grid, cs);
     default:
-        return launch_group_cfg<GroupCfg<256, 4>>(gp, grid, cs);
+        return launch_group_cfg<GroupCfg<256, 4, KIND>>(gp, grid, cs);
     }
+}
+
+// One NestedFP layer of a grouped launch: its operands and, in FP8 mode,
+// where its codes and scales go.
+struct NestedItem {
+    const void *x;
+    int64_t M, K, N;
+    const uint8_t *hi, *lo;
+    void *y;
+    uint8_t *aq;
+    float *sa;
+};
+
+// Up to kGroupMaxLayers NestedFP layers with M <= PGF8_GROUP_MAX_M through
+// one grouped launch (every SM streams an equal share of all their weight
+// planes).  FP8 mode: the f16 activations are quantised per token first
+// (one launch), the hi plane is read as E5M2; FP16 mode: the f16
+// activations are read as they are and the weights rebuilt from both
+// planes.  group_ws holds the flags and partial slots.
+static pgf8_status nested_group_chunk(const NestedItem *it, int n, pgf8_nested_mode mode, void *group_ws,
+                                      int overlap, cudaStream_t cs)
+{
+    GroupParams gp;
+    std::memset(&gp, 0, sizeof(gp));
+    int64_t units = 0;
+    int bnmax = 16;
+    const bool fp8 = (mode == PGF8_NESTED_FP8);
+    for (int i = 0; i < n; ++i) {
+        const NestedItem &l = it[i];
+        const int bn = group_bn(l.M);
+        bnmax = bn > bnmax ? bn : bnmax;
+        GroupLayer &g = gp.L[i];
+        g.unit0 = units;
+        g.M = static_cast<int>(l.M);
+        g.N = static_cast<int>(l.N);
+        g.K = static_cast<int>(l.K);
+        g.bn = bn;
+        g.y = l.y;
+        bool ok;
+        if (fp8) {
+            g.kblocks = static_cast<int>((l.K + 127) / 128);
+            g.sa = l.sa;
+            ok = make_map(&gp.tmW[i], l.hi, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(l.N),
+                          static_cast<uint64_t>(l.K), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
+                 make_map(&gp.tmX[i], l.aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(l.M),
+                          static_cast<uint64_t>(l.K), 128, static_cast<uint32_t>(bn), CU_TENSOR_MAP_SWIZZLE_128B);
+        } else {
+            g.kblocks = static_cast<int>((l.K * 2 + 127) / 128);
+            ok = make_map(&gp.tmW[i], l.hi, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(l.N),
+                          static_cast<uint64_t>(l.K), 64, 128, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                 make_map(&gp.tmW2[i], l.lo, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(l.N),
+                          static_cast<uint64_t>(l.K), 64, 128, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                 make_map(&gp.tmX[i], l.x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, static_cast<uint64_t>(l.M),
+                          static_cast<uint64_t>(l.K), 64, static_cast<uint32_t>(bn), CU_TENSOR_MAP_SWIZZLE_128B);
+        }
+        if (!ok)
+            return PGF8_ERR_UNSUPPORTED;
+        units += static_cast<int64_t>((l.N + 127) / 128) * g.kblocks;
+    }
+    gp.nlayers = n;
+    gp.units = units;
+    gp.flags = static_cast<unsigned *>(group_ws);
+    gp.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(group_ws) + kGroupFlagBytes);
+    if (!fp8) {
+        gp.prefetch_w = overlap;   // the weight planes may come from the kernel before (the split)
+        return launch_group<kNested16>(gp, bnmax, cs);
+    }
+    gp.prefetch_w = 1;   // the quantisation before writes only codes and scales
+    if (n == 1) {
+        // one layer: the row kernels, which signal the grouped GEMM at once
+        // (it loads its first weight tiles while the activations are quantised)
+        const pgf8_status st = quantize_launch(it[0].x, PGF8_F16, it[0].M, it[0].K, it[0].K, it[0].aq, it[0].sa, 0,
+                                               cs, overlap, 1);
+        if (st != PGF8_OK)
+            return st;
+        return launch_group<kNested8>(gp, bnmax, cs);
+    }
+    QuantGroupParams qp;
+    std::memset(&qp, 0, sizeof(qp));
+    int64_t rows = 0;
+    for (int i = 0; i < n; ++i) {
+        QuantGroupLayer &q = qp.L[i];
+        q.x = it[i].x;
+        q.ldx = it[i].K;
+        q.cols = it[i].K;
+        q.row0 = rows;
+        q.rows = it[i].M;
+        q.q = it[i].aq;
+        q.scales = it[i].sa;
+        q.xdt = 1;
+        rows += it[i].M;
+    }
+    qp.nlayers = n;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(rows));
+    cfg.blockDim = dim3(kQuantThreads);
+    cfg.stream = cs;
+    cudaLaunchAttribute attr[1];
+    if (overlap) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, quantize_group_kernel, qp);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    return launch_group<kNested8>(gp, bnmax, cs);
+}
+
+// A NestedFP layer with M <= PGF8_GROUP_MAX_M through the grouped kernel
+// alone: the workspace holds the flags and partial slots at offset 0 and, in
+// FP8 mode, the codes and scales after them.
+static pgf8_status nested_group_one(const void *x, int64_t M, int64_t K, const uint8_t *hi, const uint8_t *lo,
+                                    int64_t N, pgf8_nested_mode mode, void *y, void *workspace, int overlap,
+                                    cudaStream_t cs)
+{
+    NestedItem it;
+    it.x = x;
+    it.M = M;
+    it.K = K;
+    it.N = N;
+    it.hi = hi;
+    it.lo = lo;
+    it.y = y;
+    it.aq = static_cast<uint8_t *>(workspace) + nested8_codes_offset(M);
+    it.sa = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + nested8_scales_offset(M, K));
+    return nested_group_chunk(&it, 1, mode, workspace, overlap, cs);
 }
 
 // One grouped launch pair for up to kGroupMaxLayers small-M layers: the
@@ -1815,18 +1979,41 @@ pgf8_status pgf8_nestedfp_split(const void *w, int64_t N, int64_t K, uint8_t *hi
 
 size_t pgf8_nestedfp_linear_workspace_size(int64_t M, int64_t N, int64_t K, pgf8_nested_mode mode)
 {
-    if (mode == PGF8_NESTED_FP8)
-        return pgf8_fp8_linear_dynamic_workspace_size(M, N, K);
-    return streamk_bytes_for(M);
+    if (mode == PGF8_NESTED_FP8) {
+        if (M < 0 || K < 0)
+            return 0;
+        const size_t dyn = pgf8_fp8_linear_dynamic_workspace_size(M, N, K);
+        const size_t grp = nested8_scales_offset(M, K) + round_up(static_cast<size_t>(M) * 4, 256);
+        return M >= 1 && M <= PGF8_GROUP_MAX_M && grp > dyn ? grp : dyn;
+    }
+    return group_one_ws_bytes(M);
 }
 
 pgf8_status pgf8_nestedfp_linear_ex(const void *x, int64_t M, int64_t K, const uint8_t *hi, const uint8_t *lo,
                                     int64_t N, pgf8_nested_mode mode, void *y, void *workspace,
                                     size_t workspace_bytes, const pgf8_linear_opts *opts, void *stream)
 {
-    if (mode == PGF8_NESTED_FP8)
-        return linear_dynamic_impl(x, PGF8_F16, M, K, K, hi, nullptr, nullptr, N, y, workspace, workspace_bytes,
-                                   opts, stream, kNested8);
+    const pgf8_linear_opts o = opts_or_default(opts);
+    // automatic choice, 16 < M <= 256: the grouped weight-streaming kernel
+    // with this one layer (measured on B200 faster than the split-K skinny
+    // kernel from M = 128 on every 7B / 70B shape; at M <= 16 the skinny
+    // kernel's shorter start and end win for a layer called alone)
+    const bool grouped = M > 16 && M <= PGF8_GROUP_MAX_M && o.path == PGF8_PATH_AUTO && o.split_k == 0 &&
+                         o.tile_n == 0 && !(o.flags & PGF8_FLAG_FUSED_QUANT);
+    const int overlap = (o.flags & PGF8_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
+    if (mode == PGF8_NESTED_FP8) {
+        if (!grouped)
+            return linear_dynamic_impl(x, PGF8_F16, M, K, K, hi, nullptr, nullptr, N, y, workspace, workspace_bytes,
+                                       opts, stream, kNested8);
+        pgf8_status st = check_linear_dynamic(x, PGF8_F16, M, K, K, hi, nullptr, N, y, workspace, workspace_bytes,
+                                              kNested8);
+        if (st != PGF8_OK)
+            return st;
+        if (workspace_bytes < pgf8_nestedfp_linear_workspace_size(M, N, K, mode))
+            return PGF8_ERR_INVALID_ARG;
+        return nested_group_one(x, M, K, hi, nullptr, N, mode, y, workspace, overlap,
+                                static_cast<cudaStream_t>(stream));
+    }
     if (mode != PGF8_NESTED_FP16)
         return PGF8_ERR_INVALID_ARG;
     pgf8_status st = check_dims(M, N, K);
@@ -1836,6 +2023,11 @@ pgf8_status pgf8_nestedfp_linear_ex(const void *x, int64_t M, int64_t K, const u
         return PGF8_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(hi) || !aligned16(lo) || !aligned16(y) || !aligned16(workspace))
         return PGF8_ERR_ALIGNMENT;
+    if (grouped) {
+        if (!workspace || workspace_bytes < pgf8_nestedfp_linear_workspace_size(M, N, K, mode))
+            return PGF8_ERR_INVALID_ARG;
+        return nested_group_one(x, M, K, hi, lo, N, mode, y, workspace, overlap, static_cast<cudaStream_t>(stream));
+    }
     GemmLaunch L;
     L.ws = workspace;
     L.ws_bytes = workspace ? workspace_bytes : 0;
@@ -1861,6 +2053,114 @@ pgf8_status pgf8_nestedfp_linear(const void *x, int64_t M, int64_t K, const uint
                                  void *stream)
 {
     return pgf8_nestedfp_linear_ex(x, M, K, hi, lo, N, mode, y, workspace, workspace_bytes, nullptr, stream);
+}
+
+pgf8_status pgf8_nestedfp_linear_group(const pgf8_nested_layer *layers, int64_t count, pgf8_nested_mode mode,
+                                       void *group_workspace, size_t group_workspace_bytes,
+                                       const pgf8_linear_opts *opts, void *stream)
+{
+    if (count < 0 || (count > 0 && !layers))
+        return PGF8_ERR_INVALID_ARG;
+    if (mode != PGF8_NESTED_FP16 && mode != PGF8_NESTED_FP8)
+        return PGF8_ERR_INVALID_ARG;
+    const bool fp8 = (mode == PGF8_NESTED_FP8);
+    int64_t max_small = 0;
+    for (int64_t i = 0; i < count; ++i) {
+        const pgf8_nested_layer &l = layers[i];
+        pgf8_status st;
+        if (fp8) {
+            st = check_linear_dynamic(l.x_f16, PGF8_F16, l.M, l.K, l.K, l.hi, nullptr, l.N, l.y_f16, l.workspace,
+                                      l.workspace_bytes, kNested8);
+            if (st == PGF8_OK && l.workspace_bytes < pgf8_nestedfp_linear_workspace_size(l.M, l.N, l.K, mode))
+                st = PGF8_ERR_INVALID_ARG;
+        } else {
+            st = check_dims(l.M, l.N, l.K);
+            if (st == PGF8_OK && (!l.x_f16 || !l.hi || !l.lo || !l.y_f16))
+                st = PGF8_ERR_INVALID_ARG;
+            if (st == PGF8_OK && (!aligned16(l.x_f16) || !aligned16(l.hi) || !aligned16(l.lo) || !aligned16(l.y_f16)))
+                st = PGF8_ERR_ALIGNMENT;
+        }
+        if (st != PGF8_OK)
+            return st;
+        if (l.M <= PGF8_GROUP_MAX_M && l.M > max_small)
+            max_small = l.M;
+    }
+    // independent layers only: no layer writes (y, workspace) what another
+    // layer reads or writes
+    for (int64_t i = 0; i < count; ++i) {
+        const pgf8_nested_layer &a = layers[i];
+        const size_t ya = static_cast<size_t>(a.M) * static_cast<size_t>(a.N) * 2;
+        const size_t wa = fp8 ? a.workspace_bytes : 0;
+        for (int64_t j = 0; j < count; ++j) {
+            const pgf8_nested_layer &b = layers[j];
+            const size_t xb = static_cast<size_t>(b.M) * static_cast<size_t>(b.K) * 2;
+            if (ranges_overlap(a.y_f16, ya, b.x_f16, xb) || (wa && ranges_overlap(a.workspace, wa, b.x_f16, xb)))
+                return PGF8_ERR_INVALID_ARG;
+            const size_t wb = fp8 ? b.workspace_bytes : 0;
+            if (i != j && (ranges_overlap(a.y_f16, ya, b.y_f16, static_cast<size_t>(b.M) * static_cast<size_t>(b.N) * 2) ||
+                           (wa && wb && ranges_overlap(a.workspace, wa, b.workspace, wb)) ||
+                           (wb && ranges_overlap(a.y_f16, ya, b.workspace, wb))))
+                return PGF8_ERR_INVALID_ARG;
+        }
+    }
+    if (max_small > 0) {
+        if (!group_workspace || group_workspace_bytes < pgf8_fp8_linear_group_workspace_size(max_small))
+            return PGF8_ERR_INVALID_ARG;
+        if (!aligned16(group_workspace))
+            return PGF8_ERR_ALIGNMENT;
+    }
+    pgf8_linear_opts o = opts_or_default(opts);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    int pdl = (o.flags & PGF8_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
+    // small layers: grouped as in pgf8_fp8_linear_dynamic_group, codes and
+    // scales (FP8 mode) at the dynamic layout's offsets of each workspace
+    NestedItem chunk[kGroupMaxLayers];
+    for (int pass = 0; pass < 2; ++pass) {
+        const int64_t lo = pass == 0 ? 0 : 128, hi = pass == 0 ? 128 : PGF8_GROUP_MAX_M;
+        int n = 0;
+        for (int64_t i = 0; i <= count; ++i) {
+            if (i < count && layers[i].M > lo && layers[i].M <= hi) {
+                const pgf8_nested_layer &l = layers[i];
+                NestedItem &it = chunk[n++];
+                it.x = l.x_f16;
+                it.M = l.M;
+                it.K = l.K;
+                it.N = l.N;
+                it.hi = l.hi;
+                it.lo = l.lo;
+                it.y = l.y_f16;
+                it.aq = fp8 ? static_cast<uint8_t *>(l.workspace) + pgf8_fp8_linear_dynamic_codes_offset(l.M, l.K)
+                            : nullptr;
+                it.sa = fp8 ? reinterpret_cast<float *>(static_cast<uint8_t *>(l.workspace) +
+                                                        pgf8_fp8_linear_dynamic_scales_offset(l.M, l.K))
+                            : nullptr;
+            }
+            if (n == kGroupMaxLayers || (i == count && n > 0)) {
+                const pgf8_status st = nested_group_chunk(chunk, n, mode, group_workspace, pdl, cs);
+                if (st != PGF8_OK)
+                    return st;
+                n = 0;
+                pdl = 1;
+            }
+        }
+    }
+    // large layers: one call each (the tiled kernels), overlapping the previous one
+    for (int64_t i = 0; i < count; ++i) {
+        const pgf8_nested_layer &l = layers[i];
+        if (l.M <= PGF8_GROUP_MAX_M)
+            continue;
+        pgf8_linear_opts ol = o;
+        ol.path = PGF8_PATH_AUTO;
+        ol.split_k = 0;
+        ol.tile_n = 0;
+        ol.flags = pdl ? PGF8_FLAG_OVERLAP_PREVIOUS : 0;
+        const pgf8_status st = pgf8_nestedfp_linear_ex(l.x_f16, l.M, l.K, l.hi, fp8 ? nullptr : l.lo, l.N, mode,
+                                                       l.y_f16, l.workspace, l.workspace_bytes, &ol, stream);
+        if (st != PGF8_OK)
+            return st;
+        pdl = 1;
+    }
+    return PGF8_OK;
 }
 
 pgf8_status pgf8_last_cuda_error(int *cuda_err)

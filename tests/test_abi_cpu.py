@@ -39,7 +39,9 @@ def test_workspace_sizes():
         assert off % 256 == 0 and off >= c0 + M * 4096
         ws = pg.lib.pgf8_fp8_linear_dynamic_workspace_size(M, 4096, 4096)
         assert ws >= off + 4 * M and ws % 256 == 0
-    assert pg.nestedfp_linear_workspace_size(64, 4096, 4096, pg.NESTED_FP16) == 0
+    # NestedFP FP16 mode up to 256 tokens: the grouped kernel's flags and partial slots
+    assert pg.nestedfp_linear_workspace_size(64, 4096, 4096, pg.NESTED_FP16) == 1024 + 256 * 64 * 128 * 4
+    assert pg.nestedfp_linear_workspace_size(300, 4096, 4096, pg.NESTED_FP16) == 0
     assert pg.nestedfp_linear_workspace_size(8, 4096, 4096, pg.NESTED_FP16) == \
         pg.lib.pgf8_fp8_linear_workspace_size(8, 4096, 4096)
     assert pg.nestedfp_linear_workspace_size(8, 4096, 4096, pg.NESTED_FP8) == \
@@ -116,6 +118,10 @@ def test_dynamic_and_nested_reject_bad_args():
     assert n(A16, 4, 512, B16, None, 512, pg.NESTED_FP16, D16, None, 0, None) == pg.ERR_INVALID_ARG
     assert n(A16, 4, 512, B16, C16, 512, 7, D16, None, 0, None) == pg.ERR_INVALID_ARG
     assert n(A16, 4, 512, B16, None, 512, pg.NESTED_FP8, D16, None, 0, None) == pg.ERR_INVALID_ARG
+    # FP16 mode on SM pairs: 256-wide tiles only; refused before any device call
+    pair128 = pg.LinearOpts(pg.PATH_TILED_PAIR, 0, 128, 0)
+    assert pg.lib.pgf8_nestedfp_linear_ex(A16, 300, 512, B16, C16, 512, pg.NESTED_FP16, D16, None, 0,
+                                          ctypes.byref(pair128), None) == pg.ERR_UNSUPPORTED
     s = pg.lib.pgf8_nestedfp_split
     assert s(None, 16, 16, B16, C16, None) == pg.ERR_INVALID_ARG
     assert s(A16, 3, 5, B16, C16, None) == pg.ERR_ALIGNMENT
@@ -177,6 +183,40 @@ def test_dynamic_group_checks_layers_aliasing_and_workspace_first():
     assert f(ok2, 2, gws + 8, ws_need, None, None) == pg.ERR_ALIGNMENT
     assert f(None, 2, gws, ws_need, None, None) == pg.ERR_INVALID_ARG
     assert f(None, 0, None, 0, None, None) == pg.OK
+
+
+def test_nested_group_checks_layers_aliasing_and_workspace_first():
+    """pgf8_nestedfp_linear_group: the mode, every layer (FP8 mode: with its
+    workspace), independence and the group workspace checked before anything
+    is enqueued."""
+    f = pg.lib.pgf8_nestedfp_linear_group
+    ws_need = pg.lib.pgf8_fp8_linear_group_workspace_size(64)
+    base = 1 << 33
+    x0, x1, y0, y1, hi, lo, wsp0, wsp1, gws = (base + i * (1 << 27) for i in range(9))
+    lw = pg.nestedfp_linear_workspace_size(64, 512, 512, pg.NESTED_FP8)
+    l0 = pg.NestedLayer(x0, hi, lo, y0, wsp0, lw, 64, 512, 512)
+    l1 = pg.NestedLayer(x1, hi, lo, y1, wsp1, lw, 8, 512, 512)     # layers may share weight planes
+    ok2 = (pg.NestedLayer * 2)(l0, l1)
+    for mode in (pg.NESTED_FP16, pg.NESTED_FP8):
+        assert f(ok2, 2, 7, gws, ws_need, None, None) == pg.ERR_INVALID_ARG          # mode
+        assert f(ok2, 2, mode, None, 0, None, None) == pg.ERR_INVALID_ARG           # group workspace missing
+        assert f(ok2, 2, mode, gws, ws_need - 16, None, None) == pg.ERR_INVALID_ARG
+        assert f(ok2, 2, mode, gws + 8, ws_need, None, None) == pg.ERR_ALIGNMENT
+        dep = pg.NestedLayer(y0, hi, lo, y1, wsp1, lw, 8, 512, 512)                 # reads layer 0's output
+        assert f((pg.NestedLayer * 2)(l0, dep), 2, mode, gws, ws_need, None, None) == pg.ERR_INVALID_ARG
+        same_y = pg.NestedLayer(x1, hi, lo, y0, wsp1, lw, 8, 512, 512)
+        assert f((pg.NestedLayer * 2)(l0, same_y), 2, mode, gws, ws_need, None, None) == pg.ERR_INVALID_ARG
+        bad_k = pg.NestedLayer(x1, hi, lo, y1, wsp1, lw, 8, 520, 512)               # K % 16
+        assert f((pg.NestedLayer * 2)(l0, bad_k), 2, mode, gws, ws_need, None, None) == pg.ERR_ALIGNMENT
+        assert f(None, 2, mode, gws, ws_need, None, None) == pg.ERR_INVALID_ARG
+        assert f(None, 0, mode, None, 0, None, None) == pg.OK
+    # FP16 mode needs the lo plane; FP8 mode needs each layer's workspace
+    no_lo = pg.NestedLayer(x1, hi, None, y1, None, 0, 8, 512, 512)
+    assert f((pg.NestedLayer * 1)(no_lo), 1, pg.NESTED_FP16, gws, ws_need, None, None) == pg.ERR_INVALID_ARG
+    small_ws = pg.NestedLayer(x1, hi, None, y1, wsp1, lw - 256, 64, 512, 512)
+    assert f((pg.NestedLayer * 1)(small_ws), 1, pg.NESTED_FP8, gws, ws_need, None, None) == pg.ERR_INVALID_ARG
+    shared_ws = pg.NestedLayer(x1, hi, None, y1, wsp0, lw, 8, 512, 512)
+    assert f((pg.NestedLayer * 2)(l0, shared_ws), 2, pg.NESTED_FP8, gws, ws_need, None, None) == pg.ERR_INVALID_ARG
 
 
 def test_tensor_parallel_blocks_argument_checks():

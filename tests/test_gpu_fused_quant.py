@@ -180,15 +180,20 @@ def test_fused_chain_reads_previous_output():
 
 def test_nested_fp8_mode_fused():
     """NestedFP FP8 mode (E4M3 activations x E5M2 hi plane) with M <= 32 runs
-    the fused kernel: bit-identical to its two-kernel form."""
+    the fused kernel: bit-identical to its two-kernel form (the quantisation,
+    then the skinny kernel with the same split of K; the automatic choice
+    without the flag runs the grouped kernel, whose partial sums are added in
+    another order)."""
     M, N, K = 16, 1024, 4096
     g = np.random.default_rng(23)
     x = g.standard_normal((M, K), dtype=np.float32).astype(np.float16)
     w = synthetic.weights_f16(N, K, 0.02, g)
     hi, lo = pg.nestedfp_split(_to(w))
     xt = _to(x)
+    fused, split = pg.fp8_linear_dynamic_plan(M, N, K, torch.float16, flags=pg.FLAG_FUSED_QUANT)
+    assert fused
     y_f = pg.nestedfp_linear(xt, hi, None, mode=pg.NESTED_FP8, flags=pg.FLAG_FUSED_QUANT)
-    y_s = pg.nestedfp_linear(xt, hi, None, mode=pg.NESTED_FP8)
+    y_s = pg.nestedfp_linear(xt, hi, None, mode=pg.NESTED_FP8, path=pg.PATH_SKINNY, split_k=split)
     torch.cuda.synchronize()
     assert pg.device_status() == pg.OK
     np.testing.assert_array_equal(_bits(y_f), _bits(y_s))

@@ -145,3 +145,60 @@ def test_group_several_large_layers_after_a_producer():
     assert pg.device_status() == pg.OK
     for i, (layer, (x, w)) in enumerate(zip(layers, host)):
         _check_layer(i, layer, x, w)
+
+
+def _oracle_linear_threaded(aq, sa, wq, sw):
+    """The oracle's binary64 layer, its output channels split over host
+    threads (the oracle is a C library called through ctypes, which releases
+    the interpreter lock; the arithmetic is unchanged)."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    n = wq.shape[0]
+    parts = [p for p in np.array_split(np.arange(n), os.cpu_count() or 1) if p.size]
+    with ThreadPoolExecutor(len(parts)) as ex:
+        outs = list(ex.map(lambda p: oracle.fp8_linear(aq, sa, wq[p[0]:p[-1] + 1], sw[p[0]:p[-1] + 1]), parts))
+    return np.concatenate(outs, axis=1)
+
+
+@pytest.mark.slow
+def test_group_llama70b_streaming_layers_full_size_sampled():
+    """The llama70b step's weight-streaming part at full size: the four 70B
+    shapes at M = 1, 2, ..., 256 (36 layers, the benchmark's two grouped
+    launches), codes and scales of every layer bit-exact, outputs of every
+    token on 64 sampled output channels per layer within the bound."""
+    wl = synthetic.WORKLOADS["llama70b"]
+    ms = [m for m in wl.ms if m <= 256]
+    weights = {}
+    for si, (K, N, _) in enumerate(wl.shapes):
+        w = synthetic.weights("llama70b", si)
+        wq, sw = pg.fp8_quantize_rows(torch.from_numpy(w).to(DEV))
+        weights[si] = (w, wq, sw)
+    layers, host = [], []
+    for mi, M in enumerate(ms):
+        for si, (K, N, _) in enumerate(wl.shapes):
+            x = synthetic.acts("llama70b", si, mi)
+            w, wq, sw = weights[si]
+            y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+            ws = torch.zeros(pg.fp8_linear_dynamic_workspace_size(M, N, K), dtype=torch.uint8, device=DEV)
+            layers.append((torch.from_numpy(x).to(DEV), wq, sw, y, ws))
+            host.append((x, si))
+    grp = pg.LayerGroup(layers)
+    grp.run()
+    torch.cuda.synchronize()
+    assert pg.device_status() == pg.OK
+    rng = np.random.default_rng(4)
+    wq0s = {}
+    for i, (layer, (x, si)) in enumerate(zip(layers, host)):
+        w = weights[si][0]
+        if si not in wq0s:
+            ns = np.sort(rng.choice(w.shape[0], 64, replace=False))
+            wq0s[si] = (ns,) + oracle.quantize_rows(w[ns])
+        ns, wq0, sw0 = wq0s[si]
+        M, K = x.shape
+        aq0, sa0 = oracle.quantize_rows(x)
+        aq, sa = pg.dynamic_workspace_views(layer[4], M, K)
+        assert np.array_equal(aq.cpu().numpy(), aq0), f"layer {i}: codes"
+        assert np.array_equal(sa.cpu().numpy().view(np.uint32), sa0.view(np.uint32)), f"layer {i}: scales"
+        ref = _oracle_linear_threaded(aq0, sa0, wq0, sw0)
+        bound = linear_bound(ref, K, fp8_row_max(aq0, sa0), fp8_row_max(wq0, sw0))
+        assert_within(layer[3].float().cpu().numpy()[:, ns], ref, bound, f"70B layer {i} (M={M}, shape {si})")

@@ -41,7 +41,7 @@ def _run(x16, hi, lo, mode, **kw):
 
 
 RAGGED = [(1, 16, 16), (5, 48, 144), (16, 272, 528), (17, 144, 1040), (128, 256, 256), (130, 272, 400),
-          (257, 528, 192)]
+          (200, 400, 1040), (256, 144, 272), (257, 528, 192)]
 
 
 @pytest.mark.parametrize("M,N,K", RAGGED)
@@ -51,7 +51,9 @@ def test_nested_fp16_ragged(M, N, K):
     w16 = synthetic.weights_f16(N, K, 0.02, g)
     hi, lo = oracle.nestedfp_split(w16)
     ref, bound = _ref16(x16, hi, lo)
-    configs = [{"path": pg.PATH_TILED}, {"path": pg.PATH_TILED, "split_k": 2}, {"path": pg.PATH_TILED, "tile_n": 256}]
+    configs = [{}, {"path": pg.PATH_TILED}, {"path": pg.PATH_TILED, "split_k": 2},
+               {"path": pg.PATH_TILED, "tile_n": 256},
+               {"path": pg.PATH_TILED_PAIR}]   # {}: automatic (grouped kernel for M <= 256)
     if M <= 128:
         configs += [{"path": pg.PATH_SKINNY}, {"path": pg.PATH_SKINNY, "split_k": 3}]
     for kw in configs:
@@ -65,7 +67,7 @@ def test_nested_fp8_ragged(M, N, K):
     w16 = synthetic.weights_f16(N, K, 0.02, g)
     hi, _ = oracle.nestedfp_split(w16)
     ref, bound, _, _ = _ref8(x16, hi)
-    configs = [{"path": pg.PATH_TILED}, {"path": pg.PATH_TILED, "split_k": 2}, {"path": pg.PATH_TILED_PAIR}]
+    configs = [{}, {"path": pg.PATH_TILED}, {"path": pg.PATH_TILED, "split_k": 2}, {"path": pg.PATH_TILED_PAIR}]
     if M <= 128:
         configs += [{"path": pg.PATH_SKINNY}, {"path": pg.PATH_SKINNY, "split_k": 4}]
     for kw in configs:
@@ -84,9 +86,27 @@ def test_nested_fp16_identity_weights():
     w[np.arange(K), (np.arange(K) + 1) % K] = np.float16(2.0 ** -20)   # exercises lo bits (subnormal)
     hi, lo = oracle.nestedfp_split(w)
     ref, bound = _ref16(x16, hi, lo)
-    for kw in ({"path": pg.PATH_TILED}, {"path": pg.PATH_SKINNY}):
+    for kw in ({"path": pg.PATH_TILED}, {"path": pg.PATH_SKINNY}, {"path": pg.PATH_TILED_PAIR}):
         y = _run(x16, hi, lo, pg.NESTED_FP16, **kw)
         assert_within(y, ref, bound, str(kw))
+
+
+@pytest.mark.parametrize("M,N,K", [(600, 784, 528), (2200, 2208, 272), (1030, 4096, 1040)])
+def test_nested_fp16_pair_kernel(M, N, K):
+    """FP16 mode on SM pairs: each CTA of a pair rebuilds its half of the
+    256-row weight tile; the MMA reads both halves.  Cases: a few tiles per
+    pair, more tiles than pairs (a second round), and enough tiles for the
+    automatic choice to take the pair kernel; ragged M and N throughout."""
+    g = np.random.default_rng(M + 3 * N + K)
+    x16 = synthetic.activations("normal_f16", M, K, g)
+    w16 = synthetic.weights_f16(N, K, 0.02, g)
+    hi, lo = oracle.nestedfp_split(w16)
+    ref, bound = _ref16(x16, hi, lo)
+    first = _run(x16, hi, lo, pg.NESTED_FP16, path=pg.PATH_TILED_PAIR)
+    assert_within(first, ref, bound, f"fp16 pair M{M} N{N} K{K}")
+    again = _run(x16, hi, lo, pg.NESTED_FP16, path=pg.PATH_TILED_PAIR, flags=pg.FLAG_OVERLAP_PREVIOUS)
+    np.testing.assert_array_equal(first, again)
+    assert_within(_run(x16, hi, lo, pg.NESTED_FP16), ref, bound, f"fp16 auto M{M} N{N} K{K}")
 
 
 @pytest.mark.parametrize("shape_idx", [0, 1])
@@ -170,3 +190,51 @@ def test_nested_streamk(M, N, K, mode):
     for _ in range(2):
         y = _run(x16, hi, lo if m == pg.NESTED_FP16 else None, m, workspace=ws, path=pg.PATH_STREAMK)
         assert_within(y, ref, bound, f"{mode} stream-K M{M} N{N} K{K}")
+
+
+NESTED_GROUP = [(1, 528, 512), (16, 272, 1040), (17, 400, 144), (64, 1040, 528), (128, 256, 256),
+                (130, 272, 400), (256, 144, 272), (300, 528, 192)]   # (M, N, K): every token class, one layer past it
+
+
+@pytest.mark.parametrize("mode", ["fp16", "fp8"])
+def test_nested_group_matches_the_oracle(mode):
+    """pgf8_nestedfp_linear_group: layers of every token-tile class in one
+    group (two grouped launches) and one past it, run twice: every layer
+    within the bound of the oracle's, FP8 mode's codes and scales bit-exact,
+    the second call bit-identical, the flags left zero."""
+    m = pg.NESTED_FP16 if mode == "fp16" else pg.NESTED_FP8
+    g = np.random.default_rng(41 if mode == "fp16" else 43)
+    entries, host = [], []
+    for (M, N, K) in NESTED_GROUP:
+        x16 = synthetic.activations("normal_f16", M, K, g)
+        w16 = synthetic.weights_f16(N, K, 0.02, g)
+        hi, lo = oracle.nestedfp_split(w16)
+        y = torch.full((M, N), float("nan"), dtype=torch.float16, device=DEV)
+        ws = None
+        if m == pg.NESTED_FP8:
+            ws = torch.zeros(pg.nestedfp_linear_workspace_size(M, N, K, m), dtype=torch.uint8, device=DEV)
+        entries.append((_to(x16), _to(hi), _to(lo) if m == pg.NESTED_FP16 else None, y, ws))
+        host.append((x16, hi, lo))
+    grp = pg.NestedLayerGroup(entries, mode=m)
+    grp.run()
+    torch.cuda.synchronize()
+    assert pg.device_status() == pg.OK
+    first = [e[3].clone() for e in entries]
+    for i, ((xt, _, _, y, ws), (x16, hi, lo)) in enumerate(zip(entries, host)):
+        M, K = x16.shape
+        if m == pg.NESTED_FP16:
+            ref, bound = _ref16(x16, hi, lo)
+        else:
+            ref, bound, aq0, sa0 = _ref8(x16, hi)
+            aq, sa = pg.dynamic_workspace_views(ws, M, K)
+            assert np.array_equal(aq.cpu().numpy(), aq0), f"layer {i}: codes"
+            assert np.array_equal(sa.cpu().numpy().view(np.uint32), sa0.view(np.uint32)), f"layer {i}: scales"
+        assert_within(y.float().cpu().numpy(), ref, bound, f"{mode} group layer {i} (M={M})")
+    for e in entries:
+        e[3].fill_(float("nan"))
+    grp.run(flags=pg.FLAG_OVERLAP_PREVIOUS)
+    torch.cuda.synchronize()
+    assert pg.device_status() == pg.OK
+    for i, (e, f) in enumerate(zip(entries, first)):
+        assert torch.equal(e[3].view(torch.int16), f.view(torch.int16)), f"layer {i} differs on the second call"
+    assert not grp.group_workspace[:1024].any(), "flag words not cleared"
