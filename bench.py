@@ -67,7 +67,16 @@ WORKLOAD_TEXT = {
     "small": "single FP8 linear 16x512x512",
     "nested7b": "NestedFP 7B: 4096->12288 and 11008->4096 at M=1,16,128,1024, FP16 and FP8 modes on the "
                 "same hi/lo planes; fp16 out",
+    "nested7b_decode": "NestedFP 7B decode: the nested7b shapes at its decode sizes M=1,16, three weight copies "
+                       "(so a step streams more than 3 x L2), FP16 and FP8 modes; fp16 out",
 }
+
+# bench-only workloads: a subset of a seeded workload's layers (same inputs)
+BASE_WORKLOAD = {"nested7b_decode": "nested7b"}
+
+
+def base_workload(name):
+    return BASE_WORKLOAD.get(name, name)
 
 
 def _load_peaks():
@@ -107,13 +116,22 @@ class Layer:
 
 
 def workload_layers(name, copies):
-    wl = synthetic.WORKLOADS[name]
+    wl = synthetic.WORKLOADS[base_workload(name)]
     layers = []
     if name == "nested7b":
         for mi, M in enumerate(wl.ms):
             for si, (K, N, _) in enumerate(wl.shapes):
                 for kind in ("nested16", "nested8"):
                     layers.append(Layer(kind, M, K, N, si, mi, 0))
+        return layers
+    if name == "nested7b_decode":
+        for c in range(copies):
+            for mi, M in enumerate(wl.ms):
+                if M > 16:
+                    continue
+                for si, (K, N, _) in enumerate(wl.shapes):
+                    for kind in ("nested16", "nested8"):
+                        layers.append(Layer(kind, M, K, N, si, mi, c))
         return layers
     for mi, M in enumerate(wl.ms):
         for si, (K, N, _) in enumerate(wl.shapes):
@@ -123,7 +141,7 @@ def workload_layers(name, copies):
 
 def weight_copies(name):
     # enough distinct weight copies that a step streams more than 3 x L2
-    return {"decode7b": 3, "small": 1}.get(name, 1)
+    return {"decode7b": 3, "nested7b_decode": 3, "small": 1}.get(name, 1)
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -290,12 +308,12 @@ def setup_workload(pg, torch, dev, name):
         key = (L.shape_idx, L.copy, L.kind in ("nested16", "nested8"))
         if key in weights:
             continue
-        w = torch.from_numpy(synthetic.weights(name, L.shape_idx, copy=L.copy)).to(dev)
+        w = torch.from_numpy(synthetic.weights(base_workload(name), L.shape_idx, copy=L.copy)).to(dev)
         weights[key] = pg.nestedfp_split(w) if key[2] else pg.fp8_quantize_rows(w)
         del w
     acts_host, acts, outs, qbufs = [], [], [], []
     for L in layers:
-        x = synthetic.acts(name, L.shape_idx, L.m_idx)
+        x = synthetic.acts(base_workload(name), L.shape_idx, L.m_idx)
         xh = torch.from_numpy(x).pin_memory()
         acts_host.append(xh)
         acts.append(xh.to(dev))
@@ -569,11 +587,11 @@ def analyse_segments(layers, marks, ms_step, peaks, fp8_peak):
     roof["algorithmic_per_step"] = (f"{cls_flops[dom]:.4e} flop" if roof["bound"] == "tensor"
                                     else f"{cls_bytes[dom]:.4e} B")
 
-    def regime(pred, what):
+    def regime(pred, what, kind=None):
         t_s = wbytes = fl = ideal = 0.0
         for sg in segs:
             Ls = [layers[i] for i in sg["layers"]]
-            if Ls and all(pred(L.M) for L in Ls):
+            if Ls and all(pred(L.M) and (kind is None or L.kind == kind) for L in Ls):
                 t_s += sg["ms"] * scale * 1e-3
                 if sg["kind"] != "quant":
                     wbytes += sum(L.weight_bytes for L in Ls)
@@ -600,6 +618,14 @@ def analyse_segments(layers, marks, ms_step, peaks, fp8_peak):
             r["target"] = target
             r["pass"] = bool(frac >= target)
             regimes[key] = r
+    # NestedFP: the decode regime of each mode on its own
+    for kind, tag in (("nested16", "fp16_mode"), ("nested8", "fp8_mode")):
+        if any(L.kind == kind for L in layers):
+            r = regime(lambda m: m <= 16, "hbm", kind)
+            if r is not None:
+                r["target"] = 0.80
+                r["pass"] = bool(r["frac_hbm"] >= 0.80)
+                regimes["decode_m_le_16_" + tag] = r
     return roof, regimes, out
 
 
@@ -690,7 +716,7 @@ def run_ours(args, rank, world, local_rank):
     wbytes, flops = res["wbytes"], res["flops"]
     gbs = job_throughput(wbytes / 1e9, world, ms_step * 1e-3)        # whole job, all ranks
     tflops = job_throughput(flops / 1e12, world, ms_step * 1e-3)
-    memory_bound = name in ("decode7b", "small")
+    memory_bound = name in ("decode7b", "nested7b_decode", "small")
     roof = res["roof"]
     roof["traffic"], roof["traffic_note"] = profiled_traffic(name)
     if fp8_peak is not None:
@@ -744,11 +770,11 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- the other configurations, each timed as its own step in this run
     if not args.no_secondary and name == "llama70b":
-        for sec in ("decode7b", "prefill7b", "nested7b"):
+        for sec in ("decode7b", "prefill7b", "nested7b", "nested7b_decode"):
             wl2 = setup_workload(pg, torch, dev, sec)
-            steps2 = {"decode7b": 400, "prefill7b": 60, "nested7b": 60}[sec]
+            steps2 = {"decode7b": 400, "prefill7b": 60, "nested7b": 60, "nested7b_decode": 200}[sec]
             r2 = time_workload(pg, torch, dev, wl2, args, steps2, 10, world, peaks, fp8_peak)
-            mb = sec == "decode7b"
+            mb = sec in ("decode7b", "nested7b_decode")
             v = (r2["wbytes"] / 1e9 if mb else r2["flops"] / 1e12) / (r2["ms_step"] * 1e-3) * world
             result["secondary"][sec] = {
                 "value": round(v, 2), "unit": "GB/s" if mb else "TFLOP/s", "ms_per_step": round(r2["ms_step"], 5),
@@ -852,7 +878,7 @@ def run_e2e(pg, torch, dev, wl, args, world, wbytes, flops, memory_bound):
 
 # ----------------------------------------------------------------------------- CPU oracle
 ORACLE_SAMPLE = {  # per layer: first `rows` tokens x first `cols` output channels
-    "small": (16, 512), "decode7b": (8, 256), "prefill7b": (16, 48), "nested7b": (16, 96), "llama70b": (16, 64),
+    "small": (16, 512), "decode7b": (8, 256), "prefill7b": (16, 48), "nested7b": (16, 96), "nested7b_decode": (16, 96), "llama70b": (16, 64),
 }
 
 
@@ -868,9 +894,9 @@ def oracle_inputs(name, rows=None, cols=None):
     items = []
     for L in workload_layers(name, weight_copies(name)):
         m = min(rows, L.M)
-        x = synthetic.acts(name, L.shape_idx, L.m_idx, M=m)
+        x = synthetic.acts(base_workload(name), L.shape_idx, L.m_idx, M=m)
         nc = min(cols, L.N)
-        w = synthetic.weights(name, L.shape_idx, copy=L.copy, n_override=nc)
+        w = synthetic.weights(base_workload(name), L.shape_idx, copy=L.copy, n_override=nc)
         prep = oracle.quantize_rows(w) if L.kind == "fp8" else oracle.nestedfp_split(w)
         items.append((L, x, prep))
     desc = (f"all {len(items)} layers of one step, each on its first {rows} tokens (quantised over the full K) x "
@@ -944,7 +970,7 @@ def run_reference(args):
     from concurrent.futures import ThreadPoolExecutor
 
     name = args.workload
-    memory_bound = name in ("decode7b", "small")
+    memory_bound = name in ("decode7b", "nested7b_decode", "small")
     threads = os.cpu_count() or 1
     r0, c0 = ORACLE_SAMPLE[name]
     with ThreadPoolExecutor(threads) as pool:
@@ -1195,7 +1221,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(synthetic.WORKLOADS), default="llama70b")
+    ap.add_argument("--workload", choices=sorted(synthetic.WORKLOADS) + sorted(BASE_WORKLOAD), default="llama70b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true",
                     help="llama70b: skip timing decode7b, prefill7b and nested7b as secondary steps")

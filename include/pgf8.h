@@ -549,9 +549,12 @@ pgf8_status pgf8_nestedfp_split(const void *w_f16, int64_t N, int64_t K, uint8_t
  *     y = fp16_rn( (sum_k e4m3(aq[m,k]) * e5m2(hi[n,k])) * sa[m] ): the upper
  *     byte is read as an E5M2 code with unit scale, which is the FP16 weight
  *     with its low 8 bits cleared.  lo is ignored and may be NULL.
- * With the automatic kernel choice, M <= 256 runs the grouped
- * weight-streaming kernel on this one layer (every SM streams an equal
- * share of the weight planes); larger M runs the tiled kernels.
+ * With the automatic kernel choice, M <= 16 runs the split-K skinny
+ * kernel, 16 < M <= 256 the grouped weight-streaming kernel on this one
+ * layer (every SM streams an equal share of the weight planes), larger M
+ * the tiled kernels (FP16 mode: the one-CTA persistent kernel; its SM-pair
+ * form, PGF8_PATH_TILED_PAIR, measured slower).  Several layers of one
+ * mode: pgf8_nestedfp_linear_group.
  * ---------------------------------------------------------------------- */
 pgf8_status pgf8_nestedfp_linear(const void *x_f16, int64_t M, int64_t K, const uint8_t *hi,
                                  const uint8_t *lo, int64_t N, pgf8_nested_mode mode,

@@ -10,10 +10,12 @@
 //   S = Q_codes . K_codes^T              (Q quantised per (token, head) row
 //                                         beforehand by the row quantiser)
 //   P = E4M3(2^8 . exp2(S . sq . sk . log2(e)/sqrt(D) - m))   (online softmax)
-//   O = P . V_codes . 2^-8 . sv / l
-// l sums the unrounded probabilities.  head_dim 128.
+//   O = P . V_codes . sv / l
+// l sums the unrounded probabilities times 2^8 (the code scale cancels in
+// O; scaling by a power of two leaves the sum's rounding unchanged).
+// head_dim 128.
 //
-// One CTA per (128-query tile, query head, sequence), heaviest tiles first, 320 threads:
+// One CTA per (128-query tile, query head, sequence), heaviest tiles first, 576 threads:
 //   warp 0      TMA: the Q tile once, then per 128-key tile eight 16-row
 //               pieces of K and of V straight from the paged cache (a piece
 //               past the context, or of an out-of-range block, is read at a
@@ -21,16 +23,18 @@
 //   warp 1      TMEM (512 columns: S double buffer, PV double buffer) and
 //               the MMA issue: S_j = Q K_j^T, then PV_{j-1} = P_{j-1} V_{j-1}
 //               (V as an MN-major operand: the cache rows are d-contiguous);
-//   warps 2-9   two threads per query row (warps 2-5: keys / head-dim
-//               columns 0-63 of their TMEM lane quadrant, warps 6-9: columns
-//               64-127): scores from TMEM (two passes), causal and validity
-//               masks, online softmax in base 2 (the two halves' maxima
-//               exchanged through shared memory at a named barrier), P codes
-//               written into shared memory in the 128-byte-swizzled K-major
-//               layout, PV_{j-1} added into registers one tile late (so the
-//               PV MMA overlaps the next softmax), final 1/l and scales.
-//               Every barrier of these 8 warps also ANDs their wait results,
-//               so they leave the loop together when one of them gives up.
+//   warps 2-17  four threads per query row: warp w takes keys (and
+//               head-dim columns) 32 * ((w - 2) / 4) .. + 31 of TMEM lane
+//               quadrant w % 4: scores from TMEM (two passes), causal and
+//               validity masks (skipped for key tiles wholly below the
+//               query tile with every piece present), online softmax in
+//               base 2 (the four parts' maxima exchanged through shared
+//               memory at a named barrier), P codes written into shared
+//               memory in the 128-byte-swizzled K-major layout, PV_{j-1}
+//               added into registers one tile late (so the PV MMA overlaps
+//               the next softmax), final 1/l and scales.  Every barrier of
+//               these 16 warps also ANDs their wait results, so they leave
+//               the loop together when one of them gives up.
 // Every wait is bounded: a wait that gives up raises the CTA's abort flag
 // and the device error word; in-flight copies and MMAs are drained before
 // the CTA frees its TMEM and exits.
@@ -48,10 +52,12 @@ constexpr int kCtxK = kCtxQ + kCtxTile;
 constexpr int kCtxV = kCtxK + kCtxStages * kCtxTile;
 constexpr int kCtxP = kCtxV + kCtxStages * kCtxTile;
 constexpr int kCtxCtl = kCtxP + 2 * kCtxTile;
-constexpr int kCtxRed = kCtxCtl + 1024;         // [2 parities][2 halves][128 rows] f32: row-max exchange
-constexpr int kCtxSmemBytes = kCtxRed + 2048 + 1024 /*alignment slack*/;
-constexpr int kCtxThreads = 320;                 // producer, MMA, 8 softmax warps
-constexpr int kCtxSoftmaxThreads = 256;
+constexpr int kCtxParts = 4;                     // softmax threads per query row (32 columns each)
+constexpr int kCtxCols = 128 / kCtxParts;
+constexpr int kCtxRed = kCtxCtl + 1024;         // [2 parities][parts][128 rows] f32: row-max exchange
+constexpr int kCtxSmemBytes = kCtxRed + 2 * kCtxParts * 128 * 4 + 1024 /*alignment slack*/;
+constexpr int kCtxSoftmaxThreads = 128 * kCtxParts;
+constexpr int kCtxThreads = 64 + kCtxSoftmaxThreads;   // producer, MMA, softmax warps
 constexpr uint32_t kCtxTmemCols = 512;
 static_assert(kCtxSmemBytes <= 227 * 1024, "shared memory");
 
@@ -155,7 +161,17 @@ __device__ __forceinline__ int ctx_piece_row(const AttnCtxParams &p, int64_t s, 
     return static_cast<int>((blk * p.Hkv + hk) * p.B + key % p.B);
 }
 
-// AND of v over the 8 softmax warps (named barrier 1): also the barrier at
+// 2^x by the special-function unit (ex2.approx.ftz: a relative error of a
+// few binary32 ulps, far below the E4M3 rounding of the probabilities that
+// follows; -inf -> 0).
+__device__ __forceinline__ float ex2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// AND of v over the softmax warps (named barrier 1): also the barrier at
 // which they exchange row maxima through shared memory.
 __device__ __forceinline__ bool ctx_softmax_all(bool v)
 {
@@ -163,10 +179,10 @@ __device__ __forceinline__ bool ctx_softmax_all(bool v)
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.and.pred q, 1, 256, p;\n\t"
+        "bar.red.and.pred q, 1, %2, p;\n\t"
         "selp.u32 %0, 1, 0, q;\n\t}\n"
         : "=r"(r)
-        : "r"(static_cast<uint32_t>(v))
+        : "r"(static_cast<uint32_t>(v)), "n"(kCtxSoftmaxThreads)
         : "memory");
     return r != 0;
 }
@@ -216,10 +232,10 @@ __global__ void __launch_bounds__(kCtxThreads, 1) attn_context_kernel(const __gr
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->s_full[b], 1);
-            mbar_init(&ctl->s_free[b], 8);    // one arrival per softmax warp
-            mbar_init(&ctl->p_full[b], 8);
+            mbar_init(&ctl->s_free[b], kCtxSoftmaxThreads / 32);   // one arrival per softmax warp
+            mbar_init(&ctl->p_full[b], kCtxSoftmaxThreads / 32);
             mbar_init(&ctl->o_full[b], 1);
-            mbar_init(&ctl->o_free[b], 8);
+            mbar_init(&ctl->o_free[b], kCtxSoftmaxThreads / 32);
         }
         mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
@@ -315,21 +331,21 @@ __global__ void __launch_bounds__(kCtxThreads, 1) attn_context_kernel(const __gr
     } else {
         // ---------------------------------------------------------------- softmax (two threads per query row)
         const int qd = warp & 3;                          // TMEM lane quadrant of this warp
-        const int half = (warp - 2) >> 2;                 // 0: columns 0-63, 1: columns 64-127
+        const int part = (warp - 2) >> 2;                 // columns part * kCtxCols .. + kCtxCols - 1
         const int r = qd * 32 + lane;                     // query row of the tile
-        const int et = static_cast<int>(threadIdx.x) - 64;   // 0 .. 255
-        const int c_lo = half * 64;
+        const int et = static_cast<int>(threadIdx.x) - 64;   // 0 .. kCtxSoftmaxThreads - 1
+        const int c_lo = part * kCtxCols;
         const bool row_ok = r < nrows;
         const int pos = pos0 + r;
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
-        float *red = reinterpret_cast<float *>(smem + kCtxRed);   // [parity][half][row]
+        float *red = reinterpret_cast<float *>(smem + kCtxRed);   // [parity][part][row]
         const float scale = row_ok ? p.q_scales[(static_cast<int64_t>(q0) + qt * 128 + r) * p.Hq + h] * p.sk[hk] *
                                          (1.4426950408889634f * 0.08838834764831845f)   // log2(e) / sqrt(128)
                                    : 0.0f;
-        float m = -INFINITY, l = 0.0f, alpha_prev = 0.0f;   // l: this half's share of the row sum
-        float o[64];                                         // head-dim columns c_lo .. c_lo + 63
+        float m = -INFINITY, l = 0.0f, alpha_prev = 0.0f;   // l: this part's share of the row sum
+        float o[kCtxCols];                                   // head-dim columns c_lo .. c_lo + kCtxCols - 1
 #pragma unroll
-        for (int d = 0; d < 64; ++d)
+        for (int d = 0; d < kCtxCols; ++d)
             o[d] = 0.0f;
         bool ok = true;
 
@@ -341,7 +357,7 @@ __global__ void __launch_bounds__(kCtxThreads, 1) attn_context_kernel(const __gr
                 return false;
             tc_fence_after();
 #pragma unroll
-            for (int c0 = 0; c0 < 64; c0 += 16) {
+            for (int c0 = 0; c0 < kCtxCols; c0 += 16) {
                 uint32_t v[16];
                 tmem_ld_32x32b_x16(t_lane + 256 + b * 128 + c_lo + c0, v);
                 tmem_ld_wait();
@@ -372,56 +388,88 @@ __global__ void __launch_bounds__(kCtxThreads, 1) attn_context_kernel(const __gr
             }
             const bool w = wait_bounded(&ctl->s_full[b], static_cast<uint32_t>(k) & 1u, abort_flag);
             const uint32_t t_s = t_lane + b * 128 + c_lo;
-            // pass 1: the maximum of this half's valid scores, exchanged with the other half's
+            // Key tiles wholly below the tile's first query and with all eight
+            // pieces present need no mask (CTA-uniform).  Rows past the
+            // prompt (row_ok false) are then computed unmasked as well: their
+            // P and O rows are never stored, and nothing mixes rows.
+            const bool unmasked = piece_ok == 0xFFu && j * 128 + 127 <= pos0;
+            // pass 1: the maximum of this part's valid scores, exchanged with the other parts'
             float mx = -INFINITY;
             if (w) {
                 tc_fence_after();
+                if (unmasked) {
+                    float vmax = -INFINITY;
 #pragma unroll 1
-                for (int c0 = 0; c0 < 64; c0 += 16) {
-                    uint32_t v[16];
-                    tmem_ld_32x32b_x16(t_s + c0, v);
-                    tmem_ld_wait();
-                    const bool pok = (piece_ok >> ((c_lo + c0) >> 4)) & 1u;
+                    for (int c0 = 0; c0 < kCtxCols; c0 += 16) {
+                        uint32_t v[16];
+                        tmem_ld_32x32b_x16(t_s + c0, v);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int key = j * 128 + c_lo + c0 + e;
-                        const float sc = __uint_as_float(v[e]) * scale;
-                        mx = (pok && row_ok && key <= pos) ? fmaxf(mx, sc) : mx;
+                        for (int e = 0; e < 16; ++e)
+                            vmax = fmaxf(vmax, __uint_as_float(v[e]));
+                    }
+                    mx = vmax * scale;   // scale >= 0: rounding is monotone, the maximum commutes
+                } else {
+#pragma unroll 1
+                    for (int c0 = 0; c0 < kCtxCols; c0 += 16) {
+                        uint32_t v[16];
+                        tmem_ld_32x32b_x16(t_s + c0, v);
+                        tmem_ld_wait();
+                        const bool pok = (piece_ok >> ((c_lo + c0) >> 4)) & 1u;
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const int key = j * 128 + c_lo + c0 + e;
+                            const float sc = __uint_as_float(v[e]) * scale;
+                            mx = (pok && row_ok && key <= pos) ? fmaxf(mx, sc) : mx;
+                        }
                     }
                 }
             }
-            float *red_j = red + (j & 1) * 256;
-            red_j[half * 128 + r] = mx;
+            float *red_j = red + (j & 1) * (kCtxParts * 128);
+            red_j[part * 128 + r] = mx;
             if (!ctx_softmax_all(w)) {
                 ok = false;
                 break;
             }
-            mx = fmaxf(mx, red_j[(half ^ 1) * 128 + r]);
+#pragma unroll
+            for (int q = 0; q < kCtxParts; ++q)
+                mx = fmaxf(mx, red_j[q * 128 + r]);
             const float mn = fmaxf(m, mx);
-            const float alpha = m == -INFINITY ? 0.0f : exp2f(m - mn);
-            // pass 2: probabilities, their codes (x 2^8) into P buffer b, this half's row sum
+            const float alpha = m == -INFINITY ? 0.0f : ex2_approx(m - mn);
+            // pass 2: the probabilities times 2^8 (the E4M3 code scale, folded
+            // into the exponent), their codes into P buffer b, this part's
+            // row sum (in the same units)
+            const float nm8 = 8.0f - mn;
             float rs = 0.0f;
             uint8_t *prow = smem + kCtxP + b * kCtxTile + r * 128;
 #pragma unroll 1
-            for (int c0 = 0; c0 < 64; c0 += 16) {
+            for (int c0 = 0; c0 < kCtxCols; c0 += 16) {
                 uint32_t v[16];
                 tmem_ld_32x32b_x16(t_s + c0, v);
                 tmem_ld_wait();
                 const int cc = c_lo + c0;
-                const bool pok = (piece_ok >> (cc >> 4)) & 1u;
                 float pr[16];
+                if (unmasked) {
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int key = j * 128 + cc + e;
-                    const bool valid = pok && row_ok && key <= pos;
-                    pr[e] = valid ? exp2f(__uint_as_float(v[e]) * scale - mn) : 0.0f;
-                    rs += pr[e];
+                    for (int e = 0; e < 16; ++e) {
+                        pr[e] = ex2_approx(fmaf(__uint_as_float(v[e]), scale, nm8));
+                        rs += pr[e];
+                    }
+                } else {
+                    const bool pok = (piece_ok >> (cc >> 4)) & 1u;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int key = j * 128 + cc + e;
+                        const bool valid = pok && row_ok && key <= pos;
+                        pr[e] = valid ? ex2_approx(fmaf(__uint_as_float(v[e]), scale, nm8)) : 0.0f;
+                        rs += pr[e];
+                    }
                 }
                 uint32_t wv[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
-                    wv[u] = static_cast<uint32_t>(cvt_e4m3x2(pr[4 * u] * 256.0f, pr[4 * u + 1] * 256.0f)) |
-                            (static_cast<uint32_t>(cvt_e4m3x2(pr[4 * u + 2] * 256.0f, pr[4 * u + 3] * 256.0f)) << 16);
+                    wv[u] = static_cast<uint32_t>(cvt_e4m3x2(pr[4 * u], pr[4 * u + 1])) |
+                            (static_cast<uint32_t>(cvt_e4m3x2(pr[4 * u + 2], pr[4 * u + 3])) << 16);
                 *reinterpret_cast<uint4 *>(prow + (((cc >> 4) ^ (r & 7)) << 4)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
             }
             tc_fence_before();
@@ -460,15 +508,18 @@ __global__ void __launch_bounds__(kCtxThreads, 1) attn_context_kernel(const __gr
             ok = accumulate(nkt - 1, alpha_prev);
         if (ok) {
             // the row sum: both halves add the two shares in the same order
-            float *red_l = red + (nkt & 1) * 256;
-            red_l[half * 128 + r] = l;
+            float *red_l = red + (nkt & 1) * (kCtxParts * 128);
+            red_l[part * 128 + r] = l;
             ctx_softmax_all(true);
-            const float lsum = red_l[r] + red_l[128 + r];
+            float lsum = 0.0f;
+#pragma unroll
+            for (int q = 0; q < kCtxParts; ++q)   // the same order in every part
+                lsum += red_l[q * 128 + r];
             if (row_ok) {
-                const float f = lsum > 0.0f ? p.sv[hk] * 0.00390625f / lsum : 0.0f;   // 2^-8 undoes the P code scale
+                const float f = lsum > 0.0f ? p.sv[hk] / lsum : 0.0f;   // P and l both carry the 2^8
                 const int64_t base =
                     (static_cast<int64_t>(q0) + qt * 128 + r) * p.ldo + static_cast<int64_t>(h) * 128 + c_lo;
-                store_row<64>(p.out, base, p.odt, p.vec_out != 0, o, f);
+                store_row<kCtxCols>(p.out, base, p.odt, p.vec_out != 0, o, f);
             }
         }
     }
