@@ -634,31 +634,6 @@ static pgf8_status quantize_launch(const void *x, pgf8_dtype xdt, int64_t rows, 
     const int qflags = (trigger_early ? kQuantTriggerEarly : 0) | (no_wait ? kQuantNoWait : 0);
     if (rows == 0)
         return PGF8_OK;
-    // The largest shared-memory carveout, as the GEMM kernels run with: a
-    // quantisation that overlaps a running GEMM (trigger_early / no_wait)
-    // can then place its CTAs on the GEMM's SMs, whose L1 / shared split is
-    // already configured that way.
-    static PerDeviceSetup setup;
-    const cudaError_t attr_err = setup_once_per_device(setup, [](int, int *) {
-        const void *kernels[] = {
-            reinterpret_cast<const void *>(quantize_rows_held_kernel<float, 1, 256>),
-            reinterpret_cast<const void *>(quantize_rows_held_kernel<float, 2, 256>),
-            reinterpret_cast<const void *>(quantize_rows_held_kernel<float, 4, 256>),
-            reinterpret_cast<const void *>(quantize_rows_kernel<float>),
-            reinterpret_cast<const void *>(quantize_rows_held_kernel<__half, 1, 256>),
-            reinterpret_cast<const void *>(quantize_rows_held_kernel<__half, 2, 256>),
-            reinterpret_cast<const void *>(quantize_rows_held_kernel<__half, 4, 256>),
-            reinterpret_cast<const void *>(quantize_rows_kernel<__half>)};
-        for (const void *k : kernels) {
-            const cudaError_t e =
-                cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
-            if (e != cudaSuccess)
-                return e;
-        }
-        return cudaSuccess;
-    });
-    if (attr_err != cudaSuccess)
-        return cuda_fail(attr_err);
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(static_cast<unsigned>(rows));
