@@ -66,9 +66,10 @@ WORKLOAD_TEXT = {
                 "at M=1..4096; Student-t(3) activations; bf16 out",
     "small": "single FP8 linear 16x512x512",
     "nested7b": "NestedFP 7B: 4096->12288 and 11008->4096 at M=1,16,128,1024, FP16 and FP8 modes on the "
-                "same hi/lo planes; fp16 out",
-    "nested7b_decode": "NestedFP 7B decode: the nested7b shapes at its decode sizes M=1,16, three weight copies "
-                       "(so a step streams more than 3 x L2), FP16 and FP8 modes; fp16 out",
+                "same hi/lo planes (3 weight copies, one per M but M=1024 sharing the M=1 copy); fp16 out",
+    "nested7b_decode": "NestedFP 7B decode: the nested7b shapes at its decode sizes M=1,16, three times each, "
+                       "every (repeat, M) with its own weight copy (6 copies: no re-read from L2), FP16 and FP8 "
+                       "modes; fp16 out",
 }
 
 # bench-only workloads: a subset of a seeded workload's layers (same inputs)
@@ -122,16 +123,17 @@ def workload_layers(name, copies):
         for mi, M in enumerate(wl.ms):
             for si, (K, N, _) in enumerate(wl.shapes):
                 for kind in ("nested16", "nested8"):
-                    layers.append(Layer(kind, M, K, N, si, mi, 0))
+                    layers.append(Layer(kind, M, K, N, si, mi, mi % copies))
         return layers
     if name == "nested7b_decode":
+        # every (repeat, M) its own weight copy: no layer re-reads planes an
+        # earlier layer of its group left in L2
+        dec = [(mi, M) for mi, M in enumerate(wl.ms) if M <= 16]
         for c in range(copies):
-            for mi, M in enumerate(wl.ms):
-                if M > 16:
-                    continue
-                for si, (K, N, _) in enumerate(wl.shapes):
-                    for kind in ("nested16", "nested8"):
-                        layers.append(Layer(kind, M, K, N, si, mi, c))
+            mi, M = dec[c % len(dec)]
+            for si, (K, N, _) in enumerate(wl.shapes):
+                for kind in ("nested16", "nested8"):
+                    layers.append(Layer(kind, M, K, N, si, mi, c))
         return layers
     for mi, M in enumerate(wl.ms):
         for si, (K, N, _) in enumerate(wl.shapes):
@@ -141,7 +143,7 @@ def workload_layers(name, copies):
 
 def weight_copies(name):
     # enough distinct weight copies that a step streams more than 3 x L2
-    return {"decode7b": 3, "nested7b_decode": 3, "small": 1}.get(name, 1)
+    return {"decode7b": 3, "nested7b": 3, "nested7b_decode": 6, "small": 1}.get(name, 1)
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -200,7 +202,7 @@ class ClockSampler:
 # The GEMM kernels' sources (and the helpers they include): what a DRAM
 # traffic record describes.  The record also names the kernel configuration
 # it was taken on.
-GEMM_SOURCES = ("gemm.cuh", "gemm_2sm.cuh", "gemm_persistent.cuh", "gemm_streamk.cuh", "gemm_group.cuh",
+GEMM_SOURCES = ("gemm.cuh", "gemm_2sm.cuh", "gemm_pair_group.cuh", "gemm_persistent.cuh", "gemm_streamk.cuh", "gemm_group.cuh",
                 "quantize.cuh", "sm100_ptx.cuh")
 
 
@@ -347,10 +349,10 @@ class StepRunner:
     producers) chains one call per layer with PGF8_FLAG_OVERLAP_PREVIOUS.
 
     The bracketed step (for the roofline) runs the same launches with an
-    event between consecutive launch groups: the grouped kernel on the
-    M <= 128 layers and on the 128 < M <= 256 layers, then the quantisation
-    and the GEMM of every larger layer; its intervals are scaled to the
-    timed step."""
+    event between consecutive launch groups: the quantisation and the
+    grouped kernel on the M <= 128 layers, then the quantisation of the
+    larger layers and their tiled launch on SM pairs
+    (pgf8_fp8_linear_group); its intervals are scaled to the timed step."""
 
     def __init__(self, pg, torch, dev, wl, args, stream):
         self.pg, self.torch, self.dev, self.wl, self.args, self.stream = pg, torch, dev, wl, args, stream
@@ -366,14 +368,15 @@ class StepRunner:
         if self.grouped:
             ent = lambda i: (wl["acts"][i], *wl["weights"][_wkey(layers[i])], wl["outs"][i], wl["qbufs"][i])  # noqa: E731
             self.group = pg.LayerGroup([ent(i) for i in range(len(layers))])
-            # the library's launches for a group: the grouped kernel on the
-            # M <= 128 layers and on the 128 < M <= 256 layers (32 per
-            # launch), then each larger layer
-            self.classes = []
-            for lo, hi in ((0, 128), (128, GROUP_MAX_M)):
-                idx = [i for i, L in enumerate(layers) if lo < L.M <= hi]
-                self.classes += [idx[j:j + 32] for j in range(0, len(idx), 32)]
-            self.large = [i for i, L in enumerate(layers) if L.M > GROUP_MAX_M]
+            # the library's launches for a group: the quantisation and the
+            # grouped kernel on the M <= 128 layers (32 per launch), then the
+            # quantisation and the tiled launch on SM pairs over all the
+            # larger layers (32 per launch)
+            small = [i for i, L in enumerate(layers) if L.M <= 128]
+            large = [i for i, L in enumerate(layers) if L.M > 128]
+            self.classes = [small[j:j + 32] for j in range(0, len(small), 32)]
+            self.large_chunks = [large[j:j + 32] for j in range(0, len(large), 32)]
+            self.large = large
             self.sub = [pg.LayerGroup([ent(i) for i in idx]) for idx in self.classes]
         if self.nested_grouped:
             def nent(i):
@@ -413,7 +416,7 @@ class StepRunner:
     # -- launches -------------------------------------------------------------------------------------------------
     def launches_per_step(self):
         if self.grouped:
-            return sum(2 * ((len(c) + 31) // 32) for c in self.classes) + 2 * len(self.large)
+            return 2 * len(self.classes) + 2 * len(self.large_chunks)
         if self.nested_grouped:
             per = lambda i: 2 if self.layers[i].kind == "nested8" else 1  # noqa: E731
             return sum(per(idx[0]) for idx, _ in self.nsub) + sum(per(i) for i in self.nlarge)
@@ -478,13 +481,16 @@ class StepRunner:
             for idx, sub in zip(self.classes, self.sub):
                 mark(("group", tuple(idx)))
                 sub.run(stream=s)
-            for i in self.large:
-                L = self.layers[i]
-                W = wl["weights"][_wkey(L)]
-                mark(("quant", (i,)))
-                aq, sa = self._quantise(i, L, 0)
-                mark(("gemm", (i,)))
-                pg.fp8_linear(aq, sa, W[0], W[1], y=wl["outs"][i], workspace=self.sk_ws, stream=s)
+            for chunk in self.large_chunks:
+                mark(("quant", tuple(chunk)))
+                ops = []
+                for i in chunk:
+                    L = self.layers[i]
+                    W = wl["weights"][_wkey(L)]
+                    aq, sa = self._quantise(i, L, 0)
+                    ops.append((aq, sa, W[0], W[1], wl["outs"][i]))
+                mark(("gemm", tuple(chunk)))
+                pg.fp8_linear_group(ops, stream=s)
         elif self.nested_grouped:
             for idx, sub in self.nsub:
                 mark(("group", tuple(idx)))
@@ -517,22 +523,29 @@ def quant_bytes(L):
     return L.M * L.K * (xb + 1) + 4 * L.M
 
 
-def analyse_segments(layers, marks, ms_step, peaks, fp8_peak):
+def analyse_segments(layers, marks, ms_step, peaks, fp8_peak, long_region=True):
     """Per-segment durations of the bracketed step, scaled so that they sum
     to the timed step (a kernel's share of the step times the step), the
     dominant kernel's roofline and the regime checks of the layer's targets,
     over the segments whose layers all fall in the regime: decode (M <= 16)
-    >= 80 % of HBM; weight streaming (M <= 256, the grouped kernel and the
-    M = 256 layers) >= 75 % of HBM; prefill (M >= 512) >= 60 % of the FP8
-    tensor peak."""
+    >= 80 % of HBM; weight streaming (M <= 128: the grouped kernel; the
+    M = 256 layers join the tiled launch, at the FP8 ridge) >= 75 % of HBM;
+    prefill (M >= 512) >= 60 % of the FP8 tensor peak.
+
+    marks: (segment, event, ms since the previous mark); segment k runs
+    from mark k to mark k + 1.  Tensor peaks: the measured bf16 figure
+    (x 2 for E4M3 MMAs) sustained when the timed region ran long or under
+    the power cap (long_region), else the burst figure."""
     segs = []
-    for (seg, e0), (_, e1) in zip(marks[:-1], marks[1:]):
+    for (seg, _, _), (_, _, dt) in zip(marks[:-1], marks[1:]):
         kind, idx = seg
-        segs.append({"kind": kind, "layers": list(idx), "ms": e0.elapsed_time(e1)})
+        segs.append({"kind": kind, "layers": list(idx), "ms": dt})
     total = sum(sg["ms"] for sg in segs)
     scale = ms_step / total if total > 0 else 1.0
     hbm = float(peaks["hbm_gbs"])
     sustained = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    if not long_region:
+        sustained = float(peaks["bf16_tflops"])   # burst: a short timed region, no power cap seen
     fp8_peak_tf = 2.0 * sustained
     out = []
     cls_time, cls_bytes, cls_flops = {}, {}, {}
@@ -567,8 +580,11 @@ def analyse_segments(layers, marks, ms_step, peaks, fp8_peak):
         peak_eff = cls_flops[dom] / ideal_s / 1e12
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak_eff, 1),
                 "unit": "TFLOP/s", "frac": round(ideal_s / t, 4),
-                "peak_source": "measured bf16 sustained (MEASURED_PEAKS.json) x 2 for E4M3 MMAs (the FP8/bf16 "
-                               "nominal ratio), x 1 for FP16 MMAs; kernels timed inside a long power-capped step"}
+                "peak_source": ("measured bf16 sustained (MEASURED_PEAKS.json) x 2 for E4M3 MMAs (the FP8/bf16 "
+                                "nominal ratio), x 1 for FP16 MMAs; kernels timed inside a long power-capped "
+                                "region") if long_region else
+                               ("measured bf16 burst (MEASURED_PEAKS.json) x 2 for E4M3 MMAs, x 1 for FP16 MMAs; "
+                                "a short timed region without the power cap")}
         if fp8_peak and "sustained_tflops" in fp8_peak:
             roof["frac_of_scaled_mm_fp8_sustained"] = round(achieved / fp8_peak["sustained_tflops"], 4)
             roof["frac_of_scaled_mm_fp8_burst"] = round(achieved / fp8_peak["burst_tflops"], 4)
@@ -610,7 +626,7 @@ def analyse_segments(layers, marks, ms_step, peaks, fp8_peak):
 
     regimes = {}
     for key, pred, what, target in (("decode_m_le_16", lambda m: m <= 16, "hbm", 0.80),
-                                    ("weight_streaming_m_le_256", lambda m: m <= 256, "hbm", 0.75),
+                                    ("weight_streaming_m_le_128", lambda m: m <= 128, "hbm", 0.75),
                                     ("prefill_m_ge_512", lambda m: m >= 512, "tensor", 0.60)):
         r = regime(pred, what)
         if r is not None:
@@ -680,18 +696,44 @@ def time_workload(pg, torch, dev, wl, args, steps, warmup, world, peaks, fp8_pea
         raise RuntimeError(f"device error word raised in the timed region: {st}")
     ms_step = ms_total / steps
 
-    # bracketed steps (outside the timed region): median of 3 per segment
+    # bracketed steps (outside the timed region), replayed from a CUDA graph
+    # like the timed steps, so that no host launch gap sits between two
+    # events; 3 replays, the middle one by total time
     runs = []
-    for _ in range(3):
-        marks = []
+    bracket_mode = "graph"
+    try:
+        marks_g = []
+        bgraph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(bgraph, stream=stream):
+            runner.bracketed_step(marks_g)
         with torch.cuda.stream(stream):
-            runner.bracketed_step(marks)
+            bgraph.replay()
         stream.synchronize()
-        runs.append(marks)
+        for _ in range(3):
+            with torch.cuda.stream(stream):
+                bgraph.replay()
+            stream.synchronize()
+            runs.append([(seg, ev, seg_ev.elapsed_time(ev) if k else 0.0)
+                         for k, ((seg, ev), (_, seg_ev)) in enumerate(zip(marks_g, [marks_g[0]] + marks_g[:-1]))])
+        del bgraph
+    except RuntimeError:
+        # (events recorded inside a capture not supported): eager launches
+        torch.cuda.synchronize()
+        bracket_mode = "eager"
+        runs = []
+        for _ in range(3):
+            marks = []
+            with torch.cuda.stream(stream):
+                runner.bracketed_step(marks)
+            stream.synchronize()
+            runs.append([(seg, ev, prev.elapsed_time(ev) if k else 0.0)
+                         for k, ((seg, ev), (_, prev)) in enumerate(zip(marks, [marks[0]] + marks[:-1]))])
     # keep the middle run by total bracketed time
-    totals = [r[0][1].elapsed_time(r[-1][1]) for r in runs]
+    totals = [sum(d for (_, _, d) in r) for r in runs]
     marks = runs[sorted(range(3), key=lambda k: totals[k])[1]]
-    roof, regimes, segments = analyse_segments(layers, marks, ms_step, peaks, fp8_peak)
+    long_region = ms_total >= 200.0 or bool(clk and "sw_power_cap" in clk.get("reasons", []))
+    roof, regimes, segments = analyse_segments(layers, marks, ms_step, peaks, fp8_peak, long_region)
+    roof["bracketing"] = bracket_mode
     del graph
     wbytes = sum(L.weight_bytes for L in layers)
     flops = sum(L.flops for L in layers)

@@ -457,14 +457,18 @@ size_t pgf8_fp8_linear_dynamic_scales_offset(int64_t M, int64_t K);
  * are bit-identical to that call's, its outputs are within the same bound
  * (the f32 summation order differs).
  *
- * Layers with M <= 256 are quantised by one launch and then streamed by one
+ * Layers with M <= 128 are quantised by one launch and then streamed by one
  * persistent grouped kernel (one CTA per SM, each SM streaming an equal
- * share of all those layers' weights, up to 32 layers per launch pair; the
- * layers with 128 < M <= 256 in a launch pair of their own); larger layers
- * run one dynamic call each afterwards.  Decode-sized layers
- * are bound by their weight stream ("7B token speed on consumer GPUs" §1),
- * and one stream for the whole group pays the start and the end of a
- * launch once instead of once per layer.
+ * share of all those layers' weights, up to 32 layers per launch pair).
+ * Decode-sized layers are bound by their weight stream ("7B token speed on
+ * consumer GPUs" §1), and one stream for the whole group pays the start and
+ * the end of a launch once instead of once per layer.  The layers with
+ * M > 128 are then quantised by one launch and multiplied by one persistent
+ * launch on SM pairs over all their 256 x 256 output tiles (up to 32 layers
+ * per launch pair), so one layer's last round of tiles is filled by the
+ * next layer's.  With explicit kernel options (path, tile_n or split_k set)
+ * the layers with 128 < M <= 256 take a grouped launch pair of their own
+ * and larger layers run one dynamic call each, with those options.
  *
  * group_workspace: pgf8_fp8_linear_group_workspace_size(max M over the
  * layers) bytes of device memory, 16-byte aligned, zero-filled once before
@@ -484,6 +488,35 @@ pgf8_status pgf8_fp8_linear_dynamic_group(const pgf8_fp8_layer *layers, int64_t 
                                           void *group_workspace, size_t group_workspace_bytes,
                                           const pgf8_linear_opts *opts, void *stream);
 size_t pgf8_fp8_linear_group_workspace_size(int64_t max_m);
+
+/* One layer of pgf8_fp8_linear_group: the arguments of pgf8_fp8_linear
+ * (pre-quantised activations). */
+typedef struct {
+    const uint8_t *aq;       /* [M, K] E4M3 codes */
+    const float *sa;         /* [M] */
+    const uint8_t *wq;       /* [N, K] E4M3 codes */
+    const float *sw;         /* [N] */
+    void *y;                 /* [M, N] bf16 */
+    int64_t M, K, N;
+} pgf8_fp8_gemm_layer;
+
+/* ------------------------------------------------------------------------
+ * Independent FP8 GEMMs with their dequantising epilogue ("C++ and FP8"
+ * §3.3: E4M3 x E4M3 -> f32 -> bf16), each exactly what pgf8_fp8_linear
+ * computes (within the same bound; the f32 summation order may differ),
+ * all in one persistent launch on SM pairs over every layer's 256 x 256
+ * output tiles (up to 32 layers per launch).  The tiled kernel of the
+ * grouped dynamic call's M > 128 layers, for callers that quantise
+ * themselves; any M works, but the 256-token tiles suit M > 128.
+ * No workspace.  Errors: a layer's argument errors (as pgf8_fp8_linear) or
+ * an output overlapping any layer's operands or another layer's output
+ * (PGF8_ERR_INVALID_ARG), before anything is enqueued; opts other than the
+ * automatic choice (path, tile_n, split_k) give PGF8_ERR_UNSUPPORTED.
+ * The launch may start while the previous kernel in the stream finishes
+ * (it reads nothing before that kernel has completed).
+ * ---------------------------------------------------------------------- */
+pgf8_status pgf8_fp8_linear_group(const pgf8_fp8_gemm_layer *layers, int64_t count,
+                                  const pgf8_linear_opts *opts, void *stream);
 
 /* ------------------------------------------------------------------------
  * Building blocks of a tensor-parallel FP8 linear layer ("C++ and FP8"

@@ -56,6 +56,11 @@ class Fp8Layer(ctypes.Structure):
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
 
 
+class Fp8GemmLayer(ctypes.Structure):
+    _fields_ = [("aq", ctypes.c_void_p), ("sa", ctypes.c_void_p), ("wq", ctypes.c_void_p), ("sw", ctypes.c_void_p),
+                ("y", ctypes.c_void_p), ("M", ctypes.c_int64), ("K", ctypes.c_int64), ("N", ctypes.c_int64)]
+
+
 class NestedLayer(ctypes.Structure):
     _fields_ = [("x_f16", ctypes.c_void_p), ("hi", ctypes.c_void_p), ("lo", ctypes.c_void_p),
                 ("y_f16", ctypes.c_void_p), ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
@@ -94,6 +99,7 @@ _SIGS = {
     "pgf8_fp8_linear_dynamic_scales_offset": ([_i64, _i64], _sz),
     "pgf8_fp8_linear_dynamic_group": ([ctypes.POINTER(Fp8Layer), _i64, _vp, _sz, _optp, _vp], _i32),
     "pgf8_fp8_linear_group_workspace_size": ([_i64], _sz),
+    "pgf8_fp8_linear_group": ([ctypes.POINTER(Fp8GemmLayer), _i64, _optp, _vp], _i32),
     "pgf8_fp8_row_amax": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp], _i32),
     "pgf8_fp8_quantize_rows_amax": ([_vp, _i32, _i64, _i64, _i64, _vp, _vp, _vp], _i32),
     "pgf8_fp8_linear_partial": ([_vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _sz, _vp], _i32),
@@ -640,6 +646,25 @@ class LayerGroup(LayerSequence):
         _check(lib.pgf8_fp8_linear_dynamic_group(self._arr, self.count, _ptr(self.group_workspace),
                                                  _nbytes(self.group_workspace), _opts(flags=flags), _stream(stream)),
                "fp8_linear_dynamic_group")
+
+
+def fp8_linear_group(layers, flags=0, stream=None):
+    """pgf8_fp8_linear_group: independent pre-quantised FP8 GEMMs in one
+    launch on SM pairs.  Each entry (aq [M,K] uint8, sa [M] f32, wq [N,K]
+    uint8, sw [N] f32, y [M,N] bf16 or None); returns the outputs."""
+    arr = (Fp8GemmLayer * len(layers))()
+    outs = []
+    for i, (aq, sa, wq, sw, y) in enumerate(layers):
+        if not (aq.is_contiguous() and wq.is_contiguous() and sa.is_contiguous() and sw.is_contiguous()):
+            raise ValueError("operands must be contiguous")
+        M, K = aq.shape
+        N = wq.shape[0]
+        if y is None:
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=aq.device)
+        outs.append(y)
+        arr[i] = Fp8GemmLayer(aq.data_ptr(), sa.data_ptr(), wq.data_ptr(), sw.data_ptr(), y.data_ptr(), M, K, N)
+    _check(lib.pgf8_fp8_linear_group(arr, len(layers), _opts(flags=flags), _stream(stream)), "fp8_linear_group")
+    return outs
 
 
 def group_workspace_size(max_m: int) -> int:

@@ -185,6 +185,31 @@ def test_dynamic_group_checks_layers_aliasing_and_workspace_first():
     assert f(None, 0, None, 0, None, None) == pg.OK
 
 
+def test_fp8_linear_group_checks_first():
+    """pgf8_fp8_linear_group: every layer's arguments and the outputs'
+    independence checked before anything is enqueued; explicit kernel
+    options refused."""
+    f = pg.lib.pgf8_fp8_linear_group
+    base = 1 << 34
+    aq0, sa0, wq, sw, y0, y1, aq1, sa1 = (base + i * (1 << 26) for i in range(8))
+    l0 = pg.Fp8GemmLayer(aq0, sa0, wq, sw, y0, 300, 512, 512)
+    l1 = pg.Fp8GemmLayer(aq1, sa1, wq, sw, y1, 600, 512, 512)      # layers may share weights
+    assert f(None, 0, None, None) == pg.OK
+    assert f(None, 2, None, None) == pg.ERR_INVALID_ARG
+    bad_k = pg.Fp8GemmLayer(aq1, sa1, wq, sw, y1, 600, 520, 512)
+    assert f((pg.Fp8GemmLayer * 2)(l0, bad_k), 2, None, None) == pg.ERR_ALIGNMENT
+    mis = pg.Fp8GemmLayer(aq1 + 8, sa1, wq, sw, y1, 600, 512, 512)
+    assert f((pg.Fp8GemmLayer * 2)(l0, mis), 2, None, None) == pg.ERR_ALIGNMENT
+    no_sw = pg.Fp8GemmLayer(aq1, sa1, wq, None, y1, 600, 512, 512)
+    assert f((pg.Fp8GemmLayer * 2)(l0, no_sw), 2, None, None) == pg.ERR_INVALID_ARG
+    same_y = pg.Fp8GemmLayer(aq1, sa1, wq, sw, y0, 600, 512, 512)
+    assert f((pg.Fp8GemmLayer * 2)(l0, same_y), 2, None, None) == pg.ERR_INVALID_ARG
+    into_w = pg.Fp8GemmLayer(aq1, sa1, wq, sw, wq + 4096, 600, 512, 512)   # output over the weights
+    assert f((pg.Fp8GemmLayer * 2)(l0, into_w), 2, None, None) == pg.ERR_INVALID_ARG
+    o = pg.LinearOpts(pg.PATH_TILED, 0, 0, 0)
+    assert f((pg.Fp8GemmLayer * 2)(l0, l1), 2, ctypes.byref(o), None) == pg.ERR_UNSUPPORTED
+
+
 def test_nested_group_checks_layers_aliasing_and_workspace_first():
     """pgf8_nestedfp_linear_group: the mode, every layer (FP8 mode: with its
     workspace), independence and the group workspace checked before anything

@@ -202,3 +202,97 @@ def test_group_llama70b_streaming_layers_full_size_sampled():
         ref = _oracle_linear_threaded(aq0, sa0, wq0, sw0)
         bound = linear_bound(ref, K, fp8_row_max(aq0, sa0), fp8_row_max(wq0, sw0))
         assert_within(layer[3].float().cpu().numpy()[:, ns], ref, bound, f"70B layer {i} (M={M}, shape {si})")
+
+
+PAIR_GROUP = [(1, 512, 528), (100, 272, 400), (129, 1040, 144), (256, 656, 272), (300, 400, 528),
+              (600, 1008, 784), (513, 144, 1040)]   # (M, K, N): ragged M, N and K; one-tile and many-tile layers
+
+
+def test_fp8_linear_group_pre_quantised():
+    """pgf8_fp8_linear_group: the codes and scales the oracle gives, several
+    layers in one launch on SM pairs; every output within the layer's bound
+    of the oracle's binary64 layer, and equal to a second call bit for bit."""
+    g = np.random.default_rng(31)
+    ops, host = [], []
+    for (M, K, N) in PAIR_GROUP:
+        x = synthetic.activations("student_t3", M, K, g)
+        w = synthetic.weights_f16(N, K, 0.02, g)
+        aq0, sa0 = oracle.quantize_rows(x)
+        wq0, sw0 = oracle.quantize_rows(w)
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(DEV)  # noqa: E731
+        y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+        ops.append((t(aq0), t(sa0), t(wq0), t(sw0), y))
+        host.append((aq0, sa0, wq0, sw0))
+    pg.fp8_linear_group(ops)
+    torch.cuda.synchronize()
+    assert pg.device_status() == pg.OK
+    first = [o[4].clone() for o in ops]
+    for i, (o, (aq0, sa0, wq0, sw0)) in enumerate(zip(ops, host)):
+        ref = oracle.fp8_linear(aq0, sa0, wq0, sw0)
+        bound = linear_bound(ref, aq0.shape[1], fp8_row_max(aq0, sa0), fp8_row_max(wq0, sw0))
+        assert_within(o[4].float().cpu().numpy(), ref, bound, f"pair-group layer {i}")
+    pg.fp8_linear_group(ops, flags=pg.FLAG_OVERLAP_PREVIOUS)
+    torch.cuda.synchronize()
+    for i, (o, f) in enumerate(zip(ops, first)):
+        assert torch.equal(o[4].view(torch.int16), f.view(torch.int16)), f"layer {i} differs on the second call"
+
+
+def test_group_more_large_layers_than_one_launch_takes():
+    """40 layers with M > 128 in one grouped call: two quantisation and
+    tiled launches (32 layers per launch), each layer checked."""
+    shapes = [(129 + 7 * i, 144 + 16 * (i % 5), 144 + 32 * (i % 3)) for i in range(40)]
+    layers, host = _make_group(shapes, 37)
+    grp = pg.LayerGroup(layers)
+    grp.run()
+    torch.cuda.synchronize()
+    assert pg.device_status() == pg.OK
+    for i, (layer, (x, w)) in enumerate(zip(layers, host)):
+        _check_layer(i, layer, x, w)
+
+
+@pytest.mark.slow
+def test_group_llama70b_tiled_layers_full_size_sampled():
+    """The llama70b step's tiled part at full size: the four 70B shapes at
+    M = 256, 512, ..., 4096 (20 layers, one quantisation launch and one tiled
+    launch on SM pairs), codes and scales bit-exact on 6 sampled rows of
+    every layer, outputs of those rows on 64 sampled channels within the
+    bound."""
+    wl = synthetic.WORKLOADS["llama70b"]
+    mis = [mi for mi, m in enumerate(wl.ms) if m >= 256]
+    weights = {}
+    for si, (K, N, _) in enumerate(wl.shapes):
+        w = synthetic.weights("llama70b", si)
+        wq, sw = pg.fp8_quantize_rows(torch.from_numpy(w).to(DEV))
+        weights[si] = (w, wq, sw)
+    layers, host = [], []
+    for mi in mis:
+        M = wl.ms[mi]
+        for si, (K, N, _) in enumerate(wl.shapes):
+            x = synthetic.acts("llama70b", si, mi)
+            w, wq, sw = weights[si]
+            y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+            ws = torch.zeros(pg.fp8_linear_dynamic_workspace_size(M, N, K), dtype=torch.uint8, device=DEV)
+            layers.append((torch.from_numpy(x).to(DEV), wq, sw, y, ws))
+            host.append((x, si))
+    grp = pg.LayerGroup(layers)
+    grp.run()
+    torch.cuda.synchronize()
+    assert pg.device_status() == pg.OK
+    rng = np.random.default_rng(8)
+    wq0s = {}
+    for i, (layer, (x, si)) in enumerate(zip(layers, host)):
+        w = weights[si][0]
+        if si not in wq0s:
+            ns = np.sort(rng.choice(w.shape[0], 64, replace=False))
+            wq0s[si] = (ns,) + oracle.quantize_rows(w[ns])
+        ns, wq0, sw0 = wq0s[si]
+        M, K = x.shape
+        ms = np.sort(rng.choice(M, 6, replace=False))
+        aq0, sa0 = oracle.quantize_rows(x[ms])
+        aq, sa = pg.dynamic_workspace_views(layer[4], M, K)
+        assert np.array_equal(aq.cpu().numpy()[ms], aq0), f"layer {i}: codes"
+        assert np.array_equal(sa.cpu().numpy()[ms].view(np.uint32), sa0.view(np.uint32)), f"layer {i}: scales"
+        ref = oracle.fp8_linear(aq0, sa0, wq0, sw0)
+        bound = linear_bound(ref, K, fp8_row_max(aq0, sa0), fp8_row_max(wq0, sw0))
+        got = layer[3].float().cpu().numpy()[np.ix_(ms, ns)]
+        assert_within(got, ref, bound, f"70B tiled layer {i} (M={M}, shape {si})")
