@@ -463,10 +463,10 @@ size_t pgf8_fp8_linear_dynamic_scales_offset(int64_t M, int64_t K);
  * Decode-sized layers are bound by their weight stream ("7B token speed on
  * consumer GPUs" §1), and one stream for the whole group pays the start and
  * the end of a launch once instead of once per layer.  The layers with
- * M > 128 are then quantised by one launch and multiplied by one persistent
- * launch on SM pairs over all their 256 x 256 output tiles (up to 32 layers
- * per launch pair), so one layer's last round of tiles is filled by the
- * next layer's.  With explicit kernel options (path, tile_n or split_k set)
+ * M > 128 are then quantised by one launch and multiplied as
+ * pgf8_fp8_linear_group multiplies them (the layers with a few rounds of
+ * tiles in one launch on SM pairs, so one layer's last round is filled by
+ * the next layer's; larger layers one tiled launch each).  With explicit kernel options (path, tile_n or split_k set)
  * the layers with 128 < M <= 256 take a grouped launch pair of their own
  * and larger layers run one dynamic call each, with those options.
  *
@@ -503,9 +503,11 @@ typedef struct {
 /* ------------------------------------------------------------------------
  * Independent FP8 GEMMs with their dequantising epilogue ("C++ and FP8"
  * §3.3: E4M3 x E4M3 -> f32 -> bf16), each exactly what pgf8_fp8_linear
- * computes (within the same bound; the f32 summation order may differ),
- * all in one persistent launch on SM pairs over every layer's 256 x 256
- * output tiles (up to 32 layers per launch).  The tiled kernel of the
+ * computes (within the same bound; the f32 summation order may differ).
+ * The layers with at most 296 tiles of 256 x 256 (four rounds of the
+ * B200's 74 SM pairs) share one persistent launch on SM pairs over all
+ * their tiles (up to 32 layers per launch); each larger layer runs its own
+ * tiled launch (measured faster for those).  The tiled GEMMs of the
  * grouped dynamic call's M > 128 layers, for callers that quantise
  * themselves; any M works, but the 256-token tiles suit M > 128.
  * No workspace.  Errors: a layer's argument errors (as pgf8_fp8_linear) or

@@ -1744,16 +1744,90 @@ static pgf8_status nested_group_one(const void *x, int64_t M, int64_t K, const u
 // One grouped launch pair for up to kGroupMaxLayers small-M layers: the
 // per-token quantisation of all of them, then the grouped GEMM, which
 // streams its first ring of weights while the quantisation runs.
+// Layers with more 256 x 256 tiles than this (four rounds of the 74 SM
+// pairs) run one launch each: measured on B200 over the llama70b step, one
+// launch over every M > 128 layer ran 8 % slower than one launch per layer
+// (8.24 against 7.62 ms), while on the 7B prefill layers (a few rounds
+// each) the shared launch was 9 % faster.
+constexpr int64_t kPairGroupMaxTiles = 296;
+
+// Up to kPairGroupMaxLayers pre-quantised FP8 GEMMs: one persistent launch
+// on SM pairs over all the 256 x 256 tiles of the layers with at most
+// kPairGroupMaxTiles tiles, then one tiled launch for each larger layer (all
+// with programmatic stream serialization: nothing is read before the
+// previous kernel has completed).
+static pgf8_status tiled_group_launch(const pgf8_fp8_gemm_layer *ls, int n, cudaStream_t cs)
+{
+    PairGroupParams gp;   // about 10 KB: passed by value as the kernel's parameter block
+    std::memset(&gp, 0, sizeof(gp));
+    int64_t tiles = 0;
+    int ng = 0;
+    auto ntiles = [](const pgf8_fp8_gemm_layer &l) { return ((l.M + 255) / 256) * ((l.N + 255) / 256); };
+    for (int i = 0; i < n; ++i) {
+        const pgf8_fp8_gemm_layer &l = ls[i];
+        if (ntiles(l) > kPairGroupMaxTiles)
+            continue;
+        const int gi = ng++;
+        PairGroupLayer &g = gp.L[gi];
+        g.M = static_cast<int>(l.M);
+        g.N = static_cast<int>(l.N);
+        g.kblocks = static_cast<int>((l.K + 127) / 128);
+        g.m_tiles = static_cast<int>((l.M + 255) / 256);
+        g.tile0 = static_cast<int>(tiles);
+        g.sa = l.sa;
+        g.sw = l.sw;
+        g.y = l.y;
+        tiles += ntiles(l);
+        if (!make_map(&gp.tmX[gi], l.aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(l.M),
+                      static_cast<uint64_t>(l.K), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&gp.tmW[gi], l.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(l.N),
+                      static_cast<uint64_t>(l.K), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+            return PGF8_ERR_UNSUPPORTED;
+    }
+    if (ng > 0) {
+        gp.nlayers = ng;
+        gp.total = static_cast<int>(tiles);
+        const pgf8_status st = launch_pair_group(gp, cs);
+        if (st != PGF8_OK)
+            return st;
+    }
+    for (int i = 0; i < n; ++i) {
+        const pgf8_fp8_gemm_layer &l = ls[i];
+        if (ntiles(l) <= kPairGroupMaxTiles)
+            continue;
+        GemmLaunch L;
+        L.ws = nullptr;
+        L.ws_bytes = 0;
+        L.kind = kE4M3;
+        L.x = l.aq;
+        L.w = l.wq;
+        L.w2 = nullptr;
+        L.sa = l.sa;
+        L.sw = l.sw;
+        L.y = l.y;
+        L.M = static_cast<int>(l.M);
+        L.N = static_cast<int>(l.N);
+        L.K = static_cast<int>(l.K);
+        L.pdl = 1;
+        L.prefetch_w = 1;   // nothing before writes the weights
+        L.opts = opts_or_default(nullptr);
+        L.stream = cs;
+        const pgf8_status st = launch_gemm<kE4M3>(L);
+        if (st != PGF8_OK)
+            return st;
+    }
+    return PGF8_OK;
+}
+
 // Up to kPairGroupMaxLayers tiled layers (M > 128): the per-token
-// quantisation of all of them (one launch), then one persistent launch on SM
-// pairs over all their 256 x 256 tiles.
+// quantisation of all of them (one launch), then their GEMMs as
+// tiled_group_launch runs them.
 static pgf8_status pair_group_chunk(const pgf8_fp8_layer *const *ls, int n, int first_pdl, cudaStream_t cs)
 {
     QuantGroupParams qp;
     std::memset(&qp, 0, sizeof(qp));
-    PairGroupParams gp;   // about 10 KB: passed by value as the kernel's parameter block
-    std::memset(&gp, 0, sizeof(gp));
-    int64_t rows = 0, tiles = 0;
+    pgf8_fp8_gemm_layer gl[kPairGroupMaxLayers];
+    int64_t rows = 0;
     for (int i = 0; i < n; ++i) {
         const pgf8_fp8_layer &l = *ls[i];
         uint8_t *aq = static_cast<uint8_t *>(l.workspace) + pgf8_fp8_linear_dynamic_codes_offset(l.M, l.K);
@@ -1769,29 +1843,18 @@ static pgf8_status pair_group_chunk(const pgf8_fp8_layer *const *ls, int n, int 
         q.scales = sa;
         q.xdt = l.xdt == PGF8_F32 ? 0 : 1;
         rows += l.M;
-
-        PairGroupLayer &g = gp.L[i];
-        g.M = static_cast<int>(l.M);
-        g.N = static_cast<int>(l.N);
-        g.kblocks = static_cast<int>((l.K + 127) / 128);
-        g.m_tiles = static_cast<int>((l.M + 255) / 256);
-        g.tile0 = static_cast<int>(tiles);
-        g.sa = sa;
-        g.sw = l.sw;
-        g.y = l.y;
-        tiles += static_cast<int64_t>(g.m_tiles) * ((l.N + 255) / 256);
-        if (!make_map(&gp.tmX[i], aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(l.M),
-                      static_cast<uint64_t>(l.K), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_map(&gp.tmW[i], l.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(l.N),
-                      static_cast<uint64_t>(l.K), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B))
-            return PGF8_ERR_UNSUPPORTED;
+        gl[i].aq = aq;
+        gl[i].sa = sa;
+        gl[i].wq = l.wq;
+        gl[i].sw = l.sw;
+        gl[i].y = l.y;
+        gl[i].M = l.M;
+        gl[i].K = l.K;
+        gl[i].N = l.N;
     }
-    if (tiles > (1ll << 30) || rows > (1ll << 31) - 1)
+    if (rows > (1ll << 31) - 1)
         return PGF8_ERR_UNSUPPORTED;
     qp.nlayers = n;
-    gp.nlayers = n;
-    gp.total = static_cast<int>(tiles);
-
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(static_cast<unsigned>(rows));
@@ -1807,7 +1870,7 @@ static pgf8_status pair_group_chunk(const pgf8_fp8_layer *const *ls, int n, int 
     const cudaError_t e = cudaLaunchKernelEx(&cfg, quantize_group_kernel, qp);
     if (e != cudaSuccess)
         return cuda_fail(e);
-    return launch_pair_group(gp, cs);
+    return tiled_group_launch(gl, n, cs);
 }
 
 static pgf8_status group_chunk(const pgf8_fp8_layer *const *ls, int n, void *group_ws, int first_pdl,
@@ -2031,34 +2094,9 @@ pgf8_status pgf8_fp8_linear_group(const pgf8_fp8_gemm_layer *layers, int64_t cou
     if (o.path != PGF8_PATH_AUTO || o.split_k != 0 || o.tile_n != 0)
         return PGF8_ERR_UNSUPPORTED;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    PairGroupParams gp;
     for (int64_t c0 = 0; c0 < count; c0 += kPairGroupMaxLayers) {
         const int n = static_cast<int>(count - c0 < kPairGroupMaxLayers ? count - c0 : kPairGroupMaxLayers);
-        std::memset(&gp, 0, sizeof(gp));
-        int64_t tiles = 0;
-        for (int i = 0; i < n; ++i) {
-            const pgf8_fp8_gemm_layer &l = layers[c0 + i];
-            PairGroupLayer &g = gp.L[i];
-            g.M = static_cast<int>(l.M);
-            g.N = static_cast<int>(l.N);
-            g.kblocks = static_cast<int>((l.K + 127) / 128);
-            g.m_tiles = static_cast<int>((l.M + 255) / 256);
-            g.tile0 = static_cast<int>(tiles);
-            g.sa = l.sa;
-            g.sw = l.sw;
-            g.y = l.y;
-            tiles += static_cast<int64_t>(g.m_tiles) * ((l.N + 255) / 256);
-            if (!make_map(&gp.tmX[i], l.aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(l.M),
-                          static_cast<uint64_t>(l.K), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-                !make_map(&gp.tmW[i], l.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(l.N),
-                          static_cast<uint64_t>(l.K), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B))
-                return PGF8_ERR_UNSUPPORTED;
-        }
-        if (tiles > (1ll << 30))
-            return PGF8_ERR_UNSUPPORTED;
-        gp.nlayers = n;
-        gp.total = static_cast<int>(tiles);
-        const pgf8_status st = launch_pair_group(gp, cs);
+        const pgf8_status st = tiled_group_launch(layers + c0, n, cs);
         if (st != PGF8_OK)
             return st;
     }
