@@ -1763,8 +1763,22 @@ static pgf8_status tiled_group_launch(const pgf8_fp8_gemm_layer *ls, int n, cuda
     int64_t tiles = 0;
     int ng = 0;
     auto ntiles = [](const pgf8_fp8_gemm_layer &l) { return ((l.M + 255) / 256) * ((l.N + 255) / 256); };
-    for (int i = 0; i < n; ++i) {
-        const pgf8_fp8_gemm_layer &l = ls[i];
+    // The shared list takes the layers in order of K (stable): the pairs
+    // walk it round-robin, and tiles of one length keep them in step, so the
+    // tiles in flight at any time stay neighbours (their operands shared in
+    // L2); a pair that met a longer tile would otherwise fall behind its
+    // neighbours for the rest of the list.
+    int order[kPairGroupMaxLayers];
+    for (int i = 0; i < n; ++i)
+        order[i] = i;
+    for (int i = 1; i < n; ++i)
+        for (int j = i; j > 0 && ls[order[j - 1]].K > ls[order[j]].K; --j) {
+            const int t = order[j];
+            order[j] = order[j - 1];
+            order[j - 1] = t;
+        }
+    for (int oi = 0; oi < n; ++oi) {
+        const pgf8_fp8_gemm_layer &l = ls[order[oi]];
         if (ntiles(l) > kPairGroupMaxTiles)
             continue;
         const int gi = ng++;
