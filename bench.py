@@ -816,6 +816,7 @@ def run_ours(args, rank, world, local_rank):
             wl2 = setup_workload(pg, torch, dev, sec)
             steps2 = {"decode7b": 400, "prefill7b": 60, "nested7b": 60, "nested7b_decode": 200}[sec]
             r2 = time_workload(pg, torch, dev, wl2, args, steps2, 10, world, peaks, fp8_peak)
+            r2["roof"]["traffic"], r2["roof"]["traffic_note"] = profiled_traffic(sec)
             mb = sec in ("decode7b", "nested7b_decode")
             v = (r2["wbytes"] / 1e9 if mb else r2["flops"] / 1e12) / (r2["ms_step"] * 1e-3) * world
             result["secondary"][sec] = {
