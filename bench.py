@@ -47,12 +47,7 @@ if ROOT not in sys.path:
 
 import synthetic  # noqa: E402
 
-METRIC = None
-try:
-    with open(os.path.join(ROOT, "BASELINE.json")) as _f:
-        METRIC = json.load(_f)["metric"]
-except Exception:
-    METRIC = "FP8 linear TFLOPS & weight GB/s vs B200 roofline, 7B/70B shapes, M=1–4096"
+METRIC = "FP8 linear TFLOPS & weight GB/s vs B200 roofline, 7B/70B shapes, M=1–4096"
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
