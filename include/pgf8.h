@@ -624,9 +624,9 @@ typedef struct {
  * in that mode (FP8 mode: its codes and scales bit-identical; its outputs
  * within the same bound, the f32 summation order differs).
  * Layers with M <= 256 stream their weight planes through the grouped
- * kernel as pgf8_fp8_linear_dynamic_group does (FP8 mode: one quantisation
- * launch first; one launch for the layers with M <= 128 and one for
- * 128 < M <= 256, up to 32 layers each); larger layers run one call each.
+ * weight-streaming kernel (FP8 mode: one quantisation launch first; one
+ * launch for the layers with M <= 128 and one for 128 < M <= 256, up to 32
+ * layers each); larger layers run one call each.
  *   group_workspace: pgf8_fp8_linear_group_workspace_size(max M of the
  *     layers with M <= 256) bytes, zero-filled once before first use and
  *     left zero by every call; may be NULL when no layer has M <= 256.
