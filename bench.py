@@ -194,9 +194,10 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- profiled traffic
-# The GEMM kernels' sources (and the helpers they include): what a DRAM
-# traffic record describes.  The record also names the kernel configuration
-# it was taken on.
+# The sources of the kernels the recorded FP8 steps run (and the helpers
+# they include): what a DRAM traffic record describes.  The record also
+# names the kernel configuration it was taken on.  (The NestedFP-only
+# swapped FP16 kernel, gemm_persistent_swap.cuh, runs in none of them.)
 GEMM_SOURCES = ("gemm.cuh", "gemm_2sm.cuh", "gemm_pair_group.cuh", "gemm_persistent.cuh", "gemm_streamk.cuh", "gemm_group.cuh",
                 "quantize.cuh", "sm100_ptx.cuh")
 

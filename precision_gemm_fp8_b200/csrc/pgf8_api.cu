@@ -18,6 +18,7 @@
 #include "gemm_2sm.cuh"
 #include "gemm_group.cuh"
 #include "gemm_pair_group.cuh"
+#include "gemm_persistent_swap.cuh"
 #include "quantize.cuh"
 
 // Pipeline depths and stream-K occupancy (compile-time tuning constants).
@@ -298,6 +299,37 @@ template <class C> static pgf8_status launch_persistent(const GemmLaunch &L)
     cudaLaunchAttribute attrs[2];
     fill_attrs(cfg, attrs, 1, L.pdl);
     cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_persistent_kernel<C>, tmX, tmW, tmW2, p);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    return PGF8_OK;
+}
+
+// NestedFP FP16 mode, swapped orientation: one CTA per SM (at most one per
+// tile of 128 weight rows x BN tokens).
+template <class C> static pgf8_status launch_persistent_swap(const GemmLaunch &L)
+{
+    static PerDeviceSetup setup;
+    const cudaError_t attr_err = setup_once_per_device(setup, [](int, int *) {
+        return cudaFuncSetAttribute(gemm_persistent_swap_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    C::kSmemBytes);
+    });
+    if (attr_err != cudaSuccess)
+        return cuda_fail(attr_err);
+    CUtensorMap tmX, tmW, tmW2;
+    if (!make_operand_maps<C>(L, tmX, tmW, tmW2))
+        return PGF8_ERR_UNSUPPORTED;
+    const GemmParams p = make_params(L, 1);
+    const int64_t tiles = static_cast<int64_t>((L.M + C::BN - 1) / C::BN) * ((L.N + 127) / 128);
+    const int sms = num_sms();
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles < sms ? tiles : sms), 1, 1);
+    cfg.blockDim = dim3(C::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = L.stream;
+    cudaLaunchAttribute attrs[2];
+    fill_attrs(cfg, attrs, 1, L.pdl);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_persistent_swap_kernel<C>, tmX, tmW, tmW2, p);
     if (e != cudaSuccess)
         return cuda_fail(e);
     return PGF8_OK;
@@ -616,10 +648,20 @@ template <int KIND> static pgf8_status launch_gemm(const GemmLaunch &L)
     // 70B shape (M = 256 .. 4096): with 40 or more tiles it is the fastest or
     // within 3 %; with 32 tiles the one-CTA persistent kernel below is
     // faster (more SMs busy on 128-row tiles).
-    // (NestedFP FP16 mode stays on the one-CTA kernels: its pair form
-    // measured 1.6-1.8x slower on B200 at every 7B / 70B shape, M = 512 ..
-    // 4096; it stays selectable through PGF8_PATH_TILED_PAIR)
-    if constexpr (KIND != kNested16) {
+    // NestedFP FP16 mode, automatic choice, M > 256 with at least 96 tiles
+    // of 128 weight rows x 256 tokens: the one-CTA kernel with the rebuilt
+    // weights as the 128-row operand (less shared-memory traffic per
+    // k-step).  Measured on B200 over the 7B / 70B shapes at M = 512 ..
+    // 4096: 20-28 % faster from M = 1024 on (7B QKV at M = 1024: 891 against
+    // 735 TFLOP/s), slower only with 64 tiles (7B down at M = 512: 103
+    // against 81 us).  (The SM-pair form measured 1.6-1.8x slower at every
+    // shape; it stays selectable through PGF8_PATH_TILED_PAIR, the
+    // tokens-as-A kernel through path / tile_n.)
+    if constexpr (KIND == kNested16) {
+        const int64_t swap_tiles = static_cast<int64_t>((L.M + 255) / 256) * ((L.N + 127) / 128);
+        if (L.opts.path == PGF8_PATH_AUTO && bn == 0 && splits == 0 && L.M > 256 && swap_tiles >= 96)
+            return launch_persistent_swap<PersistSwapCfg<256, 4>>(L);
+    } else {
         const int64_t tiles_pair = static_cast<int64_t>((L.M + 255) / 256) * ((L.N + 255) / 256);
         // (the 192 / 128 widths fill the last round better but measured slower
         // per tile than 256 on nearly every 7B / 70B shape; they stay
