@@ -694,7 +694,9 @@ def time_workload(pg, torch, dev, wl, args, steps, warmup, world, peaks, fp8_pea
 
     # bracketed steps (outside the timed region), replayed from a CUDA graph
     # like the timed steps, so that no host launch gap sits between two
-    # events; 3 replays, the middle one by total time
+    # events: first as many replays back to back as the timed region had
+    # steps (the GPU reaches the same power state, under the power cap the
+    # same clocks), then 3 measured replays, the middle one by total time
     runs = []
     bracket_mode = "graph"
     try:
@@ -703,7 +705,8 @@ def time_workload(pg, torch, dev, wl, args, steps, warmup, world, peaks, fp8_pea
         with torch.cuda.graph(bgraph, stream=stream):
             runner.bracketed_step(marks_g)
         with torch.cuda.stream(stream):
-            bgraph.replay()
+            for _ in range(steps):
+                bgraph.replay()
         stream.synchronize()
         for _ in range(3):
             with torch.cuda.stream(stream):
