@@ -156,6 +156,14 @@ def _ptr(t: torch.Tensor | None):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _dptr(t: torch.Tensor) -> int:
+    """The device address of a tensor bound into a layer record (the
+    library reads it on the GPU later): device tensors only."""
+    if not t.is_cuda:
+        raise ValueError("pgf8 takes device tensors")
+    return t.data_ptr()
+
+
 def _stream(stream) -> ctypes.c_void_p:
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -614,8 +622,8 @@ class LayerSequence:
         for i, (x, wq, sw, y, ws) in enumerate(self._keep):
             if x.stride(1) != 1:
                 raise ValueError("x rows must be contiguous")
-            arr[i] = Fp8Layer(x.data_ptr(), _dtype_code(x), 0, x.shape[0], x.shape[1], _lead(x), wq.shape[0],
-                              wq.data_ptr(), sw.data_ptr(), y.data_ptr(), ws.data_ptr(), _nbytes(ws))
+            arr[i] = Fp8Layer(_dptr(x), _dtype_code(x), 0, x.shape[0], x.shape[1], _lead(x), wq.shape[0],
+                              _dptr(wq), _dptr(sw), _dptr(y), _dptr(ws), _nbytes(ws))
         self._arr = arr
         self.count = len(self._keep)
 
@@ -662,7 +670,7 @@ def fp8_linear_group(layers, flags=0, stream=None):
         if y is None:
             y = torch.empty((M, N), dtype=torch.bfloat16, device=aq.device)
         outs.append(y)
-        arr[i] = Fp8GemmLayer(aq.data_ptr(), sa.data_ptr(), wq.data_ptr(), sw.data_ptr(), y.data_ptr(), M, K, N)
+        arr[i] = Fp8GemmLayer(_dptr(aq), _dptr(sa), _dptr(wq), _dptr(sw), _dptr(y), M, K, N)
     _check(lib.pgf8_fp8_linear_group(arr, len(layers), _opts(flags=flags), _stream(stream)), "fp8_linear_group")
     return outs
 
@@ -734,8 +742,8 @@ class NestedLayerGroup:
         for i, (x, hi, lo, y, ws) in enumerate(self._keep):
             if x.dtype != torch.float16 or not x.is_contiguous():
                 raise ValueError("x must be a contiguous float16 tensor")
-            arr[i] = NestedLayer(x.data_ptr(), hi.data_ptr(), lo.data_ptr() if lo is not None else None,
-                                 y.data_ptr(), ws.data_ptr() if ws is not None else None, _nbytes(ws),
+            arr[i] = NestedLayer(_dptr(x), _dptr(hi), _dptr(lo) if lo is not None else None,
+                                 _dptr(y), _dptr(ws) if ws is not None else None, _nbytes(ws),
                                  x.shape[0], x.shape[1], hi.shape[0])
         self._arr = arr
         self.count = len(self._keep)

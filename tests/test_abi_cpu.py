@@ -507,3 +507,20 @@ def test_binding_constants_match_the_header():
         assert getattr(pg, n) == values["PGF8_" + n], n
     flags = [values[k] for k in values if k.startswith("PGF8_FLAG_")]
     assert len(set(flags)) == len(flags) and all(f & (f - 1) == 0 for f in flags)   # distinct single bits
+
+
+def test_layer_records_take_device_tensors_only():
+    """The grouped bindings store device addresses the GPU reads later: host
+    tensors are refused before any record is built."""
+    import torch
+    x = torch.zeros(4, 64)
+    wq = torch.zeros(64, 64, dtype=torch.uint8)
+    sw = torch.ones(64)
+    y = torch.zeros(4, 64, dtype=torch.bfloat16)
+    ws = torch.zeros(1 << 12, dtype=torch.uint8)
+    with pytest.raises(ValueError):
+        pg.LayerSequence([(x, wq, sw, y, ws)])
+    with pytest.raises(ValueError):
+        pg.NestedLayerGroup([(x.half(), wq, wq, y.half(), None)], group_workspace=ws)
+    with pytest.raises(ValueError):
+        pg.fp8_linear_group([(wq[:4], sw[:4], wq, sw, y)])
