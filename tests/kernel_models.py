@@ -12,7 +12,9 @@ CPU run checks the kernels' design against the oracle before a GPU does.
   fragment layouts (A: rows g / g+8, cols 2q+e / 2q+8+e; B: rows 2q+e /
   2q+8+e, col g; C: rows g / g+8, cols 2q+e; g = lane / 4, q = lane % 4).
 - context: attn_context_kernel (128-query tiles, 16-row pieces, E4M3
-  probabilities x 2^8, V rows past the context cleared, PV one tile late).
+  probabilities x 2^8 with the scale folded into the exponent, two softmax
+  threads per row each summing its half of l, V rows past the context
+  cleared, PV one tile late).
 
 E4M3 values come from torch's float8_e4m3fn; binary16 rounding from numpy.
 """
@@ -315,7 +317,7 @@ def context(qc, qs, q_start, lens, kc, vc, sk, sv, tables, max_ctx, max_q_len):
             row_ok, pos = rows < nrows, pos0 + rows
             sq = np.array([qs[(q0 + qt * 128 + r) * Hq + h] if r < nrows else 0 for r in range(128)], np.float32)
             scale = (sq * f32(sk[hk]) * (f32(LOG2E) * f32(0.08838834764831845))).astype(np.float32)
-            m, l = np.full(128, -np.inf, np.float32), np.zeros(128, np.float32)
+            m, l = np.full(128, -np.inf, np.float32), np.zeros((2, 128), np.float32)
             o = np.zeros((128, D), np.float32)
             pending = alpha_prev = None
             for j in range(nkt):
@@ -341,17 +343,24 @@ def context(qc, qs, q_start, lens, kc, vc, sk, sv, tables, max_ctx, max_q_len):
                 mn = np.maximum(m, np.where(valid, sc, -np.inf).max(axis=1)).astype(np.float32)
                 safe = np.where(m == -np.inf, 0, m - np.where(m == -np.inf, 0, mn))
                 alpha = np.where(m == -np.inf, 0, np.exp2(safe)).astype(np.float32)
-                pr = np.where(valid, np.exp2(np.where(valid, sc - mn[:, None], 0)), 0).astype(np.float32)
-                P = _e4m3_round(pr * f32(256))
+                # probabilities times 2^8 (the code scale folded into the exponent:
+                # exp2(fma(S, scale, 8 - m))), l in the same units
+                nm8 = (f32(8) - mn).astype(np.float32)
+                arg = np.where(valid, S.astype(np.float64) * scale[:, None] + nm8[:, None], 0).astype(np.float32)
+                pr = np.where(valid, np.exp2(arg), 0).astype(np.float32)
+                P = _e4m3_round(pr)
                 cut = ctx - j * 128
                 if 0 < cut < 128 and cut % 16 and (piece_ok >> (cut // 16)) & 1:
                     Vt[cut:(cut // 16 + 1) * 16] = 0
                 PV = (P.astype(np.float64) @ Vt).astype(np.float32)
-                m, l = mn, (l * alpha + pr.sum(axis=1, dtype=np.float32)).astype(np.float32)
+                # each of the two softmax threads of a row keeps its half's share
+                rs = np.stack([pr[:, :64].sum(axis=1, dtype=np.float32), pr[:, 64:].sum(axis=1, dtype=np.float32)])
+                m, l = mn, (l * alpha[None, :] + rs).astype(np.float32)
                 if pending is not None:
                     o = (o * alpha_prev[:, None] + pending).astype(np.float32)
                 pending, alpha_prev = PV, alpha
             o = (o * alpha_prev[:, None] + pending).astype(np.float32)
-            f = np.where(l > 0, sv[hk] * f32(0.00390625) / np.where(l > 0, l, 1), 0).astype(np.float32)
+            lsum = (l[0] + l[1]).astype(np.float32)
+            f = np.where(lsum > 0, sv[hk] / np.where(lsum > 0, lsum, 1), 0).astype(np.float32)
             out[q0 + qt * 128:q0 + qt * 128 + nrows, h] = o[:nrows] * f[:nrows, None]
     return out
